@@ -1,0 +1,308 @@
+/*
+ * ckda_oracle.c -- float64 sequential CPU oracle for the Complex KDA (CKDA) recurrence.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or call this file:
+ * it exists so that tests/, the smoke check and bench.py's cpu_baseline leg have a plain,
+ * slow, obviously correct definition to compare the CUDA library against.  It shares no
+ * code, header, table or constant with gated_delta_rule_82_b200/csrc.
+ *
+ * What it computes (per batch b and head h, independently; sequentially over t):
+ *
+ *   S := h0[b,h] or 0                                  S in R^{dk x dv}
+ *   for t = 0 .. T-1:
+ *     q, k := q[b,t,h,:], k[b,t,h,:]
+ *     if rope_theta > 0:  rotate (q, k) by angles p * rope_theta^(-2i/dk), p = pos_offset + t
+ *     if l2norm:          x <- x / sqrt(sum x^2 + 1e-6)       (per head, for q and k)
+ *     S <- Diag(alpha_t) S                              (row c of S scaled by alpha_t[c])
+ *     w <- S^T k
+ *     S <- S + beta_t k (v_t - w)^T                     i.e. S_t = (I - b k k^T) Diag(a) S_{t-1} + b k v^T
+ *     out[b,t,h,:] <- scale * S^T q                     (S after the update)
+ *   hT[b,h] := S
+ *
+ * Sources (page title, section / equation):
+ *  - "Complex KDA" paper summary (picx.dev), Background: the gated delta-rule transition
+ *    A_t = (I - beta_t k_t k_t^T) Diag(alpha_t); "CKDA Definition": alpha in [-1,1]^n, beta in [0,2].
+ *  - the recurrence's write term beta k v^T and read-out scale dk^-1/2 * S_t^T q_t complete the
+ *    transition into a layer (the FLA KDA operator the "RoPE into the KDA q/k path" review studies).
+ *  - "RoPE into the KDA q/k path" review, sections 2-3: the q/k L2 norm is a kernel-side step and
+ *    the rotation is applied before it; section 5: inverse frequencies 1/base^(2i/dim).
+ *  - the same review, section 3 (rotate_half, optional interleaved pairing) and the ferrox "mla"
+ *    module doc (interleaved convention): pair layout of the rotation.
+ *
+ * Readings where the pages are silent (each also listed in the design notes):
+ *  - L2 norm epsilon: x / sqrt(sum x^2 + 1e-6); the zero vector stays zero.
+ *  - alpha gates the dk (key) rows of S; Diag(alpha) is applied before the rank-one correction.
+ *  - the output reads S_t, after the update.
+ *  - RoPE position p = pos_offset + t, 0-based.
+ *
+ * Planted mistakes (CKDA_ORACLE_MUTANT=n at compile time) exist only so that the test suite can
+ * prove its pins catch each class of error; the default build (0) is the oracle.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifndef CKDA_ORACLE_MUTANT
+#define CKDA_ORACLE_MUTANT 0
+#endif
+
+/* mutant ids (see tests/test_oracle_mutants.py) */
+#define MUT_DH_ORDER 1      /* apply Diag(alpha) after the Householder-like factor */
+#define MUT_ABS_ALPHA 2     /* drop the sign of alpha */
+#define MUT_BETA_CLAMP 3    /* clamp beta to [0,1] */
+#define MUT_OUT_PREV 4      /* read the output from S_{t-1} */
+#define MUT_NO_SCALE 5      /* forget the dk^-1/2 read-out scale */
+#define MUT_FREQ_NO2 6      /* rope frequency exponent without its factor 2 */
+#define MUT_ROPE_Q_ONLY 7   /* rotate q but not k */
+#define MUT_THETA_1000 8    /* rope base 1000 instead of the given one */
+#define MUT_NO_L2 9         /* skip the L2 norm */
+#define MUT_NORM_AFTER 10   /* L2 norm over q and k jointly instead of per vector */
+
+#define L2_EPS 1e-6
+
+static const int g_mutant = CKDA_ORACLE_MUTANT;
+
+int ckda_oracle_mutant(void) { return g_mutant; }
+
+/* Rotate one head vector x[0..d) in place by position p (see header comment for the pairing). */
+static void rope_rotate(double* x, int d, long long p, double theta, int convention) {
+    if (g_mutant == MUT_THETA_1000) theta = 1000.0;
+    int half = d / 2;
+    for (int i = 0; i < half; ++i) {
+        double expo = (g_mutant == MUT_FREQ_NO2) ? (double)i / (double)d : 2.0 * (double)i / (double)d;
+        double omega = pow(theta, -expo);
+        double phi = (double)p * omega;
+        double c = cos(phi), s = sin(phi);
+        int a, b;
+        if (convention == 0) { a = i; b = i + half; }       /* half-split: (x_i, x_{i+d/2}) */
+        else                 { a = 2 * i; b = 2 * i + 1; }  /* interleaved: (x_{2i}, x_{2i+1}) */
+        double xa = x[a], xb = x[b];
+        x[a] = xa * c - xb * s;
+        x[b] = xb * c + xa * s;
+    }
+}
+
+static void l2_normalise(double* x, int d) {
+    double ss = 0.0;
+    for (int i = 0; i < d; ++i) ss += x[i] * x[i];
+    double r = 1.0 / sqrt(ss + L2_EPS);
+    for (int i = 0; i < d; ++i) x[i] *= r;
+}
+
+/* The q/k prologue for one token of one head: optional rotation, then optional L2 norm. */
+static void prologue_pair(double* q, double* k, int dk, long long p, int l2norm, double theta,
+                          int convention) {
+    if (theta > 0.0) {
+        rope_rotate(q, dk, p, theta, convention);
+        if (g_mutant != MUT_ROPE_Q_ONLY) rope_rotate(k, dk, p, theta, convention);
+    }
+    if (l2norm && g_mutant != MUT_NO_L2) {
+        if (g_mutant == MUT_NORM_AFTER) {
+            double ss = 0.0;
+            for (int i = 0; i < dk; ++i) ss += q[i] * q[i] + k[i] * k[i];
+            double r = 1.0 / sqrt(ss + L2_EPS);
+            for (int i = 0; i < dk; ++i) { q[i] *= r; k[i] *= r; }
+        } else {
+            l2_normalise(q, dk);
+            l2_normalise(k, dk);
+        }
+    }
+}
+
+/* One token of the recurrence on state S (dk x dv, row-major), given prepared q, k. */
+static void recurrence_token(double* S, const double* q, const double* k, const double* v,
+                             const double* alpha, double beta, double scale, int dk, int dv,
+                             double* w, double* o) {
+    if (g_mutant == MUT_BETA_CLAMP && beta > 1.0) beta = 1.0;
+    if (g_mutant == MUT_OUT_PREV) {
+        for (int j = 0; j < dv; ++j) {
+            double acc = 0.0;
+            for (int c = 0; c < dk; ++c) acc += S[(size_t)c * dv + j] * q[c];
+            o[j] = scale * acc;
+        }
+    }
+    if (g_mutant == MUT_DH_ORDER) {
+        /* S <- Diag(a) (I - b k k^T) S + b k v^T  (factors in the wrong order) */
+        for (int j = 0; j < dv; ++j) {
+            double acc = 0.0;
+            for (int c = 0; c < dk; ++c) acc += S[(size_t)c * dv + j] * k[c];
+            w[j] = acc;
+        }
+        for (int c = 0; c < dk; ++c) {
+            double a = alpha[c];
+            for (int j = 0; j < dv; ++j) {
+                double s = S[(size_t)c * dv + j] - beta * k[c] * w[j];
+                S[(size_t)c * dv + j] = a * s + beta * k[c] * v[j];
+            }
+        }
+    } else {
+        /* Diag(alpha_t) S_{t-1} */
+        for (int c = 0; c < dk; ++c) {
+            double a = (g_mutant == MUT_ABS_ALPHA) ? fabs(alpha[c]) : alpha[c];
+            for (int j = 0; j < dv; ++j) S[(size_t)c * dv + j] *= a;
+        }
+        /* w = S^T k */
+        for (int j = 0; j < dv; ++j) {
+            double acc = 0.0;
+            for (int c = 0; c < dk; ++c) acc += S[(size_t)c * dv + j] * k[c];
+            w[j] = acc;
+        }
+        /* S += beta k (v - w)^T */
+        for (int c = 0; c < dk; ++c) {
+            double bk = beta * k[c];
+            for (int j = 0; j < dv; ++j) S[(size_t)c * dv + j] += bk * (v[j] - w[j]);
+        }
+    }
+    if (g_mutant != MUT_OUT_PREV) {
+        for (int j = 0; j < dv; ++j) {
+            double acc = 0.0;
+            for (int c = 0; c < dk; ++c) acc += S[(size_t)c * dv + j] * q[c];
+            o[j] = scale * acc;
+        }
+    }
+    if (g_mutant == MUT_NO_SCALE && scale != 0.0) {
+        for (int j = 0; j < dv; ++j) o[j] /= scale;
+    }
+}
+
+typedef struct {
+    const double *q, *k, *v, *alpha, *beta, *h0;
+    double *out, *hT;
+    int B, T, H, dk, dv, l2norm, convention;
+    double theta, scale;
+    long long pos_offset;
+    int next;                 /* next (b,h) pair to process */
+    pthread_mutex_t lock;
+    int status;
+} fwd_job;
+
+static int take_pair(fwd_job* J) {
+    pthread_mutex_lock(&J->lock);
+    int p = J->next++;
+    pthread_mutex_unlock(&J->lock);
+    return p;
+}
+
+static void* fwd_worker(void* arg) {
+    fwd_job* J = (fwd_job*)arg;
+    int dk = J->dk, dv = J->dv, H = J->H, T = J->T;
+    double* S = (double*)malloc(sizeof(double) * (size_t)dk * dv);
+    double* qb = (double*)malloc(sizeof(double) * dk);
+    double* kb = (double*)malloc(sizeof(double) * dk);
+    double* w = (double*)malloc(sizeof(double) * dv);
+    double* o = (double*)malloc(sizeof(double) * dv);
+    if (!S || !qb || !kb || !w || !o) {
+        J->status = -2;
+        free(S); free(qb); free(kb); free(w); free(o);
+        return NULL;
+    }
+    for (;;) {
+        int pair = take_pair(J);
+        if (pair >= J->B * H) break;
+        int b = pair / H, h = pair % H;
+        size_t sofs = ((size_t)b * H + h) * (size_t)dk * dv;
+        if (J->h0) memcpy(S, J->h0 + sofs, sizeof(double) * (size_t)dk * dv);
+        else memset(S, 0, sizeof(double) * (size_t)dk * dv);
+        for (int t = 0; t < T; ++t) {
+            size_t row = ((size_t)b * T + t) * H + h;
+            memcpy(qb, J->q + row * dk, sizeof(double) * dk);
+            memcpy(kb, J->k + row * dk, sizeof(double) * dk);
+            prologue_pair(qb, kb, dk, J->pos_offset + t, J->l2norm, J->theta, J->convention);
+            recurrence_token(S, qb, kb, J->v + row * dv, J->alpha + row * dk, J->beta[row], J->scale,
+                             dk, dv, w, o);
+            memcpy(J->out + row * dv, o, sizeof(double) * dv);
+        }
+        if (J->hT) memcpy(J->hT + sofs, S, sizeof(double) * (size_t)dk * dv);
+    }
+    free(S); free(qb); free(kb); free(w); free(o);
+    return NULL;
+}
+
+/*
+ * Chunk-free forward over a whole sequence batch.
+ *   q, k, alpha: [B, T, H, dk];  v, out: [B, T, H, dv];  beta: [B, T, H];
+ *   h0, hT: [B, H, dk, dv] (h0 may be NULL for a zero state, hT may be NULL).
+ * Returns 0 on success, -1 on bad arguments, -2 on allocation failure.
+ */
+int ckda_oracle_fwd(const double* q, const double* k, const double* v, const double* alpha,
+                    const double* beta, const double* h0, double* out, double* hT, int B, int T,
+                    int H, int dk, int dv, int l2norm, double rope_theta, int rope_convention,
+                    double scale, long long pos_offset, int nthreads) {
+    if (!q || !k || !v || !alpha || !beta || !out) return -1;
+    if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return -1;
+    if (rope_theta > 0.0 && (dk % 2) != 0) return -1;
+    fwd_job J;
+    J.q = q; J.k = k; J.v = v; J.alpha = alpha; J.beta = beta; J.h0 = h0; J.out = out; J.hT = hT;
+    J.B = B; J.T = T; J.H = H; J.dk = dk; J.dv = dv; J.l2norm = l2norm;
+    J.convention = rope_convention; J.theta = rope_theta; J.scale = scale;
+    J.pos_offset = pos_offset; J.next = 0; J.status = 0;
+    pthread_mutex_init(&J.lock, NULL);
+    int pairs = B * H;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > pairs) nthreads = pairs > 0 ? pairs : 1;
+    pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    if (!th) { pthread_mutex_destroy(&J.lock); return -2; }
+    int started = 0;
+    for (int i = 1; i < nthreads; ++i) {
+        if (pthread_create(&th[i], NULL, fwd_worker, &J) == 0) ++started; else break;
+    }
+    fwd_worker(&J);
+    for (int i = 1; i <= started; ++i) pthread_join(th[i], NULL);
+    free(th);
+    pthread_mutex_destroy(&J.lock);
+    return J.status;
+}
+
+/*
+ * One decode step for N independent sequences: the same token body as the forward, applied
+ * in place to state [N, H, dk, dv] with the rotation at position pos[n] (pos may be NULL when
+ * rope_theta <= 0).  q, k, alpha: [N, H, dk]; v, out: [N, H, dv]; beta: [N, H].
+ */
+int ckda_oracle_decode(const double* q, const double* k, const double* v, const double* alpha,
+                       const double* beta, double* state, double* out, const long long* pos,
+                       int N, int H, int dk, int dv, int l2norm, double rope_theta,
+                       int rope_convention, double scale) {
+    if (!q || !k || !v || !alpha || !beta || !state || !out) return -1;
+    if (rope_theta > 0.0 && (!pos || (dk % 2) != 0)) return -1;
+    double* qb = (double*)malloc(sizeof(double) * dk);
+    double* kb = (double*)malloc(sizeof(double) * dk);
+    double* w = (double*)malloc(sizeof(double) * dv);
+    if (!qb || !kb || !w) { free(qb); free(kb); free(w); return -2; }
+    for (int n = 0; n < N; ++n) {
+        for (int h = 0; h < H; ++h) {
+            size_t row = (size_t)n * H + h;
+            memcpy(qb, q + row * dk, sizeof(double) * dk);
+            memcpy(kb, k + row * dk, sizeof(double) * dk);
+            prologue_pair(qb, kb, dk, rope_theta > 0.0 ? pos[n] : 0, l2norm, rope_theta,
+                          rope_convention);
+            recurrence_token(state + row * (size_t)dk * dv, qb, kb, v + row * dv, alpha + row * dk,
+                             beta[row], scale, dk, dv, w, out + row * dv);
+        }
+    }
+    free(qb); free(kb); free(w);
+    return 0;
+}
+
+/*
+ * The q/k prologue alone on one tensor x [B, T, H, d] -> y: rotation at p = pos_offset + t
+ * (if rope_theta > 0), then the per-head L2 norm (if l2norm).
+ */
+int ckda_oracle_prologue(const double* x, double* y, int B, int T, int H, int d, int l2norm,
+                         double rope_theta, int rope_convention, long long pos_offset) {
+    if (!x || !y || d <= 0) return -1;
+    if (rope_theta > 0.0 && (d % 2) != 0) return -1;
+    double* buf = (double*)malloc(sizeof(double) * d);
+    if (!buf) return -2;
+    for (int b = 0; b < B; ++b)
+        for (int t = 0; t < T; ++t)
+            for (int h = 0; h < H; ++h) {
+                size_t row = ((size_t)b * T + t) * H + h;
+                memcpy(buf, x + row * d, sizeof(double) * d);
+                if (rope_theta > 0.0) rope_rotate(buf, d, pos_offset + t, rope_theta, rope_convention);
+                if (l2norm && g_mutant != MUT_NO_L2) l2_normalise(buf, d);
+                memcpy(y + row * d, buf, sizeof(double) * d);
+            }
+    free(buf);
+    return 0;
+}

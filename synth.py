@@ -1,0 +1,138 @@
+"""Seeded synthetic inputs for the CKDA library, its tests and its benchmark.
+
+This module only draws random numbers and rounds them to the storage types; it holds none of the
+recurrence's arithmetic, and both the CUDA library's tests and the float64 oracle consume what it
+returns.  Draws use numpy's Philox counter-based generator (keyed by seed and tensor id), are
+shaped in float64, rounded to float32 (round-to-nearest-even) and, for bf16 tensors, rounded
+again to bf16 (round-to-nearest-even on the float32 bit pattern).  The oracle reads exactly the
+rounded values.
+
+Workload recipes (gate value distributions of the "Complex KDA" paper summary, "CKDA
+Definition": alpha in [-1, 1]^dk, beta in [0, 2]):
+
+  ``tiny``     q, k, v ~ N(0,1); alpha = s*m, s = +-1 (p = 1/2), m ~ U[0.05, 1]; beta ~ U[0, 2]
+  ``ckda``     alpha = s*exp(-softplus(z)), z ~ N(0,1), |alpha| >= 1e-3; beta = 2*sigmoid(N(0,1))
+  ``kda``      alpha = exp(-softplus(z)) in (0, 1]; beta = sigmoid(N(0,1)) in [0, 1]
+"""
+from __future__ import annotations
+
+import numpy as np
+
+TENSOR_IDS = {"q": 1, "k": 2, "v": 3, "alpha": 4, "beta": 5, "h0": 6, "pos": 7}
+
+
+def _gen(seed: int, tensor: str) -> np.random.Generator:
+    return np.random.Generator(np.random.Philox(key=[int(seed) & (2**64 - 1), TENSOR_IDS[tensor]]))
+
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to bf16 (nearest-even); returns the uint16 bit patterns."""
+    b = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    rounded = (b + 0x7FFF + ((b >> 16) & 1)) >> 16
+    return rounded.astype(np.uint16)
+
+
+def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    return (np.ascontiguousarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def _normal(seed, tensor, shape):
+    return _gen(seed, tensor).standard_normal(size=shape, dtype=np.float64)
+
+
+def _softplus(z):
+    return np.logaddexp(0.0, z)
+
+
+def _sigmoid(z):
+    return 0.5 * (1.0 + np.tanh(0.5 * z))
+
+
+def gates(kind: str, shape_alpha, shape_beta, seed: int):
+    """(alpha float32 [.., dk], beta float32 [..]) for one of the recipes above."""
+    ga, gb = _gen(seed, "alpha"), _gen(seed, "beta")
+    if kind == "tiny":
+        s = np.where(ga.random(size=shape_alpha) < 0.5, -1.0, 1.0)
+        m = ga.uniform(0.05, 1.0, size=shape_alpha)
+        alpha = s * m
+        beta = gb.uniform(0.0, 2.0, size=shape_beta)
+    elif kind == "ckda":
+        z = ga.standard_normal(size=shape_alpha)
+        s = np.where(ga.random(size=shape_alpha) < 0.5, -1.0, 1.0)
+        alpha = s * np.maximum(np.exp(-_softplus(z)), 1e-3)
+        beta = 2.0 * _sigmoid(gb.standard_normal(size=shape_beta))
+    elif kind == "kda":
+        z = ga.standard_normal(size=shape_alpha)
+        alpha = np.exp(-_softplus(z))
+        beta = _sigmoid(gb.standard_normal(size=shape_beta))
+    else:
+        raise ValueError(f"unknown gate recipe {kind!r}")
+    return alpha.astype(np.float32), beta.astype(np.float32)
+
+
+def _activation(seed, tensor, shape, dtype):
+    x = _normal(seed, tensor, shape).astype(np.float32)
+    if dtype == "bf16":
+        bits = f32_to_bf16_bits(x)
+        return bf16_bits_to_f32(bits), bits
+    return x, None
+
+
+def fwd_inputs(B, T, H, dk, dv, *, kind="ckda", dtype="bf16", h0_std=0.0, seed=0):
+    """Inputs of one chunked forward call.
+
+    Returns a dict of numpy arrays: q, k [B,T,H,dk], v [B,T,H,dv] as float32 holding the exact
+    values the library reads (bf16-representable when dtype == "bf16"), their bf16 bit patterns
+    under q_bits/k_bits/v_bits (bf16 only), alpha [B,T,H,dk] float32, beta [B,T,H] float32 and
+    h0 [B,H,dk,dv] float32 (None when h0_std == 0).
+    """
+    d = {}
+    for name, last in (("q", dk), ("k", dk), ("v", dv)):
+        val, bits = _activation(seed, name, (B, T, H, last), dtype)
+        d[name] = val
+        d[name + "_bits"] = bits
+    d["alpha"], d["beta"] = gates(kind, (B, T, H, dk), (B, T, H), seed)
+    if h0_std > 0:
+        d["h0"] = (h0_std * _normal(seed, "h0", (B, H, dk, dv))).astype(np.float32)
+    else:
+        d["h0"] = None
+    d["meta"] = dict(B=B, T=T, H=H, dk=dk, dv=dv, kind=kind, dtype=dtype, seed=seed)
+    return d
+
+
+def decode_inputs(N, H, dk, dv, *, kind="ckda", dtype="bf16", state_std=0.0, seed=0,
+                  with_pos=False, max_pos=65536):
+    """Inputs of one decode step (same conventions as fwd_inputs, without the T axis)."""
+    d = fwd_inputs(N, 1, H, dk, dv, kind=kind, dtype=dtype, seed=seed)
+    out = {}
+    for name in ("q", "k", "v", "alpha"):
+        out[name] = d[name][:, 0]
+    for name in ("q_bits", "k_bits", "v_bits"):
+        out[name] = None if d[name] is None else d[name][:, 0]
+    out["beta"] = d["beta"][:, 0]
+    if state_std > 0:
+        out["state"] = (state_std * _normal(seed, "h0", (N, H, dk, dv))).astype(np.float32)
+    else:
+        out["state"] = np.zeros((N, H, dk, dv), np.float32)
+    out["pos"] = (_gen(seed, "pos").integers(0, max_pos, size=(N,), dtype=np.int64)
+                  if with_pos else None)
+    return out
+
+
+# Named workloads: shapes and recipes of the benchmark and parity configurations.
+WORKLOADS = {
+    # tiny fp32 forward (oracle finishes instantly)
+    "tiny_fp32": dict(B=1, T=64, H=2, dk=16, dv=16, chunk=16, kind="tiny", dtype="f32",
+                      rope_theta=0.0, h0_std=0.0),
+    # 1.3B-layer-shaped forward, CKDA gate range
+    "layer_ckda_bf16": dict(B=2, T=2048, H=16, dk=128, dv=128, chunk=64, kind="ckda",
+                            dtype="bf16", rope_theta=0.0, h0_std=0.0),
+    # same shape, standard KDA gate range
+    "layer_kda_bf16": dict(B=2, T=2048, H=16, dk=128, dv=128, chunk=64, kind="kda",
+                           dtype="bf16", rope_theta=0.0, h0_std=0.0),
+    # long context with RoPE (theta 10000, half-split) and a nonzero initial state
+    "long_rope_bf16": dict(B=1, T=65536, H=16, dk=128, dv=128, chunk=64, kind="ckda",
+                           dtype="bf16", rope_theta=10000.0, h0_std=0.02),
+    # batched decode: 256 sequences x 32 heads, 1024 steps
+    "decode_bf16": dict(N=256, H=32, dk=128, dv=128, steps=1024, kind="ckda", dtype="bf16"),
+}

@@ -1,0 +1,213 @@
+"""Python binding of the B200 CKDA library (``libckda.so``, C ABI in ``include/ckda.h``).
+
+Argument marshalling only: every step of the computation runs in the library's CUDA kernels.
+PyTorch supplies device memory and the current stream.  There is no CPU fallback: if the
+compiled library is missing or no CUDA device is present, the calls raise.
+
+Build the library with ``python -m gated_delta_rule_82_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = ["CkdaError", "library_path", "abi_version", "qk_prologue", "workspace_bytes",
+           "fwd_chunked", "decode_step", "selftest_umma", "PATHS"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libckda.so")
+_lib = None
+
+PATHS = {"auto": 0, "simt": 1, "tc": 2}
+_F32, _BF16 = 0, 1
+
+
+class CkdaError(RuntimeError):
+    def __init__(self, func, status):
+        self.status = status
+        msg = _load().ckda_strerror(status).decode()
+        super().__init__(f"{func} failed: status {status} ({msg})")
+
+
+class _Flags(ctypes.Structure):
+    _fields_ = [("l2norm", ctypes.c_int), ("rope_theta", ctypes.c_float),
+                ("rope_convention", ctypes.c_int), ("scale", ctypes.c_float),
+                ("path", ctypes.c_int)]
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError(f"CKDA CUDA library not built: {_LIB_PATH} is missing "
+                           "(run python -m gated_delta_rule_82_b200.build)")
+    lib = ctypes.CDLL(_LIB_PATH)
+    P, I, LL, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_size_t
+    lib.ckda_abi_version.restype = I
+    lib.ckda_abi_version.argtypes = []
+    lib.ckda_strerror.restype = ctypes.c_char_p
+    lib.ckda_strerror.argtypes = [I]
+    lib.ckda_qk_prologue.restype = I
+    lib.ckda_qk_prologue.argtypes = [P, P, P, P, I, I, I, I, _Flags, I, LL, P]
+    lib.ckda_fwd_workspace_bytes.restype = SZ
+    lib.ckda_fwd_workspace_bytes.argtypes = [I, I, I, I, I, I, I, I]
+    lib.ckda_fwd_chunked.restype = I
+    lib.ckda_fwd_chunked.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, _Flags, I, LL, P,
+                                     SZ, P]
+    lib.ckda_decode_step.restype = I
+    lib.ckda_decode_step.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, _Flags, I, P]
+    lib.ckda_selftest_umma.restype = I
+    lib.ckda_selftest_umma.argtypes = [P, P, P, I, I, I, I, P]
+    _lib = lib
+    return lib
+
+
+def abi_version() -> int:
+    return _load().ckda_abi_version()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return _BF16
+    if t.dtype == torch.float32:
+        return _F32
+    raise TypeError(f"q/k/v must be bfloat16 or float32, got {t.dtype}")
+
+
+def _check(t: torch.Tensor, name: str, dtype=None, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (the library has no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _flags(l2norm, rope_theta, rope_convention, scale, path=0):
+    return _Flags(int(bool(l2norm)), float(rope_theta), int(rope_convention), float(scale),
+                  int(path))
+
+
+def _raise(func, status):
+    if status != 0:
+        raise CkdaError(func, status)
+
+
+def qk_prologue(q, k, *, l2norm=True, rope_theta=0.0, rope_convention=0, pos_offset=0,
+                q_out=None, k_out=None):
+    """Rotation at positions pos_offset + t, then per-head L2 norm, of q and k [B, T, H, dk]."""
+    _check(q, "q")
+    _check(k, "k", dtype=q.dtype, shape=q.shape)
+    B, T, H, dk = q.shape
+    q_out = torch.empty_like(q) if q_out is None else q_out
+    k_out = torch.empty_like(k) if k_out is None else k_out
+    _check(q_out, "q_out", dtype=q.dtype, shape=q.shape)
+    _check(k_out, "k_out", dtype=q.dtype, shape=q.shape)
+    st = _load().ckda_qk_prologue(_ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out), B, T, H, dk,
+                                  _flags(l2norm, rope_theta, rope_convention, 0.0),
+                                  _dtype_code(q), int(pos_offset), _stream(q.device))
+    _raise("ckda_qk_prologue", st)
+    return q_out, k_out
+
+
+def workspace_bytes(B, T, H, dk, dv, chunk=64, dtype=torch.bfloat16, path="auto") -> int:
+    code = _BF16 if dtype == torch.bfloat16 else _F32
+    n = _load().ckda_fwd_workspace_bytes(B, T, H, dk, dv, chunk, code, PATHS[path])
+    if n == ctypes.c_size_t(-1).value:
+        raise ValueError("unsupported problem for ckda_fwd_chunked")
+    return int(n)
+
+
+def fwd_chunked(q, k, v, alpha, beta, h0=None, *, chunk=64, l2norm=True, rope_theta=0.0,
+                rope_convention=0, scale=0.0, pos_offset=0, path="auto", want_state=True,
+                out=None, hT=None, workspace=None):
+    """Chunked CKDA forward.  Returns (out [B, T, H, dv], hT [B, H, dk, dv] or None).
+
+    q, k: [B, T, H, dk] (bf16 or fp32); v: [B, T, H, dv] same dtype; alpha: [B, T, H, dk]
+    fp32; beta: [B, T, H] fp32; h0: [B, H, dk, dv] fp32 or None.
+    """
+    _check(q, "q")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    _check(k, "k", dtype=q.dtype, shape=q.shape)
+    _check(v, "v", dtype=q.dtype, shape=(B, T, H, dv))
+    _check(alpha, "alpha", dtype=torch.float32, shape=(B, T, H, dk))
+    _check(beta, "beta", dtype=torch.float32, shape=(B, T, H))
+    if h0 is not None:
+        _check(h0, "h0", dtype=torch.float32, shape=(B, H, dk, dv))
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    _check(out, "out", dtype=q.dtype, shape=(B, T, H, dv))
+    if want_state and hT is None:
+        hT = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    if hT is not None:
+        _check(hT, "hT", dtype=torch.float32, shape=(B, H, dk, dv))
+    code = _dtype_code(q)
+    need = workspace_bytes(B, T, H, dk, dv, chunk, q.dtype, path)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _load().ckda_fwd_chunked(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(h0), _ptr(out), _ptr(hT),
+        B, T, H, dk, dv, int(chunk), _flags(l2norm, rope_theta, rope_convention, scale,
+                                           PATHS[path]),
+        code, int(pos_offset), _ptr(workspace), wbytes, _stream(q.device))
+    _raise("ckda_fwd_chunked", st)
+    return out, hT
+
+
+def decode_step(q, k, v, alpha, beta, state, pos=None, *, l2norm=True, rope_theta=0.0,
+                rope_convention=0, scale=0.0, out=None):
+    """One decode step, in place on state [N, H, dk, dv] fp32.  Returns out [N, H, dv]."""
+    _check(q, "q")
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    _check(k, "k", dtype=q.dtype, shape=q.shape)
+    _check(v, "v", dtype=q.dtype, shape=(N, H, dv))
+    _check(alpha, "alpha", dtype=torch.float32, shape=(N, H, dk))
+    _check(beta, "beta", dtype=torch.float32, shape=(N, H))
+    _check(state, "state", dtype=torch.float32, shape=(N, H, dk, dv))
+    if pos is not None:
+        _check(pos, "pos", dtype=torch.int64, shape=(N,))
+    if out is None:
+        out = torch.empty((N, H, dv), dtype=q.dtype, device=q.device)
+    _check(out, "out", dtype=q.dtype, shape=(N, H, dv))
+    st = _load().ckda_decode_step(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(state), _ptr(out), _ptr(pos),
+        N, H, dk, dv, _flags(l2norm, rope_theta, rope_convention, scale), _dtype_code(q),
+        _stream(q.device))
+    _raise("ckda_decode_step", st)
+    return out
+
+
+def selftest_umma(A, B, b_mn_major=False):
+    """fp32 A @ B^T (b_mn_major=False, B [N, K]) or A @ B (B [K, N]) via the library's tcgen05
+    wrappers, for bf16 A [M, K] and B."""
+    _check(A, "A", dtype=torch.bfloat16)
+    _check(B, "B", dtype=torch.bfloat16)
+    M, K = A.shape
+    N = B.shape[1] if b_mn_major else B.shape[0]
+    D = torch.empty((M, N), dtype=torch.float32, device=A.device)
+    st = _load().ckda_selftest_umma(_ptr(A), _ptr(B), _ptr(D), M, N, K, int(bool(b_mn_major)),
+                                    _stream(A.device))
+    _raise("ckda_selftest_umma", st)
+    return D

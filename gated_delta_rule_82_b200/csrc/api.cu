@@ -1,0 +1,206 @@
+// api.cu -- the C ABI declared in include/ckda.h: argument validation and dispatch.
+//
+// Everything here runs on the host before any launch.  The library allocates nothing: device
+// memory (inputs, outputs, states, workspace) belongs to the caller.
+#include <math.h>
+#include <string.h>
+
+#include "internal.cuh"
+
+using namespace ckda;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool supported_dim(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+bool supported_chunk(int c) { return c == 16 || c == 32 || c == 64; }
+
+size_t elem_size(ckda_dtype t) { return t == CKDA_BF16 ? 2 : 4; }
+
+// [lo, lo + bytes) intervals intersect?
+bool overlap(const void* a, size_t an, const void* b, size_t bn) {
+    if (!a || !b || an == 0 || bn == 0) return false;
+    uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + bn && y < x + an;
+}
+
+ckda_status make_rope(const ckda_flags& f, int dk, RopeParams* rp) {
+    memset(rp, 0, sizeof(*rp));
+    if (!(f.rope_theta > 0.f)) return CKDA_OK;  // also rejects NaN as "off"
+    if (!isfinite(f.rope_theta)) return CKDA_ERR_ARG;
+    if (f.rope_convention != 0 && f.rope_convention != 1) return CKDA_ERR_ARG;
+    rp->enabled = 1;
+    rp->convention = f.rope_convention;
+    for (int i = 0; i < dk / 2; ++i)
+        rp->inv_freq[i] = pow((double)f.rope_theta, -2.0 * (double)i / (double)dk);
+    return CKDA_OK;
+}
+
+float resolve_scale(const ckda_flags& f, int dk) {
+    return f.scale != 0.f ? f.scale : (float)(1.0 / sqrt((double)dk));
+}
+
+bool tc_eligible(int dk, int dv, int chunk, ckda_dtype dtype) {
+    return dtype == CKDA_BF16 && dk == 128 && dv == 128 && chunk == 64;
+}
+
+// 0 = SIMT, 2 = TC, -1 = unsupported request
+int choose_path(int path, int dk, int dv, int chunk, ckda_dtype dtype) {
+    if (path == CKDA_PATH_SIMT) return CKDA_PATH_SIMT;
+    if (path == CKDA_PATH_TC) return tc_eligible(dk, dv, chunk, dtype) ? CKDA_PATH_TC : -1;
+    if (path == CKDA_PATH_AUTO) return tc_eligible(dk, dv, chunk, dtype) ? CKDA_PATH_TC : CKDA_PATH_SIMT;
+    return -1;
+}
+
+ckda_status from_cuda(cudaError_t e) { return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int ckda_abi_version(void) { return CKDA_ABI_VERSION; }
+
+const char* ckda_strerror(ckda_status s) {
+    switch (s) {
+        case CKDA_OK: return "success";
+        case CKDA_ERR_NULL: return "a required pointer is NULL";
+        case CKDA_ERR_SHAPE: return "a size is out of range";
+        case CKDA_ERR_UNSUPPORTED: return "head size, chunk, dtype or path not supported";
+        case CKDA_ERR_ALIGN: return "an array pointer is not 16-byte aligned";
+        case CKDA_ERR_WORKSPACE: return "workspace missing or too small";
+        case CKDA_ERR_CUDA: return "a CUDA runtime call failed";
+        case CKDA_ERR_ARG: return "invalid argument";
+    }
+    return "unknown status";
+}
+
+ckda_status ckda_qk_prologue(const void* q, const void* k, void* q_out, void* k_out, int B, int T,
+                             int H, int dk, ckda_flags flags, ckda_dtype dtype,
+                             long long pos_offset, ckda_stream_t stream) {
+    if (!q || !k || !q_out || !k_out) return CKDA_ERR_NULL;
+    if (dtype != CKDA_F32 && dtype != CKDA_BF16) return CKDA_ERR_UNSUPPORTED;
+    if (B < 1 || T < 1 || H < 1) return CKDA_ERR_SHAPE;
+    if ((long long)B * T * H * dk > (1ll << 40)) return CKDA_ERR_SHAPE;
+    if (!supported_dim(dk)) return CKDA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(q_out) || !aligned16(k_out)) return CKDA_ERR_ALIGN;
+    size_t bytes = (size_t)B * T * H * dk * elem_size(dtype);
+    // in-place is allowed; partial overlaps and q_out aliasing k are not
+    if ((q_out != q && overlap(q_out, bytes, q, bytes)) || overlap(q_out, bytes, k, bytes) ||
+        (k_out != k && overlap(k_out, bytes, k, bytes)) || overlap(k_out, bytes, q, bytes) ||
+        overlap(q_out, bytes, k_out, bytes))
+        return CKDA_ERR_ARG;
+    RopeParams rp;
+    ckda_status st = make_rope(flags, dk, &rp);
+    if (st != CKDA_OK) return st;
+    return from_cuda(launch_qk_prologue(q, k, q_out, k_out, B, T, H, dk, flags.l2norm ? 1 : 0, rp,
+                                        pos_offset, dtype, (cudaStream_t)stream));
+}
+
+size_t ckda_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, ckda_dtype dtype,
+                                int path) {
+    if (B < 1 || T < 1 || H < 1) return (size_t)-1;
+    if (!supported_dim(dk) || !supported_dim(dv) || !supported_chunk(chunk)) return (size_t)-1;
+    if (dtype != CKDA_F32 && dtype != CKDA_BF16) return (size_t)-1;
+    int p = choose_path(path, dk, dv, chunk, dtype);
+    if (p < 0) return (size_t)-1;
+    if (p == CKDA_PATH_TC) return chunk_tc_workspace_bytes(B, T, H);
+    return 0;
+}
+
+ckda_status ckda_fwd_chunked(const void* q, const void* k, const void* v, const float* alpha,
+                             const float* beta, const float* h0, void* out, float* hT, int B,
+                             int T, int H, int dk, int dv, int chunk, ckda_flags flags,
+                             ckda_dtype dtype, long long pos_offset, void* workspace,
+                             size_t workspace_bytes, ckda_stream_t stream) {
+    if (!q || !k || !v || !alpha || !beta || !out) return CKDA_ERR_NULL;
+    if (dtype != CKDA_F32 && dtype != CKDA_BF16) return CKDA_ERR_UNSUPPORTED;
+    if (B < 1 || T < 1 || H < 1) return CKDA_ERR_SHAPE;
+    if ((long long)B * T * H * 128 > (1ll << 40)) return CKDA_ERR_SHAPE;
+    if ((long long)B * H * ((T + 15) / 16) > 0x7fffffffll) return CKDA_ERR_SHAPE;
+    if (!supported_dim(dk) || !supported_dim(dv) || !supported_chunk(chunk)) return CKDA_ERR_UNSUPPORTED;
+    int p = choose_path(flags.path, dk, dv, chunk, dtype);
+    if (p < 0) return flags.path == CKDA_PATH_TC ? CKDA_ERR_UNSUPPORTED : CKDA_ERR_ARG;
+    const void* ptrs[] = {q, k, v, alpha, beta, h0, out, hT};
+    for (const void* ptr : ptrs)
+        if (ptr && !aligned16(ptr)) return CKDA_ERR_ALIGN;
+    const size_t es = elem_size(dtype);
+    const size_t nqk = (size_t)B * T * H * dk, nv = (size_t)B * T * H * dv;
+    const size_t nst = (size_t)B * H * dk * dv;
+    // outputs must not overlap any input (hT == h0 exactly is allowed: each (b, h) is read
+    // completely before it is written)
+    const void* ins[] = {q, k, v, alpha, beta};
+    const size_t insz[] = {nqk * es, nqk * es, nv * es, nqk * 4, (size_t)B * T * H * 4};
+    for (int i = 0; i < 5; ++i) {
+        if (overlap(out, nv * es, ins[i], insz[i])) return CKDA_ERR_ARG;
+        if (hT && overlap(hT, nst * 4, ins[i], insz[i])) return CKDA_ERR_ARG;
+    }
+    if (hT && overlap(hT, nst * 4, out, nv * es)) return CKDA_ERR_ARG;
+    if (h0 && overlap(h0, nst * 4, out, nv * es)) return CKDA_ERR_ARG;
+    if (h0 && hT && hT != h0 && overlap(hT, nst * 4, h0, nst * 4)) return CKDA_ERR_ARG;
+    RopeParams rp;
+    ckda_status st = make_rope(flags, dk, &rp);
+    if (st != CKDA_OK) return st;
+    const float scale = resolve_scale(flags, dk);
+    const int l2 = flags.l2norm ? 1 : 0;
+    if (p == CKDA_PATH_TC) {
+        size_t need = chunk_tc_workspace_bytes(B, T, H);
+        if (need > 0 && (!workspace || workspace_bytes < need)) return CKDA_ERR_WORKSPACE;
+        if (workspace && !aligned16(workspace)) return CKDA_ERR_ALIGN;
+        const void* all[] = {q, k, v, alpha, beta, h0, out, hT};
+        const size_t allsz[] = {nqk * es, nqk * es, nv * es, nqk * 4, (size_t)B * T * H * 4,
+                                nst * 4, nv * es, nst * 4};
+        for (int i = 0; i < 8; ++i)
+            if (all[i] && overlap(workspace, need, all[i], allsz[i])) return CKDA_ERR_ARG;
+        return from_cuda(launch_chunk_tc(q, k, v, alpha, beta, h0, out, hT, B, T, H, l2, rp,
+                                         scale, pos_offset, workspace, (cudaStream_t)stream));
+    }
+    return from_cuda(launch_chunk_simt(q, k, v, alpha, beta, h0, out, hT, B, T, H, dk, dv, chunk,
+                                       l2, rp, scale, pos_offset, dtype, (cudaStream_t)stream));
+}
+
+ckda_status ckda_decode_step(const void* q, const void* k, const void* v, const float* alpha,
+                             const float* beta, float* state, void* out, const long long* pos,
+                             int N, int H, int dk, int dv, ckda_flags flags, ckda_dtype dtype,
+                             ckda_stream_t stream) {
+    if (!q || !k || !v || !alpha || !beta || !state || !out) return CKDA_ERR_NULL;
+    if (dtype != CKDA_F32 && dtype != CKDA_BF16) return CKDA_ERR_UNSUPPORTED;
+    if (N < 1 || H < 1) return CKDA_ERR_SHAPE;
+    if ((long long)N * H * dk * dv > (1ll << 40)) return CKDA_ERR_SHAPE;
+    if (!supported_dim(dk) || !supported_dim(dv)) return CKDA_ERR_UNSUPPORTED;
+    RopeParams rp;
+    ckda_status st = make_rope(flags, dk, &rp);
+    if (st != CKDA_OK) return st;
+    if (rp.enabled && !pos) return CKDA_ERR_NULL;
+    const void* ptrs[] = {q, k, v, alpha, beta, state, out};
+    for (const void* ptr : ptrs)
+        if (!aligned16(ptr)) return CKDA_ERR_ALIGN;
+    if (rp.enabled && (reinterpret_cast<uintptr_t>(pos) & 7u)) return CKDA_ERR_ALIGN;
+    const size_t es = elem_size(dtype);
+    const size_t nst = (size_t)N * H * dk * dv * 4;
+    const void* ins[] = {q, k, v, alpha, beta};
+    const size_t insz[] = {(size_t)N * H * dk * es, (size_t)N * H * dk * es,
+                           (size_t)N * H * dv * es, (size_t)N * H * dk * 4, (size_t)N * H * 4};
+    for (int i = 0; i < 5; ++i) {
+        if (overlap(out, (size_t)N * H * dv * es, ins[i], insz[i])) return CKDA_ERR_ARG;
+        if (overlap(state, nst, ins[i], insz[i])) return CKDA_ERR_ARG;
+    }
+    if (overlap(state, nst, out, (size_t)N * H * dv * es)) return CKDA_ERR_ARG;
+    return from_cuda(launch_decode(q, k, v, alpha, beta, state, out, rp.enabled ? pos : nullptr,
+                                   N, H, dk, dv, flags.l2norm ? 1 : 0, rp,
+                                   resolve_scale(flags, dk), dtype, (cudaStream_t)stream));
+}
+
+ckda_status ckda_selftest_umma(const void* A, const void* B, float* D, int M, int N, int K,
+                               int b_mn_major, ckda_stream_t stream) {
+    if (!A || !B || !D) return CKDA_ERR_NULL;
+    if (M != 64 && M != 128) return CKDA_ERR_UNSUPPORTED;
+    if (N < 16 || N > 256 || N % 16) return CKDA_ERR_UNSUPPORTED;
+    if (K < 64 || K > 256 || K % 64) return CKDA_ERR_UNSUPPORTED;
+    if (b_mn_major && N % 64) return CKDA_ERR_UNSUPPORTED;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(D)) return CKDA_ERR_ALIGN;
+    return from_cuda(launch_umma_selftest(A, B, D, M, N, K, b_mn_major ? 1 : 0,
+                                          (cudaStream_t)stream));
+}
+
+}  // extern "C"

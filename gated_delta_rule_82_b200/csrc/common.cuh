@@ -1,0 +1,99 @@
+// common.cuh -- small device helpers shared by the CKDA kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ckda.h"
+
+namespace ckda {
+
+constexpr float kL2Eps = 1e-6f;  // x / sqrt(sum x^2 + eps), per head
+constexpr int kMaxHalfDim = 64;  // dk <= 128
+
+// Inverse rotary frequencies omega_i = theta^(-2i/dk), computed in double on the host and
+// passed by value, so that concurrent calls with different bases never share state.
+struct RopeParams {
+    double inv_freq[kMaxHalfDim];
+    int enabled;     // rope_theta > 0
+    int convention;  // 0 half-split, 1 interleaved
+};
+
+// Position angle p * omega, reduced to [-pi, pi] in double, then sin/cos in fp32.  The angle
+// reaches ~6.5e4 rad at 64k tokens: an fp32 product would carry ~4e-3 rad of error there.
+__device__ __forceinline__ void rope_sincos(long long p, double omega, float* s, float* c) {
+    const double two_pi = 6.283185307179586476925286766559;
+    double phi = (double)p * omega;
+    double n = rint(phi * (1.0 / two_pi));
+    float r = (float)fma(-n, two_pi, phi);
+    sincosf(r, s, c);
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+// Sum over aligned groups of G lanes (G a power of two <= 32).
+template <int G>
+__device__ __forceinline__ float group_sum(float x) {
+#pragma unroll
+    for (int o = G / 2; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+// ---- element loads / stores -------------------------------------------------------------
+// Load N consecutive elements (16 bytes total) as floats.
+template <typename T, int N>
+struct Vec16;
+
+template <>
+struct Vec16<float, 4> {
+    __device__ __forceinline__ static void load(const float* p, float* x) {
+        float4 v = *reinterpret_cast<const float4*>(p);
+        x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+    }
+    __device__ __forceinline__ static void store(float* p, const float* x) {
+        *reinterpret_cast<float4*>(p) = make_float4(x[0], x[1], x[2], x[3]);
+    }
+};
+
+template <>
+struct Vec16<__nv_bfloat16, 8> {
+    __device__ __forceinline__ static void load(const __nv_bfloat16* p, float* x) {
+        uint4 v = *reinterpret_cast<const uint4*>(p);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            x[2 * i] = __uint_as_float(w[i] << 16);
+            x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+    __device__ __forceinline__ static void store(__nv_bfloat16* p, const float* x) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+            w[i] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+};
+
+template <typename T>
+struct ElemsPer16 { static constexpr int value = 16 / (int)sizeof(T); };
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T>
+__device__ __forceinline__ T from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+}  // namespace ckda

@@ -1,0 +1,33 @@
+// internal.cuh -- launchers shared between the C-ABI layer and the kernel files.
+#pragma once
+
+#include "common.cuh"
+
+namespace ckda {
+
+cudaError_t launch_qk_prologue(const void* q, const void* k, void* qo, void* ko, int B, int T_len,
+                               int H, int dk, int l2norm, const RopeParams& rp,
+                               long long pos_offset, ckda_dtype dtype, cudaStream_t stream);
+
+cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* alpha,
+                          const float* beta, float* state, void* out, const long long* pos, int N,
+                          int H, int dk, int dv, int l2norm, const RopeParams& rp, float scale,
+                          ckda_dtype dtype, cudaStream_t stream);
+
+cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const float* alpha,
+                              const float* beta, const float* h0, void* out, float* hT, int B,
+                              int T_len, int H, int dk, int dv, int chunk, int l2norm,
+                              const RopeParams& rp, float scale, long long pos_offset,
+                              ckda_dtype dtype, cudaStream_t stream);
+
+// Tensor-core chunked forward (bf16, dk = dv = 128, chunk = 64).
+size_t chunk_tc_workspace_bytes(int B, int T_len, int H);
+cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const float* alpha,
+                            const float* beta, const float* h0, void* out, float* hT, int B,
+                            int T_len, int H, int l2norm, const RopeParams& rp, float scale,
+                            long long pos_offset, void* workspace, cudaStream_t stream);
+
+cudaError_t launch_umma_selftest(const void* A, const void* B, float* D, int M, int N, int K,
+                                 int b_mn_major, cudaStream_t stream);
+
+}  // namespace ckda

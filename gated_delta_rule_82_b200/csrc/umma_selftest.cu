@@ -1,0 +1,104 @@
+// umma_selftest.cu -- one-CTA bf16 GEMM through the library's tcgen05 wrappers.
+//
+// Exercises exactly the pieces the chunked forward relies on: swizzled K-major and MN-major
+// shared-memory tiles written by threads, the shared-memory and instruction descriptors,
+// single-thread tcgen05.mma issue, tcgen05.commit to an mbarrier, and the TMEM read-back for
+// both M = 128 (row m in lane m) and M = 64 (row m in lane (m % 16) + 32 (m / 16)).
+#include "internal.cuh"
+#include "tc_sm100.cuh"
+
+namespace ckda {
+
+namespace {
+
+constexpr int kSelftestTmemCols = 256;
+
+__global__ void __launch_bounds__(128)
+umma_selftest_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16* __restrict__ B,
+                     float* __restrict__ D, int M, int N, int K, int b_mn) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = base;
+    uint8_t* sB = base + (size_t)M * K * 2;
+    __shared__ uint64_t bar;
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int e = tid; e < M * K; e += 128) {
+        int m = e / K, kk = e % K;
+        *reinterpret_cast<__nv_bfloat16*>(sA + tc::sw128_kmajor(m, kk, M)) = A[e];
+    }
+    if (!b_mn) {
+        for (int e = tid; e < N * K; e += 128) {
+            int n = e / K, kk = e % K;
+            *reinterpret_cast<__nv_bfloat16*>(sB + tc::sw128_kmajor(n, kk, N)) = B[e];
+        }
+    } else {
+        for (int e = tid; e < N * K; e += 128) {
+            int kk = e / N, n = e % N;
+            *reinterpret_cast<__nv_bfloat16*>(sB + tc::sw128_mnmajor(kk, n, K)) = B[e];
+        }
+    }
+    tc::fence_proxy_async_smem();
+    if (warp == 0) {
+        tc::tmem_alloc(&tmem_base, kSelftestTmemCols);
+        tc::tmem_relinquish();
+    }
+    if (tid == 0) {
+        tc::mbar_init(&bar, 1);
+        tc::fence_mbar_init();
+        abort_flag = 0;
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tbase = tmem_base;
+
+    if (tid == 0) {
+        const uint32_t idesc = tc::idesc_bf16_f32(M, N, 0, b_mn);
+        const uint32_t a0 = tc::smem_u32(sA), b0 = tc::smem_u32(sB);
+        for (int ks = 0; ks < K / 16; ++ks) {
+            uint64_t ad = tc::smem_desc_sw128(a0 + (ks >> 2) * M * 128 + (ks & 3) * 32, 16, 1024);
+            uint64_t bd = b_mn ? tc::smem_desc_sw128(b0 + ks * 2048, K * 128, 1024)
+                               : tc::smem_desc_sw128(b0 + (ks >> 2) * N * 128 + (ks & 3) * 32, 16, 1024);
+            tc::mma_bf16(tbase, ad, bd, idesc, ks > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(&bar);
+    }
+    tc::mbar_wait(&bar, 0, &abort_flag);
+    tc::tc_fence_after();
+
+    int row = -1;
+    if (M == 128) row = warp * 32 + lane;
+    else if (lane < 16) row = warp * 16 + lane;
+    for (int col = 0; col < N; col += 16) {
+        float v[16];
+        tc::tmem_ld16(tc::tmem_addr(tbase, warp * 32, col), v);
+        tc::tmem_ld_wait();
+        if (row >= 0 && !abort_flag) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) D[(size_t)row * N + col + i] = v[i];
+        }
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tbase, kSelftestTmemCols);
+}
+
+}  // namespace
+
+cudaError_t launch_umma_selftest(const void* A, const void* B, float* D, int M, int N, int K,
+                                 int b_mn_major, cudaStream_t stream) {
+    size_t smem = (size_t)(M + N) * K * 2 + 1024;
+    cudaError_t e = cudaFuncSetAttribute(umma_selftest_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    umma_selftest_kernel<<<1, 128, smem, stream>>>(static_cast<const __nv_bfloat16*>(A),
+                                                   static_cast<const __nv_bfloat16*>(B), D, M, N,
+                                                   K, b_mn_major);
+    return cudaGetLastError();
+}
+
+}  // namespace ckda

@@ -1,0 +1,162 @@
+/*
+ * ckda.h -- C ABI of the B200 (sm_100a) Complex KDA (CKDA) recurrence library.
+ *
+ * The recurrence (per batch b and head h, sequential over tokens t):
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,   S in R^{dk x dv}
+ *     o_t = scale * S_t^T q_t,                                                 scale = dk^-1/2
+ *
+ * with a signed channel-wise gate alpha_t in [-1, 1]^dk and beta_t in [0, 2].  The transition
+ * (I - beta k k^T) Diag(alpha) is the gated delta-rule transition of the "Complex KDA" paper
+ * summary (picx.dev), "Background"; the ranges are its "CKDA Definition".  Before the recurrence
+ * q_t and k_t are optionally rotated (rotary embedding at position pos_offset + t, inverse
+ * frequencies rope_theta^(-2i/dk), "RoPE into the KDA q/k path" review, section 5) and then
+ * L2-normalised per head, x / sqrt(sum x^2 + 1e-6) (the same review, sections 2-3: the norm is
+ * a kernel-side step and the rotation comes before it).
+ *
+ * Conventions shared by every entry point:
+ *  - Every array pointer is CALLER-OWNED DEVICE memory (cudaMalloc / torch) on the current
+ *    device.  The library never allocates, frees or retains memory.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy default stream).
+ *    A returned CKDA_OK means the arguments were valid and the kernels were enqueued; kernel
+ *    execution errors surface at the next synchronisation, as with any CUDA launch.
+ *  - Arguments are validated on the host before anything is launched; on any error nothing is
+ *    launched and no output is touched.  Values are not inspected: NaN/Inf propagate, and
+ *    alpha outside [-1, 1] or beta outside [0, 2] are accepted as given.
+ *  - Array pointers must be 16-byte aligned.  Outputs must not overlap inputs (except the
+ *    decode state, which is updated in place by design).
+ *  - Layouts are dense row-major with the last index fastest:
+ *        q, k, alpha : [B, T, H, dk]     v, out : [B, T, H, dv]     beta : [B, T, H]
+ *        h0, hT, decode state : [B or N, H, dk, dv]  (fp32 always)
+ *    q, k, v, out have the element type `dtype`; alpha, beta and states are fp32.
+ *  - Supported sizes: dk, dv in {16, 32, 64, 128}; chunk in {16, 32, 64}; any T >= 1 (a
+ *    partial last chunk is handled exactly).  B*H, N*H >= 1.
+ */
+#ifndef CKDA_H
+#define CKDA_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define CKDA_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define CKDA_API __attribute__((visibility("default")))
+#else
+#define CKDA_API
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* ckda_stream_t;
+
+typedef enum {
+    CKDA_OK = 0,
+    CKDA_ERR_NULL = 1,        /* a required pointer is NULL */
+    CKDA_ERR_SHAPE = 2,       /* a size is out of range (T < 1, B*H < 1, overflow, ...) */
+    CKDA_ERR_UNSUPPORTED = 3, /* dk, dv, chunk, dtype or path outside the compiled set */
+    CKDA_ERR_ALIGN = 4,       /* an array pointer is not 16-byte aligned */
+    CKDA_ERR_WORKSPACE = 5,   /* workspace NULL or smaller than ckda_fwd_workspace_bytes() */
+    CKDA_ERR_CUDA = 6,        /* a CUDA runtime call failed while configuring or launching */
+    CKDA_ERR_ARG = 7          /* any other invalid argument (flags, overlapping buffers) */
+} ckda_status;
+
+typedef enum {
+    CKDA_F32 = 0,  /* q, k, v, out are float32 */
+    CKDA_BF16 = 1  /* q, k, v, out are bfloat16; all arithmetic accumulates in fp32 */
+} ckda_dtype;
+
+typedef enum {
+    CKDA_PATH_AUTO = 0,  /* tensor-core path where compiled (bf16, dk = dv = 128, chunk = 64) */
+    CKDA_PATH_SIMT = 1,  /* fp32 CUDA-core chunked path, every supported size and dtype */
+    CKDA_PATH_TC = 2     /* tensor-core path (tcgen05); CKDA_ERR_UNSUPPORTED elsewhere */
+} ckda_path;
+
+typedef struct {
+    int l2norm;          /* nonzero: L2-normalise q and k per head, after the rotation */
+    float rope_theta;    /* > 0: rotary base (10000 is the usual); <= 0: no rotation */
+    int rope_convention; /* 0: half-split pairs (x_i, x_{i+dk/2}); 1: interleaved (x_{2i}, x_{2i+1}) */
+    float scale;         /* read-out scale; 0 selects dk^-1/2 */
+    int path;            /* ckda_path; ckda_fwd_chunked only, ignored elsewhere */
+} ckda_flags;
+
+/* Version of this ABI (CKDA_ABI_VERSION of the build). */
+CKDA_API int ckda_abi_version(void);
+
+/* Human-readable text for a status code (static storage, never NULL). */
+CKDA_API const char* ckda_strerror(ckda_status status);
+
+/*
+ * Prologue alone: q_out = L2(rope(q)), k_out = L2(rope(k)) per head, with the rotation at
+ * position pos_offset + t.  q, k, q_out, k_out: [B, T, H, dk] of `dtype` (arithmetic in fp32).
+ * The rotary embedding and the placement of the norm after it follow the "RoPE into the KDA
+ * q/k path" review, sections 2, 3 and 5.  In-place use (q_out == q, k_out == k) is allowed.
+ * dk in {16, 32, 64, 128}.
+ */
+CKDA_API ckda_status ckda_qk_prologue(const void* q, const void* k, void* q_out, void* k_out, int B, int T,
+                             int H, int dk, ckda_flags flags, ckda_dtype dtype,
+                             long long pos_offset, ckda_stream_t stream);
+
+/*
+ * Bytes of device workspace ckda_fwd_chunked needs for this problem and path selection
+ * (`path` as in ckda_flags).  Returns 0 when no workspace is needed, and (size_t)-1 when the
+ * sizes are invalid or unsupported for that path.
+ */
+CKDA_API size_t ckda_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, ckda_dtype dtype,
+                                int path);
+
+/*
+ * Chunked forward over whole sequences.
+ *   q, k   : [B, T, H, dk] dtype          v   : [B, T, H, dv] dtype
+ *   alpha  : [B, T, H, dk] fp32 (signed)  beta: [B, T, H] fp32
+ *   h0     : [B, H, dk, dv] fp32, or NULL for a zero initial state
+ *   out    : [B, T, H, dv] dtype (written)
+ *   hT     : [B, H, dk, dv] fp32 final state, or NULL to skip it (may equal h0: read before write
+ *            is guaranteed per (b, h))
+ *   chunk  : tokens per chunk of the chunked evaluation (16, 32 or 64; the tensor-core path
+ *            needs 64); the result does not depend on it beyond rounding.
+ *   pos_offset : rotary position of token t is pos_offset + t (used when rope_theta > 0).
+ *   workspace / workspace_bytes : device scratch of at least ckda_fwd_workspace_bytes(...),
+ *            16-byte aligned; may be NULL when that is 0.  Owned by the caller; it must not be
+ *            shared by calls that can run concurrently.
+ * The computation is the recurrence above, evaluated chunk by chunk: within a chunk a WY/UT
+ * representation of the product of transitions, across chunks an fp32 state.
+ */
+CKDA_API ckda_status ckda_fwd_chunked(const void* q, const void* k, const void* v, const float* alpha,
+                             const float* beta, const float* h0, void* out, float* hT, int B,
+                             int T, int H, int dk, int dv, int chunk, ckda_flags flags,
+                             ckda_dtype dtype, long long pos_offset, void* workspace,
+                             size_t workspace_bytes, ckda_stream_t stream);
+
+/*
+ * One decode step for N independent sequences, in place on the caller's fp32 state:
+ *   q, k, alpha : [N, H, dk]    v, out : [N, H, dv]    beta : [N, H]
+ *   state       : [N, H, dk, dv] fp32, read and overwritten with S_t
+ *   pos         : [N] int64 rotary positions (required when rope_theta > 0, else ignored)
+ * out = scale * S_t^T q_t, with S_t = (I - beta k k^T) Diag(alpha) S_{t-1} + beta k v^T.
+ * Each head's state is streamed through the SM exactly once (read once, written once).
+ */
+CKDA_API ckda_status ckda_decode_step(const void* q, const void* k, const void* v, const float* alpha,
+                             const float* beta, float* state, void* out, const long long* pos,
+                             int N, int H, int dk, int dv, ckda_flags flags, ckda_dtype dtype,
+                             ckda_stream_t stream);
+
+/*
+ * Diagnostic: D[M, N] (fp32, row-major) = A[M, K] * B for bf16 A (row-major, K contiguous),
+ * computed by the library's own tcgen05 tensor-core wrappers (shared-memory operand
+ * descriptors with the 128-byte swizzle, TMEM accumulator, one CTA).
+ *   b_mn_major == 0: B is [N, K] row-major (K contiguous), D = A B^T  (K-major B operand)
+ *   b_mn_major == 1: B is [K, N] row-major (N contiguous), D = A B    (MN-major B operand)
+ * M in {64, 128}; N a multiple of 16 in [16, 256] (a multiple of 64 when b_mn_major);
+ * K a multiple of 64 in [64, 256].  Lets a user check the tensor-core path on a device.
+ */
+CKDA_API ckda_status ckda_selftest_umma(const void* A, const void* B, float* D, int M, int N, int K,
+                               int b_mn_major, ckda_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CKDA_H */

@@ -1,0 +1,141 @@
+"""The C-ABI library: it loads, exports every entry point its header declares, and validates
+arguments on the host.  CPU only: every call below carries at least one invalid argument, so the
+library rejects it before any launch (nothing here ever reaches a kernel)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_delta_rule_82_b200 as ck
+from gated_delta_rule_82_b200 import build as ckbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ckda.h")
+
+OK, NULL, SHAPE, UNSUP, ALIGN, WORKSPACE, CUDA, ARG = range(8)
+P = 0x10000  # a 16-byte-aligned fake address; never dereferenced (calls fail validation first)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    ckbuild.build()
+    return ck._load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ckda_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for want in ("ckda_fwd_chunked", "ckda_decode_step", "ckda_fwd_workspace_bytes",
+                 "ckda_qk_prologue", "ckda_strerror", "ckda_abi_version"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in ckda.h but not exported"
+
+
+def test_only_declared_symbols_are_exported(lib):
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", ck.library_path()], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l and "ckda" in l}
+    assert exported == set(declared_functions())
+
+
+def test_version_and_strerror(lib):
+    assert ck.abi_version() == 1
+    for s in range(8):
+        assert lib.ckda_strerror(s)
+    assert lib.ckda_strerror(99) == b"unknown status"
+
+
+def flags(**kw):
+    f = dict(l2norm=1, rope_theta=0.0, rope_convention=0, scale=0.0, path=0)
+    f.update(kw)
+    return ck._Flags(f["l2norm"], f["rope_theta"], f["rope_convention"], f["scale"], f["path"])
+
+
+def fwd(lib, q=P, k=2 * P, v=3 * P, a=4 * P, b=5 * P, h0=None, out=6 * P, hT=None, B=1, T=8,
+        H=1, dk=16, dv=16, chunk=16, fl=None, dtype=1, pos=0, ws=None, wsb=0):
+    fl = fl or flags()
+    c = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.ckda_fwd_chunked(c(q), c(k), c(v), c(a), c(b), c(h0), c(out), c(hT), B, T, H, dk,
+                                dv, chunk, fl, dtype, pos, c(ws), wsb, None)
+
+
+# each case is invalid in exactly the stated way
+@pytest.mark.parametrize("kw,want", [
+    (dict(q=None), NULL), (dict(v=None), NULL), (dict(out=None), NULL), (dict(b=None), NULL),
+    (dict(T=0), SHAPE), (dict(B=0), SHAPE), (dict(H=-1), SHAPE),
+    (dict(dk=24), UNSUP), (dict(dv=256), UNSUP), (dict(chunk=128), UNSUP), (dict(dtype=7), UNSUP),
+    (dict(q=P + 8), ALIGN), (dict(a=4 * P + 4), ALIGN), (dict(hT=7 * P + 2), ALIGN),
+    (dict(out=P), ARG),                       # out aliases q
+    (dict(fl=flags(path=2)), UNSUP),          # tensor-core path needs bf16 128/128/64
+    (dict(fl=flags(path=9)), ARG),
+    (dict(fl=flags(rope_theta=1e4, rope_convention=3)), ARG),
+    (dict(dk=128, dv=128, chunk=64, T=64, q=P, k=P * 9, v=P * 17, a=P * 25, b=P * 40,
+          out=P * 50, ws=None), WORKSPACE),   # tensor-core path without workspace
+])
+def test_fwd_validation(lib, kw, want):
+    assert fwd(lib, **kw) == want
+
+
+def test_workspace_query(lib):
+    n = lib.ckda_fwd_workspace_bytes(2, 2048, 16, 128, 128, 64, 1, 0)
+    assert 0 < n < (1 << 40)
+    assert lib.ckda_fwd_workspace_bytes(2, 2048, 16, 128, 128, 64, 1, 1) == 0  # SIMT: none
+    assert lib.ckda_fwd_workspace_bytes(1, 64, 2, 16, 16, 16, 0, 0) == 0
+    bad = ctypes.c_size_t(-1).value
+    assert lib.ckda_fwd_workspace_bytes(1, 64, 2, 16, 16, 16, 0, 2) == bad
+    assert lib.ckda_fwd_workspace_bytes(1, 0, 2, 16, 16, 16, 0, 0) == bad
+    assert lib.ckda_fwd_workspace_bytes(1, 64, 2, 48, 16, 16, 0, 0) == bad
+
+
+def dec(lib, q=P, k=2 * P, v=3 * P, a=4 * P, b=5 * P, st=6 * P, out=7 * P, pos=None, N=2, H=2,
+        dk=16, dv=16, fl=None, dtype=1):
+    fl = fl or flags()
+    c = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.ckda_decode_step(c(q), c(k), c(v), c(a), c(b), c(st), c(out), c(pos), N, H, dk,
+                                dv, fl, dtype, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(st=None), NULL), (dict(q=None), NULL),
+    (dict(fl=flags(rope_theta=1e4)), NULL),   # rotation needs positions
+    (dict(N=0), SHAPE), (dict(dk=8), UNSUP), (dict(dtype=3), UNSUP),
+    (dict(st=6 * P + 4), ALIGN), (dict(out=3 * P), ARG),
+])
+def test_decode_validation(lib, kw, want):
+    assert dec(lib, **kw) == want
+
+
+def test_prologue_validation(lib):
+    c = ctypes.c_void_p
+    f = flags()
+    assert lib.ckda_qk_prologue(None, c(P), c(2 * P), c(3 * P), 1, 4, 1, 16, f, 1, 0, None) == NULL
+    assert lib.ckda_qk_prologue(c(P), c(2 * P), c(3 * P), c(4 * P), 1, 4, 1, 12, f, 1, 0, None) == UNSUP
+    assert lib.ckda_qk_prologue(c(P), c(2 * P), c(3 * P + 2), c(4 * P), 1, 4, 1, 16, f, 1, 0, None) == ALIGN
+    assert lib.ckda_qk_prologue(c(P), c(2 * P), c(2 * P), c(4 * P), 1, 4, 1, 16, f, 1, 0, None) == ARG
+    assert lib.ckda_qk_prologue(c(P), c(2 * P), c(3 * P), c(4 * P), 0, 4, 1, 16, f, 1, 0, None) == SHAPE
+
+
+def test_selftest_validation(lib):
+    c = ctypes.c_void_p
+    assert lib.ckda_selftest_umma(c(P), c(2 * P), None, 64, 64, 64, 0, None) == NULL
+    assert lib.ckda_selftest_umma(c(P), c(2 * P), c(3 * P), 32, 64, 64, 0, None) == UNSUP
+    assert lib.ckda_selftest_umma(c(P), c(2 * P), c(3 * P), 64, 48, 64, 1, None) == UNSUP
+    assert lib.ckda_selftest_umma(c(P), c(2 * P), c(3 * P), 64, 64, 96, 0, None) == UNSUP
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 4, 1, 16)
+    with pytest.raises(ValueError, match="CUDA"):
+        ck.qk_prologue(x, x)

@@ -1,0 +1,163 @@
+"""Tensor-core (tcgen05) chunked forward vs the float64 oracle (GPU).
+
+bf16 q/k/v with fp32 accumulation: max|o - o_ref| / max|o_ref| <= 1e-2, same bound on hT.
+"""
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_82_b200 as ck
+import oracle
+import synth
+from helpers import dev_f32, fwd_case, oracle_fwd, rel_err
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    from gated_delta_rule_82_b200 import build
+    build.build()
+
+
+def run_tc(g, **kw):
+    out, hT = ck.fwd_chunked(g["q"], g["k"], g["v"], g["alpha"], g["beta"], g["h0"], chunk=64,
+                             path="tc", **kw)
+    torch.cuda.synchronize()
+    return out, hT
+
+
+def check(B, T, H, *, kind="ckda", h0_std=0.0, rope=(0.0, 0), pos=0, seed=0, tol=TOL):
+    theta, conv = rope
+    d, g = fwd_case(B, T, H, 128, 128, kind=kind, dtype="bf16", h0_std=h0_std, seed=seed)
+    out, hT = run_tc(g, rope_theta=theta, rope_convention=conv, pos_offset=pos)
+    o_ref, s_ref = oracle_fwd(d, rope_theta=theta, rope_convention=conv, pos_offset=pos)
+    eo, es = rel_err(out, o_ref), rel_err(hT, s_ref)
+    assert eo < tol and es < tol, f"out {eo:.3e} hT {es:.3e}"
+    return eo, es
+
+
+def test_workspace_size():
+    n = ck.workspace_bytes(2, 2048, 16, 128, 128, 64, torch.bfloat16, "tc")
+    assert n == 2 * 16 * 32 * 82432
+
+
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 150, 257])
+def test_tc_ragged(T):
+    check(1, T, 2, h0_std=0.02, seed=T)
+
+
+@pytest.mark.parametrize("kind", ["ckda", "kda"])
+def test_tc_gate_ranges(kind):
+    check(2, 512, 3, kind=kind, h0_std=0.02, seed=3)
+
+
+@pytest.mark.parametrize("conv,pos", [(0, 0), (1, 0), (0, 65000)])
+def test_tc_rope(conv, pos):
+    check(1, 300, 2, rope=(10000.0, conv), pos=pos, h0_std=0.02, seed=7)
+
+
+def test_tc_layer_shape_ckda():
+    """The 1.3B-layer-shaped workload (B=2, T=2048, H=16, dk=dv=128), CKDA gate range, compared
+    element by element over the whole output and final state."""
+    w = synth.WORKLOADS["layer_ckda_bf16"]
+    check(w["B"], w["T"], w["H"], kind=w["kind"], seed=101)
+
+
+def test_tc_layer_shape_kda():
+    w = synth.WORKLOADS["layer_kda_bf16"]
+    check(w["B"], w["T"], w["H"], kind=w["kind"], seed=102)
+
+
+def test_tc_long_rope_sampled_heads():
+    """The long-context workload (T=65536, H=16, RoPE theta 10000 half-split, h0 ~ N(0, 0.02)),
+    run in full on the GPU; the oracle recomputes two of the heads end to end."""
+    w = synth.WORKLOADS["long_rope_bf16"]
+    d, g = fwd_case(w["B"], w["T"], w["H"], 128, 128, kind=w["kind"], dtype="bf16",
+                    h0_std=w["h0_std"], seed=103)
+    out, hT = run_tc(g, rope_theta=w["rope_theta"], rope_convention=0)
+    heads = [0, 11]
+    sub = {key: d[key][:, :, heads] for key in ("q", "k", "v", "alpha", "beta")}
+    sub["h0"] = d["h0"][:, heads]
+    o_ref, s_ref = oracle.fwd(sub["q"], sub["k"], sub["v"], sub["alpha"], sub["beta"], sub["h0"],
+                              rope_theta=w["rope_theta"], rope_convention=0)
+    assert rel_err(out[:, :, heads], o_ref) < TOL
+    assert rel_err(hT[:, heads], s_ref) < TOL
+
+
+def test_tc_matches_simt_path():
+    d, g = fwd_case(1, 200, 2, 128, 128, kind="ckda", dtype="bf16", h0_std=0.02, seed=9)
+    o1, s1 = run_tc(g)
+    o2, s2 = ck.fwd_chunked(g["q"], g["k"], g["v"], g["alpha"], g["beta"], g["h0"], chunk=64,
+                            path="simt")
+    torch.cuda.synchronize()
+    assert rel_err(o1, o2.float().cpu().numpy()) < TOL
+    assert rel_err(s1, s2.cpu().numpy()) < TOL
+
+
+def test_tc_exact_zero_gates_take_the_exact_diagonal_path():
+    """Exact-zero and tiny gates push a 16-row block's gate total below 2^-60, which switches that
+    diagonal block to the exact CUDA-core recomputation; the result must still match."""
+    d, g = fwd_case(1, 192, 2, 128, 128, kind="ckda", dtype="bf16", h0_std=0.02, seed=13)
+    a = d["alpha"]
+    a[:, 5:9] *= 1e-6          # block 0 of chunk 0 collapses (tiny gates)
+    a[:, 70, :, ::3] = 0.0     # exact zeros in chunk 1
+    a[:, 140:160] = np.sign(a[:, 140:160]) * 1e-4  # a whole stretch of strong decay
+    g["alpha"] = dev_f32(a)
+    out, hT = run_tc(g)
+    o_ref, s_ref = oracle_fwd(d)
+    assert rel_err(out, o_ref) < TOL
+    assert rel_err(hT, s_ref) < TOL
+
+
+def test_tc_orthogonal_chain():
+    """|alpha| = 1 and beta = 2 everywhere (every transition orthogonal, Theorem 1): with v = 0
+    the state norm is preserved across 2048 tokens and the output still matches the oracle."""
+    d, g = fwd_case(1, 2048, 2, 128, 128, kind="ckda", dtype="bf16", h0_std=0.05, seed=17)
+    rng = np.random.default_rng(0)
+    a = rng.choice([-1.0, 1.0], size=d["alpha"].shape).astype(np.float32)
+    b = np.full(d["beta"].shape, 2.0, np.float32)
+    d["alpha"], d["beta"] = a, b
+    d["v"] = np.zeros_like(d["v"])
+    d["v_bits"] = np.zeros_like(d["v_bits"])
+    g["alpha"], g["beta"] = dev_f32(a), dev_f32(b)
+    g["v"] = torch.zeros_like(g["v"])
+    out, hT = run_tc(g)
+    o_ref, s_ref = oracle_fwd(d)
+    n0 = np.linalg.norm(d["h0"].reshape(2, -1), axis=1)
+    n1 = np.linalg.norm(hT.cpu().numpy().reshape(2, -1), axis=1)
+    assert np.allclose(n0, n1, rtol=2e-2)
+    assert rel_err(hT, s_ref) < 5e-2  # orthogonal chains keep every rounding error alive
+    assert rel_err(out, o_ref) < 5e-2
+
+
+def test_tc_resume_equals_one_pass():
+    """fwd(T1) then fwd(T2, h0 = hT1, pos_offset = T1) equals fwd(T1 + T2) (RoPE on)."""
+    d, g = fwd_case(1, 320, 2, 128, 128, kind="ckda", dtype="bf16", h0_std=0.02, seed=19)
+    kw = dict(rope_theta=10000.0, rope_convention=0)
+    o_all, s_all = run_tc(g, **kw)
+    t1 = 192
+    part = lambda x: x[:, :t1].contiguous()
+    rest = lambda x: x[:, t1:].contiguous()
+    o1, s1 = ck.fwd_chunked(part(g["q"]), part(g["k"]), part(g["v"]), part(g["alpha"]),
+                            part(g["beta"]), g["h0"], path="tc", **kw)
+    o2, s2 = ck.fwd_chunked(rest(g["q"]), rest(g["k"]), rest(g["v"]), rest(g["alpha"]),
+                            rest(g["beta"]), s1, path="tc", pos_offset=t1, **kw)
+    torch.cuda.synchronize()
+    assert rel_err(torch.cat([o1, o2], 1), o_all.float().cpu().numpy()) < TOL
+    assert rel_err(s2, s_all.cpu().numpy()) < TOL
+
+
+def test_tc_state_in_place():
+    """hT may alias h0: each (batch, head, dv tile) is read before it is written."""
+    d, g = fwd_case(2, 130, 2, 128, 128, kind="ckda", dtype="bf16", h0_std=0.02, seed=23)
+    st = g["h0"].clone()
+    out, _ = ck.fwd_chunked(g["q"], g["k"], g["v"], g["alpha"], g["beta"], st, hT=st, path="tc")
+    torch.cuda.synchronize()
+    o_ref, s_ref = oracle_fwd(d)
+    assert rel_err(out, o_ref) < TOL
+    assert rel_err(st, s_ref) < TOL

@@ -1,0 +1,437 @@
+#!/usr/bin/env python
+"""Benchmark of the CKDA recurrence library on one node.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Headline: chunked-forward throughput (Mtok/s, tokens = B*T) on the 1.3B-layer-shaped workload
+(B=2, T=2048, H=16, dk=dv=128, bf16, chunk 64, CKDA gate range).  One step = one
+ckda_fwd_chunked call over that batch (q/k prologue, gate prep, intra-chunk factors, state pass
+and output: the whole forward path).  Every rank runs its own replica on its own synthetic batch
+(weak scaling, no collective on the data path); rank 0 prints one JSON line with the whole-job
+throughput (all ranks' tokens / the slowest rank's device time).
+
+The line also carries: the roofline of the dominant kernel and of the whole forward (against the
+measured HBM bandwidth), the decode step's HBM throughput on the batched-decode workload, the
+CKDA/KDA-range throughput ratio, an end-to-end figure through the C ABI with host buffers, SM
+clocks sampled during the timed region, and (rank 0, one GPU) the float64 CPU oracle's
+throughput on a bounded sample of the same workload.
+
+--impl reference times that float64 CPU oracle (the only reference implementation there is)
+on the same workload, metric and unit.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "CKDA chunked-fwd Mtok/s (H=16,d=128,bf16) + decode GB/s, % of roofline"
+WORKLOAD = dict(name="layer_ckda_bf16", B=2, T=2048, H=16, dk=128, dv=128, chunk=64,
+                kind="ckda", dtype="bf16")
+# algorithmic bytes per head-token of the forward: q, k, v bf16 + alpha fp32 + beta fp32 + out bf16
+FWD_BYTES_PER_HT = 3 * 256 + 512 + 4 + 256
+INTRA_BYTES_PER_HT = 3 * 256 + 512 + 4          # what the chunk-factor kernel must read
+STATE_BYTES_PER_HT = 256                        # what the state pass must write (plus states)
+N_ROTATE = 4                                    # input sets cycled so no step finds its inputs in L2
+
+
+def parse():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--decode-steps", type=int, default=1024)
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip decode / KDA-ratio / e2e / CPU-baseline legs")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+# ---- clocks ----------------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sms, maxes, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sms.append(float(f[1]))
+                maxes.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sms:
+            return None
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxes),
+                "reasons": sorted(reasons), "samples": len(sms)}
+
+
+# ---- helpers ---------------------------------------------------------------------------------
+
+def event_time_ms(fn, steps, stream):
+    """Device time of `steps` calls of fn, CUDA events recorded on the launching stream."""
+    import torch
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(steps):
+        fn(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gated_delta_rule_82_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel):
+    """DRAM bytes per launch for `kernel` from the committed ncu summary, if the kernel sources
+    are unchanged since that capture (else None)."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    if d.get("source_hash") != kernel_source_hash():
+        return None
+    ent = d.get("kernels", {}).get(kernel)
+    return None if ent is None else ent.get("dram_bytes_per_launch")
+
+
+# ---- the reference arm: float64 CPU oracle ---------------------------------------------------
+
+def cpu_oracle_leg(steps, warmup, budget_s=20.0):
+    """Time the float64 oracle on a bounded sample of the headline workload.  The sample is the
+    first `heads` (batch, head) pairs of the workload over the full sequence length; tokens/s is
+    scaled to the workload's tokens (B*T tokens of H heads each)."""
+    import numpy as np
+    import oracle
+    import synth
+    w = WORKLOAD
+    d = synth.fwd_inputs(w["B"], w["T"], w["H"], w["dk"], w["dv"], kind=w["kind"],
+                         dtype=w["dtype"], seed=4242)
+    cores = os.cpu_count() or 1
+    heads = max(1, min(w["H"], cores))
+    sub = {k: np.ascontiguousarray(d[k][:1, :, :heads]) for k in ("q", "k", "v", "alpha", "beta")}
+    run = lambda: oracle.fwd(sub["q"], sub["k"], sub["v"], sub["alpha"], sub["beta"], None,
+                             nthreads=cores, want_state=True)
+    for _ in range(warmup):
+        run()
+    times = []
+    t_start = time.perf_counter()
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        run()
+        times.append(time.perf_counter() - t0)
+        if time.perf_counter() - t_start > budget_s:
+            break
+    sec = statistics.median(times)
+    head_tokens = w["T"] * heads
+    mtok = head_tokens / w["H"] / sec / 1e6
+    sample = (f"float64 oracle, batch 0 heads 0..{heads - 1} of the workload, T={w['T']}, "
+              f"{len(times)} timed runs, median {sec * 1e3:.1f} ms")
+    return mtok, cores, sample, len(times), sec
+
+
+def reference_main(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    mtok, cores, sample, n, sec = cpu_oracle_leg(max(1, args.steps), max(0, min(args.warmup, 2)),
+                                                 budget_s=120.0)
+    w = WORKLOAD
+    line = {"impl": "reference", "metric": METRIC, "value": round(mtok, 6), "unit": "Mtok/s",
+            "n_gpus": args.gpus, "steps": n, "warmup": args.warmup,
+            "ms_per_step": round(sec * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{w['name']} (B={w['B']},T={w['T']},H={w['H']},"
+                                   f"dk=dv={w['dk']},chunk={w['chunk']},{w['kind']} gates)",
+                       "global_batch": w["B"], "seq_len": w["T"], "parallelism": "host threads"},
+            "cpu_baseline": {"value": round(mtok, 6), "unit": "Mtok/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(mtok, 6), "unit": "Mtok/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---- our arm -----------------------------------------------------------------------------------
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return reference_main(args)
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        print(json.dumps({"metric": METRIC, "error": "no CUDA device"}))
+        return 1
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    from gated_delta_rule_82_b200 import build as ckbuild
+    if rank == 0:
+        ckbuild.build()
+    if world > 1:
+        dist.barrier()
+    import gated_delta_rule_82_b200 as ck
+    import synth
+
+    hbm_peak, tc_peak, peak_src = peaks()
+    w = WORKLOAD
+    B, T, H, dk, dv, C = w["B"], w["T"], w["H"], w["dk"], w["dv"], w["chunk"]
+    stream = torch.cuda.current_stream(dev)
+
+    # ---- inputs: N_ROTATE independent synthetic batches, resident in HBM --------------------
+    sets = [synth.torch_fwd_inputs(B, T, H, dk, dv, kind=w["kind"], dtype=w["dtype"],
+                                   seed=1000 * (rank + 1) + i, device=dev) for i in range(N_ROTATE)]
+    out = torch.empty((B, T, H, dv), dtype=torch.bfloat16, device=dev)
+    hT = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    ws = torch.empty(ck.workspace_bytes(B, T, H, dk, dv, C, torch.bfloat16, "tc"),
+                     dtype=torch.uint8, device=dev)
+
+    def step(i, stages=0, inputs=None):
+        s = (inputs or sets)[i % N_ROTATE]
+        ck.fwd_chunked(s["q"], s["k"], s["v"], s["alpha"], s["beta"], None, chunk=C, path="tc",
+                       out=out, hT=hT, workspace=ws, stages=stages)
+
+    for i in range(max(3, args.warmup)):
+        step(i)
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ms = event_time_ms(step, args.steps, stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    ms_per_step = ms / args.steps
+    if world > 1:
+        t = torch.tensor([ms_per_step], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_per_step = float(t.item())
+    tokens_per_step = B * T * world
+    value = tokens_per_step / (ms_per_step / 1e3) / 1e6
+
+    # ---- per-kernel device times (each stage alone, same stream, same rotation) --------------
+    ms_intra = event_time_ms(lambda i: step(i, stages=1), args.steps, stream) / args.steps
+    ms_state = event_time_ms(lambda i: step(i, stages=2), args.steps, stream) / args.steps
+    ht = B * T * H
+    intra_gbs = ht * INTRA_BYTES_PER_HT / (ms_intra / 1e3) / 1e9
+    state_gbs = (ht * STATE_BYTES_PER_HT) / (ms_state / 1e3) / 1e9
+    path_gbs = ht * FWD_BYTES_PER_HT / (ms_per_step / 1e3) / 1e9
+    dominant = "ckda_tc_intra" if ms_intra >= ms_state else "ckda_tc_state"
+    if dominant == "ckda_tc_intra":
+        achieved, dom_ms, per_launch = intra_gbs, ms_intra, ht * INTRA_BYTES_PER_HT
+    else:
+        achieved, dom_ms, per_launch = state_gbs, ms_state, ht * STATE_BYTES_PER_HT
+    roofline = {"kernel": dominant, "bound": "hbm", "achieved": round(achieved, 1),
+                "peak": hbm_peak, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
+                "traffic": ncu_traffic(dominant), "algorithmic_bytes_per_launch": per_launch,
+                "ms_per_launch": round(dom_ms, 4), "peak_source": peak_src}
+    kernels = {"ckda_tc_intra": {"ms": round(ms_intra, 4), "alg_GBps": round(intra_gbs, 1)},
+               "ckda_tc_state": {"ms": round(ms_state, 4), "alg_GBps": round(state_gbs, 1)}}
+    path_roofline = {"bound": "hbm", "achieved": round(path_gbs, 1), "peak": hbm_peak,
+                     "unit": "GB/s", "frac": round(path_gbs / hbm_peak, 4),
+                     "roofline_mtok_s": round(hbm_peak * 1e9 / (H * FWD_BYTES_PER_HT) / 1e6, 1)}
+
+    extras = {}
+    if not args.no_extras:
+        # ---- KDA gate range at the same shape: CKDA/KDA throughput ratio --------------------
+        kda_sets = [synth.torch_fwd_inputs(B, T, H, dk, dv, kind="kda", dtype="bf16",
+                                           seed=7000 + 10 * rank + i, device=dev)
+                    for i in range(N_ROTATE)]
+        for i in range(3):
+            step(i, inputs=kda_sets)
+        ms_kda = event_time_ms(lambda i: step(i, inputs=kda_sets), args.steps, stream) / args.steps
+        extras["kda_range"] = {"mtok_s": round(B * T / (ms_kda / 1e3) / 1e6, 2),
+                               "ckda_over_kda": round(ms_kda / (ms_per_step if world == 1 else ms / args.steps), 4)}
+        del kda_sets
+
+        # ---- long-context forward with RoPE and an initial state (one call per step) -------
+        wl = synth.WORKLOADS["long_rope_bf16"]
+        L = synth.torch_fwd_inputs(wl["B"], wl["T"], wl["H"], 128, 128, kind="ckda",
+                                   dtype="bf16", h0_std=wl["h0_std"], seed=9000 + rank, device=dev)
+        wsL = torch.empty(ck.workspace_bytes(wl["B"], wl["T"], wl["H"], 128, 128),
+                          dtype=torch.uint8, device=dev)
+        outL = torch.empty_like(L["v"])
+        hL = torch.empty_like(L["h0"])
+        fnL = lambda i: ck.fwd_chunked(L["q"], L["k"], L["v"], L["alpha"], L["beta"], L["h0"],
+                                       rope_theta=wl["rope_theta"], path="tc", out=outL, hT=hL,
+                                       workspace=wsL)
+        for i in range(2):
+            fnL(i)
+        nL = max(3, args.steps // 10)
+        ms_long = event_time_ms(fnL, nL, stream) / nL
+        htL = wl["B"] * wl["T"] * wl["H"]
+        extras["long_context"] = {
+            "workload": "long_rope_bf16 (B=1,T=65536,H=16,dk=dv=128,RoPE 1e4 half-split,h0)",
+            "ms": round(ms_long, 3), "mtok_s": round(wl["B"] * wl["T"] / (ms_long / 1e3) / 1e6, 2),
+            "hbm_frac": round(htL * FWD_BYTES_PER_HT / (ms_long / 1e3) / 1e9 / hbm_peak, 4)}
+        del L, wsL, outL, hL
+
+        # ---- batched decode: 256 sequences x 32 heads, dk = dv = 128 ------------------------
+        wd = synth.WORKLOADS["decode_bf16"]
+        N, Hd, steps_d = wd["N"], wd["H"], args.decode_steps
+        Din = synth.torch_decode_inputs(steps_d, N, Hd, 128, 128, kind="ckda", dtype="bf16",
+                                        seed=5000 + rank, device=dev)
+        state = 0.02 * torch.randn((N, Hd, 128, 128), device=dev)
+        outd = torch.empty((N, Hd, 128), dtype=torch.bfloat16, device=dev)
+        fnD = lambda i: ck.decode_step(Din["q"][i], Din["k"][i], Din["v"][i], Din["alpha"][i],
+                                       Din["beta"][i], state, out=outd)
+        for i in range(3):
+            fnD(i)
+        ms_dec = event_time_ms(fnD, steps_d, stream) / steps_d
+        bytes_step = N * Hd * (2 * 128 * 128 * 4 + 3 * 256 + 512 + 4 + 256)
+        dec_gbs = bytes_step / (ms_dec / 1e3) / 1e9
+        extras["decode"] = {
+            "workload": f"decode_bf16 (N={N},H={Hd},dk=dv=128, {steps_d} sequential steps)",
+            "us_per_step": round(ms_dec * 1e3, 2), "GBps": round(dec_gbs, 1),
+            "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": hbm_peak,
+                         "unit": "GB/s", "frac": round(dec_gbs / hbm_peak, 4),
+                         "traffic": ncu_traffic("decode_kernel"),
+                         "algorithmic_bytes_per_launch": bytes_step}}
+        del Din, state
+
+    # ---- end to end through the C ABI with host buffers --------------------------------------
+    e2e = None
+    if not args.no_extras:
+        host = []
+        for i in range(2):
+            s = sets[i]
+            host.append({k: s[k].cpu().pin_memory() for k in ("q", "k", "v", "alpha", "beta")})
+        out_host = torch.empty((B, T, H, dv), dtype=torch.bfloat16).pin_memory()
+        dev_in = {k: torch.empty_like(sets[0][k]) for k in ("q", "k", "v", "alpha", "beta")}
+        h2d = sum(t.numel() * t.element_size() for t in host[0].values())
+        d2h = out_host.numel() * out_host.element_size()
+
+        def e2e_step(i):
+            hs = host[i % 2]
+            for k in dev_in:
+                dev_in[k].copy_(hs[k], non_blocking=True)
+            ck.fwd_chunked(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["alpha"],
+                           dev_in["beta"], None, chunk=C, path="tc", out=out, hT=hT, workspace=ws)
+            out_host.copy_(out, non_blocking=True)
+
+        for i in range(3):
+            e2e_step(i)
+        n_e2e = max(5, args.steps // 5)
+        ms_e2e = event_time_ms(e2e_step, n_e2e, stream) / n_e2e
+        if world > 1:
+            t = torch.tensor([ms_e2e], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        e2e = {"value": round(B * T * world / (ms_e2e / 1e3) / 1e6, 3), "unit": "Mtok/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": round(ms_e2e, 4)}
+
+    # ---- CPU baseline: the float64 oracle on a bounded sample (rank 0, one GPU) --------------
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_extras:
+        mtok, cores, sample, _, _ = cpu_oracle_leg(20, 1, budget_s=20.0)
+        cpu = {"value": round(mtok, 6), "unit": "Mtok/s", "cores": cores, "kind": "oracle",
+               "sample": sample}
+
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": "Mtok/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": f"{w['name']} (B={B},T={T},H={H},dk=dv={dk},chunk={C},"
+                                   f"{w['kind']} gates, no RoPE, h0=0)",
+                       "global_batch": B * world, "seq_len": T, "heads": H,
+                       "parallelism": f"replicas x{world} (independent batches, no collective)",
+                       "l2": f"{N_ROTATE} input sets rotated per step "
+                             f"({N_ROTATE * 80} MB > 126 MB L2)"},
+            "roofline": roofline, "path_roofline": path_roofline, "kernels": kernels,
+            "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": 2 * args.steps,
+            "clocks": clocks, **extras}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

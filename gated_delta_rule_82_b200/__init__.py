@@ -34,7 +34,7 @@ class CkdaError(RuntimeError):
 class _Flags(ctypes.Structure):
     _fields_ = [("l2norm", ctypes.c_int), ("rope_theta", ctypes.c_float),
                 ("rope_convention", ctypes.c_int), ("scale", ctypes.c_float),
-                ("path", ctypes.c_int)]
+                ("path", ctypes.c_int), ("stages", ctypes.c_int)]
 
 
 def library_path() -> str:
@@ -102,9 +102,9 @@ def _stream(device) -> ctypes.c_void_p:
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
-def _flags(l2norm, rope_theta, rope_convention, scale, path=0):
+def _flags(l2norm, rope_theta, rope_convention, scale, path=0, stages=0):
     return _Flags(int(bool(l2norm)), float(rope_theta), int(rope_convention), float(scale),
-                  int(path))
+                  int(path), int(stages))
 
 
 def _raise(func, status):
@@ -139,7 +139,7 @@ def workspace_bytes(B, T, H, dk, dv, chunk=64, dtype=torch.bfloat16, path="auto"
 
 def fwd_chunked(q, k, v, alpha, beta, h0=None, *, chunk=64, l2norm=True, rope_theta=0.0,
                 rope_convention=0, scale=0.0, pos_offset=0, path="auto", want_state=True,
-                out=None, hT=None, workspace=None):
+                out=None, hT=None, workspace=None, stages=0):
     """Chunked CKDA forward.  Returns (out [B, T, H, dv], hT [B, H, dk, dv] or None).
 
     q, k: [B, T, H, dk] (bf16 or fp32); v: [B, T, H, dv] same dtype; alpha: [B, T, H, dk]
@@ -169,7 +169,7 @@ def fwd_chunked(q, k, v, alpha, beta, h0=None, *, chunk=64, l2norm=True, rope_th
     st = _load().ckda_fwd_chunked(
         _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(h0), _ptr(out), _ptr(hT),
         B, T, H, dk, dv, int(chunk), _flags(l2norm, rope_theta, rope_convention, scale,
-                                           PATHS[path]),
+                                           PATHS[path], stages),
         code, int(pos_offset), _ptr(workspace), wbytes, _stream(q.device))
     _raise("ckda_fwd_chunked", st)
     return out, hT

@@ -138,6 +138,7 @@ ckda_status ckda_fwd_chunked(const void* q, const void* k, const void* v, const 
     if (hT && overlap(hT, nst * 4, out, nv * es)) return CKDA_ERR_ARG;
     if (h0 && overlap(h0, nst * 4, out, nv * es)) return CKDA_ERR_ARG;
     if (h0 && hT && hT != h0 && overlap(hT, nst * 4, h0, nst * 4)) return CKDA_ERR_ARG;
+    if (flags.stages < 0 || flags.stages > 3) return CKDA_ERR_ARG;
     RopeParams rp;
     ckda_status st = make_rope(flags, dk, &rp);
     if (st != CKDA_OK) return st;
@@ -153,7 +154,8 @@ ckda_status ckda_fwd_chunked(const void* q, const void* k, const void* v, const 
         for (int i = 0; i < 8; ++i)
             if (all[i] && overlap(workspace, need, all[i], allsz[i])) return CKDA_ERR_ARG;
         return from_cuda(launch_chunk_tc(q, k, v, alpha, beta, h0, out, hT, B, T, H, l2, rp,
-                                         scale, pos_offset, workspace, (cudaStream_t)stream));
+                                         scale, pos_offset, workspace, flags.stages,
+                                         (cudaStream_t)stream));
     }
     return from_cuda(launch_chunk_simt(q, k, v, alpha, beta, h0, out, hT, B, T, H, dk, dv, chunk,
                                        l2, rp, scale, pos_offset, dtype, (cudaStream_t)stream));

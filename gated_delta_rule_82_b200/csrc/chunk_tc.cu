@@ -752,7 +752,8 @@ size_t chunk_tc_workspace_bytes(int B, int T_len, int H) {
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const float* alpha,
                             const float* beta, const float* h0, void* out, float* hT, int B,
                             int T_len, int H, int l2norm, const RopeParams& rp, float scale,
-                            long long pos_offset, void* workspace, cudaStream_t stream) {
+                            long long pos_offset, void* workspace, int stages,
+                            cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(ckda_tc_intra, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)P1_BYTES);
     if (e != cudaSuccess) return e;
@@ -760,15 +761,21 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const f
     if (e != cudaSuccess) return e;
     const int NT = (T_len + kC - 1) / kC;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
+    if (stages == 0) stages = 3;
+    if (stages & 1) {
     ckda_tc_intra<<<(unsigned)(NT * B * H), 256, P1_BYTES, stream>>>(
         static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
         static_cast<const __nv_bfloat16*>(v), alpha, beta, ws, T_len, H, NT, l2norm, rp,
         pos_offset);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    ckda_tc_state<<<(unsigned)(kNTile * B * H), 160, P2_BYTES, stream>>>(
-        ws, h0, static_cast<__nv_bfloat16*>(out), hT, T_len, H, NT, scale);
-    return cudaGetLastError();
+    }
+    if (stages & 2) {
+        ckda_tc_state<<<(unsigned)(kNTile * B * H), 160, P2_BYTES, stream>>>(
+            ws, h0, static_cast<__nv_bfloat16*>(out), hT, T_len, H, NT, scale);
+        e = cudaGetLastError();
+    }
+    return e;
 }
 
 }  // namespace ckda

@@ -25,7 +25,8 @@ size_t chunk_tc_workspace_bytes(int B, int T_len, int H);
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const float* alpha,
                             const float* beta, const float* h0, void* out, float* hT, int B,
                             int T_len, int H, int l2norm, const RopeParams& rp, float scale,
-                            long long pos_offset, void* workspace, cudaStream_t stream);
+                            long long pos_offset, void* workspace, int stages,
+                            cudaStream_t stream);
 
 cudaError_t launch_umma_selftest(const void* A, const void* B, float* D, int M, int N, int K,
                                  int b_mn_major, cudaStream_t stream);

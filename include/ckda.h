@@ -80,6 +80,10 @@ typedef struct {
     int rope_convention; /* 0: half-split pairs (x_i, x_{i+dk/2}); 1: interleaved (x_{2i}, x_{2i+1}) */
     float scale;         /* read-out scale; 0 selects dk^-1/2 */
     int path;            /* ckda_path; ckda_fwd_chunked only, ignored elsewhere */
+    int stages;          /* ckda_fwd_chunked on the tensor-core path only (profiling aid):
+                            0 or 3 = both kernels; 1 = only the chunk-parallel factor kernel
+                            (fills the workspace); 2 = only the serial state pass (reads a
+                            workspace filled by a stage-1 call with the same arguments) */
 } ckda_flags;
 
 /* Version of this ABI (CKDA_ABI_VERSION of the build). */

@@ -136,3 +136,57 @@ WORKLOADS = {
     # batched decode: 256 sequences x 32 heads, 1024 steps
     "decode_bf16": dict(N=256, H=32, dk=128, dv=128, steps=1024, kind="ckda", dtype="bf16"),
 }
+
+
+# ---- device-side generation for benchmark-sized inputs -----------------------------------------
+# Same recipes as above, drawn with torch's seeded CUDA generator (Philox) so that multi-GB
+# inputs never pass through the host.  Values follow the same distributions but are not the
+# same numbers as the numpy stream; parity tests use the numpy path.
+
+def torch_gates(kind, shape_alpha, shape_beta, gen, device):
+    import torch
+    if kind == "ckda":
+        z = torch.randn(shape_alpha, generator=gen, device=device, dtype=torch.float32)
+        s = torch.where(torch.rand(shape_alpha, generator=gen, device=device) < 0.5, -1.0, 1.0)
+        alpha = s * torch.clamp(torch.exp(-torch.nn.functional.softplus(z)), min=1e-3)
+        beta = 2.0 * torch.sigmoid(torch.randn(shape_beta, generator=gen, device=device))
+    elif kind == "kda":
+        z = torch.randn(shape_alpha, generator=gen, device=device, dtype=torch.float32)
+        alpha = torch.exp(-torch.nn.functional.softplus(z))
+        beta = torch.sigmoid(torch.randn(shape_beta, generator=gen, device=device))
+    elif kind == "tiny":
+        s = torch.where(torch.rand(shape_alpha, generator=gen, device=device) < 0.5, -1.0, 1.0)
+        alpha = s * (0.05 + 0.95 * torch.rand(shape_alpha, generator=gen, device=device))
+        beta = 2.0 * torch.rand(shape_beta, generator=gen, device=device)
+    else:
+        raise ValueError(kind)
+    return alpha.contiguous(), beta.contiguous()
+
+
+def torch_fwd_inputs(B, T, H, dk, dv, *, kind="ckda", dtype="bf16", h0_std=0.0, seed=0,
+                     device="cuda"):
+    import torch
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(seed))
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    d = {}
+    for name, last in (("q", dk), ("k", dk), ("v", dv)):
+        d[name] = torch.randn((B, T, H, last), generator=gen, device=device).to(tdt)
+    d["alpha"], d["beta"] = torch_gates(kind, (B, T, H, dk), (B, T, H), gen, device)
+    d["h0"] = (h0_std * torch.randn((B, H, dk, dv), generator=gen, device=device)
+               if h0_std > 0 else None)
+    return d
+
+
+def torch_decode_inputs(steps, N, H, dk, dv, *, kind="ckda", dtype="bf16", seed=0,
+                        device="cuda"):
+    """Per-step decode inputs for `steps` steps, stacked on a leading axis."""
+    import torch
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(seed))
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    d = {}
+    for name, last in (("q", dk), ("k", dk), ("v", dv)):
+        d[name] = torch.randn((steps, N, H, last), generator=gen, device=device).to(tdt)
+    d["alpha"], d["beta"] = torch_gates(kind, (steps, N, H, dk), (steps, N, H), gen, device)
+    return d

@@ -57,9 +57,10 @@ def test_version_and_strerror(lib):
 
 
 def flags(**kw):
-    f = dict(l2norm=1, rope_theta=0.0, rope_convention=0, scale=0.0, path=0)
+    f = dict(l2norm=1, rope_theta=0.0, rope_convention=0, scale=0.0, path=0, stages=0)
     f.update(kw)
-    return ck._Flags(f["l2norm"], f["rope_theta"], f["rope_convention"], f["scale"], f["path"])
+    return ck._Flags(f["l2norm"], f["rope_theta"], f["rope_convention"], f["scale"], f["path"],
+                     f["stages"])
 
 
 def fwd(lib, q=P, k=2 * P, v=3 * P, a=4 * P, b=5 * P, h0=None, out=6 * P, hT=None, B=1, T=8,
@@ -79,6 +80,7 @@ def fwd(lib, q=P, k=2 * P, v=3 * P, a=4 * P, b=5 * P, h0=None, out=6 * P, hT=Non
     (dict(out=P), ARG),                       # out aliases q
     (dict(fl=flags(path=2)), UNSUP),          # tensor-core path needs bf16 128/128/64
     (dict(fl=flags(path=9)), ARG),
+    (dict(fl=flags(stages=4)), ARG),
     (dict(fl=flags(rope_theta=1e4, rope_convention=3)), ARG),
     (dict(dk=128, dv=128, chunk=64, T=64, q=P, k=P * 9, v=P * 17, a=P * 25, b=P * 40,
           out=P * 50, ws=None), WORKSPACE),   # tensor-core path without workspace

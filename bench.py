@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--no-extras", action="store_true",
                     help="skip decode / KDA-ratio / e2e / CPU-baseline legs")
+    ap.add_argument("--profile-case", choices=["fwd", "decode", "prologue"], default=None,
+                    help="run only a few calls of one entry point (for ncu captures) and exit")
     return ap.parse_args()
 
 
@@ -74,17 +76,20 @@ class ClockSampler:
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index):
-        self.index = index
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
         self.proc = None
         self.lines = []
+        self.error = None
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            cmd = ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                   "-lms", "100"]
+            if self.gpu_id:
+                cmd.insert(1, f"--id={self.gpu_id}")
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT,
+                                         text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
         except Exception:
@@ -117,7 +122,7 @@ class ClockSampler:
                 if val.lower() == "active":
                     reasons.add(name)
         if not sms:
-            return None
+            return {"error": "no clock samples", "raw": self.lines[:3]}
         return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxes),
                 "reasons": sorted(reasons), "samples": len(sms)}
 
@@ -220,6 +225,39 @@ def reference_main(args):
     return 0
 
 
+# ---- profiling cases (a few plain calls, no timing) ----------------------------------------------
+
+def profile_case(case, calls, dev):
+    """A few calls of one entry point on its benchmark workload, for ncu.  The first calls are
+    the ones to capture (ncu -c); nothing is timed or printed."""
+    import torch
+    import gated_delta_rule_82_b200 as ck
+    import synth
+    calls = max(1, calls)
+    if case == "fwd":
+        w = WORKLOAD
+        s = synth.torch_fwd_inputs(w["B"], w["T"], w["H"], w["dk"], w["dv"], kind=w["kind"],
+                                   seed=1, device=dev)
+        ws = torch.empty(ck.workspace_bytes(w["B"], w["T"], w["H"], w["dk"], w["dv"]),
+                         dtype=torch.uint8, device=dev)
+        for _ in range(calls):
+            ck.fwd_chunked(s["q"], s["k"], s["v"], s["alpha"], s["beta"], None, path="tc",
+                           workspace=ws)
+    elif case == "decode":
+        wd = synth.WORKLOADS["decode_bf16"]
+        d = synth.torch_decode_inputs(calls, wd["N"], wd["H"], 128, 128, seed=5, device=dev)
+        state = 0.02 * torch.randn((wd["N"], wd["H"], 128, 128), device=dev)
+        for i in range(calls):
+            ck.decode_step(d["q"][i], d["k"][i], d["v"][i], d["alpha"][i], d["beta"][i], state)
+    else:
+        w = WORKLOAD
+        s = synth.torch_fwd_inputs(w["B"], w["T"], w["H"], w["dk"], w["dv"], seed=1, device=dev)
+        for _ in range(calls):
+            ck.qk_prologue(s["q"], s["k"], rope_theta=10000.0)
+    torch.cuda.synchronize()
+    return 0
+
+
 # ---- our arm -----------------------------------------------------------------------------------
 
 def main():
@@ -250,6 +288,9 @@ def main():
     import gated_delta_rule_82_b200 as ck
     import synth
 
+    if args.profile_case:
+        return profile_case(args.profile_case, args.steps, dev)
+
     hbm_peak, tc_peak, peak_src = peaks()
     w = WORKLOAD
     B, T, H, dk, dv, C = w["B"], w["T"], w["H"], w["dk"], w["dv"], w["chunk"]
@@ -272,7 +313,12 @@ def main():
         step(i)
     torch.cuda.synchronize()
 
-    sampler = ClockSampler(local)
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        gpu_id = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    except Exception:
+        gpu_id = None
+    sampler = ClockSampler(gpu_id)
     sampler.start()
     if world > 1:
         dist.barrier()

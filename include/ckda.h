@@ -159,6 +159,32 @@ CKDA_API ckda_status ckda_decode_step(const void* q, const void* k, const void* 
 CKDA_API ckda_status ckda_selftest_umma(const void* A, const void* B, float* D, int M, int N, int K,
                                int b_mn_major, ckda_stream_t stream);
 
+/*
+ * ckda_fwd_chunked without a caller-supplied workspace (the paper has no counterpart; this is a
+ * deployment convenience).  For callers that cannot allocate device memory where they run the
+ * forward -- inside CUDA-graph stream capture, under a fixed start-up memory pool, or on a
+ * real-time path that must not call cudaMalloc/cudaFree -- the scratch lives in a fixed device
+ * array of CKDA_NOALLOC_MAX_WORKSPACE bytes inside the library, held by every GPU that loads it
+ * until the process exits.  The function allocates nothing.
+ *   Arguments and results: as ckda_fwd_chunked, minus workspace / workspace_bytes.
+ *   Limit: problems whose ckda_fwd_workspace_bytes(...) exceeds CKDA_NOALLOC_MAX_WORKSPACE are
+ *          rejected with CKDA_ERR_WORKSPACE before anything is launched (16 MiB holds 203
+ *          chunk-heads of the tensor-core path: B * H * ceil(T / 64) <= 203).
+ *   Set-up: the first call on a device looks up the array's device address (cudaGetSymbolAddress,
+ *          with that device current); make that first call before any stream capture.
+ *   Sharing: every call uses the same array, which keeps the last call's contents (no part of it
+ *          needs to start at zero).  Calls whose work overlaps on the GPU race on it: issue them
+ *          on one stream, or otherwise order them.
+ */
+#define CKDA_NOALLOC_MAX_WORKSPACE (16u << 20)
+
+CKDA_API ckda_status ckda_fwd_chunked_noalloc(const void* q, const void* k, const void* v,
+                                              const float* alpha, const float* beta,
+                                              const float* h0, void* out, float* hT, int B,
+                                              int T, int H, int dk, int dv, int chunk,
+                                              ckda_flags flags, ckda_dtype dtype,
+                                              long long pos_offset, ckda_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,37 +1,48 @@
 // chunk_tc.cu -- chunked CKDA forward on the sm_100a tensor cores (bf16 q/k/v, dk = dv = 128,
 // chunk C = 64), fp32 accumulation in Tensor Memory and an fp32 inter-chunk state.
 //
-// Chunk algebra (see chunk_simt.cu for the derivation from the transition of the "Complex KDA"
-// paper summary, "Background").  For a chunk with entering state S0 and the per-channel gate
-// products gamma_r = prod_{tau<=r} alpha_tau:
+// Chunk algebra (derived from the transition of the "Complex KDA" paper summary, "Background",
+// A_t = (I - beta_t k_t k_t^T) Diag(alpha_t); see chunk_simt.cu for the derivation).  For a chunk
+// with entering state S0 and per-channel gate products gamma_r = prod_{tau<=r} alpha_tau:
 //     A_rj = beta_r k_r^T Diag(gamma_r/gamma_j) k_j (j < r),  M_rj = q_r^T Diag(gamma_r/gamma_j) k_j (j <= r)
 //     T = (I + A)^-1,  W = T diag(beta) K_gamma,  U~ = T diag(beta) V
-//     Q' = Q_gamma - M W,  O_loc = M U~                       (state-independent, chunk-parallel)
-//     [O; U] = [scale (Q' S0 + O_loc); U~ - W S0],  S_C = Diag(gamma_C) S0 + K_end^T U   (serial)
+//     Q' = Q_gamma - M W,  O_loc = M U~
+//     A_c = Diag(gamma_C) - K_end^T W,   B_c = K_end^T U~          (K_end,j = (gamma_C/gamma_j) k_j)
+// and then, serially over chunks,
+//     O = scale (Q' S0 + O_loc),      S_C = A_c S0 + B_c.
+// Everything above the line is state-independent and runs chunk-parallel; the serial chain is a
+// single 128 x 128 x dv product per chunk.
 //
 // Gates.  The sign of gamma is a parity absorbed into q and k (q' = sigma q, k' = sigma k; the
-// paper's compiled-PyTorch variant, sign-magnitude split of its Proposition 2), so that every
-// ratio gamma_r/gamma_j (j <= r) becomes a product of |alpha| over (j, r].  Those products are
-// formed block-locally on 16-row blocks, never by dividing chunk-long products:
-//   fb_r  = prod |alpha| from the block start to r (inclusive)       <= 1
-//   bb_j  = prod |alpha| over (j, block end]                          <= 1
+// compiled-PyTorch variant of the paper summary's "Implementation", i.e. the sign-magnitude split
+// of its Proposition 2), so every ratio gamma_r/gamma_j (j <= r) is a product of |alpha| over
+// (j, r].  Those products are formed block-locally on 16-row blocks and never by dividing
+// chunk-long products:
+//   fb_r  = prod |alpha| from the block start to r (inclusive)        <= 1
+//   bb_j  = prod |alpha| over (j, block end]                           <= 1
 //   P_I   = block total;  off-diagonal block (I > J):  ratio = fb_r * prod_{J<J'<I} P_J' * bb_j
-// so both GEMM operands stay in [0, 1] and nothing overflows.  Inside a diagonal block the ratio
-// is fb_r / fb_j, which is bounded by 2^60 when the block total is >= 2^-60 (always the case for
-// gates with |alpha| >= 2^-3.75 on average); a block whose total is smaller (exact zeros, very
-// strong decay) is recomputed exactly on CUDA cores with running products.
+// so both GEMM operands of an off-diagonal block lie in [0, 1].  Inside a diagonal block the ratio
+// is fb_r / fb_j, bounded by 2^60 while the block total is >= 2^-60 (gates averaging |alpha| >=
+// 2^-3.75); a block below that (exact zeros, very strong decay) is recomputed exactly on CUDA
+// cores with running products from the inputs in global memory.
 //
-// Kernel 1 (ckda_tc_intra) -- one CTA per (chunk, batch*head), chunk-parallel:
-//   q/k prologue (rotation by an angle recurrence, L2 norm from the unrotated row sums -- the
-//   rotation preserves the norm), gate prep, operand tiles in swizzled shared memory, tcgen05
-//   GEMMs for A and M (4 block-rows), T by blocked forward substitution in fp32, tcgen05 GEMMs for
-//   [W | U~] = T' [K_gamma | V] and M [W | U~].  It writes, per chunk, UMMA-ready images of
-//   [Q'; W] (128 x 128) and K_end^T (128 x 64), the dv tiles of U~ and O_loc, and gamma_C.
-// Kernel 2 (ckda_tc_state) -- one CTA per (dv tile of 32 columns, batch*head), serial over chunks:
-//   1-D bulk (TMA) copies of the chunk's images into a double-buffered stage, then
-//   D1 = [Q'; W] S (tcgen05, M = 128, N = 32, K = 128), the epilogue turns D1 into O (written to
-//   HBM) and U (written transposed to shared memory), D2 = K_end^T U (M = 128, N = 32, K = 64),
-//   and the epilogue updates the fp32 master state held in registers, S = gamma_C * S + D2.
+// Kernel 1 (ckda_tc_intra) -- one CTA of 512 threads per (batch*head, chunk):
+//   A  alpha staged in shared memory; channel pass (thread per channel and 16-row block) forms the
+//      signed block prefix fb (sign = block-local parity), the suffix bb and the block totals;
+//      row pass (thread per row and 16 channels: a RoPE pair of 8-channel groups) loads q, k with
+//      16-byte loads, rotates, normalises, absorbs the signs and writes every operand tile with
+//      16-byte stores: L (k'fb | q'fb per block), the B tiles, K_gamma, K_end, Q_gamma, V.
+//   B  tcgen05: A and M block-rows (M = 64, K = 128) into TMEM; read back by 8 warps.
+//   C  T = (I + A)^-1 by blocked forward substitution in fp32; T' = T diag(beta) in bf16.
+//   D  tcgen05: [W | U~] = T' [K_gamma | V]  (M = 64, N = 2 x 128, MN-major B).
+//   F  tcgen05: M [W | U~] (M = 64) and K_end^T [W | U~] (M = 128, MN-major A).
+//   G  write Q', O_loc, A_c, B_c as UMMA-ready images / dv tiles of the workspace.
+// Kernel 2 (ckda_tc_state) -- one CTA per (batch*head, dv tile of 32 columns), serial over chunks:
+//   a three-stage pipeline of 1-D bulk (TMA) copies of each chunk's A_c, Q', B_c and O_loc; per
+//   chunk one tcgen05 product D_c = A_c S (M = 128, N = 32, K = 128) on the critical path, whose
+//   epilogue adds B_c to form the fp32 master state (one row per thread, in registers) and writes
+//   its bf16 copy for the next product, and one off-path product D_o = Q' S (M = 64) that becomes
+//   the chunk's output.
 #include "internal.cuh"
 #include "tc_sm100.cuh"
 
@@ -42,54 +53,129 @@ namespace {
 constexpr int kC = 64, kDK = 128, kDV = 128, kDVT = 32, kNTile = kDV / kDVT;
 
 // ---- workspace image of one chunk-head (bytes) ------------------------------------------------
-constexpr uint32_t WS_QW = 0;         // [Q'; W] bf16, K-major swizzled, 128 rows x 128
-constexpr uint32_t WS_KE = 32768;     // K_end^T bf16, K-major swizzled, 128 rows x 64
-constexpr uint32_t WS_UO = 49152;     // per dv tile t: U~[64][32] bf16 then O_loc[64][32] bf16
-constexpr uint32_t WS_G = 81920;      // gamma_C fp32 [128]
-constexpr uint32_t WS_CHUNK = 82432;
-constexpr uint32_t WS_UO_TILE = 8192;
+constexpr uint32_t WS_AC = 0;          // A_c bf16, K-major swizzled, 128 rows x 128
+constexpr uint32_t WS_QP = 32768;      // Q'  bf16, K-major swizzled, 64 rows x 128
+constexpr uint32_t WS_TILES = 49152;   // per dv tile t: B_c [128][32] bf16, then O_loc [64][32] bf16
+constexpr uint32_t WS_TILE = 12288;
+constexpr uint32_t WS_TILE_O = 8192;
+constexpr uint32_t WS_CHUNK = WS_TILES + kNTile * WS_TILE;  // 98304
 
 // ---- kernel 1 shared memory (bytes from a 1024-aligned base) ---------------------------------
-constexpr uint32_t P1_QF = 0;         // q' fp32 [64][128]; later Q_gamma
-constexpr uint32_t P1_KF = 32768;     // k' fp32 [64][128]; later T fp32 [64][65], T' bf16, X
-constexpr uint32_t P1_L = 65536;      // L tile bf16 K-major 128 x 128; later A fp32 [64][65], M bf16
-constexpr uint32_t P1_B = 98304;      // B tiles (16+32+48+64 rows x 128); later [W|U~] MN-major
-constexpr uint32_t P1_KV = 139264;    // [K_gamma | V] MN-major, 64 K-rows x 256
-constexpr uint32_t P1_SM = 172032;    // small arrays
-constexpr uint32_t P1_BYTES = P1_SM + 8192 + 1024;
+constexpr uint32_t S_FB = 0;         // alpha, then signed fb (fp32 [64][128]); later A, T, M, T', X
+constexpr uint32_t S_BB = 32768;     // bb (fp32 [64][128])
+constexpr uint32_t S_L = 65536;      // L tile (K-major, 128 rows); later W and U~ tiles (MN-major)
+constexpr uint32_t S_B = 98304;      // B tiles (16 + 32 + 48 + 64 rows); later fallback scratch
+constexpr uint32_t S_KG = 139264;    // K_gamma (MN-major, 64 K-rows x 128)
+constexpr uint32_t S_V = 155648;     // V (MN-major, 64 x 128)
+constexpr uint32_t S_KE = 172032;    // K_end (MN-major, 64 x 128): the MN-major A of K_end^T
+constexpr uint32_t S_QG = 188416;    // Q_gamma (K-major, 64 rows x 128)
+constexpr uint32_t S_SM = 204800;    // small arrays (below)
+constexpr uint32_t S_BYTES = S_SM + 10240 + 1024;
 
-constexpr uint32_t P1_T = P1_KF;              // fp32 [64][65]
-constexpr uint32_t P1_TB = P1_KF + 17408;     // T' bf16 K-major 64 x 64 (8 KB)
-constexpr uint32_t P1_X = P1_KF + 26624;      // fp32 [16][48]
-constexpr uint32_t P1_A = P1_L;               // fp32 [64][65]
-constexpr uint32_t P1_M = P1_L + 17408;       // M bf16 K-major 64 x 64 (8 KB)
-constexpr uint32_t P1_WU = P1_B;              // [W | U~] MN-major 64 K-rows x 256 (32 KB)
+constexpr int kStrideA = 68;                     // fp32 row stride of A and T
+constexpr uint32_t S_A = 0;                      // A  fp32 [64][68]
+constexpr uint32_t S_T = 17408;                  // T  fp32 [64][68]
+constexpr uint32_t S_M = 35840;                  // M  bf16 K-major 64 x 64
+constexpr uint32_t S_TB = 44032;                 // T' bf16 K-major 64 x 64
+constexpr uint32_t S_X = 52224;                  // X  fp32 [16][48]
+constexpr uint32_t S_W = S_L;                    // W  MN-major 64 x 128
+constexpr uint32_t S_U = S_L + 16384;            // U~ MN-major 64 x 128
+constexpr uint32_t S_FQ = S_B;                   // fallback q' fp32 [16][128]
+constexpr uint32_t S_FK = S_B + 8192;            // fallback k' fp32 [16][128]
+// small arrays
+constexpr uint32_t SM_P = S_SM;                  // P   fp32 [4][128]  block totals
+constexpr uint32_t SM_PAR = S_SM + 2048;         // PAR fp32 [4][128]  block parity (+-1)
+constexpr uint32_t SM_GC = S_SM + 4096;          // gamma_C fp32 [128]
+constexpr uint32_t SM_B = S_SM + 4608;           // beta fp32 [64]
+constexpr uint32_t SM_FLAGS = S_SM + 4864;       // int unsafe[4], abort, tmem slot, mbarrier
+
 __host__ __device__ constexpr uint32_t btile_off(int I) { return I == 0 ? 0u : I == 1 ? 4096u : I == 2 ? 12288u : 24576u; }
 __host__ __device__ constexpr uint32_t amcol(int I) { return I == 0 ? 0u : I == 1 ? 16u : I == 2 ? 48u : 96u; }
-constexpr int kStrideA = 65;
 
 constexpr float kDiagSafe = 8.673617379884035e-19f;  // 2^-60
 
-__device__ __forceinline__ void st_bf16(uint8_t* base, uint32_t off, float x) {
-    *reinterpret_cast<__nv_bfloat16*>(base + off) = __float2bfloat16_rn(x);
-}
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
     return *reinterpret_cast<uint32_t*>(&h);
 }
-// 8 floats -> one 16-byte chunk of bf16
 __device__ __forceinline__ uint4 pack8(const float* x) {
     return make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
                       pack_bf16(x[6], x[7]));
 }
+__device__ __forceinline__ void unpack8(uint4 v, float* x) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        x[2 * i] = __uint_as_float(w[i] << 16);
+        x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+__device__ __forceinline__ void st16(uint8_t* base, uint32_t off, const float* x) {
+    *reinterpret_cast<uint4*>(base + off) = pack8(x);
+}
+__device__ __forceinline__ void ld_f8(const float* p, float* x) {
+    float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
 
 __device__ int g_tc_error;  // nonzero after a bounded wait ran out (diagnostic)
 
-__device__ __forceinline__ float bf16_at(const __nv_bfloat16* p, size_t i) {
-    return __bfloat162float(p[i]);
+// Recompute one row of q' and k' (rotation, L2 norm, chunk-local sign parity) straight from the
+// inputs; used only by the exact fallback of a collapsed diagonal block.  One warp per row.
+__device__ void fallback_row(const __nv_bfloat16* q, const __nv_bfloat16* k, const float* alpha,
+                             size_t row0, size_t rs, int r, int lane, const RopeParams& rp,
+                             long long pos, int l2norm, float* fq, float* fk) {
+    float qv[4], kv[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const int c = lane + 32 * m;
+        qv[m] = __bfloat162float(q[(row0 + (size_t)r * rs) * kDK + c]);
+        kv[m] = __bfloat162float(k[(row0 + (size_t)r * rs) * kDK + c]);
+    }
+    if (rp.enabled) {
+        float qn[4], kn[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const int c = lane + 32 * m;
+            int i;
+            bool first;
+            float qp, kp;
+            if (rp.convention == 0) {   // partner c ^ 64: same lane, m ^ 2
+                i = c & 63; first = c < 64; qp = qv[m ^ 2]; kp = kv[m ^ 2];
+            } else {                    // partner c ^ 1: neighbouring lane
+                i = c >> 1; first = (c & 1) == 0;
+                qp = __shfl_xor_sync(0xffffffffu, qv[m], 1);
+                kp = __shfl_xor_sync(0xffffffffu, kv[m], 1);
+            }
+            float sn, cs;
+            rope_sincos(pos, rp.inv_freq[i], &sn, &cs);
+            qn[m] = first ? qv[m] * cs - qp * sn : qv[m] * cs + qp * sn;
+            kn[m] = first ? kv[m] * cs - kp * sn : kv[m] * cs + kp * sn;
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m) { qv[m] = qn[m]; kv[m] = kn[m]; }
+    }
+    if (l2norm) {
+        float a = 0.f, b = 0.f;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) { a += qv[m] * qv[m]; b += kv[m] * kv[m]; }
+        a = rsqrtf(warp_sum(a) + kL2Eps);
+        b = rsqrtf(warp_sum(b) + kL2Eps);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) { qv[m] *= a; kv[m] *= b; }
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const int c = lane + 32 * m;
+        float sg = 1.f;
+        for (int tau = 0; tau <= r; ++tau)
+            if (alpha[(row0 + (size_t)tau * rs) * kDK + c] < 0.f) sg = -sg;
+        fq[c] = sg * qv[m];
+        fk[c] = sg * kv[m];
+    }
 }
 
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(512, 1)
 ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
               const __nv_bfloat16* __restrict__ v, const float* __restrict__ alpha,
               const float* __restrict__ beta, uint8_t* __restrict__ ws, int T_len, int H, int NT,
@@ -97,13 +183,13 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float* QF = reinterpret_cast<float*>(sm + P1_QF);
-    float* KF = reinterpret_cast<float*>(sm + P1_KF);
-    float* gP = reinterpret_cast<float*>(sm + P1_SM);          // [4][128]
-    float* gS = gP + 512;                                      // [4][128]
-    float* red = gS + 512;                                     // [4][2][32]
-    float* sb = red + 256;                                     // [64]
-    int* unsafe = reinterpret_cast<int*>(sb + 64);             // [4]
+    float* FB = reinterpret_cast<float*>(sm + S_FB);
+    float* BB = reinterpret_cast<float*>(sm + S_BB);
+    float* gP = reinterpret_cast<float*>(sm + SM_P);
+    float* gPar = reinterpret_cast<float*>(sm + SM_PAR);
+    float* gGC = reinterpret_cast<float*>(sm + SM_GC);
+    float* sb = reinterpret_cast<float*>(sm + SM_B);
+    int* unsafe = reinterpret_cast<int*>(sm + SM_FLAGS);
     volatile int* abort_flag = unsafe + 4;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(unsafe + 8);
     uint64_t* bar = reinterpret_cast<uint64_t*>(unsafe + 16);
@@ -114,10 +200,11 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
     const int t0 = ch * kC;
     const int nvalid = min(kC, T_len - t0);
     uint8_t* wsc = ws + ((size_t)bh * NT + ch) * WS_CHUNK;
-    auto grow = [&](int r) -> size_t { return ((size_t)b * T_len + t0 + r) * H + h; };
+    const size_t row0 = ((size_t)b * T_len + t0) * H + h;  // row (b, t0, h) of [B*T*H]
+    const size_t rs = (size_t)H;                            // stride between tokens, in rows
 
     if (warp == 0) {
-        tc::tmem_alloc(tmem_slot, 256);
+        tc::tmem_alloc(tmem_slot, 512);
         tc::tmem_relinquish();
     }
     if (tid == 32) {
@@ -126,195 +213,192 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
         *abort_flag = 0;
     }
     if (tid < 4) unsafe[tid] = 0;
-    if (tid < 64) sb[tid] = tid < nvalid ? beta[grow(tid)] : 0.f;
+    if (tid < 64) sb[tid] = tid < nvalid ? beta[row0 + tid * rs] : 0.f;
 
-    // ======== phase A: per-thread channel pair (ca, cb) x 16-row block I ========
-    const int p = tid & 63, I = tid >> 6, r0 = 16 * I;
-    const bool inter = rp.enabled && rp.convention == 1;
-    const int ca = inter ? 2 * p : p, cb = inter ? 2 * p + 1 : p + 64;
-    uint8_t* KV = sm + P1_KV;
-    uint8_t* Lt = sm + P1_L;
-    uint8_t* Bt = sm + P1_B;
-
-    // V into the MN-major [K_gamma | V] tile (N offset 128)
-#pragma unroll 4
-    for (int rl = 0; rl < 16; ++rl) {
-        int r = r0 + rl;
-        float va = 0.f, vb = 0.f;
-        if (r < nvalid) {
-            va = bf16_at(v, grow(r) * kDV + ca);
-            vb = bf16_at(v, grow(r) * kDV + cb);
-        }
-        st_bf16(KV, tc::sw128_mnmajor(r, 128 + ca, 64), va);
-        st_bf16(KV, tc::sw128_mnmajor(r, 128 + cb, 64), vb);
+    // ======== A1: alpha into shared memory (identity gates on padding rows), V tile ========
+    for (int e = tid; e < 64 * 32; e += 512) {
+        const int r = e >> 5, c4 = (e & 31) * 4;
+        float4 a = make_float4(1.f, 1.f, 1.f, 1.f);
+        if (r < nvalid) a = *reinterpret_cast<const float4*>(alpha + (row0 + r * rs) * kDK + c4);
+        *reinterpret_cast<float4*>(FB + r * 128 + c4) = a;
     }
-
-    float qa[16], qb[16], ka[16], kb[16];
-#pragma unroll
-    for (int rl = 0; rl < 16; ++rl) {
-        int r = r0 + rl;
-        if (r < nvalid) {
-            size_t o = grow(r) * kDK;
-            qa[rl] = bf16_at(q, o + ca); qb[rl] = bf16_at(q, o + cb);
-            ka[rl] = bf16_at(k, o + ca); kb[rl] = bf16_at(k, o + cb);
-        } else {
-            qa[rl] = qb[rl] = ka[rl] = kb[rl] = 0.f;
-        }
-    }
-    // row sums of squares (the rotation preserves them): transposed butterfly, lane l ends
-    // with the warp total of value l (l < 16: q row l, else k row l - 16)
-    {
-        float x[32];
-#pragma unroll
-        for (int rl = 0; rl < 16; ++rl) {
-            x[rl] = qa[rl] * qa[rl] + qb[rl] * qb[rl];
-            x[16 + rl] = ka[rl] * ka[rl] + kb[rl] * kb[rl];
-        }
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) {
-            const bool upper = (lane & o) != 0;
-#pragma unroll
-            for (int i = 0; i < o; ++i) {
-                float send = upper ? x[i] : x[i + o];
-                float keep = upper ? x[i + o] : x[i];
-                x[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-            }
-        }
-        red[(I * 2 + (warp & 1)) * 32 + lane] = x[0];
-    }
-    if (rp.enabled) {
-        const double om = rp.inv_freq[p];
-        float sn, cs, s1, c1;
-        rope_sincos(pos_offset + t0 + r0, om, &sn, &cs);
-        rope_sincos(1, om, &s1, &c1);
-#pragma unroll
-        for (int rl = 0; rl < 16; ++rl) {
-            float x0 = qa[rl], x1 = qb[rl];
-            qa[rl] = x0 * cs - x1 * sn; qb[rl] = x1 * cs + x0 * sn;
-            x0 = ka[rl]; x1 = kb[rl];
-            ka[rl] = x0 * cs - x1 * sn; kb[rl] = x1 * cs + x0 * sn;
-            float cn = cs * c1 - sn * s1;
-            sn = sn * c1 + cs * s1;
-            cs = cn;
-        }
+    for (int e = tid; e < 64 * 16; e += 512) {
+        const int r = e >> 4, n8 = (e & 15) * 8;
+        uint4 x = make_uint4(0, 0, 0, 0);
+        if (r < nvalid) x = *reinterpret_cast<const uint4*>(v + (row0 + r * rs) * kDV + n8);
+        *reinterpret_cast<uint4*>(sm + S_V + tc::sw128_mnmajor(r, n8, 64)) = x;
     }
     __syncthreads();
-    if (l2norm) {
-#pragma unroll
-        for (int rl = 0; rl < 16; ++rl) {
-            float sq = red[(I * 2) * 32 + rl] + red[(I * 2 + 1) * 32 + rl];
-            float sk = red[(I * 2) * 32 + 16 + rl] + red[(I * 2 + 1) * 32 + 16 + rl];
-            float fq = rsqrtf(sq + kL2Eps), fk = rsqrtf(sk + kL2Eps);
-            qa[rl] *= fq; qb[rl] *= fq; ka[rl] *= fk; kb[rl] *= fk;
-        }
-    }
 
-    // gates: block-prefix fb (inclusive), block-suffix bb (exclusive), block totals; the
-    // block-local sign parity is absorbed into q and k at once
-    float faa[16], fab[16], bba[16], bbb[16];
+    // ======== A2: channel pass -- thread (channel c, block I) ========
     {
-        float aa[16], ab[16];
-#pragma unroll
-        for (int rl = 0; rl < 16; ++rl) {
-            int r = r0 + rl;
-            if (r < nvalid) {
-                aa[rl] = alpha[grow(r) * kDK + ca];
-                ab[rl] = alpha[grow(r) * kDK + cb];
-            } else {
-                aa[rl] = ab[rl] = 1.f;
-            }
-        }
-        float pa = 1.f, pb = 1.f, sa = 1.f, sbb = 1.f;
-#pragma unroll
-        for (int rl = 0; rl < 16; ++rl) {
-            pa *= fabsf(aa[rl]); pb *= fabsf(ab[rl]);
-            sa = aa[rl] < 0.f ? -sa : sa;
-            sbb = ab[rl] < 0.f ? -sbb : sbb;
-            faa[rl] = pa; fab[rl] = pb;
-            qa[rl] *= sa; ka[rl] *= sa; qb[rl] *= sbb; kb[rl] *= sbb;
-        }
-        float ba = 1.f, bbv = 1.f;
+        const int c = tid & 127, I = tid >> 7;
+        float bbv = 1.f;
 #pragma unroll
         for (int rl = 15; rl >= 0; --rl) {
-            bba[rl] = ba; bbb[rl] = bbv;
-            ba *= fabsf(aa[rl]); bbv *= fabsf(ab[rl]);
+            const int r = 16 * I + rl;
+            BB[r * 128 + c] = bbv;
+            bbv *= fabsf(FB[r * 128 + c]);
         }
-        gP[I * 128 + ca] = pa; gP[I * 128 + cb] = pb;
-        gS[I * 128 + ca] = sa; gS[I * 128 + cb] = sbb;
-        if (!(pa >= kDiagSafe) || !(pb >= kDiagSafe)) unsafe[I] = 1;
+        float p = 1.f;
+        bool neg = false;
+#pragma unroll
+        for (int rl = 0; rl < 16; ++rl) {
+            const int r = 16 * I + rl;
+            const float a = FB[r * 128 + c];
+            p *= fabsf(a);
+            neg ^= (a < 0.f);
+            FB[r * 128 + c] = neg ? -p : p;   // a signed zero keeps the parity when p underflows
+        }
+        gP[I * 128 + c] = p;
+        gPar[I * 128 + c] = neg ? -1.f : 1.f;
+        if (!(p >= kDiagSafe)) unsafe[I] = 1;
     }
     __syncthreads();
 
-    // cross-block prefixes: magnitude before / after this block, parity before it, totals
-    float preA = 1.f, preB = 1.f, sufA = 1.f, sufB = 1.f, spA = 1.f, spB = 1.f;
-    float allA = 1.f, allB = 1.f, salA = 1.f, salB = 1.f;
-#pragma unroll
-    for (int J = 0; J < 4; ++J) {
-        float PA = gP[J * 128 + ca], PB = gP[J * 128 + cb];
-        float SA = gS[J * 128 + ca], SB = gS[J * 128 + cb];
-        allA *= PA; allB *= PB; salA *= SA; salB *= SB;
-        if (J < I) { preA *= PA; preB *= PB; spA *= SA; spB *= SB; }
-        if (J > I) { sufA *= PA; sufB *= PB; }
-    }
-    const bool diag_ok = !unsafe[I];
-    float gA[16], gB[16];  // |gamma_r| for Q_gamma, kept until phase C
-#pragma unroll
-    for (int rl = 0; rl < 16; ++rl) {
-        const int r = r0 + rl;
-        const float qpa = spA * qa[rl], qpb = spB * qb[rl];
-        const float kpa = spA * ka[rl], kpb = spB * kb[rl];
-        QF[r * 128 + ca] = qpa; QF[r * 128 + cb] = qpb;
-        KF[r * 128 + ca] = kpa; KF[r * 128 + cb] = kpb;
-        // A/M left operands: rows 32I + rl (k) and 32I + 16 + rl (q)
-        st_bf16(Lt, tc::sw128_kmajor(32 * I + rl, ca, 128), kpa * faa[rl]);
-        st_bf16(Lt, tc::sw128_kmajor(32 * I + rl, cb, 128), kpb * fab[rl]);
-        st_bf16(Lt, tc::sw128_kmajor(32 * I + 16 + rl, ca, 128), qpa * faa[rl]);
-        st_bf16(Lt, tc::sw128_kmajor(32 * I + 16 + rl, cb, 128), qpb * fab[rl]);
-        // right operand of the diagonal block I
-        {
-            const int n = 16 * (I + 1);
-            float da = diag_ok ? kpa / faa[rl] : 0.f, db = diag_ok ? kpb / fab[rl] : 0.f;
-            st_bf16(Bt + btile_off(I), tc::sw128_kmajor(r, ca, n), da);
-            st_bf16(Bt + btile_off(I), tc::sw128_kmajor(r, cb, n), db);
-        }
-        // right operands of the off-diagonal blocks (I2 > I)
-        float midA = 1.f, midB = 1.f;
-#pragma unroll
-        for (int I2 = 1; I2 < 4; ++I2) {
-            if (I2 > I) {
-                const int n = 16 * (I2 + 1);
-                st_bf16(Bt + btile_off(I2), tc::sw128_kmajor(r, ca, n), kpa * bba[rl] * midA);
-                st_bf16(Bt + btile_off(I2), tc::sw128_kmajor(r, cb, n), kpb * bbb[rl] * midB);
-                midA *= gP[I2 * 128 + ca];
-                midB *= gP[I2 * 128 + cb];
-            }
-        }
-        gA[rl] = preA * faa[rl];
-        gB[rl] = preB * fab[rl];
-        st_bf16(KV, tc::sw128_mnmajor(r, ca, 64), gA[rl] * kpa);
-        st_bf16(KV, tc::sw128_mnmajor(r, cb, 64), gB[rl] * kpb);
-    }
-    // K_end^T image: rows ca, cb; columns r0 .. r0 + 15 (two 16-byte chunks per row);
-    // K_end,j = sigma_C (gamma_C / gamma_j) k'_j, from this thread's own k' values in KF
+    // ======== A3: row pass -- thread (row r, 8-channel groups g and g + 8) ========
     {
-        uint8_t* ke = wsc + WS_KE;
+        const int r = tid >> 3, g = tid & 7;
+        const int I = r >> 4, rl = r & 15;
+        const int cA = 8 * g, cB = 64 + 8 * g;
+        float qa[8], qb[8], ka[8], kb[8];
+        if (r < nvalid) {
+            const size_t o = (row0 + r * rs) * kDK;
+            unpack8(*reinterpret_cast<const uint4*>(q + o + cA), qa);
+            unpack8(*reinterpret_cast<const uint4*>(q + o + cB), qb);
+            unpack8(*reinterpret_cast<const uint4*>(k + o + cA), ka);
+            unpack8(*reinterpret_cast<const uint4*>(k + o + cB), kb);
+        } else {
 #pragma unroll
-        for (int hc = 0; hc < 2; ++hc) {
-            float ea[8], eb[8];
+            for (int i = 0; i < 8; ++i) qa[i] = qb[i] = ka[i] = kb[i] = 0.f;
+        }
+        // row norms (the rotation preserves them): reduce over the 8 threads of the row
+        float sq = 0.f, sk = 0.f;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int rl = 8 * hc + e;
-                ea[e] = salA * sufA * bba[rl] * KF[(r0 + rl) * 128 + ca];
-                eb[e] = salB * sufB * bbb[rl] * KF[(r0 + rl) * 128 + cb];
+        for (int i = 0; i < 8; ++i) {
+            sq += qa[i] * qa[i] + qb[i] * qb[i];
+            sk += ka[i] * ka[i] + kb[i] * kb[i];
+        }
+        sq = group_sum<8>(sq);
+        sk = group_sum<8>(sk);
+        if (rp.enabled) {
+            const long long pos = pos_offset + t0 + r;
+            if (rp.convention == 0) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {   // pairs (cA + i, cB + i), frequency 8g + i
+                    float sn, cs;
+                    rope_sincos(pos, rp.inv_freq[8 * g + i], &sn, &cs);
+                    float x0 = qa[i], x1 = qb[i];
+                    qa[i] = x0 * cs - x1 * sn; qb[i] = x1 * cs + x0 * sn;
+                    x0 = ka[i]; x1 = kb[i];
+                    ka[i] = x0 * cs - x1 * sn; kb[i] = x1 * cs + x0 * sn;
+                }
+            } else {
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {   // pairs (c, c + 1) inside each 8-channel group
+                    float sn, cs;
+                    rope_sincos(pos, rp.inv_freq[4 * g + m], &sn, &cs);
+                    float x0 = qa[2 * m], x1 = qa[2 * m + 1];
+                    qa[2 * m] = x0 * cs - x1 * sn; qa[2 * m + 1] = x1 * cs + x0 * sn;
+                    x0 = ka[2 * m]; x1 = ka[2 * m + 1];
+                    ka[2 * m] = x0 * cs - x1 * sn; ka[2 * m + 1] = x1 * cs + x0 * sn;
+                    rope_sincos(pos, rp.inv_freq[32 + 4 * g + m], &sn, &cs);
+                    x0 = qb[2 * m]; x1 = qb[2 * m + 1];
+                    qb[2 * m] = x0 * cs - x1 * sn; qb[2 * m + 1] = x1 * cs + x0 * sn;
+                    x0 = kb[2 * m]; x1 = kb[2 * m + 1];
+                    kb[2 * m] = x0 * cs - x1 * sn; kb[2 * m + 1] = x1 * cs + x0 * sn;
+                }
             }
-            *reinterpret_cast<uint4*>(ke + tc::sw128_kmajor(ca, r0 + 8 * hc, 128)) = pack8(ea);
-            *reinterpret_cast<uint4*>(ke + tc::sw128_kmajor(cb, r0 + 8 * hc, 128)) = pack8(eb);
         }
-        if (I == 0) {
-            float* G = reinterpret_cast<float*>(wsc + WS_G);
-            G[ca] = salA * allA;
-            G[cb] = salB * allB;
+        const float fq = l2norm ? rsqrtf(sq + kL2Eps) : 1.f;
+        const float fk = l2norm ? rsqrtf(sk + kL2Eps) : 1.f;
+        const bool diag_ok = !unsafe[I];
+
+        // the two 8-channel halves of this thread: cA.. and cB..
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int c0 = hh ? cB : cA;
+            const float* qx = hh ? qb : qa;
+            const float* kx = hh ? kb : ka;
+            float fb[8], kp[8], qp[8], acc[8], t8[8];
+            ld_f8(FB + r * 128 + c0, fb);
+            // parity before this block
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = 1.f;
+            for (int J = 0; J < I; ++J) {
+                ld_f8(gPar + J * 128 + c0, t8);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] *= t8[i];
+            }
+            // k', q' with the full-chunk parity (sign(fb) is the block-local parity); |fb|
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float s = signbit(fb[i]) ? -acc[i] : acc[i];
+                kp[i] = kx[i] * fk * s;
+                qp[i] = qx[i] * fq * s;
+                fb[i] = fabsf(fb[i]);
+            }
+            // L tile: k' fb and q' fb
+#pragma unroll
+            for (int i = 0; i < 8; ++i) t8[i] = kp[i] * fb[i];
+            st16(sm + S_L, tc::sw128_kmajor(32 * I + rl, c0, 128), t8);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) t8[i] = qp[i] * fb[i];
+            st16(sm + S_L, tc::sw128_kmajor(32 * I + 16 + rl, c0, 128), t8);
+            // right operand of the diagonal block: k' / fb
+#pragma unroll
+            for (int i = 0; i < 8; ++i) t8[i] = diag_ok ? kp[i] * __frcp_rn(fb[i]) : 0.f;
+            st16(sm + S_B + btile_off(I), tc::sw128_kmajor(r, c0, 16 * (I + 1)), t8);
+            // right operands of the off-diagonal blocks I2 > I: k' bb prod_{I<J<I2} P_J
+            ld_f8(BB + r * 128 + c0, acc);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] *= kp[i];
+            for (int I2 = I + 1; I2 < 4; ++I2) {
+                st16(sm + S_B + btile_off(I2), tc::sw128_kmajor(r, c0, 16 * (I2 + 1)), acc);
+                if (I2 < 3) {
+                    ld_f8(gP + I2 * 128 + c0, t8);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) acc[i] *= t8[i];
+                }
+            }
+            // K_end = sigma_C (|gamma_C| / |gamma_r|) k' = sigma_C bb prod_{J>I} P_J k'
+            ld_f8(BB + r * 128 + c0, acc);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] *= kp[i];
+#pragma unroll
+            for (int J = 0; J < 4; ++J) {
+                ld_f8(gPar + J * 128 + c0, t8);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] *= t8[i];
+                if (J > I) {
+                    ld_f8(gP + J * 128 + c0, t8);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) acc[i] *= t8[i];
+                }
+            }
+            st16(sm + S_KE, tc::sw128_mnmajor(r, c0, 64), acc);
+            // |gamma_r| = prod_{J<I} P_J * fb:  K_gamma = |gamma_r| k', Q_gamma = |gamma_r| q'
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = fb[i];
+            for (int J = 0; J < I; ++J) {
+                ld_f8(gP + J * 128 + c0, t8);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] *= t8[i];
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) t8[i] = acc[i] * kp[i];
+            st16(sm + S_KG, tc::sw128_mnmajor(r, c0, 64), t8);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) t8[i] = acc[i] * qp[i];
+            st16(sm + S_QG, tc::sw128_kmajor(r, c0, 64), t8);
         }
+    }
+    // gamma_C (signed) per channel, for the diagonal of A_c
+    if (tid < 128) {
+        float gc = 1.f;
+#pragma unroll
+        for (int J = 0; J < 4; ++J) gc *= gP[J * 128 + tid] * gPar[J * 128 + tid];
+        gGC[tid] = gc;
     }
     tc::fence_proxy_async_smem();
     tc::tc_fence_before();
@@ -322,9 +406,9 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    // ======== phase B: A and M block-rows on the tensor cores ========
+    // ======== B: A and M block-rows on the tensor cores ========
     if (tid == 0) {
-        const uint32_t l0 = tc::smem_u32(Lt), b0 = tc::smem_u32(Bt);
+        const uint32_t l0 = tc::smem_u32(sm + S_L), b0 = tc::smem_u32(sm + S_B);
 #pragma unroll
         for (int J = 0; J < 4; ++J) {
             const int n = 16 * (J + 1);
@@ -340,45 +424,44 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
     }
     tc::mbar_wait(bar, 0, abort_flag);
     tc::tc_fence_after();
-    float* sA = reinterpret_cast<float*>(sm + P1_A);
-    uint8_t* sM = sm + P1_M;
-    if (warp < 2) {
-        // warp 0: lanes 0..15 hold the k rows (A); warp 1: lanes 32..47 hold the q rows (M)
-        const int l = lane;
-#pragma unroll
-        for (int J = 0; J < 4; ++J) {
-            const int r = 16 * J + (l & 15);
+    float* sA = reinterpret_cast<float*>(sm + S_A);
+    uint8_t* sM = sm + S_M;
+    {
+        // M = 64 accumulator of block-row J: k rows in lanes 0..15, q rows in lanes 32..47.
+        // Warp w reads TMEM lanes 32 (w % 4) ..: w % 4 == 0 -> A part, 1 -> M part; J = w / 4.
+        const int quarter = warp & 3, J = warp >> 2;
+        if (quarter < 2) {
             const int n = 16 * (J + 1);
+            const int r = 16 * J + (lane & 15);
             for (int c0 = 0; c0 < n; c0 += 16) {
                 float x[16];
-                tc::tmem_ld16(tc::tmem_addr(tmem, 32 * warp, amcol(J) + c0), x);
+                tc::tmem_ld16(tc::tmem_addr(tmem, 32 * quarter, amcol(J) + c0), x);
                 tc::tmem_ld_wait();
-                if (l < 16) {
-                    if (warp == 0) {
+                if (lane < 16) {
+                    if (quarter == 0) {
                         const float br = sb[r];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const int j = c0 + i;
-                            sA[r * kStrideA + j] = j < r ? br * x[i] : 0.f;
-                        }
+                        for (int i = 0; i < 16; ++i) x[i] = (c0 + i) < r ? br * x[i] : 0.f;
+#pragma unroll
+                        for (int i = 0; i < 16; i += 4)
+                            *reinterpret_cast<float4*>(sA + r * kStrideA + c0 + i) =
+                                make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
                     } else {
 #pragma unroll
-                        for (int i = 0; i < 16; i += 8) {
-                            float y[8];
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) y[e] = (c0 + i + e) <= r ? x[i + e] : 0.f;
-                            *reinterpret_cast<uint4*>(sM + tc::sw128_kmajor(r, c0 + i, 64)) = pack8(y);
-                        }
+                        for (int i = 0; i < 16; ++i) x[i] = (c0 + i) <= r ? x[i] : 0.f;
+                        st16(sM, tc::sw128_kmajor(r, c0, 64), x);
+                        st16(sM, tc::sw128_kmajor(r, c0 + 8, 64), x + 8);
                     }
                 }
             }
-            if (l < 16) {
+            if (lane < 16) {
+                const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
                 for (int j = n; j < 64; j += 8) {
-                    if (warp == 0) {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) sA[r * kStrideA + j + e] = 0.f;
+                    if (quarter == 0) {
+                        *reinterpret_cast<float4*>(sA + r * kStrideA + j) = make_float4(0.f, 0.f, 0.f, 0.f);
+                        *reinterpret_cast<float4*>(sA + r * kStrideA + j + 4) = make_float4(0.f, 0.f, 0.f, 0.f);
                     } else {
-                        *reinterpret_cast<uint4*>(sM + tc::sw128_kmajor(r, j, 64)) = make_uint4(0, 0, 0, 0);
+                        st16(sM, tc::sw128_kmajor(r, j, 64), z);
                     }
                 }
             }
@@ -387,10 +470,21 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
     tc::tc_fence_before();
     __syncthreads();
 
-    // exact recomputation of diagonal blocks whose gate total fell below 2^-60
+    // exact recomputation of diagonal blocks whose gate total fell below 2^-60 (rare)
     for (int J = 0; J < 4; ++J) {
         if (!unsafe[J]) continue;
-        for (int pr = tid; pr < 136; pr += 256) {
+        float* fq = reinterpret_cast<float*>(sm + S_FQ);
+        float* fk = reinterpret_cast<float*>(sm + S_FK);
+        {
+            const int rl = warp, r = 16 * J + rl;
+            if (r < nvalid)
+                fallback_row(q, k, alpha, row0, rs, r, lane, rp, pos_offset + t0 + r, l2norm,
+                             fq + rl * 128, fk + rl * 128);
+            else
+                for (int c = lane; c < 128; c += 32) fq[rl * 128 + c] = fk[rl * 128 + c] = 0.f;
+        }
+        __syncthreads();
+        for (int pr = tid; pr < 136; pr += 512) {
             int rl = 0;
             while ((rl + 1) * (rl + 2) / 2 <= pr) ++rl;
             const int jl = pr - rl * (rl + 1) / 2;
@@ -399,26 +493,21 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
             for (int c = 0; c < kDK; ++c) {
                 float f = 1.f;
                 for (int tau = j + 1; tau <= r; ++tau)
-                    f *= tau < nvalid ? fabsf(alpha[grow(tau) * kDK + c]) : 1.f;
-                const float kj = KF[j * 128 + c] * f;
-                accA += KF[r * 128 + c] * kj;
-                accM += QF[r * 128 + c] * kj;
+                    f *= tau < nvalid ? fabsf(alpha[(row0 + tau * rs) * kDK + c]) : 1.f;
+                const float kj = fk[jl * 128 + c] * f;
+                accA += fk[rl * 128 + c] * kj;
+                accM += fq[rl * 128 + c] * kj;
             }
             sA[r * kStrideA + j] = j < r ? sb[r] * accA : 0.f;
-            st_bf16(sM, tc::sw128_kmajor(r, j, 64), accM);
+            *reinterpret_cast<__nv_bfloat16*>(sM + tc::sw128_kmajor(r, j, 64)) = __float2bfloat16_rn(accM);
         }
+        __syncthreads();
     }
-    __syncthreads();
 
-    // ======== phase C: T = (I + A)^-1 (fp32), T' = T diag(beta); Q_gamma in place of q' ========
-    float* sT = reinterpret_cast<float*>(sm + P1_T);
-    float* sX = reinterpret_cast<float*>(sm + P1_X);
-#pragma unroll
-    for (int rl = 0; rl < 16; ++rl) {
-        QF[(r0 + rl) * 128 + ca] *= gA[rl];
-        QF[(r0 + rl) * 128 + cb] *= gB[rl];
-    }
-    for (int e = tid; e < 64 * 64; e += 256) {
+    // ======== C: T = (I + A)^-1 (fp32), T' = T diag(beta) (bf16) ========
+    float* sT = reinterpret_cast<float*>(sm + S_T);
+    float* sX = reinterpret_cast<float*>(sm + S_X);
+    for (int e = tid; e < 64 * 64; e += 512) {
         const int r = e >> 6, j = e & 63;
         if ((j >> 4) > (r >> 4)) sT[r * kStrideA + j] = 0.f;
     }
@@ -427,85 +516,88 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
         float tcol[16];
 #pragma unroll
         for (int rr = 0; rr < 16; ++rr) {
-            float acc = 0.f;
+            float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-            for (int m = 0; m < 16; ++m)
-                if (m < rr) acc += sA[(base + rr) * kStrideA + base + m] * tcol[m];
-            tcol[rr] = rr < l ? 0.f : (rr == l ? 1.f : -acc);
+            for (int m = 0; m < 16; m += 2) {
+                if (m < rr) a0 += sA[(base + rr) * kStrideA + base + m] * tcol[m];
+                if (m + 1 < rr) a1 += sA[(base + rr) * kStrideA + base + m + 1] * tcol[m + 1];
+            }
+            tcol[rr] = rr < l ? 0.f : (rr == l ? 1.f : -(a0 + a1));
         }
 #pragma unroll
         for (int rr = 0; rr < 16; ++rr) sT[(base + rr) * kStrideA + base + l] = tcol[rr];
     }
     __syncthreads();
     for (int Ib = 1; Ib < 4; ++Ib) {
-        const int ncol = 16 * Ib;
-        for (int e = tid; e < 16 * ncol; e += 256) {
-            const int rl = e / ncol, jj = e % ncol;
-            const int Jb = jj >> 4;
-            float x = 0.f;
-            for (int m = 16 * Jb; m < 16 * Ib; ++m) x += sA[(16 * Ib + rl) * kStrideA + m] * sT[m * kStrideA + jj];
-            sX[rl * 48 + jj] = x;
+        const int nq = 4 * Ib;   // column quads in [0, 16 Ib)
+        // X = sum_{K = J..Ib-1} A_{Ib,K} T_{K,J}: thread per (row rl, 4 columns)
+        for (int e = tid; e < 16 * nq; e += 512) {
+            const int rl = e / nq, j0 = 4 * (e % nq);
+            const int m0 = 16 * (j0 >> 4);
+            float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
+            for (int m = m0; m < 16 * Ib; ++m) {
+                const float a = sA[(16 * Ib + rl) * kStrideA + m];
+                const float4 t = *reinterpret_cast<const float4*>(sT + m * kStrideA + j0);
+                x0 += a * t.x; x1 += a * t.y; x2 += a * t.z; x3 += a * t.w;
+            }
+            *reinterpret_cast<float4*>(sX + rl * 48 + j0) = make_float4(x0, x1, x2, x3);
         }
         __syncthreads();
-        for (int e = tid; e < 16 * ncol; e += 256) {
-            const int rl = e / ncol, jj = e % ncol;
-            float y = 0.f;
+        for (int e = tid; e < 16 * nq; e += 512) {
+            const int rl = e / nq, j0 = 4 * (e % nq);
+            float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
 #pragma unroll
-            for (int m = 0; m < 16; ++m) y += sT[(16 * Ib + rl) * kStrideA + 16 * Ib + m] * sX[m * 48 + jj];
-            sT[(16 * Ib + rl) * kStrideA + jj] = -y;
+            for (int m = 0; m < 16; ++m) {
+                const float a = sT[(16 * Ib + rl) * kStrideA + 16 * Ib + m];
+                const float4 x = *reinterpret_cast<const float4*>(sX + m * 48 + j0);
+                y0 += a * x.x; y1 += a * x.y; y2 += a * x.z; y3 += a * x.w;
+            }
+            *reinterpret_cast<float4*>(sT + (16 * Ib + rl) * kStrideA + j0) = make_float4(-y0, -y1, -y2, -y3);
         }
         __syncthreads();
     }
-    uint8_t* sTb = sm + P1_TB;
-    for (int e = tid; e < 64 * 8; e += 256) {
+    for (int e = tid; e < 64 * 8; e += 512) {
         const int r = e >> 3, j0 = (e & 7) * 8;
         float y[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) y[i] = sT[r * kStrideA + j0 + i] * sb[j0 + i];
-        *reinterpret_cast<uint4*>(sTb + tc::sw128_kmajor(r, j0, 64)) = pack8(y);
+        st16(sm + S_TB, tc::sw128_kmajor(r, j0, 64), y);
     }
     tc::fence_proxy_async_smem();
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
 
-    // ======== phase D: [W | U~] = T' [K_gamma | V]  (M = 64, N = 256, K = 64) ========
+    // ======== D: W = T' K_gamma, U~ = T' V  (M = 64, N = 128 each, K = 64) ========
     if (tid == 0) {
-        const uint32_t a0 = tc::smem_u32(sTb), b0 = tc::smem_u32(KV);
-        const uint32_t idesc = tc::idesc_bf16_f32(64, 256, 0, 1);
+        const uint32_t a0 = tc::smem_u32(sm + S_TB);
+        const uint32_t kg = tc::smem_u32(sm + S_KG), vv = tc::smem_u32(sm + S_V);
+        const uint32_t idesc = tc::idesc_bf16_f32(64, 128, 0, 1);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-            uint64_t ad = tc::smem_desc_sw128(a0 + ks * 32, 16, 1024);
-            uint64_t bd = tc::smem_desc_sw128(b0 + ks * 2048, 64 * 128, 1024);
-            tc::mma_bf16(tmem, ad, bd, idesc, ks > 0 ? 1u : 0u);
+            const uint64_t ad = tc::smem_desc_sw128(a0 + ks * 32, 16, 1024);
+            tc::mma_bf16(tmem, ad, tc::smem_desc_sw128(kg + ks * 2048, 8192, 1024), idesc, ks > 0);
+            tc::mma_bf16(tmem + 128, ad, tc::smem_desc_sw128(vv + ks * 2048, 8192, 1024), idesc, ks > 0);
         }
         tc::mma_commit(bar);
     }
     tc::mbar_wait(bar, 1, abort_flag);
     tc::tc_fence_after();
-    uint8_t* WU = sm + P1_WU;
     {
-        // M = 64 accumulator: row m in lane (m % 16) + 32 (m / 16).  Warps w and w + 4 share lanes
-        // 32 (w % 4) ..; warp w < 4 takes columns 0..127 (W), warp w + 4 columns 128..255 (U~).
-        const int wq = warp & 3, half = warp >> 2;
-        const int r = 16 * wq + (lane & 15);
-        for (int c0 = 0; c0 < 128; c0 += 16) {
+        // warp w: rows 16 (w % 4) + lane (lane < 16); 64-column slice w / 4:
+        // slices 0, 1 -> W columns 0..127, slices 2, 3 -> U~ columns 0..127
+        const int quarter = warp & 3, slice = warp >> 2;
+        const int r = 16 * quarter + (lane & 15);
+        uint8_t* dst = sm + (slice < 2 ? S_W : S_U);
+        const int n0 = 64 * (slice & 1);
+#pragma unroll
+        for (int c0 = 0; c0 < 64; c0 += 16) {
             float x[16];
-            tc::tmem_ld16(tc::tmem_addr(tmem, 32 * wq, 128 * half + c0), x);
+            tc::tmem_ld16(tc::tmem_addr(tmem, 32 * quarter, 64 * slice + c0), x);
             tc::tmem_ld_wait();
             if (lane < 16) {
-#pragma unroll
-                for (int hc = 0; hc < 2; ++hc) {
-                    const uint4 pk = pack8(x + 8 * hc);
-                    const int n = 128 * half + c0 + 8 * hc;
-                    *reinterpret_cast<uint4*>(WU + tc::sw128_mnmajor(r, n, 64)) = pk;
-                    if (half == 0) {
-                        *reinterpret_cast<uint4*>(wsc + WS_QW + tc::sw128_kmajor(64 + r, c0 + 8 * hc, 128)) = pk;
-                    } else {
-                        const int nn = c0 + 8 * hc, tile = nn >> 5;
-                        *reinterpret_cast<uint4*>(wsc + WS_UO + tile * WS_UO_TILE + (r * 32 + (nn & 31)) * 2) = pk;
-                    }
-                }
+                st16(dst, tc::sw128_mnmajor(r, n0 + c0, 64), x);
+                st16(dst, tc::sw128_mnmajor(r, n0 + c0 + 8, 64), x + 8);
             }
         }
     }
@@ -514,40 +606,77 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
     __syncthreads();
     tc::tc_fence_after();
 
-    // ======== phase F: M [W | U~]  (M = 64, N = 256, K = 64) ========
+    // ======== F: M [W | U~] (M = 64) and K_end^T [W | U~] (M = 128, MN-major A) ========
     if (tid == 0) {
-        const uint32_t a0 = tc::smem_u32(sM), b0 = tc::smem_u32(WU);
-        const uint32_t idesc = tc::idesc_bf16_f32(64, 256, 0, 1);
+        const uint32_t am = tc::smem_u32(sm + S_M), ke = tc::smem_u32(sm + S_KE);
+        const uint32_t w0 = tc::smem_u32(sm + S_W), u0 = tc::smem_u32(sm + S_U);
+        const uint32_t id64 = tc::idesc_bf16_f32(64, 128, 0, 1);
+        const uint32_t id128 = tc::idesc_bf16_f32(128, 128, 1, 1);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-            uint64_t ad = tc::smem_desc_sw128(a0 + ks * 32, 16, 1024);
-            uint64_t bd = tc::smem_desc_sw128(b0 + ks * 2048, 64 * 128, 1024);
-            tc::mma_bf16(tmem, ad, bd, idesc, ks > 0 ? 1u : 0u);
+            const uint64_t bw = tc::smem_desc_sw128(w0 + ks * 2048, 8192, 1024);
+            const uint64_t bu = tc::smem_desc_sw128(u0 + ks * 2048, 8192, 1024);
+            const uint64_t adm = tc::smem_desc_sw128(am + ks * 32, 16, 1024);
+            const uint64_t ade = tc::smem_desc_sw128(ke + ks * 2048, 8192, 1024);
+            tc::mma_bf16(tmem, adm, bw, id64, ks > 0);
+            tc::mma_bf16(tmem + 128, adm, bu, id64, ks > 0);
+            tc::mma_bf16(tmem + 256, ade, bw, id128, ks > 0);
+            tc::mma_bf16(tmem + 384, ade, bu, id128, ks > 0);
         }
         tc::mma_commit(bar);
     }
     tc::mbar_wait(bar, 0, abort_flag);
     tc::tc_fence_after();
     {
-        const int wq = warp & 3, half = warp >> 2;
-        const int r = 16 * wq + (lane & 15);
-        for (int c0 = 0; c0 < 128; c0 += 16) {
-            float x[16];
-            tc::tmem_ld16(tc::tmem_addr(tmem, 32 * wq, 128 * half + c0), x);
-            tc::tmem_ld_wait();
-            if (lane < 16) {
+        const int quarter = warp & 3, slice = warp >> 2;
+        // (1) M = 64 products: rows 16 quarter + lane; slices 0, 1 -> Q', 2, 3 -> O_loc
+        {
+            const int r = 16 * quarter + (lane & 15);
+            const int n0 = 64 * (slice & 1);
+#pragma unroll
+            for (int c0 = 0; c0 < 64; c0 += 16) {
+                float x[16];
+                tc::tmem_ld16(tc::tmem_addr(tmem, 32 * quarter, 64 * slice + c0), x);
+                tc::tmem_ld_wait();
+                if (lane < 16) {
+#pragma unroll
+                    for (int hc = 0; hc < 2; ++hc) {
+                        const int n = n0 + c0 + 8 * hc;
+                        if (slice < 2) {
+                            float qg[8];
+                            unpack8(*reinterpret_cast<const uint4*>(sm + S_QG + tc::sw128_kmajor(r, n, 64)), qg);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) qg[i] -= x[8 * hc + i];
+                            *reinterpret_cast<uint4*>(wsc + WS_QP + tc::sw128_kmajor(r, n, 64)) = pack8(qg);
+                        } else {
+                            *reinterpret_cast<uint4*>(wsc + WS_TILES + (n >> 5) * WS_TILE + WS_TILE_O +
+                                                      (r * 32 + (n & 31)) * 2) = pack8(x + 8 * hc);
+                        }
+                    }
+                }
+            }
+        }
+        // (2) M = 128 products: row c' = 32 quarter + lane; slices 0, 1 -> A_c, 2, 3 -> B_c
+        {
+            const int cr = 32 * quarter + lane;
+            const int n0 = 64 * (slice & 1);
+            const float gc = gGC[cr];
+#pragma unroll
+            for (int c0 = 0; c0 < 64; c0 += 16) {
+                float x[16];
+                tc::tmem_ld16(tc::tmem_addr(tmem, 32 * quarter, 256 + 64 * slice + c0), x);
+                tc::tmem_ld_wait();
 #pragma unroll
                 for (int hc = 0; hc < 2; ++hc) {
-                    const int n = c0 + 8 * hc;
+                    const int n = n0 + c0 + 8 * hc;
                     float y[8];
-                    if (half == 0) {
+                    if (slice < 2) {
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) y[e] = QF[r * 128 + n + e] - x[8 * hc + e];
-                        *reinterpret_cast<uint4*>(wsc + WS_QW + tc::sw128_kmajor(r, n, 128)) = pack8(y);
+                        for (int i = 0; i < 8; ++i) y[i] = (n + i == cr ? gc : 0.f) - x[8 * hc + i];
+                        *reinterpret_cast<uint4*>(wsc + WS_AC + tc::sw128_kmajor(cr, n, 128)) = pack8(y);
                     } else {
-                        const int tile = n >> 5;
-                        *reinterpret_cast<uint4*>(wsc + WS_UO + tile * WS_UO_TILE + 4096 + (r * 32 + (n & 31)) * 2) =
-                            pack8(x + 8 * hc);
+                        *reinterpret_cast<uint4*>(wsc + WS_TILES + (n >> 5) * WS_TILE +
+                                                  (cr * 32 + (n & 31)) * 2) = pack8(x + 8 * hc);
                     }
                 }
             }
@@ -556,16 +685,16 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
     tc::tc_fence_before();
     __syncthreads();
     if (*abort_flag && tid == 0) atomicExch(&g_tc_error, 1);
-    if (warp == 0) tc::tmem_dealloc(tmem, 256);
+    if (warp == 0) tc::tmem_dealloc(tmem, 512);
 }
 
-// ---- kernel 2 ---------------------------------------------------------------------------------
-constexpr uint32_t P2_STAGE = 58368;
-constexpr uint32_t P2_QW = 0, P2_KE = 32768, P2_UO = 49152, P2_G = 57344;
-constexpr uint32_t P2_LOAD_BYTES = 32768 + 16384 + WS_UO_TILE + 512;
-constexpr uint32_t P2_ST = 2 * P2_STAGE;          // S^T bf16 K-major 32 rows x 128 (8 KB)
-constexpr uint32_t P2_UT = P2_ST + 8192;          // U^T bf16 K-major 32 rows x 64 (4 KB)
-constexpr uint32_t P2_SM = P2_UT + 4096;
+// ---- kernel 2: the serial state pass ------------------------------------------------------------
+constexpr int kStages = 3;
+constexpr uint32_t P2_STAGE = 61440;                    // A_c 32 KB, Q' 16 KB, B_c 8 KB, O_loc 4 KB
+constexpr uint32_t P2_AC = 0, P2_QP = 32768, P2_BC = 49152, P2_OL = 57344;
+constexpr uint32_t P2_LOAD_BYTES = 32768 + 16384 + WS_TILE;
+constexpr uint32_t P2_ST = kStages * P2_STAGE;          // S operand bf16, K-major 32 rows x 128
+constexpr uint32_t P2_SM = P2_ST + 8192;
 constexpr uint32_t P2_BYTES = P2_SM + 256 + 1024;
 
 __global__ void __launch_bounds__(160, 1)
@@ -575,13 +704,13 @@ ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(sm + P2_SM);  // [2]
-    uint64_t* mma1 = full + 2;
-    uint64_t* mma2 = full + 3;
-    uint64_t* epi1 = full + 4;
-    uint64_t* epi2 = full + 5;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(full + 6);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(full + 7);
+    uint64_t* full = reinterpret_cast<uint64_t*>(sm + P2_SM);  // [3]
+    uint64_t* empty = full + 3;                                // [3]
+    uint64_t* mma_c = full + 6;
+    uint64_t* mma_o = full + 7;
+    uint64_t* epi = full + 8;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(full + 9);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(full + 10);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int tile = blockIdx.x % kNTile, bh = blockIdx.x / kNTile;
@@ -589,19 +718,19 @@ ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
     const int n0 = tile * kDVT;
     const uint8_t* wsh = ws + (size_t)bh * NT * WS_CHUNK;
     uint8_t* sST = sm + P2_ST;
-    uint8_t* sUT = sm + P2_UT;
 
     if (warp == 0) {
-        tc::tmem_alloc(tmem_slot, 64);
+        tc::tmem_alloc(tmem_slot, 128);
         tc::tmem_relinquish();
     }
     if (tid == 128) {
-        tc::mbar_init(&full[0], 1);
-        tc::mbar_init(&full[1], 1);
-        tc::mbar_init(mma1, 1);
-        tc::mbar_init(mma2, 1);
-        tc::mbar_init(epi1, 128);
-        tc::mbar_init(epi2, 128);
+        for (int s = 0; s < kStages; ++s) {
+            tc::mbar_init(&full[s], 1);
+            tc::mbar_init(&empty[s], 128);
+        }
+        tc::mbar_init(mma_c, 1);
+        tc::mbar_init(mma_o, 1);
+        tc::mbar_init(epi, 128);
         tc::fence_mbar_init();
         *abort_flag = 0;
     }
@@ -609,10 +738,11 @@ ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t d1 = tmem, d2 = tmem + 32;
+    const uint32_t dc = tmem;                 // D_c: 128 lanes x 32 columns
+    const uint32_t dob = tmem + 32;           // D_o: two buffers of 32 columns (M = 64 layout)
 
     if (tid < 128) {
-        // ---- epilogue warps: thread t owns TMEM lane t (a row of D1, a channel of D2) ----
+        // ---- epilogue: thread t owns state row t (TMEM lane t of D_c) ----
         const int t = tid;
         float S[kDVT];
         if (h0) {
@@ -627,56 +757,60 @@ ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
             for (int j = 0; j < kDVT; ++j) S[j] = 0.f;
         }
 #pragma unroll
-        for (int j = 0; j < kDVT; ++j) st_bf16(sST, tc::sw128_kmajor(j, t, 32), S[j]);
+        for (int j = 0; j < kDVT; ++j)
+            *reinterpret_cast<__nv_bfloat16*>(sST + tc::sw128_kmajor(j, t, 32)) = __float2bfloat16_rn(S[j]);
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
-        tc::mbar_arrive(epi2);
+        tc::mbar_arrive(epi);
         for (int ch = 0; ch < NT; ++ch) {
-            const int st = ch & 1;
+            const int st = ch % kStages;
             const uint8_t* stg = sm + st * P2_STAGE;
-            const int t0 = ch * kC;
-            tc::mbar_wait(&full[st], (ch >> 1) & 1, abort_flag);
-            tc::mbar_wait(mma1, ch & 1, abort_flag);
+            // chain: S = D_c + B_c
+            tc::mbar_wait(mma_c, ch & 1, abort_flag);
+            tc::mbar_wait(&full[st], (ch / kStages) & 1, abort_flag);
             tc::tc_fence_after();
             float d[32];
-            tc::tmem_ld16(tc::tmem_addr(d1, 32 * warp, 0), d);
-            tc::tmem_ld16(tc::tmem_addr(d1, 32 * warp, 16), d + 16);
+            tc::tmem_ld16(tc::tmem_addr(dc, 32 * warp, 0), d);
+            tc::tmem_ld16(tc::tmem_addr(dc, 32 * warp, 16), d + 16);
             tc::tmem_ld_wait();
-            if (t < 64) {
-                const int r = t;
-                const __nv_bfloat16* ol = reinterpret_cast<const __nv_bfloat16*>(stg + P2_UO + 4096) + r * 32;
-                float o[32];
+            const uint4* bc = reinterpret_cast<const uint4*>(stg + P2_BC + t * 64);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) o[j] = scale * (d[j] + __bfloat162float(ol[j]));
+            for (int j = 0; j < 4; ++j) {
+                float y[8];
+                unpack8(bc[j], y);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) S[8 * j + i] = d[8 * j + i] + y[i];
+            }
+#pragma unroll
+            for (int j = 0; j < kDVT; ++j)
+                *reinterpret_cast<__nv_bfloat16*>(sST + tc::sw128_kmajor(j, t, 32)) = __float2bfloat16_rn(S[j]);
+            tc::fence_proxy_async_smem();
+            tc::tc_fence_before();
+            tc::mbar_arrive(epi);
+            // output (off the critical path): O = scale (D_o + O_loc), rows in the M = 64 layout
+            tc::mbar_wait(mma_o, ch & 1, abort_flag);
+            tc::tc_fence_after();
+            tc::tmem_ld16(tc::tmem_addr(dob + 32 * (ch & 1), 32 * warp, 0), d);
+            tc::tmem_ld16(tc::tmem_addr(dob + 32 * (ch & 1), 32 * warp, 16), d + 16);
+            tc::tmem_ld_wait();
+            if (lane < 16) {
+                const int r = 16 * warp + lane;
+                const int t0 = ch * kC;
                 if (t0 + r < T_len) {
+                    const uint4* ol = reinterpret_cast<const uint4*>(stg + P2_OL + r * 64);
                     uint4* dst = reinterpret_cast<uint4*>(out + (((size_t)b * T_len + t0 + r) * H + h) * kDV + n0);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) dst[j] = pack8(o + 8 * j);
+                    for (int j = 0; j < 4; ++j) {
+                        float y[8];
+                        unpack8(ol[j], y);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) y[i] = scale * (d[8 * j + i] + y[i]);
+                        dst[j] = pack8(y);
+                    }
                 }
-            } else {
-                const int r = t - 64;
-                const __nv_bfloat16* ut = reinterpret_cast<const __nv_bfloat16*>(stg + P2_UO) + r * 32;
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    st_bf16(sUT, tc::sw128_kmajor(j, r, 32), __bfloat162float(ut[j]) - d[j]);
             }
-            tc::fence_proxy_async_smem();
             tc::tc_fence_before();
-            tc::mbar_arrive(epi1);
-            tc::mbar_wait(mma2, ch & 1, abort_flag);
-            tc::tc_fence_after();
-            tc::tmem_ld16(tc::tmem_addr(d2, 32 * warp, 0), d);
-            tc::tmem_ld16(tc::tmem_addr(d2, 32 * warp, 16), d + 16);
-            tc::tmem_ld_wait();
-            const float g = reinterpret_cast<const float*>(stg + P2_G)[t];
-#pragma unroll
-            for (int j = 0; j < kDVT; ++j) {
-                S[j] = g * S[j] + d[j];
-                st_bf16(sST, tc::sw128_kmajor(j, t, 32), S[j]);
-            }
-            tc::fence_proxy_async_smem();
-            tc::tc_fence_before();
-            tc::mbar_arrive(epi2);
+            tc::mbar_arrive(&empty[st]);
         }
         if (hT) {
             float4* dst = reinterpret_cast<float4*>(hT + ((size_t)bh * kDK + t) * kDV + n0);
@@ -687,59 +821,59 @@ ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
     } else if (tid == 128) {
         // ---- control thread: stage loads (1-D bulk copies) and MMA issue ----
         auto load = [&](int c) {
-            const int st = c & 1;
+            const int st = c % kStages;
             uint8_t* stg = sm + st * P2_STAGE;
             const uint8_t* src = wsh + (size_t)c * WS_CHUNK;
             tc::mbar_arrive_expect_tx(&full[st], P2_LOAD_BYTES);
-            tc::bulk_g2s(stg + P2_QW, src + WS_QW, 32768, &full[st]);
-            tc::bulk_g2s(stg + P2_KE, src + WS_KE, 16384, &full[st]);
-            tc::bulk_g2s(stg + P2_UO, src + WS_UO + tile * WS_UO_TILE, WS_UO_TILE, &full[st]);
-            tc::bulk_g2s(stg + P2_G, src + WS_G, 512, &full[st]);
+            tc::bulk_g2s(stg + P2_AC, src + WS_AC, 32768, &full[st]);
+            tc::bulk_g2s(stg + P2_QP, src + WS_QP, 16384, &full[st]);
+            tc::bulk_g2s(stg + P2_BC, src + WS_TILES + tile * WS_TILE, WS_TILE, &full[st]);
         };
-        int loaded = 0;
-        load(0);
-        loaded = 1;
-        const uint32_t id1 = tc::idesc_bf16_f32(128, kDVT, 0, 0);
-        const uint32_t st_addr = tc::smem_u32(sST), ut_addr = tc::smem_u32(sUT);
+        int issued = 0;
+        for (; issued < kStages && issued < NT; ++issued) load(issued);
+        const uint32_t idc = tc::idesc_bf16_f32(128, kDVT, 0, 0);
+        const uint32_t ido = tc::idesc_bf16_f32(64, kDVT, 0, 0);
+        const uint32_t s_addr = tc::smem_u32(sST);
         for (int ch = 0; ch < NT; ++ch) {
-            const int st = ch & 1;
+            const int st = ch % kStages;
             const uint32_t stg = tc::smem_u32(sm + st * P2_STAGE);
-            if (!tc::mbar_wait(epi2, ch & 1, abort_flag)) break;
-            if (ch + 1 < NT) { load(ch + 1); loaded = ch + 2; }
-            if (!tc::mbar_wait(&full[st], (ch >> 1) & 1, abort_flag)) break;
+            if (!tc::mbar_wait(epi, ch & 1, abort_flag)) break;            // S operand ready
+            if (!tc::mbar_wait(&full[st], (ch / kStages) & 1, abort_flag)) break;
             tc::tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
-                uint64_t ad = tc::smem_desc_sw128(stg + P2_QW + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-                uint64_t bd = tc::smem_desc_sw128(st_addr + (ks >> 2) * 4096 + (ks & 3) * 32, 16, 1024);
-                tc::mma_bf16(d1, ad, bd, id1, ks > 0 ? 1u : 0u);
+                const uint64_t bd = tc::smem_desc_sw128(s_addr + (ks >> 2) * 4096 + (ks & 3) * 32, 16, 1024);
+                const uint64_t ad = tc::smem_desc_sw128(stg + P2_AC + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+                tc::mma_bf16(dc, ad, bd, idc, ks > 0 ? 1u : 0u);
             }
-            tc::mma_commit(mma1);
-            if (!tc::mbar_wait(epi1, ch & 1, abort_flag)) break;
-            tc::tc_fence_after();
+            tc::mma_commit(mma_c);
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                uint64_t ad = tc::smem_desc_sw128(stg + P2_KE + ks * 32, 16, 1024);
-                uint64_t bd = tc::smem_desc_sw128(ut_addr + ks * 32, 16, 1024);
-                tc::mma_bf16(d2, ad, bd, id1, ks > 0 ? 1u : 0u);
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint64_t bd = tc::smem_desc_sw128(s_addr + (ks >> 2) * 4096 + (ks & 3) * 32, 16, 1024);
+                const uint64_t ad = tc::smem_desc_sw128(stg + P2_QP + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
+                tc::mma_bf16(dob + 32 * (ch & 1), ad, bd, ido, ks > 0 ? 1u : 0u);
             }
-            tc::mma_commit(mma2);
+            tc::mma_commit(mma_o);
+            // refill the stage of chunk ch - 1 once its epilogue has consumed it
+            if (ch >= 1 && issued < NT) {
+                const int prev = ch - 1;
+                if (!tc::mbar_wait(&empty[prev % kStages], (prev / kStages) & 1, abort_flag)) break;
+                load(issued);
+                ++issued;
+            }
         }
-        // drain: the final epilogue arrival, then any copy still in flight
-        tc::mbar_wait(epi2, NT & 1, abort_flag);
+        // drain: the last output epilogue, then any copy still in flight
+        if (NT > 0) tc::mbar_wait(&empty[(NT - 1) % kStages], ((NT - 1) / kStages) & 1, abort_flag);
         if (*abort_flag) {
             atomicExch(&g_tc_error, 2);
-            // only the latest fill of each stage can still be in flight
-            for (int c = loaded > 2 ? loaded - 2 : 0; c < loaded; ++c) {
+            for (int c = issued > kStages ? issued - kStages : 0; c < issued; ++c)
                 for (uint32_t i = 0; i < tc::kSpinLimit; ++i)
-                    if (tc::mbar_try_wait(&full[c & 1], (c >> 1) & 1)) break;
-            }
+                    if (tc::mbar_try_wait(&full[c % kStages], (c / kStages) & 1)) break;
         }
     }
     tc::tc_fence_before();
     __syncthreads();
-    if (warp == 0) tc::tmem_dealloc(tmem, 64);
-    (void)lane;
+    if (warp == 0) tc::tmem_dealloc(tmem, 128);
 }
 
 }  // namespace
@@ -755,7 +889,7 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const f
                             long long pos_offset, void* workspace, int stages,
                             cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(ckda_tc_intra, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)P1_BYTES);
+                                         (int)S_BYTES);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(ckda_tc_state, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P2_BYTES);
     if (e != cudaSuccess) return e;
@@ -763,12 +897,12 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const f
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     if (stages == 0) stages = 3;
     if (stages & 1) {
-    ckda_tc_intra<<<(unsigned)(NT * B * H), 256, P1_BYTES, stream>>>(
-        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-        static_cast<const __nv_bfloat16*>(v), alpha, beta, ws, T_len, H, NT, l2norm, rp,
-        pos_offset);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+        ckda_tc_intra<<<(unsigned)(NT * B * H), 512, S_BYTES, stream>>>(
+            static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+            static_cast<const __nv_bfloat16*>(v), alpha, beta, ws, T_len, H, NT, l2norm, rp,
+            pos_offset);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
     }
     if (stages & 2) {
         ckda_tc_state<<<(unsigned)(kNTile * B * H), 160, P2_BYTES, stream>>>(

@@ -48,7 +48,7 @@ def _call(f, g, out, hT, B, T, H):
 
 
 def test_noalloc_matches_the_workspace_entry_point_on_two_calls(noalloc):
-    B, T, H = 1, 700, 16  # 16 heads x 11 chunks = 176 chunk-heads, 14.5 MB of scratch
+    B, T, H = 1, 640, 16  # 16 heads x 10 chunks = 160 chunk-heads, 15.7 MB of scratch
     assert ck.workspace_bytes(B, T, H, 128, 128, 64, torch.bfloat16, "tc") <= LIMIT
     d, g = fwd_case(B, T, H, 128, 128, kind="ckda", dtype="bf16", h0_std=0.02, seed=31)
     ref_out, ref_hT = ck.fwd_chunked(g["q"], g["k"], g["v"], g["alpha"], g["beta"], g["h0"],

@@ -72,59 +72,74 @@ def peaks():
 # ---- clocks ----------------------------------------------------------------------------------
 
 class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples with host timestamps.  Started well before the
+    timed region (nvidia-smi takes a moment to produce its first line); window(t0, t1) keeps the
+    samples taken while the timed region ran, widened to the nearest sample on each side when the
+    region is shorter than the sampling interval."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, gpu_id):
         self.gpu_id = gpu_id
         self.proc = None
-        self.lines = []
-        self.error = None
+        self.samples = []   # (host time, sm MHz, max MHz, reasons)
+        self.raw = []
 
-    def start(self):
+    def start(self, wait_first=5.0):
         try:
             cmd = ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                   "-lms", "100"]
+                   "-lms", "50"]
             if self.gpu_id:
                 cmd.insert(1, f"--id={self.gpu_id}")
             self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT,
                                          text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
-        except Exception:
+            t = time.time()
+            while not self.samples and time.time() - t < wait_first and self.proc.poll() is None:
+                time.sleep(0.02)
+        except Exception as e:
             self.proc = None
+            self.raw.append(repr(e))
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
-    def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        sms, maxes, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
+            now = time.time()
             f = [x.strip() for x in line.split(",")]
             if len(f) < 9:
+                self.raw.append(line.strip())
                 continue
             try:
-                sms.append(float(f[1]))
-                maxes.append(float(f[2]))
+                sm, mx = float(f[1]), float(f[2])
             except ValueError:
+                self.raw.append(line.strip())
                 continue
-            for name, val in zip(names, f[5:9]):
-                if val.lower() == "active":
-                    reasons.add(name)
-        if not sms:
-            return {"error": "no clock samples", "raw": self.lines[:3]}
-        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxes),
-                "reasons": sorted(reasons), "samples": len(sms)}
+            reasons = {n for n, val in zip(self.NAMES, f[5:9]) if val.lower() == "active"}
+            self.samples.append((now, sm, mx, reasons))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def window(self, t0, t1):
+        if not self.samples:
+            return {"error": "no clock samples", "raw": self.raw[:3]}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not inside:   # region shorter than the interval: nearest sample on each side
+            before = [s for s in self.samples if s[0] < t0][-1:]
+            after = [s for s in self.samples if s[0] > t1][:1]
+            inside = before + after
+        sms = [s[1] for s in inside]
+        reasons = set().union(*[s[3] for s in inside]) if inside else set()
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(s[2] for s in inside),
+                "reasons": sorted(reasons), "samples": len(inside),
+                "window_ms": round((t1 - t0) * 1e3, 2)}
 
 
 # ---- helpers ---------------------------------------------------------------------------------
@@ -320,14 +335,20 @@ def main():
         gpu_id = None
     sampler = ClockSampler(gpu_id)
     sampler.start()
+    for i in range(2):
+        step(i)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    t_host0 = time.time()
     ms = event_time_ms(step, args.steps, stream)
     torch.cuda.synchronize()
+    t_host1 = time.time()
     if world > 1:
         dist.barrier()
-    clocks = sampler.stop()
+    time.sleep(0.12)
+    sampler.stop()
+    clocks = sampler.window(t_host0, t_host1)
     ms_per_step = ms / args.steps
     if world > 1:
         t = torch.tensor([ms_per_step], device=dev)

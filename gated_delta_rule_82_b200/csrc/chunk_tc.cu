@@ -70,7 +70,7 @@ constexpr uint32_t S_V = 155648;     // V (MN-major, 64 x 128)
 constexpr uint32_t S_KE = 172032;    // K_end (MN-major, 64 x 128): the MN-major A of K_end^T
 constexpr uint32_t S_QG = 188416;    // Q_gamma (K-major, 64 rows x 128)
 constexpr uint32_t S_SM = 204800;    // small arrays (below)
-constexpr uint32_t S_BYTES = S_SM + 10240 + 1024;
+constexpr uint32_t S_BYTES = S_SM + 13312 + 1024;
 
 constexpr int kStrideA = 68;                     // fp32 row stride of A and T
 constexpr uint32_t S_A = 0;                      // A  fp32 [64][68]
@@ -78,16 +78,22 @@ constexpr uint32_t S_T = 17408;                  // T  fp32 [64][68]
 constexpr uint32_t S_M = 35840;                  // M  bf16 K-major 64 x 64
 constexpr uint32_t S_TB = 44032;                 // T' bf16 K-major 64 x 64
 constexpr uint32_t S_X = 52224;                  // X  fp32 [16][48]
+constexpr uint32_t S_PT = 55296;                 // partial block products fp32 [6][16][16]
 constexpr uint32_t S_W = S_L;                    // W  MN-major 64 x 128
 constexpr uint32_t S_U = S_L + 16384;            // U~ MN-major 64 x 128
 constexpr uint32_t S_FQ = S_B;                   // fallback q' fp32 [16][128]
 constexpr uint32_t S_FK = S_B + 8192;            // fallback k' fp32 [16][128]
+constexpr uint32_t S_OUT = 0;                    // staging of the chunk's workspace image (96 KB)
 // small arrays
-constexpr uint32_t SM_P = S_SM;                  // P   fp32 [4][128]  block totals
-constexpr uint32_t SM_PAR = S_SM + 2048;         // PAR fp32 [4][128]  block parity (+-1)
-constexpr uint32_t SM_GC = S_SM + 4096;          // gamma_C fp32 [128]
-constexpr uint32_t SM_B = S_SM + 4608;           // beta fp32 [64]
-constexpr uint32_t SM_FLAGS = S_SM + 4864;       // int unsafe[4], abort, tmem slot, mbarrier
+constexpr uint32_t SM_P = S_SM;                  // P    fp32 [4][128]  block totals of |alpha|
+constexpr uint32_t SM_PAR = S_SM + 2048;         // PAR  fp32 [4][128]  block parity (+-1)
+constexpr uint32_t SM_PRE = S_SM + 4096;         // PRE  fp32 [4][128]  prod_{J<I} P_J
+constexpr uint32_t SM_KEF = S_SM + 6144;         // KEF  fp32 [4][128]  sigma_C prod_{J>I} P_J
+constexpr uint32_t SM_OFF2 = S_SM + 8192;        // OFF2 fp32 [4][128]  P_{I+1}
+constexpr uint32_t SM_OFF3 = S_SM + 10240;       // OFF3 fp32 [4][128]  P_{I+1} P_{I+2}
+constexpr uint32_t SM_GC = S_SM + 12288;         // gamma_C fp32 [128]
+constexpr uint32_t SM_B = S_SM + 12800;          // beta fp32 [64]
+constexpr uint32_t SM_FLAGS = S_SM + 13056;      // int unsafe[4], abort, tmem slot, mbarrier
 
 __host__ __device__ constexpr uint32_t btile_off(int I) { return I == 0 ? 0u : I == 1 ? 4096u : I == 2 ? 12288u : 24576u; }
 __host__ __device__ constexpr uint32_t amcol(int I) { return I == 0 ? 0u : I == 1 ? 16u : I == 2 ? 48u : 96u; }
@@ -175,11 +181,87 @@ __device__ void fallback_row(const __nv_bfloat16* q, const __nv_bfloat16* k, con
     }
 }
 
+
+// One block-row Ib (1..3) of T = (I + A)^-1 below the diagonal, given the diagonal blocks and
+// the block-rows above it:  T_{Ib,J} = -T_{Ib,Ib} sum_{K = J..Ib-1} A_{Ib,K} T_{K,J}.
+// Pass 1: warp w computes one 16 x 16 x 16 product A_{Ib,K} T_{K,J} for the w-th pair J <= K < Ib;
+// pass 2 sums the pairs into X; pass 3: warp J computes -T_{Ib,Ib} X_J.  Every loop is fully
+// unrolled, a thread owns a 2 x 4 output tile.
+template <int Ib>
+__device__ __forceinline__ void t_offdiag_level(const float* sA, float* sT, float* sX, float* sPt,
+                                                int tid) {
+    constexpr int NP = Ib * (Ib + 1) / 2;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int rp = lane >> 2, jq = lane & 3;
+    if (warp < NP) {
+        int K = 0, J = warp;
+        while (J > K) { J -= K + 1; ++K; }
+        const float* a0 = sA + (16 * Ib + 2 * rp) * kStrideA + 16 * K;
+        const float* a1 = a0 + kStrideA;
+        const float* tb = sT + (16 * K) * kStrideA + 16 * J + 4 * jq;
+        float4 x0 = make_float4(0.f, 0.f, 0.f, 0.f), x1 = x0, y0 = x0, y1 = x0;
+#pragma unroll
+        for (int m = 0; m < 16; m += 2) {
+            const float4 ta = *reinterpret_cast<const float4*>(tb + m * kStrideA);
+            const float4 tc4 = *reinterpret_cast<const float4*>(tb + (m + 1) * kStrideA);
+            const float2 aa = *reinterpret_cast<const float2*>(a0 + m);
+            const float2 ab = *reinterpret_cast<const float2*>(a1 + m);
+            x0.x += aa.x * ta.x; x0.y += aa.x * ta.y; x0.z += aa.x * ta.z; x0.w += aa.x * ta.w;
+            y0.x += aa.y * tc4.x; y0.y += aa.y * tc4.y; y0.z += aa.y * tc4.z; y0.w += aa.y * tc4.w;
+            x1.x += ab.x * ta.x; x1.y += ab.x * ta.y; x1.z += ab.x * ta.z; x1.w += ab.x * ta.w;
+            y1.x += ab.y * tc4.x; y1.y += ab.y * tc4.y; y1.z += ab.y * tc4.z; y1.w += ab.y * tc4.w;
+        }
+        float* pt = sPt + warp * 256;
+        *reinterpret_cast<float4*>(pt + (2 * rp) * 16 + 4 * jq) =
+            make_float4(x0.x + y0.x, x0.y + y0.y, x0.z + y0.z, x0.w + y0.w);
+        *reinterpret_cast<float4*>(pt + (2 * rp + 1) * 16 + 4 * jq) =
+            make_float4(x1.x + y1.x, x1.y + y1.y, x1.z + y1.z, x1.w + y1.w);
+    }
+    __syncthreads();
+    if (tid < 16 * 4 * Ib) {
+        const int rl = tid / (4 * Ib), quad = tid % (4 * Ib);
+        const int J = quad >> 2, c = 4 * (quad & 3);
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int K = 0; K < Ib; ++K) {
+            if (K >= J) {
+                const float4 p = *reinterpret_cast<const float4*>(sPt + (K * (K + 1) / 2 + J) * 256 + rl * 16 + c);
+                x.x += p.x; x.y += p.y; x.z += p.z; x.w += p.w;
+            }
+        }
+        *reinterpret_cast<float4*>(sX + rl * 48 + 16 * J + c) = x;
+    }
+    __syncthreads();
+    if (warp < Ib) {
+        const int J = warp;
+        const float* t0r = sT + (16 * Ib + 2 * rp) * kStrideA + 16 * Ib;
+        const float* t1r = t0r + kStrideA;
+        const float* xb = sX + 16 * J + 4 * jq;
+        float4 x0 = make_float4(0.f, 0.f, 0.f, 0.f), x1 = x0, y0 = x0, y1 = x0;
+#pragma unroll
+        for (int m = 0; m < 16; m += 2) {
+            const float4 xa = *reinterpret_cast<const float4*>(xb + m * 48);
+            const float4 xc = *reinterpret_cast<const float4*>(xb + (m + 1) * 48);
+            const float2 aa = *reinterpret_cast<const float2*>(t0r + m);
+            const float2 ab = *reinterpret_cast<const float2*>(t1r + m);
+            x0.x += aa.x * xa.x; x0.y += aa.x * xa.y; x0.z += aa.x * xa.z; x0.w += aa.x * xa.w;
+            y0.x += aa.y * xc.x; y0.y += aa.y * xc.y; y0.z += aa.y * xc.z; y0.w += aa.y * xc.w;
+            x1.x += ab.x * xa.x; x1.y += ab.x * xa.y; x1.z += ab.x * xa.z; x1.w += ab.x * xa.w;
+            y1.x += ab.y * xc.x; y1.y += ab.y * xc.y; y1.z += ab.y * xc.z; y1.w += ab.y * xc.w;
+        }
+        *reinterpret_cast<float4*>(sT + (16 * Ib + 2 * rp) * kStrideA + 16 * J + 4 * jq) =
+            make_float4(-(x0.x + y0.x), -(x0.y + y0.y), -(x0.z + y0.z), -(x0.w + y0.w));
+        *reinterpret_cast<float4*>(sT + (16 * Ib + 2 * rp + 1) * kStrideA + 16 * J + 4 * jq) =
+            make_float4(-(x1.x + y1.x), -(x1.y + y1.y), -(x1.z + y1.z), -(x1.w + y1.w));
+    }
+    __syncthreads();
+}
+
 __global__ void __launch_bounds__(512, 1)
 ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
               const __nv_bfloat16* __restrict__ v, const float* __restrict__ alpha,
               const float* __restrict__ beta, uint8_t* __restrict__ ws, int T_len, int H, int NT,
-              int l2norm, RopeParams rp, long long pos_offset) {
+              int total, int l2norm, RopeParams rp, long long pos_offset) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -187,21 +269,24 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
     float* BB = reinterpret_cast<float*>(sm + S_BB);
     float* gP = reinterpret_cast<float*>(sm + SM_P);
     float* gPar = reinterpret_cast<float*>(sm + SM_PAR);
+    float* gPre = reinterpret_cast<float*>(sm + SM_PRE);
+    float* gKef = reinterpret_cast<float*>(sm + SM_KEF);
+    float* gOff2 = reinterpret_cast<float*>(sm + SM_OFF2);
+    float* gOff3 = reinterpret_cast<float*>(sm + SM_OFF3);
     float* gGC = reinterpret_cast<float*>(sm + SM_GC);
     float* sb = reinterpret_cast<float*>(sm + SM_B);
     int* unsafe = reinterpret_cast<int*>(sm + SM_FLAGS);
     volatile int* abort_flag = unsafe + 4;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(unsafe + 8);
     uint64_t* bar = reinterpret_cast<uint64_t*>(unsafe + 16);
+    float* sA = reinterpret_cast<float*>(sm + S_A);
+    float* sT = reinterpret_cast<float*>(sm + S_T);
+    float* sX = reinterpret_cast<float*>(sm + S_X);
+    uint8_t* sM = sm + S_M;
+    uint8_t* out = sm + S_OUT;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int ch = blockIdx.x % NT, bh = blockIdx.x / NT;
-    const int b = bh / H, h = bh % H;
-    const int t0 = ch * kC;
-    const int nvalid = min(kC, T_len - t0);
-    uint8_t* wsc = ws + ((size_t)bh * NT + ch) * WS_CHUNK;
-    const size_t row0 = ((size_t)b * T_len + t0) * H + h;  // row (b, t0, h) of [B*T*H]
-    const size_t rs = (size_t)H;                            // stride between tokens, in rows
+    const size_t rs = (size_t)H;   // stride between tokens, in rows of [B*T*H]
 
     if (warp == 0) {
         tc::tmem_alloc(tmem_slot, 512);
@@ -212,476 +297,516 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
         tc::fence_mbar_init();
         *abort_flag = 0;
     }
-    if (tid < 4) unsafe[tid] = 0;
-    if (tid < 64) sb[tid] = tid < nvalid ? beta[row0 + tid * rs] : 0.f;
-
-    // ======== A1: alpha into shared memory (identity gates on padding rows), V tile ========
-    for (int e = tid; e < 64 * 32; e += 512) {
-        const int r = e >> 5, c4 = (e & 31) * 4;
-        float4 a = make_float4(1.f, 1.f, 1.f, 1.f);
-        if (r < nvalid) a = *reinterpret_cast<const float4*>(alpha + (row0 + r * rs) * kDK + c4);
-        *reinterpret_cast<float4*>(FB + r * 128 + c4) = a;
-    }
-    for (int e = tid; e < 64 * 16; e += 512) {
-        const int r = e >> 4, n8 = (e & 15) * 8;
-        uint4 x = make_uint4(0, 0, 0, 0);
-        if (r < nvalid) x = *reinterpret_cast<const uint4*>(v + (row0 + r * rs) * kDV + n8);
-        *reinterpret_cast<uint4*>(sm + S_V + tc::sw128_mnmajor(r, n8, 64)) = x;
-    }
-    __syncthreads();
-
-    // ======== A2: channel pass -- thread (channel c, block I) ========
-    {
-        const int c = tid & 127, I = tid >> 7;
-        float bbv = 1.f;
-#pragma unroll
-        for (int rl = 15; rl >= 0; --rl) {
-            const int r = 16 * I + rl;
-            BB[r * 128 + c] = bbv;
-            bbv *= fabsf(FB[r * 128 + c]);
-        }
-        float p = 1.f;
-        bool neg = false;
-#pragma unroll
-        for (int rl = 0; rl < 16; ++rl) {
-            const int r = 16 * I + rl;
-            const float a = FB[r * 128 + c];
-            p *= fabsf(a);
-            neg ^= (a < 0.f);
-            FB[r * 128 + c] = neg ? -p : p;   // a signed zero keeps the parity when p underflows
-        }
-        gP[I * 128 + c] = p;
-        gPar[I * 128 + c] = neg ? -1.f : 1.f;
-        if (!(p >= kDiagSafe)) unsafe[I] = 1;
-    }
-    __syncthreads();
-
-    // ======== A3: row pass -- thread (row r, 8-channel groups g and g + 8) ========
-    {
-        const int r = tid >> 3, g = tid & 7;
-        const int I = r >> 4, rl = r & 15;
-        const int cA = 8 * g, cB = 64 + 8 * g;
-        float qa[8], qb[8], ka[8], kb[8];
-        if (r < nvalid) {
-            const size_t o = (row0 + r * rs) * kDK;
-            unpack8(*reinterpret_cast<const uint4*>(q + o + cA), qa);
-            unpack8(*reinterpret_cast<const uint4*>(q + o + cB), qb);
-            unpack8(*reinterpret_cast<const uint4*>(k + o + cA), ka);
-            unpack8(*reinterpret_cast<const uint4*>(k + o + cB), kb);
-        } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) qa[i] = qb[i] = ka[i] = kb[i] = 0.f;
-        }
-        // row norms (the rotation preserves them): reduce over the 8 threads of the row
-        float sq = 0.f, sk = 0.f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            sq += qa[i] * qa[i] + qb[i] * qb[i];
-            sk += ka[i] * ka[i] + kb[i] * kb[i];
-        }
-        sq = group_sum<8>(sq);
-        sk = group_sum<8>(sk);
-        if (rp.enabled) {
-            const long long pos = pos_offset + t0 + r;
-            if (rp.convention == 0) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {   // pairs (cA + i, cB + i), frequency 8g + i
-                    float sn, cs;
-                    rope_sincos(pos, rp.inv_freq[8 * g + i], &sn, &cs);
-                    float x0 = qa[i], x1 = qb[i];
-                    qa[i] = x0 * cs - x1 * sn; qb[i] = x1 * cs + x0 * sn;
-                    x0 = ka[i]; x1 = kb[i];
-                    ka[i] = x0 * cs - x1 * sn; kb[i] = x1 * cs + x0 * sn;
-                }
-            } else {
-#pragma unroll
-                for (int m = 0; m < 4; ++m) {   // pairs (c, c + 1) inside each 8-channel group
-                    float sn, cs;
-                    rope_sincos(pos, rp.inv_freq[4 * g + m], &sn, &cs);
-                    float x0 = qa[2 * m], x1 = qa[2 * m + 1];
-                    qa[2 * m] = x0 * cs - x1 * sn; qa[2 * m + 1] = x1 * cs + x0 * sn;
-                    x0 = ka[2 * m]; x1 = ka[2 * m + 1];
-                    ka[2 * m] = x0 * cs - x1 * sn; ka[2 * m + 1] = x1 * cs + x0 * sn;
-                    rope_sincos(pos, rp.inv_freq[32 + 4 * g + m], &sn, &cs);
-                    x0 = qb[2 * m]; x1 = qb[2 * m + 1];
-                    qb[2 * m] = x0 * cs - x1 * sn; qb[2 * m + 1] = x1 * cs + x0 * sn;
-                    x0 = kb[2 * m]; x1 = kb[2 * m + 1];
-                    kb[2 * m] = x0 * cs - x1 * sn; kb[2 * m + 1] = x1 * cs + x0 * sn;
-                }
-            }
-        }
-        const float fq = l2norm ? rsqrtf(sq + kL2Eps) : 1.f;
-        const float fk = l2norm ? rsqrtf(sk + kL2Eps) : 1.f;
-        const bool diag_ok = !unsafe[I];
-
-        // the two 8-channel halves of this thread: cA.. and cB..
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            const int c0 = hh ? cB : cA;
-            const float* qx = hh ? qb : qa;
-            const float* kx = hh ? kb : ka;
-            float fb[8], kp[8], qp[8], acc[8], t8[8];
-            ld_f8(FB + r * 128 + c0, fb);
-            // parity before this block
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] = 1.f;
-            for (int J = 0; J < I; ++J) {
-                ld_f8(gPar + J * 128 + c0, t8);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] *= t8[i];
-            }
-            // k', q' with the full-chunk parity (sign(fb) is the block-local parity); |fb|
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float s = signbit(fb[i]) ? -acc[i] : acc[i];
-                kp[i] = kx[i] * fk * s;
-                qp[i] = qx[i] * fq * s;
-                fb[i] = fabsf(fb[i]);
-            }
-            // L tile: k' fb and q' fb
-#pragma unroll
-            for (int i = 0; i < 8; ++i) t8[i] = kp[i] * fb[i];
-            st16(sm + S_L, tc::sw128_kmajor(32 * I + rl, c0, 128), t8);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) t8[i] = qp[i] * fb[i];
-            st16(sm + S_L, tc::sw128_kmajor(32 * I + 16 + rl, c0, 128), t8);
-            // right operand of the diagonal block: k' / fb
-#pragma unroll
-            for (int i = 0; i < 8; ++i) t8[i] = diag_ok ? kp[i] * __frcp_rn(fb[i]) : 0.f;
-            st16(sm + S_B + btile_off(I), tc::sw128_kmajor(r, c0, 16 * (I + 1)), t8);
-            // right operands of the off-diagonal blocks I2 > I: k' bb prod_{I<J<I2} P_J
-            ld_f8(BB + r * 128 + c0, acc);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] *= kp[i];
-            for (int I2 = I + 1; I2 < 4; ++I2) {
-                st16(sm + S_B + btile_off(I2), tc::sw128_kmajor(r, c0, 16 * (I2 + 1)), acc);
-                if (I2 < 3) {
-                    ld_f8(gP + I2 * 128 + c0, t8);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) acc[i] *= t8[i];
-                }
-            }
-            // K_end = sigma_C (|gamma_C| / |gamma_r|) k' = sigma_C bb prod_{J>I} P_J k'
-            ld_f8(BB + r * 128 + c0, acc);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] *= kp[i];
-#pragma unroll
-            for (int J = 0; J < 4; ++J) {
-                ld_f8(gPar + J * 128 + c0, t8);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] *= t8[i];
-                if (J > I) {
-                    ld_f8(gP + J * 128 + c0, t8);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) acc[i] *= t8[i];
-                }
-            }
-            st16(sm + S_KE, tc::sw128_mnmajor(r, c0, 64), acc);
-            // |gamma_r| = prod_{J<I} P_J * fb:  K_gamma = |gamma_r| k', Q_gamma = |gamma_r| q'
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] = fb[i];
-            for (int J = 0; J < I; ++J) {
-                ld_f8(gP + J * 128 + c0, t8);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] *= t8[i];
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) t8[i] = acc[i] * kp[i];
-            st16(sm + S_KG, tc::sw128_mnmajor(r, c0, 64), t8);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) t8[i] = acc[i] * qp[i];
-            st16(sm + S_QG, tc::sw128_kmajor(r, c0, 64), t8);
-        }
-    }
-    // gamma_C (signed) per channel, for the diagonal of A_c
-    if (tid < 128) {
-        float gc = 1.f;
-#pragma unroll
-        for (int J = 0; J < 4; ++J) gc *= gP[J * 128 + tid] * gPar[J * 128 + tid];
-        gGC[tid] = gc;
-    }
-    tc::fence_proxy_async_smem();
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    uint32_t phase = 0;   // completions of `bar` so far
 
-    // ======== B: A and M block-rows on the tensor cores ========
-    if (tid == 0) {
-        const uint32_t l0 = tc::smem_u32(sm + S_L), b0 = tc::smem_u32(sm + S_B);
+    // persistent loop over chunk-heads ci = (batch*head) * NT + chunk
+    for (int ci = blockIdx.x; ci < total; ci += gridDim.x) {
+        const int ch = ci % NT, bh = ci / NT;
+        const int b = bh / H, h = bh % H;
+        const int t0 = ch * kC;
+        const int nvalid = min(kC, T_len - t0);
+        uint8_t* wsc = ws + (size_t)ci * WS_CHUNK;
+        const size_t row0 = ((size_t)b * T_len + t0) * H + h;
+
+        // ---- all global loads of this chunk-head, issued together (registers only) ----
+        const int rr = tid >> 3, g = tid & 7;               // row-pass coordinates
+        uint4 qkraw[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0),
+                          make_uint4(0, 0, 0, 0)};
+        if (rr < nvalid) {
+            const size_t o = (row0 + rr * rs) * kDK;
+            qkraw[0] = *reinterpret_cast<const uint4*>(q + o + 8 * g);
+            qkraw[1] = *reinterpret_cast<const uint4*>(q + o + 64 + 8 * g);
+            qkraw[2] = *reinterpret_cast<const uint4*>(k + o + 8 * g);
+            qkraw[3] = *reinterpret_cast<const uint4*>(k + o + 64 + 8 * g);
+        }
+        float4 araw[4];
 #pragma unroll
-        for (int J = 0; J < 4; ++J) {
-            const int n = 16 * (J + 1);
-            const uint32_t idesc = tc::idesc_bf16_f32(64, n, 0, 0);
+        for (int u = 0; u < 4; ++u) {
+            const int e = tid + 512 * u, r = e >> 5, c4 = (e & 31) * 4;
+            araw[u] = make_float4(1.f, 1.f, 1.f, 1.f);   // identity gates on padding rows
+            if (r < nvalid) araw[u] = *reinterpret_cast<const float4*>(alpha + (row0 + r * rs) * kDK + c4);
+        }
+        uint4 vraw[2];
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                uint64_t ad = tc::smem_desc_sw128(l0 + 4096 * J + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-                uint64_t bd = tc::smem_desc_sw128(b0 + btile_off(J) + (ks >> 2) * n * 128 + (ks & 3) * 32, 16, 1024);
-                tc::mma_bf16(tmem + amcol(J), ad, bd, idesc, ks > 0 ? 1u : 0u);
+        for (int u = 0; u < 2; ++u) {
+            const int e = tid + 512 * u, r = e >> 4, n8 = (e & 15) * 8;
+            vraw[u] = make_uint4(0, 0, 0, 0);
+            if (r < nvalid) vraw[u] = *reinterpret_cast<const uint4*>(v + (row0 + r * rs) * kDV + n8);
+        }
+        const float bval = (tid < 64 && tid < nvalid) ? beta[row0 + tid * rs] : 0.f;
+        // bring the next chunk-head of this CTA into L2 while this one computes: 640 lines of
+        // 128 bytes (q, k, v: 2 per row; alpha: 4 per row), one or two per thread
+        {
+            const int nci = ci + gridDim.x;
+            if (nci < total) {
+                const int nch = nci % NT, nbh = nci / NT;
+                const int nt0 = nch * kC, nv = min(kC, T_len - nt0);
+                const size_t nrow0 = ((size_t)(nbh / H) * T_len + nt0) * H + (nbh % H);
+                for (int li = tid; li < 640; li += 512) {
+                    const char* p;
+                    int r;
+                    if (li < 384) {
+                        const int which = li >> 7, rem = li & 127;
+                        r = rem >> 1;
+                        const __nv_bfloat16* base = which == 0 ? q : which == 1 ? k : v;
+                        p = reinterpret_cast<const char*>(base + (nrow0 + r * rs) * kDK) + 128 * (rem & 1);
+                    } else {
+                        const int rem = li - 384;
+                        r = rem >> 2;
+                        p = reinterpret_cast<const char*>(alpha + (nrow0 + r * rs) * kDK) + 128 * (rem & 3);
+                    }
+                    if (r < nv) tc::prefetch_line_l2(p);
+                }
             }
         }
-        tc::mma_commit(bar);
-    }
-    tc::mbar_wait(bar, 0, abort_flag);
-    tc::tc_fence_after();
-    float* sA = reinterpret_cast<float*>(sm + S_A);
-    uint8_t* sM = sm + S_M;
-    {
-        // M = 64 accumulator of block-row J: k rows in lanes 0..15, q rows in lanes 32..47.
-        // Warp w reads TMEM lanes 32 (w % 4) ..: w % 4 == 0 -> A part, 1 -> M part; J = w / 4.
-        const int quarter = warp & 3, J = warp >> 2;
-        if (quarter < 2) {
-            const int n = 16 * (J + 1);
-            const int r = 16 * J + (lane & 15);
-            for (int c0 = 0; c0 < n; c0 += 16) {
-                float x[16];
-                tc::tmem_ld16(tc::tmem_addr(tmem, 32 * quarter, amcol(J) + c0), x);
-                tc::tmem_ld_wait();
-                if (lane < 16) {
-                    if (quarter == 0) {
-                        const float br = sb[r];
+        // the previous chunk-head's bulk store must have finished reading shared memory
+        if (tid == 0) tc::bulk_wait_read_all();
+        __syncthreads();
+
+        // ======== A1: alpha and V into shared memory ========
+        if (tid < 4) unsafe[tid] = 0;
+        if (tid < 64) sb[tid] = bval;
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) x[i] = (c0 + i) < r ? br * x[i] : 0.f;
+        for (int u = 0; u < 4; ++u) {
+            const int e = tid + 512 * u, r = e >> 5, c4 = (e & 31) * 4;
+            *reinterpret_cast<float4*>(FB + r * 128 + c4) = araw[u];
+        }
 #pragma unroll
-                        for (int i = 0; i < 16; i += 4)
-                            *reinterpret_cast<float4*>(sA + r * kStrideA + c0 + i) =
-                                make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
-                    } else {
+        for (int u = 0; u < 2; ++u) {
+            const int e = tid + 512 * u, r = e >> 4, n8 = (e & 15) * 8;
+            *reinterpret_cast<uint4*>(sm + S_V + tc::sw128_mnmajor(r, n8, 64)) = vraw[u];
+        }
+        __syncthreads();
+
+        // ======== A2: channel pass -- thread (channel c, block I) ========
+        const int cc = tid & 127, cI = tid >> 7;
+        {
+            float bbv = 1.f;
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) x[i] = (c0 + i) <= r ? x[i] : 0.f;
-                        st16(sM, tc::sw128_kmajor(r, c0, 64), x);
-                        st16(sM, tc::sw128_kmajor(r, c0 + 8, 64), x + 8);
+            for (int rl = 15; rl >= 0; --rl) {
+                const int r = 16 * cI + rl;
+                BB[r * 128 + cc] = bbv;
+                bbv *= fabsf(FB[r * 128 + cc]);
+            }
+            float p = 1.f;
+            bool neg = false;
+#pragma unroll
+            for (int rl = 0; rl < 16; ++rl) {
+                const int r = 16 * cI + rl;
+                const float a = FB[r * 128 + cc];
+                p *= fabsf(a);
+                neg ^= (a < 0.f);
+                FB[r * 128 + cc] = neg ? -p : p;   // a signed zero keeps the parity on underflow
+            }
+            gP[cI * 128 + cc] = p;
+            gPar[cI * 128 + cc] = neg ? -1.f : 1.f;
+            if (!(p >= kDiagSafe)) unsafe[cI] = 1;
+        }
+        __syncthreads();
+        // A2b: per-(block, channel) factors; the parity before the block goes into FB's sign
+        {
+            float spre = 1.f, pre = 1.f, suf = 1.f, sC = 1.f, all = 1.f;
+#pragma unroll
+            for (int J = 0; J < 4; ++J) {
+                const float P = gP[J * 128 + cc], S = gPar[J * 128 + cc];
+                sC *= S;
+                all *= P;
+                if (J < cI) { spre *= S; pre *= P; }
+                if (J > cI) suf *= P;
+            }
+            if (spre < 0.f) {
+#pragma unroll
+                for (int rl = 0; rl < 16; ++rl) FB[(16 * cI + rl) * 128 + cc] = -FB[(16 * cI + rl) * 128 + cc];
+            }
+            gPre[cI * 128 + cc] = pre;
+            gKef[cI * 128 + cc] = sC * suf;
+            gOff2[cI * 128 + cc] = cI + 1 < 4 ? gP[(cI + 1) * 128 + cc] : 0.f;
+            gOff3[cI * 128 + cc] = cI + 2 < 4 ? gP[(cI + 1) * 128 + cc] * gP[(cI + 2) * 128 + cc] : 0.f;
+            if (cI == 0) gGC[cc] = sC * all;   // gamma_C (signed)
+        }
+        __syncthreads();
+
+        // ======== A3: row pass -- thread (row r, 8-channel groups g and g + 8) ========
+        {
+            const int r = rr, I = r >> 4, rl = r & 15;
+            const int cA = 8 * g, cB = 64 + 8 * g;
+            float qa[8], qb[8], ka[8], kb[8];
+            unpack8(qkraw[0], qa);
+            unpack8(qkraw[1], qb);
+            unpack8(qkraw[2], ka);
+            unpack8(qkraw[3], kb);
+            // row norms (the rotation preserves them): reduce over the 8 threads of the row
+            float sq = 0.f, sk = 0.f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                sq += qa[i] * qa[i] + qb[i] * qb[i];
+                sk += ka[i] * ka[i] + kb[i] * kb[i];
+            }
+            sq = group_sum<8>(sq);
+            sk = group_sum<8>(sk);
+            if (rp.enabled) {
+                const long long pos = pos_offset + t0 + r;
+                if (rp.convention == 0) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {   // pairs (cA + i, cB + i), frequency 8g + i
+                        float sn, cs;
+                        rope_sincos(pos, rp.inv_freq[8 * g + i], &sn, &cs);
+                        float x0 = qa[i], x1 = qb[i];
+                        qa[i] = x0 * cs - x1 * sn; qb[i] = x1 * cs + x0 * sn;
+                        x0 = ka[i]; x1 = kb[i];
+                        ka[i] = x0 * cs - x1 * sn; kb[i] = x1 * cs + x0 * sn;
+                    }
+                } else {
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {   // pairs (c, c + 1) inside each 8-channel group
+                        float sn, cs;
+                        rope_sincos(pos, rp.inv_freq[4 * g + m], &sn, &cs);
+                        float x0 = qa[2 * m], x1 = qa[2 * m + 1];
+                        qa[2 * m] = x0 * cs - x1 * sn; qa[2 * m + 1] = x1 * cs + x0 * sn;
+                        x0 = ka[2 * m]; x1 = ka[2 * m + 1];
+                        ka[2 * m] = x0 * cs - x1 * sn; ka[2 * m + 1] = x1 * cs + x0 * sn;
+                        rope_sincos(pos, rp.inv_freq[32 + 4 * g + m], &sn, &cs);
+                        x0 = qb[2 * m]; x1 = qb[2 * m + 1];
+                        qb[2 * m] = x0 * cs - x1 * sn; qb[2 * m + 1] = x1 * cs + x0 * sn;
+                        x0 = kb[2 * m]; x1 = kb[2 * m + 1];
+                        kb[2 * m] = x0 * cs - x1 * sn; kb[2 * m + 1] = x1 * cs + x0 * sn;
                     }
                 }
             }
-            if (lane < 16) {
-                const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                for (int j = n; j < 64; j += 8) {
-                    if (quarter == 0) {
-                        *reinterpret_cast<float4*>(sA + r * kStrideA + j) = make_float4(0.f, 0.f, 0.f, 0.f);
-                        *reinterpret_cast<float4*>(sA + r * kStrideA + j + 4) = make_float4(0.f, 0.f, 0.f, 0.f);
-                    } else {
-                        st16(sM, tc::sw128_kmajor(r, j, 64), z);
-                    }
+            const float fq = l2norm ? rsqrtf(sq + kL2Eps) : 1.f;
+            const float fk = l2norm ? rsqrtf(sk + kL2Eps) : 1.f;
+            const bool diag_ok = !unsafe[I];
+            // A3a: the operands of the A / M products (L and B tiles)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int c0 = hh ? cB : cA;
+                const float* qx = hh ? qb : qa;
+                const float* kx = hh ? kb : ka;
+                float fb[8], kp[8], qp[8], acc[8], t8[8];
+                ld_f8(FB + r * 128 + c0, fb);   // |fb| with the full-chunk parity as its sign
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float sg = signbit(fb[i]) ? -1.f : 1.f;
+                    kp[i] = kx[i] * fk * sg;
+                    qp[i] = qx[i] * fq * sg;
+                    fb[i] = fabsf(fb[i]);
+                }
+                // L tile: k' fb and q' fb
+#pragma unroll
+                for (int i = 0; i < 8; ++i) t8[i] = kp[i] * fb[i];
+                st16(sm + S_L, tc::sw128_kmajor(32 * I + rl, c0, 128), t8);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) t8[i] = qp[i] * fb[i];
+                st16(sm + S_L, tc::sw128_kmajor(32 * I + 16 + rl, c0, 128), t8);
+                // right operand of the diagonal block: k' / fb
+#pragma unroll
+                for (int i = 0; i < 8; ++i) t8[i] = diag_ok ? kp[i] * __frcp_rn(fb[i]) : 0.f;
+                st16(sm + S_B + btile_off(I), tc::sw128_kmajor(r, c0, 16 * (I + 1)), t8);
+                // off-diagonal right operands k' bb prod_{I<J<I2} P_J
+                ld_f8(BB + r * 128 + c0, acc);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] *= kp[i];
+                if (I < 3) st16(sm + S_B + btile_off(I + 1), tc::sw128_kmajor(r, c0, 16 * (I + 2)), acc);
+                if (I < 2) {
+                    ld_f8(gOff2 + I * 128 + c0, t8);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) t8[i] *= acc[i];
+                    st16(sm + S_B + btile_off(I + 2), tc::sw128_kmajor(r, c0, 16 * (I + 3)), t8);
+                }
+                if (I < 1) {
+                    ld_f8(gOff3 + I * 128 + c0, t8);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) t8[i] *= acc[i];
+                    st16(sm + S_B + btile_off(3), tc::sw128_kmajor(r, c0, 64), t8);
                 }
             }
-        }
-    }
-    tc::tc_fence_before();
-    __syncthreads();
+            tc::fence_proxy_async_smem();
+            tc::tc_fence_before();
+            __syncthreads();
+            tc::tc_fence_after();
 
-    // exact recomputation of diagonal blocks whose gate total fell below 2^-60 (rare)
-    for (int J = 0; J < 4; ++J) {
-        if (!unsafe[J]) continue;
-        float* fq = reinterpret_cast<float*>(sm + S_FQ);
-        float* fk = reinterpret_cast<float*>(sm + S_FK);
+            // ======== B: A and M block-rows on the tensor cores (overlaps A3b) ========
+            if (tid == 0) {
+                const uint32_t l0 = tc::smem_u32(sm + S_L), b0 = tc::smem_u32(sm + S_B);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+#pragma unroll
+                    for (int J = 0; J < 4; ++J) {
+                        const int n = 16 * (J + 1);
+                        const uint64_t ad = tc::smem_desc_sw128(l0 + 4096 * J + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+                        const uint64_t bd = tc::smem_desc_sw128(b0 + btile_off(J) + (ks >> 2) * n * 128 + (ks & 3) * 32, 16, 1024);
+                        tc::mma_bf16(tmem + amcol(J), ad, bd, tc::idesc_bf16_f32(64, n, 0, 0), ks > 0 ? 1u : 0u);
+                    }
+                }
+                tc::mma_commit(bar);
+            }
+
+            // A3b: K_end = k' bb KEF, K_gamma = |gamma_r| k', Q_gamma = |gamma_r| q'
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int c0 = hh ? cB : cA;
+                const float* qx = hh ? qb : qa;
+                const float* kx = hh ? kb : ka;
+                float fb[8], kp[8], qp[8], acc[8], t8[8];
+                ld_f8(FB + r * 128 + c0, fb);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float sg = signbit(fb[i]) ? -1.f : 1.f;
+                    kp[i] = kx[i] * fk * sg;
+                    qp[i] = qx[i] * fq * sg;
+                    fb[i] = fabsf(fb[i]);
+                }
+                ld_f8(BB + r * 128 + c0, acc);
+                ld_f8(gKef + I * 128 + c0, t8);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) t8[i] *= acc[i] * kp[i];
+                st16(sm + S_KE, tc::sw128_mnmajor(r, c0, 64), t8);
+                ld_f8(gPre + I * 128 + c0, acc);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) { acc[i] *= fb[i]; t8[i] = acc[i] * kp[i]; }
+                st16(sm + S_KG, tc::sw128_mnmajor(r, c0, 64), t8);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) t8[i] = acc[i] * qp[i];
+                st16(sm + S_QG, tc::sw128_kmajor(r, c0, 64), t8);
+            }
+        }
+        tc::mbar_wait(bar, phase & 1, abort_flag);
+        ++phase;
+        tc::tc_fence_after();
         {
-            const int rl = warp, r = 16 * J + rl;
-            if (r < nvalid)
-                fallback_row(q, k, alpha, row0, rs, r, lane, rp, pos_offset + t0 + r, l2norm,
-                             fq + rl * 128, fk + rl * 128);
-            else
-                for (int c = lane; c < 128; c += 32) fq[rl * 128 + c] = fk[rl * 128 + c] = 0.f;
-        }
-        __syncthreads();
-        for (int pr = tid; pr < 136; pr += 512) {
-            int rl = 0;
-            while ((rl + 1) * (rl + 2) / 2 <= pr) ++rl;
-            const int jl = pr - rl * (rl + 1) / 2;
-            const int r = 16 * J + rl, j = 16 * J + jl;
-            float accA = 0.f, accM = 0.f;
-            for (int c = 0; c < kDK; ++c) {
-                float f = 1.f;
-                for (int tau = j + 1; tau <= r; ++tau)
-                    f *= tau < nvalid ? fabsf(alpha[(row0 + tau * rs) * kDK + c]) : 1.f;
-                const float kj = fk[jl * 128 + c] * f;
-                accA += fk[rl * 128 + c] * kj;
-                accM += fq[rl * 128 + c] * kj;
-            }
-            sA[r * kStrideA + j] = j < r ? sb[r] * accA : 0.f;
-            *reinterpret_cast<__nv_bfloat16*>(sM + tc::sw128_kmajor(r, j, 64)) = __float2bfloat16_rn(accM);
-        }
-        __syncthreads();
-    }
-
-    // ======== C: T = (I + A)^-1 (fp32), T' = T diag(beta) (bf16) ========
-    float* sT = reinterpret_cast<float*>(sm + S_T);
-    float* sX = reinterpret_cast<float*>(sm + S_X);
-    for (int e = tid; e < 64 * 64; e += 512) {
-        const int r = e >> 6, j = e & 63;
-        if ((j >> 4) > (r >> 4)) sT[r * kStrideA + j] = 0.f;
-    }
-    if (warp < 4 && lane < 16) {
-        const int J = warp, l = lane, base = 16 * J;
-        float tcol[16];
+            // M = 64 accumulator of block-row J: k rows in lanes 0..15, q rows in lanes 32..47.
+            // Warp w reads TMEM lanes 32 (w % 4) ..: w % 4 == 0 -> A part, 1 -> M part; J = w / 4.
+            const int quarter = warp & 3, J = warp >> 2;
+            if (quarter < 2) {
+                const int n = 16 * (J + 1);
+                const int r = 16 * J + (lane & 15);
+                for (int c0 = 0; c0 < n; c0 += 16) {
+                    float x[16];
+                    tc::tmem_ld16_sync(tc::tmem_addr(tmem, 32 * quarter, amcol(J) + c0), x);
+                    if (lane < 16) {
+                        if (quarter == 0) {
+                            const float br = sb[r];
 #pragma unroll
-        for (int rr = 0; rr < 16; ++rr) {
-            float a0 = 0.f, a1 = 0.f;
+                            for (int i = 0; i < 16; ++i) x[i] = (c0 + i) < r ? br * x[i] : 0.f;
 #pragma unroll
-            for (int m = 0; m < 16; m += 2) {
-                if (m < rr) a0 += sA[(base + rr) * kStrideA + base + m] * tcol[m];
-                if (m + 1 < rr) a1 += sA[(base + rr) * kStrideA + base + m + 1] * tcol[m + 1];
-            }
-            tcol[rr] = rr < l ? 0.f : (rr == l ? 1.f : -(a0 + a1));
-        }
-#pragma unroll
-        for (int rr = 0; rr < 16; ++rr) sT[(base + rr) * kStrideA + base + l] = tcol[rr];
-    }
-    __syncthreads();
-    for (int Ib = 1; Ib < 4; ++Ib) {
-        const int nq = 4 * Ib;   // column quads in [0, 16 Ib)
-        // X = sum_{K = J..Ib-1} A_{Ib,K} T_{K,J}: thread per (row rl, 4 columns)
-        for (int e = tid; e < 16 * nq; e += 512) {
-            const int rl = e / nq, j0 = 4 * (e % nq);
-            const int m0 = 16 * (j0 >> 4);
-            float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
-            for (int m = m0; m < 16 * Ib; ++m) {
-                const float a = sA[(16 * Ib + rl) * kStrideA + m];
-                const float4 t = *reinterpret_cast<const float4*>(sT + m * kStrideA + j0);
-                x0 += a * t.x; x1 += a * t.y; x2 += a * t.z; x3 += a * t.w;
-            }
-            *reinterpret_cast<float4*>(sX + rl * 48 + j0) = make_float4(x0, x1, x2, x3);
-        }
-        __syncthreads();
-        for (int e = tid; e < 16 * nq; e += 512) {
-            const int rl = e / nq, j0 = 4 * (e % nq);
-            float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
-#pragma unroll
-            for (int m = 0; m < 16; ++m) {
-                const float a = sT[(16 * Ib + rl) * kStrideA + 16 * Ib + m];
-                const float4 x = *reinterpret_cast<const float4*>(sX + m * 48 + j0);
-                y0 += a * x.x; y1 += a * x.y; y2 += a * x.z; y3 += a * x.w;
-            }
-            *reinterpret_cast<float4*>(sT + (16 * Ib + rl) * kStrideA + j0) = make_float4(-y0, -y1, -y2, -y3);
-        }
-        __syncthreads();
-    }
-    for (int e = tid; e < 64 * 8; e += 512) {
-        const int r = e >> 3, j0 = (e & 7) * 8;
-        float y[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) y[i] = sT[r * kStrideA + j0 + i] * sb[j0 + i];
-        st16(sm + S_TB, tc::sw128_kmajor(r, j0, 64), y);
-    }
-    tc::fence_proxy_async_smem();
-    tc::tc_fence_before();
-    __syncthreads();
-    tc::tc_fence_after();
-
-    // ======== D: W = T' K_gamma, U~ = T' V  (M = 64, N = 128 each, K = 64) ========
-    if (tid == 0) {
-        const uint32_t a0 = tc::smem_u32(sm + S_TB);
-        const uint32_t kg = tc::smem_u32(sm + S_KG), vv = tc::smem_u32(sm + S_V);
-        const uint32_t idesc = tc::idesc_bf16_f32(64, 128, 0, 1);
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t ad = tc::smem_desc_sw128(a0 + ks * 32, 16, 1024);
-            tc::mma_bf16(tmem, ad, tc::smem_desc_sw128(kg + ks * 2048, 8192, 1024), idesc, ks > 0);
-            tc::mma_bf16(tmem + 128, ad, tc::smem_desc_sw128(vv + ks * 2048, 8192, 1024), idesc, ks > 0);
-        }
-        tc::mma_commit(bar);
-    }
-    tc::mbar_wait(bar, 1, abort_flag);
-    tc::tc_fence_after();
-    {
-        // warp w: rows 16 (w % 4) + lane (lane < 16); 64-column slice w / 4:
-        // slices 0, 1 -> W columns 0..127, slices 2, 3 -> U~ columns 0..127
-        const int quarter = warp & 3, slice = warp >> 2;
-        const int r = 16 * quarter + (lane & 15);
-        uint8_t* dst = sm + (slice < 2 ? S_W : S_U);
-        const int n0 = 64 * (slice & 1);
-#pragma unroll
-        for (int c0 = 0; c0 < 64; c0 += 16) {
-            float x[16];
-            tc::tmem_ld16(tc::tmem_addr(tmem, 32 * quarter, 64 * slice + c0), x);
-            tc::tmem_ld_wait();
-            if (lane < 16) {
-                st16(dst, tc::sw128_mnmajor(r, n0 + c0, 64), x);
-                st16(dst, tc::sw128_mnmajor(r, n0 + c0 + 8, 64), x + 8);
-            }
-        }
-    }
-    tc::fence_proxy_async_smem();
-    tc::tc_fence_before();
-    __syncthreads();
-    tc::tc_fence_after();
-
-    // ======== F: M [W | U~] (M = 64) and K_end^T [W | U~] (M = 128, MN-major A) ========
-    if (tid == 0) {
-        const uint32_t am = tc::smem_u32(sm + S_M), ke = tc::smem_u32(sm + S_KE);
-        const uint32_t w0 = tc::smem_u32(sm + S_W), u0 = tc::smem_u32(sm + S_U);
-        const uint32_t id64 = tc::idesc_bf16_f32(64, 128, 0, 1);
-        const uint32_t id128 = tc::idesc_bf16_f32(128, 128, 1, 1);
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t bw = tc::smem_desc_sw128(w0 + ks * 2048, 8192, 1024);
-            const uint64_t bu = tc::smem_desc_sw128(u0 + ks * 2048, 8192, 1024);
-            const uint64_t adm = tc::smem_desc_sw128(am + ks * 32, 16, 1024);
-            const uint64_t ade = tc::smem_desc_sw128(ke + ks * 2048, 8192, 1024);
-            tc::mma_bf16(tmem, adm, bw, id64, ks > 0);
-            tc::mma_bf16(tmem + 128, adm, bu, id64, ks > 0);
-            tc::mma_bf16(tmem + 256, ade, bw, id128, ks > 0);
-            tc::mma_bf16(tmem + 384, ade, bu, id128, ks > 0);
-        }
-        tc::mma_commit(bar);
-    }
-    tc::mbar_wait(bar, 0, abort_flag);
-    tc::tc_fence_after();
-    {
-        const int quarter = warp & 3, slice = warp >> 2;
-        // (1) M = 64 products: rows 16 quarter + lane; slices 0, 1 -> Q', 2, 3 -> O_loc
-        {
-            const int r = 16 * quarter + (lane & 15);
-            const int n0 = 64 * (slice & 1);
-#pragma unroll
-            for (int c0 = 0; c0 < 64; c0 += 16) {
-                float x[16];
-                tc::tmem_ld16(tc::tmem_addr(tmem, 32 * quarter, 64 * slice + c0), x);
-                tc::tmem_ld_wait();
-                if (lane < 16) {
-#pragma unroll
-                    for (int hc = 0; hc < 2; ++hc) {
-                        const int n = n0 + c0 + 8 * hc;
-                        if (slice < 2) {
-                            float qg[8];
-                            unpack8(*reinterpret_cast<const uint4*>(sm + S_QG + tc::sw128_kmajor(r, n, 64)), qg);
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) qg[i] -= x[8 * hc + i];
-                            *reinterpret_cast<uint4*>(wsc + WS_QP + tc::sw128_kmajor(r, n, 64)) = pack8(qg);
+                            for (int i = 0; i < 16; i += 4)
+                                *reinterpret_cast<float4*>(sA + r * kStrideA + c0 + i) =
+                                    make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
                         } else {
-                            *reinterpret_cast<uint4*>(wsc + WS_TILES + (n >> 5) * WS_TILE + WS_TILE_O +
-                                                      (r * 32 + (n & 31)) * 2) = pack8(x + 8 * hc);
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) x[i] = (c0 + i) <= r ? x[i] : 0.f;
+                            st16(sM, tc::sw128_kmajor(r, c0, 64), x);
+                            st16(sM, tc::sw128_kmajor(r, c0 + 8, 64), x + 8);
+                        }
+                    }
+                }
+                if (lane < 16) {
+                    const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    for (int j = n; j < 64; j += 8) {
+                        if (quarter == 0) {
+                            *reinterpret_cast<float4*>(sA + r * kStrideA + j) = make_float4(0.f, 0.f, 0.f, 0.f);
+                            *reinterpret_cast<float4*>(sA + r * kStrideA + j + 4) = make_float4(0.f, 0.f, 0.f, 0.f);
+                        } else {
+                            st16(sM, tc::sw128_kmajor(r, j, 64), z);
                         }
                     }
                 }
             }
         }
-        // (2) M = 128 products: row c' = 32 quarter + lane; slices 0, 1 -> A_c, 2, 3 -> B_c
+        tc::tc_fence_before();
+        __syncthreads();
+
+        // exact recomputation of diagonal blocks whose gate total fell below 2^-60 (rare)
+        for (int J = 0; J < 4; ++J) {
+            if (!unsafe[J]) continue;
+            float* fq = reinterpret_cast<float*>(sm + S_FQ);
+            float* fk = reinterpret_cast<float*>(sm + S_FK);
+            {
+                const int rl = warp, r = 16 * J + rl;
+                if (r < nvalid)
+                    fallback_row(q, k, alpha, row0, rs, r, lane, rp, pos_offset + t0 + r, l2norm,
+                                 fq + rl * 128, fk + rl * 128);
+                else
+                    for (int c = lane; c < 128; c += 32) fq[rl * 128 + c] = fk[rl * 128 + c] = 0.f;
+            }
+            __syncthreads();
+            for (int pr = tid; pr < 136; pr += 512) {
+                int rl = 0;
+                while ((rl + 1) * (rl + 2) / 2 <= pr) ++rl;
+                const int jl = pr - rl * (rl + 1) / 2;
+                const int r = 16 * J + rl, j = 16 * J + jl;
+                float accA = 0.f, accM = 0.f;
+                for (int c = 0; c < kDK; ++c) {
+                    float f = 1.f;
+                    for (int tau = j + 1; tau <= r; ++tau)
+                        f *= tau < nvalid ? fabsf(alpha[(row0 + tau * rs) * kDK + c]) : 1.f;
+                    const float kj = fk[jl * 128 + c] * f;
+                    accA += fk[rl * 128 + c] * kj;
+                    accM += fq[rl * 128 + c] * kj;
+                }
+                sA[r * kStrideA + j] = j < r ? sb[r] * accA : 0.f;
+                *reinterpret_cast<__nv_bfloat16*>(sM + tc::sw128_kmajor(r, j, 64)) = __float2bfloat16_rn(accM);
+            }
+            __syncthreads();
+        }
+
+        // ======== C: T = (I + A)^-1 (fp32), T' = T diag(beta) (bf16) ========
+        for (int e = tid; e < 64 * 64; e += 512) {
+            const int r = e >> 6, j = e & 63;
+            if ((j >> 4) > (r >> 4)) sT[r * kStrideA + j] = 0.f;
+        }
+        if (warp < 4 && lane < 16) {
+            const int J = warp, l = lane, base = 16 * J;
+            float tcol[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+                for (int m = 0; m < 16; m += 2) {
+                    if (m < i) a0 += sA[(base + i) * kStrideA + base + m] * tcol[m];
+                    if (m + 1 < i) a1 += sA[(base + i) * kStrideA + base + m + 1] * tcol[m + 1];
+                }
+                tcol[i] = i < l ? 0.f : (i == l ? 1.f : -(a0 + a1));
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) sT[(base + i) * kStrideA + base + l] = tcol[i];
+        }
+        __syncthreads();
         {
-            const int cr = 32 * quarter + lane;
+            float* sPt = reinterpret_cast<float*>(sm + S_PT);
+            t_offdiag_level<1>(sA, sT, sX, sPt, tid);
+            t_offdiag_level<2>(sA, sT, sX, sPt, tid);
+            t_offdiag_level<3>(sA, sT, sX, sPt, tid);
+        }
+        for (int e = tid; e < 64 * 8; e += 512) {
+            const int r = e >> 3, j0 = (e & 7) * 8;
+            float y[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) y[i] = sT[r * kStrideA + j0 + i] * sb[j0 + i];
+            st16(sm + S_TB, tc::sw128_kmajor(r, j0, 64), y);
+        }
+        tc::fence_proxy_async_smem();
+        tc::tc_fence_before();
+        __syncthreads();
+        tc::tc_fence_after();
+
+        // ======== D: W = T' K_gamma, U~ = T' V  (M = 64, N = 128 each, K = 64) ========
+        if (tid == 0) {
+            const uint32_t a0 = tc::smem_u32(sm + S_TB);
+            const uint32_t kg = tc::smem_u32(sm + S_KG), vv = tc::smem_u32(sm + S_V);
+            const uint32_t idesc = tc::idesc_bf16_f32(64, 128, 0, 1);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                const uint64_t ad = tc::smem_desc_sw128(a0 + ks * 32, 16, 1024);
+                tc::mma_bf16(tmem, ad, tc::smem_desc_sw128(kg + ks * 2048, 8192, 1024), idesc, ks > 0);
+                tc::mma_bf16(tmem + 128, ad, tc::smem_desc_sw128(vv + ks * 2048, 8192, 1024), idesc, ks > 0);
+            }
+            tc::mma_commit(bar);
+        }
+        tc::mbar_wait(bar, phase & 1, abort_flag);
+        ++phase;
+        tc::tc_fence_after();
+        {
+            // warp w: rows 16 (w % 4) + lane (lane < 16); 64-column slice w / 4:
+            // slices 0, 1 -> W columns 0..127, slices 2, 3 -> U~ columns 0..127
+            const int quarter = warp & 3, slice = warp >> 2;
+            const int r = 16 * quarter + (lane & 15);
+            uint8_t* dst = sm + (slice < 2 ? S_W : S_U);
             const int n0 = 64 * (slice & 1);
-            const float gc = gGC[cr];
+            float x[64];
+            tc::tmem_ld64_sync(tc::tmem_addr(tmem, 32 * quarter, 64 * slice), x);
+            if (lane < 16) {
 #pragma unroll
-            for (int c0 = 0; c0 < 64; c0 += 16) {
-                float x[16];
-                tc::tmem_ld16(tc::tmem_addr(tmem, 32 * quarter, 256 + 64 * slice + c0), x);
-                tc::tmem_ld_wait();
+                for (int c0 = 0; c0 < 64; c0 += 8) st16(dst, tc::sw128_mnmajor(r, n0 + c0, 64), x + c0);
+            }
+        }
+        tc::fence_proxy_async_smem();
+        tc::tc_fence_before();
+        __syncthreads();
+        tc::tc_fence_after();
+
+        // ======== F: M [W | U~] (M = 64) and K_end^T [W | U~] (M = 128, MN-major A) ========
+        if (tid == 0) {
+            const uint32_t am = tc::smem_u32(sm + S_M), ke = tc::smem_u32(sm + S_KE);
+            const uint32_t w0 = tc::smem_u32(sm + S_W), u0 = tc::smem_u32(sm + S_U);
+            const uint32_t id64 = tc::idesc_bf16_f32(64, 128, 0, 1);
+            const uint32_t id128 = tc::idesc_bf16_f32(128, 128, 1, 1);
 #pragma unroll
-                for (int hc = 0; hc < 2; ++hc) {
-                    const int n = n0 + c0 + 8 * hc;
-                    float y[8];
+            for (int ks = 0; ks < 4; ++ks) {
+                const uint64_t bw = tc::smem_desc_sw128(w0 + ks * 2048, 8192, 1024);
+                const uint64_t bu = tc::smem_desc_sw128(u0 + ks * 2048, 8192, 1024);
+                const uint64_t adm = tc::smem_desc_sw128(am + ks * 32, 16, 1024);
+                const uint64_t ade = tc::smem_desc_sw128(ke + ks * 2048, 8192, 1024);
+                tc::mma_bf16(tmem, adm, bw, id64, ks > 0);
+                tc::mma_bf16(tmem + 128, adm, bu, id64, ks > 0);
+                tc::mma_bf16(tmem + 256, ade, bw, id128, ks > 0);
+                tc::mma_bf16(tmem + 384, ade, bu, id128, ks > 0);
+            }
+            tc::mma_commit(bar);
+        }
+        tc::mbar_wait(bar, phase & 1, abort_flag);
+        ++phase;
+        tc::tc_fence_after();
+        // ======== G: results into the shared staging image, then one bulk store ========
+        {
+            const int quarter = warp & 3, slice = warp >> 2;
+            // (1) M = 64 products: rows 16 quarter + lane; slices 0, 1 -> Q', 2, 3 -> O_loc
+            {
+                const int r = 16 * quarter + (lane & 15);
+                const int n0 = 64 * (slice & 1);
+                float x[64];
+                tc::tmem_ld64_sync(tc::tmem_addr(tmem, 32 * quarter, 64 * slice), x);
+                if (lane < 16) {
+#pragma unroll
+                    for (int c0 = 0; c0 < 64; c0 += 8) {
+                        const int n = n0 + c0;
+                        if (slice < 2) {
+                            float qg[8];
+                            unpack8(*reinterpret_cast<const uint4*>(sm + S_QG + tc::sw128_kmajor(r, n, 64)), qg);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) qg[i] -= x[c0 + i];
+                            st16(out, WS_QP + tc::sw128_kmajor(r, n, 64), qg);
+                        } else {
+                            st16(out, WS_TILES + (n >> 5) * WS_TILE + WS_TILE_O + (r * 32 + (n & 31)) * 2, x + c0);
+                        }
+                    }
+                }
+            }
+            // (2) M = 128 products: row c' = 32 quarter + lane; slices 0, 1 -> A_c, 2, 3 -> B_c
+            {
+                const int cr = 32 * quarter + lane;
+                const int n0 = 64 * (slice & 1);
+                const float gc = gGC[cr];
+                float x[64];
+                tc::tmem_ld64_sync(tc::tmem_addr(tmem, 32 * quarter, 256 + 64 * slice), x);
+#pragma unroll
+                for (int c0 = 0; c0 < 64; c0 += 8) {
+                    const int n = n0 + c0;
                     if (slice < 2) {
+                        float y[8];
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) y[i] = (n + i == cr ? gc : 0.f) - x[8 * hc + i];
-                        *reinterpret_cast<uint4*>(wsc + WS_AC + tc::sw128_kmajor(cr, n, 128)) = pack8(y);
+                        for (int i = 0; i < 8; ++i) y[i] = (n + i == cr ? gc : 0.f) - x[c0 + i];
+                        st16(out, WS_AC + tc::sw128_kmajor(cr, n, 128), y);
                     } else {
-                        *reinterpret_cast<uint4*>(wsc + WS_TILES + (n >> 5) * WS_TILE +
-                                                  (cr * 32 + (n & 31)) * 2) = pack8(x + 8 * hc);
+                        st16(out, WS_TILES + (n >> 5) * WS_TILE + (cr * 32 + (n & 31)) * 2, x + c0);
                     }
                 }
             }
         }
+        tc::fence_proxy_async_smem();
+        tc::tc_fence_before();
+        __syncthreads();
+        tc::tc_fence_after();
+        if (tid == 0) {
+            tc::bulk_s2g(wsc, out, WS_CHUNK);
+            tc::bulk_commit();
+        }
     }
+    if (tid == 0) tc::bulk_wait_all();
     tc::tc_fence_before();
     __syncthreads();
     if (*abort_flag && tid == 0) atomicExch(&g_tc_error, 1);
@@ -770,9 +895,7 @@ ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
             tc::mbar_wait(&full[st], (ch / kStages) & 1, abort_flag);
             tc::tc_fence_after();
             float d[32];
-            tc::tmem_ld16(tc::tmem_addr(dc, 32 * warp, 0), d);
-            tc::tmem_ld16(tc::tmem_addr(dc, 32 * warp, 16), d + 16);
-            tc::tmem_ld_wait();
+            tc::tmem_ld32_sync(tc::tmem_addr(dc, 32 * warp, 0), d);
             const uint4* bc = reinterpret_cast<const uint4*>(stg + P2_BC + t * 64);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -790,9 +913,7 @@ ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
             // output (off the critical path): O = scale (D_o + O_loc), rows in the M = 64 layout
             tc::mbar_wait(mma_o, ch & 1, abort_flag);
             tc::tc_fence_after();
-            tc::tmem_ld16(tc::tmem_addr(dob + 32 * (ch & 1), 32 * warp, 0), d);
-            tc::tmem_ld16(tc::tmem_addr(dob + 32 * (ch & 1), 32 * warp, 16), d + 16);
-            tc::tmem_ld_wait();
+            tc::tmem_ld32_sync(tc::tmem_addr(dob + 32 * (ch & 1), 32 * warp, 0), d);
             if (lane < 16) {
                 const int r = 16 * warp + lane;
                 const int t0 = ch * kC;
@@ -897,9 +1018,14 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const f
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     if (stages == 0) stages = 3;
     if (stages & 1) {
-        ckda_tc_intra<<<(unsigned)(NT * B * H), 512, S_BYTES, stream>>>(
+        int dev = 0, nsm = 148;
+        if (cudaGetDevice(&dev) == cudaSuccess)
+            cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+        const int total = NT * B * H;
+        const int grid = total < nsm ? total : nsm;
+        ckda_tc_intra<<<(unsigned)grid, 512, S_BYTES, stream>>>(
             static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-            static_cast<const __nv_bfloat16*>(v), alpha, beta, ws, T_len, H, NT, l2norm, rp,
+            static_cast<const __nv_bfloat16*>(v), alpha, beta, ws, T_len, H, NT, total, l2norm, rp,
             pos_offset);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;

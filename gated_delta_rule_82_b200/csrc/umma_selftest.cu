@@ -75,8 +75,7 @@ umma_selftest_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16* _
     else if (lane < 16) row = warp * 16 + lane;
     for (int col = 0; col < N; col += 16) {
         float v[16];
-        tc::tmem_ld16(tc::tmem_addr(tbase, warp * 32, col), v);
-        tc::tmem_ld_wait();
+        tc::tmem_ld16_sync(tc::tmem_addr(tbase, warp * 32, col), v);
         if (row >= 0 && !abort_flag) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) D[(size_t)row * N + col + i] = v[i];

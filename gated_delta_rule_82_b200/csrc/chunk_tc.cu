@@ -15,28 +15,29 @@
 //
 // Gates.  The sign of gamma is a parity absorbed into q and k (q' = sigma q, k' = sigma k; the
 // compiled-PyTorch variant of the paper summary's "Implementation", i.e. the sign-magnitude split
-// of its Proposition 2), so every ratio gamma_r/gamma_j (j <= r) is a product of |alpha| over
-// (j, r].  Those products are formed block-locally on 16-row blocks and never by dividing
-// chunk-long products:
-//   fb_r  = prod |alpha| from the block start to r (inclusive)        <= 1
-//   bb_j  = prod |alpha| over (j, block end]                           <= 1
-//   P_I   = block total;  off-diagonal block (I > J):  ratio = fb_r * prod_{J<J'<I} P_J' * bb_j
-// so both GEMM operands of an off-diagonal block lie in [0, 1].  Inside a diagonal block the ratio
-// is fb_r / fb_j, bounded by 2^60 while the block total is >= 2^-60 (gates averaging |alpha| >=
-// 2^-3.75); a block below that (exact zeros, very strong decay) is recomputed exactly on CUDA
-// cores with running products from the inputs in global memory.
+// of its Proposition 2), so every ratio gamma_r/gamma_j (j <= r) is g_r / g_j with g = |gamma|, a
+// product of |alpha| over (j, r].  g is formed per channel as block-local running products (16
+// rows) times the totals of the earlier blocks, never as a division.  When the chunk's total
+// decay g_C stays >= 2^-118 in every channel, the ratio factors exactly in floating point as
+//     k'_r^T Diag(g_r / g_j) k'_j = (g_r k'_r) . (k'_j / g_j),
+// with every factor inside the bf16 / fp32 exponent range (|k'/g| <= 2^118, and the products
+// that are masked out, j > r, stay below 2^127), so A and M come from ONE tcgen05 product of
+// L = [g k'; g q'] (128 x 128) and R = k' / g (64 x 128).  L also holds K_gamma and Q_gamma, and
+// K_end = gamma_C R.  A chunk whose decay falls below 2^-118 somewhere (exact zeros, long
+// stretches of tiny gates) takes an exact CUDA-core path for A and M instead, evaluating
+// g_r / g_j = exp2(L_r - L_j) from an fp32 log2 prefix with non-positive exponents only.
 //
-// Kernel 1 (ckda_tc_intra) -- one CTA of 512 threads per (batch*head, chunk):
-//   A  alpha staged in shared memory; channel pass (thread per channel and 16-row block) forms the
-//      signed block prefix fb (sign = block-local parity), the suffix bb and the block totals;
-//      row pass (thread per row and 16 channels: a RoPE pair of 8-channel groups) loads q, k with
-//      16-byte loads, rotates, normalises, absorbs the signs and writes every operand tile with
-//      16-byte stores: L (k'fb | q'fb per block), the B tiles, K_gamma, K_end, Q_gamma, V.
-//   B  tcgen05: A and M block-rows (M = 64, K = 128) into TMEM; read back by 8 warps.
+// Kernel 1 (ckda_tc_intra) -- persistent, one CTA of 512 threads per SM, loops over
+// (batch*head, chunk):
+//   A  global loads of the next chunk-head issued together (and the one after prefetched into
+//      L2); channel pass (thread per channel and 16-row block) forms the signed prefix gamma_r;
+//      row pass (thread per row and two 8-channel groups, a RoPE pair) rotates and normalises q, k,
+//      absorbs the signs and writes L, R, K_end with 16-byte stores.
+//   B  tcgen05: [A | M] = L R^T  (M = 128, N = 64, K = 128), read back by all 16 warps.
 //   C  T = (I + A)^-1 by blocked forward substitution in fp32; T' = T diag(beta) in bf16.
 //   D  tcgen05: [W | U~] = T' [K_gamma | V]  (M = 64, N = 2 x 128, MN-major B).
 //   F  tcgen05: M [W | U~] (M = 64) and K_end^T [W | U~] (M = 128, MN-major A).
-//   G  write Q', O_loc, A_c, B_c as UMMA-ready images / dv tiles of the workspace.
+//   G  Q', O_loc, A_c, B_c staged in shared memory and written with three bulk (TMA) stores.
 // Kernel 2 (ckda_tc_state) -- one CTA per (batch*head, dv tile of 32 columns), serial over chunks:
 //   a three-stage pipeline of 1-D bulk (TMA) copies of each chunk's A_c, Q', B_c and O_loc; per
 //   chunk one tcgen05 product D_c = A_c S (M = 128, N = 32, K = 128) on the critical path, whose
@@ -61,44 +62,35 @@ constexpr uint32_t WS_TILE_O = 8192;
 constexpr uint32_t WS_CHUNK = WS_TILES + kNTile * WS_TILE;  // 98304
 
 // ---- kernel 1 shared memory (bytes from a 1024-aligned base) ---------------------------------
-constexpr uint32_t S_FB = 0;         // alpha, then signed fb (fp32 [64][128]); later A, T, M, T', X
-constexpr uint32_t S_BB = 32768;     // bb (fp32 [64][128])
-constexpr uint32_t S_L = 65536;      // L tile (K-major, 128 rows); later W and U~ tiles (MN-major)
-constexpr uint32_t S_B = 98304;      // B tiles (16 + 32 + 48 + 64 rows); later fallback scratch
-constexpr uint32_t S_KG = 139264;    // K_gamma (MN-major, 64 K-rows x 128)
-constexpr uint32_t S_V = 155648;     // V (MN-major, 64 x 128)
-constexpr uint32_t S_KE = 172032;    // K_end (MN-major, 64 x 128): the MN-major A of K_end^T
-constexpr uint32_t S_QG = 188416;    // Q_gamma (K-major, 64 rows x 128)
-constexpr uint32_t S_SM = 204800;    // small arrays (below)
-constexpr uint32_t S_BYTES = S_SM + 13312 + 1024;
-
-constexpr int kStrideA = 68;                     // fp32 row stride of A and T
-constexpr uint32_t S_A = 0;                      // A  fp32 [64][68]
-constexpr uint32_t S_T = 17408;                  // T  fp32 [64][68]
-constexpr uint32_t S_M = 35840;                  // M  bf16 K-major 64 x 64
-constexpr uint32_t S_TB = 44032;                 // T' bf16 K-major 64 x 64
-constexpr uint32_t S_X = 52224;                  // X  fp32 [16][48]
-constexpr uint32_t S_PT = 55296;                 // partial block products fp32 [6][16][16]
-constexpr uint32_t S_W = S_L;                    // W  MN-major 64 x 128
-constexpr uint32_t S_U = S_L + 16384;            // U~ MN-major 64 x 128
-constexpr uint32_t S_FQ = S_B;                   // fallback q' fp32 [16][128]
-constexpr uint32_t S_FK = S_B + 8192;            // fallback k' fp32 [16][128]
-constexpr uint32_t S_OUT = 0;                    // staging of the chunk's workspace image (96 KB)
+constexpr uint32_t S_G = 0;          // alpha, then the signed prefix gamma (fp32 [64][128])
+constexpr uint32_t S_L = 32768;      // L: rows 0..63 g k', rows 64..127 g q' (K-major, 128 rows)
+constexpr uint32_t S_R = 65536;      // R = k' / g (K-major, 64 rows)
+constexpr uint32_t S_V = 81920;      // V (MN-major, 64 K-rows x 128)
+constexpr uint32_t S_KE = 98304;     // K_end (MN-major, 64 x 128): the MN-major A of K_end^T
+constexpr uint32_t S_A = 114688;     // A fp32 [64][68]
+constexpr uint32_t S_T = 132096;     // T fp32 [64][68]
+constexpr uint32_t S_M = 149504;     // M bf16 K-major 64 x 64
+constexpr uint32_t S_TB = 157696;    // T' bf16 K-major 64 x 64
+constexpr uint32_t S_X = 165888;     // X fp32 [16][48]
+constexpr uint32_t S_PT = 168960;    // partial block products fp32 [6][16][16]
+constexpr uint32_t S_W = 175104;     // W MN-major 64 x 128   (exact path: log2 prefix fp32 [64][128]
+constexpr uint32_t S_U = 191488;     // U~ MN-major 64 x 128   spanning S_W and S_U)
+constexpr uint32_t S_SM = 207872;    // small arrays (below)
+constexpr uint32_t S_BYTES = S_SM + 5120 + 1024;
+constexpr int kStrideA = 68;         // fp32 row stride of A and T
+// staging of the chunk's workspace image, over buffers that are dead by then
+constexpr uint32_t S_OUT_AC = S_G;   // A_c image (32 KB)
+constexpr uint32_t S_OUT_QP = S_R;   // Q' image (16 KB)
+constexpr uint32_t S_OUT_TL = S_A;   // dv tiles (48 KB, over A, T, M and part of T')
 // small arrays
-constexpr uint32_t SM_P = S_SM;                  // P    fp32 [4][128]  block totals of |alpha|
-constexpr uint32_t SM_PAR = S_SM + 2048;         // PAR  fp32 [4][128]  block parity (+-1)
-constexpr uint32_t SM_PRE = S_SM + 4096;         // PRE  fp32 [4][128]  prod_{J<I} P_J
-constexpr uint32_t SM_KEF = S_SM + 6144;         // KEF  fp32 [4][128]  sigma_C prod_{J>I} P_J
-constexpr uint32_t SM_OFF2 = S_SM + 8192;        // OFF2 fp32 [4][128]  P_{I+1}
-constexpr uint32_t SM_OFF3 = S_SM + 10240;       // OFF3 fp32 [4][128]  P_{I+1} P_{I+2}
-constexpr uint32_t SM_GC = S_SM + 12288;         // gamma_C fp32 [128]
-constexpr uint32_t SM_B = S_SM + 12800;          // beta fp32 [64]
-constexpr uint32_t SM_FLAGS = S_SM + 13056;      // int unsafe[4], abort, tmem slot, mbarrier
+constexpr uint32_t SM_P = S_SM;                  // P   fp32 [4][128]  block totals of |alpha|
+constexpr uint32_t SM_PAR = S_SM + 2048;         // PAR fp32 [4][128]  block parity (+-1)
+constexpr uint32_t SM_GC = S_SM + 4096;          // gamma_C fp32 [128] (signed)
+constexpr uint32_t SM_B = S_SM + 4608;           // beta fp32 [64]
+constexpr uint32_t SM_FLAGS = S_SM + 4864;       // int exact_path, abort, tmem slot, mbarrier
 
-__host__ __device__ constexpr uint32_t btile_off(int I) { return I == 0 ? 0u : I == 1 ? 4096u : I == 2 ? 12288u : 24576u; }
-__host__ __device__ constexpr uint32_t amcol(int I) { return I == 0 ? 0u : I == 1 ? 16u : I == 2 ? 48u : 96u; }
+constexpr float kSafeDecay = 3.009265538105056e-36f;  // 2^-118
 
-constexpr float kDiagSafe = 8.673617379884035e-19f;  // 2^-60
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -125,62 +117,6 @@ __device__ __forceinline__ void ld_f8(const float* p, float* x) {
 }
 
 __device__ int g_tc_error;  // nonzero after a bounded wait ran out (diagnostic)
-
-// Recompute one row of q' and k' (rotation, L2 norm, chunk-local sign parity) straight from the
-// inputs; used only by the exact fallback of a collapsed diagonal block.  One warp per row.
-__device__ void fallback_row(const __nv_bfloat16* q, const __nv_bfloat16* k, const float* alpha,
-                             size_t row0, size_t rs, int r, int lane, const RopeParams& rp,
-                             long long pos, int l2norm, float* fq, float* fk) {
-    float qv[4], kv[4];
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-        const int c = lane + 32 * m;
-        qv[m] = __bfloat162float(q[(row0 + (size_t)r * rs) * kDK + c]);
-        kv[m] = __bfloat162float(k[(row0 + (size_t)r * rs) * kDK + c]);
-    }
-    if (rp.enabled) {
-        float qn[4], kn[4];
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const int c = lane + 32 * m;
-            int i;
-            bool first;
-            float qp, kp;
-            if (rp.convention == 0) {   // partner c ^ 64: same lane, m ^ 2
-                i = c & 63; first = c < 64; qp = qv[m ^ 2]; kp = kv[m ^ 2];
-            } else {                    // partner c ^ 1: neighbouring lane
-                i = c >> 1; first = (c & 1) == 0;
-                qp = __shfl_xor_sync(0xffffffffu, qv[m], 1);
-                kp = __shfl_xor_sync(0xffffffffu, kv[m], 1);
-            }
-            float sn, cs;
-            rope_sincos(pos, rp.inv_freq[i], &sn, &cs);
-            qn[m] = first ? qv[m] * cs - qp * sn : qv[m] * cs + qp * sn;
-            kn[m] = first ? kv[m] * cs - kp * sn : kv[m] * cs + kp * sn;
-        }
-#pragma unroll
-        for (int m = 0; m < 4; ++m) { qv[m] = qn[m]; kv[m] = kn[m]; }
-    }
-    if (l2norm) {
-        float a = 0.f, b = 0.f;
-#pragma unroll
-        for (int m = 0; m < 4; ++m) { a += qv[m] * qv[m]; b += kv[m] * kv[m]; }
-        a = rsqrtf(warp_sum(a) + kL2Eps);
-        b = rsqrtf(warp_sum(b) + kL2Eps);
-#pragma unroll
-        for (int m = 0; m < 4; ++m) { qv[m] *= a; kv[m] *= b; }
-    }
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-        const int c = lane + 32 * m;
-        float sg = 1.f;
-        for (int tau = 0; tau <= r; ++tau)
-            if (alpha[(row0 + (size_t)tau * rs) * kDK + c] < 0.f) sg = -sg;
-        fq[c] = sg * qv[m];
-        fk[c] = sg * kv[m];
-    }
-}
-
 
 // One block-row Ib (1..3) of T = (I + A)^-1 below the diagonal, given the diagonal blocks and
 // the block-rows above it:  T_{Ib,J} = -T_{Ib,Ib} sum_{K = J..Ib-1} A_{Ib,K} T_{K,J}.
@@ -265,25 +201,22 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float* FB = reinterpret_cast<float*>(sm + S_FB);
-    float* BB = reinterpret_cast<float*>(sm + S_BB);
+    float* G = reinterpret_cast<float*>(sm + S_G);
     float* gP = reinterpret_cast<float*>(sm + SM_P);
     float* gPar = reinterpret_cast<float*>(sm + SM_PAR);
-    float* gPre = reinterpret_cast<float*>(sm + SM_PRE);
-    float* gKef = reinterpret_cast<float*>(sm + SM_KEF);
-    float* gOff2 = reinterpret_cast<float*>(sm + SM_OFF2);
-    float* gOff3 = reinterpret_cast<float*>(sm + SM_OFF3);
     float* gGC = reinterpret_cast<float*>(sm + SM_GC);
     float* sb = reinterpret_cast<float*>(sm + SM_B);
-    int* unsafe = reinterpret_cast<int*>(sm + SM_FLAGS);
-    volatile int* abort_flag = unsafe + 4;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(unsafe + 8);
-    uint64_t* bar = reinterpret_cast<uint64_t*>(unsafe + 16);
+    int* exact_path = reinterpret_cast<int*>(sm + SM_FLAGS);
+    volatile int* abort_flag = exact_path + 4;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(exact_path + 8);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(exact_path + 16);
     float* sA = reinterpret_cast<float*>(sm + S_A);
     float* sT = reinterpret_cast<float*>(sm + S_T);
     float* sX = reinterpret_cast<float*>(sm + S_X);
+    float* sPt = reinterpret_cast<float*>(sm + S_PT);
+    float* sLg = reinterpret_cast<float*>(sm + S_W);   // exact path only
     uint8_t* sM = sm + S_M;
-    uint8_t* out = sm + S_OUT;
+    uint8_t* sL = sm + S_L;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const size_t rs = (size_t)H;   // stride between tokens, in rows of [B*T*H]
@@ -363,17 +296,17 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
                 }
             }
         }
-        // the previous chunk-head's bulk store must have finished reading shared memory
+        // the previous chunk-head's bulk stores must have finished reading shared memory
         if (tid == 0) tc::bulk_wait_read_all();
         __syncthreads();
 
         // ======== A1: alpha and V into shared memory ========
-        if (tid < 4) unsafe[tid] = 0;
+        if (tid == 0) *exact_path = 0;
         if (tid < 64) sb[tid] = bval;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const int e = tid + 512 * u, r = e >> 5, c4 = (e & 31) * 4;
-            *reinterpret_cast<float4*>(FB + r * 128 + c4) = araw[u];
+            *reinterpret_cast<float4*>(G + r * 128 + c4) = araw[u];
         }
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
@@ -382,57 +315,47 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
         }
         __syncthreads();
 
-        // ======== A2: channel pass -- thread (channel c, block I) ========
+        // ======== A2: channel pass -- thread (channel c, block I): signed prefix gamma ========
         const int cc = tid & 127, cI = tid >> 7;
         {
-            float bbv = 1.f;
-#pragma unroll
-            for (int rl = 15; rl >= 0; --rl) {
-                const int r = 16 * cI + rl;
-                BB[r * 128 + cc] = bbv;
-                bbv *= fabsf(FB[r * 128 + cc]);
-            }
             float p = 1.f;
             bool neg = false;
 #pragma unroll
             for (int rl = 0; rl < 16; ++rl) {
                 const int r = 16 * cI + rl;
-                const float a = FB[r * 128 + cc];
+                const float a = G[r * 128 + cc];
                 p *= fabsf(a);
                 neg ^= (a < 0.f);
-                FB[r * 128 + cc] = neg ? -p : p;   // a signed zero keeps the parity on underflow
+                G[r * 128 + cc] = neg ? -p : p;   // a signed zero keeps the parity on underflow
             }
             gP[cI * 128 + cc] = p;
             gPar[cI * 128 + cc] = neg ? -1.f : 1.f;
-            if (!(p >= kDiagSafe)) unsafe[cI] = 1;
         }
         __syncthreads();
-        // A2b: per-(block, channel) factors; the parity before the block goes into FB's sign
         {
-            float spre = 1.f, pre = 1.f, suf = 1.f, sC = 1.f, all = 1.f;
+            float pre = 1.f, all = 1.f, sC = 1.f;
 #pragma unroll
             for (int J = 0; J < 4; ++J) {
                 const float P = gP[J * 128 + cc], S = gPar[J * 128 + cc];
                 sC *= S;
                 all *= P;
-                if (J < cI) { spre *= S; pre *= P; }
-                if (J > cI) suf *= P;
+                if (J < cI) pre *= P * S;
             }
-            if (spre < 0.f) {
+            if (pre != 1.f) {
 #pragma unroll
-                for (int rl = 0; rl < 16; ++rl) FB[(16 * cI + rl) * 128 + cc] = -FB[(16 * cI + rl) * 128 + cc];
+                for (int rl = 0; rl < 16; ++rl) G[(16 * cI + rl) * 128 + cc] *= pre;
             }
-            gPre[cI * 128 + cc] = pre;
-            gKef[cI * 128 + cc] = sC * suf;
-            gOff2[cI * 128 + cc] = cI + 1 < 4 ? gP[(cI + 1) * 128 + cc] : 0.f;
-            gOff3[cI * 128 + cc] = cI + 2 < 4 ? gP[(cI + 1) * 128 + cc] * gP[(cI + 2) * 128 + cc] : 0.f;
-            if (cI == 0) gGC[cc] = sC * all;   // gamma_C (signed)
+            if (cI == 0) {
+                gGC[cc] = sC * all;
+                if (!(all >= kSafeDecay)) *exact_path = 1;
+            }
         }
         __syncthreads();
+        const bool exact = *exact_path != 0;
 
         // ======== A3: row pass -- thread (row r, 8-channel groups g and g + 8) ========
         {
-            const int r = rr, I = r >> 4, rl = r & 15;
+            const int r = rr;
             const int cA = 8 * g, cB = 64 + 8 * g;
             float qa[8], qb[8], ka[8], kb[8];
             unpack8(qkraw[0], qa);
@@ -479,180 +402,129 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
             }
             const float fq = l2norm ? rsqrtf(sq + kL2Eps) : 1.f;
             const float fk = l2norm ? rsqrtf(sk + kL2Eps) : 1.f;
-            const bool diag_ok = !unsafe[I];
-            // A3a: the operands of the A / M products (L and B tiles)
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 const int c0 = hh ? cB : cA;
                 const float* qx = hh ? qb : qa;
                 const float* kx = hh ? kb : ka;
-                float fb[8], kp[8], qp[8], acc[8], t8[8];
-                ld_f8(FB + r * 128 + c0, fb);   // |fb| with the full-chunk parity as its sign
+                float gm[8], kp[8], qp[8], t8[8];
+                ld_f8(G + r * 128 + c0, gm);   // gamma_r: |gamma| with the parity as its sign
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    const float sg = signbit(fb[i]) ? -1.f : 1.f;
-                    kp[i] = kx[i] * fk * sg;
-                    qp[i] = qx[i] * fq * sg;
-                    fb[i] = fabsf(fb[i]);
+                    const float sg = signbit(gm[i]) ? -1.f : 1.f;
+                    kp[i] = kx[i] * fk * sg;   // k'
+                    qp[i] = qx[i] * fq * sg;   // q'
+                    gm[i] = fabsf(gm[i]);      // g
                 }
-                // L tile: k' fb and q' fb
+                if (!exact) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) t8[i] = kp[i] * fb[i];
-                st16(sm + S_L, tc::sw128_kmajor(32 * I + rl, c0, 128), t8);
+                    for (int i = 0; i < 8; ++i) t8[i] = kp[i] * gm[i];
+                    st16(sL, tc::sw128_kmajor(r, c0, 128), t8);          // g k'  (= K_gamma)
 #pragma unroll
-                for (int i = 0; i < 8; ++i) t8[i] = qp[i] * fb[i];
-                st16(sm + S_L, tc::sw128_kmajor(32 * I + 16 + rl, c0, 128), t8);
-                // right operand of the diagonal block: k' / fb
+                    for (int i = 0; i < 8; ++i) t8[i] = qp[i] * gm[i];
+                    st16(sL, tc::sw128_kmajor(64 + r, c0, 128), t8);     // g q'  (= Q_gamma)
+                    float ke[8];
+                    ld_f8(gGC + c0, ke);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) t8[i] = diag_ok ? kp[i] * __frcp_rn(fb[i]) : 0.f;
-                st16(sm + S_B + btile_off(I), tc::sw128_kmajor(r, c0, 16 * (I + 1)), t8);
-                // off-diagonal right operands k' bb prod_{I<J<I2} P_J
-                ld_f8(BB + r * 128 + c0, acc);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] *= kp[i];
-                if (I < 3) st16(sm + S_B + btile_off(I + 1), tc::sw128_kmajor(r, c0, 16 * (I + 2)), acc);
-                if (I < 2) {
-                    ld_f8(gOff2 + I * 128 + c0, t8);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) t8[i] *= acc[i];
-                    st16(sm + S_B + btile_off(I + 2), tc::sw128_kmajor(r, c0, 16 * (I + 3)), t8);
-                }
-                if (I < 1) {
-                    ld_f8(gOff3 + I * 128 + c0, t8);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) t8[i] *= acc[i];
-                    st16(sm + S_B + btile_off(3), tc::sw128_kmajor(r, c0, 64), t8);
+                    for (int i = 0; i < 8; ++i) {
+                        t8[i] = kp[i] * __frcp_rn(gm[i]);                // k' / g
+                        ke[i] *= t8[i];                                  // gamma_C k' / g
+                    }
+                    st16(sm + S_R, tc::sw128_kmajor(r, c0, 64), t8);
+                    st16(sm + S_KE, tc::sw128_mnmajor(r, c0, 64), ke);   // K_end
+                } else {
+                    // exact path: unscaled k', q' for the CUDA-core A and M
+                    st16(sL, tc::sw128_kmajor(r, c0, 128), kp);
+                    st16(sL, tc::sw128_kmajor(64 + r, c0, 128), qp);
                 }
             }
-            tc::fence_proxy_async_smem();
-            tc::tc_fence_before();
-            __syncthreads();
-            tc::tc_fence_after();
+        }
+        tc::fence_proxy_async_smem();
+        tc::tc_fence_before();
+        __syncthreads();
+        tc::tc_fence_after();
 
-            // ======== B: A and M block-rows on the tensor cores (overlaps A3b) ========
+        if (!exact) {
+            // ======== B: [A | M] = L R^T on the tensor cores (M = 128, N = 64, K = 128) ========
             if (tid == 0) {
-                const uint32_t l0 = tc::smem_u32(sm + S_L), b0 = tc::smem_u32(sm + S_B);
+                const uint32_t l0 = tc::smem_u32(sL), r0a = tc::smem_u32(sm + S_R);
+                const uint32_t idesc = tc::idesc_bf16_f32(128, 64, 0, 0);
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
-#pragma unroll
-                    for (int J = 0; J < 4; ++J) {
-                        const int n = 16 * (J + 1);
-                        const uint64_t ad = tc::smem_desc_sw128(l0 + 4096 * J + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-                        const uint64_t bd = tc::smem_desc_sw128(b0 + btile_off(J) + (ks >> 2) * n * 128 + (ks & 3) * 32, 16, 1024);
-                        tc::mma_bf16(tmem + amcol(J), ad, bd, tc::idesc_bf16_f32(64, n, 0, 0), ks > 0 ? 1u : 0u);
-                    }
+                    const uint64_t ad = tc::smem_desc_sw128(l0 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+                    const uint64_t bd = tc::smem_desc_sw128(r0a + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
+                    tc::mma_bf16(tmem, ad, bd, idesc, ks > 0 ? 1u : 0u);
                 }
                 tc::mma_commit(bar);
             }
-
-            // A3b: K_end = k' bb KEF, K_gamma = |gamma_r| k', Q_gamma = |gamma_r| q'
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int c0 = hh ? cB : cA;
-                const float* qx = hh ? qb : qa;
-                const float* kx = hh ? kb : ka;
-                float fb[8], kp[8], qp[8], acc[8], t8[8];
-                ld_f8(FB + r * 128 + c0, fb);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float sg = signbit(fb[i]) ? -1.f : 1.f;
-                    kp[i] = kx[i] * fk * sg;
-                    qp[i] = qx[i] * fq * sg;
-                    fb[i] = fabsf(fb[i]);
-                }
-                ld_f8(BB + r * 128 + c0, acc);
-                ld_f8(gKef + I * 128 + c0, t8);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) t8[i] *= acc[i] * kp[i];
-                st16(sm + S_KE, tc::sw128_mnmajor(r, c0, 64), t8);
-                ld_f8(gPre + I * 128 + c0, acc);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) { acc[i] *= fb[i]; t8[i] = acc[i] * kp[i]; }
-                st16(sm + S_KG, tc::sw128_mnmajor(r, c0, 64), t8);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) t8[i] = acc[i] * qp[i];
-                st16(sm + S_QG, tc::sw128_kmajor(r, c0, 64), t8);
-            }
-        }
-        tc::mbar_wait(bar, phase & 1, abort_flag);
-        ++phase;
-        tc::tc_fence_after();
-        {
-            // M = 64 accumulator of block-row J: k rows in lanes 0..15, q rows in lanes 32..47.
-            // Warp w reads TMEM lanes 32 (w % 4) ..: w % 4 == 0 -> A part, 1 -> M part; J = w / 4.
-            const int quarter = warp & 3, J = warp >> 2;
-            if (quarter < 2) {
-                const int n = 16 * (J + 1);
-                const int r = 16 * J + (lane & 15);
-                for (int c0 = 0; c0 < n; c0 += 16) {
-                    float x[16];
-                    tc::tmem_ld16_sync(tc::tmem_addr(tmem, 32 * quarter, amcol(J) + c0), x);
-                    if (lane < 16) {
-                        if (quarter == 0) {
-                            const float br = sb[r];
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) x[i] = (c0 + i) < r ? br * x[i] : 0.f;
-#pragma unroll
-                            for (int i = 0; i < 16; i += 4)
-                                *reinterpret_cast<float4*>(sA + r * kStrideA + c0 + i) =
-                                    make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
-                        } else {
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) x[i] = (c0 + i) <= r ? x[i] : 0.f;
-                            st16(sM, tc::sw128_kmajor(r, c0, 64), x);
-                            st16(sM, tc::sw128_kmajor(r, c0 + 8, 64), x + 8);
-                        }
-                    }
-                }
-                if (lane < 16) {
-                    const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                    for (int j = n; j < 64; j += 8) {
-                        if (quarter == 0) {
-                            *reinterpret_cast<float4*>(sA + r * kStrideA + j) = make_float4(0.f, 0.f, 0.f, 0.f);
-                            *reinterpret_cast<float4*>(sA + r * kStrideA + j + 4) = make_float4(0.f, 0.f, 0.f, 0.f);
-                        } else {
-                            st16(sM, tc::sw128_kmajor(r, j, 64), z);
-                        }
-                    }
-                }
-            }
-        }
-        tc::tc_fence_before();
-        __syncthreads();
-
-        // exact recomputation of diagonal blocks whose gate total fell below 2^-60 (rare)
-        for (int J = 0; J < 4; ++J) {
-            if (!unsafe[J]) continue;
-            float* fq = reinterpret_cast<float*>(sm + S_FQ);
-            float* fk = reinterpret_cast<float*>(sm + S_FK);
+            tc::mbar_wait(bar, phase & 1, abort_flag);
+            ++phase;
+            tc::tc_fence_after();
             {
-                const int rl = warp, r = 16 * J + rl;
-                if (r < nvalid)
-                    fallback_row(q, k, alpha, row0, rs, r, lane, rp, pos_offset + t0 + r, l2norm,
-                                 fq + rl * 128, fk + rl * 128);
-                else
-                    for (int c = lane; c < 128; c += 32) fq[rl * 128 + c] = fk[rl * 128 + c] = 0.f;
+                // TMEM lanes 0..63: rows of A (k rows); lanes 64..127: rows of M (q rows).
+                // Warp w: lanes 32 (w % 4) .., columns 16 (w / 4) ..
+                const int quarter = warp & 3, c0 = 16 * (warp >> 2);
+                float x[16];
+                tc::tmem_ld16_sync(tc::tmem_addr(tmem, 32 * quarter, c0), x);
+                const int r = 32 * (quarter & 1) + lane;
+                if (quarter < 2) {
+                    const float br = sb[r];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) x[i] = (c0 + i) < r ? br * x[i] : 0.f;
+#pragma unroll
+                    for (int i = 0; i < 16; i += 4)
+                        *reinterpret_cast<float4*>(sA + r * kStrideA + c0 + i) =
+                            make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) x[i] = (c0 + i) <= r ? x[i] : 0.f;
+                    st16(sM, tc::sw128_kmajor(r, c0, 64), x);
+                    st16(sM, tc::sw128_kmajor(r, c0 + 8, 64), x + 8);
+                }
+            }
+        } else {
+            // ======== exact path for A and M (chunks whose decay leaves the bf16 range) ========
+            // log2 prefix L_r = sum_{tau <= r} log2 max(|alpha_tau|, FLT_MIN), straight from alpha
+            if (tid < 128) {
+                float L = 0.f;
+                for (int r = 0; r < 64; ++r) {
+                    const float a = r < nvalid ? alpha[(row0 + r * rs) * kDK + tid] : 1.f;
+                    L += log2f(fmaxf(fabsf(a), 1.17549435e-38f));
+                    sLg[r * 128 + tid] = L;
+                }
             }
             __syncthreads();
-            for (int pr = tid; pr < 136; pr += 512) {
-                int rl = 0;
-                while ((rl + 1) * (rl + 2) / 2 <= pr) ++rl;
-                const int jl = pr - rl * (rl + 1) / 2;
-                const int r = 16 * J + rl, j = 16 * J + jl;
+            for (int pr = tid; pr < 64 * 64; pr += 512) {
+                const int r = pr >> 6, j = pr & 63;
                 float accA = 0.f, accM = 0.f;
-                for (int c = 0; c < kDK; ++c) {
-                    float f = 1.f;
-                    for (int tau = j + 1; tau <= r; ++tau)
-                        f *= tau < nvalid ? fabsf(alpha[(row0 + tau * rs) * kDK + c]) : 1.f;
-                    const float kj = fk[jl * 128 + c] * f;
-                    accA += fk[rl * 128 + c] * kj;
-                    accM += fq[rl * 128 + c] * kj;
+                if (j <= r) {
+                    for (int c = 0; c < kDK; ++c) {
+                        const float e = exp2f(sLg[r * 128 + c] - sLg[j * 128 + c]);
+                        const float kj = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sL + tc::sw128_kmajor(j, c, 128))) * e;
+                        accA += __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sL + tc::sw128_kmajor(r, c, 128))) * kj;
+                        accM += __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sL + tc::sw128_kmajor(64 + r, c, 128))) * kj;
+                    }
                 }
                 sA[r * kStrideA + j] = j < r ? sb[r] * accA : 0.f;
                 *reinterpret_cast<__nv_bfloat16*>(sM + tc::sw128_kmajor(r, j, 64)) = __float2bfloat16_rn(accM);
             }
             __syncthreads();
+            // rescale L to (g k', g q') with g = exp2(L_r) and form K_end = sigma_C exp2(L_C - L_j) k'
+            for (int e = tid; e < 64 * 128; e += 512) {
+                const int r = e >> 7, c = e & 127;
+                const float gr = exp2f(sLg[r * 128 + c]);
+                __nv_bfloat16* kr = reinterpret_cast<__nv_bfloat16*>(sL + tc::sw128_kmajor(r, c, 128));
+                __nv_bfloat16* qr = reinterpret_cast<__nv_bfloat16*>(sL + tc::sw128_kmajor(64 + r, c, 128));
+                const float kv = __bfloat162float(*kr), qv = __bfloat162float(*qr);
+                const float sC = signbit(gGC[c]) ? -1.f : 1.f;
+                *reinterpret_cast<__nv_bfloat16*>(sm + S_KE + tc::sw128_mnmajor(r, c, 64)) =
+                    __float2bfloat16_rn(sC * exp2f(sLg[63 * 128 + c] - sLg[r * 128 + c]) * kv);
+                *kr = __float2bfloat16_rn(gr * kv);
+                *qr = __float2bfloat16_rn(gr * qv);
+            }
         }
+        tc::tc_fence_before();
+        __syncthreads();
 
         // ======== C: T = (I + A)^-1 (fp32), T' = T diag(beta) (bf16) ========
         for (int e = tid; e < 64 * 64; e += 512) {
@@ -676,12 +548,9 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
             for (int i = 0; i < 16; ++i) sT[(base + i) * kStrideA + base + l] = tcol[i];
         }
         __syncthreads();
-        {
-            float* sPt = reinterpret_cast<float*>(sm + S_PT);
-            t_offdiag_level<1>(sA, sT, sX, sPt, tid);
-            t_offdiag_level<2>(sA, sT, sX, sPt, tid);
-            t_offdiag_level<3>(sA, sT, sX, sPt, tid);
-        }
+        t_offdiag_level<1>(sA, sT, sX, sPt, tid);
+        t_offdiag_level<2>(sA, sT, sX, sPt, tid);
+        t_offdiag_level<3>(sA, sT, sX, sPt, tid);
         for (int e = tid; e < 64 * 8; e += 512) {
             const int r = e >> 3, j0 = (e & 7) * 8;
             float y[8];
@@ -695,14 +564,15 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
         tc::tc_fence_after();
 
         // ======== D: W = T' K_gamma, U~ = T' V  (M = 64, N = 128 each, K = 64) ========
+        // K_gamma is rows 0..63 of L, read as an MN-major operand: 64-column blocks 16 KB apart.
         if (tid == 0) {
             const uint32_t a0 = tc::smem_u32(sm + S_TB);
-            const uint32_t kg = tc::smem_u32(sm + S_KG), vv = tc::smem_u32(sm + S_V);
+            const uint32_t kg = tc::smem_u32(sL), vv = tc::smem_u32(sm + S_V);
             const uint32_t idesc = tc::idesc_bf16_f32(64, 128, 0, 1);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
                 const uint64_t ad = tc::smem_desc_sw128(a0 + ks * 32, 16, 1024);
-                tc::mma_bf16(tmem, ad, tc::smem_desc_sw128(kg + ks * 2048, 8192, 1024), idesc, ks > 0);
+                tc::mma_bf16(tmem, ad, tc::smem_desc_sw128(kg + ks * 2048, 16384, 1024), idesc, ks > 0);
                 tc::mma_bf16(tmem + 128, ad, tc::smem_desc_sw128(vv + ks * 2048, 8192, 1024), idesc, ks > 0);
             }
             tc::mma_commit(bar);
@@ -751,7 +621,7 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
         tc::mbar_wait(bar, phase & 1, abort_flag);
         ++phase;
         tc::tc_fence_after();
-        // ======== G: results into the shared staging image, then one bulk store ========
+        // ======== G: results into shared staging images, then three bulk stores ========
         {
             const int quarter = warp & 3, slice = warp >> 2;
             // (1) M = 64 products: rows 16 quarter + lane; slices 0, 1 -> Q', 2, 3 -> O_loc
@@ -766,12 +636,12 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
                         const int n = n0 + c0;
                         if (slice < 2) {
                             float qg[8];
-                            unpack8(*reinterpret_cast<const uint4*>(sm + S_QG + tc::sw128_kmajor(r, n, 64)), qg);
+                            unpack8(*reinterpret_cast<const uint4*>(sL + tc::sw128_kmajor(64 + r, n, 128)), qg);
 #pragma unroll
                             for (int i = 0; i < 8; ++i) qg[i] -= x[c0 + i];
-                            st16(out, WS_QP + tc::sw128_kmajor(r, n, 64), qg);
+                            st16(sm + S_OUT_QP, tc::sw128_kmajor(r, n, 64), qg);
                         } else {
-                            st16(out, WS_TILES + (n >> 5) * WS_TILE + WS_TILE_O + (r * 32 + (n & 31)) * 2, x + c0);
+                            st16(sm + S_OUT_TL, (n >> 5) * WS_TILE + WS_TILE_O + (r * 32 + (n & 31)) * 2, x + c0);
                         }
                     }
                 }
@@ -790,9 +660,9 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
                         float y[8];
 #pragma unroll
                         for (int i = 0; i < 8; ++i) y[i] = (n + i == cr ? gc : 0.f) - x[c0 + i];
-                        st16(out, WS_AC + tc::sw128_kmajor(cr, n, 128), y);
+                        st16(sm + S_OUT_AC, tc::sw128_kmajor(cr, n, 128), y);
                     } else {
-                        st16(out, WS_TILES + (n >> 5) * WS_TILE + (cr * 32 + (n & 31)) * 2, x + c0);
+                        st16(sm + S_OUT_TL, (n >> 5) * WS_TILE + (cr * 32 + (n & 31)) * 2, x + c0);
                     }
                 }
             }
@@ -802,7 +672,9 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
         __syncthreads();
         tc::tc_fence_after();
         if (tid == 0) {
-            tc::bulk_s2g(wsc, out, WS_CHUNK);
+            tc::bulk_s2g(wsc + WS_AC, sm + S_OUT_AC, 32768);
+            tc::bulk_s2g(wsc + WS_QP, sm + S_OUT_QP, 16384);
+            tc::bulk_s2g(wsc + WS_TILES, sm + S_OUT_TL, kNTile * WS_TILE);
             tc::bulk_commit();
         }
     }

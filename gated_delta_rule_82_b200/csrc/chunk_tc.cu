@@ -44,6 +44,9 @@
 //   epilogue adds B_c to form the fp32 master state (one row per thread, in registers) and writes
 //   its bf16 copy for the next product, and one off-path product D_o = Q' S (M = 64) that becomes
 //   the chunk's output.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "internal.cuh"
 #include "tc_sm100.cuh"
 
@@ -62,35 +65,38 @@ constexpr uint32_t WS_TILE_O = 8192;
 constexpr uint32_t WS_CHUNK = WS_TILES + kNTile * WS_TILE;  // 98304
 
 // ---- kernel 1 shared memory (bytes from a 1024-aligned base) ---------------------------------
-constexpr uint32_t S_G = 0;          // alpha, then the signed prefix gamma (fp32 [64][128])
-constexpr uint32_t S_L = 32768;      // L: rows 0..63 g k', rows 64..127 g q' (K-major, 128 rows)
-constexpr uint32_t S_R = 65536;      // R = k' / g (K-major, 64 rows)
-constexpr uint32_t S_V = 81920;      // V (MN-major, 64 K-rows x 128)
-constexpr uint32_t S_KE = 98304;     // K_end (MN-major, 64 x 128): the MN-major A of K_end^T
-constexpr uint32_t S_A = 114688;     // A fp32 [64][68]
-constexpr uint32_t S_T = 132096;     // T fp32 [64][68]
-constexpr uint32_t S_M = 149504;     // M bf16 K-major 64 x 64
-constexpr uint32_t S_TB = 157696;    // T' bf16 K-major 64 x 64
-constexpr uint32_t S_X = 165888;     // X fp32 [16][48]
-constexpr uint32_t S_PT = 168960;    // partial block products fp32 [6][16][16]
-constexpr uint32_t S_W = 175104;     // W MN-major 64 x 128   (exact path: log2 prefix fp32 [64][128]
-constexpr uint32_t S_U = 191488;     // U~ MN-major 64 x 128   spanning S_W and S_U)
-constexpr uint32_t S_SM = 207872;    // small arrays (below)
-constexpr uint32_t S_BYTES = S_SM + 5120 + 1024;
+constexpr uint32_t S_G = 0;          // alpha (TMA), then the signed prefix gamma (fp32 [64][128])
+constexpr uint32_t S_QR = 32768;     // raw q (TMA), bf16 [64][128] row-major
+constexpr uint32_t S_KR = 49152;     // raw k (TMA), bf16 [64][128] row-major
+constexpr uint32_t S_L = 65536;      // L: rows 0..63 g k', rows 64..127 g q' (K-major, 128 rows)
+constexpr uint32_t S_R = 98304;      // R = k' / g (K-major, 64 rows); later T', X, Y; then Q' image
+constexpr uint32_t S_V = 114688;     // V (TMA, 128-byte swizzle = MN-major, 64 K-rows x 128)
+constexpr uint32_t S_KE = 131072;    // K_end (MN-major, 64 x 128): the MN-major A of K_end^T
+constexpr uint32_t S_M = 147456;     // M bf16 K-major 64 x 64
+constexpr uint32_t S_A = 155648;     // A fp32 [64][68]
+constexpr uint32_t S_T = 173056;     // T fp32 [64][68]
+constexpr uint32_t S_W = 190464;     // W MN-major 64 x 128   (exact path: log2 prefix fp32 [64][128]
+constexpr uint32_t S_U = 206848;     // U~ MN-major 64 x 128   spanning S_W and S_U)
+constexpr uint32_t S_SM = 223232;    // small arrays (below)
+constexpr uint32_t S_BYTES = S_SM + 3072 + 1024;
 constexpr int kStrideA = 68;         // fp32 row stride of A and T
+// T solve scratch inside R (dead after the [A | M] product)
+constexpr uint32_t S_TB = S_R;               // T' bf16 K-major 64 x 64
+constexpr uint32_t S_X = S_R + 8192;         // X0, X1 fp32 [16][16] each
+constexpr uint32_t S_Y = S_R + 10240;        // Y fp32 [32][36]
 // staging of the chunk's workspace image, over buffers that are dead by then
-constexpr uint32_t S_OUT_AC = S_G;   // A_c image (32 KB)
+constexpr uint32_t S_OUT_AC = S_W;   // A_c image (32 KB, over W and U)
 constexpr uint32_t S_OUT_QP = S_R;   // Q' image (16 KB)
-constexpr uint32_t S_OUT_TL = S_A;   // dv tiles (48 KB, over A, T, M and part of T')
+constexpr uint32_t S_OUT_TL = S_KE;  // dv tiles (48 KB, over K_end, M, A and part of T)
 // small arrays
-constexpr uint32_t SM_P = S_SM;                  // P   fp32 [4][128]  block totals of |alpha|
-constexpr uint32_t SM_PAR = S_SM + 2048;         // PAR fp32 [4][128]  block parity (+-1)
-constexpr uint32_t SM_GC = S_SM + 4096;          // gamma_C fp32 [128] (signed)
-constexpr uint32_t SM_B = S_SM + 4608;           // beta fp32 [64]
-constexpr uint32_t SM_FLAGS = S_SM + 4864;       // int exact_path, abort, tmem slot, mbarrier
+constexpr uint32_t SM_P = S_SM;                  // signed block totals of alpha, fp32 [4][128]
+constexpr uint32_t SM_GC = S_SM + 2048;          // gamma_C fp32 [128] (signed)
+constexpr uint32_t SM_B = S_SM + 2560;           // beta fp32 [64]
+constexpr uint32_t SM_FLAGS = S_SM + 2816;       // exact flag, abort flag, TMEM slot, 3 mbarriers
+constexpr uint32_t kInBytes = 32768 + 2 * 16384; // alpha, q, k of one chunk-head
+constexpr uint32_t kVBytes = 16384;
 
 constexpr float kSafeDecay = 3.009265538105056e-36f;  // 2^-118
-
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -115,87 +121,166 @@ __device__ __forceinline__ void ld_f8(const float* p, float* x) {
     float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
     x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
 }
+__device__ __forceinline__ void st_bf16(uint8_t* base, uint32_t off, float x) {
+    *reinterpret_cast<__nv_bfloat16*>(base + off) = __float2bfloat16_rn(x);
+}
 
 __device__ int g_tc_error;  // nonzero after a bounded wait ran out (diagnostic)
 
-// One block-row Ib (1..3) of T = (I + A)^-1 below the diagonal, given the diagonal blocks and
-// the block-rows above it:  T_{Ib,J} = -T_{Ib,Ib} sum_{K = J..Ib-1} A_{Ib,K} T_{K,J}.
-// Pass 1: warp w computes one 16 x 16 x 16 product A_{Ib,K} T_{K,J} for the w-th pair J <= K < Ib;
-// pass 2 sums the pairs into X; pass 3: warp J computes -T_{Ib,Ib} X_J.  Every loop is fully
-// unrolled, a thread owns a 2 x 4 output tile.
-template <int Ib>
-__device__ __forceinline__ void t_offdiag_level(const float* sA, float* sT, float* sX, float* sPt,
-                                                int tid) {
-    constexpr int NP = Ib * (Ib + 1) / 2;
-    const int warp = tid >> 5, lane = tid & 31;
-    const int rp = lane >> 2, jq = lane & 3;
-    if (warp < NP) {
-        int K = 0, J = warp;
-        while (J > K) { J -= K + 1; ++K; }
-        const float* a0 = sA + (16 * Ib + 2 * rp) * kStrideA + 16 * K;
-        const float* a1 = a0 + kStrideA;
-        const float* tb = sT + (16 * K) * kStrideA + 16 * J + 4 * jq;
-        float4 x0 = make_float4(0.f, 0.f, 0.f, 0.f), x1 = x0, y0 = x0, y1 = x0;
+// Tensor maps of one forward call: q, k, v (bf16) and alpha (fp32) as 4-D arrays
+// {channel, head, token, batch}; boxes of 64 tokens of one (batch, head).
+struct TcMaps {
+    CUtensorMap q, k, v, alpha;
+};
+
+// Issue the TMA loads of chunk-head ci: alpha -> G, q -> QR, k -> KR on bar_in; V (two 64-column
+// halves, 128-byte swizzle) on bar_v when with_v.  Rows past the sequence end read as zeros.
+__device__ __forceinline__ void issue_inputs(const TcMaps& m, uint8_t* sm, uint64_t* bar_in,
+                                             int ci, int NT, int H) {
+    const int ch = ci % NT, bh = ci / NT;
+    const int b = bh / H, h = bh % H, t0 = ch * kC;
+    tc::mbar_arrive_expect_tx(bar_in, kInBytes);
+    tc::tma_load_4d(sm + S_G, &m.alpha, 0, h, t0, b, bar_in);
+    tc::tma_load_4d(sm + S_QR, &m.q, 0, h, t0, b, bar_in);
+    tc::tma_load_4d(sm + S_KR, &m.k, 0, h, t0, b, bar_in);
+}
+__device__ __forceinline__ void issue_v(const TcMaps& m, uint8_t* sm, uint64_t* bar_v, int ci,
+                                        int NT, int H) {
+    const int ch = ci % NT, bh = ci / NT;
+    const int b = bh / H, h = bh % H, t0 = ch * kC;
+    tc::mbar_arrive_expect_tx(bar_v, kVBytes);
+    tc::tma_load_4d(sm + S_V, &m.v, 0, h, t0, b, bar_v);
+    tc::tma_load_4d(sm + S_V + 8192, &m.v, 64, h, t0, b, bar_v);
+}
+
+// out[0..3] (+)= sum_{k < K} a[k] * b[k][0..3]: a row of K floats (16-byte aligned), b rows
+// `bstride` floats apart; both in shared memory.  Four independent accumulators per k quad.
+template <int K>
+__device__ __forceinline__ float4 row_x_cols4(const float* a, const float* b, int bstride) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int m = 0; m < 16; m += 2) {
-            const float4 ta = *reinterpret_cast<const float4*>(tb + m * kStrideA);
-            const float4 tc4 = *reinterpret_cast<const float4*>(tb + (m + 1) * kStrideA);
-            const float2 aa = *reinterpret_cast<const float2*>(a0 + m);
-            const float2 ab = *reinterpret_cast<const float2*>(a1 + m);
-            x0.x += aa.x * ta.x; x0.y += aa.x * ta.y; x0.z += aa.x * ta.z; x0.w += aa.x * ta.w;
-            y0.x += aa.y * tc4.x; y0.y += aa.y * tc4.y; y0.z += aa.y * tc4.z; y0.w += aa.y * tc4.w;
-            x1.x += ab.x * ta.x; x1.y += ab.x * ta.y; x1.z += ab.x * ta.z; x1.w += ab.x * ta.w;
-            y1.x += ab.y * tc4.x; y1.y += ab.y * tc4.y; y1.z += ab.y * tc4.z; y1.w += ab.y * tc4.w;
-        }
-        float* pt = sPt + warp * 256;
-        *reinterpret_cast<float4*>(pt + (2 * rp) * 16 + 4 * jq) =
-            make_float4(x0.x + y0.x, x0.y + y0.y, x0.z + y0.z, x0.w + y0.w);
-        *reinterpret_cast<float4*>(pt + (2 * rp + 1) * 16 + 4 * jq) =
-            make_float4(x1.x + y1.x, x1.y + y1.y, x1.z + y1.z, x1.w + y1.w);
+    for (int k = 0; k < K; k += 4) {
+        const float4 av = *reinterpret_cast<const float4*>(a + k);
+        const float4 b0 = *reinterpret_cast<const float4*>(b + (k + 0) * bstride);
+        const float4 b1 = *reinterpret_cast<const float4*>(b + (k + 1) * bstride);
+        const float4 b2 = *reinterpret_cast<const float4*>(b + (k + 2) * bstride);
+        const float4 b3 = *reinterpret_cast<const float4*>(b + (k + 3) * bstride);
+        acc.x += av.x * b0.x + av.y * b1.x + av.z * b2.x + av.w * b3.x;
+        acc.y += av.x * b0.y + av.y * b1.y + av.z * b2.y + av.w * b3.y;
+        acc.z += av.x * b0.z + av.y * b1.z + av.z * b2.z + av.w * b3.z;
+        acc.w += av.x * b0.w + av.y * b1.w + av.z * b2.w + av.w * b3.w;
     }
-    __syncthreads();
-    if (tid < 16 * 4 * Ib) {
-        const int rl = tid / (4 * Ib), quad = tid % (4 * Ib);
-        const int J = quad >> 2, c = 4 * (quad & 3);
-        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    return acc;
+}
+__device__ __forceinline__ void st_tb4(uint8_t* sTB, int r, int c, float4 t, const float* sb) {
+    const float4 bj = *reinterpret_cast<const float4*>(sb + c);
+    *reinterpret_cast<uint2*>(sTB + tc::sw128_kmajor(r, c, 64)) =
+        make_uint2(pack_bf16(t.x * bj.x, t.y * bj.y), pack_bf16(t.z * bj.z, t.w * bj.w));
+}
+
+// T = (I + A)^-1 for the strictly lower-triangular 64 x 64 A (fp32), by block doubling over
+// 16 x 16 blocks T_IJ (I, J = 0..3):
+//   phase 0  diagonal blocks T_JJ by forward substitution;
+//   phase 1  X0 = A_10 T_00,  X1 = A_32 T_22,  Y = [A_{[2:4],0} T_00 | A_{[2:4],1} T_11];
+//   phase 2  T_10 = -T_11 X0,  T_32 = -T_33 X1,  Y_left -= Y_right X0
+//            (then Y = A_{[2:4],[0:2]} T_{[0:2],[0:2]}, since T_10 = -T_11 X0);
+//   phase 3  T_{[2:4],[0:2]} = -T_{[2:4],[2:4]} Y.
+// Each finished block is also written as T' = T diag(beta) in bf16 (K-major, 64 x 64), the A
+// operand of the W and U~ products.  A thread owns a 1 x 4 output tile; operands are read as
+// float4 (rows of A and T at a stride of 68 floats, of Y at 36: no bank conflicts).
+constexpr int kStrideY = 36;
+__device__ __forceinline__ void t_solve(const float* sA, float* sT, const float* sb, uint8_t* sTB,
+                                        float* sX, float* sY, int tid) {
+    float* sX0 = sX;         // [16][16]
+    float* sX1 = sX + 256;   // [16][16]
+    // ---- phase 0: diagonal blocks (threads 0..63: block J = tid / 16, column l = tid % 16);
+    // the others zero block (2,3) of T and the blocks of T' above the diagonal
+    if (tid < 64) {
+        const int J = tid >> 4, l = tid & 15, base = 16 * J;
+        float tcol[16];
 #pragma unroll
-        for (int K = 0; K < Ib; ++K) {
-            if (K >= J) {
-                const float4 p = *reinterpret_cast<const float4*>(sPt + (K * (K + 1) / 2 + J) * 256 + rl * 16 + c);
-                x.x += p.x; x.y += p.y; x.z += p.z; x.w += p.w;
+        for (int i = 0; i < 16; ++i) {
+            float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+            for (int m = 0; m < 16; m += 2) {
+                if (m < i) a0 += sA[(base + i) * kStrideA + base + m] * tcol[m];
+                if (m + 1 < i) a1 += sA[(base + i) * kStrideA + base + m + 1] * tcol[m + 1];
             }
+            tcol[i] = i < l ? 0.f : (i == l ? 1.f : -(a0 + a1));
         }
-        *reinterpret_cast<float4*>(sX + rl * 48 + 16 * J + c) = x;
-    }
-    __syncthreads();
-    if (warp < Ib) {
-        const int J = warp;
-        const float* t0r = sT + (16 * Ib + 2 * rp) * kStrideA + 16 * Ib;
-        const float* t1r = t0r + kStrideA;
-        const float* xb = sX + 16 * J + 4 * jq;
-        float4 x0 = make_float4(0.f, 0.f, 0.f, 0.f), x1 = x0, y0 = x0, y1 = x0;
+        const float bl = sb[base + l];
 #pragma unroll
-        for (int m = 0; m < 16; m += 2) {
-            const float4 xa = *reinterpret_cast<const float4*>(xb + m * 48);
-            const float4 xc = *reinterpret_cast<const float4*>(xb + (m + 1) * 48);
-            const float2 aa = *reinterpret_cast<const float2*>(t0r + m);
-            const float2 ab = *reinterpret_cast<const float2*>(t1r + m);
-            x0.x += aa.x * xa.x; x0.y += aa.x * xa.y; x0.z += aa.x * xa.z; x0.w += aa.x * xa.w;
-            y0.x += aa.y * xc.x; y0.y += aa.y * xc.y; y0.z += aa.y * xc.z; y0.w += aa.y * xc.w;
-            x1.x += ab.x * xa.x; x1.y += ab.x * xa.y; x1.z += ab.x * xa.z; x1.w += ab.x * xa.w;
-            y1.x += ab.y * xc.x; y1.y += ab.y * xc.y; y1.z += ab.y * xc.z; y1.w += ab.y * xc.w;
+        for (int i = 0; i < 16; ++i) {
+            sT[(base + i) * kStrideA + base + l] = tcol[i];
+            st_bf16(sTB, tc::sw128_kmajor(base + i, base + l, 64), tcol[i] * bl);
         }
-        *reinterpret_cast<float4*>(sT + (16 * Ib + 2 * rp) * kStrideA + 16 * J + 4 * jq) =
-            make_float4(-(x0.x + y0.x), -(x0.y + y0.y), -(x0.z + y0.z), -(x0.w + y0.w));
-        *reinterpret_cast<float4*>(sT + (16 * Ib + 2 * rp + 1) * kStrideA + 16 * J + 4 * jq) =
-            make_float4(-(x1.x + y1.x), -(x1.y + y1.y), -(x1.z + y1.z), -(x1.w + y1.w));
+    } else {
+        const int e = tid - 64;   // 0..447
+        if (e < 64) {             // T block (2,3): rows 32..47, columns 48..63
+            const int rr = e >> 2, c4 = 4 * (e & 3);
+            *reinterpret_cast<float4*>(sT + (32 + rr) * kStrideA + 48 + c4) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        // T' above the diagonal blocks: 192 chunks of 8 columns
+        // (rows 0..15: 6 chunks each, rows 16..31: 4, rows 32..47: 2)
+        for (int u = e; u < 192; u += 448) {
+            int r, c8;
+            if (u < 96) { r = u / 6; c8 = 16 + 8 * (u % 6); }
+            else if (u < 160) { r = 16 + (u - 96) / 4; c8 = 32 + 8 * ((u - 96) % 4); }
+            else { r = 32 + (u - 160) / 2; c8 = 48 + 8 * ((u - 160) % 2); }
+            *reinterpret_cast<uint4*>(sTB + tc::sw128_kmajor(r, c8, 64)) = make_uint4(0, 0, 0, 0);
+        }
     }
     __syncthreads();
+    // ---- phase 1: 96 output rows x 4 column quads (threads 0..383)
+    if (tid < 384) {
+        const int ri = tid >> 2, c0 = 4 * (tid & 3);
+        if (ri < 48) {            // [X0; Y_left] = A_{[1:4],0} T_00
+            const int row = 16 + ri;
+            const float4 x = row_x_cols4<16>(sA + row * kStrideA, sT + c0, kStrideA);
+            float* dst = ri < 16 ? sX0 + ri * 16 + c0 : sY + (ri - 16) * kStrideY + c0;
+            *reinterpret_cast<float4*>(dst) = x;
+        } else if (ri < 80) {     // Y_right = A_{[2:4],1} T_11
+            const int i = ri - 48;
+            const float4 x = row_x_cols4<16>(sA + (32 + i) * kStrideA + 16, sT + 16 * kStrideA + 16 + c0, kStrideA);
+            *reinterpret_cast<float4*>(sY + i * kStrideY + 16 + c0) = x;
+        } else {                  // X1 = A_32 T_22
+            const int i = ri - 80;
+            const float4 x = row_x_cols4<16>(sA + (48 + i) * kStrideA + 32, sT + 32 * kStrideA + 32 + c0, kStrideA);
+            *reinterpret_cast<float4*>(sX1 + i * 16 + c0) = x;
+        }
+    }
+    __syncthreads();
+    // ---- phase 2: 64 output rows x 4 column quads (threads 0..255)
+    if (tid < 256) {
+        const int ri = tid >> 2, c0 = 4 * (tid & 3);
+        if (ri < 16) {            // T_10 = -T_11 X0
+            const float4 x = row_x_cols4<16>(sT + (16 + ri) * kStrideA + 16, sX0 + c0, 16);
+            st_tb4(sTB, 16 + ri, c0, make_float4(-x.x, -x.y, -x.z, -x.w), sb);   // T' only
+        } else if (ri < 32) {     // T_32 = -T_33 X1
+            const int i = ri - 16;
+            const float4 x = row_x_cols4<16>(sT + (48 + i) * kStrideA + 48, sX1 + c0, 16);
+            const float4 t = make_float4(-x.x, -x.y, -x.z, -x.w);
+            *reinterpret_cast<float4*>(sT + (48 + i) * kStrideA + 32 + c0) = t;
+            st_tb4(sTB, 48 + i, 32 + c0, t, sb);
+        } else {                  // Y_left -= Y_right X0
+            const int i = ri - 32;
+            const float4 x = row_x_cols4<16>(sY + i * kStrideY + 16, sX0 + c0, 16);
+            float4* y = reinterpret_cast<float4*>(sY + i * kStrideY + c0);
+            const float4 z = *y;
+            *y = make_float4(z.x - x.x, z.y - x.y, z.z - x.z, z.w - x.w);
+        }
+    }
+    __syncthreads();
+    // ---- phase 3: T_{[2:4],[0:2]} = -T_{[2:4],[2:4]} Y, 32 rows x 8 column quads (threads 0..255)
+    if (tid < 256) {
+        const int i = tid >> 3, c0 = 4 * (tid & 7);
+        const float4 x = row_x_cols4<32>(sT + (32 + i) * kStrideA + 32, sY + c0, kStrideY);
+        st_tb4(sTB, 32 + i, c0, make_float4(-x.x, -x.y, -x.z, -x.w), sb);
+    }
 }
 
 __global__ void __launch_bounds__(512, 1)
-ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-              const __nv_bfloat16* __restrict__ v, const float* __restrict__ alpha,
+ckda_tc_intra(const __grid_constant__ TcMaps maps, const float* __restrict__ alpha,
               const float* __restrict__ beta, uint8_t* __restrict__ ws, int T_len, int H, int NT,
               int total, int l2norm, RopeParams rp, long long pos_offset) {
     extern __shared__ uint8_t smem_raw[];
@@ -203,17 +288,16 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float* G = reinterpret_cast<float*>(sm + S_G);
     float* gP = reinterpret_cast<float*>(sm + SM_P);
-    float* gPar = reinterpret_cast<float*>(sm + SM_PAR);
     float* gGC = reinterpret_cast<float*>(sm + SM_GC);
     float* sb = reinterpret_cast<float*>(sm + SM_B);
     int* exact_path = reinterpret_cast<int*>(sm + SM_FLAGS);
     volatile int* abort_flag = exact_path + 4;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(exact_path + 8);
-    uint64_t* bar = reinterpret_cast<uint64_t*>(exact_path + 16);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(exact_path + 16);   // tensor-core completions
+    uint64_t* bar_in = bar + 1;                                     // alpha, q, k landed
+    uint64_t* bar_v = bar + 2;                                      // V landed
     float* sA = reinterpret_cast<float*>(sm + S_A);
     float* sT = reinterpret_cast<float*>(sm + S_T);
-    float* sX = reinterpret_cast<float*>(sm + S_X);
-    float* sPt = reinterpret_cast<float*>(sm + S_PT);
     float* sLg = reinterpret_cast<float*>(sm + S_W);   // exact path only
     uint8_t* sM = sm + S_M;
     uint8_t* sL = sm + S_L;
@@ -227,6 +311,8 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
     }
     if (tid == 32) {
         tc::mbar_init(bar, 1);
+        tc::mbar_init(bar_in, 1);
+        tc::mbar_init(bar_v, 1);
         tc::fence_mbar_init();
         *abort_flag = 0;
     }
@@ -235,133 +321,70 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     uint32_t phase = 0;   // completions of `bar` so far
+    if (tid == 0 && (int)blockIdx.x < total) {
+        tc::prefetch_tensormap(&maps.q);
+        tc::prefetch_tensormap(&maps.k);
+        tc::prefetch_tensormap(&maps.v);
+        tc::prefetch_tensormap(&maps.alpha);
+        issue_inputs(maps, sm, bar_in, blockIdx.x, NT, H);
+        issue_v(maps, sm, bar_v, blockIdx.x, NT, H);
+    }
 
     // persistent loop over chunk-heads ci = (batch*head) * NT + chunk
-    for (int ci = blockIdx.x; ci < total; ci += gridDim.x) {
+    uint32_t it = 0;
+    for (int ci = blockIdx.x; ci < total; ci += gridDim.x, ++it) {
         const int ch = ci % NT, bh = ci / NT;
-        const int b = bh / H, h = bh % H;
+        const int h = bh % H;
         const int t0 = ch * kC;
         const int nvalid = min(kC, T_len - t0);
+        const int nci = ci + gridDim.x;
         uint8_t* wsc = ws + (size_t)ci * WS_CHUNK;
-        const size_t row0 = ((size_t)b * T_len + t0) * H + h;
-
-        // ---- all global loads of this chunk-head, issued together (registers only) ----
-        const int rr = tid >> 3, g = tid & 7;               // row-pass coordinates
-        uint4 qkraw[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0),
-                          make_uint4(0, 0, 0, 0)};
-        if (rr < nvalid) {
-            const size_t o = (row0 + rr * rs) * kDK;
-            qkraw[0] = *reinterpret_cast<const uint4*>(q + o + 8 * g);
-            qkraw[1] = *reinterpret_cast<const uint4*>(q + o + 64 + 8 * g);
-            qkraw[2] = *reinterpret_cast<const uint4*>(k + o + 8 * g);
-            qkraw[3] = *reinterpret_cast<const uint4*>(k + o + 64 + 8 * g);
-        }
-        float4 araw[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int e = tid + 512 * u, r = e >> 5, c4 = (e & 31) * 4;
-            araw[u] = make_float4(1.f, 1.f, 1.f, 1.f);   // identity gates on padding rows
-            if (r < nvalid) araw[u] = *reinterpret_cast<const float4*>(alpha + (row0 + r * rs) * kDK + c4);
-        }
-        uint4 vraw[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int e = tid + 512 * u, r = e >> 4, n8 = (e & 15) * 8;
-            vraw[u] = make_uint4(0, 0, 0, 0);
-            if (r < nvalid) vraw[u] = *reinterpret_cast<const uint4*>(v + (row0 + r * rs) * kDV + n8);
-        }
+        const size_t row0 = ((size_t)(bh / H) * T_len + t0) * H + h;
         const float bval = (tid < 64 && tid < nvalid) ? beta[row0 + tid * rs] : 0.f;
-        // bring the next chunk-head of this CTA into L2 while this one computes: 640 lines of
-        // 128 bytes (q, k, v: 2 per row; alpha: 4 per row), one or two per thread
-        {
-            const int nci = ci + gridDim.x;
-            if (nci < total) {
-                const int nch = nci % NT, nbh = nci / NT;
-                const int nt0 = nch * kC, nv = min(kC, T_len - nt0);
-                const size_t nrow0 = ((size_t)(nbh / H) * T_len + nt0) * H + (nbh % H);
-                for (int li = tid; li < 640; li += 512) {
-                    const char* p;
-                    int r;
-                    if (li < 384) {
-                        const int which = li >> 7, rem = li & 127;
-                        r = rem >> 1;
-                        const __nv_bfloat16* base = which == 0 ? q : which == 1 ? k : v;
-                        p = reinterpret_cast<const char*>(base + (nrow0 + r * rs) * kDK) + 128 * (rem & 1);
-                    } else {
-                        const int rem = li - 384;
-                        r = rem >> 2;
-                        p = reinterpret_cast<const char*>(alpha + (nrow0 + r * rs) * kDK) + 128 * (rem & 3);
-                    }
-                    if (r < nv) tc::prefetch_line_l2(p);
-                }
-            }
-        }
-        // the previous chunk-head's bulk stores must have finished reading shared memory
-        if (tid == 0) tc::bulk_wait_read_all();
-        __syncthreads();
 
-        // ======== A1: alpha and V into shared memory ========
-        if (tid == 0) *exact_path = 0;
-        if (tid < 64) sb[tid] = bval;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int e = tid + 512 * u, r = e >> 5, c4 = (e & 31) * 4;
-            *reinterpret_cast<float4*>(G + r * 128 + c4) = araw[u];
-        }
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int e = tid + 512 * u, r = e >> 4, n8 = (e & 15) * 8;
-            *reinterpret_cast<uint4*>(sm + S_V + tc::sw128_mnmajor(r, n8, 64)) = vraw[u];
-        }
-        __syncthreads();
+        tc::mbar_wait(bar_in, it & 1, abort_flag);
 
-        // ======== A2: channel pass -- thread (channel c, block I): signed prefix gamma ========
+        // ======== A2: channel pass -- thread (channel c, 16-row block I): signed prefix ========
+        // gamma_r as a running product within the block; the sign carries the parity (a signed
+        // zero keeps it on underflow).  Rows past the sequence end are identity gates.
         const int cc = tid & 127, cI = tid >> 7;
+        if (tid == 0) *exact_path = 0;
         {
             float p = 1.f;
-            bool neg = false;
 #pragma unroll
             for (int rl = 0; rl < 16; ++rl) {
                 const int r = 16 * cI + rl;
-                const float a = G[r * 128 + cc];
-                p *= fabsf(a);
-                neg ^= (a < 0.f);
-                G[r * 128 + cc] = neg ? -p : p;   // a signed zero keeps the parity on underflow
+                const float a = r < nvalid ? G[r * 128 + cc] : 1.f;
+                p *= a;
+                G[r * 128 + cc] = p;
             }
             gP[cI * 128 + cc] = p;
-            gPar[cI * 128 + cc] = neg ? -1.f : 1.f;
         }
         __syncthreads();
-        {
-            float pre = 1.f, all = 1.f, sC = 1.f;
-#pragma unroll
-            for (int J = 0; J < 4; ++J) {
-                const float P = gP[J * 128 + cc], S = gPar[J * 128 + cc];
-                sC *= S;
-                all *= P;
-                if (J < cI) pre *= P * S;
-            }
-            if (pre != 1.f) {
-#pragma unroll
-                for (int rl = 0; rl < 16; ++rl) G[(16 * cI + rl) * 128 + cc] *= pre;
-            }
-            if (cI == 0) {
-                gGC[cc] = sC * all;
-                if (!(all >= kSafeDecay)) *exact_path = 1;
-            }
+        if (tid < 128) {
+            const float gc = gP[tid] * gP[128 + tid] * gP[256 + tid] * gP[384 + tid];
+            gGC[tid] = gc;
+            if (!(fabsf(gc) >= kSafeDecay)) *exact_path = 1;
         }
+        if (tid < 64) sb[tid] = bval;
+        // the previous chunk-head's bulk stores must have finished reading R, K_end and the rest
+        if (tid == 0) tc::bulk_wait_read_all();
         __syncthreads();
         const bool exact = *exact_path != 0;
 
         // ======== A3: row pass -- thread (row r, 8-channel groups g and g + 8) ========
         {
-            const int r = rr;
+            const int r = tid >> 3, g = tid & 7;
             const int cA = 8 * g, cB = 64 + 8 * g;
             float qa[8], qb[8], ka[8], kb[8];
-            unpack8(qkraw[0], qa);
-            unpack8(qkraw[1], qb);
-            unpack8(qkraw[2], ka);
-            unpack8(qkraw[3], kb);
+            {
+                const uint8_t* qrow = sm + S_QR + r * 256;
+                const uint8_t* krow = sm + S_KR + r * 256;
+                unpack8(*reinterpret_cast<const uint4*>(qrow + 16 * g), qa);
+                unpack8(*reinterpret_cast<const uint4*>(qrow + 128 + 16 * g), qb);
+                unpack8(*reinterpret_cast<const uint4*>(krow + 16 * g), ka);
+                unpack8(*reinterpret_cast<const uint4*>(krow + 128 + 16 * g), kb);
+            }
             // row norms (the rotation preserves them): reduce over the 8 threads of the row
             float sq = 0.f, sk = 0.f;
 #pragma unroll
@@ -402,15 +425,28 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
             }
             const float fq = l2norm ? rsqrtf(sq + kL2Eps) : 1.f;
             const float fk = l2norm ? rsqrtf(sk + kL2Eps) : 1.f;
+            const int rb = r >> 4;
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 const int c0 = hh ? cB : cA;
                 const float* qx = hh ? qb : qa;
                 const float* kx = hh ? kb : ka;
-                float gm[8], kp[8], qp[8], t8[8];
-                ld_f8(G + r * 128 + c0, gm);   // gamma_r: |gamma| with the parity as its sign
+                float gm[8], pre[8], kp[8], qp[8], t8[8];
+                ld_f8(G + r * 128 + c0, gm);   // block-local gamma
+#pragma unroll
+                for (int i = 0; i < 8; ++i) pre[i] = 1.f;
+#pragma unroll
+                for (int J = 0; J < 3; ++J) {
+                    if (J < rb) {
+                        float pj[8];
+                        ld_f8(gP + J * 128 + c0, pj);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) pre[i] *= pj[i];
+                    }
+                }
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
+                    gm[i] *= pre[i];                          // gamma_r, signed
                     const float sg = signbit(gm[i]) ? -1.f : 1.f;
                     kp[i] = kx[i] * fk * sg;   // k'
                     qp[i] = qx[i] * fq * sg;   // q'
@@ -443,6 +479,8 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
         tc::tc_fence_before();
         __syncthreads();
         tc::tc_fence_after();
+        // alpha, q, k of this chunk-head are consumed: bring in the next one's
+        if (tid == 0 && nci < total) issue_inputs(maps, sm, bar_in, nci, NT, H);
 
         if (!exact) {
             // ======== B: [A | M] = L R^T on the tensor cores (M = 128, N = 64, K = 128) ========
@@ -506,7 +544,7 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
                     }
                 }
                 sA[r * kStrideA + j] = j < r ? sb[r] * accA : 0.f;
-                *reinterpret_cast<__nv_bfloat16*>(sM + tc::sw128_kmajor(r, j, 64)) = __float2bfloat16_rn(accM);
+                st_bf16(sM, tc::sw128_kmajor(r, j, 64), accM);
             }
             __syncthreads();
             // rescale L to (g k', g q') with g = exp2(L_r) and form K_end = sigma_C exp2(L_C - L_j) k'
@@ -517,47 +555,16 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
                 __nv_bfloat16* qr = reinterpret_cast<__nv_bfloat16*>(sL + tc::sw128_kmajor(64 + r, c, 128));
                 const float kv = __bfloat162float(*kr), qv = __bfloat162float(*qr);
                 const float sC = signbit(gGC[c]) ? -1.f : 1.f;
-                *reinterpret_cast<__nv_bfloat16*>(sm + S_KE + tc::sw128_mnmajor(r, c, 64)) =
-                    __float2bfloat16_rn(sC * exp2f(sLg[63 * 128 + c] - sLg[r * 128 + c]) * kv);
+                st_bf16(sm + S_KE, tc::sw128_mnmajor(r, c, 64), sC * exp2f(sLg[63 * 128 + c] - sLg[r * 128 + c]) * kv);
                 *kr = __float2bfloat16_rn(gr * kv);
                 *qr = __float2bfloat16_rn(gr * qv);
             }
         }
-        tc::tc_fence_before();
         __syncthreads();
 
         // ======== C: T = (I + A)^-1 (fp32), T' = T diag(beta) (bf16) ========
-        for (int e = tid; e < 64 * 64; e += 512) {
-            const int r = e >> 6, j = e & 63;
-            if ((j >> 4) > (r >> 4)) sT[r * kStrideA + j] = 0.f;
-        }
-        if (warp < 4 && lane < 16) {
-            const int J = warp, l = lane, base = 16 * J;
-            float tcol[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-                for (int m = 0; m < 16; m += 2) {
-                    if (m < i) a0 += sA[(base + i) * kStrideA + base + m] * tcol[m];
-                    if (m + 1 < i) a1 += sA[(base + i) * kStrideA + base + m + 1] * tcol[m + 1];
-                }
-                tcol[i] = i < l ? 0.f : (i == l ? 1.f : -(a0 + a1));
-            }
-#pragma unroll
-            for (int i = 0; i < 16; ++i) sT[(base + i) * kStrideA + base + l] = tcol[i];
-        }
-        __syncthreads();
-        t_offdiag_level<1>(sA, sT, sX, sPt, tid);
-        t_offdiag_level<2>(sA, sT, sX, sPt, tid);
-        t_offdiag_level<3>(sA, sT, sX, sPt, tid);
-        for (int e = tid; e < 64 * 8; e += 512) {
-            const int r = e >> 3, j0 = (e & 7) * 8;
-            float y[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) y[i] = sT[r * kStrideA + j0 + i] * sb[j0 + i];
-            st16(sm + S_TB, tc::sw128_kmajor(r, j0, 64), y);
-        }
+        t_solve(sA, sT, sb, sm + S_TB, reinterpret_cast<float*>(sm + S_X),
+                reinterpret_cast<float*>(sm + S_Y), tid);
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
         __syncthreads();
@@ -566,6 +573,7 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
         // ======== D: W = T' K_gamma, U~ = T' V  (M = 64, N = 128 each, K = 64) ========
         // K_gamma is rows 0..63 of L, read as an MN-major operand: 64-column blocks 16 KB apart.
         if (tid == 0) {
+            tc::mbar_wait(bar_v, it & 1, abort_flag);
             const uint32_t a0 = tc::smem_u32(sm + S_TB);
             const uint32_t kg = tc::smem_u32(sL), vv = tc::smem_u32(sm + S_V);
             const uint32_t idesc = tc::idesc_bf16_f32(64, 128, 0, 1);
@@ -580,6 +588,8 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
         tc::mbar_wait(bar, phase & 1, abort_flag);
         ++phase;
         tc::tc_fence_after();
+        // V of this chunk-head is consumed: bring in the next one's
+        if (tid == 0 && nci < total) issue_v(maps, sm, bar_v, nci, NT, H);
         {
             // warp w: rows 16 (w % 4) + lane (lane < 16); 64-column slice w / 4:
             // slices 0, 1 -> W columns 0..127, slices 2, 3 -> U~ columns 0..127
@@ -686,48 +696,63 @@ ckda_tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
 }
 
 // ---- kernel 2: the serial state pass ------------------------------------------------------------
+// Warp roles (320 threads):
+//   warps 0-3  chain epilogue: thread t owns state row t; S_next = D_c + B_c in fp32 registers,
+//              written back as the bf16 B operand of the next product
+//   warp 4     tensor-core issue: D_c = A_c S (M = 128, N = 32) and D_o = Q' S (M = 64)
+//   warp 5     loads: 1-D bulk copies of each chunk's A_c, Q', B_c and O_loc, three stages
+//   warps 6-9  output epilogue: O = scale (D_o + O_loc), rows in the M = 64 layout
+// Only the first two roles sit on the serial path.  S alternates between two shared-memory
+// tiles, so the output product of chunk c may still read S_c while S_{c+1} is being written; the
+// output accumulator has four TMEM buffers.
 constexpr int kStages = 3;
+constexpr int kOutBufs = 4;
 constexpr uint32_t P2_STAGE = 61440;                    // A_c 32 KB, Q' 16 KB, B_c 8 KB, O_loc 4 KB
 constexpr uint32_t P2_AC = 0, P2_QP = 32768, P2_BC = 49152, P2_OL = 57344;
 constexpr uint32_t P2_LOAD_BYTES = 32768 + 16384 + WS_TILE;
-constexpr uint32_t P2_ST = kStages * P2_STAGE;          // S operand bf16, K-major 32 rows x 128
-constexpr uint32_t P2_SM = P2_ST + 8192;
+constexpr uint32_t P2_ST = kStages * P2_STAGE;          // S operands: 2 x (MN-major, 128 K-rows)
+constexpr uint32_t P2_ST_BYTES = 16384;
+constexpr uint32_t P2_SM = P2_ST + 2 * P2_ST_BYTES;
 constexpr uint32_t P2_BYTES = P2_SM + 256 + 1024;
+constexpr int kStateThreads = 320;
 
-__global__ void __launch_bounds__(160, 1)
+__global__ void __launch_bounds__(kStateThreads, 1)
 ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
               __nv_bfloat16* __restrict__ out, float* __restrict__ hT, int T_len, int H, int NT,
               float scale) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(sm + P2_SM);  // [3]
-    uint64_t* empty = full + 3;                                // [3]
-    uint64_t* mma_c = full + 6;
-    uint64_t* mma_o = full + 7;
-    uint64_t* epi = full + 8;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(full + 9);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(full + 10);
+    uint64_t* full = reinterpret_cast<uint64_t*>(sm + P2_SM);  // [kStages]
+    uint64_t* empty = full + kStages;                          // [kStages]
+    uint64_t* mma_c = empty + kStages;                         // D_c complete
+    uint64_t* epi = mma_c + 1;                                 // S operand written
+    uint64_t* mma_o = epi + 1;                                 // [kOutBufs] D_o complete
+    uint64_t* o_free = mma_o + kOutBufs;                       // [kOutBufs] D_o read back
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_free + kOutBufs);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int tile = blockIdx.x % kNTile, bh = blockIdx.x / kNTile;
     const int b = bh / H, h = bh % H;
     const int n0 = tile * kDVT;
     const uint8_t* wsh = ws + (size_t)bh * NT * WS_CHUNK;
-    uint8_t* sST = sm + P2_ST;
 
     if (warp == 0) {
-        tc::tmem_alloc(tmem_slot, 128);
+        tc::tmem_alloc(tmem_slot, 256);
         tc::tmem_relinquish();
     }
     if (tid == 128) {
         for (int s = 0; s < kStages; ++s) {
             tc::mbar_init(&full[s], 1);
-            tc::mbar_init(&empty[s], 128);
+            tc::mbar_init(&empty[s], 256);
         }
         tc::mbar_init(mma_c, 1);
-        tc::mbar_init(mma_o, 1);
         tc::mbar_init(epi, 128);
+        for (int s = 0; s < kOutBufs; ++s) {
+            tc::mbar_init(&mma_o[s], 1);
+            tc::mbar_init(&o_free[s], 128);
+        }
         tc::fence_mbar_init();
         *abort_flag = 0;
     }
@@ -736,10 +761,10 @@ ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t dc = tmem;                 // D_c: 128 lanes x 32 columns
-    const uint32_t dob = tmem + 32;           // D_o: two buffers of 32 columns (M = 64 layout)
+    const uint32_t dob = tmem + 32;           // D_o: kOutBufs buffers of 32 columns (M = 64 layout)
 
-    if (tid < 128) {
-        // ---- epilogue: thread t owns state row t (TMEM lane t of D_c) ----
+    if (warp < 4) {
+        // ---- chain epilogue: thread t owns state row t (TMEM lane t of D_c) ----
         const int t = tid;
         float S[kDVT];
         if (h0) {
@@ -753,18 +778,21 @@ ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
 #pragma unroll
             for (int j = 0; j < kDVT; ++j) S[j] = 0.f;
         }
+        // S as an MN-major B operand: K-row t holds the 32 dv values of state row t
+        auto put_s = [&](int buf) {
+            uint8_t* dst = sm + P2_ST + buf * P2_ST_BYTES;
 #pragma unroll
-        for (int j = 0; j < kDVT; ++j)
-            *reinterpret_cast<__nv_bfloat16*>(sST + tc::sw128_kmajor(j, t, 32)) = __float2bfloat16_rn(S[j]);
+            for (int j = 0; j < kDVT; j += 8) st16(dst, tc::sw128_mnmajor(t, j, kDK), S + j);
+        };
+        put_s(0);
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
         tc::mbar_arrive(epi);
         for (int ch = 0; ch < NT; ++ch) {
             const int st = ch % kStages;
             const uint8_t* stg = sm + st * P2_STAGE;
-            // chain: S = D_c + B_c
-            tc::mbar_wait(mma_c, ch & 1, abort_flag);
-            tc::mbar_wait(&full[st], (ch / kStages) & 1, abort_flag);
+            if (!tc::mbar_wait(mma_c, ch & 1, abort_flag)) break;
+            if (!tc::mbar_wait(&full[st], (ch / kStages) & 1, abort_flag)) break;
             tc::tc_fence_after();
             float d[32];
             tc::tmem_ld32_sync(tc::tmem_addr(dc, 32 * warp, 0), d);
@@ -776,18 +804,88 @@ ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
 #pragma unroll
                 for (int i = 0; i < 8; ++i) S[8 * j + i] = d[8 * j + i] + y[i];
             }
-#pragma unroll
-            for (int j = 0; j < kDVT; ++j)
-                *reinterpret_cast<__nv_bfloat16*>(sST + tc::sw128_kmajor(j, t, 32)) = __float2bfloat16_rn(S[j]);
+            put_s((ch + 1) & 1);
             tc::fence_proxy_async_smem();
             tc::tc_fence_before();
             tc::mbar_arrive(epi);
-            // output (off the critical path): O = scale (D_o + O_loc), rows in the M = 64 layout
-            tc::mbar_wait(mma_o, ch & 1, abort_flag);
+            tc::mbar_arrive(&empty[st]);
+        }
+        if (hT && !*abort_flag) {
+            float4* dst = reinterpret_cast<float4*>(hT + ((size_t)bh * kDK + t) * kDV + n0);
+#pragma unroll
+            for (int j = 0; j < kDVT / 4; ++j)
+                dst[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
+        }
+    } else if (warp == 4) {
+        if (lane == 0) {
+            // ---- tensor-core issue ----
+            const uint32_t idc = tc::idesc_bf16_f32(128, kDVT, 0, 1);
+            const uint32_t ido = tc::idesc_bf16_f32(64, kDVT, 0, 1);
+            for (int ch = 0; ch < NT; ++ch) {
+                const int st = ch % kStages, ob = ch % kOutBufs;
+                const uint32_t stg = tc::smem_u32(sm + st * P2_STAGE);
+                const uint32_t s_addr = tc::smem_u32(sm + P2_ST + (ch & 1) * P2_ST_BYTES);
+                if (!tc::mbar_wait(epi, ch & 1, abort_flag)) break;            // S_ch written
+                if (!tc::mbar_wait(&full[st], (ch / kStages) & 1, abort_flag)) break;
+                tc::tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint64_t bd = tc::smem_desc_sw128(s_addr + ks * 2048, P2_ST_BYTES, 1024);
+                    const uint64_t ad = tc::smem_desc_sw128(stg + P2_AC + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+                    tc::mma_bf16(dc, ad, bd, idc, ks > 0 ? 1u : 0u);
+                }
+                tc::mma_commit(mma_c);
+                if (ch >= kOutBufs &&
+                    !tc::mbar_wait(&o_free[ob], ((ch / kOutBufs) - 1) & 1, abort_flag))
+                    break;
+                tc::tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint64_t bd = tc::smem_desc_sw128(s_addr + ks * 2048, P2_ST_BYTES, 1024);
+                    const uint64_t ad = tc::smem_desc_sw128(stg + P2_QP + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
+                    tc::mma_bf16(dob + 32 * ob, ad, bd, ido, ks > 0 ? 1u : 0u);
+                }
+                tc::mma_commit(&mma_o[ob]);
+            }
+        }
+    } else if (warp == 5) {
+        if (lane == 0) {
+            // ---- loads ----
+            int issued = 0;
+            for (; issued < NT; ++issued) {
+                const int st = issued % kStages;
+                if (issued >= kStages &&
+                    !tc::mbar_wait(&empty[st], ((issued / kStages) - 1) & 1, abort_flag))
+                    break;
+                uint8_t* stg = sm + st * P2_STAGE;
+                const uint8_t* src = wsh + (size_t)issued * WS_CHUNK;
+                tc::mbar_arrive_expect_tx(&full[st], P2_LOAD_BYTES);
+                tc::bulk_g2s(stg + P2_AC, src + WS_AC, 32768, &full[st]);
+                tc::bulk_g2s(stg + P2_QP, src + WS_QP, 16384, &full[st]);
+                tc::bulk_g2s(stg + P2_BC, src + WS_TILES + tile * WS_TILE, WS_TILE, &full[st]);
+            }
+            if (*abort_flag) {
+                // let every copy still in flight land before the shared memory is released
+                for (int c = issued > kStages ? issued - kStages : 0; c < issued; ++c)
+                    for (uint32_t i = 0; i < tc::kSpinLimit; ++i)
+                        if (tc::mbar_try_wait(&full[c % kStages], (c / kStages) & 1)) break;
+            }
+        }
+    } else {
+        // ---- output epilogue: warp w reads TMEM lanes 32 (w % 4) .. (rows 16 (w % 4) + lane) ----
+        const int q4 = warp & 3;
+        for (int ch = 0; ch < NT; ++ch) {
+            const int st = ch % kStages, ob = ch % kOutBufs;
+            const uint8_t* stg = sm + st * P2_STAGE;
+            if (!tc::mbar_wait(&mma_o[ob], (ch / kOutBufs) & 1, abort_flag)) break;
+            if (!tc::mbar_wait(&full[st], (ch / kStages) & 1, abort_flag)) break;
             tc::tc_fence_after();
-            tc::tmem_ld32_sync(tc::tmem_addr(dob + 32 * (ch & 1), 32 * warp, 0), d);
+            float d[32];
+            tc::tmem_ld32_sync(tc::tmem_addr(dob + 32 * ob, 32 * q4, 0), d);
+            tc::tc_fence_before();
+            tc::mbar_arrive(&o_free[ob]);
             if (lane < 16) {
-                const int r = 16 * warp + lane;
+                const int r = 16 * q4 + lane;
                 const int t0 = ch * kC;
                 if (t0 + r < T_len) {
                     const uint4* ol = reinterpret_cast<const uint4*>(stg + P2_OL + r * 64);
@@ -802,74 +900,46 @@ ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
                     }
                 }
             }
-            tc::tc_fence_before();
             tc::mbar_arrive(&empty[st]);
-        }
-        if (hT) {
-            float4* dst = reinterpret_cast<float4*>(hT + ((size_t)bh * kDK + t) * kDV + n0);
-#pragma unroll
-            for (int j = 0; j < kDVT / 4; ++j)
-                dst[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
-        }
-    } else if (tid == 128) {
-        // ---- control thread: stage loads (1-D bulk copies) and MMA issue ----
-        auto load = [&](int c) {
-            const int st = c % kStages;
-            uint8_t* stg = sm + st * P2_STAGE;
-            const uint8_t* src = wsh + (size_t)c * WS_CHUNK;
-            tc::mbar_arrive_expect_tx(&full[st], P2_LOAD_BYTES);
-            tc::bulk_g2s(stg + P2_AC, src + WS_AC, 32768, &full[st]);
-            tc::bulk_g2s(stg + P2_QP, src + WS_QP, 16384, &full[st]);
-            tc::bulk_g2s(stg + P2_BC, src + WS_TILES + tile * WS_TILE, WS_TILE, &full[st]);
-        };
-        int issued = 0;
-        for (; issued < kStages && issued < NT; ++issued) load(issued);
-        const uint32_t idc = tc::idesc_bf16_f32(128, kDVT, 0, 0);
-        const uint32_t ido = tc::idesc_bf16_f32(64, kDVT, 0, 0);
-        const uint32_t s_addr = tc::smem_u32(sST);
-        for (int ch = 0; ch < NT; ++ch) {
-            const int st = ch % kStages;
-            const uint32_t stg = tc::smem_u32(sm + st * P2_STAGE);
-            if (!tc::mbar_wait(epi, ch & 1, abort_flag)) break;            // S operand ready
-            if (!tc::mbar_wait(&full[st], (ch / kStages) & 1, abort_flag)) break;
-            tc::tc_fence_after();
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint64_t bd = tc::smem_desc_sw128(s_addr + (ks >> 2) * 4096 + (ks & 3) * 32, 16, 1024);
-                const uint64_t ad = tc::smem_desc_sw128(stg + P2_AC + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-                tc::mma_bf16(dc, ad, bd, idc, ks > 0 ? 1u : 0u);
-            }
-            tc::mma_commit(mma_c);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint64_t bd = tc::smem_desc_sw128(s_addr + (ks >> 2) * 4096 + (ks & 3) * 32, 16, 1024);
-                const uint64_t ad = tc::smem_desc_sw128(stg + P2_QP + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
-                tc::mma_bf16(dob + 32 * (ch & 1), ad, bd, ido, ks > 0 ? 1u : 0u);
-            }
-            tc::mma_commit(mma_o);
-            // refill the stage of chunk ch - 1 once its epilogue has consumed it
-            if (ch >= 1 && issued < NT) {
-                const int prev = ch - 1;
-                if (!tc::mbar_wait(&empty[prev % kStages], (prev / kStages) & 1, abort_flag)) break;
-                load(issued);
-                ++issued;
-            }
-        }
-        // drain: the last output epilogue, then any copy still in flight
-        if (NT > 0) tc::mbar_wait(&empty[(NT - 1) % kStages], ((NT - 1) / kStages) & 1, abort_flag);
-        if (*abort_flag) {
-            atomicExch(&g_tc_error, 2);
-            for (int c = issued > kStages ? issued - kStages : 0; c < issued; ++c)
-                for (uint32_t i = 0; i < tc::kSpinLimit; ++i)
-                    if (tc::mbar_try_wait(&full[c % kStages], (c / kStages) & 1)) break;
         }
     }
     tc::tc_fence_before();
     __syncthreads();
-    if (warp == 0) tc::tmem_dealloc(tmem, 128);
+    if (*abort_flag && tid == 0) atomicExch(&g_tc_error, 2);
+    if (warp == 0) tc::tmem_dealloc(tmem, 256);
 }
 
 }  // namespace
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link against libcuda).
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult qr;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                             &qr) != cudaSuccess ||
+            qr != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }();
+    return fn;
+}
+
+// A [B][T][H][C] array as a 4-D tensor {C, H, T, B}; box = `box_c` channels of 64 tokens of one
+// (batch, head).  Tokens past T read as zeros.
+static bool encode_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, int C,
+                int box_c, int H, int T_len, int B, CUtensorMapSwizzle sw) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)H, (cuuint64_t)T_len, (cuuint64_t)B};
+    const cuuint64_t row = (cuuint64_t)C * esize;
+    const cuuint64_t strides[3] = {row, row * H, row * H * T_len};
+    const cuuint32_t box[4] = {(cuuint32_t)box_c, 1, (cuuint32_t)kC, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, dt, 4, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 size_t chunk_tc_workspace_bytes(int B, int T_len, int H) {
     const size_t nt = (size_t)(T_len + kC - 1) / kC;
@@ -895,15 +965,23 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const f
             cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
         const int total = NT * B * H;
         const int grid = total < nsm ? total : nsm;
-        ckda_tc_intra<<<(unsigned)grid, 512, S_BYTES, stream>>>(
-            static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-            static_cast<const __nv_bfloat16*>(v), alpha, beta, ws, T_len, H, NT, total, l2norm, rp,
-            pos_offset);
+        TcMaps maps;
+        if (!encode_map(&maps.q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK, kDK, H, T_len, B,
+                        CU_TENSOR_MAP_SWIZZLE_NONE) ||
+            !encode_map(&maps.k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK, kDK, H, T_len, B,
+                        CU_TENSOR_MAP_SWIZZLE_NONE) ||
+            !encode_map(&maps.v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDV, 64, H, T_len, B,
+                        CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !encode_map(&maps.alpha, alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kDK, kDK, H, T_len,
+                        B, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return cudaErrorInvalidValue;
+        ckda_tc_intra<<<(unsigned)grid, 512, S_BYTES, stream>>>(maps, alpha, beta, ws, T_len, H, NT,
+                                                                total, l2norm, rp, pos_offset);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
     if (stages & 2) {
-        ckda_tc_state<<<(unsigned)(kNTile * B * H), 160, P2_BYTES, stream>>>(
+        ckda_tc_state<<<(unsigned)(kNTile * B * H), kStateThreads, P2_BYTES, stream>>>(
             ws, h0, static_cast<__nv_bfloat16*>(out), hT, T_len, H, NT, scale);
         e = cudaGetLastError();
     }

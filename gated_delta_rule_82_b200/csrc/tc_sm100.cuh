@@ -1,5 +1,5 @@
 // tc_sm100.cuh -- thin inline-PTX wrappers for the sm_100a tensor-core path:
-// mbarriers, 1-D bulk (TMA) copies, Tensor Memory allocation, tcgen05.mma with shared-memory
+// mbarriers, 1-D bulk and tiled tensor (TMA) copies, Tensor Memory allocation, tcgen05.mma with shared-memory
 // operand descriptors, tcgen05.commit and tcgen05.ld.
 //
 // Operand tiles use the 128-byte swizzle.  A K-major tile (rows = M or N, K contiguous) keeps
@@ -69,6 +69,21 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
     asm volatile(
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
         ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
+
+// ---- tiled tensor copy (TMA engine), global -> shared, completing on an mbarrier ---------------
+// `map` is a CUtensorMap in kernel-parameter (grid-constant) memory; coordinates are in elements,
+// innermost first.  The innermost coordinate times the element size must be a multiple of 16.
+__device__ __forceinline__ void tma_load_4d(void* dst, const void* map, int c0, int c1, int c2,
+                                            int c3, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2),
+          "r"(c3), "r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void prefetch_tensormap(const void* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
 // ---- 1-D bulk copy, shared -> global (bulk-group completion) --------------------------------

@@ -90,7 +90,9 @@ umma_selftest_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16* _
 
 cudaError_t launch_umma_selftest(const void* A, const void* B, float* D, int M, int N, int K,
                                  int b_mn_major, cudaStream_t stream) {
-    size_t smem = (size_t)(M + N) * K * 2 + 1024;
+    // an MN-major B occupies whole 128-byte rows: ceil(N / 64) blocks of K rows
+    const size_t b_bytes = b_mn_major ? (size_t)((N + 63) / 64) * K * 128 : (size_t)N * K * 2;
+    size_t smem = (size_t)M * K * 2 + b_bytes + 1024;
     cudaError_t e = cudaFuncSetAttribute(umma_selftest_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

@@ -153,7 +153,7 @@ CKDA_API ckda_status ckda_decode_step(const void* q, const void* k, const void* 
  * descriptors with the 128-byte swizzle, TMEM accumulator, one CTA).
  *   b_mn_major == 0: B is [N, K] row-major (K contiguous), D = A B^T  (K-major B operand)
  *   b_mn_major == 1: B is [K, N] row-major (N contiguous), D = A B    (MN-major B operand)
- * M in {64, 128}; N a multiple of 16 in [16, 256] (a multiple of 64 when b_mn_major);
+ * M in {64, 128}; N a multiple of 16 in [16, 256] (32 or a multiple of 64 when b_mn_major);
  * K a multiple of 64 in [64, 256].  Lets a user check the tensor-core path on a device.
  */
 CKDA_API ckda_status ckda_selftest_umma(const void* A, const void* B, float* D, int M, int N, int K,

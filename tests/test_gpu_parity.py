@@ -30,12 +30,12 @@ def _cuda():
 # ---- tensor-core wrapper self-test ----------------------------------------------------------
 
 @pytest.mark.parametrize("M", [64, 128])
-@pytest.mark.parametrize("N", [16, 64, 128, 256])
+@pytest.mark.parametrize("N", [16, 32, 64, 128, 256])
 @pytest.mark.parametrize("K", [64, 128, 256])
 @pytest.mark.parametrize("mn", [0, 1])
 def test_umma_selftest(M, N, K, mn):
-    if mn and N % 64:
-        pytest.skip("MN-major operand needs N % 64 == 0")
+    if mn and N % 64 and N != 32:
+        pytest.skip("MN-major operand needs N = 32 or N % 64 == 0")
     g = torch.Generator().manual_seed(M * 1000 + N * 10 + K + mn)
     A = torch.randn(M, K, generator=g).bfloat16()
     B = torch.randn(K, N, generator=g).bfloat16() if mn else torch.randn(N, K, generator=g).bfloat16()

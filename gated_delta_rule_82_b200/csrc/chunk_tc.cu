@@ -479,22 +479,22 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const float* __restrict__ alp
         tc::tc_fence_before();
         __syncthreads();
         tc::tc_fence_after();
-        // alpha, q, k of this chunk-head are consumed: bring in the next one's
-        if (tid == 0 && nci < total) issue_inputs(maps, sm, bar_in, nci, NT, H);
-
         if (!exact) {
             // ======== B: [A | M] = L R^T on the tensor cores (M = 128, N = 64, K = 128) ========
-            if (tid == 0) {
-                const uint32_t l0 = tc::smem_u32(sL), r0a = tc::smem_u32(sm + S_R);
+            if (warp == 0) {
+                const uint64_t ad = tc::smem_desc_sw128(tc::smem_u32(sL), 16, 1024);
+                const uint64_t bd = tc::smem_desc_sw128(tc::smem_u32(sm + S_R), 16, 1024);
                 const uint32_t idesc = tc::idesc_bf16_f32(128, 64, 0, 0);
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint64_t ad = tc::smem_desc_sw128(l0 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-                    const uint64_t bd = tc::smem_desc_sw128(r0a + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
-                    tc::mma_bf16(tmem, ad, bd, idesc, ks > 0 ? 1u : 0u);
-                }
-                tc::mma_commit(bar);
+                for (int ks = 0; ks < 8; ++ks)
+                    tc::mma_bf16_warp(tmem, tc::desc_add(ad, (ks >> 2) * 16384 + (ks & 3) * 32),
+                                      tc::desc_add(bd, (ks >> 2) * 8192 + (ks & 3) * 32), idesc, ks > 0);
+                tc::mma_commit_warp(bar);
             }
+        }
+        // alpha, q, k of this chunk-head are consumed: bring in the next one's
+        if (tid == 0 && nci < total) issue_inputs(maps, sm, bar_in, nci, NT, H);
+        if (!exact) {
             tc::mbar_wait(bar, phase & 1, abort_flag);
             ++phase;
             tc::tc_fence_after();
@@ -572,18 +572,20 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const float* __restrict__ alp
 
         // ======== D: W = T' K_gamma, U~ = T' V  (M = 64, N = 128 each, K = 64) ========
         // K_gamma is rows 0..63 of L, read as an MN-major operand: 64-column blocks 16 KB apart.
-        if (tid == 0) {
+        if (warp == 0) {
             tc::mbar_wait(bar_v, it & 1, abort_flag);
-            const uint32_t a0 = tc::smem_u32(sm + S_TB);
-            const uint32_t kg = tc::smem_u32(sL), vv = tc::smem_u32(sm + S_V);
+            __syncwarp();
+            const uint64_t ad = tc::smem_desc_sw128(tc::smem_u32(sm + S_TB), 16, 1024);
+            const uint64_t kd = tc::smem_desc_sw128(tc::smem_u32(sL), 16384, 1024);
+            const uint64_t vd = tc::smem_desc_sw128(tc::smem_u32(sm + S_V), 8192, 1024);
             const uint32_t idesc = tc::idesc_bf16_f32(64, 128, 0, 1);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t ad = tc::smem_desc_sw128(a0 + ks * 32, 16, 1024);
-                tc::mma_bf16(tmem, ad, tc::smem_desc_sw128(kg + ks * 2048, 16384, 1024), idesc, ks > 0);
-                tc::mma_bf16(tmem + 128, ad, tc::smem_desc_sw128(vv + ks * 2048, 8192, 1024), idesc, ks > 0);
+                const uint64_t a = tc::desc_add(ad, ks * 32);
+                tc::mma_bf16_warp(tmem, a, tc::desc_add(kd, ks * 2048), idesc, ks > 0);
+                tc::mma_bf16_warp(tmem + 128, a, tc::desc_add(vd, ks * 2048), idesc, ks > 0);
             }
-            tc::mma_commit(bar);
+            tc::mma_commit_warp(bar);
         }
         tc::mbar_wait(bar, phase & 1, abort_flag);
         ++phase;
@@ -610,23 +612,23 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const float* __restrict__ alp
         tc::tc_fence_after();
 
         // ======== F: M [W | U~] (M = 64) and K_end^T [W | U~] (M = 128, MN-major A) ========
-        if (tid == 0) {
-            const uint32_t am = tc::smem_u32(sm + S_M), ke = tc::smem_u32(sm + S_KE);
-            const uint32_t w0 = tc::smem_u32(sm + S_W), u0 = tc::smem_u32(sm + S_U);
+        if (warp == 0) {
+            const uint64_t md = tc::smem_desc_sw128(tc::smem_u32(sm + S_M), 16, 1024);
+            const uint64_t ked = tc::smem_desc_sw128(tc::smem_u32(sm + S_KE), 8192, 1024);
+            const uint64_t wd = tc::smem_desc_sw128(tc::smem_u32(sm + S_W), 8192, 1024);
+            const uint64_t ud = tc::smem_desc_sw128(tc::smem_u32(sm + S_U), 8192, 1024);
             const uint32_t id64 = tc::idesc_bf16_f32(64, 128, 0, 1);
             const uint32_t id128 = tc::idesc_bf16_f32(128, 128, 1, 1);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t bw = tc::smem_desc_sw128(w0 + ks * 2048, 8192, 1024);
-                const uint64_t bu = tc::smem_desc_sw128(u0 + ks * 2048, 8192, 1024);
-                const uint64_t adm = tc::smem_desc_sw128(am + ks * 32, 16, 1024);
-                const uint64_t ade = tc::smem_desc_sw128(ke + ks * 2048, 8192, 1024);
-                tc::mma_bf16(tmem, adm, bw, id64, ks > 0);
-                tc::mma_bf16(tmem + 128, adm, bu, id64, ks > 0);
-                tc::mma_bf16(tmem + 256, ade, bw, id128, ks > 0);
-                tc::mma_bf16(tmem + 384, ade, bu, id128, ks > 0);
+                const uint64_t bw = tc::desc_add(wd, ks * 2048), bu = tc::desc_add(ud, ks * 2048);
+                const uint64_t adm = tc::desc_add(md, ks * 32), ade = tc::desc_add(ked, ks * 2048);
+                tc::mma_bf16_warp(tmem, adm, bw, id64, ks > 0);
+                tc::mma_bf16_warp(tmem + 128, adm, bu, id64, ks > 0);
+                tc::mma_bf16_warp(tmem + 256, ade, bw, id128, ks > 0);
+                tc::mma_bf16_warp(tmem + 384, ade, bu, id128, ks > 0);
             }
-            tc::mma_commit(bar);
+            tc::mma_commit_warp(bar);
         }
         tc::mbar_wait(bar, phase & 1, abort_flag);
         ++phase;
@@ -696,25 +698,35 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const float* __restrict__ alp
 }
 
 // ---- kernel 2: the serial state pass ------------------------------------------------------------
-// Warp roles (320 threads):
-//   warps 0-3  chain epilogue: thread t owns state row t; S_next = D_c + B_c in fp32 registers,
-//              written back as the bf16 B operand of the next product
-//   warp 4     tensor-core issue: D_c = A_c S (M = 128, N = 32) and D_o = Q' S (M = 64)
-//   warp 5     loads: 1-D bulk copies of each chunk's A_c, Q', B_c and O_loc, three stages
-//   warps 6-9  output epilogue: O = scale (D_o + O_loc), rows in the M = 64 layout
-// Only the first two roles sit on the serial path.  S alternates between two shared-memory
-// tiles, so the output product of chunk c may still read S_c while S_{c+1} is being written; the
-// output accumulator has four TMEM buffers.
+// Warp roles (384 threads):
+//   warps 0-3   chain epilogue: thread t owns state row t; S_next = D_c + B_c in fp32 registers,
+//               written back as the bf16 B operand of the next product
+//   warp 4      chain issue: D_c = A_c S (M = 128, N = 32)
+//   warp 5      chain loads: A_c and B_c of each chunk (1-D bulk copies, three stages)
+//   warp 6      output loads: Q' and O_loc of each chunk (three stages)
+//   warp 7      output issue: D_o = Q' S (M = 64, N = 32)
+//   warps 8-11  output epilogue: O = scale (D_o + O_loc), rows in the M = 64 layout
+// Only the first three roles are on the serial path; the output side runs behind it and never
+// holds a chain stage.  S rotates through four shared-memory buffers: S_{c+4} is written only
+// after the output product of chunk c has read S_c.  Every role issues from a converged warp
+// (one elected lane) and every wait is bounded and ends warp-uniformly.
 constexpr int kStages = 3;
 constexpr int kOutBufs = 4;
-constexpr uint32_t P2_STAGE = 61440;                    // A_c 32 KB, Q' 16 KB, B_c 8 KB, O_loc 4 KB
-constexpr uint32_t P2_AC = 0, P2_QP = 32768, P2_BC = 49152, P2_OL = 57344;
-constexpr uint32_t P2_LOAD_BYTES = 32768 + 16384 + WS_TILE;
-constexpr uint32_t P2_ST = kStages * P2_STAGE;          // S operands: 2 x (MN-major, 128 K-rows)
+constexpr int kSBufs = 4;
+constexpr uint32_t P2_CSTAGE = 40960;                    // A_c 32 KB, B_c 8 KB
+constexpr uint32_t P2_AC = 0, P2_BC = 32768;
+constexpr uint32_t P2_OSTAGE = 20480;                    // Q' 16 KB, O_loc 4 KB
+constexpr uint32_t P2_QP = 0, P2_OL = 16384;
+constexpr uint32_t P2_OBASE = kStages * P2_CSTAGE;
+// S operands: four MN-major buffers of 128 K-rows x 32 dv, two per 16 KB tile (dv columns 0..31
+// and 32..63 of the swizzled 128-byte rows)
+constexpr uint32_t P2_ST = P2_OBASE + kStages * P2_OSTAGE;
 constexpr uint32_t P2_ST_BYTES = 16384;
 constexpr uint32_t P2_SM = P2_ST + 2 * P2_ST_BYTES;
-constexpr uint32_t P2_BYTES = P2_SM + 256 + 1024;
-constexpr int kStateThreads = 320;
+constexpr uint32_t P2_BYTES = P2_SM + 512 + 1024;
+constexpr int kStateThreads = 384;
+__device__ __forceinline__ uint32_t s_tile(int buf) { return (uint32_t)(buf >> 1) * P2_ST_BYTES; }
+__device__ __forceinline__ int s_col(int buf) { return 32 * (buf & 1); }
 
 __global__ void __launch_bounds__(kStateThreads, 1)
 ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
@@ -723,13 +735,16 @@ ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(sm + P2_SM);  // [kStages]
-    uint64_t* empty = full + kStages;                          // [kStages]
-    uint64_t* mma_c = empty + kStages;                         // D_c complete
-    uint64_t* epi = mma_c + 1;                                 // S operand written
-    uint64_t* mma_o = epi + 1;                                 // [kOutBufs] D_o complete
-    uint64_t* o_free = mma_o + kOutBufs;                       // [kOutBufs] D_o read back
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_free + kOutBufs);
+    uint64_t* full_c = reinterpret_cast<uint64_t*>(sm + P2_SM);  // [kStages]
+    uint64_t* empty_c = full_c + kStages;                        // [kStages]
+    uint64_t* full_o = empty_c + kStages;                        // [kStages]
+    uint64_t* empty_o = full_o + kStages;                        // [kStages]
+    uint64_t* mma_c = empty_o + kStages;                         // D_c complete
+    uint64_t* s_ready = mma_c + 1;                               // [kSBufs] S buffer written
+    uint64_t* mma_o = s_ready + kSBufs;                          // [kOutBufs] D_o complete
+    uint64_t* o_free = mma_o + kOutBufs;                         // [kOutBufs] D_o read back
+    uint64_t* dc_issued = o_free + kOutBufs;                     // [kSBufs] D_c(c) issued
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(dc_issued + kSBufs);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -742,16 +757,21 @@ ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
         tc::tmem_alloc(tmem_slot, 256);
         tc::tmem_relinquish();
     }
-    if (tid == 128) {
+    if (tid == 32) {
         for (int s = 0; s < kStages; ++s) {
-            tc::mbar_init(&full[s], 1);
-            tc::mbar_init(&empty[s], 256);
+            tc::mbar_init(&full_c[s], 1);
+            tc::mbar_init(&empty_c[s], 4);   // one arrival per chain-epilogue warp
+            tc::mbar_init(&full_o[s], 1);
+            tc::mbar_init(&empty_o[s], 4);   // one arrival per output-epilogue warp
         }
         tc::mbar_init(mma_c, 1);
-        tc::mbar_init(epi, 128);
+        for (int s = 0; s < kSBufs; ++s) {
+            tc::mbar_init(&s_ready[s], 4);
+            tc::mbar_init(&dc_issued[s], 1);
+        }
         for (int s = 0; s < kOutBufs; ++s) {
             tc::mbar_init(&mma_o[s], 1);
-            tc::mbar_init(&o_free[s], 128);
+            tc::mbar_init(&o_free[s], 4);
         }
         tc::fence_mbar_init();
         *abort_flag = 0;
@@ -762,6 +782,11 @@ ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
     const uint32_t tmem = *tmem_slot;
     const uint32_t dc = tmem;                 // D_c: 128 lanes x 32 columns
     const uint32_t dob = tmem + 32;           // D_o: kOutBufs buffers of 32 columns (M = 64 layout)
+    auto wait = [&](uint64_t* bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, tc::mbar_wait(bar, parity, abort_flag));
+    };
+    const uint64_t s_desc0 = tc::smem_desc_sw128(tc::smem_u32(sm + P2_ST), P2_ST_BYTES, 1024);
+    auto s_desc = [&](int c) { return tc::desc_add(s_desc0, s_tile(c % kSBufs) + 2 * s_col(c % kSBufs)); };
 
     if (warp < 4) {
         // ---- chain epilogue: thread t owns state row t (TMEM lane t of D_c) ----
@@ -779,24 +804,34 @@ ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
             for (int j = 0; j < kDVT; ++j) S[j] = 0.f;
         }
         // S as an MN-major B operand: K-row t holds the 32 dv values of state row t
-        auto put_s = [&](int buf) {
-            uint8_t* dst = sm + P2_ST + buf * P2_ST_BYTES;
+        auto put_s = [&](int c) {
+            const int buf = c % kSBufs;
+            uint8_t* dst = sm + P2_ST + s_tile(buf);
 #pragma unroll
-            for (int j = 0; j < kDVT; j += 8) st16(dst, tc::sw128_mnmajor(t, j, kDK), S + j);
+            for (int j = 0; j < kDVT; j += 8) st16(dst, tc::sw128_mnmajor(t, s_col(buf) + j, kDK), S + j);
+            tc::fence_proxy_async_smem();
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&s_ready[buf]);
         };
         put_s(0);
-        tc::fence_proxy_async_smem();
-        tc::tc_fence_before();
-        tc::mbar_arrive(epi);
         for (int ch = 0; ch < NT; ++ch) {
             const int st = ch % kStages;
-            const uint8_t* stg = sm + st * P2_STAGE;
-            if (!tc::mbar_wait(mma_c, ch & 1, abort_flag)) break;
-            if (!tc::mbar_wait(&full[st], (ch / kStages) & 1, abort_flag)) break;
+            // B_c is in registers before the chain product completes
+            if (!wait(&full_c[st], (ch / kStages) & 1)) break;
+            uint4 bc[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                bc[j] = reinterpret_cast<const uint4*>(sm + st * P2_CSTAGE + P2_BC + t * 64)[j];
+            // buffer (ch + 1) % 4 last held S_{ch-3}: its output product must be done (checked
+            // before the chain product completes, off the serial path)
+            if (ch + 1 < NT && ch + 1 >= kSBufs &&
+                !wait(&mma_o[(ch - 3) % kOutBufs], ((ch - 3) / kOutBufs) & 1))
+                break;
+            if (!wait(mma_c, ch & 1)) break;
             tc::tc_fence_after();
             float d[32];
             tc::tmem_ld32_sync(tc::tmem_addr(dc, 32 * warp, 0), d);
-            const uint4* bc = reinterpret_cast<const uint4*>(stg + P2_BC + t * 64);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 float y[8];
@@ -804,11 +839,11 @@ ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
 #pragma unroll
                 for (int i = 0; i < 8; ++i) S[8 * j + i] = d[8 * j + i] + y[i];
             }
-            put_s((ch + 1) & 1);
-            tc::fence_proxy_async_smem();
-            tc::tc_fence_before();
-            tc::mbar_arrive(epi);
-            tc::mbar_arrive(&empty[st]);
+            if (ch + 1 < NT) put_s(ch + 1);
+            else tc::tc_fence_before();
+            // A_c was read (D_c done) and B_c is in registers: release the chain stage
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&empty_c[st]);
         }
         if (hT && !*abort_flag) {
             float4* dst = reinterpret_cast<float4*>(hT + ((size_t)bh * kDK + t) * kDV + n0);
@@ -817,73 +852,90 @@ ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
                 dst[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
         }
     } else if (warp == 4) {
-        if (lane == 0) {
-            // ---- tensor-core issue ----
-            const uint32_t idc = tc::idesc_bf16_f32(128, kDVT, 0, 1);
-            const uint32_t ido = tc::idesc_bf16_f32(64, kDVT, 0, 1);
-            for (int ch = 0; ch < NT; ++ch) {
-                const int st = ch % kStages, ob = ch % kOutBufs;
-                const uint32_t stg = tc::smem_u32(sm + st * P2_STAGE);
-                const uint32_t s_addr = tc::smem_u32(sm + P2_ST + (ch & 1) * P2_ST_BYTES);
-                if (!tc::mbar_wait(epi, ch & 1, abort_flag)) break;            // S_ch written
-                if (!tc::mbar_wait(&full[st], (ch / kStages) & 1, abort_flag)) break;
-                tc::tc_fence_after();
+        // ---- chain issue ----
+        const uint32_t idc = tc::idesc_bf16_f32(128, kDVT, 0, 1);
+        const uint64_t c_desc0 = tc::smem_desc_sw128(tc::smem_u32(sm), 16, 1024);
+        for (int ch = 0; ch < NT; ++ch) {
+            const int st = ch % kStages;
+            if (!wait(&full_c[st], (ch / kStages) & 1)) break;
+            if (!wait(&s_ready[ch % kSBufs], (ch / kSBufs) & 1)) break;
+            tc::tc_fence_after();
+            const uint64_t ad = tc::desc_add(c_desc0, st * P2_CSTAGE + P2_AC);
+            const uint64_t sd = s_desc(ch);
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint64_t bd = tc::smem_desc_sw128(s_addr + ks * 2048, P2_ST_BYTES, 1024);
-                    const uint64_t ad = tc::smem_desc_sw128(stg + P2_AC + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-                    tc::mma_bf16(dc, ad, bd, idc, ks > 0 ? 1u : 0u);
-                }
-                tc::mma_commit(mma_c);
-                if (ch >= kOutBufs &&
-                    !tc::mbar_wait(&o_free[ob], ((ch / kOutBufs) - 1) & 1, abort_flag))
-                    break;
-                tc::tc_fence_after();
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint64_t bd = tc::smem_desc_sw128(s_addr + ks * 2048, P2_ST_BYTES, 1024);
-                    const uint64_t ad = tc::smem_desc_sw128(stg + P2_QP + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
-                    tc::mma_bf16(dob + 32 * ob, ad, bd, ido, ks > 0 ? 1u : 0u);
-                }
-                tc::mma_commit(&mma_o[ob]);
-            }
+            for (int ks = 0; ks < 8; ++ks)
+                tc::mma_bf16_warp(dc, tc::desc_add(ad, (ks >> 2) * 16384 + (ks & 3) * 32),
+                                  tc::desc_add(sd, ks * 2048), idc, ks > 0 ? 1u : 0u);
+            tc::mma_commit_warp(mma_c);
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&dc_issued[ch % kSBufs]);   // D_o(ch) may follow it
         }
-    } else if (warp == 5) {
+    } else if (warp == 5 || warp == 6) {
+        // ---- loads: warp 5 the chain ring (A_c, B_c), warp 6 the output ring (Q', O_loc) ----
         if (lane == 0) {
-            // ---- loads ----
+            const bool chain = warp == 5;
+            uint64_t* fullb = chain ? full_c : full_o;
+            uint64_t* emptyb = chain ? empty_c : empty_o;
             int issued = 0;
             for (; issued < NT; ++issued) {
                 const int st = issued % kStages;
                 if (issued >= kStages &&
-                    !tc::mbar_wait(&empty[st], ((issued / kStages) - 1) & 1, abort_flag))
+                    !tc::mbar_wait(&emptyb[st], ((issued / kStages) - 1) & 1, abort_flag))
                     break;
-                uint8_t* stg = sm + st * P2_STAGE;
                 const uint8_t* src = wsh + (size_t)issued * WS_CHUNK;
-                tc::mbar_arrive_expect_tx(&full[st], P2_LOAD_BYTES);
-                tc::bulk_g2s(stg + P2_AC, src + WS_AC, 32768, &full[st]);
-                tc::bulk_g2s(stg + P2_QP, src + WS_QP, 16384, &full[st]);
-                tc::bulk_g2s(stg + P2_BC, src + WS_TILES + tile * WS_TILE, WS_TILE, &full[st]);
+                const uint8_t* tl = src + WS_TILES + tile * WS_TILE;
+                if (chain) {
+                    uint8_t* stg = sm + st * P2_CSTAGE;
+                    tc::mbar_arrive_expect_tx(&fullb[st], 32768 + WS_TILE_O);
+                    tc::bulk_g2s(stg + P2_AC, src + WS_AC, 32768, &fullb[st]);
+                    tc::bulk_g2s(stg + P2_BC, tl, WS_TILE_O, &fullb[st]);
+                } else {
+                    uint8_t* stg = sm + P2_OBASE + st * P2_OSTAGE;
+                    tc::mbar_arrive_expect_tx(&fullb[st], 16384 + (WS_TILE - WS_TILE_O));
+                    tc::bulk_g2s(stg + P2_QP, src + WS_QP, 16384, &fullb[st]);
+                    tc::bulk_g2s(stg + P2_OL, tl + WS_TILE_O, WS_TILE - WS_TILE_O, &fullb[st]);
+                }
             }
             if (*abort_flag) {
                 // let every copy still in flight land before the shared memory is released
                 for (int c = issued > kStages ? issued - kStages : 0; c < issued; ++c)
                     for (uint32_t i = 0; i < tc::kSpinLimit; ++i)
-                        if (tc::mbar_try_wait(&full[c % kStages], (c / kStages) & 1)) break;
+                        if (tc::mbar_try_wait(&fullb[c % kStages], (c / kStages) & 1)) break;
             }
+        }
+    } else if (warp == 7) {
+        // ---- output issue ----
+        const uint32_t ido = tc::idesc_bf16_f32(64, kDVT, 0, 1);
+        const uint64_t o_desc0 = tc::smem_desc_sw128(tc::smem_u32(sm + P2_OBASE), 16, 1024);
+        for (int ch = 0; ch < NT; ++ch) {
+            const int st = ch % kStages, ob = ch % kOutBufs;
+            if (!wait(&full_o[st], (ch / kStages) & 1)) break;
+            // issued right behind D_c(ch), so it runs while the chain epilogue works
+            if (!wait(&dc_issued[ch % kSBufs], (ch / kSBufs) & 1)) break;
+            if (ch >= kOutBufs && !wait(&o_free[ob], ((ch / kOutBufs) - 1) & 1)) break;
+            tc::tc_fence_after();
+            const uint64_t qd = tc::desc_add(o_desc0, st * P2_OSTAGE + P2_QP);
+            const uint64_t sd = s_desc(ch);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                tc::mma_bf16_warp(dob + 32 * ob, tc::desc_add(qd, (ks >> 2) * 8192 + (ks & 3) * 32),
+                                  tc::desc_add(sd, ks * 2048), ido, ks > 0 ? 1u : 0u);
+            tc::mma_commit_warp(&mma_o[ob]);
         }
     } else {
         // ---- output epilogue: warp w reads TMEM lanes 32 (w % 4) .. (rows 16 (w % 4) + lane) ----
         const int q4 = warp & 3;
         for (int ch = 0; ch < NT; ++ch) {
             const int st = ch % kStages, ob = ch % kOutBufs;
-            const uint8_t* stg = sm + st * P2_STAGE;
-            if (!tc::mbar_wait(&mma_o[ob], (ch / kOutBufs) & 1, abort_flag)) break;
-            if (!tc::mbar_wait(&full[st], (ch / kStages) & 1, abort_flag)) break;
+            const uint8_t* stg = sm + P2_OBASE + st * P2_OSTAGE;
+            if (!wait(&mma_o[ob], (ch / kOutBufs) & 1)) break;
+            if (!wait(&full_o[st], (ch / kStages) & 1)) break;
             tc::tc_fence_after();
             float d[32];
             tc::tmem_ld32_sync(tc::tmem_addr(dob + 32 * ob, 32 * q4, 0), d);
             tc::tc_fence_before();
-            tc::mbar_arrive(&o_free[ob]);
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&o_free[ob]);
             if (lane < 16) {
                 const int r = 16 * q4 + lane;
                 const int t0 = ch * kC;
@@ -900,7 +952,8 @@ ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
                     }
                 }
             }
-            tc::mbar_arrive(&empty[st]);
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&empty_o[st]);
         }
     }
     tc::tc_fence_before();

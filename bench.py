@@ -273,6 +273,42 @@ def profile_case(case, calls, dev):
     return 0
 
 
+# ---- rank plumbing (one process per GPU; also exercised by CPU tests with the gloo backend) ---
+
+PG_TIMEOUT_S = 120
+
+
+def init_ranks(world, backend="nccl", device=None, timeout_s=PG_TIMEOUT_S):
+    """Join the process group of a world-size > 1 run (rendezvous from MASTER_ADDR/MASTER_PORT).
+    A short timeout makes ranks that wait on a missing peer fail instead of hanging."""
+    import datetime
+    import torch.distributed as dist
+    kw = {"device_id": device} if device is not None else {}
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+
+
+def max_over_ranks(x, device, world):
+    """The maximum of the scalar x over all ranks (one all_reduce(MAX)); x itself when world == 1."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_mtok_s(tokens_per_rank, world, ms_per_step_max):
+    """Whole-job throughput: every rank processes its own batch of tokens_per_rank tokens per
+    step; the job's step time is the slowest rank's."""
+    return tokens_per_rank * world / (ms_per_step_max / 1e3) / 1e6
+
+
+def input_seed(rank, i):
+    """Seed of the i-th rotated input set on `rank`: disjoint synthetic batches per replica."""
+    return 1000 * (rank + 1) + i
+
+
 # ---- our arm -----------------------------------------------------------------------------------
 
 def main():
@@ -292,8 +328,7 @@ def main():
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
+        init_ranks(world, "nccl", dev)
 
     from gated_delta_rule_82_b200 import build as ckbuild
     if rank == 0:
@@ -313,7 +348,7 @@ def main():
 
     # ---- inputs: N_ROTATE independent synthetic batches, resident in HBM --------------------
     sets = [synth.torch_fwd_inputs(B, T, H, dk, dv, kind=w["kind"], dtype=w["dtype"],
-                                   seed=1000 * (rank + 1) + i, device=dev) for i in range(N_ROTATE)]
+                                   seed=input_seed(rank, i), device=dev) for i in range(N_ROTATE)]
     out = torch.empty((B, T, H, dv), dtype=torch.bfloat16, device=dev)
     hT = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
     ws = torch.empty(ck.workspace_bytes(B, T, H, dk, dv, C, torch.bfloat16, "tc"),
@@ -349,13 +384,8 @@ def main():
     time.sleep(0.12)
     sampler.stop()
     clocks = sampler.window(t_host0, t_host1)
-    ms_per_step = ms / args.steps
-    if world > 1:
-        t = torch.tensor([ms_per_step], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_per_step = float(t.item())
-    tokens_per_step = B * T * world
-    value = tokens_per_step / (ms_per_step / 1e3) / 1e6
+    ms_per_step = max_over_ranks(ms / args.steps, dev, world)
+    value = weak_scaling_mtok_s(B * T, world, ms_per_step)
 
     # ---- per-kernel device times (each stage alone, same stream, same rotation) --------------
     ms_intra = event_time_ms(lambda i: step(i, stages=1), args.steps, stream) / args.steps
@@ -461,11 +491,8 @@ def main():
             e2e_step(i)
         n_e2e = max(5, args.steps // 5)
         ms_e2e = event_time_ms(e2e_step, n_e2e, stream) / n_e2e
-        if world > 1:
-            t = torch.tensor([ms_e2e], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
-        e2e = {"value": round(B * T * world / (ms_e2e / 1e3) / 1e6, 3), "unit": "Mtok/s",
+        ms_e2e = max_over_ranks(ms_e2e, dev, world)
+        e2e = {"value": round(weak_scaling_mtok_s(B * T, world, ms_e2e), 3), "unit": "Mtok/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": round(ms_e2e, 4)}
 

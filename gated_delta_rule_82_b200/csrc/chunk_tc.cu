@@ -125,6 +125,26 @@ __device__ __forceinline__ void st_bf16(uint8_t* base, uint32_t off, float x) {
     *reinterpret_cast<__nv_bfloat16*>(base + off) = __float2bfloat16_rn(x);
 }
 
+// 1/x by the hardware approximation (about 1 ulp); the result is rounded to bf16 afterwards.
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// v[lane] for a register array of 32 values, by a select tree on the lane bits (no local memory).
+__device__ __forceinline__ float select_lane(const float* v, int lane) {
+    float a[16], b[8], c[4], d[2];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) a[i] = (lane & 1) ? v[2 * i + 1] : v[2 * i];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) b[i] = (lane & 2) ? a[2 * i + 1] : a[2 * i];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) c[i] = (lane & 4) ? b[2 * i + 1] : b[2 * i];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) d[i] = (lane & 8) ? c[2 * i + 1] : c[2 * i];
+    return (lane & 16) ? d[1] : d[0];
+}
+
 __device__ int g_tc_error;  // nonzero after a bounded wait ran out (diagnostic)
 
 // Tensor maps of one forward call: q, k, v (bf16) and alpha (fp32) as 4-D arrays
@@ -362,13 +382,20 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const float* __restrict__ alp
         }
         __syncthreads();
         if (tid < 128) {
-            const float gc = gP[tid] * gP[128 + tid] * gP[256 + tid] * gP[384 + tid];
+            // block prefix factors (the product of the earlier blocks' totals), in place
+            const float p0 = gP[tid], p1 = gP[128 + tid], p2 = gP[256 + tid], p3 = gP[384 + tid];
+            const float pre2 = p0 * p1, pre3 = pre2 * p2, gc = pre3 * p3;
+            gP[tid] = 1.f;
+            gP[128 + tid] = p0;
+            gP[256 + tid] = pre2;
+            gP[384 + tid] = pre3;
             gGC[tid] = gc;
             if (!(fabsf(gc) >= kSafeDecay)) *exact_path = 1;
         }
         if (tid < 64) sb[tid] = bval;
-        // the previous chunk-head's bulk stores must have finished reading R, K_end and the rest
-        if (tid == 0) tc::bulk_wait_read_all();
+        // the previous chunk-head's first store group (the Q' image over R, tiles 0-1 over
+        // K_end and M) must have finished reading before the row pass rewrites R and K_end
+        if (tid == 0) tc::bulk_wait_read<1>();
         __syncthreads();
         const bool exact = *exact_path != 0;
 
@@ -432,18 +459,8 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const float* __restrict__ alp
                 const float* qx = hh ? qb : qa;
                 const float* kx = hh ? kb : ka;
                 float gm[8], pre[8], kp[8], qp[8], t8[8];
-                ld_f8(G + r * 128 + c0, gm);   // block-local gamma
-#pragma unroll
-                for (int i = 0; i < 8; ++i) pre[i] = 1.f;
-#pragma unroll
-                for (int J = 0; J < 3; ++J) {
-                    if (J < rb) {
-                        float pj[8];
-                        ld_f8(gP + J * 128 + c0, pj);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) pre[i] *= pj[i];
-                    }
-                }
+                ld_f8(G + r * 128 + c0, gm);       // block-local gamma
+                ld_f8(gP + rb * 128 + c0, pre);    // product of the earlier blocks' totals
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     gm[i] *= pre[i];                          // gamma_r, signed
@@ -463,7 +480,7 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const float* __restrict__ alp
                     ld_f8(gGC + c0, ke);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        t8[i] = kp[i] * __frcp_rn(gm[i]);                // k' / g
+                        t8[i] = kp[i] * rcp_approx(gm[i]);               // k' / g
                         ke[i] *= t8[i];                                  // gamma_C k' / g
                     }
                     st16(sm + S_R, tc::sw128_kmajor(r, c0, 64), t8);
@@ -477,6 +494,9 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const float* __restrict__ alp
         }
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
+        // the rest of the previous chunk-head's images (over A, T, W and U) must be read out
+        // before the [A | M] read-back or the exact path rewrites them
+        if (tid == 0) tc::bulk_wait_read<0>();
         __syncthreads();
         tc::tc_fence_after();
         if (!exact) {
@@ -671,11 +691,17 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const float* __restrict__ alp
                     if (slice < 2) {
                         float y[8];
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) y[i] = (n + i == cr ? gc : 0.f) - x[c0 + i];
+                        for (int i = 0; i < 8; ++i) y[i] = -x[c0 + i];
                         st16(sm + S_OUT_AC, tc::sw128_kmajor(cr, n, 128), y);
                     } else {
                         st16(sm + S_OUT_TL, (n >> 5) * WS_TILE + (cr * 32 + (n & 31)) * 2, x + c0);
                     }
+                }
+                // A_c = Diag(gamma_C) - K_end^T W: row c' holds its diagonal element in this slice
+                // when c' / 64 == slice, at x[32 (quarter % 2) + lane]
+                if (slice < 2 && slice == (quarter >> 1)) {
+                    const float dx = (quarter & 1) ? select_lane(x + 32, lane) : select_lane(x, lane);
+                    st_bf16(sm + S_OUT_AC, tc::sw128_kmajor(cr, cr, 128), gc - dx);
                 }
             }
         }
@@ -684,9 +710,13 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const float* __restrict__ alp
         __syncthreads();
         tc::tc_fence_after();
         if (tid == 0) {
-            tc::bulk_s2g(wsc + WS_AC, sm + S_OUT_AC, 32768);
+            // group 1: the images over buffers the next row pass rewrites first
             tc::bulk_s2g(wsc + WS_QP, sm + S_OUT_QP, 16384);
-            tc::bulk_s2g(wsc + WS_TILES, sm + S_OUT_TL, kNTile * WS_TILE);
+            tc::bulk_s2g(wsc + WS_TILES, sm + S_OUT_TL, 2 * WS_TILE);
+            tc::bulk_commit();
+            // group 2: the rest
+            tc::bulk_s2g(wsc + WS_TILES + 2 * WS_TILE, sm + S_OUT_TL + 2 * WS_TILE, 2 * WS_TILE);
+            tc::bulk_s2g(wsc + WS_AC, sm + S_OUT_AC, 32768);
             tc::bulk_commit();
         }
     }

@@ -82,8 +82,8 @@ constexpr uint32_t S_BYTES = S_SM + 3072 + 1024;
 constexpr int kStrideA = 68;         // fp32 row stride of A and T
 // T solve scratch inside R (dead after the [A | M] product)
 constexpr uint32_t S_TB = S_R;               // T' bf16 K-major 64 x 64
-constexpr uint32_t S_X = S_R + 8192;         // X0, X1 fp32 [16][16] each
-constexpr uint32_t S_Y = S_R + 10240;        // Y fp32 [32][36]
+constexpr uint32_t S_X = S_R + 8192;         // X0, X1 fp32 [16][24] each
+constexpr uint32_t S_Y = S_R + 11264;        // Y fp32 [32][40]
 // staging of the chunk's workspace image, over buffers that are dead by then
 constexpr uint32_t S_OUT_AC = S_W;   // A_c image (32 KB, over W and U)
 constexpr uint32_t S_OUT_QP = S_R;   // Q' image (16 KB)
@@ -173,46 +173,68 @@ __device__ __forceinline__ void issue_v(const TcMaps& m, uint8_t* sm, uint64_t* 
     tc::tma_load_4d(sm + S_V + 8192, &m.v, 64, h, t0, b, bar_v);
 }
 
-// out[0..3] (+)= sum_{k < K} a[k] * b[k][0..3]: a row of K floats (16-byte aligned), b rows
-// `bstride` floats apart; both in shared memory.  Four independent accumulators per k quad.
-template <int K>
-__device__ __forceinline__ float4 row_x_cols4(const float* a, const float* b, int bstride) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int k = 0; k < K; k += 4) {
-        const float4 av = *reinterpret_cast<const float4*>(a + k);
-        const float4 b0 = *reinterpret_cast<const float4*>(b + (k + 0) * bstride);
-        const float4 b1 = *reinterpret_cast<const float4*>(b + (k + 1) * bstride);
-        const float4 b2 = *reinterpret_cast<const float4*>(b + (k + 2) * bstride);
-        const float4 b3 = *reinterpret_cast<const float4*>(b + (k + 3) * bstride);
-        acc.x += av.x * b0.x + av.y * b1.x + av.z * b2.x + av.w * b3.x;
-        acc.y += av.x * b0.y + av.y * b1.y + av.z * b2.y + av.w * b3.y;
-        acc.z += av.x * b0.z + av.y * b1.z + av.z * b2.z + av.w * b3.z;
-        acc.w += av.x * b0.w + av.y * b1.w + av.z * b2.w + av.w * b3.w;
-    }
-    return acc;
+// ---- T = (I + A)^-1 ----------------------------------------------------------------------------
+// Merge products of 16 x 16 and 32 x 32 blocks run on the warp-level tensor-core instruction
+// (mma.sync m16n8k8, tf32 operands rounded to nearest, fp32 accumulation): these blocks are below
+// the smallest tcgen05 tile (M = 64).  tf32 keeps 10 mantissa bits (the results become bf16 T').
+// Fragment layout (PTX ISA, mma.m16n8k8 .tf32), g = lane / 4, t = lane % 4:
+//   A (16 x 8, row-major)  a0 = A[g][t], a1 = A[g+8][t], a2 = A[g][t+4], a3 = A[g+8][t+4]
+//   B (8 x 8)              b0 = B[t][g], b1 = B[t+4][g]
+//   C, D (16 x 8, fp32)    c0 = D[g][2t], c1 = D[g][2t+1], c2 = D[g+8][2t], c3 = D[g+8][2t+1]
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
 }
-__device__ __forceinline__ void st_tb4(uint8_t* sTB, int r, int c, float4 t, const float* sb) {
-    const float4 bj = *reinterpret_cast<const float4*>(sb + c);
-    *reinterpret_cast<uint2*>(sTB + tc::sw128_kmajor(r, c, 64)) =
-        make_uint2(pack_bf16(t.x * bj.x, t.y * bj.y), pack_bf16(t.z * bj.z, t.w * bj.w));
+// c (+)= A[16 x K] B[K x 8]: A rows `lda` floats apart, B rows `ldb` floats apart (shared memory)
+template <int K>
+__device__ __forceinline__ void mma_tile_tf32(float c[4], const float* a, int lda, const float* b,
+                                              int ldb, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        const uint32_t a0 = to_tf32(a[g * lda + k0 + t]), a1 = to_tf32(a[(g + 8) * lda + k0 + t]);
+        const uint32_t a2 = to_tf32(a[g * lda + k0 + t + 4]), a3 = to_tf32(a[(g + 8) * lda + k0 + t + 4]);
+        const uint32_t b0 = to_tf32(b[(k0 + t) * ldb + g]), b1 = to_tf32(b[(k0 + t + 4) * ldb + g]);
+        asm volatile(
+            "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
+            "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    }
+}
+// store a D fragment (times `s`) to fp32 rows `ld` apart
+__device__ __forceinline__ void st_tile_f32(float* d, int ld, const float c[4], float s, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    *reinterpret_cast<float2*>(d + g * ld + 2 * t) = make_float2(s * c[0], s * c[1]);
+    *reinterpret_cast<float2*>(d + (g + 8) * ld + 2 * t) = make_float2(s * c[2], s * c[3]);
+}
+// store -D diag(beta) as bf16 T' (K-major, 64 x 64) at rows r0.., columns n0..
+__device__ __forceinline__ void st_tile_tb(uint8_t* sTB, int r0, int n0, const float c[4],
+                                           const float* sb, int lane) {
+    const int g = lane >> 2, t = lane & 3, n = n0 + 2 * t;
+    const float b0 = sb[n], b1 = sb[n + 1];
+    *reinterpret_cast<uint32_t*>(sTB + tc::sw128_kmajor(r0 + g, n, 64)) = pack_bf16(-c[0] * b0, -c[1] * b1);
+    *reinterpret_cast<uint32_t*>(sTB + tc::sw128_kmajor(r0 + g + 8, n, 64)) = pack_bf16(-c[2] * b0, -c[3] * b1);
 }
 
 // T = (I + A)^-1 for the strictly lower-triangular 64 x 64 A (fp32), by block doubling over
 // 16 x 16 blocks T_IJ (I, J = 0..3):
-//   phase 0  diagonal blocks T_JJ by forward substitution;
+//   phase 0  diagonal blocks T_JJ by forward substitution (fp32, CUDA cores);
 //   phase 1  X0 = A_10 T_00,  X1 = A_32 T_22,  Y = [A_{[2:4],0} T_00 | A_{[2:4],1} T_11];
 //   phase 2  T_10 = -T_11 X0,  T_32 = -T_33 X1,  Y_left -= Y_right X0
 //            (then Y = A_{[2:4],[0:2]} T_{[0:2],[0:2]}, since T_10 = -T_11 X0);
 //   phase 3  T_{[2:4],[0:2]} = -T_{[2:4],[2:4]} Y.
 // Each finished block is also written as T' = T diag(beta) in bf16 (K-major, 64 x 64), the A
-// operand of the W and U~ products.  A thread owns a 1 x 4 output tile; operands are read as
-// float4 (rows of A and T at a stride of 68 floats, of Y at 36: no bank conflicts).
-constexpr int kStrideY = 36;
+// operand of the W and U~ products.  Phases 1-3 are 12, 8 and 8 warp tiles of 16 x 8 outputs.
+// Strides keep the fragment loads free of bank conflicts: A and T rows 68 floats apart (A-side),
+// X0, X1 rows 24 apart and Y rows 40 apart (B-side).
+constexpr int kStrideX = 24, kStrideY = 40;
 __device__ __forceinline__ void t_solve(const float* sA, float* sT, const float* sb, uint8_t* sTB,
                                         float* sX, float* sY, int tid) {
-    float* sX0 = sX;         // [16][16]
-    float* sX1 = sX + 256;   // [16][16]
+    float* sX0 = sX;                    // [16][24]
+    float* sX1 = sX + 16 * kStrideX;    // [16][24]
+    const int warp = tid >> 5, lane = tid & 31;
     // ---- phase 0: diagonal blocks (threads 0..63: block J = tid / 16, column l = tid % 16);
     // the others zero block (2,3) of T and the blocks of T' above the diagonal
     if (tid < 64) {
@@ -251,51 +273,56 @@ __device__ __forceinline__ void t_solve(const float* sA, float* sT, const float*
         }
     }
     __syncthreads();
-    // ---- phase 1: 96 output rows x 4 column quads (threads 0..383)
-    if (tid < 384) {
-        const int ri = tid >> 2, c0 = 4 * (tid & 3);
-        if (ri < 48) {            // [X0; Y_left] = A_{[1:4],0} T_00
-            const int row = 16 + ri;
-            const float4 x = row_x_cols4<16>(sA + row * kStrideA, sT + c0, kStrideA);
-            float* dst = ri < 16 ? sX0 + ri * 16 + c0 : sY + (ri - 16) * kStrideY + c0;
-            *reinterpret_cast<float4*>(dst) = x;
-        } else if (ri < 80) {     // Y_right = A_{[2:4],1} T_11
-            const int i = ri - 48;
-            const float4 x = row_x_cols4<16>(sA + (32 + i) * kStrideA + 16, sT + 16 * kStrideA + 16 + c0, kStrideA);
-            *reinterpret_cast<float4*>(sY + i * kStrideY + 16 + c0) = x;
+    // ---- phase 1: 12 tiles (warps 0..11)
+    if (warp < 12) {
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        const int n = 8 * (warp & 1);
+        if (warp < 6) {           // [X0; Y_left] = A_{[1:4],0} T_00: row tiles 16, 32, 48
+            const int m = 16 + 16 * (warp >> 1);
+            mma_tile_tf32<16>(c, sA + m * kStrideA, kStrideA, sT + n, kStrideA, lane);
+            if (m == 16) st_tile_f32(sX0 + n, kStrideX, c, 1.f, lane);
+            else st_tile_f32(sY + (m - 32) * kStrideY + n, kStrideY, c, 1.f, lane);
+        } else if (warp < 10) {   // Y_right = A_{[2:4],1} T_11: row tiles 32, 48
+            const int m = 32 + 16 * ((warp - 6) >> 1);
+            mma_tile_tf32<16>(c, sA + m * kStrideA + 16, kStrideA, sT + 16 * kStrideA + 16 + n, kStrideA, lane);
+            st_tile_f32(sY + (m - 32) * kStrideY + 16 + n, kStrideY, c, 1.f, lane);
         } else {                  // X1 = A_32 T_22
-            const int i = ri - 80;
-            const float4 x = row_x_cols4<16>(sA + (48 + i) * kStrideA + 32, sT + 32 * kStrideA + 32 + c0, kStrideA);
-            *reinterpret_cast<float4*>(sX1 + i * 16 + c0) = x;
+            mma_tile_tf32<16>(c, sA + 48 * kStrideA + 32, kStrideA, sT + 32 * kStrideA + 32 + n, kStrideA, lane);
+            st_tile_f32(sX1 + n, kStrideX, c, 1.f, lane);
         }
     }
     __syncthreads();
-    // ---- phase 2: 64 output rows x 4 column quads (threads 0..255)
-    if (tid < 256) {
-        const int ri = tid >> 2, c0 = 4 * (tid & 3);
-        if (ri < 16) {            // T_10 = -T_11 X0
-            const float4 x = row_x_cols4<16>(sT + (16 + ri) * kStrideA + 16, sX0 + c0, 16);
-            st_tb4(sTB, 16 + ri, c0, make_float4(-x.x, -x.y, -x.z, -x.w), sb);   // T' only
-        } else if (ri < 32) {     // T_32 = -T_33 X1
-            const int i = ri - 16;
-            const float4 x = row_x_cols4<16>(sT + (48 + i) * kStrideA + 48, sX1 + c0, 16);
-            const float4 t = make_float4(-x.x, -x.y, -x.z, -x.w);
-            *reinterpret_cast<float4*>(sT + (48 + i) * kStrideA + 32 + c0) = t;
-            st_tb4(sTB, 48 + i, 32 + c0, t, sb);
-        } else {                  // Y_left -= Y_right X0
-            const int i = ri - 32;
-            const float4 x = row_x_cols4<16>(sY + i * kStrideY + 16, sX0 + c0, 16);
-            float4* y = reinterpret_cast<float4*>(sY + i * kStrideY + c0);
-            const float4 z = *y;
-            *y = make_float4(z.x - x.x, z.y - x.y, z.z - x.z, z.w - x.w);
+    // ---- phase 2: 8 tiles (warps 0..7)
+    if (warp < 8) {
+        const int n = 8 * (warp & 1);
+        if (warp < 2) {           // T_10 = -T_11 X0 (T' only)
+            float c[4] = {0.f, 0.f, 0.f, 0.f};
+            mma_tile_tf32<16>(c, sT + 16 * kStrideA + 16, kStrideA, sX0 + n, kStrideX, lane);
+            st_tile_tb(sTB, 16, n, c, sb, lane);
+        } else if (warp < 4) {    // T_32 = -T_33 X1 (T and T')
+            float c[4] = {0.f, 0.f, 0.f, 0.f};
+            mma_tile_tf32<16>(c, sT + 48 * kStrideA + 48, kStrideA, sX1 + n, kStrideX, lane);
+            st_tile_f32(sT + 48 * kStrideA + 32 + n, kStrideA, c, -1.f, lane);
+            st_tile_tb(sTB, 48, 32 + n, c, sb, lane);
+        } else {                  // Y_left -= Y_right X0: row tiles 0, 16 of Y
+            const int m = 16 * ((warp - 4) >> 1);
+            const int g = lane >> 2, t = lane & 3;
+            float* y = sY + m * kStrideY + n;
+            float c[4] = {0.f, 0.f, 0.f, 0.f};
+            mma_tile_tf32<16>(c, sY + m * kStrideY + 16, kStrideY, sX0 + n, kStrideX, lane);
+            const float2 y0 = *reinterpret_cast<const float2*>(y + g * kStrideY + 2 * t);
+            const float2 y1 = *reinterpret_cast<const float2*>(y + (g + 8) * kStrideY + 2 * t);
+            const float d[4] = {y0.x - c[0], y0.y - c[1], y1.x - c[2], y1.y - c[3]};
+            st_tile_f32(y, kStrideY, d, 1.f, lane);
         }
     }
     __syncthreads();
-    // ---- phase 3: T_{[2:4],[0:2]} = -T_{[2:4],[2:4]} Y, 32 rows x 8 column quads (threads 0..255)
-    if (tid < 256) {
-        const int i = tid >> 3, c0 = 4 * (tid & 7);
-        const float4 x = row_x_cols4<32>(sT + (32 + i) * kStrideA + 32, sY + c0, kStrideY);
-        st_tb4(sTB, 32 + i, c0, make_float4(-x.x, -x.y, -x.z, -x.w), sb);
+    // ---- phase 3: T_{[2:4],[0:2]} = -T_{[2:4],[2:4]} Y, 8 tiles (warps 0..7), T' only
+    if (warp < 8) {
+        const int m = 16 * (warp >> 2), n = 8 * (warp & 3);
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_tile_tf32<32>(c, sT + (32 + m) * kStrideA + 32, kStrideA, sY + n, kStrideY, lane);
+        st_tile_tb(sTB, 32 + m, n, c, sb, lane);
     }
 }
 
@@ -737,7 +764,8 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const float* __restrict__ alp
 //   warp 7      output issue: D_o = Q' S (M = 64, N = 32)
 //   warps 8-11  output epilogue: O = scale (D_o + O_loc), rows in the M = 64 layout
 // Only the first three roles are on the serial path; the output side runs behind it and never
-// holds a chain stage.  S rotates through four shared-memory buffers: S_{c+4} is written only
+// holds a chain stage: the output product of chunk c is issued when the chain product of chunk c
+// has completed, i.e. while the chain epilogue forms S_{c+1}.  S rotates through four shared-memory buffers: S_{c+4} is written only
 // after the output product of chunk c has read S_c.  Every role issues from a converged warp
 // (one elected lane) and every wait is bounded and ends warp-uniformly.
 constexpr int kStages = 3;
@@ -773,8 +801,8 @@ ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
     uint64_t* s_ready = mma_c + 1;                               // [kSBufs] S buffer written
     uint64_t* mma_o = s_ready + kSBufs;                          // [kOutBufs] D_o complete
     uint64_t* o_free = mma_o + kOutBufs;                         // [kOutBufs] D_o read back
-    uint64_t* dc_issued = o_free + kOutBufs;                     // [kSBufs] D_c(c) issued
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(dc_issued + kSBufs);
+    uint64_t* dc_done = o_free + kOutBufs;                       // [kSBufs] D_c(c) complete
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(dc_done + kSBufs);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -797,7 +825,7 @@ ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
         tc::mbar_init(mma_c, 1);
         for (int s = 0; s < kSBufs; ++s) {
             tc::mbar_init(&s_ready[s], 4);
-            tc::mbar_init(&dc_issued[s], 1);
+            tc::mbar_init(&dc_done[s], 1);
         }
         for (int s = 0; s < kOutBufs; ++s) {
             tc::mbar_init(&mma_o[s], 1);
@@ -859,6 +887,7 @@ ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
                 !wait(&mma_o[(ch - 3) % kOutBufs], ((ch - 3) / kOutBufs) & 1))
                 break;
             if (!wait(mma_c, ch & 1)) break;
+            if (tid == 0) tc::mbar_arrive(&dc_done[ch % kSBufs]);   // the output product may run
             tc::tc_fence_after();
             float d[32];
             tc::tmem_ld32_sync(tc::tmem_addr(dc, 32 * warp, 0), d);
@@ -897,8 +926,6 @@ ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
                 tc::mma_bf16_warp(dc, tc::desc_add(ad, (ks >> 2) * 16384 + (ks & 3) * 32),
                                   tc::desc_add(sd, ks * 2048), idc, ks > 0 ? 1u : 0u);
             tc::mma_commit_warp(mma_c);
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&dc_issued[ch % kSBufs]);   // D_o(ch) may follow it
         }
     } else if (warp == 5 || warp == 6) {
         // ---- loads: warp 5 the chain ring (A_c, B_c), warp 6 the output ring (Q', O_loc) ----
@@ -940,8 +967,9 @@ ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
         for (int ch = 0; ch < NT; ++ch) {
             const int st = ch % kStages, ob = ch % kOutBufs;
             if (!wait(&full_o[st], (ch / kStages) & 1)) break;
-            // issued right behind D_c(ch), so it runs while the chain epilogue works
-            if (!wait(&dc_issued[ch % kSBufs], (ch / kSBufs) & 1)) break;
+            // issued once D_c(ch) has completed, so it runs while the chain epilogue works and
+            // never shares the tensor pipe with a chain product
+            if (!wait(&dc_done[ch % kSBufs], (ch / kSBufs) & 1)) break;
             if (ch >= kOutBufs && !wait(&o_free[ob], ((ch / kOutBufs) - 1) & 1)) break;
             tc::tc_fence_after();
             const uint64_t qd = tc::desc_add(o_desc0, st * P2_OSTAGE + P2_QP);

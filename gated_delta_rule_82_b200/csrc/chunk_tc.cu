@@ -60,6 +60,9 @@ constexpr int kC = 64, kDK = 128, kDV = 128, kDVT = 32, kNTile = kDV / kDVT;
 constexpr uint32_t WS_AC = 0;          // A_c bf16, K-major swizzled, 128 rows x 128
 constexpr uint32_t WS_QP = 32768;      // Q'  bf16, K-major swizzled, 64 rows x 128
 constexpr uint32_t WS_TILES = 49152;   // per dv tile t: B_c [128][32] bf16, then O_loc [64][32] bf16
+// Both tile images have 64-byte rows whose four 16-byte chunks are swizzled by row, so that the
+// lanes of a warp reading (or writing) one chunk of 8 consecutive rows hit distinct banks.
+__host__ __device__ constexpr uint32_t bc_chunk(int row, int j) { return (uint32_t)((j ^ ((row >> 1) & 3)) << 4); }
 constexpr uint32_t WS_TILE = 12288;
 constexpr uint32_t WS_TILE_O = 8192;
 constexpr uint32_t WS_CHUNK = WS_TILES + kNTile * WS_TILE;  // 98304
@@ -75,8 +78,8 @@ constexpr uint32_t S_KE = 131072;    // K_end (MN-major, 64 x 128): the MN-major
 constexpr uint32_t S_M = 147456;     // M bf16 K-major 64 x 64
 constexpr uint32_t S_A = 155648;     // A fp32 [64][68]
 constexpr uint32_t S_T = 173056;     // T fp32 [64][68]
-constexpr uint32_t S_W = 190464;     // W MN-major 64 x 128   (exact path: log2 prefix fp32 [64][128]
-constexpr uint32_t S_U = 206848;     // U~ MN-major 64 x 128   spanning S_W and S_U)
+constexpr uint32_t S_W = 190464;     // W^T K-major 128 x 64  (exact path: log2 prefix fp32 [64][128]
+constexpr uint32_t S_U = 206848;     // U~^T K-major 128 x 64  spanning S_W and S_U)
 constexpr uint32_t S_SM = 223232;    // small arrays (below)
 constexpr uint32_t S_BYTES = S_SM + 3072 + 1024;
 constexpr int kStrideA = 68;         // fp32 row stride of A and T
@@ -351,6 +354,7 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const float* __restrict__ alp
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const size_t rs = (size_t)H;   // stride between tokens, in rows of [B*T*H]
+    tc::grid_launch_dependents();   // the state pass may start its set-up early
 
     if (warp == 0) {
         tc::tmem_alloc(tmem_slot, 512);
@@ -617,20 +621,22 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const float* __restrict__ alp
         __syncthreads();
         tc::tc_fence_after();
 
-        // ======== D: W = T' K_gamma, U~ = T' V  (M = 64, N = 128 each, K = 64) ========
-        // K_gamma is rows 0..63 of L, read as an MN-major operand: 64-column blocks 16 KB apart.
+        // ======== D: W^T = K_gamma^T T'^T, U~^T = V^T T'^T  (M = 128, N = 64 each, K = 64) ========
+        // The transposed products put a channel (or dv column) in every TMEM lane.  K_gamma^T is
+        // rows 0..63 of L read as an MN-major A operand (64-channel blocks 16 KB apart), V^T the
+        // TMA-swizzled V tile (blocks 8 KB apart); T'^T is T' itself as a K-major B operand.
         if (warp == 0) {
             tc::mbar_wait(bar_v, it & 1, abort_flag);
             __syncwarp();
-            const uint64_t ad = tc::smem_desc_sw128(tc::smem_u32(sm + S_TB), 16, 1024);
+            const uint64_t bd = tc::smem_desc_sw128(tc::smem_u32(sm + S_TB), 16, 1024);
             const uint64_t kd = tc::smem_desc_sw128(tc::smem_u32(sL), 16384, 1024);
             const uint64_t vd = tc::smem_desc_sw128(tc::smem_u32(sm + S_V), 8192, 1024);
-            const uint32_t idesc = tc::idesc_bf16_f32(64, 128, 0, 1);
+            const uint32_t idesc = tc::idesc_bf16_f32(128, 64, 1, 0);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t a = tc::desc_add(ad, ks * 32);
-                tc::mma_bf16_warp(tmem, a, tc::desc_add(kd, ks * 2048), idesc, ks > 0);
-                tc::mma_bf16_warp(tmem + 128, a, tc::desc_add(vd, ks * 2048), idesc, ks > 0);
+                const uint64_t b = tc::desc_add(bd, ks * 32);
+                tc::mma_bf16_warp(tmem, tc::desc_add(kd, ks * 2048), b, idesc, ks > 0);
+                tc::mma_bf16_warp(tmem + 64, tc::desc_add(vd, ks * 2048), b, idesc, ks > 0);
             }
             tc::mma_commit_warp(bar);
         }
@@ -640,78 +646,89 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const float* __restrict__ alp
         // V of this chunk-head is consumed: bring in the next one's
         if (tid == 0 && nci < total) issue_v(maps, sm, bar_v, nci, NT, H);
         {
-            // warp w: rows 16 (w % 4) + lane (lane < 16); 64-column slice w / 4:
-            // slices 0, 1 -> W columns 0..127, slices 2, 3 -> U~ columns 0..127
+            // warp w: lanes 32 (w % 4) .. (channel, or dv column, c); 32-column slice w / 4:
+            // slices 0, 1 -> W^T tokens 0..63, slices 2, 3 -> U~^T tokens 0..63.  Both tiles are
+            // K-major (rows c, K = token): the B operand of M W, K_end^T W and K_end^T U~, and the
+            // A operand of U~^T M^T.
             const int quarter = warp & 3, slice = warp >> 2;
-            const int r = 16 * quarter + (lane & 15);
+            const int c = 32 * quarter + lane;
             uint8_t* dst = sm + (slice < 2 ? S_W : S_U);
-            const int n0 = 64 * (slice & 1);
-            float x[64];
-            tc::tmem_ld64_sync(tc::tmem_addr(tmem, 32 * quarter, 64 * slice), x);
-            if (lane < 16) {
+            const int j0 = 32 * (slice & 1);
+            float x[32];
+            tc::tmem_ld32_sync(tc::tmem_addr(tmem, 32 * quarter, 32 * slice), x);
 #pragma unroll
-                for (int c0 = 0; c0 < 64; c0 += 8) st16(dst, tc::sw128_mnmajor(r, n0 + c0, 64), x + c0);
-            }
+            for (int i = 0; i < 32; i += 8) st16(dst, tc::sw128_kmajor(c, j0 + i, 128), x + i);
         }
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
         __syncthreads();
         tc::tc_fence_after();
 
-        // ======== F: M [W | U~] (M = 64) and K_end^T [W | U~] (M = 128, MN-major A) ========
+        // ======== F: M W (M = 64) -> Q', U~^T M^T (M = 128) -> O_loc^T,
+        //             K_end^T W (M = 128) -> A_c, K_end^T U~ (M = 128) -> B_c ========
         if (warp == 0) {
             const uint64_t md = tc::smem_desc_sw128(tc::smem_u32(sm + S_M), 16, 1024);
             const uint64_t ked = tc::smem_desc_sw128(tc::smem_u32(sm + S_KE), 8192, 1024);
-            const uint64_t wd = tc::smem_desc_sw128(tc::smem_u32(sm + S_W), 8192, 1024);
-            const uint64_t ud = tc::smem_desc_sw128(tc::smem_u32(sm + S_U), 8192, 1024);
-            const uint32_t id64 = tc::idesc_bf16_f32(64, 128, 0, 1);
-            const uint32_t id128 = tc::idesc_bf16_f32(128, 128, 1, 1);
+            const uint64_t wd = tc::smem_desc_sw128(tc::smem_u32(sm + S_W), 16, 1024);
+            const uint64_t ud = tc::smem_desc_sw128(tc::smem_u32(sm + S_U), 16, 1024);
+            const uint32_t id_q = tc::idesc_bf16_f32(64, 128, 0, 0);
+            const uint32_t id_o = tc::idesc_bf16_f32(128, 64, 0, 0);
+            const uint32_t id_c = tc::idesc_bf16_f32(128, 128, 1, 0);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t bw = tc::desc_add(wd, ks * 2048), bu = tc::desc_add(ud, ks * 2048);
-                const uint64_t adm = tc::desc_add(md, ks * 32), ade = tc::desc_add(ked, ks * 2048);
-                tc::mma_bf16_warp(tmem, adm, bw, id64, ks > 0);
-                tc::mma_bf16_warp(tmem + 128, adm, bu, id64, ks > 0);
-                tc::mma_bf16_warp(tmem + 256, ade, bw, id128, ks > 0);
-                tc::mma_bf16_warp(tmem + 384, ade, bu, id128, ks > 0);
+                const uint64_t w = tc::desc_add(wd, ks * 32), u = tc::desc_add(ud, ks * 32);
+                const uint64_t m = tc::desc_add(md, ks * 32), ke = tc::desc_add(ked, ks * 2048);
+                tc::mma_bf16_warp(tmem, m, w, id_q, ks > 0);               // M W
+                tc::mma_bf16_warp(tmem + 128, u, m, id_o, ks > 0);         // U~^T M^T
+                tc::mma_bf16_warp(tmem + 192, ke, w, id_c, ks > 0);        // K_end^T W
+                tc::mma_bf16_warp(tmem + 320, ke, u, id_c, ks > 0);        // K_end^T U~
             }
             tc::mma_commit_warp(bar);
         }
         tc::mbar_wait(bar, phase & 1, abort_flag);
         ++phase;
         tc::tc_fence_after();
-        // ======== G: results into shared staging images, then three bulk stores ========
+        // ======== G: results into shared staging images, then bulk stores in two groups ========
         {
             const int quarter = warp & 3, slice = warp >> 2;
-            // (1) M = 64 products: rows 16 quarter + lane; slices 0, 1 -> Q', 2, 3 -> O_loc
+            // (1) Q' = Q_gamma - M W (M = 64 layout): rows 16 quarter + lane, 32-column slice
             {
                 const int r = 16 * quarter + (lane & 15);
-                const int n0 = 64 * (slice & 1);
-                float x[64];
-                tc::tmem_ld64_sync(tc::tmem_addr(tmem, 32 * quarter, 64 * slice), x);
+                float x[32];
+                tc::tmem_ld32_sync(tc::tmem_addr(tmem, 32 * quarter, 32 * slice), x);
                 if (lane < 16) {
 #pragma unroll
-                    for (int c0 = 0; c0 < 64; c0 += 8) {
-                        const int n = n0 + c0;
-                        if (slice < 2) {
-                            float qg[8];
-                            unpack8(*reinterpret_cast<const uint4*>(sL + tc::sw128_kmajor(64 + r, n, 128)), qg);
+                    for (int c0 = 0; c0 < 32; c0 += 8) {
+                        const int n = 32 * slice + c0;
+                        float qg[8];
+                        unpack8(*reinterpret_cast<const uint4*>(sL + tc::sw128_kmajor(64 + r, n, 128)), qg);
 #pragma unroll
-                            for (int i = 0; i < 8; ++i) qg[i] -= x[c0 + i];
-                            st16(sm + S_OUT_QP, tc::sw128_kmajor(r, n, 64), qg);
-                        } else {
-                            st16(sm + S_OUT_TL, (n >> 5) * WS_TILE + WS_TILE_O + (r * 32 + (n & 31)) * 2, x + c0);
-                        }
+                        for (int i = 0; i < 8; ++i) qg[i] -= x[c0 + i];
+                        st16(sm + S_OUT_QP, tc::sw128_kmajor(r, n, 64), qg);
                     }
                 }
             }
-            // (2) M = 128 products: row c' = 32 quarter + lane; slices 0, 1 -> A_c, 2, 3 -> B_c
+            // (2) M = 128 products, lane = row c' (A_c, B_c) or dv column (O_loc^T)
             {
                 const int cr = 32 * quarter + lane;
+                // O_loc^T: tokens 16 slice .. 16 slice + 15 of dv column cr -> tile cr / 32, stored
+                // as O_loc rows [64 tokens][32 dv] (the lanes of a warp fill 64 contiguous bytes of
+                // one token row per store)
+                {
+                    float x[16];
+                    tc::tmem_ld16_sync(tc::tmem_addr(tmem, 32 * quarter, 128 + 16 * slice), x);
+                    const int nc = cr & 31;
+                    uint8_t* o = sm + S_OUT_TL + (cr >> 5) * WS_TILE + WS_TILE_O + (nc & 7) * 2;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int r = 16 * slice + i;
+                        st_bf16(o, r * 64 + bc_chunk(r, nc >> 3), x[i]);
+                    }
+                }
                 const int n0 = 64 * (slice & 1);
                 const float gc = gGC[cr];
                 float x[64];
-                tc::tmem_ld64_sync(tc::tmem_addr(tmem, 32 * quarter, 256 + 64 * slice), x);
+                tc::tmem_ld64_sync(tc::tmem_addr(tmem, 32 * quarter, (slice < 2 ? 192 : 320) + n0), x);
 #pragma unroll
                 for (int c0 = 0; c0 < 64; c0 += 8) {
                     const int n = n0 + c0;
@@ -721,7 +738,7 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const float* __restrict__ alp
                         for (int i = 0; i < 8; ++i) y[i] = -x[c0 + i];
                         st16(sm + S_OUT_AC, tc::sw128_kmajor(cr, n, 128), y);
                     } else {
-                        st16(sm + S_OUT_TL, (n >> 5) * WS_TILE + (cr * 32 + (n & 31)) * 2, x + c0);
+                        st16(sm + S_OUT_TL, (n >> 5) * WS_TILE + cr * 64 + bc_chunk(cr, (n & 31) >> 3), x + c0);
                     }
                 }
                 // A_c = Diag(gamma_C) - K_end^T W: row c' holds its diagonal element in this slice
@@ -837,6 +854,9 @@ ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
+    // set-up above may overlap the factor kernel's tail; everything below reads its workspace
+    // or touches caller memory, so it waits for that grid to complete
+    tc::grid_dependency_wait();
     const uint32_t tmem = *tmem_slot;
     const uint32_t dc = tmem;                 // D_c: 128 lanes x 32 columns
     const uint32_t dob = tmem + 32;           // D_o: kOutBufs buffers of 32 columns (M = 64 layout)
@@ -880,7 +900,7 @@ ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
             uint4 bc[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-                bc[j] = reinterpret_cast<const uint4*>(sm + st * P2_CSTAGE + P2_BC + t * 64)[j];
+                bc[j] = *reinterpret_cast<const uint4*>(sm + st * P2_CSTAGE + P2_BC + t * 64 + bc_chunk(t, j));
             // buffer (ch + 1) % 4 last held S_{ch-3}: its output product must be done (checked
             // before the chain product completes, off the serial path)
             if (ch + 1 < NT && ch + 1 >= kSBufs &&
@@ -998,12 +1018,11 @@ ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
                 const int r = 16 * q4 + lane;
                 const int t0 = ch * kC;
                 if (t0 + r < T_len) {
-                    const uint4* ol = reinterpret_cast<const uint4*>(stg + P2_OL + r * 64);
                     uint4* dst = reinterpret_cast<uint4*>(out + (((size_t)b * T_len + t0 + r) * H + h) * kDV + n0);
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         float y[8];
-                        unpack8(ol[j], y);
+                        unpack8(*reinterpret_cast<const uint4*>(stg + P2_OL + r * 64 + bc_chunk(r, j)), y);
 #pragma unroll
                         for (int i = 0; i < 8; ++i) y[i] = scale * (d[8 * j + i] + y[i]);
                         dst[j] = pack8(y);
@@ -1092,9 +1111,21 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const f
         if (e != cudaSuccess) return e;
     }
     if (stages & 2) {
-        ckda_tc_state<<<(unsigned)(kNTile * B * H), kStateThreads, P2_BYTES, stream>>>(
-            ws, h0, static_cast<__nv_bfloat16*>(out), hT, T_len, H, NT, scale);
-        e = cudaGetLastError();
+        // programmatic dependent launch: the state pass is scheduled while the factor kernel
+        // finishes, and waits for it (griddepcontrol.wait) before reading the workspace
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(kNTile * B * H));
+        cfg.blockDim = dim3(kStateThreads);
+        cfg.dynamicSmemBytes = P2_BYTES;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        __nv_bfloat16* outb = static_cast<__nv_bfloat16*>(out);
+        e = cudaLaunchKernelEx(&cfg, ckda_tc_state, static_cast<const uint8_t*>(ws), h0, outb, hT,
+                               T_len, H, NT, scale);
     }
     return e;
 }

@@ -113,6 +113,17 @@ __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
+// ---- programmatic dependent launch ----------------------------------------------------------
+// Let the next kernel in the stream (launched with programmatic stream serialisation) start its
+// prologue while this grid is still running.
+__device__ __forceinline__ void grid_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Wait until the preceding grid has completed and its memory operations are visible.
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ---- Tensor Memory ---------------------------------------------------------------------------
 // Whole-warp operations.  ncols: power of two >= 32.
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {

@@ -372,6 +372,9 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const float* __restrict__ alp
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     uint32_t phase = 0;   // completions of `bar` so far
+    // the set-up above may overlap the previous kernel in the stream; from here on the kernel
+    // reads the caller's inputs and writes the workspace, so it waits for that kernel
+    tc::grid_dependency_wait();
     if (tid == 0 && (int)blockIdx.x < total) {
         tc::prefetch_tensormap(&maps.q);
         tc::prefetch_tensormap(&maps.k);
@@ -857,6 +860,7 @@ ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
     // set-up above may overlap the factor kernel's tail; everything below reads its workspace
     // or touches caller memory, so it waits for that grid to complete
     tc::grid_dependency_wait();
+    tc::grid_launch_dependents();   // a following kernel may start its set-up early
     const uint32_t tmem = *tmem_slot;
     const uint32_t dc = tmem;                 // D_c: 128 lanes x 32 columns
     const uint32_t dob = tmem + 32;           // D_o: kOutBufs buffers of 32 columns (M = 64 layout)
@@ -1105,9 +1109,20 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const f
             !encode_map(&maps.alpha, alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kDK, kDK, H, T_len,
                         B, CU_TENSOR_MAP_SWIZZLE_NONE))
             return cudaErrorInvalidValue;
-        ckda_tc_intra<<<(unsigned)grid, 512, S_BYTES, stream>>>(maps, alpha, beta, ws, T_len, H, NT,
-                                                                total, l2norm, rp, pos_offset);
-        e = cudaGetLastError();
+        // programmatic dependent launch: CTAs may start their set-up on SMs the previous kernel
+        // has left, and wait (griddepcontrol.wait) for it before touching memory
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)grid);
+        cfg.blockDim = dim3(512);
+        cfg.dynamicSmemBytes = S_BYTES;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, ckda_tc_intra, maps, alpha, beta, ws, T_len, H, NT, total,
+                               l2norm, rp, pos_offset);
         if (e != cudaSuccess) return e;
     }
     if (stages & 2) {

@@ -61,6 +61,8 @@ def _load(mutant: int = 0) -> ctypes.CDLL:
         lib.ckda_oracle_prologue.argtypes = [D, D] + [ctypes.c_int] * 5 + [
             ctypes.c_double, ctypes.c_int, ctypes.c_longlong]
         lib.ckda_oracle_mutant.restype = ctypes.c_int
+        lib.ckda_oracle_gates.restype = ctypes.c_int
+        lib.ckda_oracle_gates.argtypes = [D, D, ctypes.c_longlong, D, D, ctypes.c_longlong]
         _libs[mutant] = lib
         return lib
 
@@ -108,6 +110,20 @@ def fwd(q, k, v, alpha, beta, h0=None, *, l2norm=True, rope_theta=0.0, rope_conv
     if rc != 0:
         raise RuntimeError(f"ckda_oracle_fwd failed with code {rc}")
     return out, hT
+
+
+def gates(a=None, b=None, *, mutant=0):
+    """Gates from logits, float64: alpha = 2 sigma(a) - 1 (same shape as a), beta = 2 sigma(b).
+    Returns (alpha or None, beta or None)."""
+    aa = None if a is None else _f64(a)
+    ba = None if b is None else _f64(b)
+    al = None if aa is None else np.empty_like(aa)
+    be = None if ba is None else np.empty_like(ba)
+    rc = _load(mutant).ckda_oracle_gates(_ptr(aa), _ptr(al), 0 if aa is None else aa.size,
+                                         _ptr(ba), _ptr(be), 0 if ba is None else ba.size)
+    if rc != 0:
+        raise RuntimeError(f"ckda_oracle_gates failed with code {rc}")
+    return al, be
 
 
 def decode(q, k, v, alpha, beta, state, pos=None, *, l2norm=True, rope_theta=0.0,

@@ -35,6 +35,10 @@
  *  - the output reads S_t, after the update.
  *  - RoPE position p = pos_offset + t, 0-based.
  *
+ * Gate activation (optional input form): the "Complex KDA" paper summary, Methodology, "CKDA
+ * Definition", parameterises the gates from unconstrained logits as beta_t = 2 sigma(b_t) and the
+ * signed gates alpha_{t,i} = 2 sigma(a_{t,i}) - 1, sigma the logistic function.
+ *
  * Planted mistakes (CKDA_ORACLE_MUTANT=n at compile time) exist only so that the test suite can
  * prove its pins catch each class of error; the default build (0) is the oracle.
  */
@@ -58,12 +62,36 @@
 #define MUT_THETA_1000 8    /* rope base 1000 instead of the given one */
 #define MUT_NO_L2 9         /* skip the L2 norm */
 #define MUT_NORM_AFTER 10   /* L2 norm over q and k jointly instead of per vector */
+#define MUT_GATE_NO_AFFINE 11 /* alpha = sigma(a), the sigmoid without its 2x - 1 map */
+#define MUT_BETA_NO2 12     /* beta = sigma(b), without the factor 2 */
 
 #define L2_EPS 1e-6
 
 static const int g_mutant = CKDA_ORACLE_MUTANT;
 
 int ckda_oracle_mutant(void) { return g_mutant; }
+
+/* logistic function, evaluated on the side where exp() cannot overflow */
+static double logistic(double x) {
+    if (x >= 0.0) return 1.0 / (1.0 + exp(-x));
+    double e = exp(x);
+    return e / (1.0 + e);
+}
+
+/*
+ * Gates from logits: alpha[i] = 2 sigma(a[i]) - 1 for i < na, beta[j] = 2 sigma(b[j]) for j < nb
+ * ("Complex KDA" paper summary, Methodology, CKDA Definition).  Either pair may be null.
+ */
+int ckda_oracle_gates(const double* a, double* alpha, long long na, const double* b, double* beta,
+                      long long nb) {
+    if (a && alpha)
+        for (long long i = 0; i < na; ++i)
+            alpha[i] = g_mutant == MUT_GATE_NO_AFFINE ? logistic(a[i]) : 2.0 * logistic(a[i]) - 1.0;
+    if (b && beta)
+        for (long long j = 0; j < nb; ++j)
+            beta[j] = g_mutant == MUT_BETA_NO2 ? logistic(b[j]) : 2.0 * logistic(b[j]);
+    return 0;
+}
 
 /* Rotate one head vector x[0..d) in place by position p (see header comment for the pairing). */
 static void rope_rotate(double* x, int d, long long p, double theta, int convention) {

@@ -360,7 +360,29 @@ def pin_decode_matches_fwd(mutant=0):
     assert np.allclose(s2, hT, atol=1e-13)
 
 
+def pin_gate_activation(mutant=0):
+    """Gates from logits ("Complex KDA" paper summary, Methodology, CKDA Definition: beta = 2 sigma(b),
+    signed alpha = 2 sigma(a) - 1), against facts outside the oracle: the identities
+    2 sigma(x) - 1 = tanh(x / 2) and 2 sigma(x) = 1 + tanh(x / 2) (numpy's tanh, another formula),
+    the values at 0, the odd / complementary symmetries and the ranges [-1, 1] and [0, 2] at the
+    ends."""
+    rng = np.random.default_rng(5)
+    a = np.concatenate([rng.normal(0.0, 3.0, 500), [0.0, -0.0, 1e-8, -1e-8, 40.0, -40.0, 745.0, -745.0]])
+    b = rng.normal(0.0, 3.0, 200)
+    al, be = oracle.gates(a, b, mutant=mutant)
+    assert np.allclose(al, np.tanh(a / 2.0), rtol=1e-14, atol=1e-15), "alpha = tanh(a/2)"
+    assert np.allclose(be, 1.0 + np.tanh(b / 2.0), rtol=1e-14, atol=1e-15), "beta = 1 + tanh(b/2)"
+    a0, b0 = oracle.gates(np.zeros(3), np.zeros(3), mutant=mutant)
+    assert np.all(a0 == 0.0) and np.all(b0 == 1.0), "alpha(0) = 0, beta(0) = 1"
+    am, bm = oracle.gates(-a, -b, mutant=mutant)
+    assert np.allclose(am, -al, rtol=0, atol=1e-15), "alpha odd"
+    assert np.allclose(bm + be, 2.0, rtol=0, atol=1e-15), "beta(b) + beta(-b) = 2"
+    ends, bends = oracle.gates(np.array([800.0, -800.0]), np.array([800.0, -800.0]), mutant=mutant)
+    assert ends[0] == 1.0 and ends[1] == -1.0, "alpha spans [-1, 1]"
+    assert bends[0] == 2.0 and bends[1] == 0.0, "beta spans [0, 2]"
+
+
 ALL_PINS = [pin_commutator, pin_2d_construction, pin_prop2_block, pin_orthogonal_norm,
             pin_delta_write, pin_identity_gates, pin_gdn_and_kda_spectra, pin_sign_absorption,
             pin_brute_force, pin_rope_closed_form, pin_rope_both_q_and_k, pin_rope_properties,
-            pin_l2norm, pin_decode_matches_fwd]
+            pin_l2norm, pin_decode_matches_fwd, pin_gate_activation]

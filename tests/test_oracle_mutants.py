@@ -4,7 +4,7 @@ The mistakes are compiled into separate copies of the oracle (CKDA_ORACLE_MUTANT
 oracle is never modified.  This shows the pins in pins.py can see each class of error: the order
 of Diag(alpha) and the rank-one factor, the gate sign, the beta range, the read-out state, the
 read-out scale, the rotary frequency, rotating only q, the rotary base, a missing L2 norm and a
-norm taken jointly over q and k.
+norm taken jointly over q and k, and the two gate activations.
 """
 import pytest
 
@@ -22,6 +22,8 @@ MUTANTS = {
     8: "rotary base 1000",
     9: "L2 norm skipped",
     10: "L2 norm over q and k jointly",
+    11: "signed gate as sigma(a), without the 2x - 1 map",
+    12: "beta as sigma(b), without the factor 2",
 }
 
 

@@ -422,6 +422,25 @@ def main():
                                "ckda_over_kda": round(ms_kda / (ms_per_step if world == 1 else ms / args.steps), 4)}
         del kda_sets
 
+        # ---- gates given as logits (alpha = 2 sigma(a) - 1 from bf16 a, beta = 2 sigma(b)) ----
+        gl_sets = [synth.torch_fwd_inputs(B, T, H, dk, dv, dtype="bf16", seed=8000 + 10 * rank + i,
+                                          device=dev, gate_logits=True) for i in range(N_ROTATE)]
+
+        def step_gl(i):
+            s = gl_sets[i % N_ROTATE]
+            ck.fwd_chunked(s["q"], s["k"], s["v"], s["alpha"], s["beta"], None, chunk=C, path="tc",
+                           out=out, hT=hT, workspace=ws, gate_logits=True)
+        for i in range(3):
+            step_gl(i)
+        ms_gl = event_time_ms(step_gl, args.steps, stream) / args.steps
+        gl_bytes = FWD_BYTES_PER_HT - 256   # alpha as bf16 logits: 256 B instead of 512 per head-token
+        extras["gate_logits"] = {
+            "workload": f"{w['name']} with bf16 gate logits a and fp32 logits b",
+            "mtok_s": round(B * T / (ms_gl / 1e3) / 1e6, 2), "ms_per_step": round(ms_gl, 4),
+            "roofline_mtok_s": round(hbm_peak * 1e9 / (H * gl_bytes) / 1e6, 1),
+            "path_hbm_frac": round(ht * gl_bytes / (ms_gl / 1e3) / 1e9 / hbm_peak, 4)}
+        del gl_sets
+
         # ---- long-context forward with RoPE and an initial state (one call per step) -------
         wl = synth.WORKLOADS["long_rope_bf16"]
         L = synth.torch_fwd_inputs(wl["B"], wl["T"], wl["H"], 128, 128, kind="ckda",

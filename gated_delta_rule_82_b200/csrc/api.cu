@@ -108,7 +108,7 @@ size_t ckda_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, 
     return 0;
 }
 
-ckda_status ckda_fwd_chunked(const void* q, const void* k, const void* v, const float* alpha,
+ckda_status ckda_fwd_chunked(const void* q, const void* k, const void* v, const void* alpha,
                              const float* beta, const float* h0, void* out, float* hT, int B,
                              int T, int H, int dk, int dv, int chunk, ckda_flags flags,
                              ckda_dtype dtype, long long pos_offset, void* workspace,
@@ -129,8 +129,10 @@ ckda_status ckda_fwd_chunked(const void* q, const void* k, const void* v, const 
     const size_t nst = (size_t)B * H * dk * dv;
     // outputs must not overlap any input (hT == h0 exactly is allowed: each (b, h) is read
     // completely before it is written)
+    if (flags.gate_logits != 0 && flags.gate_logits != 1) return CKDA_ERR_ARG;
+    const size_t asz = nqk * (flags.gate_logits ? es : 4);   // gate values fp32, logits `dtype`
     const void* ins[] = {q, k, v, alpha, beta};
-    const size_t insz[] = {nqk * es, nqk * es, nv * es, nqk * 4, (size_t)B * T * H * 4};
+    const size_t insz[] = {nqk * es, nqk * es, nv * es, asz, (size_t)B * T * H * 4};
     for (int i = 0; i < 5; ++i) {
         if (overlap(out, nv * es, ins[i], insz[i])) return CKDA_ERR_ARG;
         if (hT && overlap(hT, nst * 4, ins[i], insz[i])) return CKDA_ERR_ARG;
@@ -149,19 +151,20 @@ ckda_status ckda_fwd_chunked(const void* q, const void* k, const void* v, const 
         if (need > 0 && (!workspace || workspace_bytes < need)) return CKDA_ERR_WORKSPACE;
         if (workspace && !aligned16(workspace)) return CKDA_ERR_ALIGN;
         const void* all[] = {q, k, v, alpha, beta, h0, out, hT};
-        const size_t allsz[] = {nqk * es, nqk * es, nv * es, nqk * 4, (size_t)B * T * H * 4,
+        const size_t allsz[] = {nqk * es, nqk * es, nv * es, asz, (size_t)B * T * H * 4,
                                 nst * 4, nv * es, nst * 4};
         for (int i = 0; i < 8; ++i)
             if (all[i] && overlap(workspace, need, all[i], allsz[i])) return CKDA_ERR_ARG;
         return from_cuda(launch_chunk_tc(q, k, v, alpha, beta, h0, out, hT, B, T, H, l2, rp,
-                                         scale, pos_offset, workspace, flags.stages,
-                                         (cudaStream_t)stream));
+                                         scale, pos_offset, flags.gate_logits, workspace,
+                                         flags.stages, (cudaStream_t)stream));
     }
     return from_cuda(launch_chunk_simt(q, k, v, alpha, beta, h0, out, hT, B, T, H, dk, dv, chunk,
-                                       l2, rp, scale, pos_offset, dtype, (cudaStream_t)stream));
+                                       l2, rp, scale, pos_offset, flags.gate_logits, dtype,
+                                       (cudaStream_t)stream));
 }
 
-ckda_status ckda_decode_step(const void* q, const void* k, const void* v, const float* alpha,
+ckda_status ckda_decode_step(const void* q, const void* k, const void* v, const void* alpha,
                              const float* beta, float* state, void* out, const long long* pos,
                              int N, int H, int dk, int dv, ckda_flags flags, ckda_dtype dtype,
                              ckda_stream_t stream) {
@@ -180,9 +183,11 @@ ckda_status ckda_decode_step(const void* q, const void* k, const void* v, const 
     if (rp.enabled && (reinterpret_cast<uintptr_t>(pos) & 7u)) return CKDA_ERR_ALIGN;
     const size_t es = elem_size(dtype);
     const size_t nst = (size_t)N * H * dk * dv * 4;
+    if (flags.gate_logits != 0 && flags.gate_logits != 1) return CKDA_ERR_ARG;
     const void* ins[] = {q, k, v, alpha, beta};
     const size_t insz[] = {(size_t)N * H * dk * es, (size_t)N * H * dk * es,
-                           (size_t)N * H * dv * es, (size_t)N * H * dk * 4, (size_t)N * H * 4};
+                           (size_t)N * H * dv * es, (size_t)N * H * dk * (flags.gate_logits ? es : 4),
+                           (size_t)N * H * 4};
     for (int i = 0; i < 5; ++i) {
         if (overlap(out, (size_t)N * H * dv * es, ins[i], insz[i])) return CKDA_ERR_ARG;
         if (overlap(state, nst, ins[i], insz[i])) return CKDA_ERR_ARG;
@@ -190,7 +195,8 @@ ckda_status ckda_decode_step(const void* q, const void* k, const void* v, const 
     if (overlap(state, nst, out, (size_t)N * H * dv * es)) return CKDA_ERR_ARG;
     return from_cuda(launch_decode(q, k, v, alpha, beta, state, out, rp.enabled ? pos : nullptr,
                                    N, H, dk, dv, flags.l2norm ? 1 : 0, rp,
-                                   resolve_scale(flags, dk), dtype, (cudaStream_t)stream));
+                                   resolve_scale(flags, dk), flags.gate_logits, dtype,
+                                   (cudaStream_t)stream));
 }
 
 ckda_status ckda_selftest_umma(const void* A, const void* B, float* D, int M, int N, int K,

@@ -56,9 +56,10 @@ struct SimtShape {
 template <typename T, int DK, int DV, int C>
 __global__ void __launch_bounds__(kSimtThreads)
 chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
-                  const float* __restrict__ alpha, const float* __restrict__ beta,
+                  const void* __restrict__ alpha, const float* __restrict__ beta,
                   const float* __restrict__ h0, T* __restrict__ out, float* __restrict__ hT,
-                  int T_len, int H, int l2norm, RopeParams rp, float scale, long long pos_offset) {
+                  int T_len, int H, int l2norm, RopeParams rp, float scale, long long pos_offset,
+                  int gate_logits) {
     using Sh = SimtShape<DK, DV, C>;
     constexpr int DVS = Sh::DVS;
     extern __shared__ float smem[];
@@ -113,8 +114,11 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
             if (r < nvalid) vv = to_f32(v[(((size_t)b * T_len + t0 + r) * H + h) * DV + n0 + n]);
             sv[e] = vv;
         }
-        for (int r = tid; r < C; r += kSimtThreads)
-            sb[r] = r < nvalid ? beta[((size_t)b * T_len + t0 + r) * H + h] : 0.f;
+        for (int r = tid; r < C; r += kSimtThreads) {
+            float bv = r < nvalid ? beta[((size_t)b * T_len + t0 + r) * H + h] : 0.f;
+            if (r < nvalid && gate_logits) bv = gate_beta(bv);   // beta = 2 sigma(b)
+            sb[r] = bv;
+        }
         __syncthreads();
 
         // ---- prologue per row (one warp per row): rotation, then L2 norm ----
@@ -165,7 +169,12 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
             float L = 0.f, sg = 1.f;
             for (int r = 0; r < C; ++r) {
                 float a = 1.f;
-                if (r < nvalid) a = alpha[(((size_t)b * T_len + t0 + r) * H + h) * DK + c];
+                if (r < nvalid) {
+                    const size_t ia = (((size_t)b * T_len + t0 + r) * H + h) * DK + c;
+                    // gate values (fp32), or logits in the activation type: alpha = 2 sigma(a) - 1
+                    a = gate_logits ? gate_alpha(to_f32(static_cast<const T*>(alpha)[ia]))
+                                    : static_cast<const float*>(alpha)[ia];
+                }
                 if (a < 0.f) sg = -sg;
                 L += log2f(fmaxf(fabsf(a), 1.17549435e-38f));
                 sL[r * DK + c] = L;
@@ -266,10 +275,10 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
 }
 
 template <typename T, int DK, int DV, int C>
-cudaError_t launch_simt_t(const void* q, const void* k, const void* v, const float* alpha,
+cudaError_t launch_simt_t(const void* q, const void* k, const void* v, const void* alpha,
                           const float* beta, const float* h0, void* out, float* hT, int B,
                           int T_len, int H, int l2norm, const RopeParams& rp, float scale,
-                          long long pos_offset, cudaStream_t stream) {
+                          long long pos_offset, int gate_logits, cudaStream_t stream) {
     using Sh = SimtShape<DK, DV, C>;
     auto kern = chunk_simt_kernel<T, DK, DV, C>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -278,63 +287,63 @@ cudaError_t launch_simt_t(const void* q, const void* k, const void* v, const flo
     dim3 grid(B * H, DV / Sh::DVS);
     kern<<<grid, kSimtThreads, Sh::bytes, stream>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), alpha, beta,
-        h0, static_cast<T*>(out), hT, T_len, H, l2norm, rp, scale, pos_offset);
+        h0, static_cast<T*>(out), hT, T_len, H, l2norm, rp, scale, pos_offset, gate_logits);
     return cudaGetLastError();
 }
 
 template <typename T, int DK, int DV>
 cudaError_t dispatch_chunk(int chunk, const void* q, const void* k, const void* v,
-                           const float* alpha, const float* beta, const float* h0, void* out,
+                           const void* alpha, const float* beta, const float* h0, void* out,
                            float* hT, int B, int T_len, int H, int l2norm, const RopeParams& rp,
-                           float scale, long long pos_offset, cudaStream_t stream) {
+                           float scale, long long pos_offset, int gate_logits, cudaStream_t stream) {
     switch (chunk) {
-        case 16: return launch_simt_t<T, DK, DV, 16>(q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, stream);
-        case 32: return launch_simt_t<T, DK, DV, 32>(q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, stream);
-        case 64: return launch_simt_t<T, DK, DV, 64>(q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, stream);
+        case 16: return launch_simt_t<T, DK, DV, 16>(q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 32: return launch_simt_t<T, DK, DV, 32>(q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 64: return launch_simt_t<T, DK, DV, 64>(q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, gate_logits, stream);
     }
     return cudaErrorInvalidValue;
 }
 
 template <typename T, int DK>
 cudaError_t dispatch_dv(int dv, int chunk, const void* q, const void* k, const void* v,
-                        const float* alpha, const float* beta, const float* h0, void* out,
+                        const void* alpha, const float* beta, const float* h0, void* out,
                         float* hT, int B, int T_len, int H, int l2norm, const RopeParams& rp,
-                        float scale, long long pos_offset, cudaStream_t stream) {
+                        float scale, long long pos_offset, int gate_logits, cudaStream_t stream) {
     switch (dv) {
-        case 16: return dispatch_chunk<T, DK, 16>(chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, stream);
-        case 32: return dispatch_chunk<T, DK, 32>(chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, stream);
-        case 64: return dispatch_chunk<T, DK, 64>(chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, stream);
-        case 128: return dispatch_chunk<T, DK, 128>(chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, stream);
+        case 16: return dispatch_chunk<T, DK, 16>(chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 32: return dispatch_chunk<T, DK, 32>(chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 64: return dispatch_chunk<T, DK, 64>(chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 128: return dispatch_chunk<T, DK, 128>(chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, gate_logits, stream);
     }
     return cudaErrorInvalidValue;
 }
 
 template <typename T>
 cudaError_t dispatch_dk(int dk, int dv, int chunk, const void* q, const void* k, const void* v,
-                        const float* alpha, const float* beta, const float* h0, void* out,
+                        const void* alpha, const float* beta, const float* h0, void* out,
                         float* hT, int B, int T_len, int H, int l2norm, const RopeParams& rp,
-                        float scale, long long pos_offset, cudaStream_t stream) {
+                        float scale, long long pos_offset, int gate_logits, cudaStream_t stream) {
     switch (dk) {
-        case 16: return dispatch_dv<T, 16>(dv, chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, stream);
-        case 32: return dispatch_dv<T, 32>(dv, chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, stream);
-        case 64: return dispatch_dv<T, 64>(dv, chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, stream);
-        case 128: return dispatch_dv<T, 128>(dv, chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, stream);
+        case 16: return dispatch_dv<T, 16>(dv, chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 32: return dispatch_dv<T, 32>(dv, chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 64: return dispatch_dv<T, 64>(dv, chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 128: return dispatch_dv<T, 128>(dv, chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, gate_logits, stream);
     }
     return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const float* alpha,
+cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const void* alpha,
                               const float* beta, const float* h0, void* out, float* hT, int B,
                               int T_len, int H, int dk, int dv, int chunk, int l2norm,
                               const RopeParams& rp, float scale, long long pos_offset,
-                              ckda_dtype dtype, cudaStream_t stream) {
+                              int gate_logits, ckda_dtype dtype, cudaStream_t stream) {
     if (dtype == CKDA_BF16)
         return dispatch_dk<__nv_bfloat16>(dk, dv, chunk, q, k, v, alpha, beta, h0, out, hT, B,
-                                          T_len, H, l2norm, rp, scale, pos_offset, stream);
+                                          T_len, H, l2norm, rp, scale, pos_offset, gate_logits, stream);
     return dispatch_dk<float>(dk, dv, chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H,
-                              l2norm, rp, scale, pos_offset, stream);
+                              l2norm, rp, scale, pos_offset, gate_logits, stream);
 }
 
 }  // namespace ckda

@@ -159,11 +159,12 @@ struct TcMaps {
 // Issue the TMA loads of chunk-head ci: alpha -> G, q -> QR, k -> KR on bar_in; V (two 64-column
 // halves, 128-byte swizzle) on bar_v when with_v.  Rows past the sequence end read as zeros.
 __device__ __forceinline__ void issue_inputs(const TcMaps& m, uint8_t* sm, uint64_t* bar_in,
-                                             int ci, int NT, int H) {
+                                             int ci, int NT, int H, int gate_logits) {
     const int ch = ci % NT, bh = ci / NT;
     const int b = bh / H, h = bh % H, t0 = ch * kC;
-    tc::mbar_arrive_expect_tx(bar_in, kInBytes);
-    tc::tma_load_4d(sm + S_G, &m.alpha, 0, h, t0, b, bar_in);
+    // gate values: fp32 [64][128] into G; logits: bf16 [64][128] into the upper half of G
+    tc::mbar_arrive_expect_tx(bar_in, gate_logits ? kInBytes - 16384 : kInBytes);
+    tc::tma_load_4d(sm + S_G + (gate_logits ? 16384 : 0), &m.alpha, 0, h, t0, b, bar_in);
     tc::tma_load_4d(sm + S_QR, &m.q, 0, h, t0, b, bar_in);
     tc::tma_load_4d(sm + S_KR, &m.k, 0, h, t0, b, bar_in);
 }
@@ -329,10 +330,13 @@ __device__ __forceinline__ void t_solve(const float* sA, float* sT, const float*
     }
 }
 
+// kLogits: alpha and beta hold logits (alpha = 2 sigma(a) - 1 from bf16 a, beta = 2 sigma(b)).
+template <bool kLogits>
 __global__ void __launch_bounds__(512, 1)
-ckda_tc_intra(const __grid_constant__ TcMaps maps, const float* __restrict__ alpha,
+ckda_tc_intra(const __grid_constant__ TcMaps maps, const void* __restrict__ alpha,
               const float* __restrict__ beta, uint8_t* __restrict__ ws, int T_len, int H, int NT,
               int total, int l2norm, RopeParams rp, long long pos_offset) {
+    constexpr int gate_logits = kLogits ? 1 : 0;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -380,7 +384,7 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const float* __restrict__ alp
         tc::prefetch_tensormap(&maps.k);
         tc::prefetch_tensormap(&maps.v);
         tc::prefetch_tensormap(&maps.alpha);
-        issue_inputs(maps, sm, bar_in, blockIdx.x, NT, H);
+        issue_inputs(maps, sm, bar_in, blockIdx.x, NT, H, gate_logits);
         issue_v(maps, sm, bar_v, blockIdx.x, NT, H);
     }
 
@@ -394,7 +398,8 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const float* __restrict__ alp
         const int nci = ci + gridDim.x;
         uint8_t* wsc = ws + (size_t)ci * WS_CHUNK;
         const size_t row0 = ((size_t)(bh / H) * T_len + t0) * H + h;
-        const float bval = (tid < 64 && tid < nvalid) ? beta[row0 + tid * rs] : 0.f;
+        float bval = (tid < 64 && tid < nvalid) ? beta[row0 + tid * rs] : 0.f;
+        if (kLogits && tid < 64 && tid < nvalid) bval = gate_beta(bval);   // beta = 2 sigma(b)
 
         tc::mbar_wait(bar_in, it & 1, abort_flag);
 
@@ -404,12 +409,23 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const float* __restrict__ alp
         const int cc = tid & 127, cI = tid >> 7;
         if (tid == 0) *exact_path = 0;
         {
+            float av[16];
+            if constexpr (kLogits) {
+                // logits a (bf16) in the upper half of G: all of them into registers first, since
+                // the fp32 rows written below cover the same bytes; alpha = 2 sigma(a) - 1
+                const __nv_bfloat16* la = reinterpret_cast<const __nv_bfloat16*>(sm + S_G + 16384);
+#pragma unroll
+                for (int rl = 0; rl < 16; ++rl) av[rl] = gate_alpha(__bfloat162float(la[(16 * cI + rl) * 128 + cc]));
+                __syncthreads();
+            } else {
+#pragma unroll
+                for (int rl = 0; rl < 16; ++rl) av[rl] = G[(16 * cI + rl) * 128 + cc];
+            }
             float p = 1.f;
 #pragma unroll
             for (int rl = 0; rl < 16; ++rl) {
                 const int r = 16 * cI + rl;
-                const float a = r < nvalid ? G[r * 128 + cc] : 1.f;
-                p *= a;
+                p *= r < nvalid ? av[rl] : 1.f;
                 G[r * 128 + cc] = p;
             }
             gP[cI * 128 + cc] = p;
@@ -547,7 +563,7 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const float* __restrict__ alp
             }
         }
         // alpha, q, k of this chunk-head are consumed: bring in the next one's
-        if (tid == 0 && nci < total) issue_inputs(maps, sm, bar_in, nci, NT, H);
+        if (tid == 0 && nci < total) issue_inputs(maps, sm, bar_in, nci, NT, H, gate_logits);
         if (!exact) {
             tc::mbar_wait(bar, phase & 1, abort_flag);
             ++phase;
@@ -580,7 +596,14 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const float* __restrict__ alp
             if (tid < 128) {
                 float L = 0.f;
                 for (int r = 0; r < 64; ++r) {
-                    const float a = r < nvalid ? alpha[(row0 + r * rs) * kDK + tid] : 1.f;
+                    float a = 1.f;
+                    if (r < nvalid) {
+                        const size_t ia = (row0 + r * rs) * kDK + tid;
+                        if constexpr (kLogits)
+                            a = gate_alpha(__bfloat162float(static_cast<const __nv_bfloat16*>(alpha)[ia]));
+                        else
+                            a = static_cast<const float*>(alpha)[ia];
+                    }
                     L += log2f(fmaxf(fabsf(a), 1.17549435e-38f));
                     sLg[r * 128 + tid] = L;
                 }
@@ -1080,12 +1103,13 @@ size_t chunk_tc_workspace_bytes(int B, int T_len, int H) {
     return (size_t)B * H * nt * WS_CHUNK;
 }
 
-cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const float* alpha,
+cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const void* alpha,
                             const float* beta, const float* h0, void* out, float* hT, int B,
                             int T_len, int H, int l2norm, const RopeParams& rp, float scale,
-                            long long pos_offset, void* workspace, int stages,
+                            long long pos_offset, int gate_logits, void* workspace, int stages,
                             cudaStream_t stream) {
-    cudaError_t e = cudaFuncSetAttribute(ckda_tc_intra, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    auto intra = gate_logits ? ckda_tc_intra<true> : ckda_tc_intra<false>;
+    cudaError_t e = cudaFuncSetAttribute(intra, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)S_BYTES);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(ckda_tc_state, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P2_BYTES);
@@ -1106,8 +1130,10 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const f
                         CU_TENSOR_MAP_SWIZZLE_NONE) ||
             !encode_map(&maps.v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDV, 64, H, T_len, B,
                         CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !encode_map(&maps.alpha, alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kDK, kDK, H, T_len,
-                        B, CU_TENSOR_MAP_SWIZZLE_NONE))
+            !(gate_logits ? encode_map(&maps.alpha, alpha, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK,
+                                       kDK, H, T_len, B, CU_TENSOR_MAP_SWIZZLE_NONE)
+                          : encode_map(&maps.alpha, alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kDK,
+                                       kDK, H, T_len, B, CU_TENSOR_MAP_SWIZZLE_NONE)))
             return cudaErrorInvalidValue;
         // programmatic dependent launch: CTAs may start their set-up on SMs the previous kernel
         // has left, and wait (griddepcontrol.wait) for it before touching memory
@@ -1121,8 +1147,8 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const f
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, ckda_tc_intra, maps, alpha, beta, ws, T_len, H, NT, total,
-                               l2norm, rp, pos_offset);
+        e = cudaLaunchKernelEx(&cfg, intra, maps, alpha, beta, ws, T_len, H, NT, total, l2norm,
+                               rp, pos_offset);
         if (e != cudaSuccess) return e;
     }
     if (stages & 2) {

@@ -96,4 +96,13 @@ __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
     return __float2bfloat16_rn(x);
 }
 
+// Gates from logits ("Complex KDA" paper summary, Methodology, CKDA Definition):
+// alpha = 2 sigma(a) - 1 (= tanh(a / 2), formed as (1 - e) / (1 + e) with e = exp(-|a|), which
+// loses no precision near |alpha| = 1) and beta = 2 sigma(b).
+__device__ __forceinline__ float gate_alpha(float a) {
+    const float e = __expf(-fabsf(a));
+    return copysignf(__fdividef(1.f - e, 1.f + e), a);
+}
+__device__ __forceinline__ float gate_beta(float b) { return __fdividef(2.f, 1.f + __expf(-b)); }
+
 }  // namespace ckda

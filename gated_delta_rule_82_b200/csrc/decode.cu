@@ -41,10 +41,10 @@ __device__ __forceinline__ void st_stream(float* p, float4 v) {
                  :: "l"(p), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w) : "memory");
 }
 
-template <typename T, int DK, int DV>
+template <typename T, int DK, int DV, bool kLogits>
 __global__ void __launch_bounds__(kDecodeThreads, 2)
 decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
-              const float* __restrict__ alpha, const float* __restrict__ beta,
+              const void* __restrict__ alpha, const float* __restrict__ beta,
               float* __restrict__ state, T* __restrict__ out, const long long* __restrict__ pos,
               int NH, int H, int l2norm, RopeParams rp, float scale) {
     using S = DecodeShape<DK, DV>;
@@ -76,7 +76,11 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
         if (g < NH) {
             qv = to_f32(q[(size_t)g * DK + c]);
             kv = to_f32(k[(size_t)g * DK + c]);
-            av = alpha[(size_t)g * DK + c];
+            // gate values (fp32), or logits a in the activation type: alpha = 2 sigma(a) - 1
+            if constexpr (kLogits)
+                av = gate_alpha(to_f32(static_cast<const T*>(alpha)[(size_t)g * DK + c]));
+            else
+                av = static_cast<const float*>(alpha)[(size_t)g * DK + c];
         }
         sq[hh][c] = qv; sk[hh][c] = kv; sa[hh][c] = av;
     }
@@ -87,7 +91,8 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
     }
     if (tid < HPC) {
         int g = blockIdx.x * HPC + tid;
-        sbeta[tid] = g < NH ? beta[g] : 0.f;
+        const float bv = g < NH ? beta[g] : 0.f;
+        sbeta[tid] = (kLogits && g < NH) ? gate_beta(bv) : bv;
     }
     __syncthreads();
 
@@ -199,58 +204,59 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
 }
 
 template <typename T, int DK, int DV>
-cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const float* alpha,
+cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const void* alpha,
                             const float* beta, float* state, void* out, const long long* pos,
                             int N, int H, int l2norm, const RopeParams& rp, float scale,
-                            cudaStream_t stream) {
+                            int gate_logits, cudaStream_t stream) {
     using S = DecodeShape<DK, DV>;
     int NH = N * H;
     int grid = (NH + S::HPC - 1) / S::HPC;
-    decode_kernel<T, DK, DV><<<grid, kDecodeThreads, 0, stream>>>(
+    auto kern = gate_logits ? decode_kernel<T, DK, DV, true> : decode_kernel<T, DK, DV, false>;
+    kern<<<grid, kDecodeThreads, 0, stream>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), alpha, beta,
         state, static_cast<T*>(out), pos, NH, H, l2norm, rp, scale);
     return cudaGetLastError();
 }
 
 template <typename T, int DK>
-cudaError_t dispatch_dv(int dv, const void* q, const void* k, const void* v, const float* alpha,
+cudaError_t dispatch_dv(int dv, const void* q, const void* k, const void* v, const void* alpha,
                         const float* beta, float* state, void* out, const long long* pos, int N,
                         int H, int l2norm, const RopeParams& rp, float scale,
-                        cudaStream_t stream) {
+                        int gate_logits, cudaStream_t stream) {
     switch (dv) {
-        case 16: return launch_decode_t<T, DK, 16>(q, k, v, alpha, beta, state, out, pos, N, H, l2norm, rp, scale, stream);
-        case 32: return launch_decode_t<T, DK, 32>(q, k, v, alpha, beta, state, out, pos, N, H, l2norm, rp, scale, stream);
-        case 64: return launch_decode_t<T, DK, 64>(q, k, v, alpha, beta, state, out, pos, N, H, l2norm, rp, scale, stream);
-        case 128: return launch_decode_t<T, DK, 128>(q, k, v, alpha, beta, state, out, pos, N, H, l2norm, rp, scale, stream);
+        case 16: return launch_decode_t<T, DK, 16>(q, k, v, alpha, beta, state, out, pos, N, H, l2norm, rp, scale, gate_logits, stream);
+        case 32: return launch_decode_t<T, DK, 32>(q, k, v, alpha, beta, state, out, pos, N, H, l2norm, rp, scale, gate_logits, stream);
+        case 64: return launch_decode_t<T, DK, 64>(q, k, v, alpha, beta, state, out, pos, N, H, l2norm, rp, scale, gate_logits, stream);
+        case 128: return launch_decode_t<T, DK, 128>(q, k, v, alpha, beta, state, out, pos, N, H, l2norm, rp, scale, gate_logits, stream);
     }
     return cudaErrorInvalidValue;
 }
 
 template <typename T>
 cudaError_t dispatch_dk(int dk, int dv, const void* q, const void* k, const void* v,
-                        const float* alpha, const float* beta, float* state, void* out,
+                        const void* alpha, const float* beta, float* state, void* out,
                         const long long* pos, int N, int H, int l2norm, const RopeParams& rp,
-                        float scale, cudaStream_t stream) {
+                        float scale, int gate_logits, cudaStream_t stream) {
     switch (dk) {
-        case 16: return dispatch_dv<T, 16>(dv, q, k, v, alpha, beta, state, out, pos, N, H, l2norm, rp, scale, stream);
-        case 32: return dispatch_dv<T, 32>(dv, q, k, v, alpha, beta, state, out, pos, N, H, l2norm, rp, scale, stream);
-        case 64: return dispatch_dv<T, 64>(dv, q, k, v, alpha, beta, state, out, pos, N, H, l2norm, rp, scale, stream);
-        case 128: return dispatch_dv<T, 128>(dv, q, k, v, alpha, beta, state, out, pos, N, H, l2norm, rp, scale, stream);
+        case 16: return dispatch_dv<T, 16>(dv, q, k, v, alpha, beta, state, out, pos, N, H, l2norm, rp, scale, gate_logits, stream);
+        case 32: return dispatch_dv<T, 32>(dv, q, k, v, alpha, beta, state, out, pos, N, H, l2norm, rp, scale, gate_logits, stream);
+        case 64: return dispatch_dv<T, 64>(dv, q, k, v, alpha, beta, state, out, pos, N, H, l2norm, rp, scale, gate_logits, stream);
+        case 128: return dispatch_dv<T, 128>(dv, q, k, v, alpha, beta, state, out, pos, N, H, l2norm, rp, scale, gate_logits, stream);
     }
     return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* alpha,
+cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* alpha,
                           const float* beta, float* state, void* out, const long long* pos, int N,
                           int H, int dk, int dv, int l2norm, const RopeParams& rp, float scale,
-                          ckda_dtype dtype, cudaStream_t stream) {
+                          int gate_logits, ckda_dtype dtype, cudaStream_t stream) {
     if (dtype == CKDA_BF16)
         return dispatch_dk<__nv_bfloat16>(dk, dv, q, k, v, alpha, beta, state, out, pos, N, H,
-                                          l2norm, rp, scale, stream);
+                                          l2norm, rp, scale, gate_logits, stream);
     return dispatch_dk<float>(dk, dv, q, k, v, alpha, beta, state, out, pos, N, H, l2norm, rp,
-                              scale, stream);
+                              scale, gate_logits, stream);
 }
 
 }  // namespace ckda

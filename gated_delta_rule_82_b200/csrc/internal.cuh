@@ -9,23 +9,25 @@ cudaError_t launch_qk_prologue(const void* q, const void* k, void* qo, void* ko,
                                int H, int dk, int l2norm, const RopeParams& rp,
                                long long pos_offset, ckda_dtype dtype, cudaStream_t stream);
 
-cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* alpha,
+// alpha: fp32 gate values, or (gate_logits != 0) logits a of the activation type; with logits
+// the kernels form alpha = 2 sigma(a) - 1 and beta = 2 sigma(b) from the fp32 logits in beta.
+cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* alpha,
                           const float* beta, float* state, void* out, const long long* pos, int N,
                           int H, int dk, int dv, int l2norm, const RopeParams& rp, float scale,
-                          ckda_dtype dtype, cudaStream_t stream);
+                          int gate_logits, ckda_dtype dtype, cudaStream_t stream);
 
-cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const float* alpha,
+cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const void* alpha,
                               const float* beta, const float* h0, void* out, float* hT, int B,
                               int T_len, int H, int dk, int dv, int chunk, int l2norm,
                               const RopeParams& rp, float scale, long long pos_offset,
-                              ckda_dtype dtype, cudaStream_t stream);
+                              int gate_logits, ckda_dtype dtype, cudaStream_t stream);
 
 // Tensor-core chunked forward (bf16, dk = dv = 128, chunk = 64).
 size_t chunk_tc_workspace_bytes(int B, int T_len, int H);
-cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const float* alpha,
+cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const void* alpha,
                             const float* beta, const float* h0, void* out, float* hT, int B,
                             int T_len, int H, int l2norm, const RopeParams& rp, float scale,
-                            long long pos_offset, void* workspace, int stages,
+                            long long pos_offset, int gate_logits, void* workspace, int stages,
                             cudaStream_t stream);
 
 cudaError_t launch_umma_selftest(const void* A, const void* B, float* D, int M, int N, int K,

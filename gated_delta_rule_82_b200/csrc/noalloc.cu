@@ -40,7 +40,7 @@ void* scratch_address(int device) {
 }  // namespace
 
 extern "C" CKDA_API ckda_status ckda_fwd_chunked_noalloc(
-    const void* q, const void* k, const void* v, const float* alpha, const float* beta,
+    const void* q, const void* k, const void* v, const void* alpha, const float* beta,
     const float* h0, void* out, float* hT, int B, int T, int H, int dk, int dv, int chunk,
     ckda_flags flags, ckda_dtype dtype, long long pos_offset, ckda_stream_t stream) {
     const size_t need = ckda_fwd_workspace_bytes(B, T, H, dk, dv, chunk, dtype, flags.path);

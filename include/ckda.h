@@ -28,7 +28,8 @@
  *  - Layouts are dense row-major with the last index fastest:
  *        q, k, alpha : [B, T, H, dk]     v, out : [B, T, H, dv]     beta : [B, T, H]
  *        h0, hT, decode state : [B or N, H, dk, dv]  (fp32 always)
- *    q, k, v, out have the element type `dtype`; alpha, beta and states are fp32.
+ *    q, k, v, out have the element type `dtype`; beta and states are fp32; alpha is fp32 gate
+ *    values, or (flags.gate_logits = 1) logits of the element type `dtype`.
  *  - Supported sizes: dk, dv in {16, 32, 64, 128}; chunk in {16, 32, 64}; any T >= 1 (a
  *    partial last chunk is handled exactly).  B*H, N*H >= 1.
  */
@@ -41,7 +42,7 @@
 extern "C" {
 #endif
 
-#define CKDA_ABI_VERSION 1
+#define CKDA_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define CKDA_API __attribute__((visibility("default")))
@@ -84,6 +85,12 @@ typedef struct {
                             0 or 3 = both kernels; 1 = only the chunk-parallel factor kernel
                             (fills the workspace); 2 = only the serial state pass (reads a
                             workspace filled by a stage-1 call with the same arguments) */
+    int gate_logits;     /* 0: alpha and beta hold the gates themselves (fp32).  1: they hold
+                            logits -- alpha the logits a in the element type `dtype`, beta the
+                            logits b in fp32 -- and the kernels form the gates as
+                            alpha = 2 sigma(a) - 1 and beta = 2 sigma(b), sigma the logistic
+                            function (the parameterisation of the "Complex KDA" paper summary,
+                            Methodology, CKDA Definition).  Any other value: CKDA_ERR_ARG. */
 } ckda_flags;
 
 /* Version of this ABI (CKDA_ABI_VERSION of the build). */
@@ -114,7 +121,8 @@ CKDA_API size_t ckda_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, in
 /*
  * Chunked forward over whole sequences.
  *   q, k   : [B, T, H, dk] dtype          v   : [B, T, H, dv] dtype
- *   alpha  : [B, T, H, dk] fp32 (signed)  beta: [B, T, H] fp32
+ *   alpha  : [B, T, H, dk] fp32 gates (signed), or dtype logits when flags.gate_logits
+ *   beta   : [B, T, H] fp32 gates, or fp32 logits when flags.gate_logits
  *   h0     : [B, H, dk, dv] fp32, or NULL for a zero initial state
  *   out    : [B, T, H, dv] dtype (written)
  *   hT     : [B, H, dk, dv] fp32 final state, or NULL to skip it (may equal h0: read before write
@@ -128,7 +136,7 @@ CKDA_API size_t ckda_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, in
  * The computation is the recurrence above, evaluated chunk by chunk: within a chunk a WY/UT
  * representation of the product of transitions, across chunks an fp32 state.
  */
-CKDA_API ckda_status ckda_fwd_chunked(const void* q, const void* k, const void* v, const float* alpha,
+CKDA_API ckda_status ckda_fwd_chunked(const void* q, const void* k, const void* v, const void* alpha,
                              const float* beta, const float* h0, void* out, float* hT, int B,
                              int T, int H, int dk, int dv, int chunk, ckda_flags flags,
                              ckda_dtype dtype, long long pos_offset, void* workspace,
@@ -137,12 +145,13 @@ CKDA_API ckda_status ckda_fwd_chunked(const void* q, const void* k, const void* 
 /*
  * One decode step for N independent sequences, in place on the caller's fp32 state:
  *   q, k, alpha : [N, H, dk]    v, out : [N, H, dv]    beta : [N, H]
+ *   (alpha fp32 gates or dtype logits, beta fp32 gates or logits, as flags.gate_logits says)
  *   state       : [N, H, dk, dv] fp32, read and overwritten with S_t
  *   pos         : [N] int64 rotary positions (required when rope_theta > 0, else ignored)
  * out = scale * S_t^T q_t, with S_t = (I - beta k k^T) Diag(alpha) S_{t-1} + beta k v^T.
  * Each head's state is streamed through the SM exactly once (read once, written once).
  */
-CKDA_API ckda_status ckda_decode_step(const void* q, const void* k, const void* v, const float* alpha,
+CKDA_API ckda_status ckda_decode_step(const void* q, const void* k, const void* v, const void* alpha,
                              const float* beta, float* state, void* out, const long long* pos,
                              int N, int H, int dk, int dv, ckda_flags flags, ckda_dtype dtype,
                              ckda_stream_t stream);
@@ -179,7 +188,7 @@ CKDA_API ckda_status ckda_selftest_umma(const void* A, const void* B, float* D, 
 #define CKDA_NOALLOC_MAX_WORKSPACE (16u << 20)
 
 CKDA_API ckda_status ckda_fwd_chunked_noalloc(const void* q, const void* k, const void* v,
-                                              const float* alpha, const float* beta,
+                                              const void* alpha, const float* beta,
                                               const float* h0, void* out, float* hT, int B,
                                               int T, int H, int dk, int dv, int chunk,
                                               ckda_flags flags, ckda_dtype dtype,

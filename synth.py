@@ -13,6 +13,10 @@ Definition": alpha in [-1, 1]^dk, beta in [0, 2]):
   ``tiny``     q, k, v ~ N(0,1); alpha = s*m, s = +-1 (p = 1/2), m ~ U[0.05, 1]; beta ~ U[0, 2]
   ``ckda``     alpha = s*exp(-softplus(z)), z ~ N(0,1), |alpha| >= 1e-3; beta = 2*sigmoid(N(0,1))
   ``kda``      alpha = exp(-softplus(z)) in (0, 1]; beta = sigmoid(N(0,1)) in [0, 1]
+
+Gate logits (the optional input form whose activations 2 sigmoid(a) - 1 and 2 sigmoid(b) the
+library and the oracle form themselves): a = s * (1 + 2|z|), s = +-1 (p = 1/2), z ~ N(0,1),
+rounded to the activation dtype; b ~ N(0,1) in float32.
 """
 from __future__ import annotations
 
@@ -68,6 +72,19 @@ def gates(kind: str, shape_alpha, shape_beta, seed: int):
     else:
         raise ValueError(f"unknown gate recipe {kind!r}")
     return alpha.astype(np.float32), beta.astype(np.float32)
+
+
+def gate_logits(shape_alpha, shape_beta, seed: int, dtype: str):
+    """(a float32 values, a bf16 bits or None, b float32) for the gate-logit recipe above."""
+    ga, gb = _gen(seed, "alpha"), _gen(seed, "beta")
+    s = np.where(ga.random(size=shape_alpha) < 0.5, -1.0, 1.0)
+    a = (s * (1.0 + 2.0 * np.abs(ga.standard_normal(size=shape_alpha)))).astype(np.float32)
+    bits = None
+    if dtype == "bf16":
+        bits = f32_to_bf16_bits(a)
+        a = bf16_bits_to_f32(bits)
+    b = gb.standard_normal(size=shape_beta).astype(np.float32)
+    return a, bits, b
 
 
 def _activation(seed, tensor, shape, dtype):
@@ -164,7 +181,9 @@ def torch_gates(kind, shape_alpha, shape_beta, gen, device):
 
 
 def torch_fwd_inputs(B, T, H, dk, dv, *, kind="ckda", dtype="bf16", h0_std=0.0, seed=0,
-                     device="cuda"):
+                     device="cuda", gate_logits=False):
+    """Device-side draws of the same recipes (torch's seeded generator).  With gate_logits,
+    alpha and beta hold logits of the gate-logit recipe (alpha in the activation dtype)."""
     import torch
     gen = torch.Generator(device=device)
     gen.manual_seed(int(seed))
@@ -172,7 +191,13 @@ def torch_fwd_inputs(B, T, H, dk, dv, *, kind="ckda", dtype="bf16", h0_std=0.0, 
     d = {}
     for name, last in (("q", dk), ("k", dk), ("v", dv)):
         d[name] = torch.randn((B, T, H, last), generator=gen, device=device).to(tdt)
-    d["alpha"], d["beta"] = torch_gates(kind, (B, T, H, dk), (B, T, H), gen, device)
+    if gate_logits:
+        s = torch.where(torch.rand((B, T, H, dk), generator=gen, device=device) < 0.5, -1.0, 1.0)
+        z = torch.randn((B, T, H, dk), generator=gen, device=device)
+        d["alpha"] = (s * (1.0 + 2.0 * z.abs())).to(tdt).contiguous()
+        d["beta"] = torch.randn((B, T, H), generator=gen, device=device).contiguous()
+    else:
+        d["alpha"], d["beta"] = torch_gates(kind, (B, T, H, dk), (B, T, H), gen, device)
     d["h0"] = (h0_std * torch.randn((B, H, dk, dv), generator=gen, device=device)
                if h0_std > 0 else None)
     return d

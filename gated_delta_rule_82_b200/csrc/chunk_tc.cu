@@ -95,7 +95,7 @@ constexpr uint32_t S_OUT_TL = S_KE;  // dv tiles (48 KB, over K_end, M, A and pa
 constexpr uint32_t SM_P = S_SM;                  // signed block totals of alpha, fp32 [4][128]
 constexpr uint32_t SM_GC = S_SM + 2048;          // gamma_C fp32 [128] (signed)
 constexpr uint32_t SM_B = S_SM + 2560;           // beta fp32 [64]
-constexpr uint32_t SM_FLAGS = S_SM + 2816;       // exact flag, abort flag, TMEM slot, 3 mbarriers
+constexpr uint32_t SM_FLAGS = S_SM + 2816;       // exact flag, abort flag, TMEM slot, 5 mbarriers
 constexpr uint32_t kInBytes = 32768 + 2 * 16384; // alpha, q, k of one chunk-head
 constexpr uint32_t kVBytes = 16384;
 
@@ -350,6 +350,8 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const void* __restrict__ alph
     uint64_t* bar = reinterpret_cast<uint64_t*>(exact_path + 16);   // tensor-core completions
     uint64_t* bar_in = bar + 1;                                     // alpha, q, k landed
     uint64_t* bar_v = bar + 2;                                      // V landed
+    uint64_t* bar_w = bar + 3;                                      // W^T product complete
+    uint64_t* bar_q = bar + 4;                                      // M W (for Q') complete
     float* sA = reinterpret_cast<float*>(sm + S_A);
     float* sT = reinterpret_cast<float*>(sm + S_T);
     float* sLg = reinterpret_cast<float*>(sm + S_W);   // exact path only
@@ -368,6 +370,8 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const void* __restrict__ alph
         tc::mbar_init(bar, 1);
         tc::mbar_init(bar_in, 1);
         tc::mbar_init(bar_v, 1);
+        tc::mbar_init(bar_w, 1);
+        tc::mbar_init(bar_q, 1);
         tc::fence_mbar_init();
         *abort_flag = 0;
     }
@@ -549,6 +553,9 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const void* __restrict__ alph
         if (tid == 0) tc::bulk_wait_read<0>();
         __syncthreads();
         tc::tc_fence_after();
+        // alpha, q, k of this chunk-head are consumed: bring in the next one's.  Issued by warp 15
+        // (a TMA issue costs its thread several hundred cycles) while warp 0 issues the product.
+        if (tid == 480 && nci < total) issue_inputs(maps, sm, bar_in, nci, NT, H, gate_logits);
         if (!exact) {
             // ======== B: [A | M] = L R^T on the tensor cores (M = 128, N = 64, K = 128) ========
             if (warp == 0) {
@@ -562,8 +569,6 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const void* __restrict__ alph
                 tc::mma_commit_warp(bar);
             }
         }
-        // alpha, q, k of this chunk-head are consumed: bring in the next one's
-        if (tid == 0 && nci < total) issue_inputs(maps, sm, bar_in, nci, NT, H, gate_logits);
         if (!exact) {
             tc::mbar_wait(bar, phase & 1, abort_flag);
             ++phase;
@@ -659,18 +664,18 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const void* __restrict__ alph
             const uint64_t vd = tc::smem_desc_sw128(tc::smem_u32(sm + S_V), 8192, 1024);
             const uint32_t idesc = tc::idesc_bf16_f32(128, 64, 1, 0);
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t b = tc::desc_add(bd, ks * 32);
-                tc::mma_bf16_warp(tmem, tc::desc_add(kd, ks * 2048), b, idesc, ks > 0);
-                tc::mma_bf16_warp(tmem + 64, tc::desc_add(vd, ks * 2048), b, idesc, ks > 0);
-            }
+            for (int ks = 0; ks < 4; ++ks)
+                tc::mma_bf16_warp(tmem, tc::desc_add(kd, ks * 2048), tc::desc_add(bd, ks * 32), idesc, ks > 0);
+            tc::mma_commit_warp(bar_w);   // W^T: its read-back starts while U~^T computes
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                tc::mma_bf16_warp(tmem + 64, tc::desc_add(vd, ks * 2048), tc::desc_add(bd, ks * 32), idesc, ks > 0);
             tc::mma_commit_warp(bar);
         }
-        tc::mbar_wait(bar, phase & 1, abort_flag);
+        if ((warp >> 2) < 2) tc::mbar_wait(bar_w, it & 1, abort_flag);
+        else tc::mbar_wait(bar, phase & 1, abort_flag);
         ++phase;
         tc::tc_fence_after();
-        // V of this chunk-head is consumed: bring in the next one's
-        if (tid == 0 && nci < total) issue_v(maps, sm, bar_v, nci, NT, H);
         {
             // warp w: lanes 32 (w % 4) .. (channel, or dv column, c); 32-column slice w / 4:
             // slices 0, 1 -> W^T tokens 0..63, slices 2, 3 -> U~^T tokens 0..63.  Both tiles are
@@ -700,19 +705,26 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const void* __restrict__ alph
             const uint32_t id_q = tc::idesc_bf16_f32(64, 128, 0, 0);
             const uint32_t id_o = tc::idesc_bf16_f32(128, 64, 0, 0);
             const uint32_t id_c = tc::idesc_bf16_f32(128, 128, 1, 0);
+            // product by product, M W first: the Q' read-back overlaps the other three
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t w = tc::desc_add(wd, ks * 32), u = tc::desc_add(ud, ks * 32);
-                const uint64_t m = tc::desc_add(md, ks * 32), ke = tc::desc_add(ked, ks * 2048);
-                tc::mma_bf16_warp(tmem, m, w, id_q, ks > 0);               // M W
-                tc::mma_bf16_warp(tmem + 128, u, m, id_o, ks > 0);         // U~^T M^T
-                tc::mma_bf16_warp(tmem + 192, ke, w, id_c, ks > 0);        // K_end^T W
-                tc::mma_bf16_warp(tmem + 320, ke, u, id_c, ks > 0);        // K_end^T U~
-            }
+            for (int ks = 0; ks < 4; ++ks)                                  // M W
+                tc::mma_bf16_warp(tmem, tc::desc_add(md, ks * 32), tc::desc_add(wd, ks * 32), id_q, ks > 0);
+            tc::mma_commit_warp(bar_q);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)                                  // U~^T M^T
+                tc::mma_bf16_warp(tmem + 128, tc::desc_add(ud, ks * 32), tc::desc_add(md, ks * 32), id_o, ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)                                  // K_end^T W
+                tc::mma_bf16_warp(tmem + 192, tc::desc_add(ked, ks * 2048), tc::desc_add(wd, ks * 32), id_c, ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)                                  // K_end^T U~
+                tc::mma_bf16_warp(tmem + 320, tc::desc_add(ked, ks * 2048), tc::desc_add(ud, ks * 32), id_c, ks > 0);
             tc::mma_commit_warp(bar);
         }
-        tc::mbar_wait(bar, phase & 1, abort_flag);
-        ++phase;
+        // V of this chunk-head was consumed by the W/U~ products: bring in the next one's, from
+        // warp 14 while warp 0 issues these products
+        if (tid == 448 && nci < total) issue_v(maps, sm, bar_v, nci, NT, H);
+        tc::mbar_wait(bar_q, it & 1, abort_flag);
         tc::tc_fence_after();
         // ======== G: results into shared staging images, then bulk stores in two groups ========
         {
@@ -735,6 +747,9 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const void* __restrict__ alph
                 }
             }
             // (2) M = 128 products, lane = row c' (A_c, B_c) or dv column (O_loc^T)
+            tc::mbar_wait(bar, phase & 1, abort_flag);
+            ++phase;
+            tc::tc_fence_after();
             {
                 const int cr = 32 * quarter + lane;
                 // O_loc^T: tokens 16 slice .. 16 slice + 15 of dv column cr -> tile cr / 32, stored

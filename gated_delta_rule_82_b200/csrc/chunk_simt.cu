@@ -85,6 +85,13 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
     const int lane = tid & 31, warp = tid >> 5;
     constexpr int NW = kSimtThreads / 32;
 
+    // RoPE inverse frequencies in shared memory (lanes index them per channel; a per-lane index
+    // into the kernel-parameter array would serialise in the constant cache).  The barrier at the
+    // top of the chunk loop publishes them.
+    __shared__ double sfreq[DK / 2];
+    if (rp.enabled)
+        for (int i = tid; i < DK / 2; i += kSimtThreads) sfreq[i] = rp.inv_freq[i];
+
     // entering state slice
     for (int e = tid; e < DK * DVS; e += kSimtThreads) {
         int c = e / DVS, n = e % DVS;
@@ -140,7 +147,7 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
                         i = c / 2; first = (c & 1) == 0; partner = c ^ 1;
                     }
                     float sn, cs;
-                    rope_sincos(p, rp.inv_freq[i], &sn, &cs);
+                    rope_sincos(p, sfreq[i], &sn, &cs);
                     float qp = sq[r * DK + partner], kp = sk[r * DK + partner];
                     qr[m] = first ? qr[m] * cs - qp * sn : qr[m] * cs + qp * sn;
                     kr[m] = first ? kr[m] * cs - kp * sn : kr[m] * cs + kp * sn;

@@ -81,7 +81,7 @@ constexpr uint32_t S_T = 173056;     // T fp32 [64][68]
 constexpr uint32_t S_W = 190464;     // W^T K-major 128 x 64  (exact path: log2 prefix fp32 [64][128]
 constexpr uint32_t S_U = 206848;     // U~^T K-major 128 x 64  spanning S_W and S_U)
 constexpr uint32_t S_SM = 223232;    // small arrays (below)
-constexpr uint32_t S_BYTES = S_SM + 3072 + 1024;
+constexpr uint32_t S_BYTES = S_SM + 3584 + 1024;
 constexpr int kStrideA = 68;         // fp32 row stride of A and T
 // T solve scratch inside R (dead after the [A | M] product)
 constexpr uint32_t S_TB = S_R;               // T' bf16 K-major 64 x 64
@@ -96,6 +96,7 @@ constexpr uint32_t SM_P = S_SM;                  // signed block totals of alpha
 constexpr uint32_t SM_GC = S_SM + 2048;          // gamma_C fp32 [128] (signed)
 constexpr uint32_t SM_B = S_SM + 2560;           // beta fp32 [64]
 constexpr uint32_t SM_FLAGS = S_SM + 2816;       // exact flag, abort flag, TMEM slot, 5 mbarriers
+constexpr uint32_t SM_FREQ = S_SM + 3072;        // RoPE inverse frequencies fp64 [64]
 constexpr uint32_t kInBytes = 32768 + 2 * 16384; // alpha, q, k of one chunk-head
 constexpr uint32_t kVBytes = 16384;
 
@@ -366,6 +367,10 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const void* __restrict__ alph
         tc::tmem_alloc(tmem_slot, 512);
         tc::tmem_relinquish();
     }
+    // RoPE inverse frequencies in shared memory: lanes index them by channel group, and a
+    // per-lane index into the kernel-parameter array would serialise in the constant cache
+    double* sfreq = reinterpret_cast<double*>(sm + SM_FREQ);
+    if (tid < 64) sfreq[tid] = rp.inv_freq[tid];
     if (tid == 32) {
         tc::mbar_init(bar, 1);
         tc::mbar_init(bar_in, 1);
@@ -481,7 +486,7 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const void* __restrict__ alph
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {   // pairs (cA + i, cB + i), frequency 8g + i
                         float sn, cs;
-                        rope_sincos(pos, rp.inv_freq[8 * g + i], &sn, &cs);
+                        rope_sincos(pos, sfreq[8 * g + i], &sn, &cs);
                         float x0 = qa[i], x1 = qb[i];
                         qa[i] = x0 * cs - x1 * sn; qb[i] = x1 * cs + x0 * sn;
                         x0 = ka[i]; x1 = kb[i];
@@ -491,12 +496,12 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const void* __restrict__ alph
 #pragma unroll
                     for (int m = 0; m < 4; ++m) {   // pairs (c, c + 1) inside each 8-channel group
                         float sn, cs;
-                        rope_sincos(pos, rp.inv_freq[4 * g + m], &sn, &cs);
+                        rope_sincos(pos, sfreq[4 * g + m], &sn, &cs);
                         float x0 = qa[2 * m], x1 = qa[2 * m + 1];
                         qa[2 * m] = x0 * cs - x1 * sn; qa[2 * m + 1] = x1 * cs + x0 * sn;
                         x0 = ka[2 * m]; x1 = ka[2 * m + 1];
                         ka[2 * m] = x0 * cs - x1 * sn; ka[2 * m + 1] = x1 * cs + x0 * sn;
-                        rope_sincos(pos, rp.inv_freq[32 + 4 * g + m], &sn, &cs);
+                        rope_sincos(pos, sfreq[32 + 4 * g + m], &sn, &cs);
                         x0 = qb[2 * m]; x1 = qb[2 * m + 1];
                         qb[2 * m] = x0 * cs - x1 * sn; qb[2 * m + 1] = x1 * cs + x0 * sn;
                         x0 = kb[2 * m]; x1 = kb[2 * m + 1];

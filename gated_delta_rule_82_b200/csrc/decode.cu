@@ -52,6 +52,7 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
 
     __shared__ float sq[HPC][DK], sk[HPC][DK], sa[HPC][DK], sv[HPC][DV];
     __shared__ float sbeta[HPC], skq[HPC];
+    __shared__ double sfreq[DK / 2];   // RoPE inverse frequencies (lanes index them per channel)
     __shared__ float4 red_w[HPC][RG][C4], red_y[HPC][RG][C4];
 
     const int tid = threadIdx.x;
@@ -89,6 +90,8 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
         int g = blockIdx.x * HPC + hh;
         sv[hh][c] = g < NH ? to_f32(v[(size_t)g * DV + c]) : 0.f;
     }
+    if (rp.enabled)
+        for (int i = tid; i < DK / 2; i += kDecodeThreads) sfreq[i] = rp.inv_freq[i];
     if (tid < HPC) {
         int g = blockIdx.x * HPC + tid;
         const float bv = g < NH ? beta[g] : 0.f;
@@ -122,7 +125,7 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
                         i = c / 2; first = (c & 1) == 0; partner = c ^ 1;
                     }
                     float sn, cs;
-                    rope_sincos(p, rp.inv_freq[i], &sn, &cs);
+                    rope_sincos(p, sfreq[i], &sn, &cs);
                     float qp = sq[hh][partner], kp = sk[hh][partner];
                     qr[m] = first ? qr[m] * cs - qp * sn : qr[m] * cs + qp * sn;
                     kr[m] = first ? kr[m] * cs - kp * sn : kr[m] * cs + kp * sn;

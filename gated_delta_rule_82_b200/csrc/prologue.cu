@@ -34,11 +34,16 @@ qk_prologue_kernel(const T* __restrict__ q, const T* __restrict__ k, T* __restri
     const int tok0 = blockIdx.x * kTokPerCta;
     const int ntok = min(kTokPerCta, BT - tok0);
     if (rp.enabled) {
+        // inverse frequencies in shared memory (a per-lane index into the kernel-parameter
+        // array would serialise in the constant cache)
+        __shared__ double sfreq[HALF];
+        for (int i = threadIdx.x; i < HALF; i += blockDim.x) sfreq[i] = rp.inv_freq[i];
+        __syncthreads();
         for (int e = threadIdx.x; e < ntok * HALF; e += blockDim.x) {
             int j = e / HALF, i = e % HALF;
             int t = (tok0 + j) % T_len;
             float s, c;
-            rope_sincos(pos_offset + t, rp.inv_freq[i], &s, &c);
+            rope_sincos(pos_offset + t, sfreq[i], &s, &c);
             cs[j][i] = make_float2(c, s);
         }
         __syncthreads();

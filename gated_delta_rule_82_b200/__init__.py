@@ -203,15 +203,16 @@ def decode_step(q, k, v, alpha, beta, state, pos=None, *, l2norm=True, rope_thet
     return out
 
 
-def selftest_umma(A, B, b_mn_major=False):
+def selftest_umma(A, B, b_mn_major=False, a_tmem=False):
     """fp32 A @ B^T (b_mn_major=False, B [N, K]) or A @ B (B [K, N]) via the library's tcgen05
-    wrappers, for bf16 A [M, K] and B."""
+    wrappers, for bf16 A [M, K] and B; with a_tmem, A is staged into Tensor Memory first."""
     _check(A, "A", dtype=torch.bfloat16)
     _check(B, "B", dtype=torch.bfloat16)
     M, K = A.shape
     N = B.shape[1] if b_mn_major else B.shape[0]
     D = torch.empty((M, N), dtype=torch.float32, device=A.device)
-    st = _load().ckda_selftest_umma(_ptr(A), _ptr(B), _ptr(D), M, N, K, int(bool(b_mn_major)),
+    mode = int(bool(b_mn_major)) | (2 if a_tmem else 0)
+    st = _load().ckda_selftest_umma(_ptr(A), _ptr(B), _ptr(D), M, N, K, mode,
                                     _stream(A.device))
     _raise("ckda_selftest_umma", st)
     return D

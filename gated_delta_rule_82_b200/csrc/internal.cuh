@@ -31,6 +31,6 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
                             cudaStream_t stream);
 
 cudaError_t launch_umma_selftest(const void* A, const void* B, float* D, int M, int N, int K,
-                                 int b_mn_major, cudaStream_t stream);
+                                 int mode, cudaStream_t stream);
 
 }  // namespace ckda

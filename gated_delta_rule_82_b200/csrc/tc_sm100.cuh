@@ -191,6 +191,27 @@ __device__ __forceinline__ void mma_bf16_warp(uint32_t d_tmem, uint64_t adesc, u
         "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
         ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
 }
+// D[tmem] (+)= A[tmem] * B[smem], A (M = 128 rows in the TMEM lanes, K packed two bf16 per
+// 32-bit column) as staged by tmem_cp_128x256b; issued by a whole converged warp.
+__device__ __forceinline__ void mma_bf16_tmem_a_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                                     uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
+}
+// Copy a 128-row x 256-bit slice of a shared-memory matrix (described by an operand descriptor:
+// one 16-element K-step of a K-major bf16 tile) into TMEM at taddr (lane = row, 8 columns);
+// asynchronous, ordered with the issuing thread's tcgen05.mma.  Issued by a whole converged warp.
+__device__ __forceinline__ void tmem_cp_128x256b_warp(uint32_t taddr, uint64_t sdesc) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.cp.cta_group::1.128x256b [%0], %1;\n\t}"
+        ::"r"(taddr), "l"(sdesc) : "memory");
+}
 // Advance a shared-memory descriptor's start address by `bytes` (a multiple of 16; the start
 // field holds address / 16 in 14 bits and shared addresses stay below 256 KB, so no carry).
 __device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }

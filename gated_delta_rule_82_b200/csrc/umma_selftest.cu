@@ -11,11 +11,11 @@ namespace ckda {
 
 namespace {
 
-constexpr int kSelftestTmemCols = 256;
+constexpr int kSelftestTmemCols = 512;   // D (N <= 256 columns) + A staged in TMEM (K / 2 columns)
 
 __global__ void __launch_bounds__(128)
 umma_selftest_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16* __restrict__ B,
-                     float* __restrict__ D, int M, int N, int K, int b_mn) {
+                     float* __restrict__ D, int M, int N, int K, int b_mn, int a_tmem) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -56,7 +56,7 @@ umma_selftest_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16* _
     tc::tc_fence_after();
     const uint32_t tbase = tmem_base;
 
-    if (tid == 0) {
+    if (!a_tmem && tid == 0) {
         const uint32_t idesc = tc::idesc_bf16_f32(M, N, 0, b_mn);
         const uint32_t a0 = tc::smem_u32(sA), b0 = tc::smem_u32(sB);
         for (int ks = 0; ks < K / 16; ++ks) {
@@ -66,6 +66,20 @@ umma_selftest_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16* _
             tc::mma_bf16(tbase, ad, bd, idesc, ks > 0 ? 1u : 0u);
         }
         tc::mma_commit(&bar);
+    }
+    if (a_tmem && warp == 0) {
+        // A (M = 128) staged into TMEM columns 256.. by tcgen05.cp, one 16-element K-step per copy
+        const uint32_t idesc = tc::idesc_bf16_f32(M, N, 0, b_mn);
+        const uint32_t a0 = tc::smem_u32(sA), b0 = tc::smem_u32(sB);
+        const uint32_t ta = tbase + 256;
+        for (int ks = 0; ks < K / 16; ++ks)
+            tc::tmem_cp_128x256b_warp(ta + ks * 8, tc::smem_desc_sw128(a0 + (ks >> 2) * M * 128 + (ks & 3) * 32, 16, 1024));
+        for (int ks = 0; ks < K / 16; ++ks) {
+            uint64_t bd = b_mn ? tc::smem_desc_sw128(b0 + ks * 2048, K * 128, 1024)
+                               : tc::smem_desc_sw128(b0 + (ks >> 2) * N * 128 + (ks & 3) * 32, 16, 1024);
+            tc::mma_bf16_tmem_a_warp(tbase, ta + ks * 8, bd, idesc, ks > 0 ? 1u : 0u);
+        }
+        tc::mma_commit_warp(&bar);
     }
     tc::mbar_wait(&bar, 0, &abort_flag);
     tc::tc_fence_after();
@@ -89,7 +103,8 @@ umma_selftest_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16* _
 }  // namespace
 
 cudaError_t launch_umma_selftest(const void* A, const void* B, float* D, int M, int N, int K,
-                                 int b_mn_major, cudaStream_t stream) {
+                                 int mode, cudaStream_t stream) {
+    const int b_mn_major = mode & 1, a_tmem = (mode >> 1) & 1;
     // an MN-major B occupies whole 128-byte rows: ceil(N / 64) blocks of K rows
     const size_t b_bytes = b_mn_major ? (size_t)((N + 63) / 64) * K * 128 : (size_t)N * K * 2;
     size_t smem = (size_t)M * K * 2 + b_bytes + 1024;
@@ -98,7 +113,7 @@ cudaError_t launch_umma_selftest(const void* A, const void* B, float* D, int M, 
     if (e != cudaSuccess) return e;
     umma_selftest_kernel<<<1, 128, smem, stream>>>(static_cast<const __nv_bfloat16*>(A),
                                                    static_cast<const __nv_bfloat16*>(B), D, M, N,
-                                                   K, b_mn_major);
+                                                   K, b_mn_major, a_tmem);
     return cudaGetLastError();
 }
 

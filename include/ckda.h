@@ -160,8 +160,11 @@ CKDA_API ckda_status ckda_decode_step(const void* q, const void* k, const void* 
  * Diagnostic: D[M, N] (fp32, row-major) = A[M, K] * B for bf16 A (row-major, K contiguous),
  * computed by the library's own tcgen05 tensor-core wrappers (shared-memory operand
  * descriptors with the 128-byte swizzle, TMEM accumulator, one CTA).
- *   b_mn_major == 0: B is [N, K] row-major (K contiguous), D = A B^T  (K-major B operand)
- *   b_mn_major == 1: B is [K, N] row-major (N contiguous), D = A B    (MN-major B operand)
+ *   b_mn_major bit 0 clear: B is [N, K] row-major (K contiguous), D = A B^T  (K-major B operand)
+ *   b_mn_major bit 0 set:   B is [K, N] row-major (N contiguous), D = A B    (MN-major B operand)
+ *   b_mn_major bit 1 set:   A is staged from shared memory into Tensor Memory with
+ *                           tcgen05.cp and read by the product from there (M = 128 only)
+ *   other bits: CKDA_ERR_ARG.
  * M in {64, 128}; N a multiple of 16 in [16, 256] (32 or a multiple of 64 when b_mn_major);
  * K a multiple of 64 in [64, 256].  Lets a user check the tensor-core path on a device.
  */

@@ -205,13 +205,14 @@ def decode_step(q, k, v, alpha, beta, state, pos=None, *, l2norm=True, rope_thet
 
 def selftest_umma(A, B, b_mn_major=False, a_tmem=False):
     """fp32 A @ B^T (b_mn_major=False, B [N, K]) or A @ B (B [K, N]) via the library's tcgen05
-    wrappers, for bf16 A [M, K] and B; with a_tmem, A is staged into Tensor Memory first."""
+    wrappers, for bf16 A [M, K] and B.  a_tmem: False (A from shared memory), True or "cp" (A
+    copied into Tensor Memory by tcgen05.cp), "st" (A written into Tensor Memory by tcgen05.st)."""
     _check(A, "A", dtype=torch.bfloat16)
     _check(B, "B", dtype=torch.bfloat16)
     M, K = A.shape
     N = B.shape[1] if b_mn_major else B.shape[0]
     D = torch.empty((M, N), dtype=torch.float32, device=A.device)
-    mode = int(bool(b_mn_major)) | (2 if a_tmem else 0)
+    mode = int(bool(b_mn_major)) | (4 if a_tmem == "st" else 2 if a_tmem else 0)
     st = _load().ckda_selftest_umma(_ptr(A), _ptr(B), _ptr(D), M, N, K, mode,
                                     _stream(A.device))
     _raise("ckda_selftest_umma", st)

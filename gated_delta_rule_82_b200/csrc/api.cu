@@ -205,9 +205,9 @@ ckda_status ckda_selftest_umma(const void* A, const void* B, float* D, int M, in
     if (M != 64 && M != 128) return CKDA_ERR_UNSUPPORTED;
     if (N < 16 || N > 256 || N % 16) return CKDA_ERR_UNSUPPORTED;
     if (K < 64 || K > 256 || K % 64) return CKDA_ERR_UNSUPPORTED;
-    if (b_mn_major & ~3) return CKDA_ERR_ARG;
+    if ((b_mn_major & ~7) || (b_mn_major & 6) == 6) return CKDA_ERR_ARG;
     if ((b_mn_major & 1) && N % 64 && N != 32) return CKDA_ERR_UNSUPPORTED;
-    if ((b_mn_major & 2) && M != 128) return CKDA_ERR_UNSUPPORTED;
+    if ((b_mn_major & 6) && M != 128) return CKDA_ERR_UNSUPPORTED;
     if (!aligned16(A) || !aligned16(B) || !aligned16(D)) return CKDA_ERR_ALIGN;
     return from_cuda(launch_umma_selftest(A, B, D, M, N, K, b_mn_major,
                                           (cudaStream_t)stream));

@@ -27,23 +27,28 @@
 // stretches of tiny gates) takes an exact CUDA-core path for A and M instead, evaluating
 // g_r / g_j = exp2(L_r - L_j) from an fp32 log2 prefix with non-positive exponents only.
 //
-// Kernel 1 (ckda_tc_intra) -- persistent, one CTA of 512 threads per SM, loops over
-// (batch*head, chunk):
+// Factor role (ckda_tc_intra alone, or the factor CTAs of ckda_tc_fused) -- persistent, one CTA
+// of 512 threads per SM, loops over chunk-heads in head groups, chunk-major inside a group:
 //   A  global loads of the next chunk-head issued together (and the one after prefetched into
 //      L2); channel pass (thread per channel and 16-row block) forms the signed prefix gamma_r;
 //      row pass (thread per row and two 8-channel groups, a RoPE pair) rotates and normalises q, k,
 //      absorbs the signs and writes L, R, K_end with 16-byte stores.
 //   B  tcgen05: [A | M] = L R^T  (M = 128, N = 64, K = 128), read back by all 16 warps.
 //   C  T = (I + A)^-1 by blocked forward substitution in fp32; T' = T diag(beta) in bf16.
-//   D  tcgen05: [W | U~] = T' [K_gamma | V]  (M = 64, N = 2 x 128, MN-major B).
-//   F  tcgen05: M [W | U~] (M = 64) and K_end^T [W | U~] (M = 128, MN-major A).
-//   G  Q', O_loc, A_c, B_c staged in shared memory and written with three bulk (TMA) stores.
-// Kernel 2 (ckda_tc_state) -- one CTA per (batch*head, dv tile of 32 columns), serial over chunks:
-//   a three-stage pipeline of 1-D bulk (TMA) copies of each chunk's A_c, Q', B_c and O_loc; per
-//   chunk one tcgen05 product D_c = A_c S (M = 128, N = 32, K = 128) on the critical path, whose
-//   epilogue adds B_c to form the fp32 master state (one row per thread, in registers) and writes
-//   its bf16 copy for the next product, and one off-path product D_o = Q' S (M = 64) that becomes
-//   the chunk's output.
+//   D  tcgen05: W^T = K_gamma^T T'^T, U~^T = V^T T'^T (M = 128, N = 64).
+//   F  tcgen05: M W (M = 64) and U~^T M^T, K_end^T W, K_end^T U~ (M = 128).
+//   G  A_c, B_c^T and Q' staged in shared memory and written with bulk (TMA) stores, next to U~^T
+//      and M straight from the operand tiles; once they have landed the chunk-head's ready flag
+//      goes up.
+// State role (ckda_tc_state alone, or the chain CTAs of ckda_tc_fused) -- one CTA per head at a
+// time (all 128 dv columns), serial over its chunks, with the state transposed in Tensor Memory:
+// per chunk one tcgen05 product D_c^T = S^T A_c^T (M = 128, N = 128, K = 128) on the critical
+// path, whose epilogue adds B_c^T to form the next state (fp32, rounded to bf16 as the next
+// operand), and one off-path accumulation D_o^T = S^T Q'^T + U~^T M^T that becomes the chunk's
+// output.
+// The fused launch is cooperative (every CTA resident at once): a few chain CTAs follow the
+// ready flags of their heads while the factor CTAs produce them, so the serial pass hides behind
+// the chunk-parallel work instead of following it.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -54,18 +59,23 @@ namespace ckda {
 
 namespace {
 
-constexpr int kC = 64, kDK = 128, kDV = 128, kDVT = 32, kNTile = kDV / kDVT;
+constexpr int kC = 64, kDK = 128, kDV = 128;
 
 // ---- workspace image of one chunk-head (bytes) ------------------------------------------------
 constexpr uint32_t WS_AC = 0;          // A_c bf16, K-major swizzled, 128 rows x 128
-constexpr uint32_t WS_QP = 32768;      // Q'  bf16, K-major swizzled, 64 rows x 128
-constexpr uint32_t WS_TILES = 49152;   // per dv tile t: B_c [128][32] bf16, then O_loc [64][32] bf16
-// Both tile images have 64-byte rows whose four 16-byte chunks are swizzled by row, so that the
-// lanes of a warp reading (or writing) one chunk of 8 consecutive rows hit distinct banks.
-__host__ __device__ constexpr uint32_t bc_chunk(int row, int j) { return (uint32_t)((j ^ ((row >> 1) & 3)) << 4); }
-constexpr uint32_t WS_TILE = 12288;
-constexpr uint32_t WS_TILE_O = 8192;
-constexpr uint32_t WS_CHUNK = WS_TILES + kNTile * WS_TILE;  // 98304
+constexpr uint32_t WS_BC = 32768;      // B_c^T bf16 [128 dv rows][128], 16-byte chunks swizzled
+constexpr uint32_t WS_QP = 65536;      // Q'  bf16, K-major swizzled, 64 rows x 128
+constexpr uint32_t WS_UT = 81920;      // U~^T bf16, K-major swizzled, 128 dv rows x 64 tokens
+constexpr uint32_t WS_M = 98304;       // M bf16, K-major swizzled, 64 x 64
+constexpr uint32_t WS_CHUNK = 106496;
+// The state pass loads [WS_AC, WS_QP) for its chain product and [WS_QP, WS_CHUNK) for the output.
+constexpr uint32_t WS_CHAIN_BYTES = WS_QP - WS_AC, WS_OUT_BYTES = WS_CHUNK - WS_QP;
+// Chunk j of row r of B_c^T (16 chunks a row) sits at position j ^ (r % 8): the lanes of a warp
+// reading (or writing) one chunk of 8 consecutive rows hit eight distinct 16-byte bank groups.
+__host__ __device__ constexpr uint32_t bc_off(int row, int j) { return (uint32_t)(row * 256 + ((j ^ (row & 7)) << 4)); }
+// Ready flags: one 32-bit word per chunk-head after the images, set to 1 once the chunk-head's
+// images are complete in global memory (cleared before every forward).
+__host__ __device__ constexpr size_t flags_offset(size_t n_chunk_heads) { return n_chunk_heads * WS_CHUNK; }
 
 // ---- kernel 1 shared memory (bytes from a 1024-aligned base) ---------------------------------
 constexpr uint32_t S_G = 0;          // alpha (TMA), then the signed prefix gamma (fp32 [64][128])
@@ -88,9 +98,12 @@ constexpr uint32_t S_TB = S_R;               // T' bf16 K-major 64 x 64
 constexpr uint32_t S_X = S_R + 8192;         // X0, X1 fp32 [16][24] each
 constexpr uint32_t S_Y = S_R + 11264;        // Y fp32 [32][40]
 // staging of the chunk's workspace image, over buffers that are dead by then
-constexpr uint32_t S_OUT_AC = S_W;   // A_c image (32 KB, over W and U)
-constexpr uint32_t S_OUT_QP = S_R;   // Q' image (16 KB)
-constexpr uint32_t S_OUT_TL = S_KE;  // dv tiles (48 KB, over K_end, M, A and part of T)
+// (U~^T and M are stored straight from S_U and S_M)
+constexpr uint32_t S_OUT_QP = S_R;            // Q' image (16 KB)
+constexpr uint32_t S_OUT_BC0 = S_KE;          // B_c^T rows 0..63 (16 KB, over K_end)
+constexpr uint32_t S_OUT_AC = S_A;            // A_c image (32 KB, over A and part of T)
+constexpr uint32_t S_OUT_BC1 = S_A + 32768;   // B_c^T rows 64..127 (16 KB, over T and part of W)
+static_assert(S_OUT_BC1 + 16384 <= S_U, "staging must stay clear of U~^T");
 // small arrays
 constexpr uint32_t SM_P = S_SM;                  // signed block totals of alpha, fp32 [4][128]
 constexpr uint32_t SM_GC = S_SM + 2048;          // gamma_C fp32 [128] (signed)
@@ -151,10 +164,10 @@ __device__ __forceinline__ float select_lane(const float* v, int lane) {
 
 __device__ int g_tc_error;  // nonzero after a bounded wait ran out (diagnostic)
 
-// Tensor maps of one forward call: q, k, v (bf16) and alpha (fp32) as 4-D arrays
-// {channel, head, token, batch}; boxes of 64 tokens of one (batch, head).
+// Tensor maps of one forward call: q, k, v (bf16), alpha (fp32, or bf16 logits) and out (bf16)
+// as 4-D arrays {channel, head, token, batch}; boxes of 64 tokens of one (batch, head).
 struct TcMaps {
-    CUtensorMap q, k, v, alpha;
+    CUtensorMap q, k, v, alpha, out;
 };
 
 // Issue the TMA loads of chunk-head ci: alpha -> G, q -> QR, k -> KR on bar_in; V (two 64-column
@@ -331,16 +344,71 @@ __device__ __forceinline__ void t_solve(const float* sA, float* sT, const float*
     }
 }
 
+// Order in which the factor role visits the chunk-heads: heads in groups of G, and inside a
+// group chunk by chunk (chunk c of every head of the group before chunk c + 1), so that the serial
+// chains of a group, which consume their chunks in order, can run behind the factor work.  Item i
+// maps to the chunk-head ci = bh * NT + c of the workspace.
+struct WorkOrder {
+    int NT, BH, G;
+    __device__ __forceinline__ int ci(int i) const {
+        const int per = G * NT;
+        const int g = i / per, r = i - g * per;
+        const int gs = min(G, BH - g * G);
+        const int c = r / gs;
+        return (g * G + (r - c * gs)) * NT + c;
+    }
+};
+
+// Ready flags.  The writer waits for its bulk stores to complete, orders them before the flag
+// (proxy fence, then a release store at GPU scope); a reader acquires the flag and fences before
+// its own bulk (async-proxy) loads of the images.
+__device__ __forceinline__ void publish_ready(int* flag) {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(flag), "r"(1u) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire(const int* flag) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+// Waits of the state role can last as long as the factor role takes to produce a head group
+// (milliseconds on long sequences), so they are bounded by time rather than by a poll count.
+constexpr uint64_t kLongWaitNs = 4000000000ull;   // 4 s
+__device__ __forceinline__ bool flag_wait(const int* flag, volatile int* abort) {
+    const uint64_t t0 = global_ns();
+    for (;;) {
+        if (ld_acquire(flag) != 0) {
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            return true;
+        }
+        if (*abort) return false;
+        if (global_ns() - t0 > kLongWaitNs) { *abort = 1; return false; }
+        __nanosleep(256);
+    }
+}
+__device__ __forceinline__ bool mbar_wait_long(uint64_t* bar, uint32_t parity, volatile int* abort) {
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 0;; ++i) {
+        if (tc::mbar_try_wait(bar, parity)) return true;
+        if (*abort) return false;
+        if ((i & 255) == 255 && global_ns() - t0 > kLongWaitNs) { *abort = 1; return false; }
+    }
+}
+
+// ---- the factor role: chunk-heads wo.ci(i) for i = rank, rank + nprog, ... ----------------------
 // kLogits: alpha and beta hold logits (alpha = 2 sigma(a) - 1 from bf16 a, beta = 2 sigma(b)).
 template <bool kLogits>
-__global__ void __launch_bounds__(512, 1)
-ckda_tc_intra(const __grid_constant__ TcMaps maps, const void* __restrict__ alpha,
-              const float* __restrict__ beta, uint8_t* __restrict__ ws, int T_len, int H, int NT,
-              int total, int l2norm, RopeParams rp, long long pos_offset) {
+__device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, const void* __restrict__ alpha,
+                                           const float* __restrict__ beta, uint8_t* __restrict__ ws,
+                                           int* __restrict__ flags, int T_len, int H, int NT, int total,
+                                           WorkOrder wo, int rank, int nprog, int l2norm,
+                                           const RopeParams& rp, long long pos_offset) {
     constexpr int gate_logits = kLogits ? 1 : 0;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float* G = reinterpret_cast<float*>(sm + S_G);
     float* gP = reinterpret_cast<float*>(sm + SM_P);
     float* gGC = reinterpret_cast<float*>(sm + SM_GC);
@@ -388,23 +456,25 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const void* __restrict__ alph
     // the set-up above may overlap the previous kernel in the stream; from here on the kernel
     // reads the caller's inputs and writes the workspace, so it waits for that kernel
     tc::grid_dependency_wait();
-    if (tid == 0 && (int)blockIdx.x < total) {
+    if (tid == 0 && rank < total) {
         tc::prefetch_tensormap(&maps.q);
         tc::prefetch_tensormap(&maps.k);
         tc::prefetch_tensormap(&maps.v);
         tc::prefetch_tensormap(&maps.alpha);
-        issue_inputs(maps, sm, bar_in, blockIdx.x, NT, H, gate_logits);
-        issue_v(maps, sm, bar_v, blockIdx.x, NT, H);
+        issue_inputs(maps, sm, bar_in, wo.ci(rank), NT, H, gate_logits);
+        issue_v(maps, sm, bar_v, wo.ci(rank), NT, H);
     }
 
-    // persistent loop over chunk-heads ci = (batch*head) * NT + chunk
+    // persistent loop over items; chunk-head ci = (batch*head) * NT + chunk
     uint32_t it = 0;
-    for (int ci = blockIdx.x; ci < total; ci += gridDim.x, ++it) {
+    int pending = -1;   // chunk-head whose images are stored but not yet flagged ready
+    for (int i = rank; i < total; i += nprog, ++it) {
+        const int ci = wo.ci(i);
         const int ch = ci % NT, bh = ci / NT;
         const int h = bh % H;
         const int t0 = ch * kC;
         const int nvalid = min(kC, T_len - t0);
-        const int nci = ci + gridDim.x;
+        const int nci = i + nprog < total ? wo.ci(i + nprog) : -1;
         uint8_t* wsc = ws + (size_t)ci * WS_CHUNK;
         const size_t row0 = ((size_t)(bh / H) * T_len + t0) * H + h;
         float bval = (tid < 64 && tid < nvalid) ? beta[row0 + tid * rs] : 0.f;
@@ -560,7 +630,7 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const void* __restrict__ alph
         tc::tc_fence_after();
         // alpha, q, k of this chunk-head are consumed: bring in the next one's.  Issued by warp 15
         // (a TMA issue costs its thread several hundred cycles) while warp 0 issues the product.
-        if (tid == 480 && nci < total) issue_inputs(maps, sm, bar_in, nci, NT, H, gate_logits);
+        if (tid == 480 && nci >= 0) issue_inputs(maps, sm, bar_in, nci, NT, H, gate_logits);
         if (!exact) {
             // ======== B: [A | M] = L R^T on the tensor cores (M = 128, N = 64, K = 128) ========
             if (warp == 0) {
@@ -573,6 +643,14 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const void* __restrict__ alph
                                       tc::desc_add(bd, (ks >> 2) * 8192 + (ks & 3) * 32), idesc, ks > 0);
                 tc::mma_commit_warp(bar);
             }
+        }
+        // the previous chunk-head's stores have had a whole row pass to land: flag it ready
+        if (pending >= 0) {
+            if (tid == 0) {
+                tc::bulk_wait_all();
+                publish_ready(flags + pending);
+            }
+            pending = -1;
         }
         if (!exact) {
             tc::mbar_wait(bar, phase & 1, abort_flag);
@@ -700,35 +778,34 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const void* __restrict__ alph
         __syncthreads();
         tc::tc_fence_after();
 
-        // ======== F: M W (M = 64) -> Q', U~^T M^T (M = 128) -> O_loc^T,
-        //             K_end^T W (M = 128) -> A_c, K_end^T U~ (M = 128) -> B_c ========
+        // ======== F: M W (M = 64) -> Q', K_end^T W (M = 128) -> A_c,
+        //             U~^T K_end (M = 128) -> B_c^T ========
+        // (the chunk's own output M U~ is left to the state pass, which accumulates it in fp32
+        // next to Q' S0 from the U~^T and M images)
         if (warp == 0) {
             const uint64_t md = tc::smem_desc_sw128(tc::smem_u32(sm + S_M), 16, 1024);
             const uint64_t ked = tc::smem_desc_sw128(tc::smem_u32(sm + S_KE), 8192, 1024);
             const uint64_t wd = tc::smem_desc_sw128(tc::smem_u32(sm + S_W), 16, 1024);
             const uint64_t ud = tc::smem_desc_sw128(tc::smem_u32(sm + S_U), 16, 1024);
             const uint32_t id_q = tc::idesc_bf16_f32(64, 128, 0, 0);
-            const uint32_t id_o = tc::idesc_bf16_f32(128, 64, 0, 0);
             const uint32_t id_c = tc::idesc_bf16_f32(128, 128, 1, 0);
-            // product by product, M W first: the Q' read-back overlaps the other three
+            const uint32_t id_b = tc::idesc_bf16_f32(128, 128, 0, 1);
+            // product by product, M W first: the Q' read-back overlaps the other two
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)                                  // M W
                 tc::mma_bf16_warp(tmem, tc::desc_add(md, ks * 32), tc::desc_add(wd, ks * 32), id_q, ks > 0);
             tc::mma_commit_warp(bar_q);
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)                                  // U~^T M^T
-                tc::mma_bf16_warp(tmem + 128, tc::desc_add(ud, ks * 32), tc::desc_add(md, ks * 32), id_o, ks > 0);
-#pragma unroll
             for (int ks = 0; ks < 4; ++ks)                                  // K_end^T W
                 tc::mma_bf16_warp(tmem + 192, tc::desc_add(ked, ks * 2048), tc::desc_add(wd, ks * 32), id_c, ks > 0);
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)                                  // K_end^T U~
-                tc::mma_bf16_warp(tmem + 320, tc::desc_add(ked, ks * 2048), tc::desc_add(ud, ks * 32), id_c, ks > 0);
+            for (int ks = 0; ks < 4; ++ks)                                  // U~^T K_end
+                tc::mma_bf16_warp(tmem + 320, tc::desc_add(ud, ks * 32), tc::desc_add(ked, ks * 2048), id_b, ks > 0);
             tc::mma_commit_warp(bar);
         }
         // V of this chunk-head was consumed by the W/U~ products: bring in the next one's, from
         // warp 14 while warp 0 issues these products
-        if (tid == 448 && nci < total) issue_v(maps, sm, bar_v, nci, NT, H);
+        if (tid == 448 && nci >= 0) issue_v(maps, sm, bar_v, nci, NT, H);
         tc::mbar_wait(bar_q, it & 1, abort_flag);
         tc::tc_fence_after();
         // ======== G: results into shared staging images, then bulk stores in two groups ========
@@ -751,26 +828,12 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const void* __restrict__ alph
                     }
                 }
             }
-            // (2) M = 128 products, lane = row c' (A_c, B_c) or dv column (O_loc^T)
+            // (2) M = 128 products, lane = row c' (A_c) or dv column (B_c^T)
             tc::mbar_wait(bar, phase & 1, abort_flag);
             ++phase;
             tc::tc_fence_after();
             {
                 const int cr = 32 * quarter + lane;
-                // O_loc^T: tokens 16 slice .. 16 slice + 15 of dv column cr -> tile cr / 32, stored
-                // as O_loc rows [64 tokens][32 dv] (the lanes of a warp fill 64 contiguous bytes of
-                // one token row per store)
-                {
-                    float x[16];
-                    tc::tmem_ld16_sync(tc::tmem_addr(tmem, 32 * quarter, 128 + 16 * slice), x);
-                    const int nc = cr & 31;
-                    uint8_t* o = sm + S_OUT_TL + (cr >> 5) * WS_TILE + WS_TILE_O + (nc & 7) * 2;
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int r = 16 * slice + i;
-                        st_bf16(o, r * 64 + bc_chunk(r, nc >> 3), x[i]);
-                    }
-                }
                 const int n0 = 64 * (slice & 1);
                 const float gc = gGC[cr];
                 float x[64];
@@ -784,7 +847,8 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const void* __restrict__ alph
                         for (int i = 0; i < 8; ++i) y[i] = -x[c0 + i];
                         st16(sm + S_OUT_AC, tc::sw128_kmajor(cr, n, 128), y);
                     } else {
-                        st16(sm + S_OUT_TL, (n >> 5) * WS_TILE + cr * 64 + bc_chunk(cr, (n & 31) >> 3), x + c0);
+                        // rows 0..63 over K_end, rows 64..127 in the second staging half
+                        st16(sm + (quarter < 2 ? S_OUT_BC0 : S_OUT_BC1 - 16384), bc_off(cr, n >> 3), x + c0);
                     }
                 }
                 // A_c = Diag(gamma_C) - K_end^T W: row c' holds its diagonal element in this slice
@@ -800,97 +864,101 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const void* __restrict__ alph
         __syncthreads();
         tc::tc_fence_after();
         if (tid == 0) {
-            // group 1: the images over buffers the next row pass rewrites first
+            // group 1: the images over buffers the next row pass rewrites first (Q' over R,
+            // the first half of B_c^T over K_end)
             tc::bulk_s2g(wsc + WS_QP, sm + S_OUT_QP, 16384);
-            tc::bulk_s2g(wsc + WS_TILES, sm + S_OUT_TL, 2 * WS_TILE);
+            tc::bulk_s2g(wsc + WS_BC, sm + S_OUT_BC0, 16384);
             tc::bulk_commit();
-            // group 2: the rest
-            tc::bulk_s2g(wsc + WS_TILES + 2 * WS_TILE, sm + S_OUT_TL + 2 * WS_TILE, 2 * WS_TILE);
+            // group 2: the rest, U~^T and M straight from the product operands
             tc::bulk_s2g(wsc + WS_AC, sm + S_OUT_AC, 32768);
+            tc::bulk_s2g(wsc + WS_BC + 16384, sm + S_OUT_BC1, 16384);
+            tc::bulk_s2g(wsc + WS_UT, sm + S_U, 16384);
+            tc::bulk_s2g(wsc + WS_M, sm + S_M, 8192);
             tc::bulk_commit();
         }
+        pending = ci;
     }
-    if (tid == 0) tc::bulk_wait_all();
+    if (tid == 0) {
+        tc::bulk_wait_all();
+        if (pending >= 0) publish_ready(flags + pending);
+    }
     tc::tc_fence_before();
     __syncthreads();
     if (*abort_flag && tid == 0) atomicExch(&g_tc_error, 1);
     if (warp == 0) tc::tmem_dealloc(tmem, 512);
 }
 
-// ---- kernel 2: the serial state pass ------------------------------------------------------------
-// Warp roles (384 threads):
-//   warps 0-3   chain epilogue: thread t owns state row t; S_next = D_c + B_c in fp32 registers,
-//               written back as the bf16 B operand of the next product
-//   warp 4      chain issue: D_c = A_c S (M = 128, N = 32)
-//   warp 5      chain loads: A_c and B_c of each chunk (1-D bulk copies, three stages)
-//   warp 6      output loads: Q' and O_loc of each chunk (three stages)
-//   warp 7      output issue: D_o = Q' S (M = 64, N = 32)
-//   warps 8-11  output epilogue: O = scale (D_o + O_loc), rows in the M = 64 layout
-// Only the first three roles are on the serial path; the output side runs behind it and never
-// holds a chain stage: the output product of chunk c is issued when the chain product of chunk c
-// has completed, i.e. while the chain epilogue forms S_{c+1}.  S rotates through four shared-memory buffers: S_{c+4} is written only
-// after the output product of chunk c has read S_c.  Every role issues from a converged warp
-// (one elected lane) and every wait is bounded and ends warp-uniformly.
-constexpr int kStages = 3;
-constexpr int kOutBufs = 4;
-constexpr int kSBufs = 4;
-constexpr uint32_t P2_CSTAGE = 40960;                    // A_c 32 KB, B_c 8 KB
-constexpr uint32_t P2_AC = 0, P2_BC = 32768;
-constexpr uint32_t P2_OSTAGE = 20480;                    // Q' 16 KB, O_loc 4 KB
-constexpr uint32_t P2_QP = 0, P2_OL = 16384;
-constexpr uint32_t P2_OBASE = kStages * P2_CSTAGE;
-// S operands: four MN-major buffers of 128 K-rows x 32 dv, two per 16 KB tile (dv columns 0..31
-// and 32..63 of the swizzled 128-byte rows)
-constexpr uint32_t P2_ST = P2_OBASE + kStages * P2_OSTAGE;
-constexpr uint32_t P2_ST_BYTES = 16384;
-constexpr uint32_t P2_SM = P2_ST + 2 * P2_ST_BYTES;
-constexpr uint32_t P2_BYTES = P2_SM + 512 + 1024;
-constexpr int kStateThreads = 384;
-__device__ __forceinline__ uint32_t s_tile(int buf) { return (uint32_t)(buf >> 1) * P2_ST_BYTES; }
-__device__ __forceinline__ int s_col(int buf) { return 32 * (buf & 1); }
+// ---- the state role: the serial pass over the chunks of heads head0, head0 + hstride, ... ---------
+// One CTA of 512 threads carries whole heads (all 128 dv columns), one head after the other; its
+// items u = k NT + c run over (head k of the CTA, chunk c).  The state is kept transposed: S^T
+// (dv x dk) lives in Tensor Memory as the A operand of both products,
+//     D_c^T = S^T A_c^T  (M = 128 dv, N = 128, K = 128)           -> S_next^T = D_c^T + B_c^T
+//     D_o^T = S^T Q'^T + U~^T M^T  (M = 128 dv, N = 64 tokens)     -> O^T = scale D_o^T
+// so the chunk's own output M U~ is accumulated in fp32 next to Q' S0 and never rounded.
+// Warp roles:
+//   warps 0-7    chain epilogue: warp w owns dv columns 32 (w % 4) .. + 31 (its TMEM lanes) and
+//                state rows 64 (w / 4) .. + 63; S_next^T in fp32, written back into TMEM as the
+//                bf16 operand of the next products (hT in fp32 after a head's last chunk)
+//   warp 8       chain issue
+//   warp 9       output issue
+//   warp 10      chain loads: A_c and B_c^T of each item (one 64 KB bulk copy, two stages)
+//   warp 11      output loads: Q', U~^T and M of each item (one 40 KB bulk copy, two stages)
+//   warps 12-15  output epilogue: lane = dv column; the chunk's 64 x 128 output tile goes through
+//                a shared-memory staging tile and leaves with one tensor (TMA) store
+// Only the chain roles are on the serial path.  The output product of item u is issued once the
+// chain product of item u has completed, so it runs while the chain epilogue works.  S^T
+// alternates between two TMEM buffers: S_{u+1}^T goes into the buffer of S_{u-1}^T once the
+// output product of item u - 1 has read it.  Every load of an item waits for the item's ready
+// flag, every role issues from a converged warp (one elected lane) and every wait is bounded.
+constexpr uint32_t SS_C = 0;             // chain stages: A_c (32 KB) then B_c^T (32 KB)
+constexpr uint32_t SS_CSTAGE = WS_CHAIN_BYTES;
+constexpr uint32_t SS_O = 2 * SS_CSTAGE; // output stages: Q' (16 KB), U~^T (16 KB), M (8 KB)
+constexpr uint32_t SS_OSTAGE = WS_OUT_BYTES;
+constexpr uint32_t SS_STG = SS_O + 2 * SS_OSTAGE;   // output tile bf16 [64 tokens][128 dv]
+constexpr uint32_t SS_BAR = SS_STG + 16384;
+constexpr uint32_t SS_BYTES = SS_BAR + 256 + 1024;
+constexpr uint32_t FUSED_BYTES = SS_BYTES > S_BYTES ? SS_BYTES : S_BYTES;
+static_assert(SS_OSTAGE % 1024 == 0 && (WS_UT - WS_QP) % 1024 == 0 && (WS_M - WS_QP) % 1024 == 0,
+              "operand tiles of a stage must stay 1024-byte aligned");
+// TMEM columns: D_c^T 0..127, S^T buffers of 64 (bf16 pairs) from 128, D_o^T buffers of 64 from 256
+constexpr uint32_t kColS = 128, kColO = 256;
 
-__global__ void __launch_bounds__(kStateThreads, 1)
-ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
-              __nv_bfloat16* __restrict__ out, float* __restrict__ hT, int T_len, int H, int NT,
-              float scale) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full_c = reinterpret_cast<uint64_t*>(sm + P2_SM);  // [kStages]
-    uint64_t* empty_c = full_c + kStages;                        // [kStages]
-    uint64_t* full_o = empty_c + kStages;                        // [kStages]
-    uint64_t* empty_o = full_o + kStages;                        // [kStages]
-    uint64_t* mma_c = empty_o + kStages;                         // D_c complete
-    uint64_t* s_ready = mma_c + 1;                               // [kSBufs] S buffer written
-    uint64_t* mma_o = s_ready + kSBufs;                          // [kOutBufs] D_o complete
-    uint64_t* o_free = mma_o + kOutBufs;                         // [kOutBufs] D_o read back
-    uint64_t* dc_done = o_free + kOutBufs;                       // [kSBufs] D_c(c) complete
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(dc_done + kSBufs);
+__device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, const uint8_t* __restrict__ ws,
+                                           const int* __restrict__ flags, const float* __restrict__ h0,
+                                           __nv_bfloat16* __restrict__ out, float* __restrict__ hT,
+                                           int T_len, int H, int NT, int BH, float scale, int head0,
+                                           int hstride) {
+    uint64_t* full_c = reinterpret_cast<uint64_t*>(sm + SS_BAR);   // [2] A_c, B_c^T landed
+    uint64_t* empty_c = full_c + 2;     // [2] chain stage consumed (8 epilogue warps)
+    uint64_t* full_o = empty_c + 2;     // [2] Q', U~^T, M landed
+    uint64_t* empty_o = full_o + 2;     // [2] output stage read by the output product (commit)
+    uint64_t* mma_c = empty_o + 2;      // D_c^T complete
+    uint64_t* s_ready = mma_c + 1;      // [2] S^T buffer written (8 epilogue warps)
+    uint64_t* dc_done = s_ready + 2;    // [2] D_c^T of the item using S^T buffer b complete
+    uint64_t* mma_o = dc_done + 2;      // [4] D_o^T complete
+    uint64_t* o_free = mma_o + 4;       // [4] D_o^T read back (4 output-epilogue warps)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_free + 4);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int tile = blockIdx.x % kNTile, bh = blockIdx.x / kNTile;
-    const int b = bh / H, h = bh % H;
-    const int n0 = tile * kDVT;
-    const uint8_t* wsh = ws + (size_t)bh * NT * WS_CHUNK;
+    const int nheads = head0 < BH ? (BH - head0 + hstride - 1) / hstride : 0;
+    const int U = nheads * NT;
 
     if (warp == 0) {
-        tc::tmem_alloc(tmem_slot, 256);
+        tc::tmem_alloc(tmem_slot, 512);
         tc::tmem_relinquish();
     }
     if (tid == 32) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < 2; ++s) {
             tc::mbar_init(&full_c[s], 1);
-            tc::mbar_init(&empty_c[s], 4);   // one arrival per chain-epilogue warp
+            tc::mbar_init(&empty_c[s], 8);
             tc::mbar_init(&full_o[s], 1);
-            tc::mbar_init(&empty_o[s], 4);   // one arrival per output-epilogue warp
-        }
-        tc::mbar_init(mma_c, 1);
-        for (int s = 0; s < kSBufs; ++s) {
-            tc::mbar_init(&s_ready[s], 4);
+            tc::mbar_init(&empty_o[s], 1);
+            tc::mbar_init(&s_ready[s], 8);
             tc::mbar_init(&dc_done[s], 1);
         }
-        for (int s = 0; s < kOutBufs; ++s) {
+        tc::mbar_init(mma_c, 1);
+        for (int s = 0; s < 4; ++s) {
             tc::mbar_init(&mma_o[s], 1);
             tc::mbar_init(&o_free[s], 4);
         }
@@ -900,190 +968,238 @@ ckda_tc_state(const uint8_t* __restrict__ ws, const float* __restrict__ h0,
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
-    // set-up above may overlap the factor kernel's tail; everything below reads its workspace
-    // or touches caller memory, so it waits for that grid to complete
+    // a launch after the factor kernel waits for it here (no effect otherwise)
     tc::grid_dependency_wait();
-    tc::grid_launch_dependents();   // a following kernel may start its set-up early
+    tc::grid_launch_dependents();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t dc = tmem;                 // D_c: 128 lanes x 32 columns
-    const uint32_t dob = tmem + 32;           // D_o: kOutBufs buffers of 32 columns (M = 64 layout)
     auto wait = [&](uint64_t* bar, uint32_t parity) {
-        return __all_sync(0xffffffffu, tc::mbar_wait(bar, parity, abort_flag));
+        return __all_sync(0xffffffffu, mbar_wait_long(bar, parity, abort_flag));
     };
-    const uint64_t s_desc0 = tc::smem_desc_sw128(tc::smem_u32(sm + P2_ST), P2_ST_BYTES, 1024);
-    auto s_desc = [&](int c) { return tc::desc_add(s_desc0, s_tile(c % kSBufs) + 2 * s_col(c % kSBufs)); };
+    auto item_bh = [&](int u) { return head0 + (u / NT) * hstride; };
 
-    if (warp < 4) {
-        // ---- chain epilogue: thread t owns state row t (TMEM lane t of D_c) ----
-        const int t = tid;
-        float S[kDVT];
-        if (h0) {
-            const float4* src = reinterpret_cast<const float4*>(h0 + ((size_t)bh * kDK + t) * kDV + n0);
+    if (warp < 8) {
+        // ---- chain epilogue: lane = dv column n, state rows cb .. cb + 63 ----
+        const int q = warp & 3, hf = warp >> 2;
+        const int n = 32 * q + lane, cb = 64 * hf;
+        float S[64];   // S[j] = S(cb + j, n)
+        auto load_h0 = [&](int bh) {
+            if (h0) {
+                const float* src = h0 + ((size_t)bh * kDK + cb) * kDV + n;
 #pragma unroll
-            for (int j = 0; j < kDVT / 4; ++j) {
-                float4 x = src[j];
-                S[4 * j] = x.x; S[4 * j + 1] = x.y; S[4 * j + 2] = x.z; S[4 * j + 3] = x.w;
+                for (int j = 0; j < 64; ++j) S[j] = src[(size_t)j * kDV];
+            } else {
+#pragma unroll
+                for (int j = 0; j < 64; ++j) S[j] = 0.f;
             }
-        } else {
+        };
+        // S^T as the TMEM A operand: lane n, column 32 hf + j holds rows cb + 2j, cb + 2j + 1
+        auto put_s = [&](int u) {
+            uint32_t v[32];
 #pragma unroll
-            for (int j = 0; j < kDVT; ++j) S[j] = 0.f;
-        }
-        // S as an MN-major B operand: K-row t holds the 32 dv values of state row t
-        auto put_s = [&](int c) {
-            const int buf = c % kSBufs;
-            uint8_t* dst = sm + P2_ST + s_tile(buf);
-#pragma unroll
-            for (int j = 0; j < kDVT; j += 8) st16(dst, tc::sw128_mnmajor(t, s_col(buf) + j, kDK), S + j);
-            tc::fence_proxy_async_smem();
+            for (int j = 0; j < 32; ++j) v[j] = pack_bf16(S[2 * j], S[2 * j + 1]);
+            tc::tmem_st32(tc::tmem_addr(tmem + kColS + 64 * (u & 1) + 32 * hf, 32 * q, 0), v);
+            tc::tmem_st_wait();
             tc::tc_fence_before();
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&s_ready[buf]);
+            if (lane == 0) tc::mbar_arrive(&s_ready[u & 1]);
         };
-        put_s(0);
-        for (int ch = 0; ch < NT; ++ch) {
-            const int st = ch % kStages;
-            // B_c is in registers before the chain product completes
-            if (!wait(&full_c[st], (ch / kStages) & 1)) break;
-            uint4 bc[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                bc[j] = *reinterpret_cast<const uint4*>(sm + st * P2_CSTAGE + P2_BC + t * 64 + bc_chunk(t, j));
-            // buffer (ch + 1) % 4 last held S_{ch-3}: its output product must be done (checked
-            // before the chain product completes, off the serial path)
-            if (ch + 1 < NT && ch + 1 >= kSBufs &&
-                !wait(&mma_o[(ch - 3) % kOutBufs], ((ch - 3) / kOutBufs) & 1))
-                break;
-            if (!wait(mma_c, ch & 1)) break;
-            if (tid == 0) tc::mbar_arrive(&dc_done[ch % kSBufs]);   // the output product may run
+        if (U > 0) {
+            load_h0(item_bh(0));
+            put_s(0);
+        }
+        for (int u = 0; u < U; ++u) {
+            const int st = u & 1;
+            if (!wait(&full_c[st], (u >> 1) & 1)) break;
+            if (!wait(mma_c, u & 1)) break;
             tc::tc_fence_after();
-            float d[32];
-            tc::tmem_ld32_sync(tc::tmem_addr(dc, 32 * warp, 0), d);
+            tc::tmem_ld64_sync(tc::tmem_addr(tmem, 32 * q, cb), S);
+            const uint8_t* bcs = sm + SS_C + st * SS_CSTAGE + (WS_BC - WS_AC);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int j = 0; j < 8; ++j) {
                 float y[8];
-                unpack8(bc[j], y);
+                unpack8(*reinterpret_cast<const uint4*>(bcs + bc_off(n, 8 * hf + j)), y);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) S[8 * j + i] = d[8 * j + i] + y[i];
+                for (int i = 0; i < 8; ++i) S[8 * j + i] += y[i];
             }
-            if (ch + 1 < NT) put_s(ch + 1);
-            else tc::tc_fence_before();
-            // A_c was read (D_c done) and B_c is in registers: release the chain stage
+            // A_c was read by the finished product and B_c^T is in registers: release the stage
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&empty_c[st]);
-        }
-        if (hT && !*abort_flag) {
-            float4* dst = reinterpret_cast<float4*>(hT + ((size_t)bh * kDK + t) * kDV + n0);
+            const bool last = u % NT == NT - 1;
+            if (last && hT && !*abort_flag) {
+                float* dst = hT + ((size_t)item_bh(u) * kDK + cb) * kDV + n;
 #pragma unroll
-            for (int j = 0; j < kDVT / 4; ++j)
-                dst[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
+                for (int j = 0; j < 64; ++j) dst[(size_t)j * kDV] = S[j];
+            }
+            if (u + 1 < U) {
+                // the buffer of S_{u+1}^T held S_{u-1}^T: the output product of item u - 1 must
+                // be done with it
+                if (u >= 1 && !wait(&mma_o[(u - 1) & 3], ((u - 1) >> 2) & 1)) break;
+                if (last) load_h0(item_bh(u + 1));
+                put_s(u + 1);
+            } else {
+                tc::tc_fence_before();
+            }
         }
-    } else if (warp == 4) {
-        // ---- chain issue ----
-        const uint32_t idc = tc::idesc_bf16_f32(128, kDVT, 0, 1);
-        const uint64_t c_desc0 = tc::smem_desc_sw128(tc::smem_u32(sm), 16, 1024);
-        for (int ch = 0; ch < NT; ++ch) {
-            const int st = ch % kStages;
-            if (!wait(&full_c[st], (ch / kStages) & 1)) break;
-            if (!wait(&s_ready[ch % kSBufs], (ch / kSBufs) & 1)) break;
+    } else if (warp == 8) {
+        // ---- chain issue: A = S^T (TMEM), B = A_c^T (the K-major A_c image read as K-major B) ----
+        const uint32_t idc = tc::idesc_bf16_f32(128, 128, 0, 0);
+        const uint64_t c_desc0 = tc::smem_desc_sw128(tc::smem_u32(sm + SS_C), 16, 1024);
+        for (int u = 0; u < U; ++u) {
+            const int st = u & 1;
+            if (!wait(&full_c[st], (u >> 1) & 1)) break;
+            if (!wait(&s_ready[st], (u >> 1) & 1)) break;
             tc::tc_fence_after();
-            const uint64_t ad = tc::desc_add(c_desc0, st * P2_CSTAGE + P2_AC);
-            const uint64_t sd = s_desc(ch);
+            const uint64_t bd = tc::desc_add(c_desc0, st * SS_CSTAGE);
+            const uint32_t a = tmem + kColS + 64 * st;
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
-                tc::mma_bf16_warp(dc, tc::desc_add(ad, (ks >> 2) * 16384 + (ks & 3) * 32),
-                                  tc::desc_add(sd, ks * 2048), idc, ks > 0 ? 1u : 0u);
+                tc::mma_bf16_tmem_a_warp(tmem, a + 8 * ks, tc::desc_add(bd, (ks >> 2) * 16384 + (ks & 3) * 32),
+                                         idc, ks > 0 ? 1u : 0u);
             tc::mma_commit_warp(mma_c);
+            tc::mma_commit_warp(&dc_done[st]);
         }
-    } else if (warp == 5 || warp == 6) {
-        // ---- loads: warp 5 the chain ring (A_c, B_c), warp 6 the output ring (Q', O_loc) ----
+    } else if (warp == 9) {
+        // ---- output issue: S^T Q'^T (A in TMEM) + U~^T M^T (both from shared memory) ----
+        const uint32_t ido = tc::idesc_bf16_f32(128, 64, 0, 0);
+        const uint64_t o_desc0 = tc::smem_desc_sw128(tc::smem_u32(sm + SS_O), 16, 1024);
+        for (int u = 0; u < U; ++u) {
+            const int st = u & 1, ob = u & 3;
+            if (!wait(&full_o[st], (u >> 1) & 1)) break;
+            // issued once D_c(u) has completed, so it never shares the tensor pipe with a chain
+            // product; S_u^T is complete since D_c(u) read it
+            if (!wait(&dc_done[st], (u >> 1) & 1)) break;
+            if (u >= 4 && !wait(&o_free[ob], ((u >> 2) - 1) & 1)) break;
+            tc::tc_fence_after();
+            const uint64_t od = tc::desc_add(o_desc0, st * SS_OSTAGE);
+            const uint32_t d = tmem + kColO + 64 * ob;
+            const uint32_t a = tmem + kColS + 64 * st;
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)                                  // S^T Q'^T
+                tc::mma_bf16_tmem_a_warp(d, a + 8 * ks, tc::desc_add(od, (ks >> 2) * 8192 + (ks & 3) * 32),
+                                         ido, ks > 0 ? 1u : 0u);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)                                  // + U~^T M^T
+                tc::mma_bf16_warp(d, tc::desc_add(od, (WS_UT - WS_QP) + ks * 32),
+                                  tc::desc_add(od, (WS_M - WS_QP) + ks * 32), ido, 1u);
+            tc::mma_commit_warp(&mma_o[ob]);
+            tc::mma_commit_warp(&empty_o[st]);
+        }
+    } else if (warp == 10 || warp == 11) {
+        // ---- loads: warp 10 the chain stages, warp 11 the output stages ----
         if (lane == 0) {
-            const bool chain = warp == 5;
+            const bool chain = warp == 10;
             uint64_t* fullb = chain ? full_c : full_o;
             uint64_t* emptyb = chain ? empty_c : empty_o;
+            const uint32_t bytes = chain ? SS_CSTAGE : SS_OSTAGE;
+            uint8_t* stage0 = sm + (chain ? SS_C : SS_O);
             int issued = 0;
-            for (; issued < NT; ++issued) {
-                const int st = issued % kStages;
-                if (issued >= kStages &&
-                    !tc::mbar_wait(&emptyb[st], ((issued / kStages) - 1) & 1, abort_flag))
+            for (; issued < U; ++issued) {
+                const int st = issued & 1;
+                if (issued >= 2 && !mbar_wait_long(&emptyb[st], ((issued >> 1) - 1) & 1, abort_flag))
                     break;
-                const uint8_t* src = wsh + (size_t)issued * WS_CHUNK;
-                const uint8_t* tl = src + WS_TILES + tile * WS_TILE;
-                if (chain) {
-                    uint8_t* stg = sm + st * P2_CSTAGE;
-                    tc::mbar_arrive_expect_tx(&fullb[st], 32768 + WS_TILE_O);
-                    tc::bulk_g2s(stg + P2_AC, src + WS_AC, 32768, &fullb[st]);
-                    tc::bulk_g2s(stg + P2_BC, tl, WS_TILE_O, &fullb[st]);
-                } else {
-                    uint8_t* stg = sm + P2_OBASE + st * P2_OSTAGE;
-                    tc::mbar_arrive_expect_tx(&fullb[st], 16384 + (WS_TILE - WS_TILE_O));
-                    tc::bulk_g2s(stg + P2_QP, src + WS_QP, 16384, &fullb[st]);
-                    tc::bulk_g2s(stg + P2_OL, tl + WS_TILE_O, WS_TILE - WS_TILE_O, &fullb[st]);
-                }
+                const size_t ci = (size_t)item_bh(issued) * NT + issued % NT;
+                if (!flag_wait(flags + ci, abort_flag)) break;
+                tc::mbar_arrive_expect_tx(&fullb[st], bytes);
+                tc::bulk_g2s(stage0 + st * bytes, ws + ci * WS_CHUNK + (chain ? WS_AC : WS_QP), bytes,
+                             &fullb[st]);
             }
             if (*abort_flag) {
                 // let every copy still in flight land before the shared memory is released
-                for (int c = issued > kStages ? issued - kStages : 0; c < issued; ++c)
+                for (int c = issued > 2 ? issued - 2 : 0; c < issued; ++c)
                     for (uint32_t i = 0; i < tc::kSpinLimit; ++i)
-                        if (tc::mbar_try_wait(&fullb[c % kStages], (c / kStages) & 1)) break;
+                        if (tc::mbar_try_wait(&fullb[c & 1], (c >> 1) & 1)) break;
             }
-        }
-    } else if (warp == 7) {
-        // ---- output issue ----
-        const uint32_t ido = tc::idesc_bf16_f32(64, kDVT, 0, 1);
-        const uint64_t o_desc0 = tc::smem_desc_sw128(tc::smem_u32(sm + P2_OBASE), 16, 1024);
-        for (int ch = 0; ch < NT; ++ch) {
-            const int st = ch % kStages, ob = ch % kOutBufs;
-            if (!wait(&full_o[st], (ch / kStages) & 1)) break;
-            // issued once D_c(ch) has completed, so it runs while the chain epilogue works and
-            // never shares the tensor pipe with a chain product
-            if (!wait(&dc_done[ch % kSBufs], (ch / kSBufs) & 1)) break;
-            if (ch >= kOutBufs && !wait(&o_free[ob], ((ch / kOutBufs) - 1) & 1)) break;
-            tc::tc_fence_after();
-            const uint64_t qd = tc::desc_add(o_desc0, st * P2_OSTAGE + P2_QP);
-            const uint64_t sd = s_desc(ch);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                tc::mma_bf16_warp(dob + 32 * ob, tc::desc_add(qd, (ks >> 2) * 8192 + (ks & 3) * 32),
-                                  tc::desc_add(sd, ks * 2048), ido, ks > 0 ? 1u : 0u);
-            tc::mma_commit_warp(&mma_o[ob]);
         }
     } else {
-        // ---- output epilogue: warp w reads TMEM lanes 32 (w % 4) .. (rows 16 (w % 4) + lane) ----
-        const int q4 = warp & 3;
-        for (int ch = 0; ch < NT; ++ch) {
-            const int st = ch % kStages, ob = ch % kOutBufs;
-            const uint8_t* stg = sm + P2_OBASE + st * P2_OSTAGE;
-            if (!wait(&mma_o[ob], (ch / kOutBufs) & 1)) break;
-            if (!wait(&full_o[st], (ch / kStages) & 1)) break;
+        // ---- output epilogue: warp 12 + q reads TMEM lanes 32 q .. (dv columns n) ----
+        // The four warps move in step (named barrier 1): they leave the loop together, on a
+        // vote, so that none waits at a barrier the others have left.
+        const int q = warp & 3, n = 32 * q + lane;
+        const bool leader = warp == 12 && lane == 0;
+        uint8_t* stg = sm + SS_STG;
+        for (int u = 0; u < U; ++u) {
+            const int ob = u & 3;
+            const bool ok = mbar_wait_long(&mma_o[ob], (u >> 2) & 1, abort_flag);
+            // the previous item's tensor store must be done reading the staging tile
+            if (leader) tc::bulk_wait_read<0>();
+            __syncwarp();
+            if (tc::bar_any(1, 128, !ok)) break;
             tc::tc_fence_after();
-            float d[32];
-            tc::tmem_ld32_sync(tc::tmem_addr(dob + 32 * ob, 32 * q4, 0), d);
-            tc::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&o_free[ob]);
-            if (lane < 16) {
-                const int r = 16 * q4 + lane;
-                const int t0 = ch * kC;
-                if (t0 + r < T_len) {
-                    uint4* dst = reinterpret_cast<uint4*>(out + (((size_t)b * T_len + t0 + r) * H + h) * kDV + n0);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        float y[8];
-                        unpack8(*reinterpret_cast<const uint4*>(stg + P2_OL + r * 64 + bc_chunk(r, j)), y);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) y[i] = scale * (d[8 * j + i] + y[i]);
-                        dst[j] = pack8(y);
-                    }
+            for (int half = 0; half < 2; ++half) {
+                float d[32];
+                tc::tmem_ld32_sync(tc::tmem_addr(tmem + kColO + 64 * ob, 32 * q, 32 * half), d);
+                if (half == 1) {
+                    tc::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(&o_free[ob]);
                 }
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    st_bf16(stg, (32 * half + i) * 256 + 2 * n, scale * d[i]);
             }
+            tc::fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&empty_o[st]);
+            tc::bar_named(1, 128);
+            if (leader) {
+                // rows past the end of the sequence are clipped by the tensor store
+                const int bh = item_bh(u);
+                tc::tma_store_4d(&maps.out, stg, 0, bh % H, (u % NT) * kC, bh / H);
+                tc::bulk_commit();
+            }
         }
+        if (leader) tc::bulk_wait_all();
     }
     tc::tc_fence_before();
     __syncthreads();
     if (*abort_flag && tid == 0) atomicExch(&g_tc_error, 2);
-    if (warp == 0) tc::tmem_dealloc(tmem, 256);
+    if (warp == 0) tc::tmem_dealloc(tmem, 512);
+}
+
+__device__ __forceinline__ uint8_t* aligned_smem(uint8_t* raw) {
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+}
+
+// Factor kernel alone: persistent over every chunk-head (chunk-major over all heads).
+template <bool kLogits>
+__global__ void __launch_bounds__(512, 1)
+ckda_tc_intra(const __grid_constant__ TcMaps maps, const void* __restrict__ alpha,
+              const float* __restrict__ beta, uint8_t* __restrict__ ws, int* __restrict__ flags,
+              int T_len, int H, int NT, int BH, int l2norm, RopeParams rp, long long pos_offset) {
+    extern __shared__ uint8_t smem_raw[];
+    intra_role<kLogits>(aligned_smem(smem_raw), maps, alpha, beta, ws, flags, T_len, H, NT, BH * NT,
+                        WorkOrder{NT, BH, BH}, blockIdx.x, gridDim.x, l2norm, rp, pos_offset);
+}
+
+// State pass alone, after the factor kernel: heads blockIdx.x, blockIdx.x + gridDim.x, ...
+__global__ void __launch_bounds__(512, 1)
+ckda_tc_state(const __grid_constant__ TcMaps maps, const uint8_t* __restrict__ ws,
+              const int* __restrict__ flags, const float* __restrict__ h0,
+              __nv_bfloat16* __restrict__ out, float* __restrict__ hT, int T_len, int H, int NT,
+              int BH, float scale) {
+    extern __shared__ uint8_t smem_raw[];
+    state_role(aligned_smem(smem_raw), maps, ws, flags, h0, out, hT, T_len, H, NT, BH, scale,
+               blockIdx.x, gridDim.x);
+}
+
+// Both at once (cooperative launch, every CTA resident): CTAs 0 .. n_state - 1 carry the chains
+// of heads blockIdx.x + k n_state, the others run the factor role over the items in head groups
+// of n_state, so the chains of a group run while the group's chunks are produced.
+template <bool kLogits>
+__global__ void __launch_bounds__(512, 1)
+ckda_tc_fused(const __grid_constant__ TcMaps maps, const void* __restrict__ alpha,
+              const float* __restrict__ beta, uint8_t* __restrict__ ws, int* __restrict__ flags,
+              const float* __restrict__ h0, __nv_bfloat16* __restrict__ out, float* __restrict__ hT,
+              int T_len, int H, int NT, int BH, int n_state, int l2norm, RopeParams rp,
+              long long pos_offset, float scale) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = aligned_smem(smem_raw);
+    if ((int)blockIdx.x < n_state)
+        state_role(sm, maps, ws, flags, h0, out, hT, T_len, H, NT, BH, scale, blockIdx.x, n_state);
+    else
+        intra_role<kLogits>(sm, maps, alpha, beta, ws, flags, T_len, H, NT, BH * NT,
+                            WorkOrder{NT, BH, n_state}, blockIdx.x - n_state, gridDim.x - n_state,
+                            l2norm, rp, pos_offset);
 }
 
 }  // namespace
@@ -1120,7 +1236,45 @@ static bool encode_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt,
 
 size_t chunk_tc_workspace_bytes(int B, int T_len, int H) {
     const size_t nt = (size_t)(T_len + kC - 1) / kC;
-    return (size_t)B * H * nt * WS_CHUNK;
+    const size_t n = (size_t)B * H * nt;
+    return flags_offset(n) + ((n * 4 + 255) & ~(size_t)255);
+}
+
+// Chain CTAs of the fused launch.  Model (SM cycles, measured on B200): a factor item takes
+// t_i = 18800 and the factor CTAs work in lockstep rounds, an item is flagged ready about two
+// rounds after the round it starts in, and a chain step takes t_c = 2400.  With s chain CTAs the
+// heads form groups of s, produced one after the other (chunk-major inside a group); chain CTA 0
+// carries the first head of every group, one after the other, so it finishes last.  Its head in
+// group g cannot end before the previous head plus NT steps, before that head's first chunk plus
+// NT steps, or before its last chunk plus one step.  s minimises the later of that end and the
+// end of the factor work (the larger s on ties).
+int chunk_tc_state_ctas(int BH, int NT, int nsm) {
+    const double ti = 18800.0, tc = 2400.0;
+    const long long total = (long long)BH * NT;
+    const int smax = BH < nsm - 1 ? BH : nsm - 1;
+    int best = 1;
+    double best_t = 1e300;
+    for (int s = 1; s <= smax; ++s) {
+        const long long ni = (long long)(nsm - s) < total ? (long long)(nsm - s) : total;
+        const double factor_end = (double)((total + ni - 1) / ni) * ti;
+        double end = 0.0;
+        for (int g = 0; g * s < BH; ++g) {
+            const long long sg = BH - (long long)g * s < s ? BH - (long long)g * s : s;
+            const long long first = (long long)g * s * NT;
+            const double t_first = (double)(first / ni + 2) * ti;
+            const double t_last = (double)((first + (long long)(NT - 1) * sg) / ni + 2) * ti;
+            double e = end + NT * tc;
+            if (t_first + NT * tc > e) e = t_first + NT * tc;
+            if (t_last + tc > e) e = t_last + tc;
+            end = e;
+        }
+        const double t = end > factor_end ? end : factor_end;
+        if (t <= best_t) {
+            best_t = t;
+            best = s;
+        }
+    }
+    return best;
 }
 
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const void* alpha,
@@ -1129,21 +1283,28 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
                             long long pos_offset, int gate_logits, void* workspace, int stages,
                             cudaStream_t stream) {
     auto intra = gate_logits ? ckda_tc_intra<true> : ckda_tc_intra<false>;
-    cudaError_t e = cudaFuncSetAttribute(intra, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)S_BYTES);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(ckda_tc_state, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P2_BYTES);
+    auto fused = gate_logits ? ckda_tc_fused<true> : ckda_tc_fused<false>;
+    cudaError_t e = cudaFuncSetAttribute(intra, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S_BYTES);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(ckda_tc_state, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SS_BYTES);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)FUSED_BYTES);
     if (e != cudaSuccess) return e;
     const int NT = (T_len + kC - 1) / kC;
+    const int BH = B * H;
+    const int total = NT * BH;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    if (stages == 0) stages = 3;
-    if (stages & 1) {
-        int dev = 0, nsm = 148;
-        if (cudaGetDevice(&dev) == cudaSuccess)
-            cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-        const int total = NT * B * H;
-        const int grid = total < nsm ? total : nsm;
-        TcMaps maps;
+    int* flags = reinterpret_cast<int*>(ws + flags_offset((size_t)total));
+    __nv_bfloat16* outb = static_cast<__nv_bfloat16*>(out);
+    int dev = 0, nsm = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    if (stages == 0 && nsm < 2) stages = 3;
+    TcMaps maps;
+    if (!encode_map(&maps.out, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDV, kDV, H, T_len, B,
+                    CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    if (stages != 2) {
         if (!encode_map(&maps.q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK, kDK, H, T_len, B,
                         CU_TENSOR_MAP_SWIZZLE_NONE) ||
             !encode_map(&maps.k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK, kDK, H, T_len, B,
@@ -1155,38 +1316,54 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
                           : encode_map(&maps.alpha, alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kDK,
                                        kDK, H, T_len, B, CU_TENSOR_MAP_SWIZZLE_NONE)))
             return cudaErrorInvalidValue;
-        // programmatic dependent launch: CTAs may start their set-up on SMs the previous kernel
-        // has left, and wait (griddepcontrol.wait) for it before touching memory
+        // every ready flag starts at zero; the factor role raises them
+        e = cudaMemsetAsync(flags, 0, (size_t)total * 4, stream);
+        if (e != cudaSuccess) return e;
+    }
+    if (stages == 0) {
+        // one cooperative launch: the runtime makes every CTA resident at once, which the chain
+        // CTAs (waiting on flags the factor CTAs raise) rely on
+        const int n_state = chunk_tc_state_ctas(BH, NT, nsm);
+        const int n_intra = nsm - n_state < total ? nsm - n_state : total;
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)grid);
+        cfg.gridDim = dim3((unsigned)(n_state + n_intra));
+        cfg.blockDim = dim3(512);
+        cfg.dynamicSmemBytes = FUSED_BYTES;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, fused, maps, alpha, beta, ws, flags, h0, outb, hT, T_len, H,
+                                 NT, BH, n_state, l2norm, rp, pos_offset, scale);
+    }
+    // two kernels in sequence (profiling aid).  The factor kernel follows the flag reset in plain
+    // stream order; the state kernel uses programmatic dependent launch (its set-up overlaps the
+    // factor kernel's tail, and griddepcontrol.wait holds it back before it reads the workspace)
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    if (stages & 1) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(total < nsm ? total : nsm));
         cfg.blockDim = dim3(512);
         cfg.dynamicSmemBytes = S_BYTES;
         cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, intra, maps, alpha, beta, ws, T_len, H, NT, total, l2norm,
+        e = cudaLaunchKernelEx(&cfg, intra, maps, alpha, beta, ws, flags, T_len, H, NT, BH, l2norm,
                                rp, pos_offset);
         if (e != cudaSuccess) return e;
     }
     if (stages & 2) {
-        // programmatic dependent launch: the state pass is scheduled while the factor kernel
-        // finishes, and waits for it (griddepcontrol.wait) before reading the workspace
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)(kNTile * B * H));
-        cfg.blockDim = dim3(kStateThreads);
-        cfg.dynamicSmemBytes = P2_BYTES;
+        cfg.gridDim = dim3((unsigned)BH);
+        cfg.blockDim = dim3(512);
+        cfg.dynamicSmemBytes = SS_BYTES;
         cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        __nv_bfloat16* outb = static_cast<__nv_bfloat16*>(out);
-        e = cudaLaunchKernelEx(&cfg, ckda_tc_state, static_cast<const uint8_t*>(ws), h0, outb, hT,
-                               T_len, H, NT, scale);
+        e = cudaLaunchKernelEx(&cfg, ckda_tc_state, maps, static_cast<const uint8_t*>(ws),
+                               static_cast<const int*>(flags), h0, outb, hT, T_len, H, NT, BH, scale);
     }
     return e;
 }

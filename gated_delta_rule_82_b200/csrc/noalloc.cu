@@ -12,7 +12,8 @@
 // on each device looks the address up with cudaGetSymbolAddress (with that device current) and
 // caches it.  Every call shares the array: calls whose kernels overlap on the GPU (different
 // streams, or host threads racing) corrupt each other's scratch.  No byte of the scratch has to
-// start at zero: the chunk-factor kernel writes every byte the state-pass kernel later reads.
+// start at zero: every call clears the chunk-heads' ready flags itself, and the chunk-factor work
+// writes every other byte the state pass later reads.
 #include <mutex>
 
 #include "internal.cuh"

@@ -16,6 +16,8 @@ constexpr int kSelftestTmemCols = 512;   // D (N <= 256 columns) + A staged in T
 __global__ void __launch_bounds__(128)
 umma_selftest_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16* __restrict__ B,
                      float* __restrict__ D, int M, int N, int K, int b_mn, int a_tmem) {
+    // a_tmem: 0 = A from shared memory; 1 = A copied into TMEM by tcgen05.cp; 2 = A written into
+    // TMEM by the threads (tcgen05.st: row m in lane m, K elements 2j and 2j + 1 in column j)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -67,13 +69,33 @@ umma_selftest_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16* _
         }
         tc::mma_commit(&bar);
     }
+    if (a_tmem == 2) {
+        // thread (warp w, lane l) writes row 32 w + l of A, 64 K elements per 32-column store
+        const int m = warp * 32 + lane;
+        for (int c0 = 0; c0 < K / 2; c0 += 32) {
+            uint32_t v[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const uint16_t lo = __bfloat16_as_ushort(A[(size_t)m * K + 2 * (c0 + j)]);
+                const uint16_t hi = __bfloat16_as_ushort(A[(size_t)m * K + 2 * (c0 + j) + 1]);
+                v[j] = (uint32_t)lo | ((uint32_t)hi << 16);
+            }
+            tc::tmem_st32(tc::tmem_addr(tbase + 256, warp * 32, c0), v);
+        }
+        tc::tmem_st_wait();
+        tc::tc_fence_before();
+        __syncthreads();
+        tc::tc_fence_after();
+    }
     if (a_tmem && warp == 0) {
-        // A (M = 128) staged into TMEM columns 256.. by tcgen05.cp, one 16-element K-step per copy
+        // A (M = 128) in TMEM columns 256.. (K / 2 columns): copied there by tcgen05.cp, one
+        // 16-element K-step per copy, unless the threads wrote it above
         const uint32_t idesc = tc::idesc_bf16_f32(M, N, 0, b_mn);
         const uint32_t a0 = tc::smem_u32(sA), b0 = tc::smem_u32(sB);
         const uint32_t ta = tbase + 256;
-        for (int ks = 0; ks < K / 16; ++ks)
-            tc::tmem_cp_128x256b_warp(ta + ks * 8, tc::smem_desc_sw128(a0 + (ks >> 2) * M * 128 + (ks & 3) * 32, 16, 1024));
+        if (a_tmem == 1)
+            for (int ks = 0; ks < K / 16; ++ks)
+                tc::tmem_cp_128x256b_warp(ta + ks * 8, tc::smem_desc_sw128(a0 + (ks >> 2) * M * 128 + (ks & 3) * 32, 16, 1024));
         for (int ks = 0; ks < K / 16; ++ks) {
             uint64_t bd = b_mn ? tc::smem_desc_sw128(b0 + ks * 2048, K * 128, 1024)
                                : tc::smem_desc_sw128(b0 + (ks >> 2) * N * 128 + (ks & 3) * 32, 16, 1024);
@@ -104,7 +126,7 @@ umma_selftest_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16* _
 
 cudaError_t launch_umma_selftest(const void* A, const void* B, float* D, int M, int N, int K,
                                  int mode, cudaStream_t stream) {
-    const int b_mn_major = mode & 1, a_tmem = (mode >> 1) & 1;
+    const int b_mn_major = mode & 1, a_tmem = (mode & 2) ? 1 : (mode & 4) ? 2 : 0;
     // an MN-major B occupies whole 128-byte rows: ceil(N / 64) blocks of K rows
     const size_t b_bytes = b_mn_major ? (size_t)((N + 63) / 64) * K * 128 : (size_t)N * K * 2;
     size_t smem = (size_t)M * K * 2 + b_bytes + 1024;

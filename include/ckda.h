@@ -81,10 +81,12 @@ typedef struct {
     int rope_convention; /* 0: half-split pairs (x_i, x_{i+dk/2}); 1: interleaved (x_{2i}, x_{2i+1}) */
     float scale;         /* read-out scale; 0 selects dk^-1/2 */
     int path;            /* ckda_path; ckda_fwd_chunked only, ignored elsewhere */
-    int stages;          /* ckda_fwd_chunked on the tensor-core path only (profiling aid):
-                            0 or 3 = both kernels; 1 = only the chunk-parallel factor kernel
-                            (fills the workspace); 2 = only the serial state pass (reads a
-                            workspace filled by a stage-1 call with the same arguments) */
+    int stages;          /* ckda_fwd_chunked on the tensor-core path only: 0 = one fused
+                            launch (chunk-parallel factor work and the serial state pass run
+                            side by side); profiling aids: 3 = the two parts as two kernels in
+                            sequence, 1 = only the factor kernel (fills the workspace), 2 = only
+                            the state pass (reads a workspace filled by a stage-1 call with the
+                            same arguments) */
     int gate_logits;     /* 0: alpha and beta hold the gates themselves (fp32).  1: they hold
                             logits -- alpha the logits a in the element type `dtype`, beta the
                             logits b in fp32 -- and the kernels form the gates as
@@ -164,7 +166,10 @@ CKDA_API ckda_status ckda_decode_step(const void* q, const void* k, const void* 
  *   b_mn_major bit 0 set:   B is [K, N] row-major (N contiguous), D = A B    (MN-major B operand)
  *   b_mn_major bit 1 set:   A is staged from shared memory into Tensor Memory with
  *                           tcgen05.cp and read by the product from there (M = 128 only)
- *   other bits: CKDA_ERR_ARG.
+ *   b_mn_major bit 2 set:   A is written into Tensor Memory by the threads with tcgen05.st
+ *                           (row m in lane m, K elements 2j and 2j + 1 packed in column j) and
+ *                           read by the product from there (M = 128 only)
+ *   bits 1 and 2 together, or other bits: CKDA_ERR_ARG.
  * M in {64, 128}; N a multiple of 16 in [16, 256] (32 or a multiple of 64 when b_mn_major);
  * K a multiple of 64 in [64, 256].  Lets a user check the tensor-core path on a device.
  */
@@ -180,8 +185,8 @@ CKDA_API ckda_status ckda_selftest_umma(const void* A, const void* B, float* D, 
  * until the process exits.  The function allocates nothing.
  *   Arguments and results: as ckda_fwd_chunked, minus workspace / workspace_bytes.
  *   Limit: problems whose ckda_fwd_workspace_bytes(...) exceeds CKDA_NOALLOC_MAX_WORKSPACE are
- *          rejected with CKDA_ERR_WORKSPACE before anything is launched (16 MiB holds 170
- *          chunk-heads of the tensor-core path: B * H * ceil(T / 64) <= 170).
+ *          rejected with CKDA_ERR_WORKSPACE before anything is launched (16 MiB holds 157
+ *          chunk-heads of the tensor-core path: B * H * ceil(T / 64) <= 157).
  *   Set-up: the first call on a device looks up the array's device address (cudaGetSymbolAddress,
  *          with that device current); make that first call before any stream capture.
  *   Sharing: every call uses the same array, which keeps the last call's contents (no part of it

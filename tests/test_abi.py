@@ -138,7 +138,9 @@ def test_selftest_validation(lib):
     assert lib.ckda_selftest_umma(c(P), c(2 * P), c(3 * P), 64, 48, 64, 1, None) == UNSUP
     assert lib.ckda_selftest_umma(c(P), c(2 * P), c(3 * P), 64, 64, 96, 0, None) == UNSUP
     assert lib.ckda_selftest_umma(c(P), c(2 * P), c(3 * P), 64, 64, 64, 2, None) == UNSUP  # A in TMEM: M = 128
-    assert lib.ckda_selftest_umma(c(P), c(2 * P), c(3 * P), 128, 64, 64, 4, None) == ARG
+    assert lib.ckda_selftest_umma(c(P), c(2 * P), c(3 * P), 64, 64, 64, 4, None) == UNSUP  # A in TMEM: M = 128
+    assert lib.ckda_selftest_umma(c(P), c(2 * P), c(3 * P), 128, 64, 64, 6, None) == ARG
+    assert lib.ckda_selftest_umma(c(P), c(2 * P), c(3 * P), 128, 64, 64, 8, None) == ARG
 
 
 def test_binding_refuses_cpu_tensors():

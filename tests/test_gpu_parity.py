@@ -48,15 +48,17 @@ def test_umma_selftest(M, N, K, mn):
 @pytest.mark.parametrize("N", [32, 64, 128])
 @pytest.mark.parametrize("K", [64, 128])
 @pytest.mark.parametrize("mn", [0, 1])
-def test_umma_selftest_a_in_tmem(N, K, mn):
-    """A staged into Tensor Memory by tcgen05.cp (one 128x256b copy per K-step) and read by the
-    product from there; M = 128."""
+@pytest.mark.parametrize("how", ["cp", "st"])
+def test_umma_selftest_a_in_tmem(N, K, mn, how):
+    """A in Tensor Memory, read by the product from there (M = 128): staged by tcgen05.cp (one
+    128x256b copy per K-step), or written by the threads with tcgen05.st (row m in lane m, K
+    elements 2j and 2j + 1 in column j)."""
     if mn and N % 64 and N != 32:
         pytest.skip("MN-major operand needs N = 32 or N % 64 == 0")
     g = torch.Generator().manual_seed(7000 + N * 10 + K + mn)
     A = torch.randn(128, K, generator=g).bfloat16()
     B = torch.randn(K, N, generator=g).bfloat16() if mn else torch.randn(N, K, generator=g).bfloat16()
-    D = ck.selftest_umma(A.cuda(), B.cuda(), b_mn_major=bool(mn), a_tmem=True)
+    D = ck.selftest_umma(A.cuda(), B.cuda(), b_mn_major=bool(mn), a_tmem=how)
     torch.cuda.synchronize()
     ref = A.double() @ (B.double() if mn else B.double().T)
     assert rel_err(D, ref.numpy()) < 1e-5

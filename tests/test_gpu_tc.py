@@ -43,7 +43,7 @@ def check(B, T, H, *, kind="ckda", h0_std=0.0, rope=(0.0, 0), pos=0, seed=0, tol
 
 def test_workspace_size():
     n = ck.workspace_bytes(2, 2048, 16, 128, 128, 64, torch.bfloat16, "tc")
-    assert n == 2 * 16 * 32 * 98304
+    assert n == 2 * 16 * 32 * 106496 + 2 * 16 * 32 * 4
 
 
 @pytest.mark.parametrize("T", [1, 63, 64, 65, 150, 257])
@@ -153,7 +153,7 @@ def test_tc_resume_equals_one_pass():
 
 
 def test_tc_state_in_place():
-    """hT may alias h0: each (batch, head, dv tile) is read before it is written."""
+    """hT may alias h0: each (batch, head) is read before it is written."""
     d, g = fwd_case(2, 130, 2, 128, 128, kind="ckda", dtype="bf16", h0_std=0.02, seed=23)
     st = g["h0"].clone()
     out, _ = ck.fwd_chunked(g["q"], g["k"], g["v"], g["alpha"], g["beta"], st, hT=st, path="tc")
@@ -161,3 +161,41 @@ def test_tc_state_in_place():
     o_ref, s_ref = oracle_fwd(d)
     assert rel_err(out, o_ref) < TOL
     assert rel_err(st, s_ref) < TOL
+
+
+def _run_stages(g, stages, **kw):
+    ws = torch.empty(ck.workspace_bytes(g["q"].shape[0], g["q"].shape[1], g["q"].shape[2], 128, 128),
+                     dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(g["v"])
+    hT = torch.empty_like(g["h0"])
+    for s in stages:
+        ck.fwd_chunked(g["q"], g["k"], g["v"], g["alpha"], g["beta"], g["h0"], path="tc", out=out,
+                       hT=hT, workspace=ws, stages=s, **kw)
+    torch.cuda.synchronize()
+    return out, hT
+
+
+def test_tc_fused_equals_two_kernel_sequence():
+    """The fused launch (chain CTAs beside the factor CTAs), the two kernels in sequence and the
+    two kernels as separate calls compute the same arithmetic: identical bits, and the oracle's
+    values within tolerance."""
+    d, g = fwd_case(2, 300, 3, 128, 128, kind="ckda", dtype="bf16", h0_std=0.02, seed=29)
+    kw = dict(rope_theta=10000.0, rope_convention=1)
+    o0, s0 = _run_stages(g, [0], **kw)
+    o3, s3 = _run_stages(g, [3], **kw)
+    o12, s12 = _run_stages(g, [1, 2], **kw)
+    assert torch.equal(o0, o3) and torch.equal(s0, s3)
+    assert torch.equal(o0, o12) and torch.equal(s0, s12)
+    o_ref, s_ref = oracle_fwd(d, rope_theta=10000.0, rope_convention=1)
+    assert rel_err(o0, o_ref) < TOL and rel_err(s0, s_ref) < TOL
+
+
+def test_tc_heads_share_chain_ctas():
+    """90 heads of 3 ragged chunks: the fused launch gives each chain CTA several heads in turn
+    (each starting from its own h0 and ending in its own hT)."""
+    check(3, 130, 30, h0_std=0.02, seed=31)
+
+
+def test_tc_more_heads_than_sms():
+    """160 heads of one chunk each: more (batch, head) pairs than SMs."""
+    check(1, 64, 160, h0_std=0.02, seed=37)

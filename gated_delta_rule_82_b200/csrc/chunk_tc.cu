@@ -52,6 +52,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include "fastdiv.h"
 #include "internal.cuh"
 #include "tc_sm100.cuh"
 
@@ -114,6 +115,10 @@ constexpr uint32_t kInBytes = 32768 + 2 * 16384; // alpha, q, k of one chunk-hea
 constexpr uint32_t kVBytes = 16384;
 
 constexpr float kSafeDecay = 3.009265538105056e-36f;  // 2^-118
+// The factor role's bulk stores (and their waits, and the ready flags) all go through one thread:
+// bulk-store groups belong to the thread that commits them.  It sits in warp 15, which has no
+// product to issue.
+constexpr int kStoreTid = 480;
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -170,22 +175,19 @@ struct TcMaps {
     CUtensorMap q, k, v, alpha, out;
 };
 
-// Issue the TMA loads of chunk-head ci: alpha -> G, q -> QR, k -> KR on bar_in; V (two 64-column
-// halves, 128-byte swizzle) on bar_v when with_v.  Rows past the sequence end read as zeros.
+// Issue the TMA loads of the chunk of batch b, head h starting at token t0: alpha -> G, q -> QR,
+// k -> KR on bar_in; V (two 64-column halves, 128-byte swizzle) on bar_v.  Rows past the sequence
+// end read as zeros.
 __device__ __forceinline__ void issue_inputs(const TcMaps& m, uint8_t* sm, uint64_t* bar_in,
-                                             int ci, int NT, int H, int gate_logits) {
-    const int ch = ci % NT, bh = ci / NT;
-    const int b = bh / H, h = bh % H, t0 = ch * kC;
+                                             int b, int h, int t0, int gate_logits) {
     // gate values: fp32 [64][128] into G; logits: bf16 [64][128] into the upper half of G
     tc::mbar_arrive_expect_tx(bar_in, gate_logits ? kInBytes - 16384 : kInBytes);
     tc::tma_load_4d(sm + S_G + (gate_logits ? 16384 : 0), &m.alpha, 0, h, t0, b, bar_in);
     tc::tma_load_4d(sm + S_QR, &m.q, 0, h, t0, b, bar_in);
     tc::tma_load_4d(sm + S_KR, &m.k, 0, h, t0, b, bar_in);
 }
-__device__ __forceinline__ void issue_v(const TcMaps& m, uint8_t* sm, uint64_t* bar_v, int ci,
-                                        int NT, int H) {
-    const int ch = ci % NT, bh = ci / NT;
-    const int b = bh / H, h = bh % H, t0 = ch * kC;
+__device__ __forceinline__ void issue_v(const TcMaps& m, uint8_t* sm, uint64_t* bar_v, int b,
+                                        int h, int t0) {
     tc::mbar_arrive_expect_tx(bar_v, kVBytes);
     tc::tma_load_4d(sm + S_V, &m.v, 0, h, t0, b, bar_v);
     tc::tma_load_4d(sm + S_V + 8192, &m.v, 64, h, t0, b, bar_v);
@@ -347,17 +349,40 @@ __device__ __forceinline__ void t_solve(const float* sA, float* sT, const float*
 // Order in which the factor role visits the chunk-heads: heads in groups of G, and inside a
 // group chunk by chunk (chunk c of every head of the group before chunk c + 1), so that the serial
 // chains of a group, which consume their chunks in order, can run behind the factor work.  Item i
-// maps to the chunk-head ci = bh * NT + c of the workspace.
+// is chunk c of batch*head bh (workspace chunk-head bh * NT + c).  The divisions go through
+// multiply-shift forms of the launch's fixed divisors.
+struct Item {
+    int bh, c, b, h;
+};
 struct WorkOrder {
-    int NT, BH, G;
-    __device__ __forceinline__ int ci(int i) const {
-        const int per = G * NT;
-        const int g = i / per, r = i - g * per;
-        const int gs = min(G, BH - g * G);
-        const int c = r / gs;
-        return (g * G + (r - c * gs)) * NT + c;
+    int G, last_g;
+    FastDiv per;     // G * NT items per group
+    FastDiv gfull;   // G heads in a group
+    FastDiv glast;   // heads in the last group
+    FastDiv heads;   // H
+    __device__ __forceinline__ Item item(int i) const {
+        const uint32_t g = fastdiv(per, (uint32_t)i);
+        const uint32_t r = (uint32_t)i - g * per.d;
+        const FastDiv& gs = (int)g == last_g ? glast : gfull;
+        const uint32_t c = fastdiv(gs, r);
+        Item it;
+        it.bh = (int)(g * (uint32_t)G + (r - c * gs.d));
+        it.c = (int)c;
+        it.b = (int)fastdiv(heads, (uint32_t)it.bh);
+        it.h = it.bh - it.b * (int)heads.d;
+        return it;
     }
 };
+inline WorkOrder make_work_order(int NT, int BH, int H, int G) {
+    WorkOrder w;
+    w.G = G;
+    w.last_g = (BH - 1) / G;
+    w.per = make_fastdiv((uint32_t)(G * NT));
+    w.gfull = make_fastdiv((uint32_t)G);
+    w.glast = make_fastdiv((uint32_t)(BH - w.last_g * G));
+    w.heads = make_fastdiv((uint32_t)H);
+    return w;
+}
 
 // Ready flags.  The writer waits for its bulk stores to complete, orders them before the flag
 // (proxy fence, then a release store at GPU scope); a reader acquires the flag and fences before
@@ -461,22 +486,23 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
         tc::prefetch_tensormap(&maps.k);
         tc::prefetch_tensormap(&maps.v);
         tc::prefetch_tensormap(&maps.alpha);
-        issue_inputs(maps, sm, bar_in, wo.ci(rank), NT, H, gate_logits);
-        issue_v(maps, sm, bar_v, wo.ci(rank), NT, H);
+        const Item first = wo.item(rank);
+        issue_inputs(maps, sm, bar_in, first.b, first.h, first.c * kC, gate_logits);
+        issue_v(maps, sm, bar_v, first.b, first.h, first.c * kC);
     }
 
     // persistent loop over items; chunk-head ci = (batch*head) * NT + chunk
     uint32_t it = 0;
     int pending = -1;   // chunk-head whose images are stored but not yet flagged ready
     for (int i = rank; i < total; i += nprog, ++it) {
-        const int ci = wo.ci(i);
-        const int ch = ci % NT, bh = ci / NT;
-        const int h = bh % H;
-        const int t0 = ch * kC;
+        const Item cur = wo.item(i);
+        const int ci = cur.bh * NT + cur.c;
+        const int t0 = cur.c * kC;
         const int nvalid = min(kC, T_len - t0);
-        const int nci = i + nprog < total ? wo.ci(i + nprog) : -1;
+        const bool has_next = i + nprog < total;
+        const Item nxt = wo.item(has_next ? i + nprog : i);
         uint8_t* wsc = ws + (size_t)ci * WS_CHUNK;
-        const size_t row0 = ((size_t)(bh / H) * T_len + t0) * H + h;
+        const size_t row0 = ((size_t)cur.b * T_len + t0) * H + cur.h;
         float bval = (tid < 64 && tid < nvalid) ? beta[row0 + tid * rs] : 0.f;
         if (kLogits && tid < 64 && tid < nvalid) bval = gate_beta(bval);   // beta = 2 sigma(b)
 
@@ -524,7 +550,7 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
         if (tid < 64) sb[tid] = bval;
         // the previous chunk-head's first store group (the Q' image over R, tiles 0-1 over
         // K_end and M) must have finished reading before the row pass rewrites R and K_end
-        if (tid == 0) tc::bulk_wait_read<1>();
+        if (tid == kStoreTid) tc::bulk_wait_read<1>();
         __syncthreads();
         const bool exact = *exact_path != 0;
 
@@ -625,12 +651,12 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
         tc::tc_fence_before();
         // the rest of the previous chunk-head's images (over A, T, W and U) must be read out
         // before the [A | M] read-back or the exact path rewrites them
-        if (tid == 0) tc::bulk_wait_read<0>();
+        if (tid == kStoreTid) tc::bulk_wait_read<0>();
         __syncthreads();
         tc::tc_fence_after();
         // alpha, q, k of this chunk-head are consumed: bring in the next one's.  Issued by warp 15
         // (a TMA issue costs its thread several hundred cycles) while warp 0 issues the product.
-        if (tid == 480 && nci >= 0) issue_inputs(maps, sm, bar_in, nci, NT, H, gate_logits);
+        if (tid == 480 && has_next) issue_inputs(maps, sm, bar_in, nxt.b, nxt.h, nxt.c * kC, gate_logits);
         if (!exact) {
             // ======== B: [A | M] = L R^T on the tensor cores (M = 128, N = 64, K = 128) ========
             if (warp == 0) {
@@ -643,14 +669,6 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
                                       tc::desc_add(bd, (ks >> 2) * 8192 + (ks & 3) * 32), idesc, ks > 0);
                 tc::mma_commit_warp(bar);
             }
-        }
-        // the previous chunk-head's stores have had a whole row pass to land: flag it ready
-        if (pending >= 0) {
-            if (tid == 0) {
-                tc::bulk_wait_all();
-                publish_ready(flags + pending);
-            }
-            pending = -1;
         }
         if (!exact) {
             tc::mbar_wait(bar, phase & 1, abort_flag);
@@ -803,9 +821,17 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
                 tc::mma_bf16_warp(tmem + 320, tc::desc_add(ud, ks * 32), tc::desc_add(ked, ks * 2048), id_b, ks > 0);
             tc::mma_commit_warp(bar);
         }
+        // The previous chunk-head's stores, issued at its end, have landed by now: flag it ready.
+        // The release behind the flag takes a memory round trip, which the storing thread (in a
+        // warp with nothing else to do until M W completes) spends while the products run.
+        if (tid == kStoreTid && pending >= 0) {
+            tc::bulk_wait_all();
+            publish_ready(flags + pending);
+        }
+        pending = -1;
         // V of this chunk-head was consumed by the W/U~ products: bring in the next one's, from
         // warp 14 while warp 0 issues these products
-        if (tid == 448 && nci >= 0) issue_v(maps, sm, bar_v, nci, NT, H);
+        if (tid == 448 && has_next) issue_v(maps, sm, bar_v, nxt.b, nxt.h, nxt.c * kC);
         tc::mbar_wait(bar_q, it & 1, abort_flag);
         tc::tc_fence_after();
         // ======== G: results into shared staging images, then bulk stores in two groups ========
@@ -863,7 +889,7 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
         tc::tc_fence_before();
         __syncthreads();
         tc::tc_fence_after();
-        if (tid == 0) {
+        if (tid == kStoreTid) {
             // group 1: the images over buffers the next row pass rewrites first (Q' over R,
             // the first half of B_c^T over K_end)
             tc::bulk_s2g(wsc + WS_QP, sm + S_OUT_QP, 16384);
@@ -878,7 +904,7 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
         }
         pending = ci;
     }
-    if (tid == 0) {
+    if (tid == kStoreTid) {
         tc::bulk_wait_all();
         if (pending >= 0) publish_ready(flags + pending);
     }
@@ -975,7 +1001,7 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
     auto wait = [&](uint64_t* bar, uint32_t parity) {
         return __all_sync(0xffffffffu, mbar_wait_long(bar, parity, abort_flag));
     };
-    auto item_bh = [&](int u) { return head0 + (u / NT) * hstride; };
+    // items advance as (head k, chunk c) counters, so no step divides by NT
 
     if (warp < 8) {
         // ---- chain epilogue: lane = dv column n, state rows cb .. cb + 63 ----
@@ -1004,10 +1030,10 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
             if (lane == 0) tc::mbar_arrive(&s_ready[u & 1]);
         };
         if (U > 0) {
-            load_h0(item_bh(0));
+            load_h0(head0);
             put_s(0);
         }
-        for (int u = 0; u < U; ++u) {
+        for (int u = 0, c = 0, bh = head0; u < U; ++u) {
             const int st = u & 1;
             if (!wait(&full_c[st], (u >> 1) & 1)) break;
             if (!wait(mma_c, u & 1)) break;
@@ -1024,9 +1050,9 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
             // A_c was read by the finished product and B_c^T is in registers: release the stage
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&empty_c[st]);
-            const bool last = u % NT == NT - 1;
+            const bool last = c == NT - 1;
             if (last && hT && !*abort_flag) {
-                float* dst = hT + ((size_t)item_bh(u) * kDK + cb) * kDV + n;
+                float* dst = hT + ((size_t)bh * kDK + cb) * kDV + n;
 #pragma unroll
                 for (int j = 0; j < 64; ++j) dst[(size_t)j * kDV] = S[j];
             }
@@ -1034,10 +1060,14 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
                 // the buffer of S_{u+1}^T held S_{u-1}^T: the output product of item u - 1 must
                 // be done with it
                 if (u >= 1 && !wait(&mma_o[(u - 1) & 3], ((u - 1) >> 2) & 1)) break;
-                if (last) load_h0(item_bh(u + 1));
+                if (last) load_h0(bh + hstride);
                 put_s(u + 1);
             } else {
                 tc::tc_fence_before();
+            }
+            if (++c == NT) {
+                c = 0;
+                bh += hstride;
             }
         }
     } else if (warp == 8) {
@@ -1093,11 +1123,15 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
             const uint32_t bytes = chain ? SS_CSTAGE : SS_OSTAGE;
             uint8_t* stage0 = sm + (chain ? SS_C : SS_O);
             int issued = 0;
-            for (; issued < U; ++issued) {
+            for (int c = 0, bh = head0; issued < U; ++issued) {
                 const int st = issued & 1;
                 if (issued >= 2 && !mbar_wait_long(&emptyb[st], ((issued >> 1) - 1) & 1, abort_flag))
                     break;
-                const size_t ci = (size_t)item_bh(issued) * NT + issued % NT;
+                const size_t ci = (size_t)bh * NT + c;
+                if (++c == NT) {
+                    c = 0;
+                    bh += hstride;
+                }
                 if (!flag_wait(flags + ci, abort_flag)) break;
                 tc::mbar_arrive_expect_tx(&fullb[st], bytes);
                 tc::bulk_g2s(stage0 + st * bytes, ws + ci * WS_CHUNK + (chain ? WS_AC : WS_QP), bytes,
@@ -1117,7 +1151,7 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
         const int q = warp & 3, n = 32 * q + lane;
         const bool leader = warp == 12 && lane == 0;
         uint8_t* stg = sm + SS_STG;
-        for (int u = 0; u < U; ++u) {
+        for (int u = 0, c = 0, bh = head0; u < U; ++u) {
             const int ob = u & 3;
             const bool ok = mbar_wait_long(&mma_o[ob], (u >> 2) & 1, abort_flag);
             // the previous item's tensor store must be done reading the staging tile
@@ -1143,9 +1177,12 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
             tc::bar_named(1, 128);
             if (leader) {
                 // rows past the end of the sequence are clipped by the tensor store
-                const int bh = item_bh(u);
-                tc::tma_store_4d(&maps.out, stg, 0, bh % H, (u % NT) * kC, bh / H);
+                tc::tma_store_4d(&maps.out, stg, 0, bh % H, c * kC, bh / H);
                 tc::bulk_commit();
+            }
+            if (++c == NT) {
+                c = 0;
+                bh += hstride;
             }
         }
         if (leader) tc::bulk_wait_all();
@@ -1165,10 +1202,11 @@ template <bool kLogits>
 __global__ void __launch_bounds__(512, 1)
 ckda_tc_intra(const __grid_constant__ TcMaps maps, const void* __restrict__ alpha,
               const float* __restrict__ beta, uint8_t* __restrict__ ws, int* __restrict__ flags,
-              int T_len, int H, int NT, int BH, int l2norm, RopeParams rp, long long pos_offset) {
+              int T_len, int H, int NT, int BH, WorkOrder wo, int l2norm, RopeParams rp,
+              long long pos_offset) {
     extern __shared__ uint8_t smem_raw[];
     intra_role<kLogits>(aligned_smem(smem_raw), maps, alpha, beta, ws, flags, T_len, H, NT, BH * NT,
-                        WorkOrder{NT, BH, BH}, blockIdx.x, gridDim.x, l2norm, rp, pos_offset);
+                        wo, blockIdx.x, gridDim.x, l2norm, rp, pos_offset);
 }
 
 // State pass alone, after the factor kernel: heads blockIdx.x, blockIdx.x + gridDim.x, ...
@@ -1190,16 +1228,15 @@ __global__ void __launch_bounds__(512, 1)
 ckda_tc_fused(const __grid_constant__ TcMaps maps, const void* __restrict__ alpha,
               const float* __restrict__ beta, uint8_t* __restrict__ ws, int* __restrict__ flags,
               const float* __restrict__ h0, __nv_bfloat16* __restrict__ out, float* __restrict__ hT,
-              int T_len, int H, int NT, int BH, int n_state, int l2norm, RopeParams rp,
-              long long pos_offset, float scale) {
+              int T_len, int H, int NT, int BH, int n_state, WorkOrder wo, int l2norm,
+              RopeParams rp, long long pos_offset, float scale) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = aligned_smem(smem_raw);
     if ((int)blockIdx.x < n_state)
         state_role(sm, maps, ws, flags, h0, out, hT, T_len, H, NT, BH, scale, blockIdx.x, n_state);
     else
-        intra_role<kLogits>(sm, maps, alpha, beta, ws, flags, T_len, H, NT, BH * NT,
-                            WorkOrder{NT, BH, n_state}, blockIdx.x - n_state, gridDim.x - n_state,
-                            l2norm, rp, pos_offset);
+        intra_role<kLogits>(sm, maps, alpha, beta, ws, flags, T_len, H, NT, BH * NT, wo,
+                            blockIdx.x - n_state, gridDim.x - n_state, l2norm, rp, pos_offset);
 }
 
 }  // namespace
@@ -1336,7 +1373,8 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         return cudaLaunchKernelEx(&cfg, fused, maps, alpha, beta, ws, flags, h0, outb, hT, T_len, H,
-                                 NT, BH, n_state, l2norm, rp, pos_offset, scale);
+                                 NT, BH, n_state, make_work_order(NT, BH, H, n_state), l2norm, rp,
+                                 pos_offset, scale);
     }
     // two kernels in sequence (profiling aid).  The factor kernel follows the flag reset in plain
     // stream order; the state kernel uses programmatic dependent launch (its set-up overlaps the
@@ -1350,8 +1388,8 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
         cfg.blockDim = dim3(512);
         cfg.dynamicSmemBytes = S_BYTES;
         cfg.stream = stream;
-        e = cudaLaunchKernelEx(&cfg, intra, maps, alpha, beta, ws, flags, T_len, H, NT, BH, l2norm,
-                               rp, pos_offset);
+        e = cudaLaunchKernelEx(&cfg, intra, maps, alpha, beta, ws, flags, T_len, H, NT, BH,
+                               make_work_order(NT, BH, H, BH), l2norm, rp, pos_offset);
         if (e != cudaSuccess) return e;
     }
     if (stages & 2) {

@@ -405,6 +405,10 @@ __device__ __forceinline__ uint64_t global_ns() {
 // (milliseconds on long sequences), so they are bounded by time rather than by a poll count.
 constexpr uint64_t kLongWaitNs = 4000000000ull;   // 4 s
 __device__ __forceinline__ bool flag_wait(const int* flag, volatile int* abort) {
+    if (ld_acquire(flag) != 0) {
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        return true;
+    }
     const uint64_t t0 = global_ns();
     for (;;) {
         if (ld_acquire(flag) != 0) {
@@ -417,6 +421,7 @@ __device__ __forceinline__ bool flag_wait(const int* flag, volatile int* abort) 
     }
 }
 __device__ __forceinline__ bool mbar_wait_long(uint64_t* bar, uint32_t parity, volatile int* abort) {
+    if (tc::mbar_try_wait(bar, parity)) return true;   // the common case reads no timer
     const uint64_t t0 = global_ns();
     for (uint32_t i = 0;; ++i) {
         if (tc::mbar_try_wait(bar, parity)) return true;

@@ -36,16 +36,16 @@
 //   B  tcgen05: [A | M] = L R^T  (M = 128, N = 64, K = 128), read back by all 16 warps.
 //   C  T = (I + A)^-1 by blocked forward substitution in fp32; T' = T diag(beta) in bf16.
 //   D  tcgen05: W^T = K_gamma^T T'^T, U~^T = V^T T'^T (M = 128, N = 64).
-//   F  tcgen05: M W (M = 64) and U~^T M^T, K_end^T W, K_end^T U~ (M = 128).
-//   G  A_c, B_c^T and Q' staged in shared memory and written with bulk (TMA) stores, next to U~^T
-//      and M straight from the operand tiles; once they have landed the chunk-head's ready flag
+//   F  tcgen05: M W (M = 64) and K_end^T W (M = 128).
+//   G  A_c and Q' staged in shared memory and written with bulk (TMA) stores, next to K_end, U~^T
+//      and M straight from their operand tiles; once they have landed the chunk-head's ready flag
 //      goes up.
 // State role (ckda_tc_state alone, or the chain CTAs of ckda_tc_fused) -- one CTA per head at a
 // time (all 128 dv columns), serial over its chunks, with the state transposed in Tensor Memory:
-// per chunk one tcgen05 product D_c^T = S^T A_c^T (M = 128, N = 128, K = 128) on the critical
-// path, whose epilogue adds B_c^T to form the next state (fp32, rounded to bf16 as the next
-// operand), and one off-path accumulation D_o^T = S^T Q'^T + U~^T M^T that becomes the chunk's
-// output.
+// per chunk the accumulation D_c^T = U~^T K_end + S^T A_c^T (M = 128, N = 128), whose state-free
+// first part is issued ahead and whose second part (K = 128) is on the critical path; its
+// read-back is the next state (fp32, rounded to bf16 as the next operand).  One off-path
+// accumulation D_o^T = S^T Q'^T + U~^T M^T becomes the chunk's output.
 // The fused launch is cooperative (every CTA resident at once): a few chain CTAs follow the
 // ready flags of their heads while the factor CTAs produce them, so the serial pass hides behind
 // the chunk-parallel work instead of following it.
@@ -64,16 +64,14 @@ constexpr int kC = 64, kDK = 128, kDV = 128;
 
 // ---- workspace image of one chunk-head (bytes) ------------------------------------------------
 constexpr uint32_t WS_AC = 0;          // A_c bf16, K-major swizzled, 128 rows x 128
-constexpr uint32_t WS_BC = 32768;      // B_c^T bf16 [128 dv rows][128], 16-byte chunks swizzled
+constexpr uint32_t WS_KE = 32768;      // K_end bf16, MN-major swizzled, 64 token rows x 128
+constexpr uint32_t WS_UT = 49152;      // U~^T bf16, K-major swizzled, 128 dv rows x 64 tokens
 constexpr uint32_t WS_QP = 65536;      // Q'  bf16, K-major swizzled, 64 rows x 128
-constexpr uint32_t WS_UT = 81920;      // U~^T bf16, K-major swizzled, 128 dv rows x 64 tokens
-constexpr uint32_t WS_M = 98304;       // M bf16, K-major swizzled, 64 x 64
-constexpr uint32_t WS_CHUNK = 106496;
-// The state pass loads [WS_AC, WS_QP) for its chain product and [WS_QP, WS_CHUNK) for the output.
-constexpr uint32_t WS_CHAIN_BYTES = WS_QP - WS_AC, WS_OUT_BYTES = WS_CHUNK - WS_QP;
-// Chunk j of row r of B_c^T (16 chunks a row) sits at position j ^ (r % 8): the lanes of a warp
-// reading (or writing) one chunk of 8 consecutive rows hit eight distinct 16-byte bank groups.
-__host__ __device__ constexpr uint32_t bc_off(int row, int j) { return (uint32_t)(row * 256 + ((j ^ (row & 7)) << 4)); }
+constexpr uint32_t WS_M = 81920;       // M bf16, K-major swizzled, 64 x 64
+constexpr uint32_t WS_CHUNK = 90112;
+// The state pass loads [WS_AC, WS_QP) (A_c, K_end, U~^T) for its chain products and
+// [WS_UT, WS_CHUNK) (U~^T, Q', M) for the output: U~^T goes into both stages.
+constexpr uint32_t WS_CHAIN_BYTES = WS_QP - WS_AC, WS_OUT_BYTES = WS_CHUNK - WS_UT;
 // Ready flags: one 32-bit word per chunk-head after the images, set to 1 once the chunk-head's
 // images are complete in global memory (cleared before every forward).
 __host__ __device__ constexpr size_t flags_offset(size_t n_chunk_heads) { return n_chunk_heads * WS_CHUNK; }
@@ -99,12 +97,10 @@ constexpr uint32_t S_TB = S_R;               // T' bf16 K-major 64 x 64
 constexpr uint32_t S_X = S_R + 8192;         // X0, X1 fp32 [16][24] each
 constexpr uint32_t S_Y = S_R + 11264;        // Y fp32 [32][40]
 // staging of the chunk's workspace image, over buffers that are dead by then
-// (U~^T and M are stored straight from S_U and S_M)
+// (K_end, U~^T and M are stored straight from S_KE, S_U and S_M)
 constexpr uint32_t S_OUT_QP = S_R;            // Q' image (16 KB)
-constexpr uint32_t S_OUT_BC0 = S_KE;          // B_c^T rows 0..63 (16 KB, over K_end)
 constexpr uint32_t S_OUT_AC = S_A;            // A_c image (32 KB, over A and part of T)
-constexpr uint32_t S_OUT_BC1 = S_A + 32768;   // B_c^T rows 64..127 (16 KB, over T and part of W)
-static_assert(S_OUT_BC1 + 16384 <= S_U, "staging must stay clear of U~^T");
+static_assert(S_OUT_AC + 32768 <= S_W, "the A_c image must stay clear of W and U~^T");
 // small arrays
 constexpr uint32_t SM_P = S_SM;                  // signed block totals of alpha, fp32 [4][128]
 constexpr uint32_t SM_GC = S_SM + 2048;          // gamma_C fp32 [128] (signed)
@@ -801,19 +797,16 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
         __syncthreads();
         tc::tc_fence_after();
 
-        // ======== F: M W (M = 64) -> Q', K_end^T W (M = 128) -> A_c,
-        //             U~^T K_end (M = 128) -> B_c^T ========
-        // (the chunk's own output M U~ is left to the state pass, which accumulates it in fp32
-        // next to Q' S0 from the U~^T and M images)
+        // ======== F: M W (M = 64) -> Q', K_end^T W (M = 128) -> A_c ========
+        // (B_c = K_end^T U~ and the chunk's own output M U~ are left to the state pass, which
+        // forms them in fp32 accumulators from the K_end, U~^T and M images)
         if (warp == 0) {
             const uint64_t md = tc::smem_desc_sw128(tc::smem_u32(sm + S_M), 16, 1024);
             const uint64_t ked = tc::smem_desc_sw128(tc::smem_u32(sm + S_KE), 8192, 1024);
             const uint64_t wd = tc::smem_desc_sw128(tc::smem_u32(sm + S_W), 16, 1024);
-            const uint64_t ud = tc::smem_desc_sw128(tc::smem_u32(sm + S_U), 16, 1024);
             const uint32_t id_q = tc::idesc_bf16_f32(64, 128, 0, 0);
             const uint32_t id_c = tc::idesc_bf16_f32(128, 128, 1, 0);
-            const uint32_t id_b = tc::idesc_bf16_f32(128, 128, 0, 1);
-            // product by product, M W first: the Q' read-back overlaps the other two
+            // M W first: the Q' read-back overlaps K_end^T W
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)                                  // M W
                 tc::mma_bf16_warp(tmem, tc::desc_add(md, ks * 32), tc::desc_add(wd, ks * 32), id_q, ks > 0);
@@ -821,9 +814,6 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)                                  // K_end^T W
                 tc::mma_bf16_warp(tmem + 192, tc::desc_add(ked, ks * 2048), tc::desc_add(wd, ks * 32), id_c, ks > 0);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)                                  // U~^T K_end
-                tc::mma_bf16_warp(tmem + 320, tc::desc_add(ud, ks * 32), tc::desc_add(ked, ks * 2048), id_b, ks > 0);
             tc::mma_commit_warp(bar);
         }
         // The previous chunk-head's stores, issued at its end, have landed by now: flag it ready.
@@ -859,35 +849,26 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
                     }
                 }
             }
-            // (2) M = 128 products, lane = row c' (A_c) or dv column (B_c^T)
+            // (2) A_c = Diag(gamma_C) - K_end^T W (M = 128, lane = row c'): warp w reads columns
+            // 32 (w / 4) .. + 31 of rows 32 (w % 4) + lane
             tc::mbar_wait(bar, phase & 1, abort_flag);
             ++phase;
             tc::tc_fence_after();
             {
                 const int cr = 32 * quarter + lane;
-                const int n0 = 64 * (slice & 1);
-                const float gc = gGC[cr];
-                float x[64];
-                tc::tmem_ld64_sync(tc::tmem_addr(tmem, 32 * quarter, (slice < 2 ? 192 : 320) + n0), x);
+                const int n0 = 32 * slice;
+                float x[32];
+                tc::tmem_ld32_sync(tc::tmem_addr(tmem, 32 * quarter, 192 + n0), x);
+                // the diagonal element of row cr lies in this slice when slice == quarter, at x[lane]
+                const float dx = slice == quarter ? select_lane(x, lane) : 0.f;
 #pragma unroll
-                for (int c0 = 0; c0 < 64; c0 += 8) {
-                    const int n = n0 + c0;
-                    if (slice < 2) {
-                        float y[8];
+                for (int c0 = 0; c0 < 32; c0 += 8) {
+                    float y[8];
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) y[i] = -x[c0 + i];
-                        st16(sm + S_OUT_AC, tc::sw128_kmajor(cr, n, 128), y);
-                    } else {
-                        // rows 0..63 over K_end, rows 64..127 in the second staging half
-                        st16(sm + (quarter < 2 ? S_OUT_BC0 : S_OUT_BC1 - 16384), bc_off(cr, n >> 3), x + c0);
-                    }
+                    for (int i = 0; i < 8; ++i) y[i] = -x[c0 + i];
+                    st16(sm + S_OUT_AC, tc::sw128_kmajor(cr, n0 + c0, 128), y);
                 }
-                // A_c = Diag(gamma_C) - K_end^T W: row c' holds its diagonal element in this slice
-                // when c' / 64 == slice, at x[32 (quarter % 2) + lane]
-                if (slice < 2 && slice == (quarter >> 1)) {
-                    const float dx = (quarter & 1) ? select_lane(x + 32, lane) : select_lane(x, lane);
-                    st_bf16(sm + S_OUT_AC, tc::sw128_kmajor(cr, cr, 128), gc - dx);
-                }
+                if (slice == quarter) st_bf16(sm + S_OUT_AC, tc::sw128_kmajor(cr, cr, 128), gGC[cr] - dx);
             }
         }
         tc::fence_proxy_async_smem();
@@ -895,14 +876,13 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
         __syncthreads();
         tc::tc_fence_after();
         if (tid == kStoreTid) {
-            // group 1: the images over buffers the next row pass rewrites first (Q' over R,
-            // the first half of B_c^T over K_end)
+            // group 1: the images over buffers the next row pass rewrites first (Q' over R, K_end
+            // straight from its operand tile)
             tc::bulk_s2g(wsc + WS_QP, sm + S_OUT_QP, 16384);
-            tc::bulk_s2g(wsc + WS_BC, sm + S_OUT_BC0, 16384);
+            tc::bulk_s2g(wsc + WS_KE, sm + S_KE, 16384);
             tc::bulk_commit();
-            // group 2: the rest, U~^T and M straight from the product operands
+            // group 2: A_c, then U~^T and M straight from their operand tiles
             tc::bulk_s2g(wsc + WS_AC, sm + S_OUT_AC, 32768);
-            tc::bulk_s2g(wsc + WS_BC + 16384, sm + S_OUT_BC1, 16384);
             tc::bulk_s2g(wsc + WS_UT, sm + S_U, 16384);
             tc::bulk_s2g(wsc + WS_M, sm + S_M, 8192);
             tc::bulk_commit();
@@ -923,17 +903,20 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
 // One CTA of 512 threads carries whole heads (all 128 dv columns), one head after the other; its
 // items u = k NT + c run over (head k of the CTA, chunk c).  The state is kept transposed: S^T
 // (dv x dk) lives in Tensor Memory as the A operand of both products,
-//     D_c^T = S^T A_c^T  (M = 128 dv, N = 128, K = 128)           -> S_next^T = D_c^T + B_c^T
-//     D_o^T = S^T Q'^T + U~^T M^T  (M = 128 dv, N = 64 tokens)     -> O^T = scale D_o^T
-// so the chunk's own output M U~ is accumulated in fp32 next to Q' S0 and never rounded.
+//     D_c^T = U~^T K_end + S^T A_c^T  (M = 128 dv, N = 128)         -> S_next^T = D_c^T
+//     D_o^T = S^T Q'^T + U~^T M^T      (M = 128 dv, N = 64 tokens)  -> O^T = scale D_o^T
+// so B_c = K_end^T U~ and the chunk's own output M U~ are accumulated in fp32 and never rounded.
+// The U~^T K_end part needs no state: it is issued as soon as the epilogue has read the previous
+// accumulator, while the epilogue is still rounding and writing S^T.
 // Warp roles:
 //   warps 0-7    chain epilogue: warp w owns dv columns 32 (w % 4) .. + 31 (its TMEM lanes) and
-//                state rows 64 (w / 4) .. + 63; S_next^T in fp32, written back into TMEM as the
-//                bf16 operand of the next products (hT in fp32 after a head's last chunk)
+//                state rows 64 (w / 4) .. + 63; reads S_next^T in fp32 and writes it back into
+//                TMEM as the bf16 operand of the next products (hT in fp32 after a head's last
+//                chunk)
 //   warp 8       chain issue
 //   warp 9       output issue
-//   warp 10      chain loads: A_c and B_c^T of each item (one 64 KB bulk copy, two stages)
-//   warp 11      output loads: Q', U~^T and M of each item (one 40 KB bulk copy, two stages)
+//   warp 10      chain loads: A_c, K_end and U~^T of each item (one 64 KB bulk copy, two stages)
+//   warp 11      output loads: U~^T, Q' and M of each item (one 40 KB bulk copy, two stages)
 //   warps 12-15  output epilogue: lane = dv column; the chunk's 64 x 128 output tile goes through
 //                a shared-memory staging tile and leaves with one tensor (TMA) store
 // Only the chain roles are on the serial path.  The output product of item u is issued once the
@@ -941,15 +924,16 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
 // alternates between two TMEM buffers: S_{u+1}^T goes into the buffer of S_{u-1}^T once the
 // output product of item u - 1 has read it.  Every load of an item waits for the item's ready
 // flag, every role issues from a converged warp (one elected lane) and every wait is bounded.
-constexpr uint32_t SS_C = 0;             // chain stages: A_c (32 KB) then B_c^T (32 KB)
+constexpr uint32_t SS_C = 0;             // chain stages: A_c (32 KB), K_end (16 KB), U~^T (16 KB)
 constexpr uint32_t SS_CSTAGE = WS_CHAIN_BYTES;
-constexpr uint32_t SS_O = 2 * SS_CSTAGE; // output stages: Q' (16 KB), U~^T (16 KB), M (8 KB)
+constexpr uint32_t SS_O = 2 * SS_CSTAGE; // output stages: U~^T (16 KB), Q' (16 KB), M (8 KB)
 constexpr uint32_t SS_OSTAGE = WS_OUT_BYTES;
 constexpr uint32_t SS_STG = SS_O + 2 * SS_OSTAGE;   // output tile bf16 [64 tokens][128 dv]
 constexpr uint32_t SS_BAR = SS_STG + 16384;
 constexpr uint32_t SS_BYTES = SS_BAR + 256 + 1024;
 constexpr uint32_t FUSED_BYTES = SS_BYTES > S_BYTES ? SS_BYTES : S_BYTES;
-static_assert(SS_OSTAGE % 1024 == 0 && (WS_UT - WS_QP) % 1024 == 0 && (WS_M - WS_QP) % 1024 == 0,
+static_assert(SS_OSTAGE % 1024 == 0 && (WS_QP - WS_UT) % 1024 == 0 && (WS_M - WS_UT) % 1024 == 0 &&
+                  (WS_KE - WS_AC) % 1024 == 0 && (WS_UT - WS_AC) % 1024 == 0,
               "operand tiles of a stage must stay 1024-byte aligned");
 // TMEM columns: D_c^T 0..127, S^T buffers of 64 (bf16 pairs) from 128, D_o^T buffers of 64 from 256
 constexpr uint32_t kColS = 128, kColO = 256;
@@ -959,8 +943,8 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
                                            __nv_bfloat16* __restrict__ out, float* __restrict__ hT,
                                            int T_len, int H, int NT, int BH, float scale, int head0,
                                            int hstride) {
-    uint64_t* full_c = reinterpret_cast<uint64_t*>(sm + SS_BAR);   // [2] A_c, B_c^T landed
-    uint64_t* empty_c = full_c + 2;     // [2] chain stage consumed (8 epilogue warps)
+    uint64_t* full_c = reinterpret_cast<uint64_t*>(sm + SS_BAR);   // [2] A_c, K_end, U~^T landed
+    uint64_t* empty_c = full_c + 2;     // [2] chain stage read by the chain products (commit)
     uint64_t* full_o = empty_c + 2;     // [2] Q', U~^T, M landed
     uint64_t* empty_o = full_o + 2;     // [2] output stage read by the output product (commit)
     uint64_t* mma_c = empty_o + 2;      // D_c^T complete
@@ -968,7 +952,8 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
     uint64_t* dc_done = s_ready + 2;    // [2] D_c^T of the item using S^T buffer b complete
     uint64_t* mma_o = dc_done + 2;      // [4] D_o^T complete
     uint64_t* o_free = mma_o + 4;       // [4] D_o^T read back (4 output-epilogue warps)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_free + 4);
+    uint64_t* dc_free = o_free + 4;     // D_c^T read back (8 chain-epilogue warps)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(dc_free + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -980,9 +965,10 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
         tc::tmem_relinquish();
     }
     if (tid == 32) {
+        tc::mbar_init(dc_free, 8);
         for (int s = 0; s < 2; ++s) {
             tc::mbar_init(&full_c[s], 1);
-            tc::mbar_init(&empty_c[s], 8);
+            tc::mbar_init(&empty_c[s], 1);
             tc::mbar_init(&full_o[s], 1);
             tc::mbar_init(&empty_o[s], 1);
             tc::mbar_init(&s_ready[s], 8);
@@ -1039,22 +1025,13 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
             put_s(0);
         }
         for (int u = 0, c = 0, bh = head0; u < U; ++u) {
-            const int st = u & 1;
-            if (!wait(&full_c[st], (u >> 1) & 1)) break;
             if (!wait(mma_c, u & 1)) break;
             tc::tc_fence_after();
             tc::tmem_ld64_sync(tc::tmem_addr(tmem, 32 * q, cb), S);
-            const uint8_t* bcs = sm + SS_C + st * SS_CSTAGE + (WS_BC - WS_AC);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                float y[8];
-                unpack8(*reinterpret_cast<const uint4*>(bcs + bc_off(n, 8 * hf + j)), y);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) S[8 * j + i] += y[i];
-            }
-            // A_c was read by the finished product and B_c^T is in registers: release the stage
+            // the accumulator is read: the next item's state-free part may go in
+            tc::tc_fence_before();
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&empty_c[st]);
+            if (lane == 0) tc::mbar_arrive(dc_free);
             const bool last = c == NT - 1;
             if (last && hT && !*abort_flag) {
                 float* dst = hT + ((size_t)bh * kDK + cb) * kDV + n;
@@ -1076,12 +1053,23 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
             }
         }
     } else if (warp == 8) {
-        // ---- chain issue: A = S^T (TMEM), B = A_c^T (the K-major A_c image read as K-major B) ----
+        // ---- chain issue: D_c^T = U~^T K_end (both from the stage: K-major A, MN-major B) and
+        // then + S^T A_c^T (A = S^T from TMEM, B = the K-major A_c image read as K-major B) ----
         const uint32_t idc = tc::idesc_bf16_f32(128, 128, 0, 0);
+        const uint32_t idb = tc::idesc_bf16_f32(128, 128, 0, 1);
+        const uint64_t k_desc0 = tc::smem_desc_sw128(tc::smem_u32(sm + SS_C + (WS_KE - WS_AC)), 8192, 1024);
+        const uint64_t u_desc0 = tc::smem_desc_sw128(tc::smem_u32(sm + SS_C + (WS_UT - WS_AC)), 16, 1024);
         const uint64_t c_desc0 = tc::smem_desc_sw128(tc::smem_u32(sm + SS_C), 16, 1024);
         for (int u = 0; u < U; ++u) {
             const int st = u & 1;
             if (!wait(&full_c[st], (u >> 1) & 1)) break;
+            // the epilogue has read the previous accumulator
+            if (u >= 1 && !wait(dc_free, (u - 1) & 1)) break;
+            tc::tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                tc::mma_bf16_warp(tmem, tc::desc_add(u_desc0, st * SS_CSTAGE + ks * 32),
+                                  tc::desc_add(k_desc0, st * SS_CSTAGE + ks * 2048), idb, ks > 0 ? 1u : 0u);
             if (!wait(&s_ready[st], (u >> 1) & 1)) break;
             tc::tc_fence_after();
             const uint64_t bd = tc::desc_add(c_desc0, st * SS_CSTAGE);
@@ -1089,9 +1077,10 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
                 tc::mma_bf16_tmem_a_warp(tmem, a + 8 * ks, tc::desc_add(bd, (ks >> 2) * 16384 + (ks & 3) * 32),
-                                         idc, ks > 0 ? 1u : 0u);
+                                         idc, 1u);
             tc::mma_commit_warp(mma_c);
             tc::mma_commit_warp(&dc_done[st]);
+            tc::mma_commit_warp(&empty_c[st]);
         }
     } else if (warp == 9) {
         // ---- output issue: S^T Q'^T (A in TMEM) + U~^T M^T (both from shared memory) ----
@@ -1110,12 +1099,13 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
             const uint32_t a = tmem + kColS + 64 * st;
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)                                  // S^T Q'^T
-                tc::mma_bf16_tmem_a_warp(d, a + 8 * ks, tc::desc_add(od, (ks >> 2) * 8192 + (ks & 3) * 32),
+                tc::mma_bf16_tmem_a_warp(d, a + 8 * ks,
+                                         tc::desc_add(od, (WS_QP - WS_UT) + (ks >> 2) * 8192 + (ks & 3) * 32),
                                          ido, ks > 0 ? 1u : 0u);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)                                  // + U~^T M^T
-                tc::mma_bf16_warp(d, tc::desc_add(od, (WS_UT - WS_QP) + ks * 32),
-                                  tc::desc_add(od, (WS_M - WS_QP) + ks * 32), ido, 1u);
+                tc::mma_bf16_warp(d, tc::desc_add(od, ks * 32), tc::desc_add(od, (WS_M - WS_UT) + ks * 32),
+                                  ido, 1u);
             tc::mma_commit_warp(&mma_o[ob]);
             tc::mma_commit_warp(&empty_o[st]);
         }
@@ -1139,7 +1129,7 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
                 }
                 if (!flag_wait(flags + ci, abort_flag)) break;
                 tc::mbar_arrive_expect_tx(&fullb[st], bytes);
-                tc::bulk_g2s(stage0 + st * bytes, ws + ci * WS_CHUNK + (chain ? WS_AC : WS_QP), bytes,
+                tc::bulk_g2s(stage0 + st * bytes, ws + ci * WS_CHUNK + (chain ? WS_AC : WS_UT), bytes,
                              &fullb[st]);
             }
             if (*abort_flag) {

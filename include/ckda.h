@@ -185,8 +185,8 @@ CKDA_API ckda_status ckda_selftest_umma(const void* A, const void* B, float* D, 
  * until the process exits.  The function allocates nothing.
  *   Arguments and results: as ckda_fwd_chunked, minus workspace / workspace_bytes.
  *   Limit: problems whose ckda_fwd_workspace_bytes(...) exceeds CKDA_NOALLOC_MAX_WORKSPACE are
- *          rejected with CKDA_ERR_WORKSPACE before anything is launched (16 MiB holds 157
- *          chunk-heads of the tensor-core path: B * H * ceil(T / 64) <= 157).
+ *          rejected with CKDA_ERR_WORKSPACE before anything is launched (16 MiB holds 186
+ *          chunk-heads of the tensor-core path: B * H * ceil(T / 64) <= 186).
  *   Set-up: the first call on a device looks up the array's device address (cudaGetSymbolAddress,
  *          with that device current); make that first call before any stream capture.
  *   Sharing: every call uses the same array, which keeps the last call's contents (no part of it

@@ -90,7 +90,7 @@ def test_replicas_reduce_max_and_use_disjoint_inputs(tmp_path):
     for r in (0, 1):
         assert out[r]["ms_max"] == pytest.approx(0.40)
         assert out[r]["value"] == pytest.approx(4096 * 2 / 0.40e-3 / 1e6)
-        assert out[r]["ws"] == 2 * 16 * 32 * 106496 + 2 * 16 * 32 * 4
+        assert out[r]["ws"] == 2 * 16 * 32 * 90112 + 2 * 16 * 32 * 4
     assert not set(out[0]["seeds"]) & set(out[1]["seeds"])
 
 

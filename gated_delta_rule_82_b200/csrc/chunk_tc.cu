@@ -50,6 +50,7 @@
 // ready flags of their heads while the factor CTAs produce them, so the serial pass hides behind
 // the chunk-parallel work instead of following it.
 #include <cuda.h>
+#include <mutex>
 #include <cudaTypedefs.h>
 
 #include "fastdiv.h"
@@ -369,6 +370,15 @@ struct WorkOrder {
         return it;
     }
 };
+// The items one factor CTA takes: a leading run start1, start1 + stride1, ... (n1 of them), then
+// start2, start2 + stride2, ... up to `total` (none when start2 >= total).
+struct ItemSeq {
+    int start1, stride1, n1, start2, stride2, total;
+    __device__ __forceinline__ int at(int k) const {
+        const int i = k < n1 ? start1 + k * stride1 : start2 + (k - n1) * stride2;
+        return i < total ? i : -1;
+    }
+};
 inline WorkOrder make_work_order(int NT, int BH, int H, int G) {
     WorkOrder w;
     w.G = G;
@@ -426,14 +436,14 @@ __device__ __forceinline__ bool mbar_wait_long(uint64_t* bar, uint32_t parity, v
     }
 }
 
-// ---- the factor role: chunk-heads wo.ci(i) for i = rank, rank + nprog, ... ----------------------
+// ---- the factor role: chunk-heads wo.item(i) for the items i of `seq` -----------------------------
 // kLogits: alpha and beta hold logits (alpha = 2 sigma(a) - 1 from bf16 a, beta = 2 sigma(b)).
 template <bool kLogits>
 __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, const void* __restrict__ alpha,
                                            const float* __restrict__ beta, uint8_t* __restrict__ ws,
-                                           int* __restrict__ flags, int T_len, int H, int NT, int total,
-                                           WorkOrder wo, int rank, int nprog, int l2norm,
-                                           const RopeParams& rp, long long pos_offset) {
+                                           int* __restrict__ flags, int T_len, int H, int NT,
+                                           WorkOrder wo, ItemSeq seq, int l2norm,
+                                           const RopeParams& rp, long long pos_offset, uint32_t tmem) {
     constexpr int gate_logits = kLogits ? 1 : 0;
     float* G = reinterpret_cast<float*>(sm + S_G);
     float* gP = reinterpret_cast<float*>(sm + SM_P);
@@ -441,7 +451,6 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
     float* sb = reinterpret_cast<float*>(sm + SM_B);
     int* exact_path = reinterpret_cast<int*>(sm + SM_FLAGS);
     volatile int* abort_flag = exact_path + 4;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(exact_path + 8);
     uint64_t* bar = reinterpret_cast<uint64_t*>(exact_path + 16);   // tensor-core completions
     uint64_t* bar_in = bar + 1;                                     // alpha, q, k landed
     uint64_t* bar_v = bar + 2;                                      // V landed
@@ -457,10 +466,6 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
     const size_t rs = (size_t)H;   // stride between tokens, in rows of [B*T*H]
     tc::grid_launch_dependents();   // the state pass may start its set-up early
 
-    if (warp == 0) {
-        tc::tmem_alloc(tmem_slot, 512);
-        tc::tmem_relinquish();
-    }
     // RoPE inverse frequencies in shared memory: lanes index them by channel group, and a
     // per-lane index into the kernel-parameter array would serialise in the constant cache
     double* sfreq = reinterpret_cast<double*>(sm + SM_FREQ);
@@ -477,17 +482,17 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
     uint32_t phase = 0;   // completions of `bar` so far
     // the set-up above may overlap the previous kernel in the stream; from here on the kernel
     // reads the caller's inputs and writes the workspace, so it waits for that kernel
     tc::grid_dependency_wait();
-    if (tid == 0 && rank < total) {
+    const int i0 = seq.at(0);
+    if (tid == 0 && i0 >= 0) {
         tc::prefetch_tensormap(&maps.q);
         tc::prefetch_tensormap(&maps.k);
         tc::prefetch_tensormap(&maps.v);
         tc::prefetch_tensormap(&maps.alpha);
-        const Item first = wo.item(rank);
+        const Item first = wo.item(i0);
         issue_inputs(maps, sm, bar_in, first.b, first.h, first.c * kC, gate_logits);
         issue_v(maps, sm, bar_v, first.b, first.h, first.c * kC);
     }
@@ -495,13 +500,14 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
     // persistent loop over items; chunk-head ci = (batch*head) * NT + chunk
     uint32_t it = 0;
     int pending = -1;   // chunk-head whose images are stored but not yet flagged ready
-    for (int i = rank; i < total; i += nprog, ++it) {
+    for (int k = 0, i = i0; i >= 0; i = seq.at(++k), ++it) {
         const Item cur = wo.item(i);
         const int ci = cur.bh * NT + cur.c;
         const int t0 = cur.c * kC;
         const int nvalid = min(kC, T_len - t0);
-        const bool has_next = i + nprog < total;
-        const Item nxt = wo.item(has_next ? i + nprog : i);
+        const int inext = seq.at(k + 1);
+        const bool has_next = inext >= 0;
+        const Item nxt = wo.item(has_next ? inext : i);
         uint8_t* wsc = ws + (size_t)ci * WS_CHUNK;
         const size_t row0 = ((size_t)cur.b * T_len + t0) * H + cur.h;
         float bval = (tid < 64 && tid < nvalid) ? beta[row0 + tid * rs] : 0.f;
@@ -896,7 +902,17 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
     tc::tc_fence_before();
     __syncthreads();
     if (*abort_flag && tid == 0) atomicExch(&g_tc_error, 1);
-    if (warp == 0) tc::tmem_dealloc(tmem, 512);
+    // the CTA may go on to another role over this shared memory, whose copies (async proxy) must
+    // come after this role's plain writes
+    tc::fence_proxy_async_smem();
+    if (tid == 32) {
+        tc::mbar_inval(bar);
+        tc::mbar_inval(bar_in);
+        tc::mbar_inval(bar_v);
+        tc::mbar_inval(bar_w);
+        tc::mbar_inval(bar_q);
+    }
+    __syncthreads();
 }
 
 // ---- the state role: the serial pass over the chunks of heads head0, head0 + hstride, ... ---------
@@ -942,7 +958,7 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
                                            const int* __restrict__ flags, const float* __restrict__ h0,
                                            __nv_bfloat16* __restrict__ out, float* __restrict__ hT,
                                            int T_len, int H, int NT, int BH, float scale, int head0,
-                                           int hstride) {
+                                           int hstride, uint32_t tmem) {
     uint64_t* full_c = reinterpret_cast<uint64_t*>(sm + SS_BAR);   // [2] A_c, K_end, U~^T landed
     uint64_t* empty_c = full_c + 2;     // [2] chain stage read by the chain products (commit)
     uint64_t* full_o = empty_c + 2;     // [2] Q', U~^T, M landed
@@ -953,17 +969,12 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
     uint64_t* mma_o = dc_done + 2;      // [4] D_o^T complete
     uint64_t* o_free = mma_o + 4;       // [4] D_o^T read back (4 output-epilogue warps)
     uint64_t* dc_free = o_free + 4;     // D_c^T read back (8 chain-epilogue warps)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(dc_free + 1);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(dc_free + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nheads = head0 < BH ? (BH - head0 + hstride - 1) / hstride : 0;
     const int U = nheads * NT;
 
-    if (warp == 0) {
-        tc::tmem_alloc(tmem_slot, 512);
-        tc::tmem_relinquish();
-    }
     if (tid == 32) {
         tc::mbar_init(dc_free, 8);
         for (int s = 0; s < 2; ++s) {
@@ -988,7 +999,6 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
     // a launch after the factor kernel waits for it here (no effect otherwise)
     tc::grid_dependency_wait();
     tc::grid_launch_dependents();
-    const uint32_t tmem = *tmem_slot;
     auto wait = [&](uint64_t* bar, uint32_t parity) {
         return __all_sync(0xffffffffu, mbar_wait_long(bar, parity, abort_flag));
     };
@@ -1185,11 +1195,29 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
     tc::tc_fence_before();
     __syncthreads();
     if (*abort_flag && tid == 0) atomicExch(&g_tc_error, 2);
-    if (warp == 0) tc::tmem_dealloc(tmem, 512);
 }
 
 __device__ __forceinline__ uint8_t* aligned_smem(uint8_t* raw) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+}
+
+// Tensor Memory belongs to the kernel, not to a role: one allocation of all 512 columns (one CTA
+// per SM), after which the CTA gives up its permit to allocate, so a CTA that changes role keeps
+// the same columns.
+__device__ __forceinline__ uint32_t kernel_tmem_alloc(uint32_t* slot) {
+    if ((threadIdx.x >> 5) == 0) {
+        tc::tmem_alloc(slot, 512);
+        tc::tmem_relinquish();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    return *slot;
+}
+__device__ __forceinline__ void kernel_tmem_free(uint32_t tmem) {
+    tc::tc_fence_before();
+    __syncthreads();
+    if ((threadIdx.x >> 5) == 0) tc::tmem_dealloc(tmem, 512);
 }
 
 // Factor kernel alone: persistent over every chunk-head (chunk-major over all heads).
@@ -1200,8 +1228,12 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const void* __restrict__ alph
               int T_len, int H, int NT, int BH, WorkOrder wo, int l2norm, RopeParams rp,
               long long pos_offset) {
     extern __shared__ uint8_t smem_raw[];
-    intra_role<kLogits>(aligned_smem(smem_raw), maps, alpha, beta, ws, flags, T_len, H, NT, BH * NT,
-                        wo, blockIdx.x, gridDim.x, l2norm, rp, pos_offset);
+    __shared__ uint32_t tmem_slot;
+    const uint32_t tmem = kernel_tmem_alloc(&tmem_slot);
+    const ItemSeq seq{(int)blockIdx.x, (int)gridDim.x, 1 << 30, 0, 1, BH * NT};
+    intra_role<kLogits>(aligned_smem(smem_raw), maps, alpha, beta, ws, flags, T_len, H, NT, wo, seq,
+                        l2norm, rp, pos_offset, tmem);
+    kernel_tmem_free(tmem);
 }
 
 // State pass alone, after the factor kernel: heads blockIdx.x, blockIdx.x + gridDim.x, ...
@@ -1211,27 +1243,40 @@ ckda_tc_state(const __grid_constant__ TcMaps maps, const uint8_t* __restrict__ w
               __nv_bfloat16* __restrict__ out, float* __restrict__ hT, int T_len, int H, int NT,
               int BH, float scale) {
     extern __shared__ uint8_t smem_raw[];
+    __shared__ uint32_t tmem_slot;
+    const uint32_t tmem = kernel_tmem_alloc(&tmem_slot);
     state_role(aligned_smem(smem_raw), maps, ws, flags, h0, out, hT, T_len, H, NT, BH, scale,
-               blockIdx.x, gridDim.x);
+               blockIdx.x, gridDim.x, tmem);
+    kernel_tmem_free(tmem);
 }
 
-// Both at once (cooperative launch, every CTA resident): CTAs 0 .. n_state - 1 carry the chains
-// of heads blockIdx.x + k n_state, the others run the factor role over the items in head groups
-// of n_state, so the chains of a group run while the group's chunks are produced.
+// Both at once (cooperative launch, every CTA resident).  Every CTA first takes `lead` rounds of
+// factor items (item blockIdx.x + r gridDim.x, r < lead); then CTAs 0 .. n_state - 1 carry the
+// chains of heads blockIdx.x + k n_state, and the others take the remaining items in turn.  The
+// items run in head groups of n_state, chunk-major inside a group, so the chains of a group run
+// while the group's chunks are produced.  A chain CTA waits only on flags that factor work
+// raises, and factor work never waits on a chain, so every wait ends.
 template <bool kLogits>
 __global__ void __launch_bounds__(512, 1)
 ckda_tc_fused(const __grid_constant__ TcMaps maps, const void* __restrict__ alpha,
               const float* __restrict__ beta, uint8_t* __restrict__ ws, int* __restrict__ flags,
               const float* __restrict__ h0, __nv_bfloat16* __restrict__ out, float* __restrict__ hT,
-              int T_len, int H, int NT, int BH, int n_state, WorkOrder wo, int l2norm,
+              int T_len, int H, int NT, int BH, int n_state, int lead, WorkOrder wo, int l2norm,
               RopeParams rp, long long pos_offset, float scale) {
     extern __shared__ uint8_t smem_raw[];
+    __shared__ uint32_t tmem_slot;
     uint8_t* sm = aligned_smem(smem_raw);
-    if ((int)blockIdx.x < n_state)
-        state_role(sm, maps, ws, flags, h0, out, hT, T_len, H, NT, BH, scale, blockIdx.x, n_state);
-    else
-        intra_role<kLogits>(sm, maps, alpha, beta, ws, flags, T_len, H, NT, BH * NT, wo,
-                            blockIdx.x - n_state, gridDim.x - n_state, l2norm, rp, pos_offset);
+    const uint32_t tmem = kernel_tmem_alloc(&tmem_slot);
+    const int total = BH * NT, b = blockIdx.x, nall = gridDim.x, nf = nall - n_state;
+    const bool chain = b < n_state;
+    // the leading rounds, then (factor CTAs) every nf-th of the remaining items
+    const ItemSeq seq{b, nall, lead, chain ? total : lead * nall + (b - n_state), chain ? 1 : nf, total};
+    if (seq.at(0) >= 0)
+        intra_role<kLogits>(sm, maps, alpha, beta, ws, flags, T_len, H, NT, wo, seq, l2norm, rp,
+                            pos_offset, tmem);
+    if (chain)
+        state_role(sm, maps, ws, flags, h0, out, hT, T_len, H, NT, BH, scale, b, n_state, tmem);
+    kernel_tmem_free(tmem);
 }
 
 }  // namespace
@@ -1272,41 +1317,71 @@ size_t chunk_tc_workspace_bytes(int B, int T_len, int H) {
     return flags_offset(n) + ((n * 4 + 255) & ~(size_t)255);
 }
 
-// Chain CTAs of the fused launch.  Model (SM cycles, measured on B200): a factor item takes
-// t_i = 18800 and the factor CTAs work in lockstep rounds, an item is flagged ready about two
-// rounds after the round it starts in, and a chain step takes t_c = 2400.  With s chain CTAs the
-// heads form groups of s, produced one after the other (chunk-major inside a group); chain CTA 0
-// carries the first head of every group, one after the other, so it finishes last.  Its head in
+// Split of the fused launch: `n_state` chain CTAs, and `lead` leading rounds of factor items that
+// every CTA (chain CTAs included) takes before the chains start.  Model (SM cycles, measured on
+// B200): a round of factor items takes t_i = 19000 on every CTA in step, an item is flagged ready
+// about 1.5 rounds after the round it starts in, and a chain step takes t_c = 2200.  With s chain
+// CTAs the heads form groups of s, produced one after the other (chunk-major inside a group);
+// chain CTA 0 carries the first head of every group in turn, so it finishes last.  Its head in
 // group g cannot end before the previous head plus NT steps, before that head's first chunk plus
-// NT steps, or before its last chunk plus one step.  s minimises the later of that end and the
-// end of the factor work (the larger s on ties).
-int chunk_tc_state_ctas(int BH, int NT, int nsm) {
-    const double ti = 18800.0, tc = 2400.0;
+// NT steps, or before its last chunk plus one step (and no chain starts before the leading rounds
+// are done).  The split minimises the later of that end and the end of the factor work (the
+// larger s and the smaller lead on ties).
+void chunk_tc_plan(int BH, int NT, int nsm, int* n_state, int* lead) {
+    struct Entry {
+        int BH, NT, nsm, s, lead;
+    };
+    static std::mutex m;
+    static Entry cache[16];
+    static int n_cached = 0;
+    {
+        std::lock_guard<std::mutex> g(m);
+        for (int e = 0; e < n_cached; ++e)
+            if (cache[e].BH == BH && cache[e].NT == NT && cache[e].nsm == nsm) {
+                *n_state = cache[e].s;
+                *lead = cache[e].lead;
+                return;
+            }
+    }
+    const double ti = 19000.0, tc = 2200.0, lag = 1.5;
     const long long total = (long long)BH * NT;
     const int smax = BH < nsm - 1 ? BH : nsm - 1;
-    int best = 1;
+    const int lmax = (int)((total + nsm - 1) / nsm) < 8 ? (int)((total + nsm - 1) / nsm) : 8;
+    int best_s = 1, best_l = 0;
     double best_t = 1e300;
     for (int s = 1; s <= smax; ++s) {
-        const long long ni = (long long)(nsm - s) < total ? (long long)(nsm - s) : total;
-        const double factor_end = (double)((total + ni - 1) / ni) * ti;
-        double end = 0.0;
-        for (int g = 0; g * s < BH; ++g) {
-            const long long sg = BH - (long long)g * s < s ? BH - (long long)g * s : s;
-            const long long first = (long long)g * s * NT;
-            const double t_first = (double)(first / ni + 2) * ti;
-            const double t_last = (double)((first + (long long)(NT - 1) * sg) / ni + 2) * ti;
-            double e = end + NT * tc;
-            if (t_first + NT * tc > e) e = t_first + NT * tc;
-            if (t_last + tc > e) e = t_last + tc;
-            end = e;
-        }
-        const double t = end > factor_end ? end : factor_end;
-        if (t <= best_t) {
-            best_t = t;
-            best = s;
+        const long long nf = nsm - s;
+        for (int l = 0; l <= lmax; ++l) {
+            const long long pre = (long long)l * nsm < total ? (long long)l * nsm : total;
+            const long long rest = total - pre;
+            auto round_of = [&](long long i) {
+                return i < pre ? (double)(i / nsm) : (double)l + (double)((i - pre) / nf);
+            };
+            const double factor_end =
+                ((double)((pre + nsm - 1) / nsm) + (double)((rest + nf - 1) / nf)) * ti;
+            double end = (double)l * ti;
+            for (int g = 0; (long long)g * s < BH; ++g) {
+                const long long sg = BH - (long long)g * s < s ? BH - (long long)g * s : s;
+                const long long first = (long long)g * s * NT;
+                const double t_first = (round_of(first) + lag) * ti;
+                const double t_last = (round_of(first + (long long)(NT - 1) * sg) + lag) * ti;
+                double e = end + NT * tc;
+                if (t_first + NT * tc > e) e = t_first + NT * tc;
+                if (t_last + tc > e) e = t_last + tc;
+                end = e;
+            }
+            const double t = end > factor_end ? end : factor_end;
+            if (t < best_t - 1.0 || (t <= best_t + 1.0 && s > best_s)) {
+                best_t = t;
+                best_s = s;
+                best_l = l;
+            }
         }
     }
-    return best;
+    *n_state = best_s;
+    *lead = best_l;
+    std::lock_guard<std::mutex> g(m);
+    if (n_cached < 16) cache[n_cached++] = Entry{BH, NT, nsm, best_s, best_l};
 }
 
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const void* alpha,
@@ -1355,8 +1430,10 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
     if (stages == 0) {
         // one cooperative launch: the runtime makes every CTA resident at once, which the chain
         // CTAs (waiting on flags the factor CTAs raise) rely on
-        const int n_state = chunk_tc_state_ctas(BH, NT, nsm);
-        const int n_intra = nsm - n_state < total ? nsm - n_state : total;
+        int n_state = 1, lead = 0;
+        chunk_tc_plan(BH, NT, nsm, &n_state, &lead);
+        // every CTA takes part in the leading rounds; afterwards only the factor CTAs take items
+        const int n_intra = nsm - n_state;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)(n_state + n_intra));
         cfg.blockDim = dim3(512);
@@ -1368,8 +1445,8 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         return cudaLaunchKernelEx(&cfg, fused, maps, alpha, beta, ws, flags, h0, outb, hT, T_len, H,
-                                 NT, BH, n_state, make_work_order(NT, BH, H, n_state), l2norm, rp,
-                                 pos_offset, scale);
+                                 NT, BH, n_state, lead, make_work_order(NT, BH, H, n_state), l2norm,
+                                 rp, pos_offset, scale);
     }
     // two kernels in sequence (profiling aid).  The factor kernel follows the flag reset in plain
     // stream order; the state kernel uses programmatic dependent launch (its set-up overlaps the

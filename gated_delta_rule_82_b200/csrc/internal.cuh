@@ -24,8 +24,9 @@ cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const
 
 // Tensor-core chunked forward (bf16, dk = dv = 128, chunk = 64).
 size_t chunk_tc_workspace_bytes(int B, int T_len, int H);
-// chain CTAs of the fused tensor-core launch for BH heads of NT chunks on nsm SMs
-int chunk_tc_state_ctas(int BH, int NT, int nsm);
+// split of the fused tensor-core launch for BH heads of NT chunks on nsm SMs: chain CTAs and
+// leading rounds of factor items taken by every CTA
+void chunk_tc_plan(int BH, int NT, int nsm, int* n_state, int* lead);
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const void* alpha,
                             const float* beta, const float* h0, void* out, float* hT, int B,
                             int T_len, int H, int l2norm, const RopeParams& rp, float scale,

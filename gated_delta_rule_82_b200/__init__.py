@@ -34,7 +34,8 @@ class CkdaError(RuntimeError):
 class _Flags(ctypes.Structure):
     _fields_ = [("l2norm", ctypes.c_int), ("rope_theta", ctypes.c_float),
                 ("rope_convention", ctypes.c_int), ("scale", ctypes.c_float),
-                ("path", ctypes.c_int), ("stages", ctypes.c_int), ("gate_logits", ctypes.c_int)]
+                ("path", ctypes.c_int), ("stages", ctypes.c_int), ("gate_logits", ctypes.c_int),
+                ("qk_heads", ctypes.c_int)]
 
 
 def library_path() -> str:
@@ -102,9 +103,10 @@ def _stream(device) -> ctypes.c_void_p:
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
-def _flags(l2norm, rope_theta, rope_convention, scale, path=0, stages=0, gate_logits=False):
+def _flags(l2norm, rope_theta, rope_convention, scale, path=0, stages=0, gate_logits=False,
+           qk_heads=0):
     return _Flags(int(bool(l2norm)), float(rope_theta), int(rope_convention), float(scale),
-                  int(path), int(stages), int(bool(gate_logits)))
+                  int(path), int(stages), int(bool(gate_logits)), int(qk_heads))
 
 
 def _raise(func, status):
@@ -142,16 +144,21 @@ def fwd_chunked(q, k, v, alpha, beta, h0=None, *, chunk=64, l2norm=True, rope_th
                 out=None, hT=None, workspace=None, stages=0, gate_logits=False):
     """Chunked CKDA forward.  Returns (out [B, T, H, dv], hT [B, H, dk, dv] or None).
 
-    q, k: [B, T, H, dk] (bf16 or fp32); v: [B, T, H, dv] same dtype; alpha: [B, T, H, dk]
+    q, k: [B, T, Hk, dk] (bf16 or fp32); v: [B, T, H, dv] same dtype, H a multiple of Hk (grouped
+    value heads when H > Hk: value head h reads q/k head h // (H // Hk)); alpha: [B, T, H, dk]
     fp32; beta: [B, T, H] fp32; h0: [B, H, dk, dv] fp32 or None.  With gate_logits, alpha holds
     logits a in q's dtype and beta fp32 logits b; the kernels use alpha = 2 sigma(a) - 1 and
     beta = 2 sigma(b).
     """
     _check(q, "q")
-    B, T, H, dk = q.shape
-    dv = v.shape[-1]
+    B, T, Hk, dk = q.shape
+    _check(v, "v", dtype=q.dtype)
+    if v.dim() != 4 or v.shape[:2] != (B, T):
+        raise ValueError(f"v: expected [B={B}, T={T}, H, dv], got {tuple(v.shape)}")
+    H, dv = v.shape[2], v.shape[3]
+    if H % Hk:
+        raise ValueError(f"v has {H} heads, not a multiple of q's {Hk}")
     _check(k, "k", dtype=q.dtype, shape=q.shape)
-    _check(v, "v", dtype=q.dtype, shape=(B, T, H, dv))
     _check(alpha, "alpha", dtype=q.dtype if gate_logits else torch.float32, shape=(B, T, H, dk))
     _check(beta, "beta", dtype=torch.float32, shape=(B, T, H))
     if h0 is not None:
@@ -171,7 +178,8 @@ def fwd_chunked(q, k, v, alpha, beta, h0=None, *, chunk=64, l2norm=True, rope_th
     st = _load().ckda_fwd_chunked(
         _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(h0), _ptr(out), _ptr(hT),
         B, T, H, dk, dv, int(chunk), _flags(l2norm, rope_theta, rope_convention, scale,
-                                           PATHS[path], stages, gate_logits),
+                                           PATHS[path], stages, gate_logits,
+                                           Hk if Hk != H else 0),
         code, int(pos_offset), _ptr(workspace), wbytes, _stream(q.device))
     _raise("ckda_fwd_chunked", st)
     return out, hT
@@ -180,12 +188,17 @@ def fwd_chunked(q, k, v, alpha, beta, h0=None, *, chunk=64, l2norm=True, rope_th
 def decode_step(q, k, v, alpha, beta, state, pos=None, *, l2norm=True, rope_theta=0.0,
                 rope_convention=0, scale=0.0, out=None, gate_logits=False):
     """One decode step, in place on state [N, H, dk, dv] fp32.  Returns out [N, H, dv].
-    With gate_logits, alpha holds logits a in q's dtype and beta fp32 logits b."""
+    q, k: [N, Hk, dk] with H a multiple of Hk (grouped value heads when H > Hk).  With
+    gate_logits, alpha holds logits a in q's dtype and beta fp32 logits b."""
     _check(q, "q")
-    N, H, dk = q.shape
-    dv = v.shape[-1]
+    N, Hk, dk = q.shape
+    _check(v, "v", dtype=q.dtype)
+    if v.dim() != 3 or v.shape[0] != N:
+        raise ValueError(f"v: expected [N={N}, H, dv], got {tuple(v.shape)}")
+    H, dv = v.shape[1], v.shape[2]
+    if H % Hk:
+        raise ValueError(f"v has {H} heads, not a multiple of q's {Hk}")
     _check(k, "k", dtype=q.dtype, shape=q.shape)
-    _check(v, "v", dtype=q.dtype, shape=(N, H, dv))
     _check(alpha, "alpha", dtype=q.dtype if gate_logits else torch.float32, shape=(N, H, dk))
     _check(beta, "beta", dtype=torch.float32, shape=(N, H))
     _check(state, "state", dtype=torch.float32, shape=(N, H, dk, dv))
@@ -196,7 +209,8 @@ def decode_step(q, k, v, alpha, beta, state, pos=None, *, l2norm=True, rope_thet
     _check(out, "out", dtype=q.dtype, shape=(N, H, dv))
     st = _load().ckda_decode_step(
         _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(state), _ptr(out), _ptr(pos),
-        N, H, dk, dv, _flags(l2norm, rope_theta, rope_convention, scale, 0, 0, gate_logits),
+        N, H, dk, dv, _flags(l2norm, rope_theta, rope_convention, scale, 0, 0, gate_logits,
+                             Hk if Hk != H else 0),
         _dtype_code(q),
         _stream(q.device))
     _raise("ckda_decode_step", st)

@@ -124,13 +124,16 @@ ckda_status ckda_fwd_chunked(const void* q, const void* k, const void* v, const 
     const void* ptrs[] = {q, k, v, alpha, beta, h0, out, hT};
     for (const void* ptr : ptrs)
         if (ptr && !aligned16(ptr)) return CKDA_ERR_ALIGN;
+    if (flags.qk_heads < 0 || (flags.qk_heads > 0 && H % flags.qk_heads != 0)) return CKDA_ERR_ARG;
+    const int G = flags.qk_heads > 0 ? H / flags.qk_heads : 1;   // value heads per q/k head
     const size_t es = elem_size(dtype);
-    const size_t nqk = (size_t)B * T * H * dk, nv = (size_t)B * T * H * dv;
+    const size_t nqk = (size_t)B * T * (H / G) * dk, nv = (size_t)B * T * H * dv;
+    const size_t nalpha = (size_t)B * T * H * dk;
     const size_t nst = (size_t)B * H * dk * dv;
     // outputs must not overlap any input (hT == h0 exactly is allowed: each (b, h) is read
     // completely before it is written)
     if (flags.gate_logits != 0 && flags.gate_logits != 1) return CKDA_ERR_ARG;
-    const size_t asz = nqk * (flags.gate_logits ? es : 4);   // gate values fp32, logits `dtype`
+    const size_t asz = nalpha * (flags.gate_logits ? es : 4);   // gate values fp32, logits `dtype`
     const void* ins[] = {q, k, v, alpha, beta};
     const size_t insz[] = {nqk * es, nqk * es, nv * es, asz, (size_t)B * T * H * 4};
     for (int i = 0; i < 5; ++i) {
@@ -155,11 +158,11 @@ ckda_status ckda_fwd_chunked(const void* q, const void* k, const void* v, const 
                                 nst * 4, nv * es, nst * 4};
         for (int i = 0; i < 8; ++i)
             if (all[i] && overlap(workspace, need, all[i], allsz[i])) return CKDA_ERR_ARG;
-        return from_cuda(launch_chunk_tc(q, k, v, alpha, beta, h0, out, hT, B, T, H, l2, rp,
+        return from_cuda(launch_chunk_tc(q, k, v, alpha, beta, h0, out, hT, B, T, H, G, l2, rp,
                                          scale, pos_offset, flags.gate_logits, workspace,
                                          flags.stages, (cudaStream_t)stream));
     }
-    return from_cuda(launch_chunk_simt(q, k, v, alpha, beta, h0, out, hT, B, T, H, dk, dv, chunk,
+    return from_cuda(launch_chunk_simt(q, k, v, alpha, beta, h0, out, hT, B, T, H, G, dk, dv, chunk,
                                        l2, rp, scale, pos_offset, flags.gate_logits, dtype,
                                        (cudaStream_t)stream));
 }
@@ -181,11 +184,13 @@ ckda_status ckda_decode_step(const void* q, const void* k, const void* v, const 
     for (const void* ptr : ptrs)
         if (!aligned16(ptr)) return CKDA_ERR_ALIGN;
     if (rp.enabled && (reinterpret_cast<uintptr_t>(pos) & 7u)) return CKDA_ERR_ALIGN;
+    if (flags.qk_heads < 0 || (flags.qk_heads > 0 && H % flags.qk_heads != 0)) return CKDA_ERR_ARG;
+    const int G = flags.qk_heads > 0 ? H / flags.qk_heads : 1;   // value heads per q/k head
     const size_t es = elem_size(dtype);
     const size_t nst = (size_t)N * H * dk * dv * 4;
     if (flags.gate_logits != 0 && flags.gate_logits != 1) return CKDA_ERR_ARG;
     const void* ins[] = {q, k, v, alpha, beta};
-    const size_t insz[] = {(size_t)N * H * dk * es, (size_t)N * H * dk * es,
+    const size_t insz[] = {(size_t)N * (H / G) * dk * es, (size_t)N * (H / G) * dk * es,
                            (size_t)N * H * dv * es, (size_t)N * H * dk * (flags.gate_logits ? es : 4),
                            (size_t)N * H * 4};
     for (int i = 0; i < 5; ++i) {
@@ -194,7 +199,7 @@ ckda_status ckda_decode_step(const void* q, const void* k, const void* v, const 
     }
     if (overlap(state, nst, out, (size_t)N * H * dv * es)) return CKDA_ERR_ARG;
     return from_cuda(launch_decode(q, k, v, alpha, beta, state, out, rp.enabled ? pos : nullptr,
-                                   N, H, dk, dv, flags.l2norm ? 1 : 0, rp,
+                                   N, H, G, dk, dv, flags.l2norm ? 1 : 0, rp,
                                    resolve_scale(flags, dk), flags.gate_logits, dtype,
                                    (cudaStream_t)stream));
 }

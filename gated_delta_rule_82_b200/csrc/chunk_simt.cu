@@ -58,8 +58,8 @@ __global__ void __launch_bounds__(kSimtThreads)
 chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                   const void* __restrict__ alpha, const float* __restrict__ beta,
                   const float* __restrict__ h0, T* __restrict__ out, float* __restrict__ hT,
-                  int T_len, int H, int l2norm, RopeParams rp, float scale, long long pos_offset,
-                  int gate_logits) {
+                  int T_len, int H, int G, int l2norm, RopeParams rp, float scale,
+                  long long pos_offset, int gate_logits) {
     using Sh = SimtShape<DK, DV, C>;
     constexpr int DVS = Sh::DVS;
     extern __shared__ float smem[];
@@ -108,7 +108,8 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
             int r = e / DK, c = e % DK;
             float qv = 0.f, kv = 0.f;
             if (r < nvalid) {
-                size_t row = ((size_t)b * T_len + t0 + r) * H + h;
+                // value head h reads q/k head h / G (grouped value heads; G = 1 without grouping)
+                size_t row = (((size_t)b * T_len + t0 + r) * H + h) / G;
                 qv = to_f32(q[row * DK + c]);
                 kv = to_f32(k[row * DK + c]);
             }
@@ -284,7 +285,7 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
 template <typename T, int DK, int DV, int C>
 cudaError_t launch_simt_t(const void* q, const void* k, const void* v, const void* alpha,
                           const float* beta, const float* h0, void* out, float* hT, int B,
-                          int T_len, int H, int l2norm, const RopeParams& rp, float scale,
+                          int T_len, int H, int G, int l2norm, const RopeParams& rp, float scale,
                           long long pos_offset, int gate_logits, cudaStream_t stream) {
     using Sh = SimtShape<DK, DV, C>;
     auto kern = chunk_simt_kernel<T, DK, DV, C>;
@@ -294,19 +295,19 @@ cudaError_t launch_simt_t(const void* q, const void* k, const void* v, const voi
     dim3 grid(B * H, DV / Sh::DVS);
     kern<<<grid, kSimtThreads, Sh::bytes, stream>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), alpha, beta,
-        h0, static_cast<T*>(out), hT, T_len, H, l2norm, rp, scale, pos_offset, gate_logits);
+        h0, static_cast<T*>(out), hT, T_len, H, G, l2norm, rp, scale, pos_offset, gate_logits);
     return cudaGetLastError();
 }
 
 template <typename T, int DK, int DV>
 cudaError_t dispatch_chunk(int chunk, const void* q, const void* k, const void* v,
                            const void* alpha, const float* beta, const float* h0, void* out,
-                           float* hT, int B, int T_len, int H, int l2norm, const RopeParams& rp,
+                           float* hT, int B, int T_len, int H, int G, int l2norm, const RopeParams& rp,
                            float scale, long long pos_offset, int gate_logits, cudaStream_t stream) {
     switch (chunk) {
-        case 16: return launch_simt_t<T, DK, DV, 16>(q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, gate_logits, stream);
-        case 32: return launch_simt_t<T, DK, DV, 32>(q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, gate_logits, stream);
-        case 64: return launch_simt_t<T, DK, DV, 64>(q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 16: return launch_simt_t<T, DK, DV, 16>(q, k, v, alpha, beta, h0, out, hT, B, T_len, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 32: return launch_simt_t<T, DK, DV, 32>(q, k, v, alpha, beta, h0, out, hT, B, T_len, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 64: return launch_simt_t<T, DK, DV, 64>(q, k, v, alpha, beta, h0, out, hT, B, T_len, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
     }
     return cudaErrorInvalidValue;
 }
@@ -314,13 +315,13 @@ cudaError_t dispatch_chunk(int chunk, const void* q, const void* k, const void* 
 template <typename T, int DK>
 cudaError_t dispatch_dv(int dv, int chunk, const void* q, const void* k, const void* v,
                         const void* alpha, const float* beta, const float* h0, void* out,
-                        float* hT, int B, int T_len, int H, int l2norm, const RopeParams& rp,
+                        float* hT, int B, int T_len, int H, int G, int l2norm, const RopeParams& rp,
                         float scale, long long pos_offset, int gate_logits, cudaStream_t stream) {
     switch (dv) {
-        case 16: return dispatch_chunk<T, DK, 16>(chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, gate_logits, stream);
-        case 32: return dispatch_chunk<T, DK, 32>(chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, gate_logits, stream);
-        case 64: return dispatch_chunk<T, DK, 64>(chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, gate_logits, stream);
-        case 128: return dispatch_chunk<T, DK, 128>(chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 16: return dispatch_chunk<T, DK, 16>(chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 32: return dispatch_chunk<T, DK, 32>(chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 64: return dispatch_chunk<T, DK, 64>(chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 128: return dispatch_chunk<T, DK, 128>(chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
     }
     return cudaErrorInvalidValue;
 }
@@ -328,13 +329,13 @@ cudaError_t dispatch_dv(int dv, int chunk, const void* q, const void* k, const v
 template <typename T>
 cudaError_t dispatch_dk(int dk, int dv, int chunk, const void* q, const void* k, const void* v,
                         const void* alpha, const float* beta, const float* h0, void* out,
-                        float* hT, int B, int T_len, int H, int l2norm, const RopeParams& rp,
+                        float* hT, int B, int T_len, int H, int G, int l2norm, const RopeParams& rp,
                         float scale, long long pos_offset, int gate_logits, cudaStream_t stream) {
     switch (dk) {
-        case 16: return dispatch_dv<T, 16>(dv, chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, gate_logits, stream);
-        case 32: return dispatch_dv<T, 32>(dv, chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, gate_logits, stream);
-        case 64: return dispatch_dv<T, 64>(dv, chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, gate_logits, stream);
-        case 128: return dispatch_dv<T, 128>(dv, chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 16: return dispatch_dv<T, 16>(dv, chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 32: return dispatch_dv<T, 32>(dv, chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 64: return dispatch_dv<T, 64>(dv, chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 128: return dispatch_dv<T, 128>(dv, chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
     }
     return cudaErrorInvalidValue;
 }
@@ -343,13 +344,13 @@ cudaError_t dispatch_dk(int dk, int dv, int chunk, const void* q, const void* k,
 
 cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const void* alpha,
                               const float* beta, const float* h0, void* out, float* hT, int B,
-                              int T_len, int H, int dk, int dv, int chunk, int l2norm,
+                              int T_len, int H, int G, int dk, int dv, int chunk, int l2norm,
                               const RopeParams& rp, float scale, long long pos_offset,
                               int gate_logits, ckda_dtype dtype, cudaStream_t stream) {
     if (dtype == CKDA_BF16)
         return dispatch_dk<__nv_bfloat16>(dk, dv, chunk, q, k, v, alpha, beta, h0, out, hT, B,
-                                          T_len, H, l2norm, rp, scale, pos_offset, gate_logits, stream);
-    return dispatch_dk<float>(dk, dv, chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H,
+                                          T_len, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
+    return dispatch_dk<float>(dk, dv, chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, G,
                               l2norm, rp, scale, pos_offset, gate_logits, stream);
 }
 

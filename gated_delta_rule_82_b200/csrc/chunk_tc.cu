@@ -172,16 +172,16 @@ struct TcMaps {
     CUtensorMap q, k, v, alpha, out;
 };
 
-// Issue the TMA loads of the chunk of batch b, head h starting at token t0: alpha -> G, q -> QR,
-// k -> KR on bar_in; V (two 64-column halves, 128-byte swizzle) on bar_v.  Rows past the sequence
-// end read as zeros.
+// Issue the TMA loads of the chunk of batch b, value head h (q/k head hk) starting at token t0:
+// alpha -> G, q -> QR, k -> KR on bar_in; V (two 64-column halves, 128-byte swizzle) on bar_v.
+// Rows past the sequence end read as zeros.
 __device__ __forceinline__ void issue_inputs(const TcMaps& m, uint8_t* sm, uint64_t* bar_in,
-                                             int b, int h, int t0, int gate_logits) {
+                                             int b, int h, int hk, int t0, int gate_logits) {
     // gate values: fp32 [64][128] into G; logits: bf16 [64][128] into the upper half of G
     tc::mbar_arrive_expect_tx(bar_in, gate_logits ? kInBytes - 16384 : kInBytes);
     tc::tma_load_4d(sm + S_G + (gate_logits ? 16384 : 0), &m.alpha, 0, h, t0, b, bar_in);
-    tc::tma_load_4d(sm + S_QR, &m.q, 0, h, t0, b, bar_in);
-    tc::tma_load_4d(sm + S_KR, &m.k, 0, h, t0, b, bar_in);
+    tc::tma_load_4d(sm + S_QR, &m.q, 0, hk, t0, b, bar_in);
+    tc::tma_load_4d(sm + S_KR, &m.k, 0, hk, t0, b, bar_in);
 }
 __device__ __forceinline__ void issue_v(const TcMaps& m, uint8_t* sm, uint64_t* bar_v, int b,
                                         int h, int t0) {
@@ -349,7 +349,7 @@ __device__ __forceinline__ void t_solve(const float* sA, float* sT, const float*
 // is chunk c of batch*head bh (workspace chunk-head bh * NT + c).  The divisions go through
 // multiply-shift forms of the launch's fixed divisors.
 struct Item {
-    int bh, c, b, h;
+    int bh, c, b, h, hk;   // hk: the q/k head of value head h
 };
 struct WorkOrder {
     int G, last_g;
@@ -357,6 +357,7 @@ struct WorkOrder {
     FastDiv gfull;   // G heads in a group
     FastDiv glast;   // heads in the last group
     FastDiv heads;   // H
+    FastDiv group;   // value heads per q/k head
     __device__ __forceinline__ Item item(int i) const {
         const uint32_t g = fastdiv(per, (uint32_t)i);
         const uint32_t r = (uint32_t)i - g * per.d;
@@ -367,6 +368,7 @@ struct WorkOrder {
         it.c = (int)c;
         it.b = (int)fastdiv(heads, (uint32_t)it.bh);
         it.h = it.bh - it.b * (int)heads.d;
+        it.hk = (int)fastdiv(group, (uint32_t)it.h);
         return it;
     }
 };
@@ -379,9 +381,10 @@ struct ItemSeq {
         return i < total ? i : -1;
     }
 };
-inline WorkOrder make_work_order(int NT, int BH, int H, int G) {
+inline WorkOrder make_work_order(int NT, int BH, int H, int G, int qk_group) {
     WorkOrder w;
     w.G = G;
+    w.group = make_fastdiv((uint32_t)qk_group);
     w.last_g = (BH - 1) / G;
     w.per = make_fastdiv((uint32_t)(G * NT));
     w.gfull = make_fastdiv((uint32_t)G);
@@ -493,7 +496,7 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
         tc::prefetch_tensormap(&maps.v);
         tc::prefetch_tensormap(&maps.alpha);
         const Item first = wo.item(i0);
-        issue_inputs(maps, sm, bar_in, first.b, first.h, first.c * kC, gate_logits);
+        issue_inputs(maps, sm, bar_in, first.b, first.h, first.hk, first.c * kC, gate_logits);
         issue_v(maps, sm, bar_v, first.b, first.h, first.c * kC);
     }
 
@@ -663,7 +666,7 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
         tc::tc_fence_after();
         // alpha, q, k of this chunk-head are consumed: bring in the next one's.  Issued by warp 15
         // (a TMA issue costs its thread several hundred cycles) while warp 0 issues the product.
-        if (tid == 480 && has_next) issue_inputs(maps, sm, bar_in, nxt.b, nxt.h, nxt.c * kC, gate_logits);
+        if (tid == 480 && has_next) issue_inputs(maps, sm, bar_in, nxt.b, nxt.h, nxt.hk, nxt.c * kC, gate_logits);
         if (!exact) {
             // ======== B: [A | M] = L R^T on the tensor cores (M = 128, N = 64, K = 128) ========
             if (warp == 0) {
@@ -1386,7 +1389,7 @@ void chunk_tc_plan(int BH, int NT, int nsm, int* n_state, int* lead) {
 
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const void* alpha,
                             const float* beta, const float* h0, void* out, float* hT, int B,
-                            int T_len, int H, int l2norm, const RopeParams& rp, float scale,
+                            int T_len, int H, int G, int l2norm, const RopeParams& rp, float scale,
                             long long pos_offset, int gate_logits, void* workspace, int stages,
                             cudaStream_t stream) {
     auto intra = gate_logits ? ckda_tc_intra<true> : ckda_tc_intra<false>;
@@ -1412,9 +1415,10 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
                     CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     if (stages != 2) {
-        if (!encode_map(&maps.q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK, kDK, H, T_len, B,
+        // q and k carry H / G heads (value head h reads q/k head h / G)
+        if (!encode_map(&maps.q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK, kDK, H / G, T_len, B,
                         CU_TENSOR_MAP_SWIZZLE_NONE) ||
-            !encode_map(&maps.k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK, kDK, H, T_len, B,
+            !encode_map(&maps.k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK, kDK, H / G, T_len, B,
                         CU_TENSOR_MAP_SWIZZLE_NONE) ||
             !encode_map(&maps.v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDV, 64, H, T_len, B,
                         CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -1445,7 +1449,7 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         return cudaLaunchKernelEx(&cfg, fused, maps, alpha, beta, ws, flags, h0, outb, hT, T_len, H,
-                                 NT, BH, n_state, lead, make_work_order(NT, BH, H, n_state), l2norm,
+                                 NT, BH, n_state, lead, make_work_order(NT, BH, H, n_state, G), l2norm,
                                  rp, pos_offset, scale);
     }
     // two kernels in sequence (profiling aid).  The factor kernel follows the flag reset in plain
@@ -1461,7 +1465,7 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
         cfg.dynamicSmemBytes = S_BYTES;
         cfg.stream = stream;
         e = cudaLaunchKernelEx(&cfg, intra, maps, alpha, beta, ws, flags, T_len, H, NT, BH,
-                               make_work_order(NT, BH, H, BH), l2norm, rp, pos_offset);
+                               make_work_order(NT, BH, H, BH, G), l2norm, rp, pos_offset);
         if (e != cudaSuccess) return e;
     }
     if (stages & 2) {

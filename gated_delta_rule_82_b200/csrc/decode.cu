@@ -46,7 +46,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
 decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
               const void* __restrict__ alpha, const float* __restrict__ beta,
               float* __restrict__ state, T* __restrict__ out, const long long* __restrict__ pos,
-              int NH, int H, int l2norm, RopeParams rp, float scale) {
+              int NH, int H, int G, int l2norm, RopeParams rp, float scale) {
     using S = DecodeShape<DK, DV>;
     constexpr int HPC = S::HPC, TPH = S::TPH, R = S::R, RG = S::RG, C4 = S::C4;
 
@@ -75,8 +75,9 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
         int g = blockIdx.x * HPC + hh;
         float qv = 0.f, kv = 0.f, av = 0.f;
         if (g < NH) {
-            qv = to_f32(q[(size_t)g * DK + c]);
-            kv = to_f32(k[(size_t)g * DK + c]);
+            // value head g reads q/k head g / G (grouped value heads; G = 1 without grouping)
+            qv = to_f32(q[(size_t)(g / G) * DK + c]);
+            kv = to_f32(k[(size_t)(g / G) * DK + c]);
             // gate values (fp32), or logits a in the activation type: alpha = 2 sigma(a) - 1
             if constexpr (kLogits)
                 av = gate_alpha(to_f32(static_cast<const T*>(alpha)[(size_t)g * DK + c]));
@@ -209,7 +210,7 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
 template <typename T, int DK, int DV>
 cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const void* alpha,
                             const float* beta, float* state, void* out, const long long* pos,
-                            int N, int H, int l2norm, const RopeParams& rp, float scale,
+                            int N, int H, int G, int l2norm, const RopeParams& rp, float scale,
                             int gate_logits, cudaStream_t stream) {
     using S = DecodeShape<DK, DV>;
     int NH = N * H;
@@ -217,20 +218,20 @@ cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const v
     auto kern = gate_logits ? decode_kernel<T, DK, DV, true> : decode_kernel<T, DK, DV, false>;
     kern<<<grid, kDecodeThreads, 0, stream>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), alpha, beta,
-        state, static_cast<T*>(out), pos, NH, H, l2norm, rp, scale);
+        state, static_cast<T*>(out), pos, NH, H, G, l2norm, rp, scale);
     return cudaGetLastError();
 }
 
 template <typename T, int DK>
 cudaError_t dispatch_dv(int dv, const void* q, const void* k, const void* v, const void* alpha,
                         const float* beta, float* state, void* out, const long long* pos, int N,
-                        int H, int l2norm, const RopeParams& rp, float scale,
+                        int H, int G, int l2norm, const RopeParams& rp, float scale,
                         int gate_logits, cudaStream_t stream) {
     switch (dv) {
-        case 16: return launch_decode_t<T, DK, 16>(q, k, v, alpha, beta, state, out, pos, N, H, l2norm, rp, scale, gate_logits, stream);
-        case 32: return launch_decode_t<T, DK, 32>(q, k, v, alpha, beta, state, out, pos, N, H, l2norm, rp, scale, gate_logits, stream);
-        case 64: return launch_decode_t<T, DK, 64>(q, k, v, alpha, beta, state, out, pos, N, H, l2norm, rp, scale, gate_logits, stream);
-        case 128: return launch_decode_t<T, DK, 128>(q, k, v, alpha, beta, state, out, pos, N, H, l2norm, rp, scale, gate_logits, stream);
+        case 16: return launch_decode_t<T, DK, 16>(q, k, v, alpha, beta, state, out, pos, N, H, G, l2norm, rp, scale, gate_logits, stream);
+        case 32: return launch_decode_t<T, DK, 32>(q, k, v, alpha, beta, state, out, pos, N, H, G, l2norm, rp, scale, gate_logits, stream);
+        case 64: return launch_decode_t<T, DK, 64>(q, k, v, alpha, beta, state, out, pos, N, H, G, l2norm, rp, scale, gate_logits, stream);
+        case 128: return launch_decode_t<T, DK, 128>(q, k, v, alpha, beta, state, out, pos, N, H, G, l2norm, rp, scale, gate_logits, stream);
     }
     return cudaErrorInvalidValue;
 }
@@ -238,13 +239,13 @@ cudaError_t dispatch_dv(int dv, const void* q, const void* k, const void* v, con
 template <typename T>
 cudaError_t dispatch_dk(int dk, int dv, const void* q, const void* k, const void* v,
                         const void* alpha, const float* beta, float* state, void* out,
-                        const long long* pos, int N, int H, int l2norm, const RopeParams& rp,
+                        const long long* pos, int N, int H, int G, int l2norm, const RopeParams& rp,
                         float scale, int gate_logits, cudaStream_t stream) {
     switch (dk) {
-        case 16: return dispatch_dv<T, 16>(dv, q, k, v, alpha, beta, state, out, pos, N, H, l2norm, rp, scale, gate_logits, stream);
-        case 32: return dispatch_dv<T, 32>(dv, q, k, v, alpha, beta, state, out, pos, N, H, l2norm, rp, scale, gate_logits, stream);
-        case 64: return dispatch_dv<T, 64>(dv, q, k, v, alpha, beta, state, out, pos, N, H, l2norm, rp, scale, gate_logits, stream);
-        case 128: return dispatch_dv<T, 128>(dv, q, k, v, alpha, beta, state, out, pos, N, H, l2norm, rp, scale, gate_logits, stream);
+        case 16: return dispatch_dv<T, 16>(dv, q, k, v, alpha, beta, state, out, pos, N, H, G, l2norm, rp, scale, gate_logits, stream);
+        case 32: return dispatch_dv<T, 32>(dv, q, k, v, alpha, beta, state, out, pos, N, H, G, l2norm, rp, scale, gate_logits, stream);
+        case 64: return dispatch_dv<T, 64>(dv, q, k, v, alpha, beta, state, out, pos, N, H, G, l2norm, rp, scale, gate_logits, stream);
+        case 128: return dispatch_dv<T, 128>(dv, q, k, v, alpha, beta, state, out, pos, N, H, G, l2norm, rp, scale, gate_logits, stream);
     }
     return cudaErrorInvalidValue;
 }
@@ -253,12 +254,12 @@ cudaError_t dispatch_dk(int dk, int dv, const void* q, const void* k, const void
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* alpha,
                           const float* beta, float* state, void* out, const long long* pos, int N,
-                          int H, int dk, int dv, int l2norm, const RopeParams& rp, float scale,
+                          int H, int G, int dk, int dv, int l2norm, const RopeParams& rp, float scale,
                           int gate_logits, ckda_dtype dtype, cudaStream_t stream) {
     if (dtype == CKDA_BF16)
-        return dispatch_dk<__nv_bfloat16>(dk, dv, q, k, v, alpha, beta, state, out, pos, N, H,
+        return dispatch_dk<__nv_bfloat16>(dk, dv, q, k, v, alpha, beta, state, out, pos, N, H, G,
                                           l2norm, rp, scale, gate_logits, stream);
-    return dispatch_dk<float>(dk, dv, q, k, v, alpha, beta, state, out, pos, N, H, l2norm, rp,
+    return dispatch_dk<float>(dk, dv, q, k, v, alpha, beta, state, out, pos, N, H, G, l2norm, rp,
                               scale, gate_logits, stream);
 }
 

@@ -11,14 +11,16 @@ cudaError_t launch_qk_prologue(const void* q, const void* k, void* qo, void* ko,
 
 // alpha: fp32 gate values, or (gate_logits != 0) logits a of the activation type; with logits
 // the kernels form alpha = 2 sigma(a) - 1 and beta = 2 sigma(b) from the fp32 logits in beta.
+// G: value heads per q/k head (grouped value heads; 1 = none): q and k have H / G heads and
+// value head h reads q/k head h / G.
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* alpha,
                           const float* beta, float* state, void* out, const long long* pos, int N,
-                          int H, int dk, int dv, int l2norm, const RopeParams& rp, float scale,
+                          int H, int G, int dk, int dv, int l2norm, const RopeParams& rp, float scale,
                           int gate_logits, ckda_dtype dtype, cudaStream_t stream);
 
 cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const void* alpha,
                               const float* beta, const float* h0, void* out, float* hT, int B,
-                              int T_len, int H, int dk, int dv, int chunk, int l2norm,
+                              int T_len, int H, int G, int dk, int dv, int chunk, int l2norm,
                               const RopeParams& rp, float scale, long long pos_offset,
                               int gate_logits, ckda_dtype dtype, cudaStream_t stream);
 
@@ -29,7 +31,7 @@ size_t chunk_tc_workspace_bytes(int B, int T_len, int H);
 void chunk_tc_plan(int BH, int NT, int nsm, int* n_state, int* lead);
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const void* alpha,
                             const float* beta, const float* h0, void* out, float* hT, int B,
-                            int T_len, int H, int l2norm, const RopeParams& rp, float scale,
+                            int T_len, int H, int G, int l2norm, const RopeParams& rp, float scale,
                             long long pos_offset, int gate_logits, void* workspace, int stages,
                             cudaStream_t stream);
 

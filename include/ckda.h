@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define CKDA_ABI_VERSION 2
+#define CKDA_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define CKDA_API __attribute__((visibility("default")))
@@ -93,6 +93,14 @@ typedef struct {
                             alpha = 2 sigma(a) - 1 and beta = 2 sigma(b), sigma the logistic
                             function (the parameterisation of the "Complex KDA" paper summary,
                             Methodology, CKDA Definition).  Any other value: CKDA_ERR_ARG. */
+    int qk_heads;        /* grouped value heads (GVA): 0 = q and k have the same H heads as v;
+                            otherwise q and k have qk_heads heads (which must divide H) and value
+                            head h reads q and k head h / (H / qk_heads), i.e. each q/k head is
+                            repeated H / qk_heads times on the head axis.  The rotation and the
+                            L2 norm act on q and k before the repeat ("RoPE review", section 7,
+                            on the GVA repeat).  alpha, beta, v, out and the states stay on the H
+                            value heads.  Negative, or not dividing H: CKDA_ERR_ARG.
+                            ckda_fwd_chunked and ckda_decode_step; ignored elsewhere. */
 } ckda_flags;
 
 /* Version of this ABI (CKDA_ABI_VERSION of the build). */
@@ -122,7 +130,8 @@ CKDA_API size_t ckda_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, in
 
 /*
  * Chunked forward over whole sequences.
- *   q, k   : [B, T, H, dk] dtype          v   : [B, T, H, dv] dtype
+ *   q, k   : [B, T, Hk, dk] dtype         v   : [B, T, H, dv] dtype
+ *            (Hk = flags.qk_heads, or H when that is 0)
  *   alpha  : [B, T, H, dk] fp32 gates (signed), or dtype logits when flags.gate_logits
  *   beta   : [B, T, H] fp32 gates, or fp32 logits when flags.gate_logits
  *   h0     : [B, H, dk, dv] fp32, or NULL for a zero initial state
@@ -146,7 +155,8 @@ CKDA_API ckda_status ckda_fwd_chunked(const void* q, const void* k, const void* 
 
 /*
  * One decode step for N independent sequences, in place on the caller's fp32 state:
- *   q, k, alpha : [N, H, dk]    v, out : [N, H, dv]    beta : [N, H]
+ *   q, k : [N, Hk, dk] (Hk = flags.qk_heads, or H)    alpha : [N, H, dk]
+ *   v, out : [N, H, dv]    beta : [N, H]
  *   (alpha fp32 gates or dtype logits, beta fp32 gates or logits, as flags.gate_logits says)
  *   state       : [N, H, dk, dv] fp32, read and overwritten with S_t
  *   pos         : [N] int64 rotary positions (required when rope_theta > 0, else ignored)

@@ -82,14 +82,27 @@ def default_scale(dk: int) -> float:
     return 1.0 / float(np.sqrt(dk))
 
 
+def repeat_qk_heads(x, H: int, axis: int):
+    """Grouped value heads (GVA): q or k with Hk heads on `axis`, each repeated H / Hk times in
+    place, so that value head h reads q/k head h // (H / Hk).  The pages place the L2 norm (and
+    with it the rotation) on the key-head axis, above this repeat ("RoPE review", section 7); both
+    act per head, so repeating before or after them gives the same values."""
+    Hk = x.shape[axis]
+    assert H % Hk == 0, "value heads must be a multiple of the q/k heads"
+    return x if Hk == H else np.repeat(x, H // Hk, axis=axis)
+
+
 def fwd(q, k, v, alpha, beta, h0=None, *, l2norm=True, rope_theta=0.0, rope_convention=0,
         scale=None, pos_offset=0, want_state=True, nthreads=None, mutant=0):
     """Sequential float64 forward.
 
-    q, k, alpha: [B, T, H, dk]; v: [B, T, H, dv]; beta: [B, T, H]; h0: [B, H, dk, dv] or None.
+    q, k: [B, T, Hk, dk]; alpha: [B, T, H, dk]; v: [B, T, H, dv]; beta: [B, T, H]; h0:
+    [B, H, dk, dv] or None; H a multiple of Hk (grouped value heads when H > Hk).
     Returns (out [B, T, H, dv], hT [B, H, dk, dv] or None), float64.
     """
     q, k, v, alpha, beta = (_f64(x) for x in (q, k, v, alpha, beta))
+    q = np.ascontiguousarray(repeat_qk_heads(q, v.shape[2], 2))
+    k = np.ascontiguousarray(repeat_qk_heads(k, v.shape[2], 2))
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     assert k.shape == q.shape and alpha.shape == q.shape
@@ -128,8 +141,11 @@ def gates(a=None, b=None, *, mutant=0):
 
 def decode(q, k, v, alpha, beta, state, pos=None, *, l2norm=True, rope_theta=0.0,
            rope_convention=0, scale=None, mutant=0):
-    """One float64 decode step.  Returns (out [N, H, dv], new state [N, H, dk, dv])."""
+    """One float64 decode step.  q, k: [N, Hk, dk] with H a multiple of Hk (grouped value heads
+    when H > Hk).  Returns (out [N, H, dv], new state [N, H, dk, dv])."""
     q, k, v, alpha, beta = (_f64(x) for x in (q, k, v, alpha, beta))
+    q = np.ascontiguousarray(repeat_qk_heads(q, v.shape[1], 1))
+    k = np.ascontiguousarray(repeat_qk_heads(k, v.shape[1], 1))
     N, H, dk = q.shape
     dv = v.shape[-1]
     st = _f64(state).copy()

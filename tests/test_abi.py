@@ -50,7 +50,7 @@ def test_only_declared_symbols_are_exported(lib):
 
 
 def test_version_and_strerror(lib):
-    assert ck.abi_version() == 2
+    assert ck.abi_version() == 3
     for s in range(8):
         assert lib.ckda_strerror(s)
     assert lib.ckda_strerror(99) == b"unknown status"
@@ -58,10 +58,10 @@ def test_version_and_strerror(lib):
 
 def flags(**kw):
     f = dict(l2norm=1, rope_theta=0.0, rope_convention=0, scale=0.0, path=0, stages=0,
-             gate_logits=0)
+             gate_logits=0, qk_heads=0)
     f.update(kw)
     return ck._Flags(f["l2norm"], f["rope_theta"], f["rope_convention"], f["scale"], f["path"],
-                     f["stages"], f["gate_logits"])
+                     f["stages"], f["gate_logits"], f["qk_heads"])
 
 
 def fwd(lib, q=P, k=2 * P, v=3 * P, a=4 * P, b=5 * P, h0=None, out=6 * P, hT=None, B=1, T=8,
@@ -84,6 +84,8 @@ def fwd(lib, q=P, k=2 * P, v=3 * P, a=4 * P, b=5 * P, h0=None, out=6 * P, hT=Non
     (dict(fl=flags(stages=4)), ARG),
     (dict(fl=flags(rope_theta=1e4, rope_convention=3)), ARG),
     (dict(fl=flags(gate_logits=2)), ARG),
+    (dict(fl=flags(qk_heads=-1)), ARG),
+    (dict(H=4, fl=flags(qk_heads=3)), ARG),   # q/k heads must divide the value heads
     (dict(dk=128, dv=128, chunk=64, T=64, q=P, k=P * 9, v=P * 17, a=P * 25, b=P * 40,
           out=P * 50, ws=None), WORKSPACE),   # tensor-core path without workspace
 ])
@@ -116,6 +118,7 @@ def dec(lib, q=P, k=2 * P, v=3 * P, a=4 * P, b=5 * P, st=6 * P, out=7 * P, pos=N
     (dict(N=0), SHAPE), (dict(dk=8), UNSUP), (dict(dtype=3), UNSUP),
     (dict(st=6 * P + 4), ALIGN), (dict(out=3 * P), ARG),
     (dict(fl=flags(gate_logits=-1)), ARG),
+    (dict(fl=flags(qk_heads=-2)), ARG), (dict(H=2, fl=flags(qk_heads=3)), ARG),
 ])
 def test_decode_validation(lib, kw, want):
     assert dec(lib, **kw) == want

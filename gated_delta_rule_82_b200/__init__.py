@@ -35,7 +35,7 @@ class _Flags(ctypes.Structure):
     _fields_ = [("l2norm", ctypes.c_int), ("rope_theta", ctypes.c_float),
                 ("rope_convention", ctypes.c_int), ("scale", ctypes.c_float),
                 ("path", ctypes.c_int), ("stages", ctypes.c_int), ("gate_logits", ctypes.c_int),
-                ("qk_heads", ctypes.c_int)]
+                ("rope_dims", ctypes.c_int), ("qk_heads", ctypes.c_int)]
 
 
 def library_path() -> str:
@@ -104,9 +104,9 @@ def _stream(device) -> ctypes.c_void_p:
 
 
 def _flags(l2norm, rope_theta, rope_convention, scale, path=0, stages=0, gate_logits=False,
-           qk_heads=0):
+           qk_heads=0, rope_dims=0):
     return _Flags(int(bool(l2norm)), float(rope_theta), int(rope_convention), float(scale),
-                  int(path), int(stages), int(bool(gate_logits)), int(qk_heads))
+                  int(path), int(stages), int(bool(gate_logits)), int(rope_dims), int(qk_heads))
 
 
 def _raise(func, status):
@@ -115,7 +115,7 @@ def _raise(func, status):
 
 
 def qk_prologue(q, k, *, l2norm=True, rope_theta=0.0, rope_convention=0, pos_offset=0,
-                q_out=None, k_out=None):
+                q_out=None, k_out=None, rope_dims=0):
     """Rotation at positions pos_offset + t, then per-head L2 norm, of q and k [B, T, H, dk]."""
     _check(q, "q")
     _check(k, "k", dtype=q.dtype, shape=q.shape)
@@ -125,7 +125,8 @@ def qk_prologue(q, k, *, l2norm=True, rope_theta=0.0, rope_convention=0, pos_off
     _check(q_out, "q_out", dtype=q.dtype, shape=q.shape)
     _check(k_out, "k_out", dtype=q.dtype, shape=q.shape)
     st = _load().ckda_qk_prologue(_ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out), B, T, H, dk,
-                                  _flags(l2norm, rope_theta, rope_convention, 0.0),
+                                  _flags(l2norm, rope_theta, rope_convention, 0.0,
+                                         rope_dims=rope_dims),
                                   _dtype_code(q), int(pos_offset), _stream(q.device))
     _raise("ckda_qk_prologue", st)
     return q_out, k_out
@@ -141,7 +142,7 @@ def workspace_bytes(B, T, H, dk, dv, chunk=64, dtype=torch.bfloat16, path="auto"
 
 def fwd_chunked(q, k, v, alpha, beta, h0=None, *, chunk=64, l2norm=True, rope_theta=0.0,
                 rope_convention=0, scale=0.0, pos_offset=0, path="auto", want_state=True,
-                out=None, hT=None, workspace=None, stages=0, gate_logits=False):
+                out=None, hT=None, workspace=None, stages=0, gate_logits=False, rope_dims=0):
     """Chunked CKDA forward.  Returns (out [B, T, H, dv], hT [B, H, dk, dv] or None).
 
     q, k: [B, T, Hk, dk] (bf16 or fp32); v: [B, T, H, dv] same dtype, H a multiple of Hk (grouped
@@ -179,14 +180,14 @@ def fwd_chunked(q, k, v, alpha, beta, h0=None, *, chunk=64, l2norm=True, rope_th
         _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(h0), _ptr(out), _ptr(hT),
         B, T, H, dk, dv, int(chunk), _flags(l2norm, rope_theta, rope_convention, scale,
                                            PATHS[path], stages, gate_logits,
-                                           Hk if Hk != H else 0),
+                                           Hk if Hk != H else 0, rope_dims),
         code, int(pos_offset), _ptr(workspace), wbytes, _stream(q.device))
     _raise("ckda_fwd_chunked", st)
     return out, hT
 
 
 def decode_step(q, k, v, alpha, beta, state, pos=None, *, l2norm=True, rope_theta=0.0,
-                rope_convention=0, scale=0.0, out=None, gate_logits=False):
+                rope_convention=0, scale=0.0, out=None, gate_logits=False, rope_dims=0):
     """One decode step, in place on state [N, H, dk, dv] fp32.  Returns out [N, H, dv].
     q, k: [N, Hk, dk] with H a multiple of Hk (grouped value heads when H > Hk).  With
     gate_logits, alpha holds logits a in q's dtype and beta fp32 logits b."""
@@ -210,7 +211,7 @@ def decode_step(q, k, v, alpha, beta, state, pos=None, *, l2norm=True, rope_thet
     st = _load().ckda_decode_step(
         _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(state), _ptr(out), _ptr(pos),
         N, H, dk, dv, _flags(l2norm, rope_theta, rope_convention, scale, 0, 0, gate_logits,
-                             Hk if Hk != H else 0),
+                             Hk if Hk != H else 0, rope_dims),
         _dtype_code(q),
         _stream(q.device))
     _raise("ckda_decode_step", st)

@@ -30,10 +30,13 @@ ckda_status make_rope(const ckda_flags& f, int dk, RopeParams* rp) {
     if (!(f.rope_theta > 0.f)) return CKDA_OK;  // also rejects NaN as "off"
     if (!isfinite(f.rope_theta)) return CKDA_ERR_ARG;
     if (f.rope_convention != 0 && f.rope_convention != 1) return CKDA_ERR_ARG;
+    const int rot = f.rope_dims == 0 ? dk : f.rope_dims;
+    if (rot != dk && !(rot * 2 == dk && dk >= 32)) return CKDA_ERR_ARG;
     rp->enabled = 1;
     rp->convention = f.rope_convention;
-    for (int i = 0; i < dk / 2; ++i)
-        rp->inv_freq[i] = pow((double)f.rope_theta, -2.0 * (double)i / (double)dk);
+    rp->rot_dims = rot;
+    for (int i = 0; i < rot / 2; ++i)
+        rp->inv_freq[i] = pow((double)f.rope_theta, -2.0 * (double)i / (double)rot);
     return CKDA_OK;
 }
 

@@ -139,11 +139,12 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
                 int c = lane + 32 * m;
                 qr[m] = c < DK ? sq[r * DK + c] : 0.f;
                 kr[m] = c < DK ? sk[r * DK + c] : 0.f;
-                if (rp.enabled && c < DK) {
+                if (rp.enabled && c < rp.rot_dims) {   // the first rot_dims channels rotate
                     int i, partner;
                     bool first;
                     if (rp.convention == 0) {
-                        i = c % (DK / 2); first = c < DK / 2; partner = first ? c + DK / 2 : c - DK / 2;
+                        const int half = rp.rot_dims / 2;
+                        i = c % half; first = c < half; partner = first ? c + half : c - half;
                     } else {
                         i = c / 2; first = (c & 1) == 0; partner = c ^ 1;
                     }

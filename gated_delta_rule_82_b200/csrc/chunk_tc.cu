@@ -586,7 +586,34 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
             }
             sq = group_sum<8>(sq);
             sk = group_sum<8>(sk);
-            if (rp.enabled) {
+            if (rp.enabled && rp.rot_dims != kDK) {
+                // partial rotation of channels 0..63 only (64..127 carried through)
+                const long long pos = pos_offset + t0 + r;
+                if (rp.convention == 0) {
+                    // pairs (c, c + 32), frequency c % 32: channels 8g + i of this thread pair with
+                    // those of the thread 4 lanes away in the same row (group g ^ 4)
+                    const bool first = g < 4;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        float sn, cs;
+                        rope_sincos(pos, sfreq[8 * (g & 3) + i], &sn, &cs);
+                        const float yq = __shfl_xor_sync(0xffffffffu, qa[i], 4);
+                        const float yk = __shfl_xor_sync(0xffffffffu, ka[i], 4);
+                        qa[i] = first ? qa[i] * cs - yq * sn : qa[i] * cs + yq * sn;
+                        ka[i] = first ? ka[i] * cs - yk * sn : ka[i] * cs + yk * sn;
+                    }
+                } else {
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {   // pairs (c, c + 1), frequency c / 2, c < 64
+                        float sn, cs;
+                        rope_sincos(pos, sfreq[4 * g + m], &sn, &cs);
+                        float x0 = qa[2 * m], x1 = qa[2 * m + 1];
+                        qa[2 * m] = x0 * cs - x1 * sn; qa[2 * m + 1] = x1 * cs + x0 * sn;
+                        x0 = ka[2 * m]; x1 = ka[2 * m + 1];
+                        ka[2 * m] = x0 * cs - x1 * sn; ka[2 * m + 1] = x1 * cs + x0 * sn;
+                    }
+                }
+            } else if (rp.enabled) {
                 const long long pos = pos_offset + t0 + r;
                 if (rp.convention == 0) {
 #pragma unroll

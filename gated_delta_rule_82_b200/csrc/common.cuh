@@ -15,9 +15,10 @@ constexpr int kMaxHalfDim = 64;  // dk <= 128
 // Inverse rotary frequencies omega_i = theta^(-2i/dk), computed in double on the host and
 // passed by value, so that concurrent calls with different bases never share state.
 struct RopeParams {
-    double inv_freq[kMaxHalfDim];
+    double inv_freq[kMaxHalfDim];   // theta^(-2i / rot_dims), i < rot_dims / 2 (0 beyond)
     int enabled;     // rope_theta > 0
-    int convention;  // 0 half-split, 1 interleaved
+    int convention;  // 0 half-split, 1 interleaved (both over the first rot_dims channels)
+    int rot_dims;    // channels rotated: dk, or dk / 2 (the rest carried through)
 };
 
 // Position angle p * omega, reduced to [-pi, pi] in double, then sin/cos in fp32.  The angle

@@ -117,11 +117,12 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
 #pragma unroll
             for (int m = 0; m < PER; ++m) {
                 int c = lane + 32 * m;
-                if (c < DK) {
+                if (c < rp.rot_dims) {   // the first rot_dims channels rotate
                     int i, partner;
                     bool first;
                     if (rp.convention == 0) {
-                        i = c % (DK / 2); first = c < DK / 2; partner = first ? c + DK / 2 : c - DK / 2;
+                        const int half = rp.rot_dims / 2;
+                        i = c % half; first = c < half; partner = first ? c + half : c - half;
                     } else {
                         i = c / 2; first = (c & 1) == 0; partner = c ^ 1;
                     }

@@ -69,20 +69,27 @@ qk_prologue_kernel(const T* __restrict__ q, const T* __restrict__ k, T* __restri
             for (int e = 0; e < EPL; ++e) x[e] = 0.f;
         }
         if (rp.enabled) {
+            // the first rot_dims channels rotate (all of them, or the first half of the head)
+            const int rot = rp.rot_dims;
             if (rp.convention == 0) {
+                // pairs (i, i + rot / 2): the partner's elements are dl lanes away
+                const int dl = rot == DK ? G / 2 : G / 4;
                 float y[EPL];
 #pragma unroll
-                for (int e = 0; e < EPL; ++e) y[e] = __shfl_xor_sync(0xffffffffu, x[e], G / 2);
-                const bool first = li < G / 2;
+                for (int e = 0; e < EPL; ++e) y[e] = __shfl_xor_sync(0xffffffffu, x[e], dl);
+                const bool first = li < dl;
+                if (li < 2 * dl) {
 #pragma unroll
-                for (int e = 0; e < EPL; ++e) {
-                    int i = (li * EPL + e) % HALF;
-                    float2 c = cs[j][i];
-                    x[e] = first ? (x[e] * c.x - y[e] * c.y) : (x[e] * c.x + y[e] * c.y);
+                    for (int e = 0; e < EPL; ++e) {
+                        int i = (li * EPL + e) % (rot / 2);
+                        float2 c = cs[j][i];
+                        x[e] = first ? (x[e] * c.x - y[e] * c.y) : (x[e] * c.x + y[e] * c.y);
+                    }
                 }
             } else {
 #pragma unroll
                 for (int e = 0; e < EPL; e += 2) {
+                    if (li * EPL + e >= rot) continue;
                     int i = (li * EPL + e) / 2;
                     float2 c = cs[j][i];
                     float a = x[e], b = x[e + 1];

@@ -93,6 +93,12 @@ typedef struct {
                             alpha = 2 sigma(a) - 1 and beta = 2 sigma(b), sigma the logistic
                             function (the parameterisation of the "Complex KDA" paper summary,
                             Methodology, CKDA Definition).  Any other value: CKDA_ERR_ARG. */
+    int rope_dims;       /* channels rotated when rope_theta > 0: 0 or dk = all; dk / 2 (dk >= 32)
+                            = the first half of each head's channels, as a rotation of that
+                            sub-vector on its own (pairs and frequencies theta^(-2i/(dk/2)) over
+                            those channels; the "RoPE review", section 3, partial rotation); the
+                            other channels are carried through, and the L2 norm, after it, covers
+                            all dk.  Other values: CKDA_ERR_ARG. */
     int qk_heads;        /* grouped value heads (GVA): 0 = q and k have the same H heads as v;
                             otherwise q and k have qk_heads heads (which must divide H) and value
                             head h reads q and k head h / (H / qk_heads), i.e. each q/k head is

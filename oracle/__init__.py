@@ -53,13 +53,14 @@ def _load(mutant: int = 0) -> ctypes.CDLL:
         D = ctypes.POINTER(ctypes.c_double)
         lib.ckda_oracle_fwd.restype = ctypes.c_int
         lib.ckda_oracle_fwd.argtypes = [D, D, D, D, D, D, D, D] + [ctypes.c_int] * 6 + [
-            ctypes.c_double, ctypes.c_int, ctypes.c_double, ctypes.c_longlong, ctypes.c_int]
+            ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_longlong,
+            ctypes.c_int]
         lib.ckda_oracle_decode.restype = ctypes.c_int
         lib.ckda_oracle_decode.argtypes = [D, D, D, D, D, D, D, ctypes.POINTER(ctypes.c_longlong)] + [
-            ctypes.c_int] * 5 + [ctypes.c_double, ctypes.c_int, ctypes.c_double]
+            ctypes.c_int] * 5 + [ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_double]
         lib.ckda_oracle_prologue.restype = ctypes.c_int
         lib.ckda_oracle_prologue.argtypes = [D, D] + [ctypes.c_int] * 5 + [
-            ctypes.c_double, ctypes.c_int, ctypes.c_longlong]
+            ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_longlong]
         lib.ckda_oracle_mutant.restype = ctypes.c_int
         lib.ckda_oracle_gates.restype = ctypes.c_int
         lib.ckda_oracle_gates.argtypes = [D, D, ctypes.c_longlong, D, D, ctypes.c_longlong]
@@ -93,7 +94,7 @@ def repeat_qk_heads(x, H: int, axis: int):
 
 
 def fwd(q, k, v, alpha, beta, h0=None, *, l2norm=True, rope_theta=0.0, rope_convention=0,
-        scale=None, pos_offset=0, want_state=True, nthreads=None, mutant=0):
+        rope_dims=0, scale=None, pos_offset=0, want_state=True, nthreads=None, mutant=0):
     """Sequential float64 forward.
 
     q, k: [B, T, Hk, dk]; alpha: [B, T, H, dk]; v: [B, T, H, dv]; beta: [B, T, H]; h0:
@@ -118,8 +119,8 @@ def fwd(q, k, v, alpha, beta, h0=None, *, l2norm=True, rope_theta=0.0, rope_conv
         nthreads = os.cpu_count() or 1
     rc = _load(mutant).ckda_oracle_fwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(h0a), _ptr(out), _ptr(hT),
-        B, T, H, dk, dv, int(bool(l2norm)), float(rope_theta), int(rope_convention), float(scale),
-        int(pos_offset), int(nthreads))
+        B, T, H, dk, dv, int(bool(l2norm)), float(rope_theta), int(rope_convention), int(rope_dims),
+        float(scale), int(pos_offset), int(nthreads))
     if rc != 0:
         raise RuntimeError(f"ckda_oracle_fwd failed with code {rc}")
     return out, hT
@@ -140,7 +141,7 @@ def gates(a=None, b=None, *, mutant=0):
 
 
 def decode(q, k, v, alpha, beta, state, pos=None, *, l2norm=True, rope_theta=0.0,
-           rope_convention=0, scale=None, mutant=0):
+           rope_convention=0, rope_dims=0, scale=None, mutant=0):
     """One float64 decode step.  q, k: [N, Hk, dk] with H a multiple of Hk (grouped value heads
     when H > Hk).  Returns (out [N, H, dv], new state [N, H, dk, dv])."""
     q, k, v, alpha, beta = (_f64(x) for x in (q, k, v, alpha, beta))
@@ -159,20 +160,21 @@ def decode(q, k, v, alpha, beta, state, pos=None, *, l2norm=True, rope_theta=0.0
         pp = posa.ctypes.data_as(ctypes.POINTER(ctypes.c_longlong))
     rc = _load(mutant).ckda_oracle_decode(
         _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(st), _ptr(out), pp, N, H, dk,
-        dv, int(bool(l2norm)), float(rope_theta), int(rope_convention), float(scale))
+        dv, int(bool(l2norm)), float(rope_theta), int(rope_convention), int(rope_dims), float(scale))
     if rc != 0:
         raise RuntimeError(f"ckda_oracle_decode failed with code {rc}")
     return out, st
 
 
-def prologue(x, *, l2norm=True, rope_theta=0.0, rope_convention=0, pos_offset=0, mutant=0):
+def prologue(x, *, l2norm=True, rope_theta=0.0, rope_convention=0, rope_dims=0, pos_offset=0,
+             mutant=0):
     """Rotation (if rope_theta > 0) then per-head L2 norm of x [B, T, H, d], float64."""
     x = _f64(x)
     B, T, H, d = x.shape
     y = np.empty_like(x)
     rc = _load(mutant).ckda_oracle_prologue(_ptr(x), _ptr(y), B, T, H, d, int(bool(l2norm)),
                                             float(rope_theta), int(rope_convention),
-                                            int(pos_offset))
+                                            int(rope_dims), int(pos_offset))
     if rc != 0:
         raise RuntimeError(f"ckda_oracle_prologue failed with code {rc}")
     return y

@@ -118,12 +118,14 @@ static void l2_normalise(double* x, int d) {
     for (int i = 0; i < d; ++i) x[i] *= r;
 }
 
-/* The q/k prologue for one token of one head: optional rotation, then optional L2 norm. */
-static void prologue_pair(double* q, double* k, int dk, long long p, int l2norm, double theta,
-                          int convention) {
+/* The q/k prologue for one token of one head: optional rotation of the first `rot` channels
+ * (a rotation of that sub-vector as a head of its own, the remaining channels carried through:
+ * the partial rotation of the "RoPE review", section 3), then optional L2 norm over all dk. */
+static void prologue_pair(double* q, double* k, int dk, int rot, long long p, int l2norm,
+                          double theta, int convention) {
     if (theta > 0.0) {
-        rope_rotate(q, dk, p, theta, convention);
-        if (g_mutant != MUT_ROPE_Q_ONLY) rope_rotate(k, dk, p, theta, convention);
+        rope_rotate(q, rot, p, theta, convention);
+        if (g_mutant != MUT_ROPE_Q_ONLY) rope_rotate(k, rot, p, theta, convention);
     }
     if (l2norm && g_mutant != MUT_NO_L2) {
         if (g_mutant == MUT_NORM_AFTER) {
@@ -197,7 +199,7 @@ static void recurrence_token(double* S, const double* q, const double* k, const 
 typedef struct {
     const double *q, *k, *v, *alpha, *beta, *h0;
     double *out, *hT;
-    int B, T, H, dk, dv, l2norm, convention;
+    int B, T, H, dk, dv, l2norm, convention, rot;
     double theta, scale;
     long long pos_offset;
     int next;                 /* next (b,h) pair to process */
@@ -236,7 +238,7 @@ static void* fwd_worker(void* arg) {
             size_t row = ((size_t)b * T + t) * H + h;
             memcpy(qb, J->q + row * dk, sizeof(double) * dk);
             memcpy(kb, J->k + row * dk, sizeof(double) * dk);
-            prologue_pair(qb, kb, dk, J->pos_offset + t, J->l2norm, J->theta, J->convention);
+            prologue_pair(qb, kb, dk, J->rot, J->pos_offset + t, J->l2norm, J->theta, J->convention);
             recurrence_token(S, qb, kb, J->v + row * dv, J->alpha + row * dk, J->beta[row], J->scale,
                              dk, dv, w, o);
             memcpy(J->out + row * dv, o, sizeof(double) * dv);
@@ -250,20 +252,22 @@ static void* fwd_worker(void* arg) {
 /*
  * Chunk-free forward over a whole sequence batch.
  *   q, k, alpha: [B, T, H, dk];  v, out: [B, T, H, dv];  beta: [B, T, H];
- *   h0, hT: [B, H, dk, dv] (h0 may be NULL for a zero state, hT may be NULL).
+ *   h0, hT: [B, H, dk, dv] (h0 may be NULL for a zero state, hT may be NULL);
+ *   rope_dims: channels rotated (0 = all dk; otherwise an even number up to dk).
  * Returns 0 on success, -1 on bad arguments, -2 on allocation failure.
  */
 int ckda_oracle_fwd(const double* q, const double* k, const double* v, const double* alpha,
                     const double* beta, const double* h0, double* out, double* hT, int B, int T,
                     int H, int dk, int dv, int l2norm, double rope_theta, int rope_convention,
-                    double scale, long long pos_offset, int nthreads) {
+                    int rope_dims, double scale, long long pos_offset, int nthreads) {
     if (!q || !k || !v || !alpha || !beta || !out) return -1;
     if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return -1;
-    if (rope_theta > 0.0 && (dk % 2) != 0) return -1;
+    if (rope_dims == 0) rope_dims = dk;
+    if (rope_theta > 0.0 && ((rope_dims % 2) != 0 || rope_dims < 0 || rope_dims > dk)) return -1;
     fwd_job J;
     J.q = q; J.k = k; J.v = v; J.alpha = alpha; J.beta = beta; J.h0 = h0; J.out = out; J.hT = hT;
     J.B = B; J.T = T; J.H = H; J.dk = dk; J.dv = dv; J.l2norm = l2norm;
-    J.convention = rope_convention; J.theta = rope_theta; J.scale = scale;
+    J.convention = rope_convention; J.theta = rope_theta; J.scale = scale; J.rot = rope_dims;
     J.pos_offset = pos_offset; J.next = 0; J.status = 0;
     pthread_mutex_init(&J.lock, NULL);
     int pairs = B * H;
@@ -290,9 +294,11 @@ int ckda_oracle_fwd(const double* q, const double* k, const double* v, const dou
 int ckda_oracle_decode(const double* q, const double* k, const double* v, const double* alpha,
                        const double* beta, double* state, double* out, const long long* pos,
                        int N, int H, int dk, int dv, int l2norm, double rope_theta,
-                       int rope_convention, double scale) {
+                       int rope_convention, int rope_dims, double scale) {
     if (!q || !k || !v || !alpha || !beta || !state || !out) return -1;
-    if (rope_theta > 0.0 && (!pos || (dk % 2) != 0)) return -1;
+    if (rope_dims == 0) rope_dims = dk;
+    if (rope_theta > 0.0 && (!pos || (rope_dims % 2) != 0 || rope_dims < 0 || rope_dims > dk))
+        return -1;
     double* qb = (double*)malloc(sizeof(double) * dk);
     double* kb = (double*)malloc(sizeof(double) * dk);
     double* w = (double*)malloc(sizeof(double) * dv);
@@ -302,7 +308,7 @@ int ckda_oracle_decode(const double* q, const double* k, const double* v, const 
             size_t row = (size_t)n * H + h;
             memcpy(qb, q + row * dk, sizeof(double) * dk);
             memcpy(kb, k + row * dk, sizeof(double) * dk);
-            prologue_pair(qb, kb, dk, rope_theta > 0.0 ? pos[n] : 0, l2norm, rope_theta,
+            prologue_pair(qb, kb, dk, rope_dims, rope_theta > 0.0 ? pos[n] : 0, l2norm, rope_theta,
                           rope_convention);
             recurrence_token(state + row * (size_t)dk * dv, qb, kb, v + row * dv, alpha + row * dk,
                              beta[row], scale, dk, dv, w, out + row * dv);
@@ -317,9 +323,11 @@ int ckda_oracle_decode(const double* q, const double* k, const double* v, const 
  * (if rope_theta > 0), then the per-head L2 norm (if l2norm).
  */
 int ckda_oracle_prologue(const double* x, double* y, int B, int T, int H, int d, int l2norm,
-                         double rope_theta, int rope_convention, long long pos_offset) {
+                         double rope_theta, int rope_convention, int rope_dims,
+                         long long pos_offset) {
     if (!x || !y || d <= 0) return -1;
-    if (rope_theta > 0.0 && (d % 2) != 0) return -1;
+    if (rope_dims == 0) rope_dims = d;
+    if (rope_theta > 0.0 && ((rope_dims % 2) != 0 || rope_dims < 0 || rope_dims > d)) return -1;
     double* buf = (double*)malloc(sizeof(double) * d);
     if (!buf) return -2;
     for (int b = 0; b < B; ++b)
@@ -327,7 +335,8 @@ int ckda_oracle_prologue(const double* x, double* y, int B, int T, int H, int d,
             for (int h = 0; h < H; ++h) {
                 size_t row = ((size_t)b * T + t) * H + h;
                 memcpy(buf, x + row * d, sizeof(double) * d);
-                if (rope_theta > 0.0) rope_rotate(buf, d, pos_offset + t, rope_theta, rope_convention);
+                if (rope_theta > 0.0)
+                    rope_rotate(buf, rope_dims, pos_offset + t, rope_theta, rope_convention);
                 if (l2norm && g_mutant != MUT_NO_L2) l2_normalise(buf, d);
                 memcpy(y + row * d, buf, sizeof(double) * d);
             }

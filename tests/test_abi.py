@@ -58,10 +58,10 @@ def test_version_and_strerror(lib):
 
 def flags(**kw):
     f = dict(l2norm=1, rope_theta=0.0, rope_convention=0, scale=0.0, path=0, stages=0,
-             gate_logits=0, qk_heads=0)
+             gate_logits=0, rope_dims=0, qk_heads=0)
     f.update(kw)
     return ck._Flags(f["l2norm"], f["rope_theta"], f["rope_convention"], f["scale"], f["path"],
-                     f["stages"], f["gate_logits"], f["qk_heads"])
+                     f["stages"], f["gate_logits"], f["rope_dims"], f["qk_heads"])
 
 
 def fwd(lib, q=P, k=2 * P, v=3 * P, a=4 * P, b=5 * P, h0=None, out=6 * P, hT=None, B=1, T=8,
@@ -85,6 +85,8 @@ def fwd(lib, q=P, k=2 * P, v=3 * P, a=4 * P, b=5 * P, h0=None, out=6 * P, hT=Non
     (dict(fl=flags(rope_theta=1e4, rope_convention=3)), ARG),
     (dict(fl=flags(gate_logits=2)), ARG),
     (dict(fl=flags(qk_heads=-1)), ARG),
+    (dict(dk=32, dv=16, fl=flags(rope_theta=1e4, rope_dims=12)), ARG),   # neither dk nor dk / 2
+    (dict(fl=flags(rope_theta=1e4, rope_dims=8)), ARG),                  # dk / 2 needs dk >= 32
     (dict(H=4, fl=flags(qk_heads=3)), ARG),   # q/k heads must divide the value heads
     (dict(dk=128, dv=128, chunk=64, T=64, q=P, k=P * 9, v=P * 17, a=P * 25, b=P * 40,
           out=P * 50, ws=None), WORKSPACE),   # tensor-core path without workspace

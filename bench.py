@@ -382,7 +382,6 @@ def main():
     if world > 1:
         dist.barrier()
     time.sleep(0.12)
-    sampler.stop()
     clocks = sampler.window(t_host0, t_host1)
     ms_per_step = max_over_ranks(ms / args.steps, dev, world)
     value = weak_scaling_mtok_s(B * T, world, ms_per_step)
@@ -477,7 +476,12 @@ def main():
                                        Din["beta"][i], state, out=outd)
         for i in range(3):
             fnD(i)
+        torch.cuda.synchronize()
+        t_dec0 = time.time()
         ms_dec = event_time_ms(fnD, steps_d, stream) / steps_d
+        t_dec1 = time.time()
+        time.sleep(0.12)
+        clocks_dec = sampler.window(t_dec0, t_dec1)
         bytes_step = N * Hd * (2 * 128 * 128 * 4 + 3 * 256 + 512 + 4 + 256)
         dec_gbs = bytes_step / (ms_dec / 1e3) / 1e9
         extras["decode"] = {
@@ -486,8 +490,10 @@ def main():
             "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": hbm_peak,
                          "unit": "GB/s", "frac": round(dec_gbs / hbm_peak, 4),
                          "traffic": ncu_traffic("decode_kernel"),
-                         "algorithmic_bytes_per_launch": bytes_step}}
+                         "algorithmic_bytes_per_launch": bytes_step},
+            "clocks": clocks_dec}
         del Din, state
+    sampler.stop()
 
     # ---- end to end through the C ABI with host buffers --------------------------------------
     e2e = None

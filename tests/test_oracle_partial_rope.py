@@ -1,18 +1,19 @@
 """Partial rotation (rope_dims = dk / 2) in the float64 oracle.
 
-The "RoPE review" (section 3) quotes FLA's rotary reference for a partial rotation: the first
-ro_dim channels are rotated as a vector of their own (cos/sin tables of ro_dim / 2 frequencies,
-rotate_half or interleaved pairs within them) and the remaining channels are carried through.
+The "RoPE review" (section 3) describes FLA's reference for a partial rotation: the leading
+ro_dim channels are rotated as a vector of their own (ro_dim / 2 frequencies, half-split or
+interleaved pairs among those channels) and the channels after them pass through unchanged; it
+names the fractions 0.5 and 1.0 as the ones accepted.
 Pins: the partial rotation equals the full rotation of the first dk / 2 channels as a head of
 dk / 2 channels (whose frequencies and pairings the full-rotation pins already fix), with the
 other half untouched; it differs from the full rotation; the inner product of a rotated q at
 position m and a rotated k at position n depends only on m - n; and the L2 norm commutes with it.
 
-On that last point the review says the opposite (a norm over all dims after a partial rotation
-"mixes rotated and unrotated coordinates").  The arithmetic decides: a partial rotation is
-linear and orthogonal (a rotation on the first channels, the identity on the rest), so it keeps
-the norm and commutes with a per-head scaling.  The oracle rotates first, then normalises; the
-test shows the order is free.
+On that last point the review claims that the two orders give different results once the norm
+runs over the whole head.  The arithmetic decides otherwise: a partial rotation is linear and
+orthogonal (a rotation on the leading channels, the identity on the rest), so it keeps the norm and
+commutes with a scaling of the whole head.  The oracle rotates first, then normalises; the test
+shows the order is free.
 """
 import numpy as np
 import pytest

@@ -55,6 +55,11 @@ def _load(mutant: int = 0) -> ctypes.CDLL:
         lib.ckda_oracle_fwd.argtypes = [D, D, D, D, D, D, D, D] + [ctypes.c_int] * 6 + [
             ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_longlong,
             ctypes.c_int]
+        lib.ckda_oracle_fwd_varlen.restype = ctypes.c_int
+        lib.ckda_oracle_fwd_varlen.argtypes = [D, D, D, D, D, D, D, D,
+                                               ctypes.POINTER(ctypes.c_longlong)] + [
+            ctypes.c_int] * 5 + [ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                 ctypes.c_longlong, ctypes.c_int]
         lib.ckda_oracle_decode.restype = ctypes.c_int
         lib.ckda_oracle_decode.argtypes = [D, D, D, D, D, D, D, ctypes.POINTER(ctypes.c_longlong)] + [
             ctypes.c_int] * 5 + [ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_double]
@@ -124,6 +129,50 @@ def fwd(q, k, v, alpha, beta, h0=None, *, l2norm=True, rope_theta=0.0, rope_conv
     if rc != 0:
         raise RuntimeError(f"ckda_oracle_fwd failed with code {rc}")
     return out, hT
+
+
+def fwd_varlen(q, k, v, alpha, beta, cu_seqlens, h0=None, *, l2norm=True, rope_theta=0.0,
+               rope_convention=0, rope_dims=0, scale=None, pos_offset=0, want_state=True,
+               nthreads=None, mutant=0):
+    """Sequential float64 forward over packed sequences of different lengths.
+
+    q, k: [T_total, Hk, dk] (or with a leading batch axis of 1); alpha: [T_total, H, dk];
+    v: [T_total, H, dv]; beta: [T_total, H]; cu_seqlens: [n + 1] token offsets (0 first,
+    non-decreasing, T_total last); h0: [n, H, dk, dv] or None.  Sequence s is tokens
+    cu_seqlens[s] .. cu_seqlens[s+1] - 1 with its own state and rotary positions from
+    pos_offset.  Returns (out shaped like v, hT [n, H, dk, dv] or None), float64.
+    """
+    q, k, v, alpha, beta = (_f64(x) for x in (q, k, v, alpha, beta))
+    lead = v.ndim == 4
+    if lead:
+        assert v.shape[0] == 1, "packed sequences take a batch axis of 1"
+        q, k, v, alpha, beta = q[0], k[0], v[0], alpha[0], beta[0]
+    q = np.ascontiguousarray(repeat_qk_heads(q, v.shape[1], 1))
+    k = np.ascontiguousarray(repeat_qk_heads(k, v.shape[1], 1))
+    Tt, H, dk = q.shape
+    dv = v.shape[-1]
+    assert k.shape == q.shape and alpha.shape == q.shape
+    assert v.shape == (Tt, H, dv) and beta.shape == (Tt, H)
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+    n = cu.shape[0] - 1
+    assert n >= 0 and cu[-1] == Tt
+    h0a = None if h0 is None else _f64(h0)
+    if h0a is not None:
+        assert h0a.shape == (n, H, dk, dv)
+    out = np.empty((Tt, H, dv), np.float64)
+    hT = np.empty((n, H, dk, dv), np.float64) if want_state else None
+    if scale is None:
+        scale = default_scale(dk)
+    if nthreads is None:
+        nthreads = os.cpu_count() or 1
+    rc = _load(mutant).ckda_oracle_fwd_varlen(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(h0a), _ptr(out), _ptr(hT),
+        cu.ctypes.data_as(ctypes.POINTER(ctypes.c_longlong)), n, H, dk, dv, int(bool(l2norm)),
+        float(rope_theta), int(rope_convention), int(rope_dims), float(scale), int(pos_offset),
+        int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"ckda_oracle_fwd_varlen failed with code {rc}")
+    return (out[None] if lead else out), hT
 
 
 def gates(a=None, b=None, *, mutant=0):

@@ -202,6 +202,7 @@ typedef struct {
     int B, T, H, dk, dv, l2norm, convention, rot;
     double theta, scale;
     long long pos_offset;
+    const long long* cu;      /* packed sequences: token offsets [B + 1], or NULL (batched) */
     int next;                 /* next (b,h) pair to process */
     pthread_mutex_t lock;
     int status;
@@ -231,11 +232,15 @@ static void* fwd_worker(void* arg) {
         int pair = take_pair(J);
         if (pair >= J->B * H) break;
         int b = pair / H, h = pair % H;
+        /* sequence b: tokens first .. first + len - 1 of the token axis (a packed sequence, or
+           row b of the batch); its positions start again at pos_offset */
+        long long first = J->cu ? J->cu[b] : (long long)b * T;
+        long long len = J->cu ? J->cu[b + 1] - J->cu[b] : T;
         size_t sofs = ((size_t)b * H + h) * (size_t)dk * dv;
         if (J->h0) memcpy(S, J->h0 + sofs, sizeof(double) * (size_t)dk * dv);
         else memset(S, 0, sizeof(double) * (size_t)dk * dv);
-        for (int t = 0; t < T; ++t) {
-            size_t row = ((size_t)b * T + t) * H + h;
+        for (long long t = 0; t < len; ++t) {
+            size_t row = ((size_t)(first + t)) * H + h;
             memcpy(qb, J->q + row * dk, sizeof(double) * dk);
             memcpy(kb, J->k + row * dk, sizeof(double) * dk);
             prologue_pair(qb, kb, dk, J->rot, J->pos_offset + t, J->l2norm, J->theta, J->convention);
@@ -247,6 +252,33 @@ static void* fwd_worker(void* arg) {
     }
     free(S); free(qb); free(kb); free(w); free(o);
     return NULL;
+}
+
+/* Runs the (sequence, head) pairs of J on nthreads threads (the caller's included). */
+static int run_fwd_job(fwd_job* J, int nthreads) {
+    J->next = 0;
+    J->status = 0;
+    pthread_mutex_init(&J->lock, NULL);
+    int pairs = J->B * J->H;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > pairs) nthreads = pairs > 0 ? pairs : 1;
+    pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    if (!th) { pthread_mutex_destroy(&J->lock); return -2; }
+    int started = 0;
+    for (int i = 1; i < nthreads; ++i) {
+        if (pthread_create(&th[i], NULL, fwd_worker, J) == 0) ++started; else break;
+    }
+    fwd_worker(J);
+    for (int i = 1; i <= started; ++i) pthread_join(th[i], NULL);
+    free(th);
+    pthread_mutex_destroy(&J->lock);
+    return J->status;
+}
+
+static int check_rope(int dk, double rope_theta, int* rope_dims) {
+    if (*rope_dims == 0) *rope_dims = dk;
+    if (rope_theta > 0.0 && ((*rope_dims % 2) != 0 || *rope_dims < 0 || *rope_dims > dk)) return -1;
+    return 0;
 }
 
 /*
@@ -262,28 +294,41 @@ int ckda_oracle_fwd(const double* q, const double* k, const double* v, const dou
                     int rope_dims, double scale, long long pos_offset, int nthreads) {
     if (!q || !k || !v || !alpha || !beta || !out) return -1;
     if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return -1;
-    if (rope_dims == 0) rope_dims = dk;
-    if (rope_theta > 0.0 && ((rope_dims % 2) != 0 || rope_dims < 0 || rope_dims > dk)) return -1;
+    if (check_rope(dk, rope_theta, &rope_dims) != 0) return -1;
     fwd_job J;
     J.q = q; J.k = k; J.v = v; J.alpha = alpha; J.beta = beta; J.h0 = h0; J.out = out; J.hT = hT;
     J.B = B; J.T = T; J.H = H; J.dk = dk; J.dv = dv; J.l2norm = l2norm;
     J.convention = rope_convention; J.theta = rope_theta; J.scale = scale; J.rot = rope_dims;
-    J.pos_offset = pos_offset; J.next = 0; J.status = 0;
-    pthread_mutex_init(&J.lock, NULL);
-    int pairs = B * H;
-    if (nthreads < 1) nthreads = 1;
-    if (nthreads > pairs) nthreads = pairs > 0 ? pairs : 1;
-    pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)nthreads);
-    if (!th) { pthread_mutex_destroy(&J.lock); return -2; }
-    int started = 0;
-    for (int i = 1; i < nthreads; ++i) {
-        if (pthread_create(&th[i], NULL, fwd_worker, &J) == 0) ++started; else break;
-    }
-    fwd_worker(&J);
-    for (int i = 1; i <= started; ++i) pthread_join(th[i], NULL);
-    free(th);
-    pthread_mutex_destroy(&J.lock);
-    return J.status;
+    J.pos_offset = pos_offset; J.cu = NULL;
+    return run_fwd_job(&J, nthreads);
+}
+
+/*
+ * Forward over packed sequences of different lengths (the cu_seqlens layout of the rotary that
+ * FLA's attention layer applies: "RoPE review", section 4).  Sequence s owns tokens
+ * cu[s] .. cu[s+1] - 1 of the token axis; it starts from h0[s] (or zero), ends in hT[s], and its
+ * rotary positions start again at pos_offset.  No state crosses from one sequence to the next.
+ *   q, k, alpha: [T_total, H, dk];  v, out: [T_total, H, dv];  beta: [T_total, H];
+ *   h0, hT: [n_seqs, H, dk, dv];  cu: [n_seqs + 1], cu[0] = 0, non-decreasing, cu[n_seqs] = T_total.
+ * Returns 0 on success, -1 on bad arguments, -2 on allocation failure.
+ */
+int ckda_oracle_fwd_varlen(const double* q, const double* k, const double* v,
+                           const double* alpha, const double* beta, const double* h0,
+                           double* out, double* hT, const long long* cu, int n_seqs, int H,
+                           int dk, int dv, int l2norm, double rope_theta, int rope_convention,
+                           int rope_dims, double scale, long long pos_offset, int nthreads) {
+    if (!cu || n_seqs < 0 || H < 0 || dk <= 0 || dv <= 0) return -1;
+    if (cu[0] != 0) return -1;
+    for (int s = 0; s < n_seqs; ++s)
+        if (cu[s + 1] < cu[s]) return -1;
+    if (cu[n_seqs] > 0 && (!q || !k || !v || !alpha || !beta || !out)) return -1;
+    if (check_rope(dk, rope_theta, &rope_dims) != 0) return -1;
+    fwd_job J;
+    J.q = q; J.k = k; J.v = v; J.alpha = alpha; J.beta = beta; J.h0 = h0; J.out = out; J.hT = hT;
+    J.B = n_seqs; J.T = 0; J.H = H; J.dk = dk; J.dv = dv; J.l2norm = l2norm;
+    J.convention = rope_convention; J.theta = rope_theta; J.scale = scale; J.rot = rope_dims;
+    J.pos_offset = pos_offset; J.cu = cu;
+    return run_fwd_job(&J, nthreads);
 }
 
 /*
@@ -296,9 +341,7 @@ int ckda_oracle_decode(const double* q, const double* k, const double* v, const 
                        int N, int H, int dk, int dv, int l2norm, double rope_theta,
                        int rope_convention, int rope_dims, double scale) {
     if (!q || !k || !v || !alpha || !beta || !state || !out) return -1;
-    if (rope_dims == 0) rope_dims = dk;
-    if (rope_theta > 0.0 && (!pos || (rope_dims % 2) != 0 || rope_dims < 0 || rope_dims > dk))
-        return -1;
+    if (check_rope(dk, rope_theta, &rope_dims) != 0 || (rope_theta > 0.0 && !pos)) return -1;
     double* qb = (double*)malloc(sizeof(double) * dk);
     double* kb = (double*)malloc(sizeof(double) * dk);
     double* w = (double*)malloc(sizeof(double) * dv);

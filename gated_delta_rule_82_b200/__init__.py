@@ -14,7 +14,8 @@ import os
 import torch
 
 __all__ = ["CkdaError", "library_path", "abi_version", "qk_prologue", "workspace_bytes",
-           "fwd_chunked", "decode_step", "selftest_umma", "PATHS"]
+           "fwd_chunked", "varlen_workspace_bytes", "fwd_varlen", "decode_step", "selftest_umma",
+           "PATHS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libckda.so")
@@ -62,6 +63,11 @@ def _load():
     lib.ckda_fwd_chunked.restype = I
     lib.ckda_fwd_chunked.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, _Flags, I, LL, P,
                                      SZ, P]
+    lib.ckda_fwd_varlen_workspace_bytes.restype = SZ
+    lib.ckda_fwd_varlen_workspace_bytes.argtypes = [P, I, I, I, I, I, I, I]
+    lib.ckda_fwd_varlen.restype = I
+    lib.ckda_fwd_varlen.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, _Flags, I, LL, P,
+                                    SZ, P]
     lib.ckda_decode_step.restype = I
     lib.ckda_decode_step.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, _Flags, I, P]
     lib.ckda_selftest_umma.restype = I
@@ -183,6 +189,84 @@ def fwd_chunked(q, k, v, alpha, beta, h0=None, *, chunk=64, l2norm=True, rope_th
                                            Hk if Hk != H else 0, rope_dims),
         code, int(pos_offset), _ptr(workspace), wbytes, _stream(q.device))
     _raise("ckda_fwd_chunked", st)
+    return out, hT
+
+
+def _host_offsets(cu_seqlens, cu_seqlens_cpu):
+    """int32 offsets on the device (as given) and a host copy (given, or read back: a sync)."""
+    _check(cu_seqlens, "cu_seqlens", dtype=torch.int32)
+    if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
+        raise ValueError("cu_seqlens: expected [n + 1] token offsets, n >= 1")
+    host = cu_seqlens.cpu() if cu_seqlens_cpu is None else cu_seqlens_cpu
+    host = host.to(torch.int32).contiguous()
+    if tuple(host.shape) != tuple(cu_seqlens.shape):
+        raise ValueError("cu_seqlens_cpu must have the shape of cu_seqlens")
+    return host
+
+
+def varlen_workspace_bytes(cu_seqlens_cpu, H, dk, dv, chunk, dtype, path="auto") -> int:
+    """Device workspace bytes of fwd_varlen for these host offsets (0 when none is needed)."""
+    host = cu_seqlens_cpu.to(torch.int32).contiguous()
+    code = _BF16 if dtype == torch.bfloat16 else _F32
+    n = _load().ckda_fwd_varlen_workspace_bytes(ctypes.c_void_p(host.data_ptr()), host.numel() - 1,
+                                                H, dk, dv, chunk, code, PATHS[path])
+    if n == ctypes.c_size_t(-1).value:
+        raise ValueError("unsupported sizes or invalid offsets for the packed forward")
+    return n
+
+
+def fwd_varlen(q, k, v, alpha, beta, cu_seqlens, h0=None, *, cu_seqlens_cpu=None, chunk=64,
+               l2norm=True, rope_theta=0.0, rope_convention=0, scale=0.0, pos_offset=0,
+               path="auto", want_state=True, out=None, hT=None, workspace=None, stages=0,
+               gate_logits=False, rope_dims=0):
+    """Chunked CKDA forward over packed sequences of different lengths.  Returns (out, hT).
+
+    q, k: [1, T, Hk, dk] or [T, Hk, dk]; v: [.., T, H, dv]; alpha: [.., T, H, dk]; beta:
+    [.., T, H] (the layouts of fwd_chunked with a batch of 1, or without the batch axis);
+    cu_seqlens: int32 [n + 1] on the device, token offsets of the n sequences (0 first,
+    non-decreasing, T last); cu_seqlens_cpu: the same offsets on the host (read back from the
+    device when omitted); h0 / hT: [n, H, dk, dv] fp32.  Each sequence starts from its own h0,
+    ends in its own hT, and its rotary positions start again at pos_offset.
+    """
+    _check(q, "q")
+    lead = q.dim() == 4
+    if lead and q.shape[0] != 1:
+        raise ValueError("packed sequences take a batch axis of 1 (or none)")
+    T, Hk, dk = q.shape[-3:]
+    _check(v, "v", dtype=q.dtype)
+    if v.dim() != q.dim() or v.shape[-3] != T:
+        raise ValueError(f"v: expected [.., T={T}, H, dv], got {tuple(v.shape)}")
+    H, dv = v.shape[-2], v.shape[-1]
+    if H % Hk:
+        raise ValueError(f"v has {H} heads, not a multiple of q's {Hk}")
+    pre = (1,) if lead else ()
+    _check(k, "k", dtype=q.dtype, shape=q.shape)
+    _check(alpha, "alpha", dtype=q.dtype if gate_logits else torch.float32, shape=pre + (T, H, dk))
+    _check(beta, "beta", dtype=torch.float32, shape=pre + (T, H))
+    host = _host_offsets(cu_seqlens, cu_seqlens_cpu)
+    n = host.numel() - 1
+    if int(host[-1]) != T:
+        raise ValueError(f"cu_seqlens ends at {int(host[-1])}, but the token axis holds {T}")
+    if h0 is not None:
+        _check(h0, "h0", dtype=torch.float32, shape=(n, H, dk, dv))
+    if out is None:
+        out = torch.empty(pre + (T, H, dv), dtype=q.dtype, device=q.device)
+    _check(out, "out", dtype=q.dtype, shape=pre + (T, H, dv))
+    if want_state and hT is None:
+        hT = torch.empty((n, H, dk, dv), dtype=torch.float32, device=q.device)
+    if hT is not None:
+        _check(hT, "hT", dtype=torch.float32, shape=(n, H, dk, dv))
+    need = varlen_workspace_bytes(host, H, dk, dv, chunk, q.dtype, path)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _load().ckda_fwd_varlen(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(h0), _ptr(out), _ptr(hT),
+        _ptr(cu_seqlens), ctypes.c_void_p(host.data_ptr()), n, H, dk, dv, int(chunk),
+        _flags(l2norm, rope_theta, rope_convention, scale, PATHS[path], stages, gate_logits,
+               Hk if Hk != H else 0, rope_dims),
+        _dtype_code(q), int(pos_offset), _ptr(workspace), wbytes, _stream(q.device))
+    _raise("ckda_fwd_varlen", st)
     return out, hT
 
 

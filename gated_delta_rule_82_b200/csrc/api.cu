@@ -111,16 +111,35 @@ size_t ckda_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, 
     return 0;
 }
 
-ckda_status ckda_fwd_chunked(const void* q, const void* k, const void* v, const void* alpha,
-                             const float* beta, const float* h0, void* out, float* hT, int B,
-                             int T, int H, int dk, int dv, int chunk, ckda_flags flags,
-                             ckda_dtype dtype, long long pos_offset, void* workspace,
-                             size_t workspace_bytes, ckda_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Offsets of packed sequences, checked on the host: cu[0] = 0, non-decreasing.  Returns the
+// token count cu[n], or -1.
+long long packed_tokens(const int* cu_host, int n) {
+    if (!cu_host || n < 1 || cu_host[0] != 0) return -1;
+    for (int s = 0; s < n; ++s)
+        if (cu_host[s + 1] < cu_host[s]) return -1;
+    return cu_host[n];
+}
+
+// The forward over a batch (pk.cu == nullptr: B rows of T tokens) or over packed sequences
+// (pk.n sequences on one axis of T tokens; states per sequence).
+ckda_status fwd_impl(const void* q, const void* k, const void* v, const void* alpha,
+                     const float* beta, const float* h0, void* out, float* hT, int B, int T, int H,
+                     int dk, int dv, int chunk, ckda_flags flags, ckda_dtype dtype,
+                     long long pos_offset, void* workspace, size_t workspace_bytes,
+                     const PackedSeqs& pk, cudaStream_t stream) {
+    const bool packed = pk.cu != nullptr;
     if (!q || !k || !v || !alpha || !beta || !out) return CKDA_ERR_NULL;
     if (dtype != CKDA_F32 && dtype != CKDA_BF16) return CKDA_ERR_UNSUPPORTED;
-    if (B < 1 || T < 1 || H < 1) return CKDA_ERR_SHAPE;
-    if ((long long)B * T * H * 128 > (1ll << 40)) return CKDA_ERR_SHAPE;
-    if ((long long)B * H * ((T + 15) / 16) > 0x7fffffffll) return CKDA_ERR_SHAPE;
+    if (B < 1 || T < (packed ? 0 : 1) || H < 1) return CKDA_ERR_SHAPE;
+    const long long ntok = packed ? (long long)T : (long long)B * T;   // tokens on the token axis
+    const long long nrows = packed ? (long long)pk.n : (long long)B;    // initial / final states
+    if (ntok * H * 128 > (1ll << 40) || nrows * H * 128 * 128 > (1ll << 40)) return CKDA_ERR_SHAPE;
+    const long long chunks16 = packed ? ntok / 16 + nrows : (long long)B * ((T + 15) / 16);
+    if (chunks16 * H > 0x7fffffffll) return CKDA_ERR_SHAPE;
     if (!supported_dim(dk) || !supported_dim(dv) || !supported_chunk(chunk)) return CKDA_ERR_UNSUPPORTED;
     int p = choose_path(flags.path, dk, dv, chunk, dtype);
     if (p < 0) return flags.path == CKDA_PATH_TC ? CKDA_ERR_UNSUPPORTED : CKDA_ERR_ARG;
@@ -130,15 +149,15 @@ ckda_status ckda_fwd_chunked(const void* q, const void* k, const void* v, const 
     if (flags.qk_heads < 0 || (flags.qk_heads > 0 && H % flags.qk_heads != 0)) return CKDA_ERR_ARG;
     const int G = flags.qk_heads > 0 ? H / flags.qk_heads : 1;   // value heads per q/k head
     const size_t es = elem_size(dtype);
-    const size_t nqk = (size_t)B * T * (H / G) * dk, nv = (size_t)B * T * H * dv;
-    const size_t nalpha = (size_t)B * T * H * dk;
-    const size_t nst = (size_t)B * H * dk * dv;
-    // outputs must not overlap any input (hT == h0 exactly is allowed: each (b, h) is read
+    const size_t nqk = (size_t)ntok * (H / G) * dk, nv = (size_t)ntok * H * dv;
+    const size_t nalpha = (size_t)ntok * H * dk;
+    const size_t nst = (size_t)nrows * H * dk * dv;
+    // outputs must not overlap any input (hT == h0 exactly is allowed: each state is read
     // completely before it is written)
     if (flags.gate_logits != 0 && flags.gate_logits != 1) return CKDA_ERR_ARG;
     const size_t asz = nalpha * (flags.gate_logits ? es : 4);   // gate values fp32, logits `dtype`
     const void* ins[] = {q, k, v, alpha, beta};
-    const size_t insz[] = {nqk * es, nqk * es, nv * es, asz, (size_t)B * T * H * 4};
+    const size_t insz[] = {nqk * es, nqk * es, nv * es, asz, (size_t)ntok * H * 4};
     for (int i = 0; i < 5; ++i) {
         if (overlap(out, nv * es, ins[i], insz[i])) return CKDA_ERR_ARG;
         if (hT && overlap(hT, nst * 4, ins[i], insz[i])) return CKDA_ERR_ARG;
@@ -153,21 +172,64 @@ ckda_status ckda_fwd_chunked(const void* q, const void* k, const void* v, const 
     const float scale = resolve_scale(flags, dk);
     const int l2 = flags.l2norm ? 1 : 0;
     if (p == CKDA_PATH_TC) {
-        size_t need = chunk_tc_workspace_bytes(B, T, H);
+        size_t need = packed ? chunk_tc_workspace_bytes_packed(pk.cu_host, pk.n, H)
+                             : chunk_tc_workspace_bytes(B, T, H);
         if (need > 0 && (!workspace || workspace_bytes < need)) return CKDA_ERR_WORKSPACE;
         if (workspace && !aligned16(workspace)) return CKDA_ERR_ALIGN;
         const void* all[] = {q, k, v, alpha, beta, h0, out, hT};
-        const size_t allsz[] = {nqk * es, nqk * es, nv * es, asz, (size_t)B * T * H * 4,
+        const size_t allsz[] = {nqk * es, nqk * es, nv * es, asz, (size_t)ntok * H * 4,
                                 nst * 4, nv * es, nst * 4};
         for (int i = 0; i < 8; ++i)
             if (all[i] && overlap(workspace, need, all[i], allsz[i])) return CKDA_ERR_ARG;
         return from_cuda(launch_chunk_tc(q, k, v, alpha, beta, h0, out, hT, B, T, H, G, l2, rp,
                                          scale, pos_offset, flags.gate_logits, workspace,
-                                         flags.stages, (cudaStream_t)stream));
+                                         flags.stages, pk, stream));
     }
     return from_cuda(launch_chunk_simt(q, k, v, alpha, beta, h0, out, hT, B, T, H, G, dk, dv, chunk,
-                                       l2, rp, scale, pos_offset, flags.gate_logits, dtype,
-                                       (cudaStream_t)stream));
+                                       l2, rp, scale, pos_offset, flags.gate_logits, dtype, pk,
+                                       stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+ckda_status ckda_fwd_chunked(const void* q, const void* k, const void* v, const void* alpha,
+                             const float* beta, const float* h0, void* out, float* hT, int B,
+                             int T, int H, int dk, int dv, int chunk, ckda_flags flags,
+                             ckda_dtype dtype, long long pos_offset, void* workspace,
+                             size_t workspace_bytes, ckda_stream_t stream) {
+    const PackedSeqs none{nullptr, nullptr, 0};
+    return fwd_impl(q, k, v, alpha, beta, h0, out, hT, B, T, H, dk, dv, chunk, flags, dtype,
+                    pos_offset, workspace, workspace_bytes, none, (cudaStream_t)stream);
+}
+
+size_t ckda_fwd_varlen_workspace_bytes(const int* cu_seqlens_host, int n_seqs, int H, int dk,
+                                       int dv, int chunk, ckda_dtype dtype, int path) {
+    if (packed_tokens(cu_seqlens_host, n_seqs) < 0 || H < 1) return (size_t)-1;
+    if (!supported_dim(dk) || !supported_dim(dv) || !supported_chunk(chunk)) return (size_t)-1;
+    if (dtype != CKDA_F32 && dtype != CKDA_BF16) return (size_t)-1;
+    int p = choose_path(path, dk, dv, chunk, dtype);
+    if (p < 0) return (size_t)-1;
+    if (p == CKDA_PATH_TC) return chunk_tc_workspace_bytes_packed(cu_seqlens_host, n_seqs, H);
+    return 0;
+}
+
+ckda_status ckda_fwd_varlen(const void* q, const void* k, const void* v, const void* alpha,
+                            const float* beta, const float* h0, void* out, float* hT,
+                            const int* cu_seqlens, const int* cu_seqlens_host, int n_seqs, int H,
+                            int dk, int dv, int chunk, ckda_flags flags, ckda_dtype dtype,
+                            long long pos_offset, void* workspace, size_t workspace_bytes,
+                            ckda_stream_t stream) {
+    if (!cu_seqlens || !cu_seqlens_host) return CKDA_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) return CKDA_ERR_ALIGN;
+    if (n_seqs < 1) return CKDA_ERR_SHAPE;
+    const long long T = packed_tokens(cu_seqlens_host, n_seqs);
+    if (T < 0) return CKDA_ERR_ARG;
+    if (T > 0x7fffffffll) return CKDA_ERR_SHAPE;
+    const PackedSeqs pk{cu_seqlens, cu_seqlens_host, n_seqs};
+    return fwd_impl(q, k, v, alpha, beta, h0, out, hT, 1, (int)T, H, dk, dv, chunk, flags, dtype,
+                    pos_offset, workspace, workspace_bytes, pk, (cudaStream_t)stream);
 }
 
 ckda_status ckda_decode_step(const void* q, const void* k, const void* v, const void* alpha,

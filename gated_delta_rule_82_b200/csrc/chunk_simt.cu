@@ -58,7 +58,7 @@ __global__ void __launch_bounds__(kSimtThreads)
 chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                   const void* __restrict__ alpha, const float* __restrict__ beta,
                   const float* __restrict__ h0, T* __restrict__ out, float* __restrict__ hT,
-                  int T_len, int H, int G, int l2norm, RopeParams rp, float scale,
+                  int T_len, const int* cu, int H, int G, int l2norm, RopeParams rp, float scale,
                   long long pos_offset, int gate_logits) {
     using Sh = SimtShape<DK, DV, C>;
     constexpr int DVS = Sh::DVS;
@@ -80,6 +80,10 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
 
     const int bh = blockIdx.x;
     const int b = bh / H, h = bh % H;
+    // the sequence's tokens on the token axis: batch row b, or packed sequence b (cu != nullptr:
+    // tokens cu[b] .. cu[b + 1] - 1, rotary positions again from pos_offset)
+    const size_t first = cu ? (size_t)cu[b] : (size_t)b * T_len;
+    const int len = cu ? cu[b + 1] - cu[b] : T_len;
     const int n0 = blockIdx.y * DVS;
     const int tid = threadIdx.x;
     const int lane = tid & 31, warp = tid >> 5;
@@ -98,10 +102,10 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
         sS[e] = h0 ? h0[((size_t)bh * DK + c) * DV + n0 + n] : 0.f;
     }
 
-    const int nchunks = (T_len + C - 1) / C;
+    const int nchunks = (len + C - 1) / C;
     for (int ch = 0; ch < nchunks; ++ch) {
         const int t0 = ch * C;
-        const int nvalid = min(C, T_len - t0);
+        const int nvalid = min(C, len - t0);
         __syncthreads();
         // ---- load the chunk: q, k, v slice, beta (padding rows are identity steps) ----
         for (int e = tid; e < C * DK; e += kSimtThreads) {
@@ -109,7 +113,7 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
             float qv = 0.f, kv = 0.f;
             if (r < nvalid) {
                 // value head h reads q/k head h / G (grouped value heads; G = 1 without grouping)
-                size_t row = (((size_t)b * T_len + t0 + r) * H + h) / G;
+                size_t row = ((first + t0 + r) * H + h) / G;
                 qv = to_f32(q[row * DK + c]);
                 kv = to_f32(k[row * DK + c]);
             }
@@ -119,11 +123,11 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
         for (int e = tid; e < C * DVS; e += kSimtThreads) {
             int r = e / DVS, n = e % DVS;
             float vv = 0.f;
-            if (r < nvalid) vv = to_f32(v[(((size_t)b * T_len + t0 + r) * H + h) * DV + n0 + n]);
+            if (r < nvalid) vv = to_f32(v[((first + t0 + r) * H + h) * DV + n0 + n]);
             sv[e] = vv;
         }
         for (int r = tid; r < C; r += kSimtThreads) {
-            float bv = r < nvalid ? beta[((size_t)b * T_len + t0 + r) * H + h] : 0.f;
+            float bv = r < nvalid ? beta[(first + t0 + r) * H + h] : 0.f;
             if (r < nvalid && gate_logits) bv = gate_beta(bv);   // beta = 2 sigma(b)
             sb[r] = bv;
         }
@@ -179,7 +183,7 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
             for (int r = 0; r < C; ++r) {
                 float a = 1.f;
                 if (r < nvalid) {
-                    const size_t ia = (((size_t)b * T_len + t0 + r) * H + h) * DK + c;
+                    const size_t ia = ((first + t0 + r) * H + h) * DK + c;
                     // gate values (fp32), or logits in the activation type: alpha = 2 sigma(a) - 1
                     a = gate_logits ? gate_alpha(to_f32(static_cast<const T*>(alpha)[ia]))
                                     : static_cast<const float*>(alpha)[ia];
@@ -261,7 +265,7 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
             float acc = 0.f;
             for (int c = 0; c < DK; ++c) acc += exp2f(sL[r * DK + c]) * sq[r * DK + c] * sS[c * DVS + n];
             for (int j = 0; j <= r; ++j) acc += sM[r * C + j] * sU[j * DVS + n];
-            out[(((size_t)b * T_len + t0 + r) * H + h) * DV + n0 + n] = from_f32<T>(scale * acc);
+            out[((first + t0 + r) * H + h) * DV + n0 + n] = from_f32<T>(scale * acc);
         }
         __syncthreads();
 
@@ -286,7 +290,7 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
 template <typename T, int DK, int DV, int C>
 cudaError_t launch_simt_t(const void* q, const void* k, const void* v, const void* alpha,
                           const float* beta, const float* h0, void* out, float* hT, int B,
-                          int T_len, int H, int G, int l2norm, const RopeParams& rp, float scale,
+                          int T_len, const int* cu, int H, int G, int l2norm, const RopeParams& rp, float scale,
                           long long pos_offset, int gate_logits, cudaStream_t stream) {
     using Sh = SimtShape<DK, DV, C>;
     auto kern = chunk_simt_kernel<T, DK, DV, C>;
@@ -296,19 +300,19 @@ cudaError_t launch_simt_t(const void* q, const void* k, const void* v, const voi
     dim3 grid(B * H, DV / Sh::DVS);
     kern<<<grid, kSimtThreads, Sh::bytes, stream>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), alpha, beta,
-        h0, static_cast<T*>(out), hT, T_len, H, G, l2norm, rp, scale, pos_offset, gate_logits);
+        h0, static_cast<T*>(out), hT, T_len, cu, H, G, l2norm, rp, scale, pos_offset, gate_logits);
     return cudaGetLastError();
 }
 
 template <typename T, int DK, int DV>
 cudaError_t dispatch_chunk(int chunk, const void* q, const void* k, const void* v,
                            const void* alpha, const float* beta, const float* h0, void* out,
-                           float* hT, int B, int T_len, int H, int G, int l2norm, const RopeParams& rp,
+                           float* hT, int B, int T_len, const int* cu, int H, int G, int l2norm, const RopeParams& rp,
                            float scale, long long pos_offset, int gate_logits, cudaStream_t stream) {
     switch (chunk) {
-        case 16: return launch_simt_t<T, DK, DV, 16>(q, k, v, alpha, beta, h0, out, hT, B, T_len, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
-        case 32: return launch_simt_t<T, DK, DV, 32>(q, k, v, alpha, beta, h0, out, hT, B, T_len, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
-        case 64: return launch_simt_t<T, DK, DV, 64>(q, k, v, alpha, beta, h0, out, hT, B, T_len, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 16: return launch_simt_t<T, DK, DV, 16>(q, k, v, alpha, beta, h0, out, hT, B, T_len, cu, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 32: return launch_simt_t<T, DK, DV, 32>(q, k, v, alpha, beta, h0, out, hT, B, T_len, cu, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 64: return launch_simt_t<T, DK, DV, 64>(q, k, v, alpha, beta, h0, out, hT, B, T_len, cu, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
     }
     return cudaErrorInvalidValue;
 }
@@ -316,13 +320,13 @@ cudaError_t dispatch_chunk(int chunk, const void* q, const void* k, const void* 
 template <typename T, int DK>
 cudaError_t dispatch_dv(int dv, int chunk, const void* q, const void* k, const void* v,
                         const void* alpha, const float* beta, const float* h0, void* out,
-                        float* hT, int B, int T_len, int H, int G, int l2norm, const RopeParams& rp,
+                        float* hT, int B, int T_len, const int* cu, int H, int G, int l2norm, const RopeParams& rp,
                         float scale, long long pos_offset, int gate_logits, cudaStream_t stream) {
     switch (dv) {
-        case 16: return dispatch_chunk<T, DK, 16>(chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
-        case 32: return dispatch_chunk<T, DK, 32>(chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
-        case 64: return dispatch_chunk<T, DK, 64>(chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
-        case 128: return dispatch_chunk<T, DK, 128>(chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 16: return dispatch_chunk<T, DK, 16>(chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, cu, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 32: return dispatch_chunk<T, DK, 32>(chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, cu, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 64: return dispatch_chunk<T, DK, 64>(chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, cu, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 128: return dispatch_chunk<T, DK, 128>(chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, cu, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
     }
     return cudaErrorInvalidValue;
 }
@@ -330,13 +334,13 @@ cudaError_t dispatch_dv(int dv, int chunk, const void* q, const void* k, const v
 template <typename T>
 cudaError_t dispatch_dk(int dk, int dv, int chunk, const void* q, const void* k, const void* v,
                         const void* alpha, const float* beta, const float* h0, void* out,
-                        float* hT, int B, int T_len, int H, int G, int l2norm, const RopeParams& rp,
+                        float* hT, int B, int T_len, const int* cu, int H, int G, int l2norm, const RopeParams& rp,
                         float scale, long long pos_offset, int gate_logits, cudaStream_t stream) {
     switch (dk) {
-        case 16: return dispatch_dv<T, 16>(dv, chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
-        case 32: return dispatch_dv<T, 32>(dv, chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
-        case 64: return dispatch_dv<T, 64>(dv, chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
-        case 128: return dispatch_dv<T, 128>(dv, chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 16: return dispatch_dv<T, 16>(dv, chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, cu, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 32: return dispatch_dv<T, 32>(dv, chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, cu, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 64: return dispatch_dv<T, 64>(dv, chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, cu, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
+        case 128: return dispatch_dv<T, 128>(dv, chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, cu, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
     }
     return cudaErrorInvalidValue;
 }
@@ -347,11 +351,14 @@ cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const
                               const float* beta, const float* h0, void* out, float* hT, int B,
                               int T_len, int H, int G, int dk, int dv, int chunk, int l2norm,
                               const RopeParams& rp, float scale, long long pos_offset,
-                              int gate_logits, ckda_dtype dtype, cudaStream_t stream) {
+                              int gate_logits, ckda_dtype dtype, const PackedSeqs& pk,
+                              cudaStream_t stream) {
+    const int* cu = pk.cu;
+    if (cu) B = pk.n;   // one CTA row per packed sequence
     if (dtype == CKDA_BF16)
         return dispatch_dk<__nv_bfloat16>(dk, dv, chunk, q, k, v, alpha, beta, h0, out, hT, B,
-                                          T_len, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
-    return dispatch_dk<float>(dk, dv, chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, H, G,
+                                          T_len, cu, H, G, l2norm, rp, scale, pos_offset, gate_logits, stream);
+    return dispatch_dk<float>(dk, dv, chunk, q, k, v, alpha, beta, h0, out, hT, B, T_len, cu, H, G,
                               l2norm, rp, scale, pos_offset, gate_logits, stream);
 }
 

@@ -381,6 +381,36 @@ struct ItemSeq {
         return i < total ? i : -1;
     }
 };
+// Packed sequences of different lengths: the chunk axis runs over the chunks of every sequence in
+// turn, and entry c of the chunk table (built on the device from the token offsets) says where
+// chunk c lies: x = first token on the packed token axis, y = tokens in the chunk (1..64), z = its
+// sequence, w = its index within the sequence, with kLastChunk set on the sequence's last chunk.
+// Without a table (a batch of equal lengths) chunk c starts at token 64 c of its batch row.
+constexpr int kLastChunk = 1 << 30;
+struct ChunkAt {
+    int t0, nvalid, seq, last;
+    long long pos0;   // rotary position of the chunk's first token
+};
+__device__ __forceinline__ ChunkAt chunk_at(const int4* __restrict__ ctab, int c, int T_len, int NT,
+                                            long long pos_offset) {
+    ChunkAt a;
+    if (ctab) {
+        const int4 e = ctab[c];
+        a.t0 = e.x;
+        a.nvalid = e.y;
+        a.seq = e.z;
+        a.last = (e.w & kLastChunk) != 0;
+        a.pos0 = pos_offset + (long long)(e.w & (kLastChunk - 1)) * kC;
+    } else {
+        a.t0 = c * kC;
+        a.nvalid = min(kC, T_len - a.t0);
+        a.seq = 0;
+        a.last = c == NT - 1;
+        a.pos0 = pos_offset + a.t0;
+    }
+    return a;
+}
+
 inline WorkOrder make_work_order(int NT, int BH, int H, int G, int qk_group) {
     WorkOrder w;
     w.G = G;
@@ -444,8 +474,8 @@ __device__ __forceinline__ bool mbar_wait_long(uint64_t* bar, uint32_t parity, v
 template <bool kLogits>
 __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, const void* __restrict__ alpha,
                                            const float* __restrict__ beta, uint8_t* __restrict__ ws,
-                                           int* __restrict__ flags, int T_len, int H, int NT,
-                                           WorkOrder wo, ItemSeq seq, int l2norm,
+                                           int* __restrict__ flags, const int4* __restrict__ ctab,
+                                           int T_len, int H, int NT, WorkOrder wo, ItemSeq seq, int l2norm,
                                            const RopeParams& rp, long long pos_offset, uint32_t tmem) {
     constexpr int gate_logits = kLogits ? 1 : 0;
     float* G = reinterpret_cast<float*>(sm + S_G);
@@ -496,9 +526,12 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
         tc::prefetch_tensormap(&maps.v);
         tc::prefetch_tensormap(&maps.alpha);
         const Item first = wo.item(i0);
-        issue_inputs(maps, sm, bar_in, first.b, first.h, first.hk, first.c * kC, gate_logits);
-        issue_v(maps, sm, bar_v, first.b, first.h, first.c * kC);
+        const int ft0 = chunk_at(ctab, first.c, T_len, NT, pos_offset).t0;
+        issue_inputs(maps, sm, bar_in, first.b, first.h, first.hk, ft0, gate_logits);
+        issue_v(maps, sm, bar_v, first.b, first.h, ft0);
     }
+    // where the current item's chunk lies; the next item's entry is read one item ahead
+    ChunkAt at_next = chunk_at(ctab, i0 >= 0 ? wo.item(i0).c : 0, T_len, NT, pos_offset);
 
     // persistent loop over items; chunk-head ci = (batch*head) * NT + chunk
     uint32_t it = 0;
@@ -506,11 +539,13 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
     for (int k = 0, i = i0; i >= 0; i = seq.at(++k), ++it) {
         const Item cur = wo.item(i);
         const int ci = cur.bh * NT + cur.c;
-        const int t0 = cur.c * kC;
-        const int nvalid = min(kC, T_len - t0);
+        const ChunkAt at = at_next;
+        const int t0 = at.t0;
+        const int nvalid = at.nvalid;
         const int inext = seq.at(k + 1);
         const bool has_next = inext >= 0;
         const Item nxt = wo.item(has_next ? inext : i);
+        at_next = chunk_at(ctab, nxt.c, T_len, NT, pos_offset);
         uint8_t* wsc = ws + (size_t)ci * WS_CHUNK;
         const size_t row0 = ((size_t)cur.b * T_len + t0) * H + cur.h;
         float bval = (tid < 64 && tid < nvalid) ? beta[row0 + tid * rs] : 0.f;
@@ -588,7 +623,7 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
             sk = group_sum<8>(sk);
             if (rp.enabled && rp.rot_dims != kDK) {
                 // partial rotation of channels 0..63 only (64..127 carried through)
-                const long long pos = pos_offset + t0 + r;
+                const long long pos = at.pos0 + r;
                 if (rp.convention == 0) {
                     // pairs (c, c + 32), frequency c % 32: channels 8g + i of this thread pair with
                     // those of the thread 4 lanes away in the same row (group g ^ 4)
@@ -614,7 +649,7 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
                     }
                 }
             } else if (rp.enabled) {
-                const long long pos = pos_offset + t0 + r;
+                const long long pos = at.pos0 + r;
                 if (rp.convention == 0) {
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {   // pairs (cA + i, cB + i), frequency 8g + i
@@ -693,7 +728,7 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
         tc::tc_fence_after();
         // alpha, q, k of this chunk-head are consumed: bring in the next one's.  Issued by warp 15
         // (a TMA issue costs its thread several hundred cycles) while warp 0 issues the product.
-        if (tid == 480 && has_next) issue_inputs(maps, sm, bar_in, nxt.b, nxt.h, nxt.hk, nxt.c * kC, gate_logits);
+        if (tid == 480 && has_next) issue_inputs(maps, sm, bar_in, nxt.b, nxt.h, nxt.hk, at_next.t0, gate_logits);
         if (!exact) {
             // ======== B: [A | M] = L R^T on the tensor cores (M = 128, N = 64, K = 128) ========
             if (warp == 0) {
@@ -862,7 +897,7 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
         pending = -1;
         // V of this chunk-head was consumed by the W/U~ products: bring in the next one's, from
         // warp 14 while warp 0 issues these products
-        if (tid == 448 && has_next) issue_v(maps, sm, bar_v, nxt.b, nxt.h, nxt.c * kC);
+        if (tid == 448 && has_next) issue_v(maps, sm, bar_v, nxt.b, nxt.h, at_next.t0);
         tc::mbar_wait(bar_q, it & 1, abort_flag);
         tc::tc_fence_after();
         // ======== G: results into shared staging images, then bulk stores in two groups ========
@@ -985,7 +1020,8 @@ static_assert(SS_OSTAGE % 1024 == 0 && (WS_QP - WS_UT) % 1024 == 0 && (WS_M - WS
 constexpr uint32_t kColS = 128, kColO = 256;
 
 __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, const uint8_t* __restrict__ ws,
-                                           const int* __restrict__ flags, const float* __restrict__ h0,
+                                           const int* __restrict__ flags, const int4* __restrict__ ctab,
+                                           const float* __restrict__ h0,
                                            __nv_bfloat16* __restrict__ out, float* __restrict__ hT,
                                            int T_len, int H, int NT, int BH, float scale, int head0,
                                            int hstride, uint32_t tmem) {
@@ -1039,9 +1075,11 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
         const int q = warp & 3, hf = warp >> 2;
         const int n = 32 * q + lane, cb = 64 * hf;
         float S[64];   // S[j] = S(cb + j, n)
-        auto load_h0 = [&](int bh) {
+        // state row of head unit bh at chunk c: the batch row's (b, h), or, for packed sequences
+        // (bh = h), (sequence of chunk c, h)
+        auto load_h0 = [&](int srow) {
             if (h0) {
-                const float* src = h0 + ((size_t)bh * kDK + cb) * kDV + n;
+                const float* src = h0 + ((size_t)srow * kDK + cb) * kDV + n;
 #pragma unroll
                 for (int j = 0; j < 64; ++j) S[j] = src[(size_t)j * kDV];
             } else {
@@ -1061,10 +1099,14 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
             if (lane == 0) tc::mbar_arrive(&s_ready[u & 1]);
         };
         if (U > 0) {
-            load_h0(head0);
+            load_h0(ctab ? ctab[0].z * H + head0 : head0);
             put_s(0);
         }
         for (int u = 0, c = 0, bh = head0; u < U; ++u) {
+            // this chunk's entry and the next item's (read ahead of the wait)
+            const int c2 = c + 1 < NT ? c + 1 : 0, bh2 = c + 1 < NT ? bh : bh + hstride;
+            const int4 ecur = ctab ? ctab[c] : make_int4(0, 0, 0, c == NT - 1 ? kLastChunk : 0);
+            const int4 enext = ctab ? ctab[c2] : make_int4(0, 0, 0, c2);
             if (!wait(mma_c, u & 1)) break;
             tc::tc_fence_after();
             tc::tmem_ld64_sync(tc::tmem_addr(tmem, 32 * q, cb), S);
@@ -1072,9 +1114,10 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
             tc::tc_fence_before();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(dc_free);
-            const bool last = c == NT - 1;
+            const bool last = (ecur.w & kLastChunk) != 0;
             if (last && hT && !*abort_flag) {
-                float* dst = hT + ((size_t)bh * kDK + cb) * kDV + n;
+                const int srow = ctab ? ecur.z * H + bh : bh;
+                float* dst = hT + ((size_t)srow * kDK + cb) * kDV + n;
 #pragma unroll
                 for (int j = 0; j < 64; ++j) dst[(size_t)j * kDV] = S[j];
             }
@@ -1082,7 +1125,8 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
                 // the buffer of S_{u+1}^T held S_{u-1}^T: the output product of item u - 1 must
                 // be done with it
                 if (u >= 1 && !wait(&mma_o[(u - 1) & 3], ((u - 1) >> 2) & 1)) break;
-                if (last) load_h0(bh + hstride);
+                // the next item starts a sequence: its initial state
+                if ((enext.w & (kLastChunk - 1)) == 0) load_h0(ctab ? enext.z * H + bh2 : bh2);
                 put_s(u + 1);
             } else {
                 tc::tc_fence_before();
@@ -1188,6 +1232,8 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
         uint8_t* stg = sm + SS_STG;
         for (int u = 0, c = 0, bh = head0; u < U; ++u) {
             const int ob = u & 3;
+            // the chunk's first token and length (packed sequences: from the chunk table)
+            const int4 e = ctab ? ctab[c] : make_int4(c * kC, kC, 0, 0);
             const bool ok = mbar_wait_long(&mma_o[ob], (u >> 2) & 1, abort_flag);
             // the previous item's tensor store must be done reading the staging tile
             if (leader) tc::bulk_wait_read<0>();
@@ -1210,10 +1256,26 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
             tc::fence_proxy_async_smem();
             __syncwarp();
             tc::bar_named(1, 128);
-            if (leader) {
-                // rows past the end of the sequence are clipped by the tensor store
-                tc::tma_store_4d(&maps.out, stg, 0, bh % H, c * kC, bh / H);
-                tc::bulk_commit();
+            if (e.y == kC || !ctab) {
+                // rows past the end of a batch row are clipped by the tensor store
+                if (leader) {
+                    tc::tma_store_4d(&maps.out, stg, 0, bh % H, e.x, bh / H);
+                    tc::bulk_commit();
+                }
+            } else {
+                // a packed sequence's short last chunk: the rows after it belong to the next
+                // sequence, so only its own rows are written (16-byte plain stores)
+                const int o = tid - 384;
+                for (int x = o; x < e.y * 16; x += 128) {
+                    const int r = x >> 4, col = x & 15;
+                    if (e.x + r < T_len) {
+                        const uint4 val = *reinterpret_cast<const uint4*>(stg + r * 256 + col * 16);
+                        *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(out) +
+                                                  ((size_t)(e.x + r) * H + bh) * (kDV * 2) + col * 16) = val;
+                    }
+                }
+                // the staging tile is read before the next item rewrites it
+                tc::bar_named(1, 128);
             }
             if (++c == NT) {
                 c = 0;
@@ -1255,27 +1317,27 @@ template <bool kLogits>
 __global__ void __launch_bounds__(512, 1)
 ckda_tc_intra(const __grid_constant__ TcMaps maps, const void* __restrict__ alpha,
               const float* __restrict__ beta, uint8_t* __restrict__ ws, int* __restrict__ flags,
-              int T_len, int H, int NT, int BH, WorkOrder wo, int l2norm, RopeParams rp,
-              long long pos_offset) {
+              const int4* __restrict__ ctab, int T_len, int H, int NT, int BH, WorkOrder wo,
+              int l2norm, RopeParams rp, long long pos_offset) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint32_t tmem_slot;
     const uint32_t tmem = kernel_tmem_alloc(&tmem_slot);
     const ItemSeq seq{(int)blockIdx.x, (int)gridDim.x, 1 << 30, 0, 1, BH * NT};
-    intra_role<kLogits>(aligned_smem(smem_raw), maps, alpha, beta, ws, flags, T_len, H, NT, wo, seq,
-                        l2norm, rp, pos_offset, tmem);
+    intra_role<kLogits>(aligned_smem(smem_raw), maps, alpha, beta, ws, flags, ctab, T_len, H, NT, wo,
+                        seq, l2norm, rp, pos_offset, tmem);
     kernel_tmem_free(tmem);
 }
 
 // State pass alone, after the factor kernel: heads blockIdx.x, blockIdx.x + gridDim.x, ...
 __global__ void __launch_bounds__(512, 1)
 ckda_tc_state(const __grid_constant__ TcMaps maps, const uint8_t* __restrict__ ws,
-              const int* __restrict__ flags, const float* __restrict__ h0,
-              __nv_bfloat16* __restrict__ out, float* __restrict__ hT, int T_len, int H, int NT,
-              int BH, float scale) {
+              const int* __restrict__ flags, const int4* __restrict__ ctab,
+              const float* __restrict__ h0, __nv_bfloat16* __restrict__ out,
+              float* __restrict__ hT, int T_len, int H, int NT, int BH, float scale) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint32_t tmem_slot;
     const uint32_t tmem = kernel_tmem_alloc(&tmem_slot);
-    state_role(aligned_smem(smem_raw), maps, ws, flags, h0, out, hT, T_len, H, NT, BH, scale,
+    state_role(aligned_smem(smem_raw), maps, ws, flags, ctab, h0, out, hT, T_len, H, NT, BH, scale,
                blockIdx.x, gridDim.x, tmem);
     kernel_tmem_free(tmem);
 }
@@ -1290,9 +1352,10 @@ template <bool kLogits>
 __global__ void __launch_bounds__(512, 1)
 ckda_tc_fused(const __grid_constant__ TcMaps maps, const void* __restrict__ alpha,
               const float* __restrict__ beta, uint8_t* __restrict__ ws, int* __restrict__ flags,
-              const float* __restrict__ h0, __nv_bfloat16* __restrict__ out, float* __restrict__ hT,
-              int T_len, int H, int NT, int BH, int n_state, int lead, WorkOrder wo, int l2norm,
-              RopeParams rp, long long pos_offset, float scale) {
+              const int4* __restrict__ ctab, const float* __restrict__ h0,
+              __nv_bfloat16* __restrict__ out, float* __restrict__ hT, int T_len, int H, int NT,
+              int BH, int n_state, int lead, WorkOrder wo, int l2norm, RopeParams rp,
+              long long pos_offset, float scale) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint32_t tmem_slot;
     uint8_t* sm = aligned_smem(smem_raw);
@@ -1302,11 +1365,96 @@ ckda_tc_fused(const __grid_constant__ TcMaps maps, const void* __restrict__ alph
     // the leading rounds, then (factor CTAs) every nf-th of the remaining items
     const ItemSeq seq{b, nall, lead, chain ? total : lead * nall + (b - n_state), chain ? 1 : nf, total};
     if (seq.at(0) >= 0)
-        intra_role<kLogits>(sm, maps, alpha, beta, ws, flags, T_len, H, NT, wo, seq, l2norm, rp,
-                            pos_offset, tmem);
+        intra_role<kLogits>(sm, maps, alpha, beta, ws, flags, ctab, T_len, H, NT, wo, seq, l2norm,
+                            rp, pos_offset, tmem);
     if (chain)
-        state_role(sm, maps, ws, flags, h0, out, hT, T_len, H, NT, BH, scale, b, n_state, tmem);
+        state_role(sm, maps, ws, flags, ctab, h0, out, hT, T_len, H, NT, BH, scale, b, n_state, tmem);
     kernel_tmem_free(tmem);
+}
+
+// Packed sequences: the chunk table and the ready flags of one call (one CTA of 1024 threads).
+// Sequences are taken 1024 at a time; a block-wide scan of their chunk counts gives each one its
+// first chunk.  If the device offsets do not give the host's chunk count nc (the two copies of
+// cu_seqlens differ), every entry becomes an empty chunk of sequence 0 and the error flag is set,
+// so that no later access leaves the caller's arrays.
+constexpr int kPrepThreads = 1024;
+__global__ void __launch_bounds__(kPrepThreads)
+ckda_varlen_prep(const int* __restrict__ cu, int n_seqs, int T_total, int nc, int4* __restrict__ ctab,
+                 int* __restrict__ flags, int n_flags) {
+    __shared__ int warp_sum[32];
+    __shared__ int s_bad;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int i = tid; i < n_flags; i += kPrepThreads) flags[i] = 0;
+    if (tid == 0) s_bad = (cu[0] != 0 || cu[n_seqs] != T_total) ? 1 : 0;
+    __syncthreads();
+    int base = 0;   // chunks of the sequences before this tile
+    for (int s0 = 0; s0 < n_seqs; s0 += kPrepThreads) {
+        const int sq = s0 + tid;
+        int len = 0;
+        if (sq < n_seqs) {
+            len = cu[sq + 1] - cu[sq];
+            if (len < 0) {
+                s_bad = 1;
+                len = 0;
+            }
+        }
+        const int nch = (len + kC - 1) / kC;
+        // inclusive scan of nch over the block
+        int x = nch;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, d);
+            if (lane >= d) x += y;
+        }
+        if (lane == 31) warp_sum[warp] = x;
+        __syncthreads();
+        if (warp == 0) {
+            int w = warp_sum[lane];
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, w, d);
+                if (lane >= d) w += y;
+            }
+            warp_sum[lane] = w;   // inclusive over warps
+        }
+        __syncthreads();
+        const int first = base + (warp ? warp_sum[warp - 1] : 0) + x - nch;
+        const int tile_total = warp_sum[31];
+        for (int j = 0; j < nch; ++j) {
+            const int c = first + j;
+            if (c < nc)
+                ctab[c] = make_int4(cu[sq] + j * kC, min(kC, len - j * kC), sq,
+                                    j | (j == nch - 1 ? kLastChunk : 0));
+            else
+                s_bad = 1;
+        }
+        base += tile_total;
+        __syncthreads();   // warp_sum is rewritten by the next tile
+    }
+    __syncthreads();
+    if (base != nc) s_bad = 1;
+    __syncthreads();
+    if (s_bad) {
+        for (int c = tid; c < nc; c += kPrepThreads) ctab[c] = make_int4(0, 0, 0, 0);
+        if (tid == 0) atomicExch(&g_tc_error, 3);
+    }
+}
+
+// Empty packed sequences: hT = h0 (or zero) for the listed sequences, one CTA per sequence.
+constexpr int kMaxEmptyList = 1024;
+struct EmptyList {
+    int n;
+    int seq[kMaxEmptyList];
+};
+__global__ void __launch_bounds__(256)
+ckda_varlen_empty(const __grid_constant__ EmptyList list, const float* __restrict__ h0,
+                  float* __restrict__ hT, int H) {
+    const size_t per = (size_t)H * kDK * kDV;
+    const size_t o = (size_t)list.seq[blockIdx.x] * per;
+    for (size_t i = threadIdx.x * 4; i < per; i += 256 * 4) {
+        const float4 x = h0 ? *reinterpret_cast<const float4*>(h0 + o + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4*>(hT + o + i) = x;
+    }
 }
 
 }  // namespace
@@ -1341,10 +1489,25 @@ static bool encode_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Workspace: the images of n = heads x chunks chunk-heads, their ready flags, and (packed
+// sequences) the chunk table of `ntab` entries.
+static size_t ctab_offset(size_t n) { return flags_offset(n) + ((n * 4 + 255) & ~(size_t)255); }
+static size_t tc_workspace(size_t n, size_t ntab) { return ctab_offset(n) + ntab * sizeof(int4); }
+
 size_t chunk_tc_workspace_bytes(int B, int T_len, int H) {
     const size_t nt = (size_t)(T_len + kC - 1) / kC;
-    const size_t n = (size_t)B * H * nt;
-    return flags_offset(n) + ((n * 4 + 255) & ~(size_t)255);
+    return tc_workspace((size_t)B * H * nt, 0);
+}
+
+long long packed_chunks(const int* cu_host, int n_seqs) {
+    long long nc = 0;
+    for (int s = 0; s < n_seqs; ++s) nc += (cu_host[s + 1] - cu_host[s] + kC - 1) / kC;
+    return nc;
+}
+
+size_t chunk_tc_workspace_bytes_packed(const int* cu_host, int n_seqs, int H) {
+    const size_t nc = (size_t)packed_chunks(cu_host, n_seqs);
+    return tc_workspace(nc * H, nc);
 }
 
 // Split of the fused launch: `n_state` chain CTAs, and `lead` leading rounds of factor items that
@@ -1418,7 +1581,7 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
                             const float* beta, const float* h0, void* out, float* hT, int B,
                             int T_len, int H, int G, int l2norm, const RopeParams& rp, float scale,
                             long long pos_offset, int gate_logits, void* workspace, int stages,
-                            cudaStream_t stream) {
+                            const PackedSeqs& pk, cudaStream_t stream) {
     auto intra = gate_logits ? ckda_tc_intra<true> : ckda_tc_intra<false>;
     auto fused = gate_logits ? ckda_tc_fused<true> : ckda_tc_fused<false>;
     cudaError_t e = cudaFuncSetAttribute(intra, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S_BYTES);
@@ -1427,36 +1590,64 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)FUSED_BYTES);
     if (e != cudaSuccess) return e;
-    const int NT = (T_len + kC - 1) / kC;
-    const int BH = B * H;
+    // packed sequences: one token axis (batch 1) whose chunks run sequence after sequence; a
+    // head's chain walks through all of them, starting again from h0 at each sequence
+    const bool packed = pk.cu != nullptr;
+    const int NT = packed ? (int)packed_chunks(pk.cu_host, pk.n) : (T_len + kC - 1) / kC;
+    const int BH = packed ? H : B * H;
+    const int Bm = packed ? 1 : B;
     const int total = NT * BH;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     int* flags = reinterpret_cast<int*>(ws + flags_offset((size_t)total));
+    int4* ctab = packed ? reinterpret_cast<int4*>(ws + ctab_offset((size_t)total)) : nullptr;
+    if (packed && stages != 2) {
+        if (hT) {
+            // empty sequences keep their initial state
+            EmptyList list;
+            list.n = 0;
+            for (int s = 0; s <= pk.n; ++s) {
+                if (s < pk.n && pk.cu_host[s + 1] == pk.cu_host[s]) list.seq[list.n++] = s;
+                if (list.n == kMaxEmptyList || (s == pk.n && list.n > 0)) {
+                    ckda_varlen_empty<<<list.n, 256, 0, stream>>>(list, h0, hT, H);
+                    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+                    list.n = 0;
+                }
+            }
+        }
+        if (total == 0) return cudaSuccess;
+        // the chunk table, and every ready flag at zero
+        ckda_varlen_prep<<<1, kPrepThreads, 0, stream>>>(pk.cu, pk.n, T_len, NT, ctab, flags, total);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (total == 0) return cudaSuccess;
     __nv_bfloat16* outb = static_cast<__nv_bfloat16*>(out);
     int dev = 0, nsm = 148;
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
     if (stages == 0 && nsm < 2) stages = 3;
     TcMaps maps;
-    if (!encode_map(&maps.out, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDV, kDV, H, T_len, B,
+    if (!encode_map(&maps.out, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDV, kDV, H, T_len, Bm,
                     CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     if (stages != 2) {
         // q and k carry H / G heads (value head h reads q/k head h / G)
-        if (!encode_map(&maps.q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK, kDK, H / G, T_len, B,
+        if (!encode_map(&maps.q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK, kDK, H / G, T_len, Bm,
                         CU_TENSOR_MAP_SWIZZLE_NONE) ||
-            !encode_map(&maps.k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK, kDK, H / G, T_len, B,
+            !encode_map(&maps.k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK, kDK, H / G, T_len, Bm,
                         CU_TENSOR_MAP_SWIZZLE_NONE) ||
-            !encode_map(&maps.v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDV, 64, H, T_len, B,
+            !encode_map(&maps.v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDV, 64, H, T_len, Bm,
                         CU_TENSOR_MAP_SWIZZLE_128B) ||
             !(gate_logits ? encode_map(&maps.alpha, alpha, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK,
-                                       kDK, H, T_len, B, CU_TENSOR_MAP_SWIZZLE_NONE)
+                                       kDK, H, T_len, Bm, CU_TENSOR_MAP_SWIZZLE_NONE)
                           : encode_map(&maps.alpha, alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kDK,
-                                       kDK, H, T_len, B, CU_TENSOR_MAP_SWIZZLE_NONE)))
+                                       kDK, H, T_len, Bm, CU_TENSOR_MAP_SWIZZLE_NONE)))
             return cudaErrorInvalidValue;
-        // every ready flag starts at zero; the factor role raises them
-        e = cudaMemsetAsync(flags, 0, (size_t)total * 4, stream);
-        if (e != cudaSuccess) return e;
+        // every ready flag starts at zero; the factor role raises them (packed sequences: the
+        // table kernel above cleared them)
+        if (!packed) {
+            e = cudaMemsetAsync(flags, 0, (size_t)total * 4, stream);
+            if (e != cudaSuccess) return e;
+        }
     }
     if (stages == 0) {
         // one cooperative launch: the runtime makes every CTA resident at once, which the chain
@@ -1475,9 +1666,10 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
         attr[0].val.cooperative = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        return cudaLaunchKernelEx(&cfg, fused, maps, alpha, beta, ws, flags, h0, outb, hT, T_len, H,
-                                 NT, BH, n_state, lead, make_work_order(NT, BH, H, n_state, G), l2norm,
-                                 rp, pos_offset, scale);
+        return cudaLaunchKernelEx(&cfg, fused, maps, alpha, beta, ws, flags,
+                                  static_cast<const int4*>(ctab), h0, outb, hT, T_len, H, NT, BH,
+                                  n_state, lead, make_work_order(NT, BH, H, n_state, G), l2norm, rp,
+                                  pos_offset, scale);
     }
     // two kernels in sequence (profiling aid).  The factor kernel follows the flag reset in plain
     // stream order; the state kernel uses programmatic dependent launch (its set-up overlaps the
@@ -1491,7 +1683,8 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
         cfg.blockDim = dim3(512);
         cfg.dynamicSmemBytes = S_BYTES;
         cfg.stream = stream;
-        e = cudaLaunchKernelEx(&cfg, intra, maps, alpha, beta, ws, flags, T_len, H, NT, BH,
+        e = cudaLaunchKernelEx(&cfg, intra, maps, alpha, beta, ws, flags,
+                               static_cast<const int4*>(ctab), T_len, H, NT, BH,
                                make_work_order(NT, BH, H, BH, G), l2norm, rp, pos_offset);
         if (e != cudaSuccess) return e;
     }
@@ -1504,7 +1697,8 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         e = cudaLaunchKernelEx(&cfg, ckda_tc_state, maps, static_cast<const uint8_t*>(ws),
-                               static_cast<const int*>(flags), h0, outb, hT, T_len, H, NT, BH, scale);
+                               static_cast<const int*>(flags), static_cast<const int4*>(ctab), h0,
+                               outb, hT, T_len, H, NT, BH, scale);
     }
     return e;
 }

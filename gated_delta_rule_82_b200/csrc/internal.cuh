@@ -5,6 +5,14 @@
 
 namespace ckda {
 
+// Packed sequences of different lengths on one token axis (cu == nullptr: a batch of equal
+// lengths).  Sequence s owns tokens cu[s] .. cu[s + 1] - 1; its state rows are s * H + h.
+struct PackedSeqs {
+    const int* cu;        // device token offsets [n + 1]
+    const int* cu_host;   // the same offsets in host memory (sizes the launch)
+    int n;                // sequences
+};
+
 cudaError_t launch_qk_prologue(const void* q, const void* k, void* qo, void* ko, int B, int T_len,
                                int H, int dk, int l2norm, const RopeParams& rp,
                                long long pos_offset, ckda_dtype dtype, cudaStream_t stream);
@@ -22,10 +30,14 @@ cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const
                               const float* beta, const float* h0, void* out, float* hT, int B,
                               int T_len, int H, int G, int dk, int dv, int chunk, int l2norm,
                               const RopeParams& rp, float scale, long long pos_offset,
-                              int gate_logits, ckda_dtype dtype, cudaStream_t stream);
+                              int gate_logits, ckda_dtype dtype, const PackedSeqs& pk,
+                              cudaStream_t stream);
 
 // Tensor-core chunked forward (bf16, dk = dv = 128, chunk = 64).
 size_t chunk_tc_workspace_bytes(int B, int T_len, int H);
+// chunks of packed sequences (sum of ceil(len / 64)) and their workspace
+long long packed_chunks(const int* cu_host, int n_seqs);
+size_t chunk_tc_workspace_bytes_packed(const int* cu_host, int n_seqs, int H);
 // split of the fused tensor-core launch for BH heads of NT chunks on nsm SMs: chain CTAs and
 // leading rounds of factor items taken by every CTA
 void chunk_tc_plan(int BH, int NT, int nsm, int* n_state, int* lead);
@@ -33,7 +45,7 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
                             const float* beta, const float* h0, void* out, float* hT, int B,
                             int T_len, int H, int G, int l2norm, const RopeParams& rp, float scale,
                             long long pos_offset, int gate_logits, void* workspace, int stages,
-                            cudaStream_t stream);
+                            const PackedSeqs& pk, cudaStream_t stream);
 
 cudaError_t launch_umma_selftest(const void* A, const void* B, float* D, int M, int N, int K,
                                  int mode, cudaStream_t stream);

@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define CKDA_ABI_VERSION 3
+#define CKDA_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define CKDA_API __attribute__((visibility("default")))
@@ -106,7 +106,8 @@ typedef struct {
                             L2 norm act on q and k before the repeat ("RoPE review", section 7,
                             on the GVA repeat).  alpha, beta, v, out and the states stay on the H
                             value heads.  Negative, or not dividing H: CKDA_ERR_ARG.
-                            ckda_fwd_chunked and ckda_decode_step; ignored elsewhere. */
+                            ckda_fwd_chunked, ckda_fwd_varlen and ckda_decode_step; ignored
+                            elsewhere. */
 } ckda_flags;
 
 /* Version of this ABI (CKDA_ABI_VERSION of the build). */
@@ -158,6 +159,45 @@ CKDA_API ckda_status ckda_fwd_chunked(const void* q, const void* k, const void* 
                              int T, int H, int dk, int dv, int chunk, ckda_flags flags,
                              ckda_dtype dtype, long long pos_offset, void* workspace,
                              size_t workspace_bytes, ckda_stream_t stream);
+
+/*
+ * Bytes of device workspace ckda_fwd_varlen needs for these packed sequences (cu_seqlens_host as
+ * below) and path selection.  0 when none is needed; (size_t)-1 when the offsets or sizes are
+ * invalid or unsupported for that path.
+ */
+CKDA_API size_t ckda_fwd_varlen_workspace_bytes(const int* cu_seqlens_host, int n_seqs, int H,
+                                                int dk, int dv, int chunk, ckda_dtype dtype,
+                                                int path);
+
+/*
+ * Chunked forward over packed sequences of different lengths: n_seqs sequences laid end to end
+ * on one token axis of T_total = cu_seqlens_host[n_seqs] tokens, described by token offsets
+ * (the cu_seqlens layout with which FLA's attention layer rotates packed sequences: "RoPE into
+ * the KDA q/k path" review, section 4).  Sequence s owns tokens cu[s] .. cu[s+1] - 1; it starts
+ * from h0[s] (or zero), ends in hT[s], and the rotary position of its token t (t counted from
+ * its first token) is pos_offset + t.  No state passes from one sequence to the next: the
+ * result for each sequence is the ckda_fwd_chunked result for that sequence alone.
+ *   q, k   : [T_total, Hk, dk] dtype       v, out : [T_total, H, dv] dtype
+ *   alpha  : [T_total, H, dk], beta : [T_total, H]  (values or logits as flags.gate_logits)
+ *   h0, hT : [n_seqs, H, dk, dv] fp32 (h0 may be NULL, hT may be NULL or equal h0)
+ *   cu_seqlens      : device int32 [n_seqs + 1], 4-byte aligned, read by the kernels
+ *   cu_seqlens_host : host int32 [n_seqs + 1], the same values, read before the call returns
+ *                     (it sizes the launch): cu[0] = 0 and non-decreasing, else CKDA_ERR_ARG.
+ *                     Empty sequences are allowed (their hT is h0, or zero).  If the two copies
+ *                     differ, the results are undefined, but every access stays inside the
+ *                     arrays described by cu_seqlens_host.
+ *   n_seqs >= 1; the other arguments as ckda_fwd_chunked, with workspace of at least
+ *   ckda_fwd_varlen_workspace_bytes(...).
+ * On the tensor-core path each head's chain of chunk steps runs through the sequences in turn;
+ * a sequence's last chunk may be short (its own tokens only are written).
+ */
+CKDA_API ckda_status ckda_fwd_varlen(const void* q, const void* k, const void* v,
+                                     const void* alpha, const float* beta, const float* h0,
+                                     void* out, float* hT, const int* cu_seqlens,
+                                     const int* cu_seqlens_host, int n_seqs, int H, int dk, int dv,
+                                     int chunk, ckda_flags flags, ckda_dtype dtype,
+                                     long long pos_offset, void* workspace,
+                                     size_t workspace_bytes, ckda_stream_t stream);
 
 /*
  * One decode step for N independent sequences, in place on the caller's fp32 state:

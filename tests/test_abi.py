@@ -32,7 +32,8 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for want in ("ckda_fwd_chunked", "ckda_decode_step", "ckda_fwd_workspace_bytes",
-                 "ckda_qk_prologue", "ckda_strerror", "ckda_abi_version"):
+                 "ckda_qk_prologue", "ckda_strerror", "ckda_abi_version", "ckda_fwd_varlen",
+                 "ckda_fwd_varlen_workspace_bytes"):
         assert want in names
 
 
@@ -50,7 +51,7 @@ def test_only_declared_symbols_are_exported(lib):
 
 
 def test_version_and_strerror(lib):
-    assert ck.abi_version() == 3
+    assert ck.abi_version() == 4
     for s in range(8):
         assert lib.ckda_strerror(s)
     assert lib.ckda_strerror(99) == b"unknown status"
@@ -104,6 +105,53 @@ def test_workspace_query(lib):
     assert lib.ckda_fwd_workspace_bytes(1, 64, 2, 16, 16, 16, 0, 2) == bad
     assert lib.ckda_fwd_workspace_bytes(1, 0, 2, 16, 16, 16, 0, 0) == bad
     assert lib.ckda_fwd_workspace_bytes(1, 64, 2, 48, 16, 16, 0, 0) == bad
+
+
+def host_offsets(vals):
+    return (ctypes.c_int * len(vals))(*vals)
+
+
+def fwd_varlen(lib, q=P, k=2 * P, v=3 * P, a=4 * P, b=5 * P, h0=None, out=6 * P, hT=None,
+               cu=8 * P, cu_host=(0, 5, 8), n=None, H=1, dk=16, dv=16, chunk=16, fl=None, dtype=1,
+               ws=None, wsb=0):
+    fl = fl or flags()
+    c = lambda x: None if x is None else ctypes.c_void_p(x)
+    host = None if cu_host is None else host_offsets(cu_host)
+    n = (len(cu_host) - 1 if cu_host else 1) if n is None else n
+    return lib.ckda_fwd_varlen(c(q), c(k), c(v), c(a), c(b), c(h0), c(out), c(hT), c(cu),
+                               None if host is None else ctypes.cast(host, ctypes.c_void_p), n, H,
+                               dk, dv, chunk, fl, dtype, 0, c(ws), wsb, None)
+
+
+# each case is invalid in exactly the stated way
+@pytest.mark.parametrize("kw,want", [
+    (dict(cu=None), NULL), (dict(cu_host=None), NULL), (dict(q=None), NULL),
+    (dict(cu=8 * P + 2), ALIGN),
+    (dict(n=0), SHAPE),
+    (dict(cu_host=(1, 5, 8)), ARG),          # offsets must start at 0
+    (dict(cu_host=(0, 6, 5, 8)), ARG),       # and never decrease
+    (dict(dk=24), UNSUP),
+    (dict(out=P), ARG),                      # out aliases q
+    (dict(fl=flags(qk_heads=-1)), ARG),
+    (dict(dk=128, dv=128, chunk=64, cu_host=(0, 70, 100), q=P, k=P * 9, v=P * 17, a=P * 25,
+          b=P * 40, out=P * 50, ws=None), WORKSPACE),   # tensor-core path without workspace
+])
+def test_fwd_varlen_validation(lib, kw, want):
+    assert fwd_varlen(lib, **kw) == want
+
+
+def test_varlen_workspace_query(lib):
+    q = lambda vals, H=16, path=0, dk=128: lib.ckda_fwd_varlen_workspace_bytes(
+        ctypes.cast(host_offsets(vals), ctypes.c_void_p), len(vals) - 1, H, dk, 128, 64, 1, path)
+    bad = ctypes.c_size_t(-1).value
+    one = q((0, 64))                            # one chunk per head
+    assert 0 < one < (1 << 40)
+    # chunks are counted per sequence: 70 + 30 tokens make 2 + 1 chunks, one sequence of 100 two
+    assert q((0, 70, 100)) > q((0, 100)) > one
+    assert q((0, 64, 64, 128)) == q((0, 128))   # an empty sequence adds no chunk
+    assert q((0, 100), path=1) == 0             # SIMT: none
+    assert q((0, 100), dk=48) == bad
+    assert q((0, 50, 40)) == bad                # decreasing offsets
 
 
 def dec(lib, q=P, k=2 * P, v=3 * P, a=4 * P, b=5 * P, st=6 * P, out=7 * P, pos=None, N=2, H=2,

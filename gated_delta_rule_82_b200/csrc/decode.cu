@@ -41,7 +41,9 @@ __device__ __forceinline__ void st_stream(float* p, float4 v) {
                  :: "l"(p), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w) : "memory");
 }
 
-template <typename T, int DK, int DV, bool kLogits>
+// kRope: the rotation is compiled in only where it is asked for (the step is latency-bound per CTA
+// at two CTAs per SM, so code that a call does not need is left out of its kernel).
+template <typename T, int DK, int DV, bool kLogits, bool kRope>
 __global__ void __launch_bounds__(kDecodeThreads, 2)
 decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
               const void* __restrict__ alpha, const float* __restrict__ beta,
@@ -76,8 +78,9 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
         float qv = 0.f, kv = 0.f, av = 0.f;
         if (g < NH) {
             // value head g reads q/k head g / G (grouped value heads; G = 1 without grouping)
-            qv = to_f32(q[(size_t)(g / G) * DK + c]);
-            kv = to_f32(k[(size_t)(g / G) * DK + c]);
+            const int gq = G == 1 ? g : g / G;
+            qv = to_f32(q[(size_t)gq * DK + c]);
+            kv = to_f32(k[(size_t)gq * DK + c]);
             // gate values (fp32), or logits a in the activation type: alpha = 2 sigma(a) - 1
             if constexpr (kLogits)
                 av = gate_alpha(to_f32(static_cast<const T*>(alpha)[(size_t)g * DK + c]));
@@ -91,7 +94,7 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
         int g = blockIdx.x * HPC + hh;
         sv[hh][c] = g < NH ? to_f32(v[(size_t)g * DV + c]) : 0.f;
     }
-    if (rp.enabled)
+    if (kRope)
         for (int i = tid; i < DK / 2; i += kDecodeThreads) sfreq[i] = rp.inv_freq[i];
     if (tid < HPC) {
         int g = blockIdx.x * HPC + tid;
@@ -112,7 +115,7 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
             qr[m] = c < DK ? sq[hh][c] : 0.f;
             kr[m] = c < DK ? sk[hh][c] : 0.f;
         }
-        if (rp.enabled && g < NH) {
+        if (kRope && g < NH) {
             long long p = pos[g / H];
 #pragma unroll
             for (int m = 0; m < PER; ++m) {
@@ -216,7 +219,10 @@ cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const v
     using S = DecodeShape<DK, DV>;
     int NH = N * H;
     int grid = (NH + S::HPC - 1) / S::HPC;
-    auto kern = gate_logits ? decode_kernel<T, DK, DV, true> : decode_kernel<T, DK, DV, false>;
+    auto kern = gate_logits ? (rp.enabled ? decode_kernel<T, DK, DV, true, true>
+                                          : decode_kernel<T, DK, DV, true, false>)
+                            : (rp.enabled ? decode_kernel<T, DK, DV, false, true>
+                                          : decode_kernel<T, DK, DV, false, false>);
     kern<<<grid, kDecodeThreads, 0, stream>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), alpha, beta,
         state, static_cast<T*>(out), pos, NH, H, G, l2norm, rp, scale);

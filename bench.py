@@ -443,6 +443,33 @@ def main():
             "path_hbm_frac": round(ht * gl_bytes / (ms_gl / 1e3) / 1e9 / hbm_peak, 4)}
         del gl_sets
 
+        # ---- packed sequences of different lengths (cu_seqlens), the layer shape's tokens ----
+        wp = synth.WORKLOADS["packed_bf16"]
+        Tp, n_p = sum(wp["lens"]), len(wp["lens"])
+        p_sets = [synth.torch_fwd_inputs(1, Tp, H, dk, dv, kind="ckda", dtype="bf16",
+                                         seed=8500 + 10 * rank + i, device=dev)
+                  for i in range(N_ROTATE)]
+        cu_h = torch.tensor([sum(wp["lens"][:j]) for j in range(n_p + 1)], dtype=torch.int32)
+        cu_d = cu_h.to(dev)
+        out_p = torch.empty((1, Tp, H, dv), dtype=torch.bfloat16, device=dev)
+        hT_p = torch.empty((n_p, H, dk, dv), dtype=torch.float32, device=dev)
+        ws_p = torch.empty(ck.varlen_workspace_bytes(cu_h, H, dk, dv, C, torch.bfloat16),
+                           dtype=torch.uint8, device=dev)
+
+        def step_p(i):
+            s = p_sets[i % N_ROTATE]
+            ck.fwd_varlen(s["q"], s["k"], s["v"], s["alpha"], s["beta"], cu_d, None,
+                          cu_seqlens_cpu=cu_h, chunk=C, path="tc", out=out_p, hT=hT_p,
+                          workspace=ws_p)
+        for i in range(3):
+            step_p(i)
+        ms_p = event_time_ms(step_p, args.steps, stream) / args.steps
+        extras["varlen"] = {
+            "workload": f"packed_bf16 ({n_p} sequences of {wp['lens']} tokens, H={H}, dk=dv=128)",
+            "mtok_s": round(Tp / (ms_p / 1e3) / 1e6, 2), "ms_per_step": round(ms_p, 4),
+            "path_hbm_frac": round(Tp * H * FWD_BYTES_PER_HT / (ms_p / 1e3) / 1e9 / hbm_peak, 4)}
+        del p_sets, ws_p
+
         # ---- long-context forward with RoPE and an initial state (one call per step) -------
         wl = synth.WORKLOADS["long_rope_bf16"]
         L = synth.torch_fwd_inputs(wl["B"], wl["T"], wl["H"], 128, 128, kind="ckda",

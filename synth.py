@@ -150,6 +150,10 @@ WORKLOADS = {
     # long context with RoPE (theta 10000, half-split) and a nonzero initial state
     "long_rope_bf16": dict(B=1, T=65536, H=16, dk=128, dv=128, chunk=64, kind="ckda",
                            dtype="bf16", rope_theta=10000.0, h0_std=0.02),
+    # packed sequences of different lengths (ragged ends, one short sequence) with the layer
+    # shape's token count and heads
+    "packed_bf16": dict(lens=[1536, 1024, 700, 512, 300, 24], H=16, dk=128, dv=128, chunk=64,
+                        kind="ckda", dtype="bf16"),
     # batched decode: 256 sequences x 32 heads, 1024 steps
     "decode_bf16": dict(N=256, H=32, dk=128, dv=128, steps=1024, kind="ckda", dtype="bf16"),
 }

@@ -60,6 +60,10 @@ def _load(mutant: int = 0) -> ctypes.CDLL:
                                                ctypes.POINTER(ctypes.c_longlong)] + [
             ctypes.c_int] * 5 + [ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_double,
                                  ctypes.c_longlong, ctypes.c_int]
+        lib.ckda_oracle_bwd.restype = ctypes.c_int
+        lib.ckda_oracle_bwd.argtypes = [D] * 14 + [ctypes.c_int] * 6 + [
+            ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_longlong,
+            ctypes.c_int]
         lib.ckda_oracle_decode.restype = ctypes.c_int
         lib.ckda_oracle_decode.argtypes = [D, D, D, D, D, D, D, ctypes.POINTER(ctypes.c_longlong)] + [
             ctypes.c_int] * 5 + [ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_double]
@@ -173,6 +177,45 @@ def fwd_varlen(q, k, v, alpha, beta, cu_seqlens, h0=None, *, l2norm=True, rope_t
     if rc != 0:
         raise RuntimeError(f"ckda_oracle_fwd_varlen failed with code {rc}")
     return (out[None] if lead else out), hT
+
+
+def bwd(q, k, v, alpha, beta, h0=None, dout=None, dhT=None, *, l2norm=True, rope_theta=0.0,
+        rope_convention=0, rope_dims=0, scale=None, pos_offset=0, nthreads=None):
+    """float64 gradients of L = <dout, out> + <dhT, hT> for the forward `fwd` (same arguments).
+
+    Returns a dict with dq, dk ([B, T, Hk, dk]: summed over the value heads a grouped q/k head
+    serves), dv, dalpha, dbeta and dh0 (None when h0 is None).
+    """
+    q, k, v, alpha, beta = (_f64(x) for x in (q, k, v, alpha, beta))
+    Hk, H = q.shape[2], v.shape[2]
+    qr = np.ascontiguousarray(repeat_qk_heads(q, H, 2))
+    kr = np.ascontiguousarray(repeat_qk_heads(k, H, 2))
+    B, T, _, dk = qr.shape
+    dv = v.shape[-1]
+    assert kr.shape == qr.shape and alpha.shape == qr.shape
+    assert v.shape == (B, T, H, dv) and beta.shape == (B, T, H)
+    h0a = None if h0 is None else _f64(h0)
+    do = None if dout is None else _f64(dout)
+    dh = None if dhT is None else _f64(dhT)
+    g = {n: np.zeros(shape, np.float64) for n, shape in (
+        ("dq", qr.shape), ("dk", qr.shape), ("dv", v.shape), ("dalpha", alpha.shape),
+        ("dbeta", beta.shape))}
+    g["dh0"] = None if h0a is None else np.zeros(h0a.shape, np.float64)
+    if scale is None:
+        scale = default_scale(dk)
+    if nthreads is None:
+        nthreads = os.cpu_count() or 1
+    rc = _load().ckda_oracle_bwd(
+        _ptr(qr), _ptr(kr), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(h0a), _ptr(do), _ptr(dh),
+        _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dalpha"]), _ptr(g["dbeta"]),
+        _ptr(g["dh0"]), B, T, H, dk, dv, int(bool(l2norm)), float(rope_theta),
+        int(rope_convention), int(rope_dims), float(scale), int(pos_offset), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"ckda_oracle_bwd failed with code {rc}")
+    if Hk != H:   # a q/k head serves H / Hk value heads: its gradient is their sum
+        for n in ("dq", "dk"):
+            g[n] = g[n].reshape(B, T, Hk, H // Hk, dk).sum(axis=3)
+    return g
 
 
 def gates(a=None, b=None, *, mutant=0):

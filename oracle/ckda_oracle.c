@@ -39,6 +39,9 @@
  * Definition", parameterises the gates from unconstrained logits as beta_t = 2 sigma(b_t) and the
  * signed gates alpha_{t,i} = 2 sigma(a_{t,i}) - 1, sigma the logistic function.
  *
+ * Backward (ckda_oracle_bwd, at the end of this file): reverse-mode gradients of the same forward,
+ * pinned to central finite differences of it.
+ *
  * Planted mistakes (CKDA_ORACLE_MUTANT=n at compile time) exist only so that the test suite can
  * prove its pins catch each class of error; the default build (0) is the oracle.
  */
@@ -385,4 +388,212 @@ int ckda_oracle_prologue(const double* x, double* y, int B, int T, int H, int d,
             }
     free(buf);
     return 0;
+}
+
+/*
+ * Reverse-mode gradients of the forward above, by backpropagation through the token loop, for a
+ * loss L with dL/dout = dout and dL/dhT = dhT (either may be NULL for zero).  Per (b, h) the
+ * forward is replayed with every state S_0 .. S_T kept, then the tokens are walked backwards.
+ * One token (q^, k^ the prepared vectors, S' = Diag(alpha) S_{t-1}, w = S'^T k^, u = v - w,
+ * S_t = S' + beta k^ u^T, o = scale S_t^T q^) gives, with G the gradient of S_t (future tokens
+ * plus this token's read-out, G += scale q^ do^T):
+ *   dq^ = scale S_t do,  dbeta = k^T G u,  dv = du = beta G^T k^,  dk^ = beta G u + S' dw,
+ *   dw = -du,  G' = G + k^ dw^T (gradient of S'),  dalpha_i = sum_j G'_ij S_{t-1,ij},
+ *   gradient of S_{t-1} = Diag(alpha) G'.
+ * The prologue is differentiated through: for the norm n(y) = y s, s = (|y|^2 + eps)^(-1/2),
+ * dy = s dn - s^3 (y . dn) y; the rotation is orthogonal, so dx = R^T dy, the rotation by -p.
+ * Outputs dq, dk, dalpha: [B, T, H, dk]; dv: [B, T, H, dv]; dbeta: [B, T, H]; dh0: [B, H, dk, dv]
+ * (may be NULL).  Gates are taken as values (the logit form composes with dalpha / da =
+ * (1 - alpha^2) / 2 and dbeta / db = beta (1 - beta / 2)).
+ * Returns 0 on success, -1 on bad arguments, -2 on allocation failure.
+ */
+typedef struct {
+    const double *q, *k, *v, *alpha, *beta, *h0, *dout, *dhT;
+    double *dq, *dk, *dv, *dalpha, *dbeta, *dh0;
+    int B, T, H, dk_, dv_, l2norm, convention, rot;
+    double theta, scale;
+    long long pos_offset;
+    int next;
+    pthread_mutex_t lock;
+    int status;
+} bwd_job;
+
+/* Gradient through x^ = n(R x) for one head vector: y is R x (before the norm), g the gradient of
+ * x^ on entry and of x on return. */
+static void prologue_backward(double* g, const double* y, int d, int rot, long long p, int l2norm,
+                              double theta, int convention) {
+    if (l2norm) {
+        double ss = 0.0, yg = 0.0;
+        for (int i = 0; i < d; ++i) { ss += y[i] * y[i]; yg += y[i] * g[i]; }
+        double s = 1.0 / sqrt(ss + L2_EPS);
+        for (int i = 0; i < d; ++i) g[i] = s * g[i] - s * s * s * yg * y[i];
+    }
+    if (theta > 0.0) rope_rotate(g, rot, -p, theta, convention);
+}
+
+static void* bwd_worker(void* arg) {
+    bwd_job* J = (bwd_job*)arg;
+    const int dk = J->dk_, dv = J->dv_, H = J->H, T = J->T;
+    const size_t SS = (size_t)dk * dv;
+    double* St = (double*)malloc(sizeof(double) * SS * (size_t)(T + 1));   /* S_0 .. S_T */
+    double* Y = (double*)malloc(sizeof(double) * (size_t)T * 2 * dk);      /* R q, R k per token */
+    double* QK = (double*)malloc(sizeof(double) * (size_t)T * 2 * dk);     /* q^, k^ per token */
+    double* G = (double*)malloc(sizeof(double) * SS);
+    double* Sp = (double*)malloc(sizeof(double) * SS);
+    double* w = (double*)malloc(sizeof(double) * dv);
+    double* u = (double*)malloc(sizeof(double) * dv);
+    double* du = (double*)malloc(sizeof(double) * dv);
+    double* o = (double*)malloc(sizeof(double) * dv);
+    double* gq = (double*)malloc(sizeof(double) * dk);
+    double* gk = (double*)malloc(sizeof(double) * dk);
+    if (!St || !Y || !QK || !G || !Sp || !w || !u || !du || !o || !gq || !gk) {
+        J->status = -2;
+        free(St); free(Y); free(QK); free(G); free(Sp); free(w); free(u); free(du); free(o);
+        free(gq); free(gk);
+        return NULL;
+    }
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        int pair = J->next++;
+        pthread_mutex_unlock(&J->lock);
+        if (pair >= J->B * H) break;
+        int b = pair / H, h = pair % H;
+        size_t sofs = ((size_t)b * H + h) * SS;
+        /* forward replay, keeping every state and the prepared vectors */
+        if (J->h0) memcpy(St, J->h0 + sofs, sizeof(double) * SS);
+        else memset(St, 0, sizeof(double) * SS);
+        for (int t = 0; t < T; ++t) {
+            size_t row = ((size_t)b * T + t) * H + h;
+            double* yq = Y + (size_t)t * 2 * dk;
+            double* yk = yq + dk;
+            double* qh = QK + (size_t)t * 2 * dk;
+            double* kh = qh + dk;
+            memcpy(yq, J->q + row * dk, sizeof(double) * dk);
+            memcpy(yk, J->k + row * dk, sizeof(double) * dk);
+            if (J->theta > 0.0) {
+                rope_rotate(yq, J->rot, J->pos_offset + t, J->theta, J->convention);
+                rope_rotate(yk, J->rot, J->pos_offset + t, J->theta, J->convention);
+            }
+            memcpy(qh, yq, sizeof(double) * dk);
+            memcpy(kh, yk, sizeof(double) * dk);
+            if (J->l2norm) {
+                l2_normalise(qh, dk);
+                l2_normalise(kh, dk);
+            }
+            double* S = St + (size_t)(t + 1) * SS;
+            memcpy(S, St + (size_t)t * SS, sizeof(double) * SS);
+            recurrence_token(S, qh, kh, J->v + row * dv, J->alpha + row * dk, J->beta[row],
+                             J->scale, dk, dv, w, o);
+        }
+        /* backward over the tokens */
+        if (J->dhT) memcpy(G, J->dhT + sofs, sizeof(double) * SS);
+        else memset(G, 0, sizeof(double) * SS);
+        for (int t = T - 1; t >= 0; --t) {
+            size_t row = ((size_t)b * T + t) * H + h;
+            const double* S = St + (size_t)(t + 1) * SS;
+            const double* S0 = St + (size_t)t * SS;
+            const double* qh = QK + (size_t)t * 2 * dk;
+            const double* kh = qh + dk;
+            const double* a = J->alpha + row * dk;
+            const double* vt = J->v + row * dv;
+            const double bt = J->beta[row];
+            const double* dot = J->dout ? J->dout + row * dv : NULL;
+            /* read-out: dq^ = scale S_t do, G += scale q^ do^T */
+            for (int i = 0; i < dk; ++i) {
+                double acc = 0.0;
+                if (dot)
+                    for (int j = 0; j < dv; ++j) acc += S[(size_t)i * dv + j] * dot[j];
+                gq[i] = J->scale * acc;
+            }
+            if (dot)
+                for (int i = 0; i < dk; ++i)
+                    for (int j = 0; j < dv; ++j) G[(size_t)i * dv + j] += J->scale * qh[i] * dot[j];
+            /* S' = Diag(alpha) S_{t-1}, w = S'^T k^, u = v - w */
+            for (int i = 0; i < dk; ++i)
+                for (int j = 0; j < dv; ++j) Sp[(size_t)i * dv + j] = a[i] * S0[(size_t)i * dv + j];
+            for (int j = 0; j < dv; ++j) {
+                double acc = 0.0;
+                for (int i = 0; i < dk; ++i) acc += Sp[(size_t)i * dv + j] * kh[i];
+                w[j] = acc;
+                u[j] = vt[j] - acc;
+            }
+            /* rank-one write */
+            double db = 0.0;
+            for (int i = 0; i < dk; ++i) {
+                double gu = 0.0;
+                for (int j = 0; j < dv; ++j) gu += G[(size_t)i * dv + j] * u[j];
+                db += kh[i] * gu;
+                gk[i] = bt * gu;
+            }
+            for (int j = 0; j < dv; ++j) {
+                double acc = 0.0;
+                for (int i = 0; i < dk; ++i) acc += G[(size_t)i * dv + j] * kh[i];
+                du[j] = bt * acc;
+            }
+            J->dbeta[row] = db;
+            for (int j = 0; j < dv; ++j) J->dv[row * dv + j] = du[j];
+            /* w = S'^T k^ with dw = -du: G' = G + k^ dw^T, dk^ += S' dw */
+            for (int i = 0; i < dk; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < dv; ++j) {
+                    G[(size_t)i * dv + j] -= kh[i] * du[j];
+                    acc -= Sp[(size_t)i * dv + j] * du[j];
+                }
+                gk[i] += acc;
+            }
+            /* S' = Diag(alpha) S_{t-1} */
+            for (int i = 0; i < dk; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < dv; ++j) {
+                    acc += G[(size_t)i * dv + j] * S0[(size_t)i * dv + j];
+                    G[(size_t)i * dv + j] *= a[i];
+                }
+                J->dalpha[row * dk + i] = acc;
+            }
+            /* prologue */
+            const double* yq = Y + (size_t)t * 2 * dk;
+            const double* yk = yq + dk;
+            prologue_backward(gq, yq, dk, J->rot, J->pos_offset + t, J->l2norm, J->theta, J->convention);
+            prologue_backward(gk, yk, dk, J->rot, J->pos_offset + t, J->l2norm, J->theta, J->convention);
+            memcpy(J->dq + row * dk, gq, sizeof(double) * dk);
+            memcpy(J->dk + row * dk, gk, sizeof(double) * dk);
+        }
+        if (J->dh0) memcpy(J->dh0 + sofs, G, sizeof(double) * SS);
+    }
+    free(St); free(Y); free(QK); free(G); free(Sp); free(w); free(u); free(du); free(o);
+    free(gq); free(gk);
+    return NULL;
+}
+
+int ckda_oracle_bwd(const double* q, const double* k, const double* v, const double* alpha,
+                    const double* beta, const double* h0, const double* dout, const double* dhT,
+                    double* dq, double* dk_out, double* dv_out, double* dalpha, double* dbeta,
+                    double* dh0, int B, int T, int H, int dk, int dv, int l2norm, double rope_theta,
+                    int rope_convention, int rope_dims, double scale, long long pos_offset,
+                    int nthreads) {
+    if (!q || !k || !v || !alpha || !beta || !dq || !dk_out || !dv_out || !dalpha || !dbeta)
+        return -1;
+    if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return -1;
+    if (check_rope(dk, rope_theta, &rope_dims) != 0) return -1;
+    bwd_job J;
+    J.q = q; J.k = k; J.v = v; J.alpha = alpha; J.beta = beta; J.h0 = h0; J.dout = dout;
+    J.dhT = dhT; J.dq = dq; J.dk = dk_out; J.dv = dv_out; J.dalpha = dalpha; J.dbeta = dbeta;
+    J.dh0 = dh0; J.B = B; J.T = T; J.H = H; J.dk_ = dk; J.dv_ = dv; J.l2norm = l2norm;
+    J.convention = rope_convention; J.rot = rope_dims; J.theta = rope_theta; J.scale = scale;
+    J.pos_offset = pos_offset; J.next = 0; J.status = 0;
+    pthread_mutex_init(&J.lock, NULL);
+    int pairs = B * H;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > pairs) nthreads = pairs > 0 ? pairs : 1;
+    pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    if (!th) { pthread_mutex_destroy(&J.lock); return -2; }
+    int started = 0;
+    for (int i = 1; i < nthreads; ++i) {
+        if (pthread_create(&th[i], NULL, bwd_worker, &J) == 0) ++started; else break;
+    }
+    bwd_worker(&J);
+    for (int i = 1; i <= started; ++i) pthread_join(th[i], NULL);
+    free(th);
+    pthread_mutex_destroy(&J.lock);
+    return J.status;
 }

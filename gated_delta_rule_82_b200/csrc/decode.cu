@@ -41,6 +41,20 @@ __device__ __forceinline__ void st_stream(float* p, float4 v) {
                  :: "l"(p), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w) : "memory");
 }
 
+// Loads of the small per-head vectors, as volatile asm so that they keep their place ahead of the
+// state loads: issued first, they return long before the 64 KiB of state behind them, and the
+// q/k preparation overlaps the state's arrival.
+__device__ __forceinline__ float ld_vec(const float* p) {
+    float x;
+    asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(x) : "l"(p));
+    return x;
+}
+__device__ __forceinline__ float ld_vec(const __nv_bfloat16* p) {
+    unsigned short x;
+    asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(x) : "l"(p));
+    return __bfloat162float(__ushort_as_bfloat16(x));
+}
+
 // kRope: the rotation is compiled in only where it is asked for (the step is latency-bound per CTA
 // at two CTAs per SM, so code that a call does not need is left out of its kernel).
 template <typename T, int DK, int DV, bool kLogits, bool kRope>
@@ -63,7 +77,36 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
     const int head = blockIdx.x * HPC + hl;
     const bool valid = head < NH;
 
-    // 1. stream this thread's strip of the state in (issued first, consumed last)
+    // 1. the per-head vectors (q, k, alpha: NQ elements a thread, v: NV) are requested first
+    constexpr int NQ = (HPC * DK + kDecodeThreads - 1) / kDecodeThreads;
+    constexpr int NV = (HPC * DV + kDecodeThreads - 1) / kDecodeThreads;
+    float qv[NQ], kv[NQ], av[NQ], vv[NV], bv = 0.f;
+#pragma unroll
+    for (int i = 0; i < NQ; ++i) {
+        const int e = tid + i * kDecodeThreads, hh = e / DK, c = e % DK;
+        const int g = blockIdx.x * HPC + hh;
+        qv[i] = kv[i] = av[i] = 0.f;
+        if (e < HPC * DK && g < NH) {
+            // value head g reads q/k head g / G (grouped value heads; G = 1 without grouping)
+            const int gq = G == 1 ? g : g / G;
+            qv[i] = ld_vec(q + (size_t)gq * DK + c);
+            kv[i] = ld_vec(k + (size_t)gq * DK + c);
+            // gate values (fp32), or logits a in the activation type (alpha = 2 sigma(a) - 1 below)
+            if constexpr (kLogits)
+                av[i] = ld_vec(static_cast<const T*>(alpha) + (size_t)g * DK + c);
+            else
+                av[i] = ld_vec(static_cast<const float*>(alpha) + (size_t)g * DK + c);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int e = tid + i * kDecodeThreads, hh = e / DV, c = e % DV;
+        const int g = blockIdx.x * HPC + hh;
+        vv[i] = (e < HPC * DV && g < NH) ? ld_vec(v + (size_t)g * DV + c) : 0.f;
+    }
+    if (tid < HPC && blockIdx.x * HPC + tid < NH) bv = ld_vec(beta + blockIdx.x * HPC + tid);
+
+    // 2. then this thread's strip of the state (consumed last)
     float4 s[R];
     float* sbase = state + (size_t)(valid ? head : 0) * DK * DV + c4 * 4;
     if (valid) {
@@ -71,39 +114,27 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
         for (int j = 0; j < R; ++j) s[j] = ld_stream(sbase + (size_t)(rg + j * RG) * DV);
     }
 
-    // 2. per-head vectors into shared memory (fp32)
-    for (int e = tid; e < HPC * DK; e += kDecodeThreads) {
-        int hh = e / DK, c = e % DK;
-        int g = blockIdx.x * HPC + hh;
-        float qv = 0.f, kv = 0.f, av = 0.f;
-        if (g < NH) {
-            // value head g reads q/k head g / G (grouped value heads; G = 1 without grouping)
-            const int gq = G == 1 ? g : g / G;
-            qv = to_f32(q[(size_t)gq * DK + c]);
-            kv = to_f32(k[(size_t)gq * DK + c]);
-            // gate values (fp32), or logits a in the activation type: alpha = 2 sigma(a) - 1
-            if constexpr (kLogits)
-                av = gate_alpha(to_f32(static_cast<const T*>(alpha)[(size_t)g * DK + c]));
-            else
-                av = static_cast<const float*>(alpha)[(size_t)g * DK + c];
+    // 3. the vectors into shared memory (fp32)
+#pragma unroll
+    for (int i = 0; i < NQ; ++i) {
+        const int e = tid + i * kDecodeThreads;
+        if (e < HPC * DK) {
+            sq[e / DK][e % DK] = qv[i];
+            sk[e / DK][e % DK] = kv[i];
+            sa[e / DK][e % DK] = kLogits ? gate_alpha(av[i]) : av[i];
         }
-        sq[hh][c] = qv; sk[hh][c] = kv; sa[hh][c] = av;
     }
-    for (int e = tid; e < HPC * DV; e += kDecodeThreads) {
-        int hh = e / DV, c = e % DV;
-        int g = blockIdx.x * HPC + hh;
-        sv[hh][c] = g < NH ? to_f32(v[(size_t)g * DV + c]) : 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int e = tid + i * kDecodeThreads;
+        if (e < HPC * DV) sv[e / DV][e % DV] = vv[i];
     }
     if (kRope)
         for (int i = tid; i < DK / 2; i += kDecodeThreads) sfreq[i] = rp.inv_freq[i];
-    if (tid < HPC) {
-        int g = blockIdx.x * HPC + tid;
-        const float bv = g < NH ? beta[g] : 0.f;
-        sbeta[tid] = (kLogits && g < NH) ? gate_beta(bv) : bv;
-    }
+    if (tid < HPC) sbeta[tid] = (kLogits && blockIdx.x * HPC + tid < NH) ? gate_beta(bv) : bv;
     __syncthreads();
 
-    // 3. rotation and L2 norm of q and k: one warp per head
+    // 4. rotation and L2 norm of q and k: one warp per head
     const int lane = tid & 31, warp = tid >> 5;
     for (int hh = warp; hh < HPC; hh += kDecodeThreads / 32) {
         int g = blockIdx.x * HPC + hh;
@@ -161,7 +192,7 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
     }
     __syncthreads();
 
-    // 4. gate the rows and reduce w = S'^T k, y = S'^T q over this thread's rows
+    // 5. gate the rows and reduce w = S'^T k, y = S'^T q over this thread's rows
     float4 w = make_float4(0.f, 0.f, 0.f, 0.f), y = w;
     if (valid) {
 #pragma unroll
@@ -186,7 +217,7 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
     }
     if (!valid) return;
 
-    // 5. rank-one write and read-out
+    // 6. rank-one write and read-out
     const float bt = sbeta[hl];
     float4 u;
     u.x = bt * (sv[hl][c4 * 4 + 0] - w.x);

@@ -158,10 +158,11 @@ def event_time_ms(fn, steps, stream):
     return e0.elapsed_time(e1)
 
 
-def kernel_source_hash():
+def kernel_source_hash(files=None):
+    """Hash of the named sources under csrc/ (all of them when files is None)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_delta_rule_82_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(files if files is not None else os.listdir(csrc)):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -169,18 +170,18 @@ def kernel_source_hash():
 
 
 def ncu_traffic(kernel):
-    """DRAM bytes per launch for `kernel` from the committed ncu summary, if the kernel sources
-    are unchanged since that capture (else None)."""
+    """DRAM bytes per launch for `kernel` from the committed ncu summary, if the sources the
+    kernel is built from are unchanged since that capture (else None)."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
     except Exception:
         return None
-    if d.get("source_hash") != kernel_source_hash():
-        return None
     ent = d.get("kernels", {}).get(kernel)
-    return None if ent is None else ent.get("dram_bytes_per_launch")
+    if ent is None or ent.get("source_hash") != kernel_source_hash(ent.get("sources")):
+        return None
+    return ent.get("dram_bytes_per_launch")
 
 
 # ---- the reference arm: float64 CPU oracle ---------------------------------------------------

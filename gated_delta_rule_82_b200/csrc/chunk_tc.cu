@@ -371,6 +371,18 @@ struct WorkOrder {
         it.hk = (int)fastdiv(group, (uint32_t)it.h);
         return it;
     }
+    // packed sequences: item i is entry i of the item table, (head unit, chunk of its lane)
+    __device__ __forceinline__ Item item(int i, const int2* __restrict__ itab) const {
+        if (!itab) return item(i);
+        const int2 e = itab[i];
+        Item it;
+        it.bh = e.x;
+        it.c = e.y;
+        it.b = (int)fastdiv(heads, (uint32_t)it.bh);   // the lane
+        it.h = it.bh - it.b * (int)heads.d;
+        it.hk = (int)fastdiv(group, (uint32_t)it.h);
+        return it;
+    }
 };
 // The items one factor CTA takes: a leading run start1, start1 + stride1, ... (n1 of them), then
 // start2, start2 + stride2, ... up to `total` (none when start2 >= total).
@@ -381,27 +393,42 @@ struct ItemSeq {
         return i < total ? i : -1;
     }
 };
-// Packed sequences of different lengths: the chunk axis runs over the chunks of every sequence in
-// turn, and entry c of the chunk table (built on the device from the token offsets) says where
-// chunk c lies: x = first token on the packed token axis, y = tokens in the chunk (1..64), z = its
-// sequence, w = its index within the sequence, with kLastChunk set on the sequence's last chunk.
-// Without a table (a batch of equal lengths) chunk c starts at token 64 c of its batch row.
+// Packed sequences of different lengths.  The sequences are dealt, in order, to lanes: runs of
+// whole sequences with about the same number of chunks.  A lane plays the part of a batch row:
+// head unit bh = lane * H + h, and chunk c of a unit is chunk c of its lane (the chunks of the
+// lane's sequences in turn).  Lanes hold different numbers of chunks (lane_cnt); NT is the
+// largest, and slots past a lane's count are never used.  Entry lane * NT + c of the chunk table
+// (built on the device from the token offsets) says where a chunk lies: x = first token on the
+// packed token axis, y = tokens in the chunk (1..64), z = its sequence, w = its index within the
+// sequence, with kLastChunk set on the sequence's last chunk.  The item table lists the factor
+// work, (unit, chunk) pairs, in the order the work order would give (head groups, chunk-major
+// inside a group), skipping the unused slots.  Without tables (a batch of equal lengths) chunk c
+// starts at token 64 c of batch row b.
 constexpr int kLastChunk = 1 << 30;
+struct PackedTabs {
+    const int4* ctab;      // chunk table [lanes * NT]
+    const int* lane_cnt;   // chunks of each lane [lanes]
+    const int2* itab;      // item table [items]
+};
 struct ChunkAt {
+    int b;            // batch coordinate of the tensor maps (0 for packed sequences)
     int t0, nvalid, seq, last;
     long long pos0;   // rotary position of the chunk's first token
 };
-__device__ __forceinline__ ChunkAt chunk_at(const int4* __restrict__ ctab, int c, int T_len, int NT,
-                                            long long pos_offset) {
+__device__ __forceinline__ ChunkAt chunk_at(const int4* __restrict__ ctab, const Item& it, int T_len,
+                                            int NT, long long pos_offset) {
     ChunkAt a;
+    const int c = it.c;
     if (ctab) {
-        const int4 e = ctab[c];
+        const int4 e = ctab[(size_t)it.b * NT + c];   // it.b is the lane
+        a.b = 0;
         a.t0 = e.x;
         a.nvalid = e.y;
         a.seq = e.z;
         a.last = (e.w & kLastChunk) != 0;
         a.pos0 = pos_offset + (long long)(e.w & (kLastChunk - 1)) * kC;
     } else {
+        a.b = it.b;
         a.t0 = c * kC;
         a.nvalid = min(kC, T_len - a.t0);
         a.seq = 0;
@@ -474,7 +501,7 @@ __device__ __forceinline__ bool mbar_wait_long(uint64_t* bar, uint32_t parity, v
 template <bool kLogits>
 __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, const void* __restrict__ alpha,
                                            const float* __restrict__ beta, uint8_t* __restrict__ ws,
-                                           int* __restrict__ flags, const int4* __restrict__ ctab,
+                                           int* __restrict__ flags, PackedTabs pt,
                                            int T_len, int H, int NT, WorkOrder wo, ItemSeq seq, int l2norm,
                                            const RopeParams& rp, long long pos_offset, uint32_t tmem) {
     constexpr int gate_logits = kLogits ? 1 : 0;
@@ -525,29 +552,29 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
         tc::prefetch_tensormap(&maps.k);
         tc::prefetch_tensormap(&maps.v);
         tc::prefetch_tensormap(&maps.alpha);
-        const Item first = wo.item(i0);
-        const int ft0 = chunk_at(ctab, first.c, T_len, NT, pos_offset).t0;
-        issue_inputs(maps, sm, bar_in, first.b, first.h, first.hk, ft0, gate_logits);
-        issue_v(maps, sm, bar_v, first.b, first.h, ft0);
+        const Item first = wo.item(i0, pt.itab);
+        const ChunkAt fa = chunk_at(pt.ctab, first, T_len, NT, pos_offset);
+        issue_inputs(maps, sm, bar_in, fa.b, first.h, first.hk, fa.t0, gate_logits);
+        issue_v(maps, sm, bar_v, fa.b, first.h, fa.t0);
     }
     // where the current item's chunk lies; the next item's entry is read one item ahead
-    ChunkAt at_next = chunk_at(ctab, i0 >= 0 ? wo.item(i0).c : 0, T_len, NT, pos_offset);
+    ChunkAt at_next = chunk_at(pt.ctab, wo.item(i0 >= 0 ? i0 : 0, pt.itab), T_len, NT, pos_offset);
 
     // persistent loop over items; chunk-head ci = (batch*head) * NT + chunk
     uint32_t it = 0;
     int pending = -1;   // chunk-head whose images are stored but not yet flagged ready
     for (int k = 0, i = i0; i >= 0; i = seq.at(++k), ++it) {
-        const Item cur = wo.item(i);
+        const Item cur = wo.item(i, pt.itab);
         const int ci = cur.bh * NT + cur.c;
         const ChunkAt at = at_next;
         const int t0 = at.t0;
         const int nvalid = at.nvalid;
         const int inext = seq.at(k + 1);
         const bool has_next = inext >= 0;
-        const Item nxt = wo.item(has_next ? inext : i);
-        at_next = chunk_at(ctab, nxt.c, T_len, NT, pos_offset);
+        const Item nxt = wo.item(has_next ? inext : i, pt.itab);
+        at_next = chunk_at(pt.ctab, nxt, T_len, NT, pos_offset);
         uint8_t* wsc = ws + (size_t)ci * WS_CHUNK;
-        const size_t row0 = ((size_t)cur.b * T_len + t0) * H + cur.h;
+        const size_t row0 = ((size_t)at.b * T_len + t0) * H + cur.h;
         float bval = (tid < 64 && tid < nvalid) ? beta[row0 + tid * rs] : 0.f;
         if (kLogits && tid < 64 && tid < nvalid) bval = gate_beta(bval);   // beta = 2 sigma(b)
 
@@ -728,7 +755,7 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
         tc::tc_fence_after();
         // alpha, q, k of this chunk-head are consumed: bring in the next one's.  Issued by warp 15
         // (a TMA issue costs its thread several hundred cycles) while warp 0 issues the product.
-        if (tid == 480 && has_next) issue_inputs(maps, sm, bar_in, nxt.b, nxt.h, nxt.hk, at_next.t0, gate_logits);
+        if (tid == 480 && has_next) issue_inputs(maps, sm, bar_in, at_next.b, nxt.h, nxt.hk, at_next.t0, gate_logits);
         if (!exact) {
             // ======== B: [A | M] = L R^T on the tensor cores (M = 128, N = 64, K = 128) ========
             if (warp == 0) {
@@ -897,7 +924,7 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
         pending = -1;
         // V of this chunk-head was consumed by the W/U~ products: bring in the next one's, from
         // warp 14 while warp 0 issues these products
-        if (tid == 448 && has_next) issue_v(maps, sm, bar_v, nxt.b, nxt.h, at_next.t0);
+        if (tid == 448 && has_next) issue_v(maps, sm, bar_v, at_next.b, nxt.h, at_next.t0);
         tc::mbar_wait(bar_q, it & 1, abort_flag);
         tc::tc_fence_after();
         // ======== G: results into shared staging images, then bulk stores in two groups ========
@@ -1020,7 +1047,7 @@ static_assert(SS_OSTAGE % 1024 == 0 && (WS_QP - WS_UT) % 1024 == 0 && (WS_M - WS
 constexpr uint32_t kColS = 128, kColO = 256;
 
 __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, const uint8_t* __restrict__ ws,
-                                           const int* __restrict__ flags, const int4* __restrict__ ctab,
+                                           const int* __restrict__ flags, PackedTabs pt,
                                            const float* __restrict__ h0,
                                            __nv_bfloat16* __restrict__ out, float* __restrict__ hT,
                                            int T_len, int H, int NT, int BH, float scale, int head0,
@@ -1038,8 +1065,11 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
     volatile int* abort_flag = reinterpret_cast<volatile int*>(dc_free + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int nheads = head0 < BH ? (BH - head0 + hstride - 1) / hstride : 0;
-    const int U = nheads * NT;
+    // chunks of head unit bh: NT, or (packed sequences) the count of its lane
+    const int4* __restrict__ ctab = pt.ctab;
+    auto units_chunks = [&](int bh) { return pt.lane_cnt ? pt.lane_cnt[bh / H] : NT; };
+    int U = 0;   // items of this CTA: the chunks of heads head0, head0 + hstride, ...
+    for (int bh = head0; bh < BH; bh += hstride) U += units_chunks(bh);
 
     if (tid == 32) {
         tc::mbar_init(dc_free, 8);
@@ -1098,15 +1128,22 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&s_ready[u & 1]);
         };
+        // packed sequences: unit bh is (lane bh / H, head bh % H); tab is its lane's chunk table
+        // and srow gives the state row of (sequence, head)
+        const int4* tab = ctab ? ctab + (size_t)(head0 / H) * NT : nullptr;
+        auto srow = [&](int4 e, int bh) { return ctab ? e.z * H + bh % H : bh; };
+        int nc = U > 0 ? units_chunks(head0) : 0;
         if (U > 0) {
-            load_h0(ctab ? ctab[0].z * H + head0 : head0);
+            load_h0(srow(ctab ? tab[0] : make_int4(0, 0, 0, 0), head0));
             put_s(0);
         }
         for (int u = 0, c = 0, bh = head0; u < U; ++u) {
             // this chunk's entry and the next item's (read ahead of the wait)
-            const int c2 = c + 1 < NT ? c + 1 : 0, bh2 = c + 1 < NT ? bh : bh + hstride;
-            const int4 ecur = ctab ? ctab[c] : make_int4(0, 0, 0, c == NT - 1 ? kLastChunk : 0);
-            const int4 enext = ctab ? ctab[c2] : make_int4(0, 0, 0, c2);
+            const bool same = c + 1 < nc;
+            const int c2 = same ? c + 1 : 0, bh2 = same ? bh : bh + hstride;
+            const int4* tab2 = ctab ? (same ? tab : ctab + (size_t)(bh2 / H) * NT) : nullptr;
+            const int4 ecur = ctab ? tab[c] : make_int4(0, 0, 0, c == NT - 1 ? kLastChunk : 0);
+            const int4 enext = ctab && u + 1 < U ? tab2[c2] : make_int4(0, 0, 0, c2);
             if (!wait(mma_c, u & 1)) break;
             tc::tc_fence_after();
             tc::tmem_ld64_sync(tc::tmem_addr(tmem, 32 * q, cb), S);
@@ -1116,8 +1153,7 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
             if (lane == 0) tc::mbar_arrive(dc_free);
             const bool last = (ecur.w & kLastChunk) != 0;
             if (last && hT && !*abort_flag) {
-                const int srow = ctab ? ecur.z * H + bh : bh;
-                float* dst = hT + ((size_t)srow * kDK + cb) * kDV + n;
+                float* dst = hT + ((size_t)srow(ecur, bh) * kDK + cb) * kDV + n;
 #pragma unroll
                 for (int j = 0; j < 64; ++j) dst[(size_t)j * kDV] = S[j];
             }
@@ -1126,14 +1162,16 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
                 // be done with it
                 if (u >= 1 && !wait(&mma_o[(u - 1) & 3], ((u - 1) >> 2) & 1)) break;
                 // the next item starts a sequence: its initial state
-                if ((enext.w & (kLastChunk - 1)) == 0) load_h0(ctab ? enext.z * H + bh2 : bh2);
+                if ((enext.w & (kLastChunk - 1)) == 0) load_h0(srow(enext, bh2));
                 put_s(u + 1);
             } else {
                 tc::tc_fence_before();
             }
-            if (++c == NT) {
+            if (++c == nc) {
                 c = 0;
                 bh += hstride;
+                tab = tab2;
+                if (u + 1 < U) nc = units_chunks(bh);
             }
         }
     } else if (warp == 8) {
@@ -1202,14 +1240,16 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
             const uint32_t bytes = chain ? SS_CSTAGE : SS_OSTAGE;
             uint8_t* stage0 = sm + (chain ? SS_C : SS_O);
             int issued = 0;
+            int nc = U > 0 ? units_chunks(head0) : 0;
             for (int c = 0, bh = head0; issued < U; ++issued) {
                 const int st = issued & 1;
                 if (issued >= 2 && !mbar_wait_long(&emptyb[st], ((issued >> 1) - 1) & 1, abort_flag))
                     break;
                 const size_t ci = (size_t)bh * NT + c;
-                if (++c == NT) {
+                if (++c == nc) {
                     c = 0;
                     bh += hstride;
+                    if (issued + 1 < U) nc = units_chunks(bh);
                 }
                 if (!flag_wait(flags + ci, abort_flag)) break;
                 tc::mbar_arrive_expect_tx(&fullb[st], bytes);
@@ -1230,10 +1270,12 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
         const int q = warp & 3, n = 32 * q + lane;
         const bool leader = warp == 12 && lane == 0;
         uint8_t* stg = sm + SS_STG;
+        const int4* otab = ctab ? ctab + (size_t)(head0 / H) * NT : nullptr;   // the lane's table
+        int nc = U > 0 ? units_chunks(head0) : 0;
         for (int u = 0, c = 0, bh = head0; u < U; ++u) {
             const int ob = u & 3;
             // the chunk's first token and length (packed sequences: from the chunk table)
-            const int4 e = ctab ? ctab[c] : make_int4(c * kC, kC, 0, 0);
+            const int4 e = ctab ? otab[c] : make_int4(c * kC, kC, 0, 0);
             const bool ok = mbar_wait_long(&mma_o[ob], (u >> 2) & 1, abort_flag);
             // the previous item's tensor store must be done reading the staging tile
             if (leader) tc::bulk_wait_read<0>();
@@ -1256,10 +1298,11 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
             tc::fence_proxy_async_smem();
             __syncwarp();
             tc::bar_named(1, 128);
+            const int h = bh % H;
             if (e.y == kC || !ctab) {
                 // rows past the end of a batch row are clipped by the tensor store
                 if (leader) {
-                    tc::tma_store_4d(&maps.out, stg, 0, bh % H, e.x, bh / H);
+                    tc::tma_store_4d(&maps.out, stg, 0, h, e.x, ctab ? 0 : bh / H);
                     tc::bulk_commit();
                 }
             } else {
@@ -1271,15 +1314,19 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
                     if (e.x + r < T_len) {
                         const uint4 val = *reinterpret_cast<const uint4*>(stg + r * 256 + col * 16);
                         *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(out) +
-                                                  ((size_t)(e.x + r) * H + bh) * (kDV * 2) + col * 16) = val;
+                                                  ((size_t)(e.x + r) * H + h) * (kDV * 2) + col * 16) = val;
                     }
                 }
                 // the staging tile is read before the next item rewrites it
                 tc::bar_named(1, 128);
             }
-            if (++c == NT) {
+            if (++c == nc) {
                 c = 0;
                 bh += hstride;
+                if (u + 1 < U) {
+                    nc = units_chunks(bh);
+                    if (ctab) otab = ctab + (size_t)(bh / H) * NT;
+                }
             }
         }
         if (leader) tc::bulk_wait_all();
@@ -1317,13 +1364,13 @@ template <bool kLogits>
 __global__ void __launch_bounds__(512, 1)
 ckda_tc_intra(const __grid_constant__ TcMaps maps, const void* __restrict__ alpha,
               const float* __restrict__ beta, uint8_t* __restrict__ ws, int* __restrict__ flags,
-              const int4* __restrict__ ctab, int T_len, int H, int NT, int BH, WorkOrder wo,
+              PackedTabs pt, int T_len, int H, int NT, int n_items, WorkOrder wo,
               int l2norm, RopeParams rp, long long pos_offset) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint32_t tmem_slot;
     const uint32_t tmem = kernel_tmem_alloc(&tmem_slot);
-    const ItemSeq seq{(int)blockIdx.x, (int)gridDim.x, 1 << 30, 0, 1, BH * NT};
-    intra_role<kLogits>(aligned_smem(smem_raw), maps, alpha, beta, ws, flags, ctab, T_len, H, NT, wo,
+    const ItemSeq seq{(int)blockIdx.x, (int)gridDim.x, 1 << 30, 0, 1, n_items};
+    intra_role<kLogits>(aligned_smem(smem_raw), maps, alpha, beta, ws, flags, pt, T_len, H, NT, wo,
                         seq, l2norm, rp, pos_offset, tmem);
     kernel_tmem_free(tmem);
 }
@@ -1331,13 +1378,13 @@ ckda_tc_intra(const __grid_constant__ TcMaps maps, const void* __restrict__ alph
 // State pass alone, after the factor kernel: heads blockIdx.x, blockIdx.x + gridDim.x, ...
 __global__ void __launch_bounds__(512, 1)
 ckda_tc_state(const __grid_constant__ TcMaps maps, const uint8_t* __restrict__ ws,
-              const int* __restrict__ flags, const int4* __restrict__ ctab,
+              const int* __restrict__ flags, PackedTabs pt,
               const float* __restrict__ h0, __nv_bfloat16* __restrict__ out,
               float* __restrict__ hT, int T_len, int H, int NT, int BH, float scale) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint32_t tmem_slot;
     const uint32_t tmem = kernel_tmem_alloc(&tmem_slot);
-    state_role(aligned_smem(smem_raw), maps, ws, flags, ctab, h0, out, hT, T_len, H, NT, BH, scale,
+    state_role(aligned_smem(smem_raw), maps, ws, flags, pt, h0, out, hT, T_len, H, NT, BH, scale,
                blockIdx.x, gridDim.x, tmem);
     kernel_tmem_free(tmem);
 }
@@ -1352,41 +1399,61 @@ template <bool kLogits>
 __global__ void __launch_bounds__(512, 1)
 ckda_tc_fused(const __grid_constant__ TcMaps maps, const void* __restrict__ alpha,
               const float* __restrict__ beta, uint8_t* __restrict__ ws, int* __restrict__ flags,
-              const int4* __restrict__ ctab, const float* __restrict__ h0,
+              PackedTabs pt, const float* __restrict__ h0,
               __nv_bfloat16* __restrict__ out, float* __restrict__ hT, int T_len, int H, int NT,
-              int BH, int n_state, int lead, WorkOrder wo, int l2norm, RopeParams rp,
+              int BH, int n_items, int n_state, int lead, WorkOrder wo, int l2norm, RopeParams rp,
               long long pos_offset, float scale) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint32_t tmem_slot;
     uint8_t* sm = aligned_smem(smem_raw);
     const uint32_t tmem = kernel_tmem_alloc(&tmem_slot);
-    const int total = BH * NT, b = blockIdx.x, nall = gridDim.x, nf = nall - n_state;
+    const int total = n_items, b = blockIdx.x, nall = gridDim.x, nf = nall - n_state;
     const bool chain = b < n_state;
     // the leading rounds, then (factor CTAs) every nf-th of the remaining items
     const ItemSeq seq{b, nall, lead, chain ? total : lead * nall + (b - n_state), chain ? 1 : nf, total};
     if (seq.at(0) >= 0)
-        intra_role<kLogits>(sm, maps, alpha, beta, ws, flags, ctab, T_len, H, NT, wo, seq, l2norm,
+        intra_role<kLogits>(sm, maps, alpha, beta, ws, flags, pt, T_len, H, NT, wo, seq, l2norm,
                             rp, pos_offset, tmem);
     if (chain)
-        state_role(sm, maps, ws, flags, ctab, h0, out, hT, T_len, H, NT, BH, scale, b, n_state, tmem);
+        state_role(sm, maps, ws, flags, pt, h0, out, hT, T_len, H, NT, BH, scale, b, n_state, tmem);
     kernel_tmem_free(tmem);
 }
 
-// Packed sequences: the chunk table and the ready flags of one call (one CTA of 1024 threads).
-// Sequences are taken 1024 at a time; a block-wide scan of their chunk counts gives each one its
-// first chunk.  If the device offsets do not give the host's chunk count nc (the two copies of
-// cu_seqlens differ), every entry becomes an empty chunk of sequence 0 and the error flag is set,
-// so that no later access leaves the caller's arrays.
+// How packed sequences are dealt to lanes (computed on the host from the offsets, passed by value).
+constexpr int kMaxLanes = 64;
+struct LanePlan {
+    int P;                      // lanes
+    int NTL;                    // chunks of the longest lane (the NT of the launch)
+    int total;                  // chunks of all sequences (per head)
+    int seq0[kMaxLanes + 1];    // first sequence of each lane; seq0[P] = number of sequences
+    int cbase[kMaxLanes + 1];   // chunks before each lane; cbase[P] = total
+};
+
+// Packed sequences: the tables and the ready flags of one call (one CTA of 1024 threads).
+//  1. chunk table: sequences are taken 1024 at a time; a block-wide scan of their chunk counts
+//     gives each one its first chunk in the global order, and lane l's chunk j is global chunk
+//     cbase[l] + j.  Slots past a lane's count get a harmless entry (never read).
+//  2. item table: head unit u = lane * H + h has lane_cnt[lane] chunks; units form groups of
+//     `group` (the chain CTAs of the launch), and inside a group the items run chunk-major over
+//     the units that have that chunk.  Item (u, c) sits at base(group) + sum over the group's
+//     units of min(count, c) + the number of the group's units before u that have chunk c.
+// If the device offsets do not match the plan (the two copies of cu_seqlens differ), every chunk
+// entry becomes an empty chunk of sequence 0 and the error word is set, so that no later access
+// leaves the caller's arrays.
 constexpr int kPrepThreads = 1024;
 __global__ void __launch_bounds__(kPrepThreads)
-ckda_varlen_prep(const int* __restrict__ cu, int n_seqs, int T_total, int nc, int4* __restrict__ ctab,
-                 int* __restrict__ flags, int n_flags) {
+ckda_varlen_prep(const int* __restrict__ cu, int n_seqs, int T_total, const LanePlan lp, int H,
+                 int group, int4* __restrict__ ctab, int* __restrict__ lane_cnt,
+                 int2* __restrict__ itab, int* __restrict__ flags, int n_flags) {
     __shared__ int warp_sum[32];
     __shared__ int s_bad;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    auto cnt = [&](int l) { return lp.cbase[l + 1] - lp.cbase[l]; };
     for (int i = tid; i < n_flags; i += kPrepThreads) flags[i] = 0;
+    if (tid < lp.P) lane_cnt[tid] = cnt(tid);
     if (tid == 0) s_bad = (cu[0] != 0 || cu[n_seqs] != T_total) ? 1 : 0;
     __syncthreads();
+    // 1. chunk table
     int base = 0;   // chunks of the sequences before this tile
     for (int s0 = 0; s0 < n_seqs; s0 += kPrepThreads) {
         const int sq = s0 + tid;
@@ -1420,23 +1487,52 @@ ckda_varlen_prep(const int* __restrict__ cu, int n_seqs, int T_total, int nc, in
         __syncthreads();
         const int first = base + (warp ? warp_sum[warp - 1] : 0) + x - nch;
         const int tile_total = warp_sum[31];
-        for (int j = 0; j < nch; ++j) {
-            const int c = first + j;
-            if (c < nc)
-                ctab[c] = make_int4(cu[sq] + j * kC, min(kC, len - j * kC), sq,
-                                    j | (j == nch - 1 ? kLastChunk : 0));
-            else
-                s_bad = 1;
+        if (nch > 0) {
+            int l = 0;   // the lane of sequence sq
+            while (l + 1 < lp.P && lp.seq0[l + 1] <= sq) ++l;
+            for (int j = 0; j < nch; ++j) {
+                const int jl = first + j - lp.cbase[l];
+                if (jl >= 0 && jl < cnt(l))
+                    ctab[(size_t)l * lp.NTL + jl] = make_int4(cu[sq] + j * kC, min(kC, len - j * kC),
+                                                              sq, j | (j == nch - 1 ? kLastChunk : 0));
+                else
+                    s_bad = 1;
+            }
         }
         base += tile_total;
         __syncthreads();   // warp_sum is rewritten by the next tile
     }
+    for (int x = tid; x < lp.P * lp.NTL; x += kPrepThreads) {
+        const int l = x / lp.NTL;
+        if (x - l * lp.NTL >= cnt(l)) ctab[x] = make_int4(0, 0, min(lp.seq0[l], n_seqs - 1), 1);
+    }
     __syncthreads();
-    if (base != nc) s_bad = 1;
+    if (base != lp.total) s_bad = 1;
     __syncthreads();
     if (s_bad) {
-        for (int c = tid; c < nc; c += kPrepThreads) ctab[c] = make_int4(0, 0, 0, 0);
+        for (int x = tid; x < lp.P * lp.NTL; x += kPrepThreads) ctab[x] = make_int4(0, 0, 0, 0);
         if (tid == 0) atomicExch(&g_tc_error, 3);
+    }
+    // 2. item table
+    const int BH = lp.P * H;
+    for (int u = tid; u < BH; u += kPrepThreads) {
+        const int l = u / H, n_u = cnt(l);
+        const int g0 = u - u % group, g1 = min(BH, g0 + group);
+        const int la = g0 / H, lb = (g1 - 1) / H;
+        const long long gbase = (long long)H * lp.cbase[la] + (long long)(g0 - la * H) * cnt(la);
+        const int own = u - max(g0, l * H);   // units of u's lane ahead of u in the group
+        long long S = 0;                      // sum over the group's units of min(count, c)
+        for (int c = 0; c < n_u; ++c) {
+            int rank = own, ng = 0;
+            for (int l2 = la; l2 <= lb; ++l2) {
+                const int m = min(g1, (l2 + 1) * H) - max(g0, l2 * H);   // the lane's units in the group
+                const int on = cnt(l2) > c ? m : 0;
+                ng += on;
+                if (l2 < l) rank += on;
+            }
+            itab[gbase + S + rank] = make_int2(u, c);
+            S += ng;
+        }
     }
 }
 
@@ -1491,12 +1587,13 @@ static bool encode_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt,
 
 // Workspace: the images of n = heads x chunks chunk-heads, their ready flags, and (packed
 // sequences) the chunk table of `ntab` entries.
+// Workspace: the images of n = units x NT chunk slots and their ready flags; for packed sequences
+// then the chunk table (lanes x NT entries), the lane counts and the item table.
 static size_t ctab_offset(size_t n) { return flags_offset(n) + ((n * 4 + 255) & ~(size_t)255); }
-static size_t tc_workspace(size_t n, size_t ntab) { return ctab_offset(n) + ntab * sizeof(int4); }
 
 size_t chunk_tc_workspace_bytes(int B, int T_len, int H) {
     const size_t nt = (size_t)(T_len + kC - 1) / kC;
-    return tc_workspace((size_t)B * H * nt, 0);
+    return ctab_offset((size_t)B * H * nt);
 }
 
 long long packed_chunks(const int* cu_host, int n_seqs) {
@@ -1505,9 +1602,63 @@ long long packed_chunks(const int* cu_host, int n_seqs) {
     return nc;
 }
 
+// Lanes of about kLaneChunks chunks: the sequences in order, a lane closed once it holds at least
+// its share and the next sequence has chunks (whole sequences only: a sequence's chunks form one
+// chain).  Lanes stand in for batch rows, so that P x H chains can run where one chain per head
+// would walk through every sequence.
+constexpr int kLaneChunks = 32;
+static LanePlan plan_lanes(const int* cu_host, int n) {
+    LanePlan lp;
+    memset(&lp, 0, sizeof(lp));
+    const long long total = packed_chunks(cu_host, n);
+    int nonempty = 0;
+    for (int s = 0; s < n; ++s) nonempty += cu_host[s + 1] > cu_host[s];
+    int P = (int)((total + kLaneChunks / 2) / kLaneChunks);
+    P = P < 1 ? 1 : P;
+    P = P > kMaxLanes ? kMaxLanes : P;
+    P = P > nonempty ? (nonempty > 0 ? nonempty : 1) : P;
+    const long long share = (total + P - 1) / P;
+    int l = 0;
+    long long in_lane = 0, seen = 0;
+    lp.seq0[0] = 0;
+    lp.cbase[0] = 0;
+    for (int s = 0; s < n; ++s) {
+        const long long nch = (cu_host[s + 1] - cu_host[s] + kC - 1) / kC;
+        if (nch > 0 && in_lane >= share && l < P - 1) {
+            ++l;
+            lp.seq0[l] = s;
+            lp.cbase[l] = (int)seen;
+            in_lane = 0;
+        }
+        in_lane += nch;
+        seen += nch;
+    }
+    lp.P = l + 1;
+    lp.seq0[lp.P] = n;
+    lp.cbase[lp.P] = (int)total;
+    lp.total = (int)total;
+    lp.NTL = 0;
+    for (int i = 0; i < lp.P; ++i)
+        if (lp.cbase[i + 1] - lp.cbase[i] > lp.NTL) lp.NTL = lp.cbase[i + 1] - lp.cbase[i];
+    return lp;
+}
+
+struct PackedLayout {
+    size_t images, ctab, lane_cnt, itab, bytes;   // byte offsets into the workspace, and its size
+};
+static PackedLayout packed_layout(const LanePlan& lp, int H) {
+    PackedLayout w;
+    const size_t slots = (size_t)lp.P * H * lp.NTL;
+    w.images = 0;
+    w.ctab = ctab_offset(slots);
+    w.lane_cnt = w.ctab + (size_t)lp.P * lp.NTL * sizeof(int4);
+    w.itab = w.lane_cnt + (((size_t)lp.P * 4 + 15) & ~(size_t)15);
+    w.bytes = w.itab + (size_t)H * lp.total * sizeof(int2);
+    return w;
+}
+
 size_t chunk_tc_workspace_bytes_packed(const int* cu_host, int n_seqs, int H) {
-    const size_t nc = (size_t)packed_chunks(cu_host, n_seqs);
-    return tc_workspace(nc * H, nc);
+    return packed_layout(plan_lanes(cu_host, n_seqs), H).bytes;
 }
 
 // Split of the fused launch: `n_state` chain CTAs, and `lead` leading rounds of factor items that
@@ -1590,16 +1741,32 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)FUSED_BYTES);
     if (e != cudaSuccess) return e;
-    // packed sequences: one token axis (batch 1) whose chunks run sequence after sequence; a
-    // head's chain walks through all of them, starting again from h0 at each sequence
+    // packed sequences: one token axis (batch 1); the sequences are dealt to lanes that stand in
+    // for batch rows, and a unit's chain walks through its lane's sequences, starting again from
+    // h0 at each one
     const bool packed = pk.cu != nullptr;
-    const int NT = packed ? (int)packed_chunks(pk.cu_host, pk.n) : (T_len + kC - 1) / kC;
-    const int BH = packed ? H : B * H;
+    LanePlan lp;
+    if (packed) lp = plan_lanes(pk.cu_host, pk.n);
+    const int NT = packed ? lp.NTL : (T_len + kC - 1) / kC;
+    const int BH = packed ? lp.P * H : B * H;
     const int Bm = packed ? 1 : B;
-    const int total = NT * BH;
+    const int total = NT * BH;                                 // chunk slots (images, flags)
+    const int n_items = packed ? H * lp.total : total;         // chunk-heads to produce
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     int* flags = reinterpret_cast<int*>(ws + flags_offset((size_t)total));
-    int4* ctab = packed ? reinterpret_cast<int4*>(ws + ctab_offset((size_t)total)) : nullptr;
+    PackedTabs pt{nullptr, nullptr, nullptr};
+    if (packed) {
+        const PackedLayout pl = packed_layout(lp, H);
+        pt.ctab = reinterpret_cast<const int4*>(ws + pl.ctab);
+        pt.lane_cnt = reinterpret_cast<const int*>(ws + pl.lane_cnt);
+        pt.itab = reinterpret_cast<const int2*>(ws + pl.itab);
+    }
+    int dev = 0, nsm = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    if (stages == 0 && nsm < 2) stages = 3;
+    int n_state = 1, lead = 0;
+    if (stages == 0 && n_items > 0) chunk_tc_plan(BH, NT, nsm, &n_state, &lead);
     if (packed && stages != 2) {
         if (hT) {
             // empty sequences keep their initial state
@@ -1614,17 +1781,16 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
                 }
             }
         }
-        if (total == 0) return cudaSuccess;
-        // the chunk table, and every ready flag at zero
-        ckda_varlen_prep<<<1, kPrepThreads, 0, stream>>>(pk.cu, pk.n, T_len, NT, ctab, flags, total);
+        if (n_items == 0) return cudaSuccess;
+        // the chunk and item tables (items grouped as the launch takes them: by chain CTA for the
+        // fused kernel, all units at once for the factor kernel alone), every ready flag at zero
+        ckda_varlen_prep<<<1, kPrepThreads, 0, stream>>>(
+            pk.cu, pk.n, T_len, lp, H, stages == 0 ? n_state : BH, const_cast<int4*>(pt.ctab),
+            const_cast<int*>(pt.lane_cnt), const_cast<int2*>(pt.itab), flags, total);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    if (total == 0) return cudaSuccess;
+    if (n_items == 0) return cudaSuccess;
     __nv_bfloat16* outb = static_cast<__nv_bfloat16*>(out);
-    int dev = 0, nsm = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-    if (stages == 0 && nsm < 2) stages = 3;
     TcMaps maps;
     if (!encode_map(&maps.out, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDV, kDV, H, T_len, Bm,
                     CU_TENSOR_MAP_SWIZZLE_NONE))
@@ -1652,8 +1818,6 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
     if (stages == 0) {
         // one cooperative launch: the runtime makes every CTA resident at once, which the chain
         // CTAs (waiting on flags the factor CTAs raise) rely on
-        int n_state = 1, lead = 0;
-        chunk_tc_plan(BH, NT, nsm, &n_state, &lead);
         // every CTA takes part in the leading rounds; afterwards only the factor CTAs take items
         const int n_intra = nsm - n_state;
         cudaLaunchConfig_t cfg = {};
@@ -1666,10 +1830,10 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
         attr[0].val.cooperative = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        return cudaLaunchKernelEx(&cfg, fused, maps, alpha, beta, ws, flags,
-                                  static_cast<const int4*>(ctab), h0, outb, hT, T_len, H, NT, BH,
-                                  n_state, lead, make_work_order(NT, BH, H, n_state, G), l2norm, rp,
-                                  pos_offset, scale);
+        return cudaLaunchKernelEx(&cfg, fused, maps, alpha, beta, ws, flags, pt, h0, outb, hT,
+                                  T_len, H, NT, BH, n_items, n_state, lead,
+                                  make_work_order(NT, BH, H, n_state, G), l2norm, rp, pos_offset,
+                                  scale);
     }
     // two kernels in sequence (profiling aid).  The factor kernel follows the flag reset in plain
     // stream order; the state kernel uses programmatic dependent launch (its set-up overlaps the
@@ -1679,12 +1843,11 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     if (stages & 1) {
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)(total < nsm ? total : nsm));
+        cfg.gridDim = dim3((unsigned)(n_items < nsm ? n_items : nsm));
         cfg.blockDim = dim3(512);
         cfg.dynamicSmemBytes = S_BYTES;
         cfg.stream = stream;
-        e = cudaLaunchKernelEx(&cfg, intra, maps, alpha, beta, ws, flags,
-                               static_cast<const int4*>(ctab), T_len, H, NT, BH,
+        e = cudaLaunchKernelEx(&cfg, intra, maps, alpha, beta, ws, flags, pt, T_len, H, NT, n_items,
                                make_work_order(NT, BH, H, BH, G), l2norm, rp, pos_offset);
         if (e != cudaSuccess) return e;
     }
@@ -1697,8 +1860,8 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         e = cudaLaunchKernelEx(&cfg, ckda_tc_state, maps, static_cast<const uint8_t*>(ws),
-                               static_cast<const int*>(flags), static_cast<const int4*>(ctab), h0,
-                               outb, hT, T_len, H, NT, BH, scale);
+                               static_cast<const int*>(flags), pt, h0, outb, hT, T_len, H, NT, BH,
+                               scale);
     }
     return e;
 }

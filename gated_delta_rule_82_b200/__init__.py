@@ -178,9 +178,10 @@ def fwd_chunked(q, k, v, alpha, beta, h0=None, *, chunk=64, l2norm=True, rope_th
     if hT is not None:
         _check(hT, "hT", dtype=torch.float32, shape=(B, H, dk, dv))
     code = _dtype_code(q)
-    need = workspace_bytes(B, T, H, dk, dv, chunk, q.dtype, path)
-    if need and workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if workspace is None:   # (a workspace given is checked against the need by the library)
+        need = workspace_bytes(B, T, H, dk, dv, chunk, q.dtype, path)
+        if need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = _load().ckda_fwd_chunked(
         _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(h0), _ptr(out), _ptr(hT),
@@ -256,9 +257,10 @@ def fwd_varlen(q, k, v, alpha, beta, cu_seqlens, h0=None, *, cu_seqlens_cpu=None
         hT = torch.empty((n, H, dk, dv), dtype=torch.float32, device=q.device)
     if hT is not None:
         _check(hT, "hT", dtype=torch.float32, shape=(n, H, dk, dv))
-    need = varlen_workspace_bytes(host, H, dk, dv, chunk, q.dtype, path)
-    if need and workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if workspace is None:   # (a workspace given is checked against the need by the library)
+        need = varlen_workspace_bytes(host, H, dk, dv, chunk, q.dtype, path)
+        if need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = _load().ckda_fwd_varlen(
         _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(h0), _ptr(out), _ptr(hT),

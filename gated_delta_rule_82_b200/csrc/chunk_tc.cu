@@ -557,14 +557,16 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
         issue_inputs(maps, sm, bar_in, fa.b, first.h, first.hk, fa.t0, gate_logits);
         issue_v(maps, sm, bar_v, fa.b, first.h, fa.t0);
     }
-    // where the current item's chunk lies; the next item's entry is read one item ahead
-    ChunkAt at_next = chunk_at(pt.ctab, wo.item(i0 >= 0 ? i0 : 0, pt.itab), T_len, NT, pos_offset);
+    // the current item and where its chunk lies; the next item's entries are read one item
+    // ahead, so that no table read sits at the top of an item
+    Item item_next = wo.item(i0 >= 0 ? i0 : 0, pt.itab);
+    ChunkAt at_next = chunk_at(pt.ctab, item_next, T_len, NT, pos_offset);
 
     // persistent loop over items; chunk-head ci = (batch*head) * NT + chunk
     uint32_t it = 0;
     int pending = -1;   // chunk-head whose images are stored but not yet flagged ready
     for (int k = 0, i = i0; i >= 0; i = seq.at(++k), ++it) {
-        const Item cur = wo.item(i, pt.itab);
+        const Item cur = item_next;
         const int ci = cur.bh * NT + cur.c;
         const ChunkAt at = at_next;
         const int t0 = at.t0;
@@ -572,6 +574,7 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
         const int inext = seq.at(k + 1);
         const bool has_next = inext >= 0;
         const Item nxt = wo.item(has_next ? inext : i, pt.itab);
+        item_next = nxt;
         at_next = chunk_at(pt.ctab, nxt, T_len, NT, pos_offset);
         uint8_t* wsc = ws + (size_t)ci * WS_CHUNK;
         const size_t row0 = ((size_t)at.b * T_len + t0) * H + cur.h;
@@ -1671,9 +1674,11 @@ size_t chunk_tc_workspace_bytes_packed(const int* cu_host, int n_seqs, int H) {
 // NT steps, or before its last chunk plus one step (and no chain starts before the leading rounds
 // are done).  The split minimises the later of that end and the end of the factor work (the
 // larger s and the smaller lead on ties).
-void chunk_tc_plan(int BH, int NT, int nsm, int* n_state, int* lead) {
+void chunk_tc_plan(int BH, int NT, long long n_items, int nsm, int* n_state, int* lead) {
     struct Entry {
-        int BH, NT, nsm, s, lead;
+        int BH, NT;
+        long long n_items;
+        int nsm, s, lead;
     };
     static std::mutex m;
     static Entry cache[16];
@@ -1681,14 +1686,17 @@ void chunk_tc_plan(int BH, int NT, int nsm, int* n_state, int* lead) {
     {
         std::lock_guard<std::mutex> g(m);
         for (int e = 0; e < n_cached; ++e)
-            if (cache[e].BH == BH && cache[e].NT == NT && cache[e].nsm == nsm) {
+            if (cache[e].BH == BH && cache[e].NT == NT && cache[e].n_items == n_items &&
+                cache[e].nsm == nsm) {
                 *n_state = cache[e].s;
                 *lead = cache[e].lead;
                 return;
             }
     }
     const double ti = 19000.0, tc = 2200.0, lag = 1.5;
-    const long long total = (long long)BH * NT;
+    // items: BH x NT, or fewer for packed sequences, whose lanes hold up to NT chunks each
+    const long long total = n_items;
+    const double per_unit = (double)n_items / BH;
     const int smax = BH < nsm - 1 ? BH : nsm - 1;
     const int lmax = (int)((total + nsm - 1) / nsm) < 8 ? (int)((total + nsm - 1) / nsm) : 8;
     int best_s = 1, best_l = 0;
@@ -1706,9 +1714,11 @@ void chunk_tc_plan(int BH, int NT, int nsm, int* n_state, int* lead) {
             double end = (double)l * ti;
             for (int g = 0; (long long)g * s < BH; ++g) {
                 const long long sg = BH - (long long)g * s < s ? BH - (long long)g * s : s;
-                const long long first = (long long)g * s * NT;
+                const long long first = (long long)((double)g * s * per_unit);
+                long long last_item = first + (long long)(NT - 1) * sg;
+                if (last_item > total - 1) last_item = total - 1;
                 const double t_first = (round_of(first) + lag) * ti;
-                const double t_last = (round_of(first + (long long)(NT - 1) * sg) + lag) * ti;
+                const double t_last = (round_of(last_item) + lag) * ti;
                 double e = end + NT * tc;
                 if (t_first + NT * tc > e) e = t_first + NT * tc;
                 if (t_last + tc > e) e = t_last + tc;
@@ -1725,7 +1735,7 @@ void chunk_tc_plan(int BH, int NT, int nsm, int* n_state, int* lead) {
     *n_state = best_s;
     *lead = best_l;
     std::lock_guard<std::mutex> g(m);
-    if (n_cached < 16) cache[n_cached++] = Entry{BH, NT, nsm, best_s, best_l};
+    if (n_cached < 16) cache[n_cached++] = Entry{BH, NT, n_items, nsm, best_s, best_l};
 }
 
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const void* alpha,
@@ -1766,7 +1776,7 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
         cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
     if (stages == 0 && nsm < 2) stages = 3;
     int n_state = 1, lead = 0;
-    if (stages == 0 && n_items > 0) chunk_tc_plan(BH, NT, nsm, &n_state, &lead);
+    if (stages == 0 && n_items > 0) chunk_tc_plan(BH, NT, n_items, nsm, &n_state, &lead);
     if (packed && stages != 2) {
         if (hT) {
             // empty sequences keep their initial state

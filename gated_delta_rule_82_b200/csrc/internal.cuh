@@ -38,9 +38,9 @@ size_t chunk_tc_workspace_bytes(int B, int T_len, int H);
 // chunks of packed sequences (sum of ceil(len / 64)) and their workspace
 long long packed_chunks(const int* cu_host, int n_seqs);
 size_t chunk_tc_workspace_bytes_packed(const int* cu_host, int n_seqs, int H);
-// split of the fused tensor-core launch for BH heads of NT chunks on nsm SMs: chain CTAs and
-// leading rounds of factor items taken by every CTA
-void chunk_tc_plan(int BH, int NT, int nsm, int* n_state, int* lead);
+// split of the fused tensor-core launch for BH heads of up to NT chunks (n_items chunk-heads in
+// all) on nsm SMs: chain CTAs and leading rounds of factor items taken by every CTA
+void chunk_tc_plan(int BH, int NT, long long n_items, int nsm, int* n_state, int* lead);
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const void* alpha,
                             const float* beta, const float* h0, void* out, float* hT, int B,
                             int T_len, int H, int G, int l2norm, const RopeParams& rp, float scale,

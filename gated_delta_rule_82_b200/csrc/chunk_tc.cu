@@ -54,6 +54,7 @@
 #include <cudaTypedefs.h>
 
 #include "fastdiv.h"
+#include "lanes.h"
 #include "internal.cuh"
 #include "tc_sm100.cuh"
 
@@ -1422,16 +1423,6 @@ ckda_tc_fused(const __grid_constant__ TcMaps maps, const void* __restrict__ alph
     kernel_tmem_free(tmem);
 }
 
-// How packed sequences are dealt to lanes (computed on the host from the offsets, passed by value).
-constexpr int kMaxLanes = 64;
-struct LanePlan {
-    int P;                      // lanes
-    int NTL;                    // chunks of the longest lane (the NT of the launch)
-    int total;                  // chunks of all sequences (per head)
-    int seq0[kMaxLanes + 1];    // first sequence of each lane; seq0[P] = number of sequences
-    int cbase[kMaxLanes + 1];   // chunks before each lane; cbase[P] = total
-};
-
 // Packed sequences: the tables and the ready flags of one call (one CTA of 1024 threads).
 //  1. chunk table: sequences are taken 1024 at a time; a block-wide scan of their chunk counts
 //     gives each one its first chunk in the global order, and lane l's chunk j is global chunk
@@ -1605,47 +1596,6 @@ long long packed_chunks(const int* cu_host, int n_seqs) {
     return nc;
 }
 
-// Lanes of about kLaneChunks chunks: the sequences in order, a lane closed once it holds at least
-// its share and the next sequence has chunks (whole sequences only: a sequence's chunks form one
-// chain).  Lanes stand in for batch rows, so that P x H chains can run where one chain per head
-// would walk through every sequence.
-constexpr int kLaneChunks = 32;
-static LanePlan plan_lanes(const int* cu_host, int n) {
-    LanePlan lp;
-    memset(&lp, 0, sizeof(lp));
-    const long long total = packed_chunks(cu_host, n);
-    int nonempty = 0;
-    for (int s = 0; s < n; ++s) nonempty += cu_host[s + 1] > cu_host[s];
-    int P = (int)((total + kLaneChunks / 2) / kLaneChunks);
-    P = P < 1 ? 1 : P;
-    P = P > kMaxLanes ? kMaxLanes : P;
-    P = P > nonempty ? (nonempty > 0 ? nonempty : 1) : P;
-    const long long share = (total + P - 1) / P;
-    int l = 0;
-    long long in_lane = 0, seen = 0;
-    lp.seq0[0] = 0;
-    lp.cbase[0] = 0;
-    for (int s = 0; s < n; ++s) {
-        const long long nch = (cu_host[s + 1] - cu_host[s] + kC - 1) / kC;
-        if (nch > 0 && in_lane >= share && l < P - 1) {
-            ++l;
-            lp.seq0[l] = s;
-            lp.cbase[l] = (int)seen;
-            in_lane = 0;
-        }
-        in_lane += nch;
-        seen += nch;
-    }
-    lp.P = l + 1;
-    lp.seq0[lp.P] = n;
-    lp.cbase[lp.P] = (int)total;
-    lp.total = (int)total;
-    lp.NTL = 0;
-    for (int i = 0; i < lp.P; ++i)
-        if (lp.cbase[i + 1] - lp.cbase[i] > lp.NTL) lp.NTL = lp.cbase[i + 1] - lp.cbase[i];
-    return lp;
-}
-
 struct PackedLayout {
     size_t images, ctab, lane_cnt, itab, bytes;   // byte offsets into the workspace, and its size
 };
@@ -1661,7 +1611,7 @@ static PackedLayout packed_layout(const LanePlan& lp, int H) {
 }
 
 size_t chunk_tc_workspace_bytes_packed(const int* cu_host, int n_seqs, int H) {
-    return packed_layout(plan_lanes(cu_host, n_seqs), H).bytes;
+    return packed_layout(plan_lanes(cu_host, n_seqs, kC), H).bytes;
 }
 
 // Split of the fused launch: `n_state` chain CTAs, and `lead` leading rounds of factor items that
@@ -1756,7 +1706,7 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
     // h0 at each one
     const bool packed = pk.cu != nullptr;
     LanePlan lp;
-    if (packed) lp = plan_lanes(pk.cu_host, pk.n);
+    if (packed) lp = plan_lanes(pk.cu_host, pk.n, kC);
     const int NT = packed ? lp.NTL : (T_len + kC - 1) / kC;
     const int BH = packed ? lp.P * H : B * H;
     const int Bm = packed ? 1 : B;

@@ -104,6 +104,13 @@ def test_tc_many_short_sequences():
     assert torch.equal(hT[torch.from_numpy(empty).cuda()].cpu(), torch.from_numpy(h0[empty]))
 
 
+def test_tc_uneven_lanes():
+    # 65 chunks per head: two lanes of whole sequences, 40 and 25 chunks, ragged ends
+    g, n, h0, cu = _case([1536, 1024, 700, 512, 300, 24], 2, 128, 128, "bf16", seed=535)
+    out, hT, o_ref, s_ref = _run(g, n, h0, cu, "tc", rope_theta=10000.0, rope_convention=1)
+    assert rel_err(out[0], o_ref) < TOL_BF16 and rel_err(hT, s_ref) < TOL_BF16
+
+
 @pytest.mark.parametrize("dk,dv,chunk", [(64, 64, 32), (32, 128, 16), (128, 128, 64)])
 def test_simt_mixed_lengths(dk, dv, chunk):
     g, n, h0, cu = _case(MIXED, 2, dk, dv, "f32", seed=540 + dk)

@@ -11,10 +11,12 @@ and output: the whole forward path).  Every rank runs its own replica on its own
 throughput (all ranks' tokens / the slowest rank's device time).
 
 The line also carries: the roofline of the one kernel a step launches (ckda_tc_fused, the whole
-forward; against the measured HBM bandwidth), the same work timed as two kernels in sequence, the decode step's HBM throughput on the batched-decode workload, the
-CKDA/KDA-range throughput ratio, an end-to-end figure through the C ABI with host buffers, SM
-clocks sampled during the timed region, and (rank 0, one GPU) the float64 CPU oracle's
-throughput on a bounded sample of the same workload.
+forward; against the measured HBM bandwidth), the same work timed as two kernels in sequence,
+the decode step's HBM throughput on the batched-decode workload, the standalone q/k prologue's
+HBM throughput (rotation then L2 norm at the layer shape), the CKDA/KDA-range throughput ratio,
+an end-to-end figure through the C ABI with host buffers, SM clocks sampled during the timed
+region, and (rank 0, one GPU) the float64 CPU oracle's throughput on bounded samples of the
+layer-shaped and long-context workloads, on all host cores and on one.
 
 --impl reference times that float64 CPU oracle (the only reference implementation there is)
 on the same workload, metric and unit.
@@ -191,21 +193,22 @@ def ncu_traffic(kernel):
 
 # ---- the reference arm: float64 CPU oracle ---------------------------------------------------
 
-def cpu_oracle_leg(steps, warmup, budget_s=20.0):
-    """Time the float64 oracle on a bounded sample of the headline workload.  The sample is the
-    first `heads` (batch, head) pairs of the workload over the full sequence length; tokens/s is
-    scaled to the workload's tokens (B*T tokens of H heads each)."""
+def cpu_oracle_leg(steps, warmup, budget_s=20.0, threads=None, heads=None, workload=None):
+    """Time the float64 oracle on a bounded sample of a forward workload (the headline's by
+    default).  The sample is the first `heads` (batch, head) pairs of the workload over its full
+    sequence length, on `threads` host threads (default: every core, and as many heads);
+    tokens/s is scaled to the workload's tokens (B*T tokens of H heads each)."""
     import numpy as np
     import oracle
     import synth
-    w = WORKLOAD
-    d = synth.fwd_inputs(w["B"], w["T"], w["H"], w["dk"], w["dv"], kind=w["kind"],
-                         dtype=w["dtype"], seed=4242)
+    w = workload or WORKLOAD
     cores = os.cpu_count() or 1
-    heads = max(1, min(w["H"], cores))
-    sub = {k: np.ascontiguousarray(d[k][:1, :, :heads]) for k in ("q", "k", "v", "alpha", "beta")}
-    run = lambda: oracle.fwd(sub["q"], sub["k"], sub["v"], sub["alpha"], sub["beta"], None,
-                             nthreads=cores, want_state=True)
+    threads = threads or cores
+    heads = max(1, min(w["H"], heads or threads))
+    d = synth.fwd_inputs(1, w["T"], heads, w["dk"], w["dv"], kind=w["kind"], dtype=w["dtype"],
+                         h0_std=w.get("h0_std", 0.0), seed=4242)
+    kw = dict(rope_theta=w.get("rope_theta", 0.0), nthreads=threads, want_state=True)
+    run = lambda: oracle.fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["h0"], **kw)
     for _ in range(warmup):
         run()
     times = []
@@ -219,9 +222,9 @@ def cpu_oracle_leg(steps, warmup, budget_s=20.0):
     sec = statistics.median(times)
     head_tokens = w["T"] * heads
     mtok = head_tokens / w["H"] / sec / 1e6
-    sample = (f"float64 oracle, batch 0 heads 0..{heads - 1} of the workload, T={w['T']}, "
-              f"{len(times)} timed runs, median {sec * 1e3:.1f} ms")
-    return mtok, cores, sample, len(times), sec
+    sample = (f"float64 oracle, {heads} head(s) of {w.get('name', 'the workload')}, T={w['T']}, "
+              f"{threads} thread(s), {len(times)} timed run(s), median {sec * 1e3:.1f} ms")
+    return mtok, threads, sample, len(times), sec
 
 
 def reference_main(args):
@@ -504,6 +507,30 @@ def main():
             "hbm_frac": round(htL * FWD_BYTES_PER_HT / (ms_long / 1e3) / 1e9 / hbm_peak, 4)}
         del L, wsL, outL, hL
 
+        # ---- standalone q/k prologue: rotation (theta 1e4, half-split) then the L2 norm --------
+        pq = [synth.torch_fwd_inputs(B, T, H, dk, dv, seed=6000 + 10 * rank + i, device=dev)
+              for i in range(N_ROTATE)]
+        pqo, pko = torch.empty_like(pq[0]["q"]), torch.empty_like(pq[0]["k"])
+        fnP = lambda i: ck.qk_prologue(pq[i % N_ROTATE]["q"], pq[i % N_ROTATE]["k"],
+                                       rope_theta=10000.0, q_out=pqo, k_out=pko)
+        for i in range(3):
+            fnP(i)
+        # a call's device time (~10 us) is below the host's per-call work: queue the calls behind
+        # a GPU spin so that the events time the device work back to back
+        ms_pro = event_time_ms(fnP, args.steps, stream,
+                               queue_ahead_ms=max(20.0, 0.5 * args.steps)) / args.steps
+        pro_bytes = 4 * B * T * H * dk * 2          # q and k read, q and k written (bf16)
+        pro_gbs = pro_bytes / (ms_pro / 1e3) / 1e9
+        extras["prologue"] = {
+            "workload": f"qk_prologue at the layer shape (B={B},T={T},H={H},dk={dk},bf16), "
+                        "RoPE theta 1e4 half-split, then L2 norm",
+            "us_per_call": round(ms_pro * 1e3, 2),
+            "roofline": {"bound": "hbm", "achieved": round(pro_gbs, 1), "peak": hbm_peak,
+                         "unit": "GB/s", "frac": round(pro_gbs / hbm_peak, 4),
+                         "traffic": ncu_traffic("qk_prologue_kernel"),
+                         "algorithmic_bytes_per_launch": pro_bytes}}
+        del pq, pqo, pko
+
         # ---- batched decode: 256 sequences x 32 heads, dk = dv = 128 ------------------------
         wd = synth.WORKLOADS["decode_bf16"]
         N, Hd, steps_d = wd["N"], wd["H"], args.decode_steps
@@ -569,6 +596,14 @@ def main():
         mtok, cores, sample, _, _ = cpu_oracle_leg(20, 1, budget_s=20.0)
         cpu = {"value": round(mtok, 6), "unit": "Mtok/s", "cores": cores, "kind": "oracle",
                "sample": sample}
+        # the same sample on one host thread (one head), and the long-context workload (one
+        # head per core, T = 65536, RoPE, h0) on every core
+        m1, c1, s1, _, _ = cpu_oracle_leg(5, 0, budget_s=10.0, threads=1, heads=1)
+        cpu["one_core"] = {"value": round(m1, 6), "unit": "Mtok/s", "cores": c1, "sample": s1}
+        wl = dict(synth.WORKLOADS["long_rope_bf16"], name="long_rope_bf16")
+        mL, cL, sL, _, _ = cpu_oracle_leg(1, 0, budget_s=1.0, workload=wl)
+        cpu["long_context"] = {"value": round(mL, 6), "unit": "Mtok/s", "cores": cL,
+                               "sample": sL}
 
     if world > 1:
         dist.barrier()

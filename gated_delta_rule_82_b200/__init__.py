@@ -15,7 +15,7 @@ import torch
 
 __all__ = ["CkdaError", "library_path", "abi_version", "qk_prologue", "workspace_bytes",
            "fwd_chunked", "varlen_workspace_bytes", "fwd_varlen", "decode_step", "selftest_umma",
-           "PATHS"]
+           "last_device_status", "set_wait_limit_ns", "PATHS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libckda.so")
@@ -72,6 +72,10 @@ def _load():
     lib.ckda_decode_step.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, _Flags, I, P]
     lib.ckda_selftest_umma.restype = I
     lib.ckda_selftest_umma.argtypes = [P, P, P, I, I, I, I, P]
+    lib.ckda_last_device_status.restype = I
+    lib.ckda_last_device_status.argtypes = [P, ctypes.POINTER(I)]
+    lib.ckda_set_wait_limit_ns.restype = I
+    lib.ckda_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
     _lib = lib
     return lib
 
@@ -302,6 +306,23 @@ def decode_step(q, k, v, alpha, beta, state, pos=None, *, l2norm=True, rope_thet
         _stream(q.device))
     _raise("ckda_decode_step", st)
     return out
+
+
+def last_device_status(device=None) -> int:
+    """Wait for the current stream, then read and clear the library's device status word:
+    0 = no failure recorded; 1 / 2 = a bounded wait of the tensor-core forward ran out (factor
+    work / state pass); 3 = packed-sequence offsets on the device disagreed with the host copy."""
+    code = ctypes.c_int(0)
+    st = _load().ckda_last_device_status(_stream(device), ctypes.byref(code))
+    if st not in (0, 8):   # CKDA_OK, CKDA_ERR_DEVICE_STATUS
+        raise CkdaError("ckda_last_device_status", st)
+    return int(code.value)
+
+
+def set_wait_limit_ns(ns: int = 0) -> None:
+    """Upper bound of one wait of the tensor-core forward's state pass on the current device
+    (0 restores the default of 4 s).  A diagnostic: a short limit makes a wait give up sooner."""
+    _raise("ckda_set_wait_limit_ns", _load().ckda_set_wait_limit_ns(int(ns)))
 
 
 def selftest_umma(A, B, b_mn_major=False, a_tmem=False):

@@ -1,6 +1,6 @@
 """Build the CKDA CUDA library (libckda.so) in-tree with nvcc for sm_100a.
 
-    python -m gated_delta_rule_82_b200.build [--force] [--debug]
+    python -m gated_delta_rule_82_b200.build [--force] [-v]
 
 The shared library is written next to this file and loaded by the package with ctypes.
 """
@@ -21,6 +21,8 @@ LIB = os.path.join(HERE, "libckda.so")
 BUILD_DIR = os.path.join(HERE, "_build")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-fvisibility=hidden",
+         "--expt-relaxed-constexpr"]
 
 
 def nvcc() -> str:
@@ -34,12 +36,12 @@ def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _digest(debug: bool) -> str:
+def _digest() -> str:
     """Hash of every source and header plus the flags: a copy of the tree keeps it valid."""
     import hashlib
-    h = hashlib.sha256(f"debug={int(debug)};arch={ARCH}".encode())
+    h = hashlib.sha256(f"arch={ARCH};flags={FLAGS}".encode())
     deps = sorted(sources() + glob.glob(os.path.join(CSRC, "*.cuh")) +
-                  glob.glob(os.path.join(INCLUDE, "*.h")))
+                  glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(INCLUDE, "*.h")))
     for p in deps:
         h.update(os.path.basename(p).encode())
         with open(p, "rb") as f:
@@ -47,23 +49,20 @@ def _digest(debug: bool) -> str:
     return h.hexdigest()
 
 
-def _stale(debug: bool = False) -> bool:
+def _stale() -> bool:
     stamp = LIB + ".sha256"
     if not os.path.exists(LIB) or not os.path.exists(stamp):
         return True
     with open(stamp) as f:
-        return f.read().strip() != _digest(debug)
+        return f.read().strip() != _digest()
 
 
-def build(force: bool = False, debug: bool = False, verbose: bool = False) -> str:
+def build(force: bool = False, verbose: bool = False) -> str:
     """Compile every .cu under csrc/ into libckda.so (sm_100a).  Returns the library path."""
-    if not force and not _stale(debug):
+    if not force and not _stale():
         return LIB
     os.makedirs(BUILD_DIR, exist_ok=True)
-    flags = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-fvisibility=hidden",
-                    "-I", INCLUDE, "-I", CSRC, "--expt-relaxed-constexpr"]
-    if debug:
-        flags += ["-DCKDA_DEBUG=1"]
+    flags = ARCH + FLAGS + ["-I", INCLUDE, "-I", CSRC]
     if verbose:
         flags += ["-Xptxas", "-v"]
     objs = []
@@ -88,14 +87,13 @@ def build(force: bool = False, debug: bool = False, verbose: bool = False) -> st
     subprocess.run([nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-Xcompiler", "-fPIC"], check=True)
     os.replace(tmp, LIB)
     with open(LIB + ".sha256", "w") as f:
-        f.write(_digest(debug))
+        f.write(_digest())
     return LIB
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
-    ap.add_argument("--debug", action="store_true")
     ap.add_argument("-v", "--verbose", action="store_true")
     a = ap.parse_args()
-    print(build(force=a.force, debug=a.debug, verbose=a.verbose))
+    print(build(force=a.force, verbose=a.verbose))

@@ -74,8 +74,20 @@ const char* ckda_strerror(ckda_status s) {
         case CKDA_ERR_WORKSPACE: return "workspace missing or too small";
         case CKDA_ERR_CUDA: return "a CUDA runtime call failed";
         case CKDA_ERR_ARG: return "invalid argument";
+        case CKDA_ERR_DEVICE_STATUS: return "a kernel recorded a failure on the device";
     }
     return "unknown status";
+}
+
+ckda_status ckda_last_device_status(ckda_stream_t stream, int* code) {
+    int v = 0;
+    if (device_status_take((cudaStream_t)stream, &v) != cudaSuccess) return CKDA_ERR_CUDA;
+    if (code) *code = v;
+    return v == 0 ? CKDA_OK : CKDA_ERR_DEVICE_STATUS;
+}
+
+ckda_status ckda_set_wait_limit_ns(unsigned long long ns) {
+    return from_cuda(set_wait_limit_ns(ns));
 }
 
 ckda_status ckda_qk_prologue(const void* q, const void* k, void* q_out, void* k_out, int B, int T,

@@ -165,7 +165,18 @@ __device__ __forceinline__ float select_lane(const float* v, int lane) {
     return (lane & 16) ? d[1] : d[0];
 }
 
-__device__ int g_tc_error;  // nonzero after a bounded wait ran out (diagnostic)
+// Device status word of the forward kernels: 0, or the first failure recorded since the host last
+// read it (kStatus* below).  Read and cleared by ckda_last_device_status.
+__device__ int g_tc_error;
+// Upper bound (ns) of one wait of the state role (a ready flag, or an mbarrier that may
+// legitimately wait for a whole head group to be produced); settable from the host.
+constexpr unsigned long long kDefaultWaitNs = 4000000000ull;   // 4 s
+__device__ unsigned long long g_wait_limit_ns = kDefaultWaitNs;
+// Codes of the status word (the first failure since the last read is kept).
+constexpr int kStatusFactorWait = 1;     // a wait of the factor role ran out
+constexpr int kStatusStateWait = 2;      // a wait of the state role ran out
+constexpr int kStatusPackedOffsets = 3;  // device cu_seqlens disagree with the host copy
+__device__ __forceinline__ void record_status(int code) { atomicCAS(&g_tc_error, 0, code); }
 
 // Tensor maps of one forward call: q, k, v (bf16), alpha (fp32, or bf16 logits) and out (bf16)
 // as 4-D arrays {channel, head, token, batch}; boxes of 64 tokens of one (batch, head).
@@ -469,9 +480,9 @@ __device__ __forceinline__ uint64_t global_ns() {
     return t;
 }
 // Waits of the state role can last as long as the factor role takes to produce a head group
-// (milliseconds on long sequences), so they are bounded by time rather than by a poll count.
-constexpr uint64_t kLongWaitNs = 4000000000ull;   // 4 s
-__device__ __forceinline__ bool flag_wait(const int* flag, volatile int* abort) {
+// (milliseconds on long sequences), so they are bounded by time (g_wait_limit_ns, read once per
+// kernel into `limit`) rather than by a poll count.
+__device__ __forceinline__ bool flag_wait(const int* flag, volatile int* abort, uint64_t limit) {
     if (ld_acquire(flag) != 0) {
         asm volatile("fence.proxy.async.global;" ::: "memory");
         return true;
@@ -483,17 +494,18 @@ __device__ __forceinline__ bool flag_wait(const int* flag, volatile int* abort) 
             return true;
         }
         if (*abort) return false;
-        if (global_ns() - t0 > kLongWaitNs) { *abort = 1; return false; }
+        if (global_ns() - t0 > limit) { *abort = 1; return false; }
         __nanosleep(256);
     }
 }
-__device__ __forceinline__ bool mbar_wait_long(uint64_t* bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait_long(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                               uint64_t limit) {
     if (tc::mbar_try_wait(bar, parity)) return true;   // the common case reads no timer
     const uint64_t t0 = global_ns();
     for (uint32_t i = 0;; ++i) {
         if (tc::mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if ((i & 255) == 255 && global_ns() - t0 > kLongWaitNs) { *abort = 1; return false; }
+        if ((i & 255) == 255 && global_ns() - t0 > limit) { *abort = 1; return false; }
     }
 }
 
@@ -997,7 +1009,7 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
     }
     tc::tc_fence_before();
     __syncthreads();
-    if (*abort_flag && tid == 0) atomicExch(&g_tc_error, 1);
+    if (*abort_flag && tid == 0) record_status(kStatusFactorWait);
     // the CTA may go on to another role over this shared memory, whose copies (async proxy) must
     // come after this role's plain writes
     tc::fence_proxy_async_smem();
@@ -1099,8 +1111,9 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
     // a launch after the factor kernel waits for it here (no effect otherwise)
     tc::grid_dependency_wait();
     tc::grid_launch_dependents();
+    const uint64_t limit = g_wait_limit_ns;
     auto wait = [&](uint64_t* bar, uint32_t parity) {
-        return __all_sync(0xffffffffu, mbar_wait_long(bar, parity, abort_flag));
+        return __all_sync(0xffffffffu, mbar_wait_long(bar, parity, abort_flag, limit));
     };
     // items advance as (head k, chunk c) counters, so no step divides by NT
 
@@ -1247,7 +1260,7 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
             int nc = U > 0 ? units_chunks(head0) : 0;
             for (int c = 0, bh = head0; issued < U; ++issued) {
                 const int st = issued & 1;
-                if (issued >= 2 && !mbar_wait_long(&emptyb[st], ((issued >> 1) - 1) & 1, abort_flag))
+                if (issued >= 2 && !mbar_wait_long(&emptyb[st], ((issued >> 1) - 1) & 1, abort_flag, limit))
                     break;
                 const size_t ci = (size_t)bh * NT + c;
                 if (++c == nc) {
@@ -1255,7 +1268,7 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
                     bh += hstride;
                     if (issued + 1 < U) nc = units_chunks(bh);
                 }
-                if (!flag_wait(flags + ci, abort_flag)) break;
+                if (!flag_wait(flags + ci, abort_flag, limit)) break;
                 tc::mbar_arrive_expect_tx(&fullb[st], bytes);
                 tc::bulk_g2s(stage0 + st * bytes, ws + ci * WS_CHUNK + (chain ? WS_AC : WS_UT), bytes,
                              &fullb[st]);
@@ -1280,7 +1293,7 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
             const int ob = u & 3;
             // the chunk's first token and length (packed sequences: from the chunk table)
             const int4 e = ctab ? otab[c] : make_int4(c * kC, kC, 0, 0);
-            const bool ok = mbar_wait_long(&mma_o[ob], (u >> 2) & 1, abort_flag);
+            const bool ok = mbar_wait_long(&mma_o[ob], (u >> 2) & 1, abort_flag, limit);
             // the previous item's tensor store must be done reading the staging tile
             if (leader) tc::bulk_wait_read<0>();
             __syncwarp();
@@ -1337,7 +1350,7 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
     }
     tc::tc_fence_before();
     __syncthreads();
-    if (*abort_flag && tid == 0) atomicExch(&g_tc_error, 2);
+    if (*abort_flag && tid == 0) record_status(kStatusStateWait);
 }
 
 __device__ __forceinline__ uint8_t* aligned_smem(uint8_t* raw) {
@@ -1505,7 +1518,7 @@ ckda_varlen_prep(const int* __restrict__ cu, int n_seqs, int T_total, const Lane
     __syncthreads();
     if (s_bad) {
         for (int x = tid; x < lp.P * lp.NTL; x += kPrepThreads) ctab[x] = make_int4(0, 0, 0, 0);
-        if (tid == 0) atomicExch(&g_tc_error, 3);
+        if (tid == 0) record_status(kStatusPackedOffsets);
     }
     // 2. item table
     const int BH = lp.P * H;
@@ -1824,6 +1837,28 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
                                scale);
     }
     return e;
+}
+
+// Read the status word on the current device (after `stream` has finished) and clear it.
+cudaError_t device_status_take(cudaStream_t stream, int* code) {
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_tc_error, sizeof(int), 0,
+                                              cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e == cudaSuccess && v != 0) {
+        static const int zero = 0;
+        e = cudaMemcpyToSymbolAsync(g_tc_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice,
+                                    stream);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    }
+    *code = v;
+    return e;
+}
+
+// Bound of one wait of the state role on the current device (0: the default).
+cudaError_t set_wait_limit_ns(unsigned long long ns) {
+    const unsigned long long v = ns ? ns : kDefaultWaitNs;
+    return cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v));
 }
 
 }  // namespace ckda

@@ -47,6 +47,12 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
                             long long pos_offset, int gate_logits, void* workspace, int stages,
                             const PackedSeqs& pk, cudaStream_t stream);
 
+// The forward kernels' device status word on the current device: read once `stream` has
+// finished, then cleared (0 = no failure recorded).
+cudaError_t device_status_take(cudaStream_t stream, int* code);
+// Upper bound of one wait of the fused forward's state role on the current device (0: default).
+cudaError_t set_wait_limit_ns(unsigned long long ns);
+
 cudaError_t launch_umma_selftest(const void* A, const void* B, float* D, int M, int N, int K,
                                  int mode, cudaStream_t stream);
 

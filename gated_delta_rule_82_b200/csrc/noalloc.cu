@@ -13,7 +13,8 @@
 // caches it.  Every call shares the array: calls whose kernels overlap on the GPU (different
 // streams, or host threads racing) corrupt each other's scratch.  No byte of the scratch has to
 // start at zero: every call clears the chunk-heads' ready flags itself, and the chunk-factor work
-// writes every other byte the state pass later reads.
+// writes every other byte the state pass later reads.  That holds for the whole forward (stages 0
+// and 3); the profiling stages 1 and 2, which split it across calls, are refused.
 #include <mutex>
 
 #include "internal.cuh"
@@ -44,6 +45,8 @@ extern "C" CKDA_API ckda_status ckda_fwd_chunked_noalloc(
     const void* q, const void* k, const void* v, const void* alpha, const float* beta,
     const float* h0, void* out, float* hT, int B, int T, int H, int dk, int dv, int chunk,
     ckda_flags flags, ckda_dtype dtype, long long pos_offset, ckda_stream_t stream) {
+    // the profiling stages 1 and 2 would leave or read images of the shared array across calls
+    if (flags.stages != 0 && flags.stages != 3) return CKDA_ERR_ARG;
     const size_t need = ckda_fwd_workspace_bytes(B, T, H, dk, dv, chunk, dtype, flags.path);
     if (need != (size_t)-1 && need > (size_t)CKDA_NOALLOC_MAX_WORKSPACE) return CKDA_ERR_WORKSPACE;
     void* scratch = nullptr;

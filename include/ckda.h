@@ -32,6 +32,11 @@
  *    values, or (flags.gate_logits = 1) logits of the element type `dtype`.
  *  - Supported sizes: dk, dv in {16, 32, 64, 128}; chunk in {16, 32, 64}; any T >= 1 (a
  *    partial last chunk is handled exactly).  B*H, N*H >= 1.
+ *  - Failures the kernels detect on the device (a bounded wait of the tensor-core forward that
+ *    ran out, packed-sequence offsets whose device copy disagrees with the host copy) are
+ *    recorded in a per-device status word instead of faulting: the kernel stops its work, leaves
+ *    the outputs unspecified and returns, so the context stays usable.  The call itself has
+ *    already returned CKDA_OK by then; ckda_last_device_status reports the failure.
  */
 #ifndef CKDA_H
 #define CKDA_H
@@ -42,7 +47,7 @@
 extern "C" {
 #endif
 
-#define CKDA_ABI_VERSION 4
+#define CKDA_ABI_VERSION 5
 
 #if defined(__GNUC__)
 #define CKDA_API __attribute__((visibility("default")))
@@ -61,7 +66,9 @@ typedef enum {
     CKDA_ERR_ALIGN = 4,       /* an array pointer is not 16-byte aligned */
     CKDA_ERR_WORKSPACE = 5,   /* workspace NULL or smaller than ckda_fwd_workspace_bytes() */
     CKDA_ERR_CUDA = 6,        /* a CUDA runtime call failed while configuring or launching */
-    CKDA_ERR_ARG = 7          /* any other invalid argument (flags, overlapping buffers) */
+    CKDA_ERR_ARG = 7,         /* any other invalid argument (flags, overlapping buffers) */
+    CKDA_ERR_DEVICE_STATUS = 8 /* a kernel recorded a failure in the device status word
+                                  (ckda_last_device_status) */
 } ckda_status;
 
 typedef enum {
@@ -115,6 +122,30 @@ CKDA_API int ckda_abi_version(void);
 
 /* Human-readable text for a status code (static storage, never NULL). */
 CKDA_API const char* ckda_strerror(ckda_status status);
+
+/*
+ * Device status word of the current device: waits until `stream` has finished its work, then
+ * reads the word and clears it.  The word is shared by every stream and call on the device and
+ * keeps the first failure recorded since the last read.  *code (may be NULL) receives it:
+ *   0  no failure recorded
+ *   1  a wait of the tensor-core forward's chunk-factor work ran out (a poll limit)
+ *   2  a wait of the tensor-core forward's state pass ran out (ckda_set_wait_limit_ns)
+ *   3  ckda_fwd_varlen: the device copy of cu_seqlens disagrees with the host copy
+ * Returns CKDA_OK for 0, CKDA_ERR_DEVICE_STATUS otherwise, CKDA_ERR_CUDA when the read fails.
+ * After a recorded failure the outputs of the failing call are unspecified.  There is no
+ * counterpart on the pages: it reports the bounded waits of this library's own kernels.
+ */
+CKDA_API ckda_status ckda_last_device_status(ckda_stream_t stream, int* code);
+
+/*
+ * Upper bound, in nanoseconds, of any single wait of the tensor-core forward's state pass on the
+ * current device (a wait for a chunk's factors to be produced, or for a tensor-core product).
+ * A wait that reaches it stops the kernel with status 2.  ns = 0 restores the default, 4 s,
+ * which no correct run comes near (the state pass waits at most for one head group's factors).
+ * Synchronous; affects calls enqueued afterwards.  A diagnostic, with no counterpart on the
+ * pages: a short limit lets a test make a wait run out on purpose.
+ */
+CKDA_API ckda_status ckda_set_wait_limit_ns(unsigned long long ns);
 
 /*
  * Prologue alone: q_out = L2(rope(q)), k_out = L2(rope(k)) per head, with the rotation at
@@ -248,6 +279,9 @@ CKDA_API ckda_status ckda_selftest_umma(const void* A, const void* B, float* D, 
  *   Sharing: every call uses the same array, which keeps the last call's contents (no part of it
  *          needs to start at zero).  Calls whose work overlaps on the GPU race on it: issue them
  *          on one stream, or otherwise order them.
+ *   flags.stages: 0 or 3 only (each of those clears the array's ready flags itself); the
+ *          profiling stages 1 and 2 are refused with CKDA_ERR_ARG, since a stage-2 call would
+ *          read whatever an earlier call, of any shape, left in the shared array.
  */
 #define CKDA_NOALLOC_MAX_WORKSPACE (16u << 20)
 

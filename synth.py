@@ -13,6 +13,10 @@ Definition": alpha in [-1, 1]^dk, beta in [0, 2]):
   ``tiny``     q, k, v ~ N(0,1); alpha = s*m, s = +-1 (p = 1/2), m ~ U[0.05, 1]; beta ~ U[0, 2]
   ``ckda``     alpha = s*exp(-softplus(z)), z ~ N(0,1), |alpha| >= 1e-3; beta = 2*sigmoid(N(0,1))
   ``kda``      alpha = exp(-softplus(z)) in (0, 1]; beta = sigmoid(N(0,1)) in [0, 1]
+  ``longmem``  alpha = s*m, s = +-1 (p = 1/2), m ~ U[0.95, 1]; beta ~ U[1.5, 2] (slow decay and
+               strong reflections: the state keeps a memory over many chunks)
+  ``orth``     alpha = +-1 (p = 1/2); beta = 2 (every transition orthogonal: the rotation regime
+               of the paper summary's Theorem 1, nothing decays)
 
 Gate logits (the optional input form whose activations 2 sigmoid(a) - 1 and 2 sigmoid(b) the
 library and the oracle form themselves): a = s * (1 + 2|z|), s = +-1 (p = 1/2), z ~ N(0,1),
@@ -69,6 +73,13 @@ def gates(kind: str, shape_alpha, shape_beta, seed: int):
         z = ga.standard_normal(size=shape_alpha)
         alpha = np.exp(-_softplus(z))
         beta = _sigmoid(gb.standard_normal(size=shape_beta))
+    elif kind == "longmem":
+        s = np.where(ga.random(size=shape_alpha) < 0.5, -1.0, 1.0)
+        alpha = s * ga.uniform(0.95, 1.0, size=shape_alpha)
+        beta = gb.uniform(1.5, 2.0, size=shape_beta)
+    elif kind == "orth":
+        alpha = np.where(ga.random(size=shape_alpha) < 0.5, -1.0, 1.0)
+        beta = np.full(shape_beta, 2.0)
     else:
         raise ValueError(f"unknown gate recipe {kind!r}")
     return alpha.astype(np.float32), beta.astype(np.float32)

@@ -13,7 +13,7 @@ from gated_delta_rule_82_b200 import build as ckbuild
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "ckda.h")
 
-OK, NULL, SHAPE, UNSUP, ALIGN, WORKSPACE, CUDA, ARG = range(8)
+OK, NULL, SHAPE, UNSUP, ALIGN, WORKSPACE, CUDA, ARG, DEVICE_STATUS = range(9)
 P = 0x10000  # a 16-byte-aligned fake address; never dereferenced (calls fail validation first)
 
 
@@ -33,7 +33,8 @@ def test_header_declares_the_boundary():
     names = declared_functions()
     for want in ("ckda_fwd_chunked", "ckda_decode_step", "ckda_fwd_workspace_bytes",
                  "ckda_qk_prologue", "ckda_strerror", "ckda_abi_version", "ckda_fwd_varlen",
-                 "ckda_fwd_varlen_workspace_bytes"):
+                 "ckda_fwd_varlen_workspace_bytes", "ckda_last_device_status",
+                 "ckda_set_wait_limit_ns", "ckda_fwd_chunked_noalloc"):
         assert want in names
 
 
@@ -51,8 +52,8 @@ def test_only_declared_symbols_are_exported(lib):
 
 
 def test_version_and_strerror(lib):
-    assert ck.abi_version() == 4
-    for s in range(8):
+    assert ck.abi_version() == 5
+    for s in range(9):
         assert lib.ckda_strerror(s)
     assert lib.ckda_strerror(99) == b"unknown status"
 
@@ -201,3 +202,18 @@ def test_binding_refuses_cpu_tensors():
     x = torch.zeros(1, 4, 1, 16)
     with pytest.raises(ValueError, match="CUDA"):
         ck.qk_prologue(x, x)
+
+
+@pytest.mark.parametrize("stages", [1, 2, 4, -1])
+def test_noalloc_refuses_split_stages(lib, stages):
+    """The library-owned scratch of ckda_fwd_chunked_noalloc is shared by every call, so the
+    profiling stages that split one forward across two calls (and invalid stages) are refused
+    before anything else is looked at."""
+    f = lib.ckda_fwd_chunked_noalloc
+    f.restype = ctypes.c_int
+    P_, I_ = ctypes.c_void_p, ctypes.c_int
+    f.argtypes = [P_] * 8 + [I_] * 6 + [ck._Flags, I_, ctypes.c_longlong, P_]
+    c = ctypes.c_void_p
+    st = f(c(P), c(2 * P), c(3 * P), c(4 * P), c(5 * P), None, c(6 * P), None, 1, 64, 1, 128,
+           128, 64, flags(path=2, stages=stages), 1, 0, None)
+    assert st == ARG

@@ -139,6 +139,41 @@ def test_decode_batched_full_shape():
     assert es < TOL_F32
 
 
+def test_decode_batched_all_steps():
+    """The batched-decode workload in full: 256 sequences x 32 heads, dk = dv = 128, 1024
+    sequential steps in place on the caller's fp32 state (512 MiB).  Sequences 0-7 (256 chains of
+    all 32 heads) carry seeded inputs that the oracle replays token by token -- T decode steps
+    are the forward over T tokens, a pinned identity of the oracle -- and every step's output and
+    the final state of those chains are compared.  The other 248 sequences carry random inputs
+    that keep every launch at the full shape."""
+    wd = synth.WORKLOADS["decode_bf16"]
+    N, H, steps, n_chk = wd["N"], wd["H"], wd["steps"], 8
+    d = synth.fwd_inputs(n_chk, steps, H, 128, 128, kind=wd["kind"], dtype="bf16", h0_std=0.05,
+                         seed=51)
+    o_ref, s_ref = oracle.fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["h0"])
+    step_major = lambda x: torch.from_numpy(np.ascontiguousarray(np.swapaxes(x, 0, 1)))
+    chk = {n: step_major(d[n + "_bits"]).view(torch.bfloat16).cuda() for n in ("q", "k", "v")}
+    chk["alpha"] = step_major(d["alpha"]).cuda()
+    chk["beta"] = step_major(d["beta"]).cuda()
+    pool = synth.torch_decode_inputs(4, N, H, 128, 128, kind=wd["kind"], seed=52)
+    state = 0.02 * torch.randn((N, H, 128, 128), device="cuda")
+    state[:n_chk] = dev_f32(d["h0"])
+    outs = torch.empty((steps, n_chk, H, 128), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((N, H, 128), dtype=torch.bfloat16, device="cuda")
+    for t in range(steps):
+        x = {n: pool[n][t % 4] for n in ("q", "k", "v", "alpha", "beta")}
+        for n in x:
+            x[n][:n_chk] = chk[n][t]
+        ck.decode_step(x["q"], x["k"], x["v"], x["alpha"], x["beta"], state, out=out)
+        outs[t] = out[:n_chk]
+    torch.cuda.synchronize()
+    eo = rel_err(outs.permute(1, 0, 2, 3), o_ref)
+    es = rel_err(state[:n_chk], s_ref)
+    print(f"1024 decode steps: out {eo:.3e} state {es:.3e}")
+    assert eo < TOL_BF16
+    assert es < TOL_F32
+
+
 # ---- chunked forward, CUDA-core path --------------------------------------------------------
 
 def _fwd_check(B, T, H, dk, dv, chunk, *, dtype, kind="ckda", rope=(0.0, 0), pos=0, h0_std=0.0,

@@ -73,20 +73,22 @@ def test_tc_layer_shape_kda():
     check(w["B"], w["T"], w["H"], kind=w["kind"], seed=102)
 
 
-def test_tc_long_rope_sampled_heads():
-    """The long-context workload (T=65536, H=16, RoPE theta 10000 half-split, h0 ~ N(0, 0.02)),
-    run in full on the GPU; the oracle recomputes two of the heads end to end."""
+def test_tc_long_rope_all_heads():
+    """The long-context workload (B=1, T=65536, H=16, RoPE theta 10000 half-split, h0 ~ N(0,
+    0.02)), run in full on the GPU and compared with the oracle element by element on every head:
+    all 65536 x 16 outputs and the 16 final states."""
     w = synth.WORKLOADS["long_rope_bf16"]
-    d, g = fwd_case(w["B"], w["T"], w["H"], 128, 128, kind=w["kind"], dtype="bf16",
-                    h0_std=w["h0_std"], seed=103)
-    out, hT = run_tc(g, rope_theta=w["rope_theta"], rope_convention=0)
-    heads = [0, 11]
-    sub = {key: d[key][:, :, heads] for key in ("q", "k", "v", "alpha", "beta")}
-    sub["h0"] = d["h0"][:, heads]
-    o_ref, s_ref = oracle.fwd(sub["q"], sub["k"], sub["v"], sub["alpha"], sub["beta"], sub["h0"],
-                              rope_theta=w["rope_theta"], rope_convention=0)
-    assert rel_err(out[:, :, heads], o_ref) < TOL
-    assert rel_err(hT[:, heads], s_ref) < TOL
+    check(w["B"], w["T"], w["H"], kind=w["kind"], h0_std=w["h0_std"],
+          rope=(w["rope_theta"], 0), seed=103)
+
+
+def test_tc_layer_shape_long_memory():
+    """The layer shape (B=2, T=2048, H=16) with slowly decaying signed gates (|alpha| in [0.95,
+    1], random signs) and strong reflections (beta in [1.5, 2]) from a nonzero h0: the state
+    carries information across many chunks, so the inter-chunk chain's precision shows."""
+    w = synth.WORKLOADS["layer_ckda_bf16"]
+    eo, es = check(w["B"], w["T"], w["H"], kind="longmem", h0_std=0.05, seed=41)
+    print(f"long-memory gates, layer shape: out {eo:.3e} hT {es:.3e}")
 
 
 def test_tc_matches_simt_path():
@@ -115,24 +117,35 @@ def test_tc_exact_zero_gates_take_the_exact_diagonal_path():
 
 
 def test_tc_orthogonal_chain():
-    """|alpha| = 1 and beta = 2 everywhere (every transition orthogonal, Theorem 1): with v = 0
-    the state norm is preserved across 2048 tokens and the output still matches the oracle."""
-    d, g = fwd_case(1, 2048, 2, 128, 128, kind="ckda", dtype="bf16", h0_std=0.05, seed=17)
-    rng = np.random.default_rng(0)
-    a = rng.choice([-1.0, 1.0], size=d["alpha"].shape).astype(np.float32)
-    b = np.full(d["beta"].shape, 2.0, np.float32)
-    d["alpha"], d["beta"] = a, b
+    """|alpha| = 1 and beta = 2 everywhere (every transition orthogonal, the summary's Theorem 1),
+    v = 0, 2048 tokens: nothing decays, so every rounding of every chunk survives to the end.
+
+    The tensor-core path rounds its chunk-factor operands to bf16; the rounding model
+    (precision_model.py, test_precision_model.py) places those roundings in float64 on these very
+    inputs and gives the floor any bf16-operand evaluation reaches here (about 3e-2 at 32 chunks,
+    each of seven operand roundings contributing about 1e-2).  The GPU path must stay within 1.5x
+    of that floor, and keep each head's state norm.  The fp32 CUDA-core path (which rounds only
+    its output) holds the same chain to the 1e-2 bound."""
+    from precision_model import chunked
+    d, g = fwd_case(1, 2048, 2, 128, 128, kind="orth", dtype="bf16", h0_std=0.05, seed=17)
     d["v"] = np.zeros_like(d["v"])
     d["v_bits"] = np.zeros_like(d["v_bits"])
-    g["alpha"], g["beta"] = dev_f32(a), dev_f32(b)
     g["v"] = torch.zeros_like(g["v"])
     out, hT = run_tc(g)
     o_ref, s_ref = oracle_fwd(d)
+    o_mod, s_mod = chunked(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["h0"])
+    floor_o, floor_s = rel_err(o_mod, o_ref), rel_err(s_mod, s_ref)
+    eo, es = rel_err(out, o_ref), rel_err(hT, s_ref)
+    print(f"orthogonal chain: tensor-core out {eo:.3e} hT {es:.3e}; "
+          f"bf16-operand floor out {floor_o:.3e} hT {floor_s:.3e}")
     n0 = np.linalg.norm(d["h0"].reshape(2, -1), axis=1)
     n1 = np.linalg.norm(hT.cpu().numpy().reshape(2, -1), axis=1)
     assert np.allclose(n0, n1, rtol=2e-2)
-    assert rel_err(hT, s_ref) < 5e-2  # orthogonal chains keep every rounding error alive
-    assert rel_err(out, o_ref) < 5e-2
+    assert eo < 1.5 * floor_o and es < 1.5 * floor_s
+    o2, s2 = ck.fwd_chunked(g["q"], g["k"], g["v"], g["alpha"], g["beta"], g["h0"], chunk=64,
+                            path="simt")
+    torch.cuda.synchronize()
+    assert rel_err(o2, o_ref) < TOL and rel_err(s2, s_ref) < TOL
 
 
 def test_tc_resume_equals_one_pass():

@@ -35,8 +35,14 @@ ckda_status make_rope(const ckda_flags& f, int dk, RopeParams* rp) {
     rp->enabled = 1;
     rp->convention = f.rope_convention;
     rp->rot_dims = rot;
-    for (int i = 0; i < rot / 2; ++i)
-        rp->inv_freq[i] = pow((double)f.rope_theta, -2.0 * (double)i / (double)rot);
+    // omega_i = theta^(-2i/rot) ("RoPE review", section 5) as turns per position in 0.64 fixed
+    // point, formed in extended precision: 2^64 frac(omega_i / 2 pi)
+    const long double two_pi = 6.283185307179586476925286766559005768L;
+    for (int i = 0; i < rot / 2; ++i) {
+        const long double omega = powl((long double)f.rope_theta, -2.0L * i / rot);
+        const long double frac = fmodl(omega / two_pi, 1.0L);
+        rp->turns[i] = (unsigned long long)ldexpl(frac, 64);   // exact scaling; truncates
+    }
     return CKDA_OK;
 }
 

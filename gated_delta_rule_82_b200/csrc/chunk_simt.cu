@@ -89,12 +89,12 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
     const int lane = tid & 31, warp = tid >> 5;
     constexpr int NW = kSimtThreads / 32;
 
-    // RoPE inverse frequencies in shared memory (lanes index them per channel; a per-lane index
+    // RoPE frequencies in shared memory (lanes index them per channel; a per-lane index
     // into the kernel-parameter array would serialise in the constant cache).  The barrier at the
     // top of the chunk loop publishes them.
-    __shared__ double sfreq[DK / 2];
+    __shared__ unsigned long long sfreq[DK / 2];
     if (rp.enabled)
-        for (int i = tid; i < DK / 2; i += kSimtThreads) sfreq[i] = rp.inv_freq[i];
+        for (int i = tid; i < DK / 2; i += kSimtThreads) sfreq[i] = rp.turns[i];
 
     // entering state slice
     for (int e = tid; e < DK * DVS; e += kSimtThreads) {

@@ -108,7 +108,7 @@ constexpr uint32_t SM_P = S_SM;                  // signed block totals of alpha
 constexpr uint32_t SM_GC = S_SM + 2048;          // gamma_C fp32 [128] (signed)
 constexpr uint32_t SM_B = S_SM + 2560;           // beta fp32 [64]
 constexpr uint32_t SM_FLAGS = S_SM + 2816;       // exact flag, abort flag, TMEM slot, 5 mbarriers
-constexpr uint32_t SM_FREQ = S_SM + 3072;        // RoPE inverse frequencies fp64 [64]
+constexpr uint32_t SM_FREQ = S_SM + 3072;        // RoPE frequencies, turns per position [64]
 constexpr uint32_t kInBytes = 32768 + 2 * 16384; // alpha, q, k of one chunk-head
 constexpr uint32_t kVBytes = 16384;
 
@@ -539,10 +539,10 @@ __device__ __forceinline__ void intra_role(uint8_t* sm, const TcMaps& maps, cons
     const size_t rs = (size_t)H;   // stride between tokens, in rows of [B*T*H]
     tc::grid_launch_dependents();   // the state pass may start its set-up early
 
-    // RoPE inverse frequencies in shared memory: lanes index them by channel group, and a
+    // RoPE frequencies in shared memory: lanes index them by channel group, and a
     // per-lane index into the kernel-parameter array would serialise in the constant cache
-    double* sfreq = reinterpret_cast<double*>(sm + SM_FREQ);
-    if (tid < 64) sfreq[tid] = rp.inv_freq[tid];
+    unsigned long long* sfreq = reinterpret_cast<unsigned long long*>(sm + SM_FREQ);
+    if (tid < 64) sfreq[tid] = rp.turns[tid];
     if (tid == 32) {
         tc::mbar_init(bar, 1);
         tc::mbar_init(bar_in, 1);

@@ -12,24 +12,26 @@ namespace ckda {
 constexpr float kL2Eps = 1e-6f;  // x / sqrt(sum x^2 + eps), per head
 constexpr int kMaxHalfDim = 64;  // dk <= 128
 
-// Inverse rotary frequencies omega_i = theta^(-2i/dk), computed in double on the host and
-// passed by value, so that concurrent calls with different bases never share state.
+// Rotary frequencies omega_i = theta^(-2i/rot_dims), computed on the host and passed by value
+// (so that concurrent calls with different bases never share state), each as a 0.64 fixed-point
+// count of turns per position: turns[i] = round(2^64 frac(omega_i / 2 pi)).
 struct RopeParams {
-    double inv_freq[kMaxHalfDim];   // theta^(-2i / rot_dims), i < rot_dims / 2 (0 beyond)
+    unsigned long long turns[kMaxHalfDim];   // i < rot_dims / 2 (0 beyond)
     int enabled;     // rope_theta > 0
     int convention;  // 0 half-split, 1 interleaved (both over the first rot_dims channels)
     int rot_dims;    // channels rotated: dk, or dk / 2 (the rest carried through)
 };
 
-// Position angle p * omega, reduced to [-pi, pi] in double, then sin/cos in fp32.  The angle
-// reaches ~6.5e4 rad at 64k tokens: an fp32 product would carry ~4e-3 rad of error there.  On
-// the reduced argument the fast hardware sin/cos is accurate to a few 1e-7 (absolute), far below
-// the bf16 resolution of the rotated activations, at a fraction of the accurate routine's cost.
-__device__ __forceinline__ void rope_sincos(long long p, double omega, float* s, float* c) {
-    const double two_pi = 6.283185307179586476925286766559;
-    double phi = (double)p * omega;
-    double n = rint(phi * (1.0 / two_pi));
-    float r = (float)fma(-n, two_pi, phi);
+// sin and cos of the position angle p * omega for a frequency given as fixed-point turns per
+// position (RopeParams::turns).  p * turns mod 2^64 is the fractional turn count of p * omega,
+// exact in integer arithmetic at any position (an fp32 product p * omega would carry ~4e-3 rad
+// of error at 64k tokens); its top 32 bits, read as a signed fraction of a turn, give the angle
+// reduced to [-pi, pi) to within 2^-32 of a turn.  On that argument the fast hardware sin/cos is
+// accurate to a few 1e-7 (absolute), far below the bf16 resolution of the rotated activations.
+__device__ __forceinline__ void rope_sincos(long long p, unsigned long long turns, float* s,
+                                            float* c) {
+    const unsigned long long t = (unsigned long long)p * turns;
+    const float r = (float)(int)(unsigned)(t >> 32) * 1.4629180792671596e-09f;   // 2 pi / 2^32
     __sincosf(r, s, c);
 }
 

@@ -68,7 +68,7 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
 
     __shared__ float sq[HPC][DK], sk[HPC][DK], sa[HPC][DK], sv[HPC][DV];
     __shared__ float sbeta[HPC], skq[HPC];
-    __shared__ double sfreq[DK / 2];   // RoPE inverse frequencies (lanes index them per channel)
+    __shared__ unsigned long long sfreq[DK / 2];   // RoPE frequencies (lanes index them per channel)
     __shared__ float4 red_w[HPC][RG][C4], red_y[HPC][RG][C4];
 
     const int tid = threadIdx.x;
@@ -130,7 +130,7 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
         if (e < HPC * DV) sv[e / DV][e % DV] = vv[i];
     }
     if (kRope)
-        for (int i = tid; i < DK / 2; i += kDecodeThreads) sfreq[i] = rp.inv_freq[i];
+        for (int i = tid; i < DK / 2; i += kDecodeThreads) sfreq[i] = rp.turns[i];
     if (tid < HPC) sbeta[tid] = (kLogits && blockIdx.x * HPC + tid < NH) ? gate_beta(bv) : bv;
     __syncthreads();
 

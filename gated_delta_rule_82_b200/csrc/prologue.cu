@@ -6,11 +6,13 @@
 //
 // Layout: one CTA handles a run of consecutive tokens (all their heads, q and k).  Each head
 // vector is held by a group of G lanes with 16-byte loads and stores (8 bf16 or 4 fp32 per lane),
-// and the norm is a G-lane shuffle reduction.  Every thread first issues the loads of all its
-// vectors (up to kMaxRounds per batch, kept as raw 16-byte words), so that many bytes are in
-// flight per SM; the sin/cos of the run's angles are computed into shared memory while they
-// arrive, shared by the 2*H head vectors of each token.  The kernel reads and writes every q/k
-// element once: it is HBM-bound.
+// and the norm is a G-lane shuffle reduction.  A lane group takes kMaxRounds consecutive head
+// vectors of the run and issues all their loads first, so that many bytes are in flight per SM.
+// Consecutive vectors are consecutive heads of one token (when H is a multiple of kMaxRounds,
+// always), so a thread needs the sin/cos of its own channels' frequencies at one position: it
+// forms them in registers, again only when the token changes.  The kernel reads and writes every
+// q/k element once: it is HBM-bound.
+#include "fastdiv.h"
 #include "internal.cuh"
 
 namespace ckda {
@@ -18,72 +20,72 @@ namespace ckda {
 namespace {
 
 constexpr int kPrologueThreads = 256;
-constexpr int kMaxRounds = 8;      // head vectors per thread per batch
-constexpr int kMaxTokPerCta = 64;  // bounds the sin/cos table (64 x 64 float2 = 32 KB)
+constexpr int kMaxRounds = 8;      // head vectors per lane group per batch
 
-// vectors of one CTA round (all warps)
+// lane groups of a CTA (vectors it loads per round)
 template <typename T, int DK>
-constexpr int vectors_per_round() {
-    return (kPrologueThreads / 32) * (32 / (DK / ElemsPer16<T>::value));
+constexpr int lane_groups() {
+    return kPrologueThreads / (DK / ElemsPer16<T>::value);
 }
 
 template <typename T, int DK>
 __global__ void __launch_bounds__(kPrologueThreads)
 qk_prologue_kernel(const T* __restrict__ q, const T* __restrict__ k, T* __restrict__ qo,
-                   T* __restrict__ ko, int BT, int T_len, int H, int tok_per_cta, int l2norm,
-                   RopeParams rp, long long pos_offset) {
+                   T* __restrict__ ko, int BT, int T_len, int H, FastDiv hdiv, int tok_per_cta,
+                   int l2norm, RopeParams rp, long long pos_offset) {
     constexpr int EPL = ElemsPer16<T>::value;  // elements per lane
     constexpr int G = DK / EPL;                // lanes per head vector
-    constexpr int VPW = 32 / G;                // head vectors per warp instruction
-    constexpr int VPR = vectors_per_round<T, DK>();
+    constexpr int NG = lane_groups<T, DK>();
     constexpr int HALF = DK / 2;
     static_assert(G >= 2 && G <= 32, "unsupported head size for this element type");
 
-    extern __shared__ float2 cs[];   // (cos, sin) [token of the run][frequency]
-    __shared__ double sfreq[HALF];
+    __shared__ unsigned long long sfreq[HALF];
 
     const int tok0 = blockIdx.x * tok_per_cta;
     const int ntok = min(tok_per_cta, BT - tok0);
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int grp = lane / G, li = lane % G;
-    const int nvec = ntok * 2 * H;  // (token, q/k, head)
-    const int two_h = 2 * H;
-    for (int b0 = 0; b0 < nvec; b0 += kMaxRounds * VPR) {
-        // 1. issue every load of this batch (vector b0 + r VPR + warp VPW + grp in round r)
+    const int lg = threadIdx.x / G, li = threadIdx.x % G;
+    // The run's q vectors are contiguous (tokens x heads x DK), and so are its k vectors: vector
+    // v < nvq is q vector v, the others k vector v - nvq; its token in the run is (v mod nvq) / H.
+    const int nvq = ntok * H;
+    const int nvec = 2 * nvq;
+    const size_t base = (size_t)tok0 * H * DK + (size_t)li * EPL;
+    // rotation: this lane's channels li EPL + e use frequency ib + e (half-split pairs (i, i +
+    // rot / 2)) or ib + e / 2 (interleaved pairs); the first rot channels rotate
+    const int rot = rp.rot_dims;
+    const bool full = rot == DK;
+    const int ib = rp.convention == 0 ? (full ? (li * EPL) % HALF : (li * EPL) % (HALF / 2))
+                                      : li * EPL / 2;
+    const bool rot_lane = rp.enabled && li * EPL < rot;   // this lane holds rotated channels
+    const int dl = full ? G / 2 : G / 4;                  // half-split partner, lanes away
+    if (rp.enabled) {
+        // frequencies in shared memory (a per-lane index into the kernel-parameter array would
+        // serialise in the constant cache)
+        for (int i = threadIdx.x; i < HALF; i += blockDim.x) sfreq[i] = rp.turns[i];
+        __syncthreads();
+    }
+    for (int b0 = 0; b0 < nvec; b0 += kMaxRounds * NG) {
+        const int v0 = b0 + lg * kMaxRounds;   // this lane group's vectors v0 .. v0 + 7
+        // 1. issue every load of this batch
         uint4 raw[kMaxRounds];
 #pragma unroll
         for (int r = 0; r < kMaxRounds; ++r) {
-            const int vid = b0 + r * VPR + warp * VPW + grp;
-            if (vid < nvec) {
-                const int j = vid / two_h, rem = vid - j * two_h;
-                const int which = rem >= H, h = which ? rem - H : rem;
-                const T* src = which ? k : q;
+            const int v = v0 + r;
+            if (v < nvec) {
+                const bool isk = v >= nvq;
                 raw[r] = __ldcs(reinterpret_cast<const uint4*>(
-                    src + ((size_t)(tok0 + j) * H + h) * DK + (size_t)li * EPL));
+                    (isk ? k : q) + base + (size_t)(isk ? v - nvq : v) * DK));
             }
         }
-        // 2. the run's sin/cos table, once, while the loads are in flight
-        if (rp.enabled && b0 == 0) {
-            for (int i = threadIdx.x; i < HALF; i += blockDim.x) sfreq[i] = rp.inv_freq[i];
-            __syncthreads();
-            for (int e = threadIdx.x; e < ntok * HALF; e += blockDim.x) {
-                const int j = e / HALF, i = e - j * HALF;
-                const int t = (tok0 + j) % T_len;
-                float sn, c;
-                rope_sincos(pos_offset + t, sfreq[i], &sn, &c);
-                cs[j * HALF + i] = make_float2(c, sn);
-            }
-            __syncthreads();
-        }
-        // 3. rotate, normalise, store
+        // 2. rotate, normalise, store
+        int jc = -1;              // token whose sin/cos are in cs_, sn_
+        float cs_[EPL], sn_[EPL];
 #pragma unroll
         for (int r = 0; r < kMaxRounds; ++r) {
-            const int vid = b0 + r * VPR + warp * VPW + grp;
-            if (b0 + r * VPR >= nvec) break;   // warp-uniform: no later round has a vector
-            const bool active = vid < nvec;
-            const int vv = active ? vid : 0;
-            const int j = vv / two_h, rem = vv - j * two_h;
-            const int which = rem >= H, h = which ? rem - H : rem;
+            const int v = v0 + r;
+            if (b0 + r >= nvec) break;   // CTA-uniform: every vector of this round is past the end
+            const bool active = v < nvec;
+            const bool isk = v >= nvq;
+            const int vi = active ? (isk ? v - nvq : v) : 0;
             float x[EPL];
             if (active) {
                 if constexpr (EPL == 8) {
@@ -102,32 +104,37 @@ qk_prologue_kernel(const T* __restrict__ q, const T* __restrict__ k, T* __restri
                 for (int e = 0; e < EPL; ++e) x[e] = 0.f;
             }
             if (rp.enabled) {
-                // the first rot_dims channels rotate (all of them, or the first half of the head)
-                const int rot = rp.rot_dims;
-                const float2* csj = cs + j * HALF;
+                const int j = (int)fastdiv(hdiv, (uint32_t)vi);
+                if (j != jc && rot_lane) {
+                    jc = j;
+                    const long long p = pos_offset + (tok0 + j) % T_len;
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) {
+                        const int fi = rp.convention == 0 ? ib + e : ib + e / 2;
+                        if (rp.convention == 0 || (e & 1) == 0)
+                            rope_sincos(p, sfreq[fi], &sn_[e], &cs_[e]);
+                        else {
+                            sn_[e] = sn_[e - 1];
+                            cs_[e] = cs_[e - 1];
+                        }
+                    }
+                }
                 if (rp.convention == 0) {
-                    // pairs (i, i + rot / 2): the partner's elements are dl lanes away
-                    const int dl = rot == DK ? G / 2 : G / 4;
                     float y[EPL];
 #pragma unroll
                     for (int e = 0; e < EPL; ++e) y[e] = __shfl_xor_sync(0xffffffffu, x[e], dl);
-                    const bool first = li < dl;
-                    if (li < 2 * dl) {
+                    if (rot_lane) {
+                        const bool first = li < dl;
 #pragma unroll
-                        for (int e = 0; e < EPL; ++e) {
-                            const int i = (li * EPL + e) % (rot / 2);
-                            const float2 c = csj[i];
-                            x[e] = first ? (x[e] * c.x - y[e] * c.y) : (x[e] * c.x + y[e] * c.y);
-                        }
+                        for (int e = 0; e < EPL; ++e)
+                            x[e] = first ? (x[e] * cs_[e] - y[e] * sn_[e]) : (x[e] * cs_[e] + y[e] * sn_[e]);
                     }
-                } else {
+                } else if (rot_lane) {
 #pragma unroll
                     for (int e = 0; e < EPL; e += 2) {
-                        if (li * EPL + e >= rot) continue;
-                        const float2 c = csj[(li * EPL + e) / 2];
                         const float a = x[e], b = x[e + 1];
-                        x[e] = a * c.x - b * c.y;
-                        x[e + 1] = b * c.x + a * c.y;
+                        x[e] = a * cs_[e] - b * sn_[e];
+                        x[e + 1] = b * cs_[e] + a * sn_[e];
                     }
                 }
             }
@@ -140,10 +147,7 @@ qk_prologue_kernel(const T* __restrict__ q, const T* __restrict__ k, T* __restri
 #pragma unroll
                 for (int e = 0; e < EPL; ++e) x[e] *= rn;
             }
-            if (active) {
-                T* dst = which ? ko : qo;
-                Vec16<T, EPL>::store(dst + ((size_t)(tok0 + j) * H + h) * DK + (size_t)li * EPL, x);
-            }
+            if (active) Vec16<T, EPL>::store((isk ? ko : qo) + base + (size_t)vi * DK, x);
         }
     }
 }
@@ -153,15 +157,15 @@ cudaError_t launch_prologue_t(const void* q, const void* k, void* qo, void* ko, 
                               int H, int l2norm, const RopeParams& rp, long long pos_offset,
                               cudaStream_t stream) {
     const int BT = B * T_len;
-    // tokens per CTA: one batch of kMaxRounds vectors per thread covers them (at least one
-    // token, at most kMaxTokPerCta)
-    constexpr int per_batch = kMaxRounds * vectors_per_round<T, DK>();
-    const int tpc = max(1, min(kMaxTokPerCta, per_batch / (2 * H)));
+    // tokens per CTA: one batch of kMaxRounds vectors per lane group covers them (at least one
+    // token)
+    constexpr int per_batch = kMaxRounds * lane_groups<T, DK>();
+    const int tpc = max(1, per_batch / (2 * H));
     const int grid = (BT + tpc - 1) / tpc;
-    const size_t smem = rp.enabled ? (size_t)tpc * (DK / 2) * sizeof(float2) : 0;
-    qk_prologue_kernel<T, DK><<<grid, kPrologueThreads, smem, stream>>>(
+    qk_prologue_kernel<T, DK><<<grid, kPrologueThreads, 0, stream>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), static_cast<T*>(qo),
-        static_cast<T*>(ko), BT, T_len, H, tpc, l2norm, rp, pos_offset);
+        static_cast<T*>(ko), BT, T_len, H, make_fastdiv((uint32_t)H), tpc, l2norm, rp,
+        pos_offset);
     return cudaGetLastError();
 }
 

@@ -15,7 +15,8 @@ import torch
 
 __all__ = ["CkdaError", "library_path", "abi_version", "qk_prologue", "workspace_bytes",
            "fwd_chunked", "varlen_workspace_bytes", "fwd_varlen", "decode_step", "selftest_umma",
-           "last_device_status", "set_wait_limit_ns", "PATHS"]
+           "last_device_status", "set_wait_limit_ns", "bwd_workspace_bytes", "bwd_chunked",
+           "PATHS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libckda.so")
@@ -72,6 +73,10 @@ def _load():
     lib.ckda_decode_step.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, _Flags, I, P]
     lib.ckda_selftest_umma.restype = I
     lib.ckda_selftest_umma.argtypes = [P, P, P, I, I, I, I, P]
+    lib.ckda_bwd_workspace_bytes.restype = SZ
+    lib.ckda_bwd_workspace_bytes.argtypes = [I, I, I, I, I]
+    lib.ckda_bwd_chunked.restype = I
+    lib.ckda_bwd_chunked.argtypes = [P] * 14 + [I] * 5 + [_Flags, I, LL, P, SZ, P]
     lib.ckda_last_device_status.restype = I
     lib.ckda_last_device_status.argtypes = [P, ctypes.POINTER(I)]
     lib.ckda_set_wait_limit_ns.restype = I
@@ -306,6 +311,55 @@ def decode_step(q, k, v, alpha, beta, state, pos=None, *, l2norm=True, rope_thet
         _stream(q.device))
     _raise("ckda_decode_step", st)
     return out
+
+
+def bwd_workspace_bytes(B, T, H, dk, dv) -> int:
+    n = _load().ckda_bwd_workspace_bytes(B, T, H, dk, dv)
+    if n == ctypes.c_size_t(-1).value:
+        raise ValueError("unsupported problem for ckda_bwd_chunked")
+    return int(n)
+
+
+def bwd_chunked(q, k, v, alpha, beta, h0, dout, dhT=None, *, l2norm=True, rope_theta=0.0,
+                rope_convention=0, scale=0.0, pos_offset=0, gate_logits=False, rope_dims=0,
+                workspace=None, want_dh0=True):
+    """Gradients of <dout, out> + <dhT, hT> for fwd_chunked with the same inputs and flags.
+
+    Returns a dict of fp32 tensors: dq, dk ([B, T, Hk, dk]), dv, dalpha, dbeta and dh0 (None
+    when want_dh0 is False).  dout has the dtype of q; dhT is fp32 [B, H, dk, dv] or None.
+    """
+    _check(q, "q")
+    B, T, Hk, dk = q.shape
+    _check(v, "v", dtype=q.dtype)
+    H, dv = v.shape[2], v.shape[3]
+    if H % Hk:
+        raise ValueError(f"v has {H} heads, not a multiple of q's {Hk}")
+    _check(k, "k", dtype=q.dtype, shape=q.shape)
+    _check(alpha, "alpha", dtype=q.dtype if gate_logits else torch.float32, shape=(B, T, H, dk))
+    _check(beta, "beta", dtype=torch.float32, shape=(B, T, H))
+    _check(dout, "dout", dtype=q.dtype, shape=(B, T, H, dv))
+    if h0 is not None:
+        _check(h0, "h0", dtype=torch.float32, shape=(B, H, dk, dv))
+    if dhT is not None:
+        _check(dhT, "dhT", dtype=torch.float32, shape=(B, H, dk, dv))
+    f32 = dict(dtype=torch.float32, device=q.device)
+    g = {"dq": torch.empty((B, T, Hk, dk), **f32), "dk": torch.empty((B, T, Hk, dk), **f32),
+         "dv": torch.empty((B, T, H, dv), **f32), "dalpha": torch.empty((B, T, H, dk), **f32),
+         "dbeta": torch.empty((B, T, H), **f32),
+         "dh0": torch.empty((B, H, dk, dv), **f32) if want_dh0 else None}
+    if workspace is None:
+        workspace = torch.empty(bwd_workspace_bytes(B, T, H, dk, dv), dtype=torch.uint8,
+                                device=q.device)
+    wbytes = workspace.numel() * workspace.element_size()
+    st = _load().ckda_bwd_chunked(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(h0), _ptr(dout), _ptr(dhT),
+        _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dalpha"]), _ptr(g["dbeta"]),
+        _ptr(g["dh0"]), B, T, H, dk, dv,
+        _flags(l2norm, rope_theta, rope_convention, scale, 0, 0, gate_logits,
+               Hk if Hk != H else 0, rope_dims),
+        _dtype_code(q), int(pos_offset), _ptr(workspace), wbytes, _stream(q.device))
+    _raise("ckda_bwd_chunked", st)
+    return g
 
 
 def last_device_status(device=None) -> int:

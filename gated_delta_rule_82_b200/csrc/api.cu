@@ -287,6 +287,64 @@ ckda_status ckda_decode_step(const void* q, const void* k, const void* v, const 
                                    (cudaStream_t)stream));
 }
 
+size_t ckda_bwd_workspace_bytes(int B, int T, int H, int dk, int dv) {
+    if (B < 1 || T < 1 || H < 1) return (size_t)-1;
+    if (!supported_dim(dk) || !supported_dim(dv)) return (size_t)-1;
+    if ((long long)B * T * H * 128 > (1ll << 40)) return (size_t)-1;
+    return bwd_layout(nullptr, B, T, H, dk, dv).bytes;
+}
+
+ckda_status ckda_bwd_chunked(const void* q, const void* k, const void* v, const void* alpha,
+                             const float* beta, const float* h0, const void* dout,
+                             const float* dhT, float* dq, float* dk, float* dv, float* dalpha,
+                             float* dbeta, float* dh0, int B, int T, int H, int dk_, int dv_,
+                             ckda_flags flags, ckda_dtype dtype, long long pos_offset,
+                             void* workspace, size_t workspace_bytes, ckda_stream_t stream) {
+    if (!q || !k || !v || !alpha || !beta || !dout || !dq || !dk || !dv || !dalpha || !dbeta)
+        return CKDA_ERR_NULL;
+    if (dtype != CKDA_F32 && dtype != CKDA_BF16) return CKDA_ERR_UNSUPPORTED;
+    if (B < 1 || T < 1 || H < 1) return CKDA_ERR_SHAPE;
+    if ((long long)B * T * H * 128 > (1ll << 40) || (long long)B * H * 128 * 128 > (1ll << 40))
+        return CKDA_ERR_SHAPE;
+    if ((long long)B * H * ((T + 15) / 16) > 0x7fffffffll) return CKDA_ERR_SHAPE;
+    if (!supported_dim(dk_) || !supported_dim(dv_)) return CKDA_ERR_UNSUPPORTED;
+    if (flags.qk_heads < 0 || (flags.qk_heads > 0 && H % flags.qk_heads != 0)) return CKDA_ERR_ARG;
+    if (flags.gate_logits != 0 && flags.gate_logits != 1) return CKDA_ERR_ARG;
+    const void* ptrs[] = {q, k, v, alpha, beta, h0, dout, dhT, dq, dk, dv, dalpha, dbeta, dh0,
+                          workspace};
+    for (const void* ptr : ptrs)
+        if (ptr && !aligned16(ptr)) return CKDA_ERR_ALIGN;
+    const size_t need = ckda_bwd_workspace_bytes(B, T, H, dk_, dv_);
+    if (!workspace || workspace_bytes < need) return CKDA_ERR_WORKSPACE;
+    const int G = flags.qk_heads > 0 ? H / flags.qk_heads : 1;
+    const size_t es = elem_size(dtype), ntok = (size_t)B * T;
+    const size_t nqk = ntok * (H / G) * dk_, nv = ntok * H * dv_, nal = ntok * H * dk_;
+    const size_t nst = (size_t)B * H * dk_ * dv_;
+    // outputs (fp32) against every input and each other; the workspace against all of them
+    const void* ins[] = {q, k, v, alpha, beta, h0, dout, dhT};
+    const size_t insz[] = {nqk * es, nqk * es, nv * es, nal * (flags.gate_logits ? es : 4),
+                           ntok * H * 4, nst * 4, nv * es, nst * 4};
+    void* outs[] = {dq, dk, dv, dalpha, dbeta, dh0, workspace};
+    const size_t outsz[] = {nqk * 4, nqk * 4, nv * 4, nal * 4, ntok * H * 4, nst * 4, need};
+    for (int i = 0; i < 7; ++i) {
+        for (int j = 0; j < 8; ++j)
+            if (outs[i] && overlap(outs[i], outsz[i], ins[j], insz[j])) return CKDA_ERR_ARG;
+        for (int j = 0; j < i; ++j)
+            if (outs[i] && outs[j] && overlap(outs[i], outsz[i], outs[j], outsz[j])) return CKDA_ERR_ARG;
+    }
+    BwdArgs a;
+    a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.beta = beta; a.h0 = h0; a.dout = dout;
+    a.dhT = dhT; a.dq_out = dq; a.dk_out = dk; a.dv = dv; a.dalpha = dalpha; a.dbeta = dbeta;
+    a.dh0 = dh0; a.B = B; a.T_len = T; a.H = H; a.G = G; a.l2norm = flags.l2norm ? 1 : 0;
+    ckda_status st = make_rope(flags, dk_, &a.rp);
+    if (st != CKDA_OK) return st;
+    a.scale = resolve_scale(flags, dk_);
+    a.pos_offset = pos_offset;
+    a.gate_logits = flags.gate_logits;
+    a.dtype = dtype;
+    return from_cuda(launch_chunk_bwd(a, dk_, dv_, workspace, (cudaStream_t)stream));
+}
+
 ckda_status ckda_selftest_umma(const void* A, const void* B, float* D, int M, int N, int K,
                                int b_mn_major, ckda_stream_t stream) {
     if (!A || !B || !D) return CKDA_ERR_NULL;

@@ -26,12 +26,52 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, const voi
                           int H, int G, int dk, int dv, int l2norm, const RopeParams& rp, float scale,
                           int gate_logits, ckda_dtype dtype, cudaStream_t stream);
 
+// Arguments of the CUDA-core chunked forward.  states: nullable; when given, the state entering
+// each chunk is written there ([B*H][ceil(T/chunk)][dk][dv] fp32).  out and hT are nullable.
+struct SimtArgs {
+    const void *q, *k, *v, *alpha;
+    const float *beta, *h0;
+    void* out;
+    float* hT;
+    float* states;
+    int B, T_len;
+    const int* cu;   // packed sequences (B = their count), or nullptr
+    int H, G, l2norm;
+    RopeParams rp;
+    float scale;
+    long long pos_offset;
+    int gate_logits;
+};
+cudaError_t launch_chunk_simt(const SimtArgs& a, int dk, int dv, int chunk, ckda_dtype dtype,
+                              cudaStream_t stream);
 cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const void* alpha,
                               const float* beta, const float* h0, void* out, float* hT, int B,
                               int T_len, int H, int G, int dk, int dv, int chunk, int l2norm,
                               const RopeParams& rp, float scale, long long pos_offset,
                               int gate_logits, ckda_dtype dtype, const PackedSeqs& pk,
                               cudaStream_t stream);
+
+// Backward of the chunked forward on CUDA cores (fp32 gradients).
+struct BwdArgs {
+    const void *q, *k, *v, *alpha;
+    const float *beta, *h0;
+    const void* dout;
+    const float* dhT;
+    float *dq_out, *dk_out, *dv, *dalpha, *dbeta, *dh0;
+    int B, T_len, H, G, l2norm;
+    RopeParams rp;
+    float scale;
+    long long pos_offset;
+    int gate_logits;
+    ckda_dtype dtype;
+};
+struct BwdLayout {
+    float *states, *dstates, *dq, *dk;
+    size_t bytes;
+};
+BwdLayout bwd_layout(void* ws, int B, int T_len, int H, int dk, int dv);
+cudaError_t launch_chunk_bwd(const BwdArgs& a, int dk, int dv, void* workspace,
+                             cudaStream_t stream);
 
 // Tensor-core chunked forward (bf16, dk = dv = 128, chunk = 64).
 size_t chunk_tc_workspace_bytes(int B, int T_len, int H);

@@ -47,7 +47,7 @@
 extern "C" {
 #endif
 
-#define CKDA_ABI_VERSION 5
+#define CKDA_ABI_VERSION 6
 
 #if defined(__GNUC__)
 #define CKDA_API __attribute__((visibility("default")))
@@ -244,6 +244,42 @@ CKDA_API ckda_status ckda_decode_step(const void* q, const void* k, const void* 
                              const float* beta, float* state, void* out, const long long* pos,
                              int N, int H, int dk, int dv, ckda_flags flags, ckda_dtype dtype,
                              ckda_stream_t stream);
+
+/*
+ * Bytes of device workspace ckda_bwd_chunked needs (never 0), or (size_t)-1 for invalid or
+ * unsupported sizes.
+ */
+CKDA_API size_t ckda_bwd_workspace_bytes(int B, int T, int H, int dk, int dv);
+
+/*
+ * Backward of ckda_fwd_chunked: the gradients of L = <dout, out> + <dhT, hT> with respect to
+ * q, k, v, the gates and h0, for the forward with the same inputs, sizes and flags (rotation,
+ * norm, scale, grouped value heads, gate logits).  Computed in fp32 on the CUDA cores by the
+ * chunked form run in reverse (16-token chunks: the forward replay keeps each chunk's entering
+ * state, a reverse chain carries the state gradient, every chunk forms its input gradients, and
+ * the prologue -- rotation, then L2 norm -- is differentiated last).  There is no backward on
+ * the pages beyond the statement that one exists ("Complex KDA" paper summary, Implementation:
+ * a hybrid TileLang backward); this is the reverse mode of the recurrence above.
+ *   q, k, v, alpha, beta, h0 : the forward's inputs (layouts and types as ckda_fwd_chunked;
+ *                              h0 may be NULL for a zero initial state)
+ *   dout : [B, T, H, dv] of `dtype`, the gradient of out (required)
+ *   dhT  : [B, H, dk, dv] fp32, the gradient of hT, or NULL for zero
+ *   dq, dk : [B, T, Hk, dk] fp32 (Hk = flags.qk_heads or H: a grouped q/k head receives the sum
+ *            over the value heads that read it)
+ *   dv   : [B, T, H, dv] fp32      dalpha : [B, T, H, dk] fp32      dbeta : [B, T, H] fp32
+ *          (with flags.gate_logits, dalpha and dbeta are the gradients of the logits a and b)
+ *   dh0  : [B, H, dk, dv] fp32, or NULL to skip it
+ *   workspace : at least ckda_bwd_workspace_bytes(B, T, H, dk, dv), 16-byte aligned, owned by
+ *               the caller and not shared with concurrent calls
+ * flags.path and flags.stages are ignored.  Outputs must not overlap the inputs or each other.
+ */
+CKDA_API ckda_status ckda_bwd_chunked(const void* q, const void* k, const void* v,
+                                      const void* alpha, const float* beta, const float* h0,
+                                      const void* dout, const float* dhT, float* dq, float* dk,
+                                      float* dv, float* dalpha, float* dbeta, float* dh0, int B,
+                                      int T, int H, int dk_, int dv_, ckda_flags flags,
+                                      ckda_dtype dtype, long long pos_offset, void* workspace,
+                                      size_t workspace_bytes, ckda_stream_t stream);
 
 /*
  * Diagnostic: D[M, N] (fp32, row-major) = A[M, K] * B for bf16 A (row-major, K contiguous),

@@ -26,7 +26,8 @@ from __future__ import annotations
 
 import numpy as np
 
-TENSOR_IDS = {"q": 1, "k": 2, "v": 3, "alpha": 4, "beta": 5, "h0": 6, "pos": 7}
+TENSOR_IDS = {"q": 1, "k": 2, "v": 3, "alpha": 4, "beta": 5, "h0": 6, "pos": 7, "dout": 8,
+              "dhT": 9}
 
 
 def _gen(seed: int, tensor: str) -> np.random.Generator:
@@ -125,6 +126,17 @@ def fwd_inputs(B, T, H, dk, dv, *, kind="ckda", dtype="bf16", h0_std=0.0, seed=0
     else:
         d["h0"] = None
     d["meta"] = dict(B=B, T=T, H=H, dk=dk, dv=dv, kind=kind, dtype=dtype, seed=seed)
+    return d
+
+
+def bwd_inputs(B, T, H, dk, dv, *, dtype="bf16", dhT_std=0.0, seed=0):
+    """Output gradients for a backward call: dout [B,T,H,dv] ~ N(0,1) in the activation dtype
+    (float32 values, bf16 bit patterns under dout_bits) and dhT [B,H,dk,dv] ~ N(0, dhT_std^2)
+    float32 (None when dhT_std == 0)."""
+    val, bits = _activation(seed, "dout", (B, T, H, dv), dtype)
+    d = {"dout": val, "dout_bits": bits}
+    d["dhT"] = ((dhT_std * _normal(seed, "dhT", (B, H, dk, dv))).astype(np.float32)
+                if dhT_std > 0 else None)
     return d
 
 

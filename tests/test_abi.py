@@ -52,7 +52,7 @@ def test_only_declared_symbols_are_exported(lib):
 
 
 def test_version_and_strerror(lib):
-    assert ck.abi_version() == 5
+    assert ck.abi_version() == 6
     for s in range(9):
         assert lib.ckda_strerror(s)
     assert lib.ckda_strerror(99) == b"unknown status"

@@ -1,6 +1,7 @@
 """A chunked form of the backward pass, restated in float64 numpy and checked against the
-oracle's gradients (which are pinned to finite differences): the algebra a GPU backward would
-evaluate chunk by chunk.
+oracle's gradients (which are pinned to finite differences): first in the plain form below, then
+in the numerically stable form that the GPU backward (ckda_bwd_chunked) evaluates chunk by chunk
+(at the end of this file).
 
 Forward per chunk (as in the chunk-algebra test; gamma the running gate products, Kg = gamma k^,
 Ki = k^ / gamma, Qg = gamma q^):
@@ -143,6 +144,129 @@ def test_chunked_backward_equals_the_oracle(T, C, theta, l2):
     dout, dhT = rng.standard_normal((T, dv)), rng.standard_normal((dk, dv))
     scale = oracle.default_scale(dk)
     got = _chunked_bwd(q, k, v, alpha, beta, h0, dout, dhT, C, scale, l2, theta, 3)
+    ref = oracle.bwd(q[None, :, None], k[None, :, None], v[None, :, None], alpha[None, :, None],
+                     beta[None, :, None], h0[None, None], dout[None, :, None], dhT[None, None],
+                     l2norm=l2, rope_theta=theta, pos_offset=3)
+    want = (ref["dq"][0, :, 0], ref["dk"][0, :, 0], ref["dv"][0, :, 0], ref["dalpha"][0, :, 0],
+            ref["dbeta"][0, :, 0], ref["dh0"][0, 0])
+    for name, x, y in zip(("dq", "dk", "dv", "dalpha", "dbeta", "dh0"), got, want):
+        err = np.abs(x - y).max() / max(np.abs(y).max(), 1e-12)
+        assert err < 1e-9, (name, err)
+
+
+
+# ---- the stable form the GPU backward evaluates -------------------------------------------------
+# The form above forms k / gamma, which overflows once the gate products underflow (long runs of
+# small gates, exact zeros).  The GPU backward instead keeps the sign of gamma absorbed into q'
+# and k' and every ratio as R_rj = |gamma_r| / |gamma_j| = 2^(L_r - L_j) <= 1 (L the running sum
+# of log2 max(|alpha|, FLT_MIN)), takes the gradients with respect to R and g = |gamma| directly,
+# and reaches the gates without dividing by alpha:
+#   dalpha_t = sign(alpha_t) [ g_{t-1} sum_{r>=t} dg_r R_rt + sum_{a>=t} R_at Z_at ],
+#   Z_{a,t} = |alpha_{t-1}| Z_{a,t-1} + dR_{a,t-1},  Z_{a,0} = 0.
+FLT_MIN = 1.17549435e-38
+
+
+def _stable_factors(qh, kh, V, a, b):
+    C = qh.shape[0]
+    sig = np.cumprod(np.where(a < 0, -1.0, 1.0), axis=0)
+    L = np.cumsum(np.log2(np.maximum(np.abs(a), FLT_MIN)), axis=0)
+    R = 2.0 ** (L[:, None, :] - L[None, :, :]) * np.tril(np.ones((C, C)))[:, :, None]
+    g = 2.0 ** L
+    kp, qp = sig * kh, sig * qh
+    P = np.einsum("rc,jc,rjc->rj", kp, kp, R) * np.tril(np.ones((C, C)), -1)
+    M = np.einsum("rc,jc,rjc->rj", qp, kp, R)
+    T = np.linalg.inv(np.eye(C) + b[:, None] * P)
+    Kg, Qg = g * kp, g * qp
+    W, U = T @ (b[:, None] * Kg), T @ (b[:, None] * V)
+    return dict(sig=sig, sC=sig[-1], gC=g[-1], R=R, g=g, kp=kp, qp=qp, P=P, M=M, T=T, Kg=Kg,
+                Qg=Qg, W=W, U=U, Kend=sig[-1] * R[-1] * kp, Qp=Qg - M @ W)
+
+
+def _stable_chunk_grads(F, V, a, b, S0, dO, dS1, scale):
+    C = V.shape[0]
+    kp, qp, R, g, T, W, U, M, Kend, Kg = (F[x] for x in ("kp", "qp", "R", "g", "T", "W", "U",
+                                                         "M", "Kend", "Kg"))
+    dQp = scale * dO @ S0.T
+    dU = scale * M.T @ dO + Kend @ dS1
+    dKend = (U - W @ S0) @ dS1.T
+    dW = -(Kend @ dS1) @ S0.T - M.T @ dQp
+    dM = np.tril(scale * dO @ U.T - dQp @ W.T)
+    dgC = (dS1 * S0).sum(1)
+    X, Y = T.T @ dW, T.T @ dU
+    dT = dW @ (b[:, None] * Kg).T + dU @ (b[:, None] * V).T
+    dA = np.tril(-T.T @ dT @ T.T, -1)
+    db = (X * Kg).sum(1) + (Y * V).sum(1) + (dA * F["P"]).sum(1)
+    E = b[:, None] * dA
+    dKg = b[:, None] * X
+    dkp = (np.einsum("rj,jc,rjc->rc", E, kp, R) + np.einsum("rj,rc,rjc->jc", E, kp, R)
+           + np.einsum("rj,rc,rjc->jc", dM, qp, R) + dKg * g + dKend * F["sC"] * R[-1])
+    dqp = np.einsum("rj,jc,rjc->rc", dM, kp, R) + dQp * g
+    dR = np.einsum("rj,rc,jc->rjc", E, kp, kp) + np.einsum("rj,rc,jc->rjc", dM, qp, kp)
+    dR[-1] += dKend * F["sC"] * kp
+    dg = dKg * kp + dQp * qp
+    dg[-1] += dgC * F["sC"]
+    am = np.maximum(np.abs(a), FLT_MIN)
+    da = np.zeros_like(a)
+    Z = np.zeros((C, a.shape[1]))
+    for t in range(C):
+        if t > 0:
+            Z = am[t - 1] * Z + dR[:, t - 1, :]
+        gprev = g[t - 1] if t > 0 else 1.0
+        da[t] = np.where(a[t] < 0, -1.0, 1.0) * (gprev * (dg[t:] * R[t:, t]).sum(0)
+                                                 + (R[t:, t] * Z[t:]).sum(0))
+    dS0 = scale * F["Qp"].T @ dO + (F["sC"] * F["gC"])[:, None] * dS1 - W.T @ (Kend @ dS1)
+    return F["sig"] * dqp, F["sig"] * dkp, b[:, None] * Y, da, db, dS0
+
+
+def _stable_chunked_bwd(q, k, v, alpha, beta, h0, dout, dhT, C, scale, l2norm, theta, pos0):
+    T, dk = q.shape
+    pos = pos0 + np.arange(T, dtype=np.float64)
+    yq = _rot(q, pos, theta) if theta > 0 else q.copy()
+    yk = _rot(k, pos, theta) if theta > 0 else k.copy()
+    nq = np.sqrt((yq ** 2).sum(1) + 1e-6)[:, None] if l2norm else np.ones((T, 1))
+    nk = np.sqrt((yk ** 2).sum(1) + 1e-6)[:, None] if l2norm else np.ones((T, 1))
+    qh, kh = yq / nq, yk / nk
+    S, S0s = h0.copy(), []
+    for c0 in range(0, T, C):
+        sl = slice(c0, min(T, c0 + C))
+        S0s.append(S.copy())
+        F = _stable_factors(qh[sl], kh[sl], v[sl], alpha[sl], beta[sl])
+        S = (np.diag(F["sC"] * F["gC"]) - F["Kend"].T @ F["W"]) @ S + F["Kend"].T @ F["U"]
+    dS = dhT.copy()
+    grads = [np.zeros_like(x) for x in (qh, kh, v, alpha, beta)]
+    for ci in reversed(range(len(S0s))):
+        sl = slice(ci * C, min(T, ci * C + C))
+        F = _stable_factors(qh[sl], kh[sl], v[sl], alpha[sl], beta[sl])
+        *gs, dS = _stable_chunk_grads(F, v[sl], alpha[sl], beta[sl], S0s[ci], dout[sl], dS,
+                                      scale)
+        for G_, x in zip(grads, gs):
+            G_[sl] = x
+
+    def back(y, n, g):
+        if l2norm:
+            g = g / n - y * ((y * g).sum(1)[:, None]) / n ** 3
+        return _rot(g, pos, theta, inverse=True) if theta > 0 else g
+    return back(yq, nq, grads[0]), back(yk, nk, grads[1]), grads[2], grads[3], grads[4], dS
+
+
+@pytest.mark.parametrize("T,C,theta,l2,amin,zeros", [(32, 8, 0.0, True, 0.4, False),
+                                                     (40, 16, 100.0, True, 1e-3, False),
+                                                     (48, 16, 0.0, True, 1e-3, True),
+                                                     (29, 16, 1000.0, False, 0.05, True)])
+def test_stable_chunked_backward_equals_the_oracle(T, C, theta, l2, amin, zeros):
+    """Gates down to 1e-3 (their products underflow within a chunk) and exact zeros."""
+    rng = np.random.default_rng(T * 7 + C)
+    dk, dv = 6, 4
+    q, k = rng.standard_normal((T, dk)), rng.standard_normal((T, dk))
+    v = rng.standard_normal((T, dv))
+    alpha = rng.choice([-1.0, 1.0], (T, dk)) * rng.uniform(amin, 1.0, (T, dk))
+    if zeros:
+        alpha[rng.random((T, dk)) < 0.1] = 0.0
+    beta = rng.uniform(0.0, 2.0, T)
+    h0 = rng.standard_normal((dk, dv))
+    dout, dhT = rng.standard_normal((T, dv)), rng.standard_normal((dk, dv))
+    scale = oracle.default_scale(dk)
+    got = _stable_chunked_bwd(q, k, v, alpha, beta, h0, dout, dhT, C, scale, l2, theta, 3)
     ref = oracle.bwd(q[None, :, None], k[None, :, None], v[None, :, None], alpha[None, :, None],
                      beta[None, :, None], h0[None, None], dout[None, :, None], dhT[None, None],
                      l2norm=l2, rope_theta=theta, pos_offset=3)

@@ -53,6 +53,7 @@ bwd_chain_kernel(const T* __restrict__ q, const T* __restrict__ k, const void* _
                  long long pos_offset, int gate_logits) {
     using Sh = ChainShape<DK, DV, C>;
     constexpr int DVS = Sh::DVS;
+    constexpr int LD = Factors<DK, C>::LD;
     extern __shared__ float smem[];
     Factors<DK, C> f;
     f.bind(smem);
@@ -85,15 +86,15 @@ bwd_chain_kernel(const T* __restrict__ q, const T* __restrict__ k, const void* _
         // Q' = Q_gamma - M W;  K_end dS_out
         for (int e = tid; e < C * DK; e += kThreads) {
             const int r = e / DK, c = e % DK;
-            float acc = exp2f(f.L[e]) * f.q[e];
-            for (int j = 0; j <= r; ++j) acc -= f.M[r * C + j] * f.W[j * DK + c];
+            float acc = exp2f(f.L[r * LD + c]) * f.q[r * LD + c];
+            for (int j = 0; j <= r; ++j) acc -= f.M[r * C + j] * f.W[j * LD + c];
             sQp[e] = acc;
         }
         for (int e = tid; e < C * DVS; e += kThreads) {
             const int j = e / DVS, n = e % DVS;
             float acc = 0.f;
             for (int c = 0; c < DK; ++c)
-                acc += f.sg[c] * exp2f(f.LC[c] - f.L[j * DK + c]) * f.k[j * DK + c] * sdS[c * DVS + n];
+                acc += f.sg[c] * exp2f(f.LC[c] - f.L[j * LD + c]) * f.k[j * LD + c] * sdS[c * DVS + n];
             sKd[e] = acc;
         }
         __syncthreads();
@@ -102,7 +103,7 @@ bwd_chain_kernel(const T* __restrict__ q, const T* __restrict__ k, const void* _
             const int c = e / DVS, n = e % DVS;
             float acc = f.sg[c] * exp2f(f.LC[c]) * sdS[e];
             for (int r = 0; r < C; ++r)
-                acc += scale * sQp[r * DK + c] * sdO[r * DVS + n] - f.W[r * DK + c] * sKd[r * DVS + n];
+                acc += scale * sQp[r * DK + c] * sdO[r * DVS + n] - f.W[r * LD + c] * sKd[r * DVS + n];
             sdS[e] = acc;   // each element is read only by its own thread above
         }
     }
@@ -116,7 +117,8 @@ bwd_chain_kernel(const T* __restrict__ q, const T* __restrict__ k, const void* _
 template <int DK, int DV, int C>
 struct GradShape {
     static constexpr int DT = DV < 32 ? DV : 32;
-    static constexpr int CD = C * DK, CC = C * C, CT = C * DT;
+    static constexpr int TP = DT + 1;   // tile rows are TP floats apart (distinct banks down a column)
+    static constexpr int CD = C * DK, CC = C * C, CT = C * TP;
     static constexpr int off_qp = Factors<DK, C>::floats;  // Q'     [C][DK]
     static constexpr int off_ke = off_qp + CD;             // K_end  [C][DK]
     static constexpr int off_dqp = off_ke + CD;            // dQ'    [C][DK]
@@ -129,9 +131,9 @@ struct GradShape {
     static constexpr int off_dT = off_dM + CC;             // dT, then E = B dA [C][C]
     static constexpr int off_Z = off_dT + CC;              // dT T^T [C][C]
     static constexpr int off_db = off_Z + CC;              // dbeta [C]
-    static constexpr int off_s0 = off_db + C;              // S0 tile      [DK][DT]
-    static constexpr int off_ds = off_s0 + DK * DT;        // dS_out tile  [DK][DT]
-    static constexpr int off_do = off_ds + DK * DT;        // dO tile [C][DT]
+    static constexpr int off_s0 = off_db + C;              // S0 tile      [DK][TP]
+    static constexpr int off_ds = off_s0 + DK * TP;        // dS_out tile  [DK][TP]
+    static constexpr int off_do = off_ds + DK * TP;        // dO tile [C][TP]
     static constexpr int off_v = off_do + CT;              // V tile
     static constexpr int off_u = off_v + CT;               // U tile
     static constexpr int off_du = off_u + CT;              // dU tile
@@ -154,6 +156,8 @@ bwd_grad_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
                 int l2norm, RopeParams rp, float scale, long long pos_offset, int gate_logits) {
     using Sh = GradShape<DK, DV, C>;
     constexpr int DT = Sh::DT;
+    constexpr int TP = Sh::TP;   // padded row stride of the tiles
+    constexpr int LD = Factors<DK, C>::LD;
     extern __shared__ float smem[];
     Factors<DK, C> f;
     f.bind(smem);
@@ -197,10 +201,10 @@ bwd_grad_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
     // Q', K_end, P, the running sign products; zero the accumulators
     for (int e = tid; e < C * DK; e += kThreads) {
         const int r = e / DK, c = e % DK;
-        float acc = exp2f(f.L[e]) * f.q[e];
-        for (int j = 0; j <= r; ++j) acc -= f.M[r * C + j] * f.W[j * DK + c];
+        float acc = exp2f(f.L[r * LD + c]) * f.q[r * LD + c];
+        for (int j = 0; j <= r; ++j) acc -= f.M[r * C + j] * f.W[j * LD + c];
         sQp[e] = acc;
-        sKe[e] = f.sg[c] * exp2f(f.LC[c] - f.L[e]) * f.k[e];
+        sKe[e] = f.sg[c] * exp2f(f.LC[c] - f.L[r * LD + c]) * f.k[r * LD + c];
         sdQp[e] = 0.f;
         sdKe[e] = 0.f;
         sdW[e] = 0.f;
@@ -218,7 +222,7 @@ bwd_grad_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
         float p = 0.f;
         if (j < r)
             for (int c = 0; c < DK; ++c)
-                p += f.k[r * DK + c] * f.k[j * DK + c] * exp2f(f.L[r * DK + c] - f.L[j * DK + c]);
+                p += f.k[r * LD + c] * f.k[j * LD + c] * exp2f(f.L[r * LD + c] - f.L[j * LD + c]);
         sP[e] = p;
         sdM[e] = 0.f;
         sdT[e] = 0.f;
@@ -232,35 +236,35 @@ bwd_grad_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
         // tiles of S0, dS_out, dO, V; U = T B V
         for (int e = tid; e < DK * DT; e += kThreads) {
             const int c = e / DT, n = e % DT;
-            tS0[e] = S0[(size_t)c * DV + n0 + n];
-            tdS[e] = dS[(size_t)c * DV + n0 + n];
+            tS0[c * TP + n] = S0[(size_t)c * DV + n0 + n];
+            tdS[c * TP + n] = dS[(size_t)c * DV + n0 + n];
         }
         for (int e = tid; e < C * DT; e += kThreads) {
             const int r = e / DT, n = e % DT;
             const size_t o = ((first + t0 + r) * H + h) * DV + n0 + n;
-            tdO[e] = r < nvalid ? to_f32(dout[o]) : 0.f;
-            tV[e] = r < nvalid ? to_f32(v[o]) : 0.f;
+            tdO[r * TP + n] = r < nvalid ? to_f32(dout[o]) : 0.f;
+            tV[r * TP + n] = r < nvalid ? to_f32(v[o]) : 0.f;
         }
         __syncthreads();
         for (int e = tid; e < C * DT; e += kThreads) {
             const int j = e / DT, n = e % DT;
             float u = 0.f, ws = 0.f, kd = 0.f;
-            for (int m = 0; m <= j; ++m) u += f.T[j * C + m] * f.b[m] * tV[m * DT + n];
+            for (int m = 0; m <= j; ++m) u += f.T[j * C + m] * f.b[m] * tV[m * TP + n];
             for (int c = 0; c < DK; ++c) {
-                ws += f.W[j * DK + c] * tS0[c * DT + n];
-                kd += sKe[j * DK + c] * tdS[c * DT + n];
+                ws += f.W[j * LD + c] * tS0[c * TP + n];
+                kd += sKe[j * DK + c] * tdS[c * TP + n];
             }
-            tU[e] = u;
-            tWS[e] = ws;
-            tKd[e] = kd;
+            tU[j * TP + n] = u;
+            tWS[j * TP + n] = ws;
+            tKd[j * TP + n] = kd;
         }
         __syncthreads();
         // dU = scale M^T dO + K_end dS_out
         for (int e = tid; e < C * DT; e += kThreads) {
             const int j = e / DT, n = e % DT;
-            float acc = tKd[e];
-            for (int r = j; r < C; ++r) acc += scale * f.M[r * C + j] * tdO[r * DT + n];
-            tdU[e] = acc;
+            float acc = tKd[j * TP + n];
+            for (int r = j; r < C; ++r) acc += scale * f.M[r * C + j] * tdO[r * TP + n];
+            tdU[j * TP + n] = acc;
         }
         __syncthreads();
         // accumulate dQ', dK_end, dW over the tile's columns
@@ -268,9 +272,9 @@ bwd_grad_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
             const int r = e / DK, c = e % DK;
             float aq = 0.f, ak = 0.f, aw = 0.f;
             for (int n = 0; n < DT; ++n) {
-                aq += tdO[r * DT + n] * tS0[c * DT + n];
-                ak += (tU[r * DT + n] - tWS[r * DT + n]) * tdS[c * DT + n];
-                aw += tKd[r * DT + n] * tS0[c * DT + n];
+                aq += tdO[r * TP + n] * tS0[c * TP + n];
+                ak += (tU[r * TP + n] - tWS[r * TP + n]) * tdS[c * TP + n];
+                aw += tKd[r * TP + n] * tS0[c * TP + n];
             }
             sdQp[e] += scale * aq;
             sdKe[e] += ak;
@@ -278,7 +282,7 @@ bwd_grad_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
         }
         for (int c = tid; c < DK; c += kThreads) {
             float acc = 0.f;
-            for (int n = 0; n < DT; ++n) acc += tdS[c * DT + n] * tS0[c * DT + n];
+            for (int n = 0; n < DT; ++n) acc += tdS[c * TP + n] * tS0[c * TP + n];
             sdgC[c] += acc;
         }
         // dM += scale dO U^T;  dT += dU (B V)^T
@@ -286,8 +290,8 @@ bwd_grad_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
             const int r = e / C, j = e % C;
             float am = 0.f, at = 0.f;
             for (int n = 0; n < DT; ++n) {
-                am += tdO[r * DT + n] * tU[j * DT + n];
-                at += tdU[r * DT + n] * tV[j * DT + n];
+                am += tdO[r * TP + n] * tU[j * TP + n];
+                at += tdU[r * TP + n] * tV[j * TP + n];
             }
             sdM[e] += scale * am;
             sdT[e] += f.b[j] * at;
@@ -296,9 +300,9 @@ bwd_grad_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
         for (int j = tid / DT; j < C; j += kThreads / DT) {
             const int n = tid % DT;
             float y = 0.f;
-            for (int r = j; r < C; ++r) y += f.T[r * C + j] * tdU[r * DT + n];
+            for (int r = j; r < C; ++r) y += f.T[r * C + j] * tdU[r * TP + n];
             if (j < nvalid) dv_out[((first + t0 + j) * H + h) * DV + n0 + n] = f.b[j] * y;
-            float yv = y * tV[j * DT + n];
+            float yv = y * tV[j * TP + n];
             for (int o = DT / 2; o > 0; o >>= 1) yv += __shfl_xor_sync(0xffffffffu, yv, o);
             if (n == 0) sdb[j] += yv;
         }
@@ -309,7 +313,7 @@ bwd_grad_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
     for (int e = tid; e < C * C; e += kThreads) {
         const int r = e / C, j = e % C;
         float acc = 0.f;
-        for (int c = 0; c < DK; ++c) acc += sdQp[r * DK + c] * f.W[j * DK + c];
+        for (int c = 0; c < DK; ++c) acc += sdQp[r * DK + c] * f.W[j * LD + c];
         sdM[e] = j <= r ? sdM[e] - acc : 0.f;   // M is lower triangular (diagonal included)
     }
     for (int e = tid; e < C * DK; e += kThreads) {
@@ -323,7 +327,7 @@ bwd_grad_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
     for (int e = tid; e < C * C; e += kThreads) {
         const int r = e / C, j = e % C;
         float acc = 0.f;
-        for (int c = 0; c < DK; ++c) acc += sdW[r * DK + c] * exp2f(f.L[j * DK + c]) * f.k[j * DK + c];
+        for (int c = 0; c < DK; ++c) acc += sdW[r * DK + c] * exp2f(f.L[j * LD + c]) * f.k[j * LD + c];
         sdT[e] += f.b[j] * acc;
     }
     __syncthreads();
@@ -354,10 +358,12 @@ bwd_grad_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
             for (int m = 0; m < C; ++m) acc -= f.T[m * C + r] * sZ[m * C + j];
         sdT[e] = acc;
     }
-    for (int j = tid; j < C; j += kThreads) {
+    for (int j = tid >> 5; j < C; j += kThreads / 32) {   // one warp per row, lanes over channels
         float acc = 0.f;
-        for (int c = 0; c < DK; ++c) acc += sdW[j * DK + c] * exp2f(f.L[j * DK + c]) * f.k[j * DK + c];
-        sdb[j] += acc;
+        for (int c = tid & 31; c < DK; c += 32)
+            acc += sdW[j * DK + c] * exp2f(f.L[j * LD + c]) * f.k[j * LD + c];
+        acc = warp_sum(acc);
+        if ((tid & 31) == 0) sdb[j] += acc;
     }
     __syncthreads();
     // A = B P:  dbeta += rowsum(dA . P);  E = B dA (in place)
@@ -378,17 +384,17 @@ bwd_grad_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
     for (int e = tid; e < C * DK; e += kThreads) {
         const int j = e / DK, c = e % DK;
         if (j >= nvalid) continue;
-        const float Lj = f.L[e];
+        const float Lj = f.L[j * LD + c];
         float dk = 0.f, dq = 0.f;
         for (int m = 0; m < j; ++m) {
-            const float R = exp2f(Lj - f.L[m * DK + c]);
-            dk += sE[j * C + m] * R * f.k[m * DK + c];
-            dq += sdM[j * C + m] * R * f.k[m * DK + c];
+            const float R = exp2f(Lj - f.L[m * LD + c]);
+            dk += sE[j * C + m] * R * f.k[m * LD + c];
+            dq += sdM[j * C + m] * R * f.k[m * LD + c];
         }
-        dq += sdM[j * C + j] * f.k[e];
+        dq += sdM[j * C + j] * f.k[j * LD + c];
         for (int r = j; r < C; ++r) {
-            const float R = exp2f(f.L[r * DK + c] - Lj);
-            dk += (sE[r * C + j] * f.k[r * DK + c] + sdM[r * C + j] * f.q[r * DK + c]) * R;
+            const float R = exp2f(f.L[r * LD + c] - Lj);
+            dk += (sE[r * C + j] * f.k[r * LD + c] + sdM[r * C + j] * f.q[r * LD + c]) * R;
         }
         const float g = exp2f(Lj);
         dk += f.b[j] * sdW[e] * g + sdKe[e] * f.sg[c] * exp2f(f.LC[c] - Lj);
@@ -408,29 +414,29 @@ bwd_grad_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
 #pragma unroll
         for (int a = 0; a < C; ++a) Z[a] = 0.f;
         auto dR = [&](int a, int bb) {
-            float x = (sE[a * C + bb] * f.k[a * DK + c] + sdM[a * C + bb] * f.q[a * DK + c]) * f.k[bb * DK + c];
-            if (a == C - 1) x += sdKe[bb * DK + c] * sC * f.k[bb * DK + c];
+            float x = (sE[a * C + bb] * f.k[a * LD + c] + sdM[a * C + bb] * f.q[a * LD + c]) * f.k[bb * LD + c];
+            if (a == C - 1) x += sdKe[bb * DK + c] * sC * f.k[bb * LD + c];
             return x;
         };
         auto dg = [&](int r) {
-            float x = f.b[r] * sdW[r * DK + c] * f.k[r * DK + c] + sdQp[r * DK + c] * f.q[r * DK + c];
+            float x = f.b[r] * sdW[r * DK + c] * f.k[r * LD + c] + sdQp[r * DK + c] * f.q[r * LD + c];
             if (r == C - 1) x += sdgC[c] * sC;
             return x;
         };
 #pragma unroll
         for (int t = 0; t < C; ++t) {
             if (t > 0) {
-                const float am = exp2f(f.L[(t - 1) * DK + c] - (t > 1 ? f.L[(t - 2) * DK + c] : 0.f));
+                const float am = exp2f(f.L[(t - 1) * LD + c] - (t > 1 ? f.L[(t - 2) * LD + c] : 0.f));
 #pragma unroll
                 for (int a = 0; a < C; ++a) Z[a] = a >= t - 1 ? am * Z[a] + dR(a, t - 1) : 0.f;
             }
-            const float Lt = f.L[t * DK + c];
-            const float gprev = t > 0 ? exp2f(f.L[(t - 1) * DK + c]) : 1.f;
+            const float Lt = f.L[t * LD + c];
+            const float gprev = t > 0 ? exp2f(f.L[(t - 1) * LD + c]) : 1.f;
             float s1 = 0.f, s2 = 0.f;
 #pragma unroll
             for (int r = 0; r < C; ++r) {
                 if (r < t) continue;
-                const float R = exp2f(f.L[r * DK + c] - Lt);
+                const float R = exp2f(f.L[r * LD + c] - Lt);
                 s1 += dg(r) * R;
                 s2 += Z[r] * R;
             }

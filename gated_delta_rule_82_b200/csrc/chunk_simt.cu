@@ -58,6 +58,7 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
     extern __shared__ float smem[];
     simt::Factors<DK, C> f;
     f.bind(smem);
+    constexpr int LD = simt::Factors<DK, C>::LD;
     float* sv = smem + Sh::off_v;
     float* sUt = smem + Sh::off_Ut;
     float* sU = smem + Sh::off_U;
@@ -117,7 +118,7 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
         for (int e = tid; e < C * DVS; e += kSimtThreads) {
             int r = e / DVS, n = e % DVS;
             float acc = sUt[e];
-            for (int c = 0; c < DK; ++c) acc -= f.W[r * DK + c] * sS[c * DVS + n];
+            for (int c = 0; c < DK; ++c) acc -= f.W[r * LD + c] * sS[c * DVS + n];
             sU[e] = acc;
         }
         __syncthreads();
@@ -128,7 +129,7 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
                 int r = e / DVS, n = e % DVS;
                 if (r >= nvalid) continue;
                 float acc = 0.f;
-                for (int c = 0; c < DK; ++c) acc += exp2f(f.L[r * DK + c]) * f.q[r * DK + c] * sS[c * DVS + n];
+                for (int c = 0; c < DK; ++c) acc += exp2f(f.L[r * LD + c]) * f.q[r * LD + c] * sS[c * DVS + n];
                 for (int j = 0; j <= r; ++j) acc += f.M[r * C + j] * sU[j * DVS + n];
                 out[((first + t0 + r) * H + h) * DV + n0 + n] = from_f32<T>(scale * acc);
             }
@@ -140,7 +141,7 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
             int c = e / DVS, n = e % DVS;
             float LC = f.LC[c];
             float acc = exp2f(LC) * sS[e];
-            for (int r = 0; r < C; ++r) acc += exp2f(LC - f.L[r * DK + c]) * f.k[r * DK + c] * sU[r * DVS + n];
+            for (int r = 0; r < C; ++r) acc += exp2f(LC - f.L[r * LD + c]) * f.k[r * LD + c] * sU[r * DVS + n];
             sS[e] = f.sg[c] * acc;
         }
     }

@@ -18,25 +18,28 @@
 namespace ckda {
 namespace simt {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 256;   // >= 128 (one thread per channel) and >= the chunk
 constexpr float kFltMin = 1.17549435e-38f;
 
-// Shared-memory arrays of one chunk's factors (floats).
+// Shared-memory arrays of one chunk's factors (floats).  The rows of q', k', L and W are LD =
+// DK + 1 floats apart, so that loops whose lanes run over rows at a fixed channel (the A and M
+// products) hit distinct banks.
 template <int DK, int C>
 struct Factors {
-    float* q;    // q'  [C][DK]
-    float* k;    // k'  [C][DK]
-    float* L;    // L   [C][DK]
-    float* W;    // W   [C][DK]
+    static constexpr int LD = DK + 1;
+    float* q;    // q'  [C][LD]
+    float* k;    // k'  [C][LD]
+    float* L;    // L   [C][LD]
+    float* W;    // W   [C][LD]
     float* A;    // A   [C][C]
     float* M;    // M   [C][C]
     float* T;    // T   [C][C]
     float* b;    // beta [C]
     float* sg;   // sigma_C [DK]
     float* LC;   // L_C [DK]
-    static constexpr int floats = 4 * C * DK + 3 * C * C + C + 2 * DK;
+    static constexpr int floats = 4 * C * LD + 3 * C * C + C + 2 * DK;
     __device__ void bind(float* p) {
-        q = p; k = q + C * DK; L = k + C * DK; W = L + C * DK; A = W + C * DK; M = A + C * C;
+        q = p; k = q + C * LD; L = k + C * LD; W = L + C * LD; A = W + C * LD; M = A + C * C;
         T = M + C * C; b = T + C * C; sg = b + C; LC = sg + DK;
     }
 };
@@ -53,23 +56,52 @@ __device__ __forceinline__ void chunk_factors(const Factors<DK, C>& f, const Tin
                                               int nvalid, int H, int h, int G, int l2norm,
                                               const RopeParams& rp, const unsigned long long* sfreq,
                                               long long pos0, int gate_logits) {
+    constexpr int LD = Factors<DK, C>::LD;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     constexpr int NW = kThreads / 32;
-    for (int e = tid; e < C * DK; e += kThreads) {
-        const int r = e / DK, c = e % DK;
-        float qv = 0.f, kv = 0.f;
-        if (r < nvalid) {
-            const size_t row = ((first + t0 + r) * H + h) / G;
-            qv = to_f32(q[row * DK + c]);
-            kv = to_f32(k[row * DK + c]);
-        }
-        f.q[e] = qv;
-        f.k[e] = kv;
+    // the chunk's global loads are issued in batches before their values are used: q and k in
+    // groups of up to 8 elements per thread, beta, and the gates of this thread's channel
+    // (thread c < DK) for the first rows (the later rows are loaded, again in batches, during
+    // the gate prefix below)
+    constexpr int NQK = (C * DK + kThreads - 1) / kThreads;
+    constexpr int QG = NQK < 8 ? NQK : 8;
+    constexpr int AG = C < 16 ? C : 16;
+    auto gate_at = [&](int r) {
+        const size_t ia = ((first + t0 + r) * H + h) * DK + tid;
+        return r >= nvalid ? 1.f
+               : gate_logits ? gate_alpha(to_f32(static_cast<const Tin*>(alpha)[ia]))
+                             : static_cast<const float*>(alpha)[ia];
+    };
+    float av[AG];
+    float bv = tid < nvalid ? beta[(first + t0 + tid) * H + h] : 0.f;
+    if (tid < DK) {
+#pragma unroll
+        for (int r = 0; r < AG; ++r) av[r] = gate_at(r);
     }
-    for (int r = tid; r < C; r += kThreads) {
-        float bv = r < nvalid ? beta[(first + t0 + r) * H + h] : 0.f;
-        if (r < nvalid && gate_logits) bv = gate_beta(bv);   // beta = 2 sigma(b)
-        f.b[r] = bv;
+    for (int i0 = 0; i0 < NQK; i0 += QG) {
+        float qv[QG], kv[QG];
+#pragma unroll
+        for (int i = 0; i < QG; ++i) {
+            const int e = tid + (i0 + i) * kThreads, r = e / DK, c = e % DK;
+            qv[i] = kv[i] = 0.f;
+            if (e < C * DK && r < nvalid) {
+                const size_t row = ((first + t0 + r) * H + h) / G;
+                qv[i] = to_f32(q[row * DK + c]);
+                kv[i] = to_f32(k[row * DK + c]);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < QG; ++i) {
+            const int e = tid + (i0 + i) * kThreads, r = e / DK, c = e % DK;
+            if (e < C * DK) {
+                f.q[r * LD + c] = qv[i];
+                f.k[r * LD + c] = kv[i];
+            }
+        }
+    }
+    if (tid < C) {
+        if (tid < nvalid && gate_logits) bv = gate_beta(bv);   // beta = 2 sigma(b)
+        f.b[tid] = bv;
     }
     __syncthreads();
     // prologue per row (one warp per row): rotation, then L2 norm
@@ -80,8 +112,8 @@ __device__ __forceinline__ void chunk_factors(const Factors<DK, C>& f, const Tin
 #pragma unroll
         for (int m = 0; m < PER; ++m) {
             const int c = lane + 32 * m;
-            qr[m] = c < DK ? f.q[r * DK + c] : 0.f;
-            kr[m] = c < DK ? f.k[r * DK + c] : 0.f;
+            qr[m] = c < DK ? f.q[r * LD + c] : 0.f;
+            kr[m] = c < DK ? f.k[r * LD + c] : 0.f;
             if (rp.enabled && c < rp.rot_dims) {   // the first rot_dims channels rotate
                 int i, partner;
                 bool lo;
@@ -93,7 +125,7 @@ __device__ __forceinline__ void chunk_factors(const Factors<DK, C>& f, const Tin
                 }
                 float sn, cs;
                 rope_sincos(p, sfreq[i], &sn, &cs);
-                const float qp = f.q[r * DK + partner], kp = f.k[r * DK + partner];
+                const float qp = f.q[r * LD + partner], kp = f.k[r * LD + partner];
                 qr[m] = lo ? qr[m] * cs - qp * sn : qr[m] * cs + qp * sn;
                 kr[m] = lo ? kr[m] * cs - kp * sn : kr[m] * cs + kp * sn;
             }
@@ -111,25 +143,29 @@ __device__ __forceinline__ void chunk_factors(const Factors<DK, C>& f, const Tin
 #pragma unroll
         for (int m = 0; m < PER; ++m) {
             const int c = lane + 32 * m;
-            if (c < DK) { f.q[r * DK + c] = qr[m]; f.k[r * DK + c] = kr[m]; }
+            if (c < DK) { f.q[r * LD + c] = qr[m]; f.k[r * LD + c] = kr[m]; }
         }
     }
     __syncthreads();
     // gate prep: sign parity and log2-magnitude prefix per channel; absorb signs
-    for (int c = tid; c < DK; c += kThreads) {
+    if (tid < DK) {
+        const int c = tid;
         float L = 0.f, sg = 1.f;
-        for (int r = 0; r < C; ++r) {
-            float a = 1.f;
-            if (r < nvalid) {
-                const size_t ia = ((first + t0 + r) * H + h) * DK + c;
-                a = gate_logits ? gate_alpha(to_f32(static_cast<const Tin*>(alpha)[ia]))
-                                : static_cast<const float*>(alpha)[ia];
+#pragma unroll
+        for (int r0 = 0; r0 < C; r0 += AG) {
+            if (r0 > 0) {
+#pragma unroll
+                for (int r = 0; r < AG; ++r) av[r] = gate_at(r0 + r);
             }
-            if (a < 0.f) sg = -sg;
-            L += log2f(fmaxf(fabsf(a), kFltMin));
-            f.L[r * DK + c] = L;
-            f.q[r * DK + c] *= sg;
-            f.k[r * DK + c] *= sg;
+#pragma unroll
+            for (int r = 0; r < AG; ++r) {
+                const float a = av[r];
+                if (a < 0.f) sg = -sg;
+                L += log2f(fmaxf(fabsf(a), kFltMin));
+                f.L[(r0 + r) * LD + c] = L;
+                f.q[(r0 + r) * LD + c] *= sg;
+                f.k[(r0 + r) * LD + c] *= sg;
+            }
         }
         f.sg[c] = sg;
         f.LC[c] = L;
@@ -141,9 +177,9 @@ __device__ __forceinline__ void chunk_factors(const Factors<DK, C>& f, const Tin
         float a = 0.f, m = 0.f;
         if (j <= r) {
             for (int c = 0; c < DK; ++c) {
-                const float kk = f.k[j * DK + c] * exp2f(f.L[r * DK + c] - f.L[j * DK + c]);
-                a += f.k[r * DK + c] * kk;
-                m += f.q[r * DK + c] * kk;
+                const float kk = f.k[j * LD + c] * exp2f(f.L[r * LD + c] - f.L[j * LD + c]);
+                a += f.k[r * LD + c] * kk;
+                m += f.q[r * LD + c] * kk;
             }
             a = (j < r) ? a * f.b[r] : 0.f;
         }
@@ -171,8 +207,8 @@ __device__ __forceinline__ void chunk_factors(const Factors<DK, C>& f, const Tin
         const int r = e / DK, c = e % DK;
         float acc = 0.f;
         for (int j = 0; j <= r; ++j)
-            acc += f.T[r * C + j] * f.b[j] * exp2f(f.L[j * DK + c]) * f.k[j * DK + c];
-        f.W[e] = acc;
+            acc += f.T[r * C + j] * f.b[j] * exp2f(f.L[j * LD + c]) * f.k[j * LD + c];
+        f.W[r * LD + c] = acc;
     }
     __syncthreads();
 }

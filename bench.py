@@ -13,7 +13,8 @@ throughput (all ranks' tokens / the slowest rank's device time).
 The line also carries: the roofline of the one kernel a step launches (ckda_tc_fused, the whole
 forward; against the measured HBM bandwidth), the same work timed as two kernels in sequence,
 the decode step's HBM throughput on the batched-decode workload, the standalone q/k prologue's
-HBM throughput (rotation then L2 norm at the layer shape), the CKDA/KDA-range throughput ratio,
+HBM throughput (rotation then L2 norm at the layer shape), the backward's time at the layer
+shape, the CKDA/KDA-range throughput ratio,
 an end-to-end figure through the C ABI with host buffers, SM clocks sampled during the timed
 region, and (rank 0, one GPU) the float64 CPU oracle's throughput on bounded samples of the
 layer-shaped and long-context workloads, on all host cores and on one.
@@ -530,6 +531,27 @@ def main():
                          "traffic": ncu_traffic("qk_prologue_kernel"),
                          "algorithmic_bytes_per_launch": pro_bytes}}
         del pq, pqo, pko
+
+        # ---- backward at the layer shape: gradients of <dout, out> + <dhT, hT> ---------------
+        bw = synth.torch_fwd_inputs(B, T, H, dk, dv, kind=w["kind"], dtype="bf16", h0_std=0.02,
+                                    seed=6500 + rank, device=dev)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(6600 + rank)
+        dout = torch.randn((B, T, H, dv), generator=gen, device=dev).to(torch.bfloat16)
+        dhT = 0.02 * torch.randn((B, H, dk, dv), generator=gen, device=dev)
+        wsb = torch.empty(ck.bwd_workspace_bytes(B, T, H, dk, dv), dtype=torch.uint8, device=dev)
+        fnB = lambda i: ck.bwd_chunked(bw["q"], bw["k"], bw["v"], bw["alpha"], bw["beta"],
+                                       bw["h0"], dout, dhT, workspace=wsb)
+        for i in range(2):
+            fnB(i)
+        nB = max(3, args.steps // 10)
+        ms_b = event_time_ms(fnB, nB, stream) / nB
+        extras["backward"] = {
+            "workload": f"{w['name']} (B={B},T={T},H={H},dk=dv={dk}) with h0, dout and dhT: dq, dk, "
+                        "dv, dalpha, dbeta, dh0 in fp32 (CUDA cores, 16-token chunks)",
+            "ms": round(ms_b, 3), "mtok_s": round(B * T / (ms_b / 1e3) / 1e6, 3),
+            "over_forward": round(ms_b / ms_local, 1)}
+        del bw, dout, dhT, wsb
 
         # ---- batched decode: 256 sequences x 32 heads, dk = dv = 128 ------------------------
         wd = synth.WORKLOADS["decode_bf16"]

@@ -57,7 +57,7 @@ def parse():
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--no-extras", action="store_true",
                     help="skip decode / KDA-ratio / e2e / CPU-baseline legs")
-    ap.add_argument("--profile-case", choices=["fwd", "decode", "prologue"], default=None,
+    ap.add_argument("--profile-case", choices=["fwd", "decode", "prologue", "bwd"], default=None,
                     help="run only a few calls of one entry point (for ncu captures) and exit")
     return ap.parse_args()
 
@@ -274,6 +274,16 @@ def profile_case(case, calls, dev):
         state = 0.02 * torch.randn((wd["N"], wd["H"], 128, 128), device=dev)
         for i in range(calls):
             ck.decode_step(d["q"][i], d["k"][i], d["v"][i], d["alpha"][i], d["beta"][i], state)
+    elif case == "bwd":
+        w = WORKLOAD
+        s = synth.torch_fwd_inputs(w["B"], w["T"], w["H"], w["dk"], w["dv"], kind=w["kind"],
+                                   h0_std=0.02, seed=1, device=dev)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(2)
+        dout = torch.randn((w["B"], w["T"], w["H"], w["dv"]), generator=gen, device=dev).bfloat16()
+        dhT = 0.02 * torch.randn((w["B"], w["H"], w["dk"], w["dv"]), generator=gen, device=dev)
+        for _ in range(calls):
+            ck.bwd_chunked(s["q"], s["k"], s["v"], s["alpha"], s["beta"], s["h0"], dout, dhT)
     else:
         w = WORKLOAD
         s = synth.torch_fwd_inputs(w["B"], w["T"], w["H"], w["dk"], w["dv"], seed=1, device=dev)

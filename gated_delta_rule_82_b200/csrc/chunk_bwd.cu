@@ -4,11 +4,14 @@
 // The backward runs the chunked form in reverse (derived from the transition of the "Complex
 // KDA" paper summary, "Background"; the chunk factors are those of simt_chunk.cuh, with the gate
 // signs absorbed into q' and k' and every gate ratio taken as R_rj = exp2(L_r - L_j) <= 1):
-//   1. the forward replays the chunks and keeps the state entering each one (chunk_simt.cu);
+//   0. every chunk's factors are computed once, chunk-parallel, into a record in the workspace
+//      (W, K_end, T, beta, gamma_C, Q', M and P = A before beta);
+//   1. the forward replays the chunks from those records and keeps the state entering each one;
 //   2. a chain over the chunks in reverse carries the gradient of the state:
 //        dS_in = scale Q'^T dO + Diag(gamma_C) dS_out - W^T (K_end dS_out)
 //      (Q' = Q_gamma - M W, K_end,j = sigma_C R_Cj k'_j), column slices of S independent;
-//   3. every chunk then forms its input gradients from its entering state, dS_out and dO:
+//   3. every chunk then forms its input gradients from its record, its entering state, dS_out and
+//      dO:
 //        dQ' = scale dO S0^T,  dM = scale dO U^T - dQ' W^T,  dU = scale M^T dO + K_end dS_out,
 //        dK_end = (U - W S0) dS_out^T,  dW = -(K_end dS_out) S0^T - M^T dQ',
 //        dgamma_C = rowsum(dS_out . S0),  dT = dW (B K_gamma)^T + dU (B V)^T,
@@ -31,14 +34,151 @@ using simt::Factors;
 using simt::kThreads;
 constexpr int kBwdC = 16;
 
+// ---- the record of a chunk's factors (fp32, rows DK floats apart) ----------------------------------
+// [W | K_end | T | beta | gamma_C | Q' | M | P]: the replay reads the prefix up to Q', the chain up to
+// M, the chunk gradients all of it.  Every offset is a multiple of 4 floats.
+template <int DK, int C>
+struct Rec {
+    static constexpr int W = 0, KE = C * DK, T = 2 * C * DK, B = T + C * C, GC = B + C;
+    static constexpr int QP = GC + DK, M = QP + C * DK, P = M + C * C, floats = P + C * C;
+};
+
+// 16-byte copies global -> shared on the load/store path, completed per thread by commit groups.
+__device__ __forceinline__ void cp16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
+                 ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+// the first `floats` floats of a chunk record into shared memory (one commit group)
+__device__ __forceinline__ void load_record(float* dst, const float* src, int floats) {
+    for (int i = threadIdx.x; i < floats / 4; i += kThreads) cp16(dst + 4 * i, src + 4 * i);
+    cp_commit();
+}
+
+// ---- 0. every chunk's factors: one CTA per (b*h, chunk) -----------------------------------------
+template <typename T, int DK, int DV, int C>
+__global__ void __launch_bounds__(kThreads)
+bwd_factors_kernel(const T* __restrict__ q, const T* __restrict__ k, const void* __restrict__ alpha,
+                   const float* __restrict__ beta, float* __restrict__ recs, int T_len, int H,
+                   int G, int l2norm, RopeParams rp, long long pos_offset, int gate_logits) {
+    using R = Rec<DK, C>;
+    constexpr int LD = Factors<DK, C>::LD;
+    extern __shared__ float smem[];
+    Factors<DK, C> f;
+    f.bind(smem);
+    __shared__ unsigned long long sfreq[DK / 2];
+    const int nchunks = (T_len + C - 1) / C;
+    const int bh = blockIdx.x / nchunks, ch = blockIdx.x % nchunks;
+    const int b = bh / H, h = bh % H;
+    const int t0 = ch * C, nvalid = min(C, T_len - t0);
+    const int tid = threadIdx.x;
+    if (rp.enabled)
+        for (int i = tid; i < DK / 2; i += kThreads) sfreq[i] = rp.turns[i];
+    float* rec = recs + ((size_t)bh * nchunks + ch) * R::floats;
+    simt::chunk_prep<T, DK, C>(f, q, k, alpha, beta, (size_t)b * T_len, t0, nvalid, H, h, G,
+                               l2norm, rp, sfreq, pos_offset + t0, gate_logits);
+    simt::chunk_products<DK, C>(f, rec + R::P);   // P = A before beta, straight to the record
+    for (int e = tid; e < C * DK; e += kThreads) {
+        const int r = e / DK, c = e % DK;
+        float qp = exp2f(f.L[r * LD + c]) * f.q[r * LD + c];   // Q' = Q_gamma - M W
+        for (int j = 0; j <= r; ++j) qp -= f.M[r * C + j] * f.W[j * LD + c];
+        rec[R::W + e] = f.W[r * LD + c];
+        rec[R::KE + e] = f.sg[c] * exp2f(f.LC[c] - f.L[r * LD + c]) * f.k[r * LD + c];
+        rec[R::QP + e] = qp;
+    }
+    for (int e = tid; e < C * C; e += kThreads) {
+        rec[R::T + e] = f.T[e];
+        rec[R::M + e] = f.M[e];
+    }
+    for (int r = tid; r < C; r += kThreads) rec[R::B + r] = f.b[r];
+    for (int c = tid; c < DK; c += kThreads) rec[R::GC + c] = f.sg[c] * exp2f(f.LC[c]);
+}
+
+// ---- 1. the forward replay: one CTA per (b*h, DVS columns of the state) ----------------------------
+//   U~ = T B V,  U = U~ - W S,  S <- Diag(gamma_C) S + K_end^T U;  the state entering every chunk is
+//   written to ws_S.  The next chunk's record is fetched while this one is used.
+template <int DK, int DV, int C>
+struct ReplayShape {
+    static constexpr int DVS = DV < 16 ? DV : 16;
+    static constexpr int REC = Rec<DK, C>::QP;               // the part of a record the replay reads
+    static constexpr int off_v = 2 * REC;                    // two record stages, then V [C][DVS]
+    static constexpr int off_ut = off_v + C * DVS;           // U~ [C][DVS]
+    static constexpr int off_u = off_ut + C * DVS;           // U  [C][DVS]
+    static constexpr int off_s = off_u + C * DVS;            // S  [DK][DVS]
+    static constexpr int total = off_s + DK * DVS;
+    static constexpr size_t bytes = sizeof(float) * (size_t)total;
+};
+
+template <typename T, int DK, int DV, int C>
+__global__ void __launch_bounds__(kThreads)
+bwd_replay_kernel(const T* __restrict__ v, const float* __restrict__ h0,
+                  const float* __restrict__ recs, float* __restrict__ ws_S, int T_len, int H) {
+    using R = Rec<DK, C>;
+    using Sh = ReplayShape<DK, DV, C>;
+    constexpr int DVS = Sh::DVS;
+    extern __shared__ float smem[];
+    float* sv = smem + Sh::off_v;
+    float* sUt = smem + Sh::off_ut;
+    float* sU = smem + Sh::off_u;
+    float* sS = smem + Sh::off_s;
+    const int bh = blockIdx.x, b = bh / H, h = bh % H;
+    const int n0 = blockIdx.y * DVS;
+    const int tid = threadIdx.x;
+    const int nchunks = (T_len + C - 1) / C;
+    const float* rec0 = recs + (size_t)bh * nchunks * R::floats;
+    for (int e = tid; e < DK * DVS; e += kThreads)
+        sS[e] = h0 ? h0[((size_t)bh * DK + e / DVS) * DV + n0 + e % DVS] : 0.f;
+    load_record(smem, rec0, Sh::REC);
+    for (int ch = 0; ch < nchunks; ++ch) {
+        const float* rf = smem + (ch & 1) * Sh::REC;
+        if (ch + 1 < nchunks) {
+            load_record(smem + ((ch + 1) & 1) * Sh::REC, rec0 + (size_t)(ch + 1) * R::floats, Sh::REC);
+            cp_wait<1>();
+        } else {
+            cp_wait<0>();
+        }
+        const int t0 = ch * C, nvalid = min(C, T_len - t0);
+        float* dst = ws_S + ((size_t)bh * nchunks + ch) * DK * DV + n0;
+        for (int e = tid; e < DK * DVS; e += kThreads) dst[(e / DVS) * DV + e % DVS] = sS[e];
+        for (int e = tid; e < C * DVS; e += kThreads) {
+            const int r = e / DVS, n = e % DVS;
+            sv[e] = r < nvalid ? to_f32(v[(((size_t)b * T_len + t0 + r) * H + h) * DV + n0 + n]) : 0.f;
+        }
+        __syncthreads();
+        for (int e = tid; e < C * DVS; e += kThreads) {
+            const int r = e / DVS, n = e % DVS;
+            float acc = 0.f;
+            for (int j = 0; j <= r; ++j) acc += rf[R::T + r * C + j] * rf[R::B + j] * sv[j * DVS + n];
+            sUt[e] = acc;
+        }
+        __syncthreads();
+        for (int e = tid; e < C * DVS; e += kThreads) {
+            const int r = e / DVS, n = e % DVS;
+            float acc = sUt[e];
+            for (int c = 0; c < DK; ++c) acc -= rf[R::W + r * DK + c] * sS[c * DVS + n];
+            sU[e] = acc;
+        }
+        __syncthreads();
+        for (int e = tid; e < DK * DVS; e += kThreads) {
+            const int c = e / DVS, n = e % DVS;
+            float acc = rf[R::GC + c] * sS[e];
+            for (int r = 0; r < C; ++r) acc += rf[R::KE + r * DK + c] * sU[r * DVS + n];
+            sS[e] = acc;
+        }
+        __syncthreads();   // this stage is refilled by the next iteration's prefetch
+    }
+}
+
 // ---- 2. the state-gradient chain: one CTA per (b*h, DVS columns of the state) ----------------
 template <int DK, int DV, int C>
 struct ChainShape {
     static constexpr int DVS = DV < 16 ? DV : 16;
-    static constexpr int off_qp = Factors<DK, C>::floats;   // Q'   [C][DK]
-    static constexpr int off_do = off_qp + C * DK;          // dO   [C][DVS]
-    static constexpr int off_kd = off_do + C * DVS;         // K_end dS_out [C][DVS]
-    static constexpr int off_ds = off_kd + C * DVS;         // dS_out [DK][DVS]
+    static constexpr int REC = Rec<DK, C>::M;                 // the part of a record the chain reads
+    static constexpr int off_do = 2 * REC;                    // two record stages, then dO [C][DVS]
+    static constexpr int off_kd = off_do + C * DVS;           // K_end dS_out [C][DVS]
+    static constexpr int off_ds = off_kd + C * DVS;           // dS_out [DK][DVS]
     static constexpr int total = off_ds + DK * DVS;
     static constexpr size_t bytes = sizeof(float) * (size_t)total;
 };
@@ -46,68 +186,57 @@ struct ChainShape {
 // ws_dS: [B*H][NT][DK][DV] fp32, the gradient with respect to each chunk's end state.
 template <typename T, int DK, int DV, int C>
 __global__ void __launch_bounds__(kThreads)
-bwd_chain_kernel(const T* __restrict__ q, const T* __restrict__ k, const void* __restrict__ alpha,
-                 const float* __restrict__ beta, const T* __restrict__ dout,
-                 const float* __restrict__ dhT, float* __restrict__ dh0, float* __restrict__ ws_dS,
-                 int T_len, int H, int G, int l2norm, RopeParams rp, float scale,
-                 long long pos_offset, int gate_logits) {
+bwd_chain_kernel(const T* __restrict__ dout, const float* __restrict__ dhT,
+                 float* __restrict__ dh0, const float* __restrict__ recs, float* __restrict__ ws_dS,
+                 int T_len, int H, float scale) {
+    using R = Rec<DK, C>;
     using Sh = ChainShape<DK, DV, C>;
     constexpr int DVS = Sh::DVS;
-    constexpr int LD = Factors<DK, C>::LD;
     extern __shared__ float smem[];
-    Factors<DK, C> f;
-    f.bind(smem);
-    float* sQp = smem + Sh::off_qp;
     float* sdO = smem + Sh::off_do;
     float* sKd = smem + Sh::off_kd;
     float* sdS = smem + Sh::off_ds;
-    __shared__ unsigned long long sfreq[DK / 2];
     const int bh = blockIdx.x, b = bh / H, h = bh % H;
     const int n0 = blockIdx.y * DVS;
     const int tid = threadIdx.x;
-    const size_t first = (size_t)b * T_len;
-    if (rp.enabled)
-        for (int i = tid; i < DK / 2; i += kThreads) sfreq[i] = rp.turns[i];
+    const int nchunks = (T_len + C - 1) / C;
+    const float* rec0 = recs + (size_t)bh * nchunks * R::floats;
     for (int e = tid; e < DK * DVS; e += kThreads)
         sdS[e] = dhT ? dhT[((size_t)bh * DK + e / DVS) * DV + n0 + e % DVS] : 0.f;
-    const int nchunks = (T_len + C - 1) / C;
-    for (int ch = nchunks - 1; ch >= 0; --ch) {
-        const int t0 = ch * C;
-        const int nvalid = min(C, T_len - t0);
-        __syncthreads();
+    load_record(smem, rec0 + (size_t)(nchunks - 1) * R::floats, Sh::REC);
+    for (int ch = nchunks - 1, it = 0; ch >= 0; --ch, ++it) {
+        const float* rf = smem + (it & 1) * Sh::REC;
+        if (ch > 0) {
+            load_record(smem + ((it + 1) & 1) * Sh::REC, rec0 + (size_t)(ch - 1) * R::floats, Sh::REC);
+            cp_wait<1>();
+        } else {
+            cp_wait<0>();
+        }
+        const int t0 = ch * C, nvalid = min(C, T_len - t0);
         float* dst = ws_dS + ((size_t)bh * nchunks + ch) * DK * DV + n0;
         for (int e = tid; e < DK * DVS; e += kThreads) dst[(e / DVS) * DV + e % DVS] = sdS[e];
         for (int e = tid; e < C * DVS; e += kThreads) {
             const int r = e / DVS, n = e % DVS;
-            sdO[e] = r < nvalid ? to_f32(dout[((first + t0 + r) * H + h) * DV + n0 + n]) : 0.f;
+            sdO[e] = r < nvalid ? to_f32(dout[(((size_t)b * T_len + t0 + r) * H + h) * DV + n0 + n]) : 0.f;
         }
-        simt::chunk_factors<T, DK, C>(f, q, k, alpha, beta, first, t0, nvalid, H, h, G, l2norm,
-                                      rp, sfreq, pos_offset + t0, gate_logits);
-        // Q' = Q_gamma - M W;  K_end dS_out
-        for (int e = tid; e < C * DK; e += kThreads) {
-            const int r = e / DK, c = e % DK;
-            float acc = exp2f(f.L[r * LD + c]) * f.q[r * LD + c];
-            for (int j = 0; j <= r; ++j) acc -= f.M[r * C + j] * f.W[j * LD + c];
-            sQp[e] = acc;
-        }
-        for (int e = tid; e < C * DVS; e += kThreads) {
+        __syncthreads();
+        for (int e = tid; e < C * DVS; e += kThreads) {   // K_end dS_out
             const int j = e / DVS, n = e % DVS;
             float acc = 0.f;
-            for (int c = 0; c < DK; ++c)
-                acc += f.sg[c] * exp2f(f.LC[c] - f.L[j * LD + c]) * f.k[j * LD + c] * sdS[c * DVS + n];
+            for (int c = 0; c < DK; ++c) acc += rf[R::KE + j * DK + c] * sdS[c * DVS + n];
             sKd[e] = acc;
         }
         __syncthreads();
         // dS_in = scale Q'^T dO + Diag(gamma_C) dS_out - W^T (K_end dS_out)
         for (int e = tid; e < DK * DVS; e += kThreads) {
             const int c = e / DVS, n = e % DVS;
-            float acc = f.sg[c] * exp2f(f.LC[c]) * sdS[e];
+            float acc = rf[R::GC + c] * sdS[e];
             for (int r = 0; r < C; ++r)
-                acc += scale * sQp[r * DK + c] * sdO[r * DVS + n] - f.W[r * LD + c] * sKd[r * DVS + n];
+                acc += scale * rf[R::QP + r * DK + c] * sdO[r * DVS + n] - rf[R::W + r * DK + c] * sKd[r * DVS + n];
             sdS[e] = acc;   // each element is read only by its own thread above
         }
+        __syncthreads();   // this stage is refilled by the next iteration's prefetch
     }
-    __syncthreads();
     if (dh0)
         for (int e = tid; e < DK * DVS; e += kThreads)
             dh0[((size_t)bh * DK + e / DVS) * DV + n0 + e % DVS] = sdS[e];
@@ -143,14 +272,16 @@ struct GradShape {
     static constexpr size_t bytes = sizeof(float) * (size_t)total;
 };
 
-// ws_S, ws_dS: [B*H][NT][DK][DV] fp32 (entering state, end-state gradient of each chunk);
-// ws_dq, ws_dk: [B*T*H][DK] fp32 gradients of the prepared q^, k^ per value head.
+// recs: the chunk records; ws_S, ws_dS: [B*H][NT][DK][DV] fp32 (entering state, end-state
+// gradient of each chunk); ws_dq, ws_dk: [B*T*H][DK] fp32 gradients of the prepared q^, k^ per
+// value head.
 template <typename T, int DK, int DV, int C>
 __global__ void __launch_bounds__(kThreads)
 bwd_grad_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                 const void* __restrict__ alpha, const float* __restrict__ beta,
-                const T* __restrict__ dout, const float* __restrict__ ws_S,
-                const float* __restrict__ ws_dS, float* __restrict__ ws_dq,
+                const T* __restrict__ dout, const float* __restrict__ recs,
+                const float* __restrict__ ws_S, const float* __restrict__ ws_dS,
+                float* __restrict__ ws_dq,
                 float* __restrict__ ws_dk, float* __restrict__ dv_out,
                 float* __restrict__ dalpha, float* __restrict__ dbeta, int T_len, int H, int G,
                 int l2norm, RopeParams rp, float scale, long long pos_offset, int gate_logits) {
@@ -191,20 +322,33 @@ bwd_grad_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
     const size_t first = (size_t)b * T_len;
     if (rp.enabled)
         for (int i = tid; i < DK / 2; i += kThreads) sfreq[i] = rp.turns[i];
-    simt::chunk_factors<T, DK, C>(f, q, k, alpha, beta, first, t0, nvalid, H, h, G, l2norm, rp,
-                                  sfreq, pos_offset + t0, gate_logits);
+    // the record's T, M, P, Q' and K_end land while the chunk's rows are prepared; W goes to its
+    // padded rows through registers
+    {
+        using R = Rec<DK, C>;
+        const float* rec = recs + ((size_t)bh * nchunks + ch) * R::floats;
+        for (int i = tid; i < C * C / 4; i += kThreads) {
+            cp16(f.T + 4 * i, rec + R::T + 4 * i);
+            cp16(f.M + 4 * i, rec + R::M + 4 * i);
+            cp16(sP + 4 * i, rec + R::P + 4 * i);
+        }
+        for (int i = tid; i < C * DK / 4; i += kThreads) {
+            cp16(sQp + 4 * i, rec + R::QP + 4 * i);
+            cp16(sKe + 4 * i, rec + R::KE + 4 * i);
+        }
+        cp_commit();
+        for (int e = tid; e < C * DK; e += kThreads) f.W[(e / DK) * LD + e % DK] = rec[R::W + e];
+    }
+    simt::chunk_prep<T, DK, C>(f, q, k, alpha, beta, first, t0, nvalid, H, h, G, l2norm, rp,
+                               sfreq, pos_offset + t0, gate_logits);
+    cp_wait<0>();
     auto gate = [&](int r, int c) {   // alpha of row r < nvalid, channel c
         const size_t ia = ((first + t0 + r) * H + h) * DK + c;
         return gate_logits ? gate_alpha(to_f32(static_cast<const T*>(alpha)[ia]))
                            : static_cast<const float*>(alpha)[ia];
     };
-    // Q', K_end, P, the running sign products; zero the accumulators
+    // the running sign products; zero the accumulators
     for (int e = tid; e < C * DK; e += kThreads) {
-        const int r = e / DK, c = e % DK;
-        float acc = exp2f(f.L[r * LD + c]) * f.q[r * LD + c];
-        for (int j = 0; j <= r; ++j) acc -= f.M[r * C + j] * f.W[j * LD + c];
-        sQp[e] = acc;
-        sKe[e] = f.sg[c] * exp2f(f.LC[c] - f.L[r * LD + c]) * f.k[r * LD + c];
         sdQp[e] = 0.f;
         sdKe[e] = 0.f;
         sdW[e] = 0.f;
@@ -218,12 +362,6 @@ bwd_grad_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
         sdgC[c] = 0.f;
     }
     for (int e = tid; e < C * C; e += kThreads) {
-        const int r = e / C, j = e % C;
-        float p = 0.f;
-        if (j < r)
-            for (int c = 0; c < DK; ++c)
-                p += f.k[r * LD + c] * f.k[j * LD + c] * exp2f(f.L[r * LD + c] - f.L[j * LD + c]);
-        sP[e] = p;
         sdM[e] = 0.f;
         sdT[e] = 0.f;
     }
@@ -537,39 +675,49 @@ bwd_prologue_kernel(const T* __restrict__ q, const T* __restrict__ k,
     }
 }
 
-template <int DK, int DV>
-struct BwdSizes {
-    static constexpr size_t chain = ChainShape<DK, DV, kBwdC>::bytes;
-    static constexpr size_t grad = GradShape<DK, DV, kBwdC>::bytes;
-};
+template <typename K>
+cudaError_t set_smem(K kernel, size_t bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
 
 template <typename T, int DK, int DV>
 cudaError_t launch_bwd_t(const BwdArgs& a, const BwdLayout& w, cudaStream_t stream) {
+    constexpr int C = kBwdC;
     const int BH = a.B * a.H;
-    const int nt = (a.T_len + kBwdC - 1) / kBwdC;
+    const int nt = (a.T_len + C - 1) / C;
+    const T* q = static_cast<const T*>(a.q);
+    const T* k = static_cast<const T*>(a.k);
+    const T* v = static_cast<const T*>(a.v);
+    const T* dout = static_cast<const T*>(a.dout);
+    // 0. every chunk's factors
+    auto factors = bwd_factors_kernel<T, DK, DV, C>;
+    constexpr size_t fbytes = sizeof(float) * Factors<DK, C>::floats;
+    cudaError_t e = set_smem(factors, fbytes);
+    if (e != cudaSuccess) return e;
+    factors<<<(unsigned)((size_t)BH * nt), kThreads, fbytes, stream>>>(
+        q, k, a.alpha, a.beta, w.records, a.T_len, a.H, a.G, a.l2norm, a.rp, a.pos_offset,
+        a.gate_logits);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // 1. the forward replay, keeping every chunk's entering state
-    SimtArgs fa{a.q, a.k, a.v, a.alpha, a.beta, a.h0, nullptr, nullptr, w.states, a.B, a.T_len,
-                nullptr, a.H, a.G, a.l2norm, a.rp, a.scale, a.pos_offset, a.gate_logits};
-    cudaError_t e = launch_chunk_simt(fa, DK, DV, kBwdC, a.dtype, stream);
-    if (e != cudaSuccess) return e;
+    using RS = ReplayShape<DK, DV, C>;
+    auto replay = bwd_replay_kernel<T, DK, DV, C>;
+    if ((e = set_smem(replay, RS::bytes)) != cudaSuccess) return e;
+    replay<<<dim3(BH, DV / RS::DVS), kThreads, RS::bytes, stream>>>(v, a.h0, w.records, w.states,
+                                                                   a.T_len, a.H);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // 2. the state-gradient chain
-    auto chain = bwd_chain_kernel<T, DK, DV, kBwdC>;
-    e = cudaFuncSetAttribute(chain, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)BwdSizes<DK, DV>::chain);
-    if (e != cudaSuccess) return e;
-    chain<<<dim3(BH, DV / ChainShape<DK, DV, kBwdC>::DVS), kThreads, BwdSizes<DK, DV>::chain,
-            stream>>>(static_cast<const T*>(a.q), static_cast<const T*>(a.k), a.alpha, a.beta,
-                      static_cast<const T*>(a.dout), a.dhT, a.dh0, w.dstates, a.T_len, a.H, a.G,
-                      a.l2norm, a.rp, a.scale, a.pos_offset, a.gate_logits);
+    using CS = ChainShape<DK, DV, C>;
+    auto chain = bwd_chain_kernel<T, DK, DV, C>;
+    if ((e = set_smem(chain, CS::bytes)) != cudaSuccess) return e;
+    chain<<<dim3(BH, DV / CS::DVS), kThreads, CS::bytes, stream>>>(
+        dout, a.dhT, a.dh0, w.records, w.dstates, a.T_len, a.H, a.scale);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // 3. every chunk's gradients
-    auto grad = bwd_grad_kernel<T, DK, DV, kBwdC>;
-    e = cudaFuncSetAttribute(grad, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)BwdSizes<DK, DV>::grad);
-    if (e != cudaSuccess) return e;
-    grad<<<(unsigned)((size_t)BH * nt), kThreads, BwdSizes<DK, DV>::grad, stream>>>(
-        static_cast<const T*>(a.q), static_cast<const T*>(a.k), static_cast<const T*>(a.v),
-        a.alpha, a.beta, static_cast<const T*>(a.dout), w.states, w.dstates, w.dq, w.dk, a.dv,
+    using GS = GradShape<DK, DV, C>;
+    auto grad = bwd_grad_kernel<T, DK, DV, C>;
+    if ((e = set_smem(grad, GS::bytes)) != cudaSuccess) return e;
+    grad<<<(unsigned)((size_t)BH * nt), kThreads, GS::bytes, stream>>>(
+        q, k, v, a.alpha, a.beta, dout, w.records, w.states, w.dstates, w.dq, w.dk, a.dv,
         a.dalpha, a.dbeta, a.T_len, a.H, a.G, a.l2norm, a.rp, a.scale, a.pos_offset,
         a.gate_logits);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -578,8 +726,8 @@ cudaError_t launch_bwd_t(const BwdArgs& a, const BwdLayout& w, cudaStream_t stre
     const long long warps = 2 * rows;
     bwd_prologue_kernel<T, DK><<<(unsigned)((warps + kThreads / 32 - 1) / (kThreads / 32)),
                                  kThreads, 0, stream>>>(
-        static_cast<const T*>(a.q), static_cast<const T*>(a.k), w.dq, w.dk, a.dq_out, a.dk_out,
-        a.T_len, a.H / a.G, a.G, rows, a.l2norm, a.rp, a.pos_offset);
+        q, k, w.dq, w.dk, a.dq_out, a.dk_out, a.T_len, a.H / a.G, a.G, rows, a.l2norm, a.rp,
+        a.pos_offset);
     return cudaGetLastError();
 }
 
@@ -608,21 +756,25 @@ cudaError_t bwd_dispatch(int dk, int dv, const BwdArgs& a, const BwdLayout& w,
 
 }  // namespace
 
-// Workspace of the backward: the entering state and the end-state gradient of every chunk of 16
-// tokens ([B*H][ceil(T/16)][dk][dv] fp32 each), then the gradients of the prepared q^ and k^ per
-// value head ([B*T*H][dk] fp32 each); every part 256-byte aligned.
+// Workspace of the backward: the factor record of every chunk of 16 tokens
+// ([B*H][ceil(T/16)][3*16*dk + 3*16*16 + 16 + dk] fp32), the entering state and the end-state
+// gradient of every chunk ([B*H][ceil(T/16)][dk][dv] fp32 each), then the gradients of the
+// prepared q^ and k^ per value head ([B*T*H][dk] fp32 each); every part 256-byte aligned.
 BwdLayout bwd_layout(void* ws, int B, int T_len, int H, int dk, int dv) {
     auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    constexpr size_t C = kBwdC;
     const size_t nt = (size_t)(T_len + kBwdC - 1) / kBwdC;
+    const size_t rec = up((size_t)B * H * nt * (3 * C * dk + 3 * C * C + C + dk) * sizeof(float));
     const size_t st = up((size_t)B * H * nt * dk * dv * sizeof(float));
     const size_t gr = up((size_t)B * T_len * H * dk * sizeof(float));
     BwdLayout w;
     uint8_t* p = static_cast<uint8_t*>(ws);
-    w.states = reinterpret_cast<float*>(p);
-    w.dstates = reinterpret_cast<float*>(p + st);
-    w.dq = reinterpret_cast<float*>(p + 2 * st);
-    w.dk = reinterpret_cast<float*>(p + 2 * st + gr);
-    w.bytes = 2 * st + 2 * gr;
+    w.records = reinterpret_cast<float*>(p);
+    w.states = reinterpret_cast<float*>(p + rec);
+    w.dstates = reinterpret_cast<float*>(p + rec + st);
+    w.dq = reinterpret_cast<float*>(p + rec + 2 * st);
+    w.dk = reinterpret_cast<float*>(p + rec + 2 * st + gr);
+    w.bytes = rec + 2 * st + 2 * gr;
     return w;
 }
 

@@ -43,15 +43,13 @@ struct SimtShape {
     static constexpr size_t bytes = sizeof(float) * (size_t)total;
 };
 
-// states: nullable; when given, the state entering each chunk ([B*H][ceil(T/C)][DK][DV] fp32,
-// the CTA's columns) is written there (the backward replays the chunks from them).  out and hT
-// are nullable.
+// out and hT are nullable.
 template <typename T, int DK, int DV, int C>
 __global__ void __launch_bounds__(kSimtThreads)
 chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                   const void* __restrict__ alpha, const float* __restrict__ beta,
                   const float* __restrict__ h0, T* __restrict__ out, float* __restrict__ hT,
-                  float* __restrict__ states, int T_len, const int* cu, int H, int G, int l2norm,
+                  int T_len, const int* cu, int H, int G, int l2norm,
                   RopeParams rp, float scale, long long pos_offset, int gate_logits) {
     using Sh = SimtShape<DK, DV, C>;
     constexpr int DVS = Sh::DVS;
@@ -91,10 +89,6 @@ chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
         const int t0 = ch * C;
         const int nvalid = min(C, len - t0);
         __syncthreads();
-        if (states) {
-            float* dst = states + ((size_t)bh * nchunks + ch) * DK * DV + n0;
-            for (int e = tid; e < DK * DVS; e += kSimtThreads) dst[(e / DVS) * DV + e % DVS] = sS[e];
-        }
         for (int e = tid; e < C * DVS; e += kSimtThreads) {
             int r = e / DVS, n = e % DVS;
             float vv = 0.f;
@@ -164,7 +158,7 @@ cudaError_t launch_simt_t(const SimtArgs& a, cudaStream_t stream) {
     dim3 grid(a.B * a.H, DV / Sh::DVS);
     kern<<<grid, kSimtThreads, Sh::bytes, stream>>>(
         static_cast<const T*>(a.q), static_cast<const T*>(a.k), static_cast<const T*>(a.v),
-        a.alpha, a.beta, a.h0, static_cast<T*>(a.out), a.hT, a.states, a.T_len, a.cu, a.H, a.G,
+        a.alpha, a.beta, a.h0, static_cast<T*>(a.out), a.hT, a.T_len, a.cu, a.H, a.G,
         a.l2norm, a.rp, a.scale, a.pos_offset, a.gate_logits);
     return cudaGetLastError();
 }
@@ -215,7 +209,7 @@ cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const
                               const RopeParams& rp, float scale, long long pos_offset,
                               int gate_logits, ckda_dtype dtype, const PackedSeqs& pk,
                               cudaStream_t stream) {
-    SimtArgs a{q, k, v, alpha, beta, h0, out, hT, nullptr,
+    SimtArgs a{q, k, v, alpha, beta, h0, out, hT,
                pk.cu ? pk.n : B,   // one CTA row per packed sequence
                T_len, pk.cu, H, G, l2norm, rp, scale, pos_offset, gate_logits};
     return launch_chunk_simt(a, dk, dv, chunk, dtype, stream);

@@ -26,14 +26,12 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, const voi
                           int H, int G, int dk, int dv, int l2norm, const RopeParams& rp, float scale,
                           int gate_logits, ckda_dtype dtype, cudaStream_t stream);
 
-// Arguments of the CUDA-core chunked forward.  states: nullable; when given, the state entering
-// each chunk is written there ([B*H][ceil(T/chunk)][dk][dv] fp32).  out and hT are nullable.
+// Arguments of the CUDA-core chunked forward.  out and hT are nullable.
 struct SimtArgs {
     const void *q, *k, *v, *alpha;
     const float *beta, *h0;
     void* out;
     float* hT;
-    float* states;
     int B, T_len;
     const int* cu;   // packed sequences (B = their count), or nullptr
     int H, G, l2norm;
@@ -66,7 +64,7 @@ struct BwdArgs {
     ckda_dtype dtype;
 };
 struct BwdLayout {
-    float *states, *dstates, *dq, *dk;
+    float *records, *states, *dstates, *dq, *dk;
     size_t bytes;
 };
 BwdLayout bwd_layout(void* ws, int B, int T_len, int H, int dk, int dv);

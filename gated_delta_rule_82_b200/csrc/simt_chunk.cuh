@@ -46,10 +46,11 @@ struct Factors {
 
 // Rows r < nvalid of q and k (value head h reads q/k row (token * H + h) / G), beta of head h,
 // alpha from fp32 values or `dtype` logits; rows past nvalid are identity steps.  Then the
-// prologue (rotation at position pos0 + r, L2 norm), the gate prefix with the signs absorbed, A,
-// M, T and W.  `first` is the token index of row 0 on the token axis.  Ends with a barrier.
+// prologue (rotation at position pos0 + r, L2 norm) and the gate prefix with the signs absorbed:
+// q', k', L, beta, sigma_C and L_C.  `first` is the token index of row 0 on the token axis.  Ends
+// with a barrier.
 template <typename Tin, int DK, int C>
-__device__ __forceinline__ void chunk_factors(const Factors<DK, C>& f, const Tin* __restrict__ q,
+__device__ __forceinline__ void chunk_prep(const Factors<DK, C>& f, const Tin* __restrict__ q,
                                               const Tin* __restrict__ k,
                                               const void* __restrict__ alpha,
                                               const float* __restrict__ beta, size_t first, int t0,
@@ -171,6 +172,14 @@ __device__ __forceinline__ void chunk_factors(const Factors<DK, C>& f, const Tin
         f.LC[c] = L;
     }
     __syncthreads();
+}
+
+// A, M, T and W of a chunk whose q', k', L and beta chunk_prep has filled in; P (nullable, [C][C])
+// receives A before the row scaling by beta.  Ends with a barrier.
+template <int DK, int C>
+__device__ __forceinline__ void chunk_products(const Factors<DK, C>& f, float* P = nullptr) {
+    constexpr int LD = Factors<DK, C>::LD;
+    const int tid = threadIdx.x;
     // A (strictly lower) and M (lower incl. diagonal)
     for (int e = tid; e < C * C; e += kThreads) {
         const int r = e / C, j = e % C;
@@ -181,9 +190,10 @@ __device__ __forceinline__ void chunk_factors(const Factors<DK, C>& f, const Tin
                 a += f.k[r * LD + c] * kk;
                 m += f.q[r * LD + c] * kk;
             }
-            a = (j < r) ? a * f.b[r] : 0.f;
+            if (j == r) a = 0.f;
         }
-        f.A[e] = a;
+        if (P) P[e] = a;
+        f.A[e] = a * f.b[r];
         f.M[e] = m;
     }
     __syncthreads();
@@ -211,6 +221,20 @@ __device__ __forceinline__ void chunk_factors(const Factors<DK, C>& f, const Tin
         f.W[r * LD + c] = acc;
     }
     __syncthreads();
+}
+
+// chunk_prep, then chunk_products: every factor of the chunk.
+template <typename Tin, int DK, int C>
+__device__ __forceinline__ void chunk_factors(const Factors<DK, C>& f, const Tin* __restrict__ q,
+                                              const Tin* __restrict__ k,
+                                              const void* __restrict__ alpha,
+                                              const float* __restrict__ beta, size_t first, int t0,
+                                              int nvalid, int H, int h, int G, int l2norm,
+                                              const RopeParams& rp, const unsigned long long* sfreq,
+                                              long long pos0, int gate_logits) {
+    chunk_prep<Tin, DK, C>(f, q, k, alpha, beta, first, t0, nvalid, H, h, G, l2norm, rp, sfreq,
+                           pos0, gate_logits);
+    chunk_products<DK, C>(f);
 }
 
 }  // namespace simt

@@ -57,7 +57,7 @@ def parse():
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--no-extras", action="store_true",
                     help="skip decode / KDA-ratio / e2e / CPU-baseline legs")
-    ap.add_argument("--profile-case", choices=["fwd", "decode", "prologue", "bwd"], default=None,
+    ap.add_argument("--profile-case", choices=["fwd", "decode", "prologue", "bwd", "seg"], default=None,
                     help="run only a few calls of one entry point (for ncu captures) and exit")
     return ap.parse_args()
 
@@ -284,6 +284,13 @@ def profile_case(case, calls, dev):
         dhT = 0.02 * torch.randn((w["B"], w["H"], w["dk"], w["dv"]), generator=gen, device=dev)
         for _ in range(calls):
             ck.bwd_chunked(s["q"], s["k"], s["v"], s["alpha"], s["beta"], s["h0"], dout, dhT)
+    elif case == "seg":
+        wl = synth.WORKLOADS["long_rope_bf16"]
+        s = synth.torch_fwd_inputs(1, wl["T"], 2, 128, 128, kind="ckda", dtype="bf16",
+                                   h0_std=wl["h0_std"], seed=1, device=dev)
+        for _ in range(calls):
+            ck.fwd_segmented(s["q"], s["k"], s["v"], s["alpha"], s["beta"], s["h0"], segments=0,
+                             rope_theta=wl["rope_theta"])
     else:
         w = WORKLOAD
         s = synth.torch_fwd_inputs(w["B"], w["T"], w["H"], w["dk"], w["dv"], seed=1, device=dev)
@@ -516,7 +523,47 @@ def main():
             "workload": "long_rope_bf16 (B=1,T=65536,H=16,dk=dv=128,RoPE 1e4 half-split,h0)",
             "ms": round(ms_long, 3), "mtok_s": round(wl["B"] * wl["T"] / (ms_long / 1e3) / 1e6, 2),
             "hbm_frac": round(htL * FWD_BYTES_PER_HT / (ms_long / 1e3) / 1e9 / hbm_peak, 4)}
-        del L, wsL, outL, hL
+        # the same workload with the segment-parallel state pass (8 segments, and the model's
+        # count, which keeps the single fused launch here)
+        wsS = torch.empty(ck.segmented_workspace_bytes(wl["B"], wl["T"], wl["H"], 128, 128, 8),
+                          dtype=torch.uint8, device=dev)
+        fnS = lambda i: ck.fwd_segmented(L["q"], L["k"], L["v"], L["alpha"], L["beta"], L["h0"],
+                                         segments=8, rope_theta=wl["rope_theta"], out=outL,
+                                         hT=hL, workspace=wsS)
+        for i in range(2):
+            fnS(i)
+        ms_seg = event_time_ms(fnS, nL, stream) / nL
+        extras["long_context"]["segments_8_ms"] = round(ms_seg, 3)
+        extras["long_context"]["segments_auto"] = ck.segments_auto(wl["B"], wl["T"], wl["H"])
+        del L, wsL, outL, hL, wsS
+
+        # ---- one long sequence on two heads (a head-sharded layer's share of the long-context
+        # workload): the single fused launch vs the segment-parallel state pass ----------------
+        H2 = 2
+        L2 = synth.torch_fwd_inputs(1, wl["T"], H2, 128, 128, kind="ckda", dtype="bf16",
+                                    h0_std=wl["h0_std"], seed=9500 + rank, device=dev)
+        P2 = ck.segments_auto(1, wl["T"], H2)
+        ws2 = torch.empty(ck.segmented_workspace_bytes(1, wl["T"], H2, 128, 128, P2),
+                          dtype=torch.uint8, device=dev)
+        out2, h2 = torch.empty_like(L2["v"]), torch.empty_like(L2["h0"])
+        fnF = lambda i: ck.fwd_chunked(L2["q"], L2["k"], L2["v"], L2["alpha"], L2["beta"],
+                                       L2["h0"], rope_theta=wl["rope_theta"], path="tc",
+                                       out=out2, hT=h2, workspace=ws2)
+        fnG = lambda i: ck.fwd_segmented(L2["q"], L2["k"], L2["v"], L2["alpha"], L2["beta"],
+                                         L2["h0"], segments=P2, rope_theta=wl["rope_theta"],
+                                         out=out2, hT=h2, workspace=ws2)
+        for i in range(2):
+            fnF(i)
+            fnG(i)
+        ms_f2 = event_time_ms(fnF, nL, stream) / nL
+        ms_g2 = event_time_ms(fnG, nL, stream) / nL
+        ht2 = wl["T"] * H2
+        extras["long_context_2_heads"] = {
+            "workload": "B=1,T=65536,H=2,dk=dv=128,RoPE 1e4 half-split,h0",
+            "fused_ms": round(ms_f2, 3), "segmented_ms": round(ms_g2, 3), "segments": P2,
+            "segmented_mtok_s": round(wl["T"] / (ms_g2 / 1e3) / 1e6, 2),
+            "segmented_hbm_frac": round(ht2 * FWD_BYTES_PER_HT / (ms_g2 / 1e3) / 1e9 / hbm_peak, 4)}
+        del L2, ws2, out2, h2
 
         # ---- standalone q/k prologue: rotation (theta 1e4, half-split) then the L2 norm --------
         pq = [synth.torch_fwd_inputs(B, T, H, dk, dv, seed=6000 + 10 * rank + i, device=dev)

@@ -64,6 +64,12 @@ def _load():
     lib.ckda_fwd_chunked.restype = I
     lib.ckda_fwd_chunked.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, _Flags, I, LL, P,
                                      SZ, P]
+    lib.ckda_fwd_segmented_workspace_bytes.restype = SZ
+    lib.ckda_fwd_segmented_workspace_bytes.argtypes = [I] * 6
+    lib.ckda_fwd_segmented.restype = I
+    lib.ckda_fwd_segmented.argtypes = [P] * 8 + [I] * 5 + [_Flags, I, LL, I, P, SZ, P]
+    lib.ckda_fwd_segments_auto.restype = I
+    lib.ckda_fwd_segments_auto.argtypes = [I, I, I]
     lib.ckda_fwd_varlen_workspace_bytes.restype = SZ
     lib.ckda_fwd_varlen_workspace_bytes.argtypes = [P, I, I, I, I, I, I, I]
     lib.ckda_fwd_varlen.restype = I
@@ -199,6 +205,61 @@ def fwd_chunked(q, k, v, alpha, beta, h0=None, *, chunk=64, l2norm=True, rope_th
                                            Hk if Hk != H else 0, rope_dims),
         code, int(pos_offset), _ptr(workspace), wbytes, _stream(q.device))
     _raise("ckda_fwd_chunked", st)
+    return out, hT
+
+
+def segments_auto(B, T, H) -> int:
+    """Segment count ckda_fwd_segments_auto picks for a batch of B x H sequences of T tokens on the
+    current device (1: the single fused launch is expected to be faster)."""
+    return int(_load().ckda_fwd_segments_auto(B, T, H))
+
+
+def segmented_workspace_bytes(B, T, H, dk, dv, segments) -> int:
+    n = _load().ckda_fwd_segmented_workspace_bytes(B, T, H, dk, dv, segments)
+    if n == ctypes.c_size_t(-1).value:
+        raise ValueError("unsupported problem for ckda_fwd_segmented")
+    return int(n)
+
+
+def fwd_segmented(q, k, v, alpha, beta, h0=None, *, segments=0, l2norm=True, rope_theta=0.0,
+                  rope_convention=0, scale=0.0, pos_offset=0, want_state=True, out=None, hT=None,
+                  workspace=None, gate_logits=False, rope_dims=0):
+    """Tensor-core forward with the segment-parallel state pass (ckda_fwd_segmented): arguments
+    and results as fwd_chunked (bf16, dk = dv = 128).  segments = 0 takes segments_auto's count.
+    Returns (out, hT)."""
+    _check(q, "q")
+    B, T, Hk, dk = q.shape
+    _check(v, "v", dtype=q.dtype)
+    if v.dim() != 4 or v.shape[:2] != (B, T):
+        raise ValueError(f"v: expected [B={B}, T={T}, H, dv], got {tuple(v.shape)}")
+    H, dv = v.shape[2], v.shape[3]
+    if H % Hk:
+        raise ValueError(f"v has {H} heads, not a multiple of q's {Hk}")
+    _check(k, "k", dtype=q.dtype, shape=q.shape)
+    _check(alpha, "alpha", dtype=q.dtype if gate_logits else torch.float32, shape=(B, T, H, dk))
+    _check(beta, "beta", dtype=torch.float32, shape=(B, T, H))
+    if h0 is not None:
+        _check(h0, "h0", dtype=torch.float32, shape=(B, H, dk, dv))
+    if segments == 0:
+        segments = segments_auto(B, T, H)
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    _check(out, "out", dtype=q.dtype, shape=(B, T, H, dv))
+    if want_state and hT is None:
+        hT = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    if hT is not None:
+        _check(hT, "hT", dtype=torch.float32, shape=(B, H, dk, dv))
+    if workspace is None:
+        workspace = torch.empty(segmented_workspace_bytes(B, T, H, dk, dv, segments),
+                                dtype=torch.uint8, device=q.device)
+    wbytes = workspace.numel() * workspace.element_size()
+    st = _load().ckda_fwd_segmented(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(h0), _ptr(out), _ptr(hT),
+        B, T, H, dk, dv, _flags(l2norm, rope_theta, rope_convention, scale, PATHS["tc"], 0,
+                                gate_logits, Hk if Hk != H else 0, rope_dims),
+        _dtype_code(q), int(pos_offset), int(segments), _ptr(workspace), wbytes,
+        _stream(q.device))
+    _raise("ckda_fwd_segmented", st)
     return out, hT
 
 

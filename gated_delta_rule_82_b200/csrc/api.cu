@@ -148,7 +148,7 @@ ckda_status fwd_impl(const void* q, const void* k, const void* v, const void* al
                      const float* beta, const float* h0, void* out, float* hT, int B, int T, int H,
                      int dk, int dv, int chunk, ckda_flags flags, ckda_dtype dtype,
                      long long pos_offset, void* workspace, size_t workspace_bytes,
-                     const PackedSeqs& pk, cudaStream_t stream) {
+                     const PackedSeqs& pk, cudaStream_t stream, int segments = 1) {
     const bool packed = pk.cu != nullptr;
     if (!q || !k || !v || !alpha || !beta || !out) return CKDA_ERR_NULL;
     if (dtype != CKDA_F32 && dtype != CKDA_BF16) return CKDA_ERR_UNSUPPORTED;
@@ -189,9 +189,11 @@ ckda_status fwd_impl(const void* q, const void* k, const void* v, const void* al
     if (st != CKDA_OK) return st;
     const float scale = resolve_scale(flags, dk);
     const int l2 = flags.l2norm ? 1 : 0;
+    if (segments != 1 && (p != CKDA_PATH_TC || packed)) return CKDA_ERR_UNSUPPORTED;
     if (p == CKDA_PATH_TC) {
-        size_t need = packed ? chunk_tc_workspace_bytes_packed(pk.cu_host, pk.n, H)
-                             : chunk_tc_workspace_bytes(B, T, H);
+        size_t need = packed          ? chunk_tc_workspace_bytes_packed(pk.cu_host, pk.n, H)
+                      : segments != 1 ? chunk_tc_seg_workspace_bytes(B, T, H, segments)
+                                      : chunk_tc_workspace_bytes(B, T, H);
         if (need > 0 && (!workspace || workspace_bytes < need)) return CKDA_ERR_WORKSPACE;
         if (workspace && !aligned16(workspace)) return CKDA_ERR_ALIGN;
         const void* all[] = {q, k, v, alpha, beta, h0, out, hT};
@@ -199,6 +201,10 @@ ckda_status fwd_impl(const void* q, const void* k, const void* v, const void* al
                                 nst * 4, nv * es, nst * 4};
         for (int i = 0; i < 8; ++i)
             if (all[i] && overlap(workspace, need, all[i], allsz[i])) return CKDA_ERR_ARG;
+        if (segments != 1)
+            return from_cuda(launch_chunk_tc_seg(q, k, v, alpha, beta, h0, out, hT, B, T, H, G, l2,
+                                                 rp, scale, pos_offset, flags.gate_logits,
+                                                 workspace, segments, stream));
         return from_cuda(launch_chunk_tc(q, k, v, alpha, beta, h0, out, hT, B, T, H, G, l2, rp,
                                          scale, pos_offset, flags.gate_logits, workspace,
                                          flags.stages, pk, stream));
@@ -220,6 +226,33 @@ ckda_status ckda_fwd_chunked(const void* q, const void* k, const void* v, const 
     const PackedSeqs none{nullptr, nullptr, 0};
     return fwd_impl(q, k, v, alpha, beta, h0, out, hT, B, T, H, dk, dv, chunk, flags, dtype,
                     pos_offset, workspace, workspace_bytes, none, (cudaStream_t)stream);
+}
+
+int ckda_fwd_segments_auto(int B, int T, int H) {
+    if (B < 1 || T < 1 || H < 1 || (long long)B * H > 0x7fffffffll) return 1;
+    int dev = 0, nsm = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    return chunk_tc_seg_plan(B * H, (T + 63) / 64, nsm);
+}
+
+size_t ckda_fwd_segmented_workspace_bytes(int B, int T, int H, int dk, int dv, int segments) {
+    if (B < 1 || T < 1 || H < 1 || segments < 1) return (size_t)-1;
+    if (dk != 128 || dv != 128) return (size_t)-1;
+    if ((long long)B * T * H * 128 > (1ll << 40)) return (size_t)-1;
+    return chunk_tc_seg_workspace_bytes(B, T, H, segments);
+}
+
+ckda_status ckda_fwd_segmented(const void* q, const void* k, const void* v, const void* alpha,
+                               const float* beta, const float* h0, void* out, float* hT, int B,
+                               int T, int H, int dk, int dv, ckda_flags flags, ckda_dtype dtype,
+                               long long pos_offset, int segments, void* workspace,
+                               size_t workspace_bytes, ckda_stream_t stream) {
+    if (segments < 1) return CKDA_ERR_ARG;
+    if (flags.path == CKDA_PATH_SIMT) return CKDA_ERR_UNSUPPORTED;
+    const PackedSeqs none{nullptr, nullptr, 0};
+    return fwd_impl(q, k, v, alpha, beta, h0, out, hT, B, T, H, dk, dv, 64, flags, dtype,
+                    pos_offset, workspace, workspace_bytes, none, (cudaStream_t)stream, segments);
 }
 
 size_t ckda_fwd_varlen_workspace_bytes(const int* cu_seqlens_host, int n_seqs, int H, int dk,

@@ -1062,12 +1062,85 @@ static_assert(SS_OSTAGE % 1024 == 0 && (WS_QP - WS_UT) % 1024 == 0 && (WS_M - WS
 // TMEM columns: D_c^T 0..127, S^T buffers of 64 (bf16 pairs) from 128, D_o^T buffers of 64 from 256
 constexpr uint32_t kColS = 128, kColO = 256;
 
+// ---- segments of the state pass (the segment-parallel chunk-transition scan) -------------------
+// The NT chunks of every head unit form P segments of L chunks (the last one may be shorter).  A
+// summary pass gives, for every segment s < P - 1, its end state E_s when entered with h0 (s = 0)
+// or with zero (s > 0), and for 0 < s < P - 1 its transition F_s, the product of its A_c (a chain
+// entered with the identity and without the B_c terms).  A scan then forms the state entering
+// every segment, S_1 = E_0 and S_{s+1} = F_s S_s + E_s, and a second pass runs every segment from
+// its entering state with its outputs.  States and transitions are fp32 [dk][dv] (or [dk][dk])
+// arrays of the workspace, indexed (unit * P + s).
+struct SegArgs {
+    int P, L;
+    int summary;          // 1: the summary pass (no outputs); 0: the pass with outputs
+    float* segE;          // end states E_s
+    float* segF;          // transitions F_s
+    const float* segS;    // entering states S_s (S_0 = h0)
+};
+struct SegUnit {
+    int bh, s, c0, c1;
+    int transition;       // 1: a transition chain (identity start, no B_c terms)
+};
+__host__ __device__ inline int seg_units(const SegArgs& a, int BH) {
+    return a.summary ? BH * (a.P - 1) + BH * (a.P > 2 ? a.P - 2 : 0) : BH * a.P;
+}
+// summary units: the end-state chains (unit, s < P - 1), then the transition chains
+// (unit, 0 < s < P - 1); pass units: (unit, s)
+__device__ __forceinline__ SegUnit seg_unit(const SegArgs& a, int vu, int BH, int NT) {
+    SegUnit u;
+    u.transition = 0;
+    if (a.summary) {
+        const int ne = BH * (a.P - 1);
+        if (vu < ne) {
+            u.bh = vu / (a.P - 1);
+            u.s = vu % (a.P - 1);
+        } else {
+            u.transition = 1;
+            u.bh = (vu - ne) / (a.P - 2);
+            u.s = 1 + (vu - ne) % (a.P - 2);
+        }
+    } else {
+        u.bh = vu / a.P;
+        u.s = vu % a.P;
+    }
+    u.c0 = u.s * a.L;
+    u.c1 = min(NT, u.c0 + a.L);
+    return u;
+}
+// The items (unit, chunk) of the units first, first + stride, ... in order.
+struct SegIter {
+    SegArgs a;
+    int BH, NT, vu, stride, nunits, c;
+    SegUnit cur;
+    __device__ SegIter(const SegArgs& a_, int first, int stride_, int BH_, int NT_)
+        : a(a_), BH(BH_), NT(NT_), vu(first), stride(stride_), nunits(seg_units(a_, BH_)), c(0) {
+        cur = SegUnit{0, 0, 0, 0, 0};
+        if (vu < nunits) {
+            cur = seg_unit(a, vu, BH, NT);
+            c = cur.c0;
+        }
+    }
+    __device__ bool unit_end() const { return c + 1 == cur.c1; }
+    __device__ void next() {
+        if (++c == cur.c1) {
+            vu += stride;
+            if (vu < nunits) {
+                cur = seg_unit(a, vu, BH, NT);
+                c = cur.c0;
+            }
+        }
+    }
+};
+
+// kSeg: the items are the chunks of segment units (SegArgs) head0, head0 + hstride, ... instead of
+// whole head units; in the summary pass there are no outputs.
+template <bool kSeg>
 __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, const uint8_t* __restrict__ ws,
                                            const int* __restrict__ flags, PackedTabs pt,
                                            const float* __restrict__ h0,
                                            __nv_bfloat16* __restrict__ out, float* __restrict__ hT,
                                            int T_len, int H, int NT, int BH, float scale, int head0,
-                                           int hstride, uint32_t tmem) {
+                                           int hstride, uint32_t tmem, SegArgs sa) {
     uint64_t* full_c = reinterpret_cast<uint64_t*>(sm + SS_BAR);   // [2] A_c, K_end, U~^T landed
     uint64_t* empty_c = full_c + 2;     // [2] chain stage read by the chain products (commit)
     uint64_t* full_o = empty_c + 2;     // [2] Q', U~^T, M landed
@@ -1085,7 +1158,16 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
     const int4* __restrict__ ctab = pt.ctab;
     auto units_chunks = [&](int bh) { return pt.lane_cnt ? pt.lane_cnt[bh / H] : NT; };
     int U = 0;   // items of this CTA: the chunks of heads head0, head0 + hstride, ...
-    for (int bh = head0; bh < BH; bh += hstride) U += units_chunks(bh);
+    if constexpr (kSeg) {
+        const int nu = seg_units(sa, BH);
+        for (int vu = head0; vu < nu; vu += hstride) {
+            const SegUnit su = seg_unit(sa, vu, BH, NT);
+            U += su.c1 - su.c0;
+        }
+    } else {
+        for (int bh = head0; bh < BH; bh += hstride) U += units_chunks(bh);
+    }
+    const bool outputs = !kSeg || !sa.summary;
 
     if (tid == 32) {
         tc::mbar_init(dc_free, 8);
@@ -1145,6 +1227,61 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&s_ready[u & 1]);
         };
+        if constexpr (kSeg) {
+            // the state entering a segment unit: S_s (pass with outputs); h0 or zero (end-state
+            // chains); the identity (transition chains)
+            auto load_init = [&](const SegUnit& su) {
+                const float* src = nullptr;
+                if (!sa.summary)
+                    src = sa.segS + ((size_t)su.bh * sa.P + su.s) * kDK * kDV;
+                else if (!su.transition && su.s == 0 && h0)
+                    src = h0 + (size_t)su.bh * kDK * kDV;
+                if (src) {
+                    src += (size_t)cb * kDV + n;
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) S[j] = src[(size_t)j * kDV];
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) S[j] = (su.transition && cb + j == n) ? 1.f : 0.f;
+                }
+            };
+            SegIter it(sa, head0, hstride, BH, NT);
+            if (U > 0) {
+                load_init(it.cur);
+                put_s(0);
+            }
+            for (int u = 0; u < U; ++u) {
+                const bool unit_end = it.unit_end();
+                if (!wait(mma_c, u & 1)) break;
+                tc::tc_fence_after();
+                tc::tmem_ld64_sync(tc::tmem_addr(tmem, 32 * q, cb), S);
+                tc::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(dc_free);
+                if (unit_end && !*abort_flag) {
+                    // the pass writes hT after a head's last chunk; the summary its E_s or F_s
+                    float* dst = nullptr;
+                    if (!sa.summary)
+                        dst = (hT && it.c == NT - 1) ? hT + (size_t)it.cur.bh * kDK * kDV : nullptr;
+                    else
+                        dst = (it.cur.transition ? sa.segF : sa.segE) +
+                              ((size_t)it.cur.bh * sa.P + it.cur.s) * kDK * kDV;
+                    if (dst) {
+                        dst += (size_t)cb * kDV + n;
+#pragma unroll
+                        for (int j = 0; j < 64; ++j) dst[(size_t)j * kDV] = S[j];
+                    }
+                }
+                if (u + 1 < U) {
+                    if (outputs && u >= 1 && !wait(&mma_o[(u - 1) & 3], ((u - 1) >> 2) & 1)) break;
+                    it.next();
+                    if (unit_end) load_init(it.cur);
+                    put_s(u + 1);
+                } else {
+                    tc::tc_fence_before();
+                }
+            }
+        } else {
         // packed sequences: unit bh is (lane bh / H, head bh % H); tab is its lane's chunk table
         // and srow gives the state row of (sequence, head)
         const int4* tab = ctab ? ctab + (size_t)(head0 / H) * NT : nullptr;
@@ -1191,6 +1328,7 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
                 if (u + 1 < U) nc = units_chunks(bh);
             }
         }
+        }
     } else if (warp == 8) {
         // ---- chain issue: D_c^T = U~^T K_end (both from the stage: K-major A, MN-major B) and
         // then + S^T A_c^T (A = S^T from TMEM, B = the K-major A_c image read as K-major B) ----
@@ -1199,16 +1337,22 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
         const uint64_t k_desc0 = tc::smem_desc_sw128(tc::smem_u32(sm + SS_C + (WS_KE - WS_AC)), 8192, 1024);
         const uint64_t u_desc0 = tc::smem_desc_sw128(tc::smem_u32(sm + SS_C + (WS_UT - WS_AC)), 16, 1024);
         const uint64_t c_desc0 = tc::smem_desc_sw128(tc::smem_u32(sm + SS_C), 16, 1024);
+        SegIter it(sa, head0, hstride, BH, NT);   // (segment units only)
         for (int u = 0; u < U; ++u) {
             const int st = u & 1;
             if (!wait(&full_c[st], (u >> 1) & 1)) break;
             // the epilogue has read the previous accumulator
             if (u >= 1 && !wait(dc_free, (u - 1) & 1)) break;
             tc::tc_fence_after();
+            // a transition chain has no B_c = K_end^T U~ term
+            bool bterm = true;
+            if constexpr (kSeg) bterm = !it.cur.transition;
+            if (bterm) {
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                tc::mma_bf16_warp(tmem, tc::desc_add(u_desc0, st * SS_CSTAGE + ks * 32),
-                                  tc::desc_add(k_desc0, st * SS_CSTAGE + ks * 2048), idb, ks > 0 ? 1u : 0u);
+                for (int ks = 0; ks < 4; ++ks)
+                    tc::mma_bf16_warp(tmem, tc::desc_add(u_desc0, st * SS_CSTAGE + ks * 32),
+                                      tc::desc_add(k_desc0, st * SS_CSTAGE + ks * 2048), idb, ks > 0 ? 1u : 0u);
+            }
             if (!wait(&s_ready[st], (u >> 1) & 1)) break;
             tc::tc_fence_after();
             const uint64_t bd = tc::desc_add(c_desc0, st * SS_CSTAGE);
@@ -1216,16 +1360,17 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
                 tc::mma_bf16_tmem_a_warp(tmem, a + 8 * ks, tc::desc_add(bd, (ks >> 2) * 16384 + (ks & 3) * 32),
-                                         idc, 1u);
+                                         idc, (bterm || ks > 0) ? 1u : 0u);
             tc::mma_commit_warp(mma_c);
             tc::mma_commit_warp(&dc_done[st]);
             tc::mma_commit_warp(&empty_c[st]);
+            if constexpr (kSeg) it.next();
         }
     } else if (warp == 9) {
         // ---- output issue: S^T Q'^T (A in TMEM) + U~^T M^T (both from shared memory) ----
         const uint32_t ido = tc::idesc_bf16_f32(128, 64, 0, 0);
         const uint64_t o_desc0 = tc::smem_desc_sw128(tc::smem_u32(sm + SS_O), 16, 1024);
-        for (int u = 0; u < U; ++u) {
+        for (int u = 0; u < (outputs ? U : 0); ++u) {
             const int st = u & 1, ob = u & 3;
             if (!wait(&full_o[st], (u >> 1) & 1)) break;
             // issued once D_c(u) has completed, so it never shares the tensor pipe with a chain
@@ -1250,23 +1395,30 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
         }
     } else if (warp == 10 || warp == 11) {
         // ---- loads: warp 10 the chain stages, warp 11 the output stages ----
-        if (lane == 0) {
+        if (lane == 0 && (warp == 10 || outputs)) {
             const bool chain = warp == 10;
             uint64_t* fullb = chain ? full_c : full_o;
             uint64_t* emptyb = chain ? empty_c : empty_o;
             const uint32_t bytes = chain ? SS_CSTAGE : SS_OSTAGE;
             uint8_t* stage0 = sm + (chain ? SS_C : SS_O);
             int issued = 0;
-            int nc = U > 0 ? units_chunks(head0) : 0;
+            int nc = U > 0 && !kSeg ? units_chunks(head0) : 0;
+            SegIter it(sa, head0, hstride, BH, NT);   // (segment units only)
             for (int c = 0, bh = head0; issued < U; ++issued) {
                 const int st = issued & 1;
                 if (issued >= 2 && !mbar_wait_long(&emptyb[st], ((issued >> 1) - 1) & 1, abort_flag, limit))
                     break;
-                const size_t ci = (size_t)bh * NT + c;
-                if (++c == nc) {
-                    c = 0;
-                    bh += hstride;
-                    if (issued + 1 < U) nc = units_chunks(bh);
+                size_t ci;
+                if constexpr (kSeg) {
+                    ci = (size_t)it.cur.bh * NT + it.c;
+                    it.next();
+                } else {
+                    ci = (size_t)bh * NT + c;
+                    if (++c == nc) {
+                        c = 0;
+                        bh += hstride;
+                        if (issued + 1 < U) nc = units_chunks(bh);
+                    }
                 }
                 if (!flag_wait(flags + ci, abort_flag, limit)) break;
                 tc::mbar_arrive_expect_tx(&fullb[st], bytes);
@@ -1288,9 +1440,14 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
         const bool leader = warp == 12 && lane == 0;
         uint8_t* stg = sm + SS_STG;
         const int4* otab = ctab ? ctab + (size_t)(head0 / H) * NT : nullptr;   // the lane's table
-        int nc = U > 0 ? units_chunks(head0) : 0;
-        for (int u = 0, c = 0, bh = head0; u < U; ++u) {
+        int nc = U > 0 && !kSeg ? units_chunks(head0) : 0;
+        SegIter it(sa, head0, hstride, BH, NT);   // (segment units only)
+        for (int u = 0, c = 0, bh = head0; u < (outputs ? U : 0); ++u) {
             const int ob = u & 3;
+            if constexpr (kSeg) {
+                c = it.c;
+                bh = it.cur.bh;
+            }
             // the chunk's first token and length (packed sequences: from the chunk table)
             const int4 e = ctab ? otab[c] : make_int4(c * kC, kC, 0, 0);
             const bool ok = mbar_wait_long(&mma_o[ob], (u >> 2) & 1, abort_flag, limit);
@@ -1337,7 +1494,9 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
                 // the staging tile is read before the next item rewrites it
                 tc::bar_named(1, 128);
             }
-            if (++c == nc) {
+            if constexpr (kSeg) {
+                it.next();
+            } else if (++c == nc) {
                 c = 0;
                 bh += hstride;
                 if (u + 1 < U) {
@@ -1401,8 +1560,8 @@ ckda_tc_state(const __grid_constant__ TcMaps maps, const uint8_t* __restrict__ w
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint32_t tmem_slot;
     const uint32_t tmem = kernel_tmem_alloc(&tmem_slot);
-    state_role(aligned_smem(smem_raw), maps, ws, flags, pt, h0, out, hT, T_len, H, NT, BH, scale,
-               blockIdx.x, gridDim.x, tmem);
+    state_role<false>(aligned_smem(smem_raw), maps, ws, flags, pt, h0, out, hT, T_len, H, NT, BH,
+                      scale, blockIdx.x, gridDim.x, tmem, SegArgs{});
     kernel_tmem_free(tmem);
 }
 
@@ -1432,8 +1591,95 @@ ckda_tc_fused(const __grid_constant__ TcMaps maps, const void* __restrict__ alph
         intra_role<kLogits>(sm, maps, alpha, beta, ws, flags, pt, T_len, H, NT, wo, seq, l2norm,
                             rp, pos_offset, tmem);
     if (chain)
-        state_role(sm, maps, ws, flags, pt, h0, out, hT, T_len, H, NT, BH, scale, b, n_state, tmem);
+        state_role<false>(sm, maps, ws, flags, pt, h0, out, hT, T_len, H, NT, BH, scale, b, n_state,
+                          tmem, SegArgs{});
     kernel_tmem_free(tmem);
+}
+
+// A pass over segment units (after the factor kernel): units blockIdx.x, blockIdx.x + gridDim.x, ...
+__global__ void __launch_bounds__(512, 1)
+ckda_tc_seg(const __grid_constant__ TcMaps maps, const uint8_t* __restrict__ ws,
+            const int* __restrict__ flags, const float* __restrict__ h0,
+            __nv_bfloat16* __restrict__ out, float* __restrict__ hT, int T_len, int H, int NT,
+            int BH, float scale, SegArgs sa) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint32_t tmem_slot;
+    const uint32_t tmem = kernel_tmem_alloc(&tmem_slot);
+    state_role<true>(aligned_smem(smem_raw), maps, ws, flags, PackedTabs{nullptr, nullptr, nullptr},
+                     h0, out, hT, T_len, H, NT, BH, scale, blockIdx.x, gridDim.x, tmem, sa);
+    kernel_tmem_free(tmem);
+}
+
+// The scan over the segments of one head unit, 8 state columns per CTA (grid BH x 16), in fp32 on
+// CUDA cores: S_0 = h0 (or zero), S_1 = E_0, S_{s+1} = F_s S_s + E_s for 0 < s < P - 1.  F_{s+1}
+// is copied into shared memory (rows 132 floats apart) while step s runs; thread (row r, column
+// group) reads its row of F_s in 16-byte pieces (eight consecutive rows of a quarter warp fall on
+// distinct bank groups) and forms 4 columns.
+constexpr int kScanCols = 8, kScanLd = kDK + 4, kScanThreads = 256;
+constexpr size_t kScanSmem = sizeof(float) * (2 * (size_t)kDK * kScanLd + (size_t)kDK * kScanCols);
+__device__ __forceinline__ void scan_load_f(float* dst, const float* F) {
+    for (int i = threadIdx.x; i < kDK * kDK / 4; i += kScanThreads) {
+        const int r = i / (kDK / 4), k4 = 4 * (i % (kDK / 4));
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
+                     ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst + r * kScanLd + k4))),
+                     "l"(F + (size_t)r * kDK + k4) : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__global__ void __launch_bounds__(kScanThreads)
+ckda_seg_scan(const float* __restrict__ h0, SegArgs sa) {
+    extern __shared__ __align__(16) float scan_sm[];
+    float* sF = scan_sm;                            // F_s, two buffers [128][132]
+    float* sS = scan_sm + 2 * kDK * kScanLd;        // S_s columns [128][8]
+    const int bh = blockIdx.x, n0 = blockIdx.y * kScanCols, tid = threadIdx.x;
+    const size_t st = (size_t)kDK * kDV, base = (size_t)bh * sa.P;
+    float* segS = const_cast<float*>(sa.segS);
+    tc::grid_dependency_wait();   // the summary pass is complete (programmatic launch)
+    // F_s goes to buffer s & 1
+    if (sa.P > 2) scan_load_f(sF + kDK * kScanLd, sa.segF + (base + 1) * st);
+    for (int e = tid; e < kDK * kScanCols; e += kScanThreads) {
+        const size_t o = (size_t)(e / kScanCols) * kDV + n0 + e % kScanCols;
+        segS[base * st + o] = h0 ? h0[(size_t)bh * st + o] : 0.f;
+        const float s1 = sa.segE[base * st + o];
+        sS[e] = s1;
+        segS[(base + 1) * st + o] = s1;
+    }
+    const int r = tid >> 1, cg = 4 * (tid & 1);
+    // this thread's part of E_s, loaded one step ahead
+    auto load_e = [&](int s) {
+        return *reinterpret_cast<const float4*>(sa.segE + (base + s) * st + (size_t)r * kDV + n0 + cg);
+    };
+    float4 e_next = sa.P > 2 ? load_e(1) : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 1; s + 1 < sa.P; ++s) {
+        const float4 e4 = e_next;
+        if (s + 2 < sa.P) e_next = load_e(s + 1);
+        if (s + 2 < sa.P) {
+            scan_load_f(sF + ((s + 1) & 1) * kDK * kScanLd, sa.segF + (base + s + 1) * st);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+        }
+        __syncthreads();   // F_s landed (every thread's copies) and S_s written
+        const float4* Fr = reinterpret_cast<const float4*>(sF + (s & 1) * kDK * kScanLd + r * kScanLd);
+        float a0 = e4.x, a1 = e4.y, a2 = e4.z, a3 = e4.w;
+#pragma unroll 8
+        for (int k4 = 0; k4 < kDK / 4; ++k4) {
+            const float4 f = Fr[k4];
+            const float fk[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const float4 sv = *reinterpret_cast<const float4*>(sS + (4 * k4 + kk) * kScanCols + cg);
+                a0 += fk[kk] * sv.x;
+                a1 += fk[kk] * sv.y;
+                a2 += fk[kk] * sv.z;
+                a3 += fk[kk] * sv.w;
+            }
+        }
+        __syncthreads();   // every thread has read S_s and F_s
+        *reinterpret_cast<float4*>(sS + r * kScanCols + cg) = make_float4(a0, a1, a2, a3);
+        *reinterpret_cast<float4*>(segS + (base + s + 1) * st + (size_t)r * kDV + n0 + cg) =
+            make_float4(a0, a1, a2, a3);
+    }
 }
 
 // Packed sequences: the tables and the ready flags of one call (one CTA of 1024 threads).
@@ -1637,11 +1883,13 @@ size_t chunk_tc_workspace_bytes_packed(const int* cu_host, int n_seqs, int H) {
 // NT steps, or before its last chunk plus one step (and no chain starts before the leading rounds
 // are done).  The split minimises the later of that end and the end of the factor work (the
 // larger s and the smaller lead on ties).
-void chunk_tc_plan(int BH, int NT, long long n_items, int nsm, int* n_state, int* lead) {
+void chunk_tc_plan(int BH, int NT, long long n_items, int nsm, int* n_state, int* lead,
+                   double* t_model) {
     struct Entry {
         int BH, NT;
         long long n_items;
         int nsm, s, lead;
+        double t;
     };
     static std::mutex m;
     static Entry cache[16];
@@ -1653,6 +1901,7 @@ void chunk_tc_plan(int BH, int NT, long long n_items, int nsm, int* n_state, int
                 cache[e].nsm == nsm) {
                 *n_state = cache[e].s;
                 *lead = cache[e].lead;
+                if (t_model) *t_model = cache[e].t;
                 return;
             }
     }
@@ -1697,8 +1946,56 @@ void chunk_tc_plan(int BH, int NT, long long n_items, int nsm, int* n_state, int
     }
     *n_state = best_s;
     *lead = best_l;
+    if (t_model) *t_model = best_t;
     std::lock_guard<std::mutex> g(m);
-    if (n_cached < 16) cache[n_cached++] = Entry{BH, NT, n_items, nsm, best_s, best_l};
+    if (n_cached < 16) cache[n_cached++] = Entry{BH, NT, n_items, nsm, best_s, best_l, best_t};
+}
+
+// Segments of the segment-parallel pass: L = ceil(NT / P) chunks each, and as many segments as
+// that needs (none empty).
+static void seg_shape(int NT, int P, int* Pe, int* L) {
+    const int l = (NT + P - 1) / P;
+    *L = l;
+    *Pe = (NT + l - 1) / l;
+}
+
+size_t chunk_tc_seg_workspace_bytes(int B, int T_len, int H, int segments) {
+    const int NT = (T_len + kC - 1) / kC;
+    int P = 1, L = NT;
+    if (segments > 1) seg_shape(NT, segments, &P, &L);
+    const size_t base = chunk_tc_workspace_bytes(B, T_len, H);
+    if (P < 2) return base;
+    return ((base + 255) & ~(size_t)255) + 3 * (size_t)B * H * P * kDK * kDV * sizeof(float);
+}
+
+// Segment count for the segment-parallel pass, from the same cycle model as chunk_tc_plan: the
+// factor kernel alone (rounds of t_i on all SMs), the summary pass (end-state and transition
+// chains, rounds of L steps of t_c), the scan (t_s per segment), the pass with outputs (rounds of
+// L steps) and t_g for the flag reset and the four launches (t_s and t_g fitted to B200 timings
+// of one sequence of 65536 tokens on 2 heads).  1 when no segment count beats the single fused
+// launch.
+int chunk_tc_seg_plan(int BH, int NT, int nsm) {
+    const double ti = 19000.0, tc = 2200.0, ts = 5000.0, tg = 35000.0;
+    if (BH < 1 || NT < 4 || nsm < 2) return 1;
+    int n_state = 1, lead = 0;
+    double fused = 0.0;
+    chunk_tc_plan(BH, NT, (long long)BH * NT, nsm, &n_state, &lead, &fused);
+    const double factor = (double)(((long long)BH * NT + nsm - 1) / nsm) * ti;
+    int best = 1;
+    double best_t = fused;
+    for (int p = 2; p <= NT && p <= 1024; ++p) {
+        int P, L;
+        seg_shape(NT, p, &P, &L);
+        if (P != p) continue;
+        const long long nsum = (long long)BH * (P - 1) + (long long)BH * (P - 2);
+        const double t = factor + (double)((nsum + nsm - 1) / nsm) * L * tc + (P - 2) * ts +
+                         (double)(((long long)BH * P + nsm - 1) / nsm) * L * tc + tg;
+        if (t < best_t) {
+            best_t = t;
+            best = P;
+        }
+    }
+    return best;
 }
 
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const void* alpha,
@@ -1739,7 +2036,7 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
         cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
     if (stages == 0 && nsm < 2) stages = 3;
     int n_state = 1, lead = 0;
-    if (stages == 0 && n_items > 0) chunk_tc_plan(BH, NT, n_items, nsm, &n_state, &lead);
+    if (stages == 0 && n_items > 0) chunk_tc_plan(BH, NT, n_items, nsm, &n_state, &lead, nullptr);
     if (packed && stages != 2) {
         if (hT) {
             // empty sequences keep their initial state
@@ -1837,6 +2134,72 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
                                scale);
     }
     return e;
+}
+
+// The forward with the segment-parallel pass (batched sequences only): the factor kernel, the
+// summary pass, the scan, and the pass with outputs, in stream order.
+cudaError_t launch_chunk_tc_seg(const void* q, const void* k, const void* v, const void* alpha,
+                                const float* beta, const float* h0, void* out, float* hT, int B,
+                                int T_len, int H, int G, int l2norm, const RopeParams& rp,
+                                float scale, long long pos_offset, int gate_logits,
+                                void* workspace, int segments, cudaStream_t stream) {
+    const int NT = (T_len + kC - 1) / kC, BH = B * H;
+    const PackedSeqs none{nullptr, nullptr, 0};
+    int P = 1, L = NT;
+    if (segments > 1) seg_shape(NT, segments, &P, &L);
+    if (P < 2)
+        return launch_chunk_tc(q, k, v, alpha, beta, h0, out, hT, B, T_len, H, G, l2norm, rp, scale,
+                               pos_offset, gate_logits, workspace, 0, none, stream);
+    // the factor kernel (with the reset of the ready flags)
+    cudaError_t e = launch_chunk_tc(q, k, v, alpha, beta, h0, out, hT, B, T_len, H, G, l2norm, rp,
+                                    scale, pos_offset, gate_logits, workspace, 1, none, stream);
+    if (e != cudaSuccess) return e;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const int* flags = reinterpret_cast<const int*>(ws + flags_offset((size_t)BH * NT));
+    float* seg = reinterpret_cast<float*>(
+        ws + ((chunk_tc_workspace_bytes(B, T_len, H) + 255) & ~(size_t)255));
+    const size_t arr = (size_t)BH * P * kDK * kDV;
+    SegArgs sa{P, L, 1, seg, seg + arr, seg + 2 * arr};
+    TcMaps maps;
+    if (!encode_map(&maps.out, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDV, kDV, H, T_len, B,
+                    CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    e = cudaFuncSetAttribute(ckda_tc_seg, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SS_BYTES);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(ckda_seg_scan, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kScanSmem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, nsm = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    __nv_bfloat16* outb = static_cast<__nv_bfloat16*>(out);
+    // programmatic dependent launches: each kernel's set-up overlaps the previous one's tail, and
+    // griddepcontrol.wait holds it back before it reads what that kernel wrote
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(512);
+    cfg.dynamicSmemBytes = SS_BYTES;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const int nsum = seg_units(sa, BH);
+    cfg.gridDim = dim3((unsigned)(nsum < nsm ? nsum : nsm));
+    e = cudaLaunchKernelEx(&cfg, ckda_tc_seg, maps, static_cast<const uint8_t*>(ws), flags, h0,
+                           outb, hT, T_len, H, NT, BH, scale, sa);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t scfg = cfg;
+    scfg.gridDim = dim3((unsigned)BH, kDV / kScanCols);
+    scfg.blockDim = dim3(kScanThreads);
+    scfg.dynamicSmemBytes = kScanSmem;
+    e = cudaLaunchKernelEx(&scfg, ckda_seg_scan, h0, sa);
+    if (e != cudaSuccess) return e;
+    sa.summary = 0;
+    const int npass = BH * P;
+    cfg.gridDim = dim3((unsigned)(npass < nsm ? npass : nsm));
+    return cudaLaunchKernelEx(&cfg, ckda_tc_seg, maps, static_cast<const uint8_t*>(ws), flags, h0,
+                              outb, hT, T_len, H, NT, BH, scale, sa);
 }
 
 // Read the status word on the current device (after `stream` has finished) and clear it.

@@ -78,7 +78,16 @@ long long packed_chunks(const int* cu_host, int n_seqs);
 size_t chunk_tc_workspace_bytes_packed(const int* cu_host, int n_seqs, int H);
 // split of the fused tensor-core launch for BH heads of up to NT chunks (n_items chunk-heads in
 // all) on nsm SMs: chain CTAs and leading rounds of factor items taken by every CTA
-void chunk_tc_plan(int BH, int NT, long long n_items, int nsm, int* n_state, int* lead);
+void chunk_tc_plan(int BH, int NT, long long n_items, int nsm, int* n_state, int* lead,
+                   double* t_model);
+// The segment-parallel pass (batched sequences): workspace, segment count model, launch.
+size_t chunk_tc_seg_workspace_bytes(int B, int T_len, int H, int segments);
+int chunk_tc_seg_plan(int BH, int NT, int nsm);
+cudaError_t launch_chunk_tc_seg(const void* q, const void* k, const void* v, const void* alpha,
+                                const float* beta, const float* h0, void* out, float* hT, int B,
+                                int T_len, int H, int G, int l2norm, const RopeParams& rp,
+                                float scale, long long pos_offset, int gate_logits,
+                                void* workspace, int segments, cudaStream_t stream);
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const void* alpha,
                             const float* beta, const float* h0, void* out, float* hT, int B,
                             int T_len, int H, int G, int l2norm, const RopeParams& rp, float scale,

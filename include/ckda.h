@@ -47,7 +47,7 @@
 extern "C" {
 #endif
 
-#define CKDA_ABI_VERSION 6
+#define CKDA_ABI_VERSION 7
 
 #if defined(__GNUC__)
 #define CKDA_API __attribute__((visibility("default")))
@@ -190,6 +190,46 @@ CKDA_API ckda_status ckda_fwd_chunked(const void* q, const void* k, const void* 
                              int T, int H, int dk, int dv, int chunk, ckda_flags flags,
                              ckda_dtype dtype, long long pos_offset, void* workspace,
                              size_t workspace_bytes, ckda_stream_t stream);
+
+/*
+ * The chunked forward with a segment-parallel state pass (tensor-core path only: bf16,
+ * dk = dv = 128, chunk 64; batched sequences).  The serial pass over the chunks of every
+ * (batch, head) is split into `segments` segments of L = ceil(ceil(T/64) / segments) chunks
+ * (as many as that needs, none empty).  Every chunk's transition is
+ *     A_c = Diag(gamma_C) - K_end^T W      (dk x dk),
+ * the chunk-level form of the product of the per-token transitions (I - beta k k^T) Diag(alpha)
+ * of the "Complex KDA" paper summary, "Background"; the summary's fixed-size state is what makes
+ * a segment's composition F_s = A_c(last) ... A_c(first) a dk x dk matrix.  A summary pass forms,
+ * in parallel over segments, each segment's end state from zero (from h0 for the first) and its
+ * transition F_s; an fp32 scan forms the state entering every segment, S_{s+1} = F_s S_s + E_s;
+ * a second parallel pass runs every segment from its entering state and writes the outputs
+ * (and hT).  The result is the recurrence's, like ckda_fwd_chunked's, up to rounding; the work
+ * on the serial path drops from ceil(T/64) chunk steps to about 3 L + segments, for about three
+ * times the state-pass products in total.  It pays when few (batch, head) pairs carry long
+ * sequences (ckda_fwd_segments_auto).
+ *   Arguments as ckda_fwd_chunked (chunk fixed at 64; flags.path must not select the CUDA-core
+ *   path, flags.stages is ignored), plus
+ *   segments : >= 1; 1 runs ckda_fwd_chunked's single fused launch.
+ *   workspace / workspace_bytes : at least ckda_fwd_segmented_workspace_bytes(...): the
+ *            tensor-core forward's workspace and three fp32 arrays of B*H*P dk x dv matrices.
+ * Errors: CKDA_ERR_UNSUPPORTED outside the tensor-core sizes (segments > 1), CKDA_ERR_ARG for
+ * segments < 1, otherwise as ckda_fwd_chunked.  hT may equal h0 (h0 is read by the first two
+ * launches, hT written by the last).
+ */
+CKDA_API size_t ckda_fwd_segmented_workspace_bytes(int B, int T, int H, int dk, int dv,
+                                                   int segments);
+CKDA_API ckda_status ckda_fwd_segmented(const void* q, const void* k, const void* v,
+                                        const void* alpha, const float* beta, const float* h0,
+                                        void* out, float* hT, int B, int T, int H, int dk,
+                                        int dv, ckda_flags flags, ckda_dtype dtype,
+                                        long long pos_offset, int segments, void* workspace,
+                                        size_t workspace_bytes, ckda_stream_t stream);
+/*
+ * Segment count for ckda_fwd_segmented on the current device from a cycle model of the four
+ * launches against the single fused launch; 1 when the fused launch is expected to be faster
+ * (many (batch, head) pairs keep every SM busy with chunk-parallel work).
+ */
+CKDA_API int ckda_fwd_segments_auto(int B, int T, int H);
 
 /*
  * Bytes of device workspace ckda_fwd_varlen needs for these packed sequences (cu_seqlens_host as

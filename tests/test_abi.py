@@ -34,7 +34,8 @@ def test_header_declares_the_boundary():
     for want in ("ckda_fwd_chunked", "ckda_decode_step", "ckda_fwd_workspace_bytes",
                  "ckda_qk_prologue", "ckda_strerror", "ckda_abi_version", "ckda_fwd_varlen",
                  "ckda_fwd_varlen_workspace_bytes", "ckda_last_device_status",
-                 "ckda_set_wait_limit_ns", "ckda_fwd_chunked_noalloc"):
+                 "ckda_set_wait_limit_ns", "ckda_fwd_chunked_noalloc", "ckda_fwd_segmented",
+                 "ckda_fwd_segmented_workspace_bytes", "ckda_fwd_segments_auto"):
         assert want in names
 
 
@@ -52,7 +53,7 @@ def test_only_declared_symbols_are_exported(lib):
 
 
 def test_version_and_strerror(lib):
-    assert ck.abi_version() == 6
+    assert ck.abi_version() == 7
     for s in range(9):
         assert lib.ckda_strerror(s)
     assert lib.ckda_strerror(99) == b"unknown status"
@@ -106,6 +107,49 @@ def test_workspace_query(lib):
     assert lib.ckda_fwd_workspace_bytes(1, 64, 2, 16, 16, 16, 0, 2) == bad
     assert lib.ckda_fwd_workspace_bytes(1, 0, 2, 16, 16, 16, 0, 0) == bad
     assert lib.ckda_fwd_workspace_bytes(1, 64, 2, 48, 16, 16, 0, 0) == bad
+
+
+def fwd_seg(lib, q=P, k=9 * P, v=17 * P, a=25 * P, b=40 * P, h0=None, out=50 * P, hT=None, B=1,
+            T=256, H=1, dk=128, dv=128, fl=None, dtype=1, pos=0, segments=2, ws=60 * P,
+            wsb=1 << 40):
+    fl = fl or flags()
+    c = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.ckda_fwd_segmented(c(q), c(k), c(v), c(a), c(b), c(h0), c(out), c(hT), B, T, H,
+                                  dk, dv, fl, dtype, pos, segments, c(ws), wsb, None)
+
+
+# each case is invalid in exactly the stated way (nothing is launched: no GPU needed)
+@pytest.mark.parametrize("kw,want", [
+    (dict(segments=0), ARG), (dict(segments=-3), ARG),
+    (dict(dtype=0), UNSUP),                   # fp32: no tensor-core path
+    (dict(dk=64, dv=64), UNSUP),
+    (dict(fl=flags(path=1)), UNSUP),          # the CUDA-core path has no segments
+    (dict(q=None), NULL), (dict(T=0), SHAPE), (dict(q=P + 8), ALIGN),
+    (dict(out=P), ARG),                       # out aliases q
+    (dict(ws=None, wsb=0), WORKSPACE),
+    (dict(wsb=1024), WORKSPACE),
+])
+def test_segmented_validation(lib, kw, want):
+    assert fwd_seg(lib, **kw) == want
+
+
+def test_segmented_workspace_and_count(lib):
+    plain = lib.ckda_fwd_workspace_bytes(1, 65536, 2, 128, 128, 64, 1, 0)
+    assert lib.ckda_fwd_segmented_workspace_bytes(1, 65536, 2, 128, 128, 1) == plain
+    # 1024 chunks in 32 segments of 32: three fp32 arrays of 2 x 32 matrices of 64 KiB beyond it
+    n32 = lib.ckda_fwd_segmented_workspace_bytes(1, 65536, 2, 128, 128, 32)
+    assert n32 >= plain + 3 * 2 * 32 * 65536 and n32 - plain < 3 * 2 * 32 * 65536 + 256
+    # 5 chunks asked for 4 segments: L = 2, so 3 segments
+    n4 = lib.ckda_fwd_segmented_workspace_bytes(1, 320, 1, 128, 128, 4)
+    assert n4 - lib.ckda_fwd_workspace_bytes(1, 320, 1, 128, 128, 64, 1, 0) < 3 * 3 * 65536 + 256
+    bad = ctypes.c_size_t(-1).value
+    assert lib.ckda_fwd_segmented_workspace_bytes(1, 256, 1, 64, 128, 2) == bad
+    assert lib.ckda_fwd_segmented_workspace_bytes(1, 256, 1, 128, 128, 0) == bad
+    # the model: few heads over a long sequence are chain-bound (segments); the layer shape's
+    # 32 heads keep every SM busy (one fused launch)
+    assert lib.ckda_fwd_segments_auto(1, 65536, 2) > 1
+    assert lib.ckda_fwd_segments_auto(2, 2048, 16) == 1
+    assert lib.ckda_fwd_segments_auto(1, 64, 1) == 1
 
 
 def host_offsets(vals):

@@ -131,21 +131,33 @@ bwd_replay_kernel(const T* __restrict__ v, const float* __restrict__ h0,
     for (int e = tid; e < DK * DVS; e += kThreads)
         sS[e] = h0 ? h0[((size_t)bh * DK + e / DVS) * DV + n0 + e % DVS] : 0.f;
     load_record(smem, rec0, Sh::REC);
+    // this thread's elements of a chunk's V slice, read one chunk ahead into registers
+    constexpr int NE = (C * DVS + kThreads - 1) / kThreads;
+    float rv[NE];
+    auto load_v = [&](int ch) {
+        const int t0 = ch * C, nvalid = min(C, T_len - t0);
+#pragma unroll
+        for (int i = 0; i < NE; ++i) {
+            const int e = tid + i * kThreads, r = e / DVS, n = e % DVS;
+            rv[i] = e < C * DVS && r < nvalid
+                        ? to_f32(v[(((size_t)b * T_len + t0 + r) * H + h) * DV + n0 + n]) : 0.f;
+        }
+    };
+    load_v(0);
     for (int ch = 0; ch < nchunks; ++ch) {
         const float* rf = smem + (ch & 1) * Sh::REC;
+#pragma unroll
+        for (int i = 0; i < NE; ++i)
+            if (tid + i * kThreads < C * DVS) sv[tid + i * kThreads] = rv[i];
         if (ch + 1 < nchunks) {
+            load_v(ch + 1);
             load_record(smem + ((ch + 1) & 1) * Sh::REC, rec0 + (size_t)(ch + 1) * R::floats, Sh::REC);
             cp_wait<1>();
         } else {
             cp_wait<0>();
         }
-        const int t0 = ch * C, nvalid = min(C, T_len - t0);
         float* dst = ws_S + ((size_t)bh * nchunks + ch) * DK * DV + n0;
         for (int e = tid; e < DK * DVS; e += kThreads) dst[(e / DVS) * DV + e % DVS] = sS[e];
-        for (int e = tid; e < C * DVS; e += kThreads) {
-            const int r = e / DVS, n = e % DVS;
-            sv[e] = r < nvalid ? to_f32(v[(((size_t)b * T_len + t0 + r) * H + h) * DV + n0 + n]) : 0.f;
-        }
         __syncthreads();
         for (int e = tid; e < C * DVS; e += kThreads) {
             const int r = e / DVS, n = e % DVS;
@@ -204,21 +216,33 @@ bwd_chain_kernel(const T* __restrict__ dout, const float* __restrict__ dhT,
     for (int e = tid; e < DK * DVS; e += kThreads)
         sdS[e] = dhT ? dhT[((size_t)bh * DK + e / DVS) * DV + n0 + e % DVS] : 0.f;
     load_record(smem, rec0 + (size_t)(nchunks - 1) * R::floats, Sh::REC);
+    // this thread's elements of a chunk's dO slice, read one chunk ahead into registers
+    constexpr int NE = (C * DVS + kThreads - 1) / kThreads;
+    float rdo[NE];
+    auto load_do = [&](int ch) {
+        const int t0 = ch * C, nvalid = min(C, T_len - t0);
+#pragma unroll
+        for (int i = 0; i < NE; ++i) {
+            const int e = tid + i * kThreads, r = e / DVS, n = e % DVS;
+            rdo[i] = e < C * DVS && r < nvalid
+                         ? to_f32(dout[(((size_t)b * T_len + t0 + r) * H + h) * DV + n0 + n]) : 0.f;
+        }
+    };
+    load_do(nchunks - 1);
     for (int ch = nchunks - 1, it = 0; ch >= 0; --ch, ++it) {
         const float* rf = smem + (it & 1) * Sh::REC;
+#pragma unroll
+        for (int i = 0; i < NE; ++i)
+            if (tid + i * kThreads < C * DVS) sdO[tid + i * kThreads] = rdo[i];
         if (ch > 0) {
+            load_do(ch - 1);
             load_record(smem + ((it + 1) & 1) * Sh::REC, rec0 + (size_t)(ch - 1) * R::floats, Sh::REC);
             cp_wait<1>();
         } else {
             cp_wait<0>();
         }
-        const int t0 = ch * C, nvalid = min(C, T_len - t0);
         float* dst = ws_dS + ((size_t)bh * nchunks + ch) * DK * DV + n0;
         for (int e = tid; e < DK * DVS; e += kThreads) dst[(e / DVS) * DV + e % DVS] = sdS[e];
-        for (int e = tid; e < C * DVS; e += kThreads) {
-            const int r = e / DVS, n = e % DVS;
-            sdO[e] = r < nvalid ? to_f32(dout[(((size_t)b * T_len + t0 + r) * H + h) * DV + n0 + n]) : 0.f;
-        }
         __syncthreads();
         for (int e = tid; e < C * DVS; e += kThreads) {   // K_end dS_out
             const int j = e / DVS, n = e % DVS;
@@ -242,41 +266,108 @@ bwd_chain_kernel(const T* __restrict__ dout, const float* __restrict__ dhT,
             dh0[((size_t)bh * DK + e / DVS) * DV + n0 + e % DVS] = sdS[e];
 }
 
+// ---- warp-level tensor-core tiles with fp32-grade products ------------------------------------
+// mma.sync m16n8k8 with tf32 operands, each operand split into a tf32 head and a tf32 tail
+// (x = hi + lo, lo the rounded remainder): a b = a_hi b_hi + a_hi b_lo + a_lo b_hi up to a relative
+// 2^-21, i.e. the product of two fp32 values to about fp32 precision ("3xTF32").  Fragment layout
+// (PTX ISA, mma.m16n8k8 .tf32), g = lane / 4, t = lane % 4: A a0 = A[g][t], a1 = A[g+8][t],
+// a2 = A[g][t+4], a3 = A[g+8][t+4]; B b0 = B[t][g], b1 = B[t+4][g]; D d0 = D[g][2t],
+// d1 = D[g][2t+1], d2 = D[g+8][2t], d3 = D[g+8][2t+1].
+__device__ __forceinline__ uint32_t f2tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+    hi = f2tf32(x);
+    lo = f2tf32(x - __uint_as_float(hi));
+}
+__device__ __forceinline__ void mma_tf32(float c[4], const uint32_t a[4], const uint32_t b[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// c (+)= A[16 x K] B[K x 8], A(m, k) and B(k, n) read through the accessors
+template <int K, typename FA, typename FB>
+__device__ __forceinline__ void mma3_tile(float c[4], FA A, FB B, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        uint32_t ah[4], al[4], bh[2], bl[2];
+        split_tf32(A(g, k0 + t), ah[0], al[0]);
+        split_tf32(A(g + 8, k0 + t), ah[1], al[1]);
+        split_tf32(A(g, k0 + t + 4), ah[2], al[2]);
+        split_tf32(A(g + 8, k0 + t + 4), ah[3], al[3]);
+        split_tf32(B(k0 + t, g), bh[0], bl[0]);
+        split_tf32(B(k0 + t + 4, g), bh[1], bl[1]);
+        mma_tf32(c, al, bh);
+        mma_tf32(c, ah, bl);
+        mma_tf32(c, ah, bh);
+    }
+}
+// D fragment (times s) into rows ld floats apart, columns col0 ..
+__device__ __forceinline__ void st_frag(float* d, int ld, int col0, const float c[4], float s,
+                                        int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    d[g * ld + col0 + 2 * t] = s * c[0];
+    d[g * ld + col0 + 2 * t + 1] = s * c[1];
+    d[(g + 8) * ld + col0 + 2 * t] = s * c[2];
+    d[(g + 8) * ld + col0 + 2 * t + 1] = s * c[3];
+}
+
 // ---- 3. the gradients of one chunk: one CTA per (b*h, chunk), all dv in tiles of DT ----------
+// The products over a dv tile are 16-row warp tiles (above): U, W S0, K_end dS_out, dU, and the
+// accumulations dQ', dK_end, dW, dM, dT, whose fragments stay in registers across the dv tiles
+// (tile q of the 3 DK/8 + 4 belongs to warp q % 8).
 template <int DK, int DV, int C>
 struct GradShape {
-    static constexpr int DT = DV < 32 ? DV : 32;
-    static constexpr int TP = DT + 1;   // tile rows are TP floats apart (distinct banks down a column)
-    static constexpr int CD = C * DK, CC = C * C, CT = C * TP;
-    static constexpr int off_qp = Factors<DK, C>::floats;  // Q'     [C][DK]
-    static constexpr int off_ke = off_qp + CD;             // K_end  [C][DK]
-    static constexpr int off_dqp = off_ke + CD;            // dQ'    [C][DK]
-    static constexpr int off_dke = off_dqp + CD;           // dK_end [C][DK]
-    static constexpr int off_dw = off_dke + CD;            // dW, then dK_gamma [C][DK]
-    static constexpr int off_sig = off_dw + CD;            // sigma  [C][DK]
-    static constexpr int off_dgc = off_sig + CD;           // dgamma_C [DK]
+    static_assert(C == 16, "the warp tiles are 16 rows: one chunk");
+    static constexpr int DT = 16;          // dv columns per tile
+    static constexpr int NTT = DT / 8;     // 8-column tiles per dv tile
+    static constexpr int TP = DT + 4;      // tile rows TP floats apart (fragment lanes on distinct banks)
+    static constexpr int KP = DK + 4;      // rows of W, K_end and K_gamma (the same)
+    static constexpr int NQ = 3 * (DK / 8) + 4;   // accumulated tiles: dQ', dK_end, dW, dM (2), dT (2)
+    static constexpr int QI = (NQ + 7) / 8;       // of them per warp
+    static constexpr int CD = C * DK, CC = C * C, CT = C * TP, CK = C * KP;
+    static constexpr int off_w = Factors<DK, C>::floats_nw;  // W       [C][KP]
+    static constexpr int off_ke = off_w + CK;              // K_end   [C][KP]
+    static constexpr int off_kg = off_ke + CK;             // K_gamma [C][KP]
+    static constexpr int off_al = off_kg + CK;             // alpha   [C][DK]
+    static constexpr int off_sm = off_al + CD;             // running-sign bits per channel [DK]
+    static constexpr int off_dgc = off_sm + DK;            // dgamma_C [DK]
     static constexpr int off_P = off_dgc + DK;             // P (A before beta) [C][C]
     static constexpr int off_dM = off_P + CC;              // dM [C][C]
     static constexpr int off_dT = off_dM + CC;             // dT, then E = B dA [C][C]
     static constexpr int off_Z = off_dT + CC;              // dT T^T [C][C]
     static constexpr int off_db = off_Z + CC;              // dbeta [C]
-    static constexpr int off_s0 = off_db + C;              // S0 tile      [DK][TP]
-    static constexpr int off_ds = off_s0 + DK * TP;        // dS_out tile  [DK][TP]
-    static constexpr int off_do = off_ds + DK * TP;        // dO tile [C][TP]
+    static constexpr int off_yb = off_db + C;              // dbeta parts of the Y tiles [NTT][C]
+    // the dv tiles; after the last one the same floats hold dQ', dK_end and dW (then X)
+    static constexpr int off_tiles = off_yb + NTT * C;
+    static constexpr int off_s0 = off_tiles;               // S0 tiles     [2][DK][TP]
+    static constexpr int off_ds = off_s0 + 2 * DK * TP;    // dS_out tiles [2][DK][TP]
+    static constexpr int off_do = off_ds + 2 * DK * TP;    // dO tile [C][TP]
     static constexpr int off_v = off_do + CT;              // V tile
     static constexpr int off_u = off_v + CT;               // U tile
     static constexpr int off_du = off_u + CT;              // dU tile
     static constexpr int off_ws = off_du + CT;             // W S0 tile
     static constexpr int off_kd = off_ws + CT;             // K_end dS_out tile
-    static constexpr int total = off_kd + CT;
+    static constexpr int off_dqp = off_tiles;              // dQ'    [C][DK]
+    static constexpr int off_dke = off_dqp + CD;           // dK_end [C][DK]
+    static constexpr int off_dw = off_dke + CD;            // dW, then X = T^T dW [C][DK]
+    static constexpr int tiles_end = off_kd + CT, post_end = off_dw + CD;
+    static constexpr int total = tiles_end > post_end ? tiles_end : post_end;
     static constexpr size_t bytes = sizeof(float) * (size_t)total;
+    static_assert(off_tiles % 4 == 0 && off_w % 4 == 0 && (DK * TP) % 4 == 0,
+                  "16-byte copies need 4-float offsets");
 };
 
 // recs: the chunk records; ws_S, ws_dS: [B*H][NT][DK][DV] fp32 (entering state, end-state
 // gradient of each chunk); ws_dq, ws_dk: [B*T*H][DK] fp32 gradients of the prepared q^, k^ per
 // value head.
 template <typename T, int DK, int DV, int C>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 bwd_grad_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                 const void* __restrict__ alpha, const float* __restrict__ beta,
                 const T* __restrict__ dout, const float* __restrict__ recs,
@@ -286,44 +377,74 @@ bwd_grad_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
                 float* __restrict__ dalpha, float* __restrict__ dbeta, int T_len, int H, int G,
                 int l2norm, RopeParams rp, float scale, long long pos_offset, int gate_logits) {
     using Sh = GradShape<DK, DV, C>;
-    constexpr int DT = Sh::DT;
-    constexpr int TP = Sh::TP;   // padded row stride of the tiles
+    constexpr int DT = Sh::DT, NTT = Sh::NTT, NQ = Sh::NQ, QI = Sh::QI;
+    constexpr int TP = Sh::TP, KP = Sh::KP;
     constexpr int LD = Factors<DK, C>::LD;
+    constexpr int Q1 = DK / 8, Q2 = 2 * (DK / 8), Q3 = 3 * (DK / 8);   // tile-kind boundaries
     extern __shared__ float smem[];
     Factors<DK, C> f;
-    f.bind(smem);
-    float* sQp = smem + Sh::off_qp;
+    f.bind_nw(smem);
+    float* sW = smem + Sh::off_w;
     float* sKe = smem + Sh::off_ke;
+    float* sKg = smem + Sh::off_kg;
     float* sdQp = smem + Sh::off_dqp;
     float* sdKe = smem + Sh::off_dke;
     float* sdW = smem + Sh::off_dw;
-    float* sSig = smem + Sh::off_sig;
+    uint32_t* sSgn = reinterpret_cast<uint32_t*>(smem + Sh::off_sm);
+    float* sAl = smem + Sh::off_al;
     float* sdgC = smem + Sh::off_dgc;
     float* sP = smem + Sh::off_P;
     float* sdM = smem + Sh::off_dM;
     float* sdT = smem + Sh::off_dT;
     float* sZ = smem + Sh::off_Z;
     float* sdb = smem + Sh::off_db;
-    float* tS0 = smem + Sh::off_s0;
-    float* tdS = smem + Sh::off_ds;
+    float* sYb = smem + Sh::off_yb;
     float* tdO = smem + Sh::off_do;
     float* tV = smem + Sh::off_v;
     float* tU = smem + Sh::off_u;
     float* tdU = smem + Sh::off_du;
     float* tWS = smem + Sh::off_ws;
     float* tKd = smem + Sh::off_kd;
-    __shared__ unsigned long long sfreq[DK / 2];
+    // RoPE frequencies for the row preparation, in the second S0 tile buffer (first written by
+    // the prefetch of the second dv tile, after the preparation); two CTAs of this kernel fit an
+    // SM at dk = 128 only without a static array
+    unsigned long long* sfreq = reinterpret_cast<unsigned long long*>(smem + Sh::off_s0 + DK * TP);
 
     const int nchunks = (T_len + C - 1) / C;
     const int bh = blockIdx.x / nchunks, ch = blockIdx.x % nchunks;
     const int b = bh / H, h = bh % H;
     const int t0 = ch * C, nvalid = min(C, T_len - t0);
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const size_t first = (size_t)b * T_len;
+    const float* S0 = ws_S + ((size_t)bh * nchunks + ch) * DK * DV;
+    const float* dS = ws_dS + ((size_t)bh * nchunks + ch) * DK * DV;
+    // the state tiles of dv columns n0 .. n0 + DT - 1 into buffer `buf` (one commit group)
+    auto load_state_tiles = [&](int n0, int buf) {
+        float* d0 = smem + Sh::off_s0 + buf * DK * TP;
+        float* d1 = smem + Sh::off_ds + buf * DK * TP;
+        for (int i = tid; i < DK * DT / 4; i += kThreads) {
+            const int c = i / (DT / 4), n4 = 4 * (i % (DT / 4));
+            cp16(d0 + c * TP + n4, S0 + (size_t)c * DV + n0 + n4);
+            cp16(d1 + c * TP + n4, dS + (size_t)c * DV + n0 + n4);
+        }
+        cp_commit();
+    };
+    // this thread's elements of the dO and V tiles, read one tile ahead into registers
+    constexpr int NE = (C * DT + kThreads - 1) / kThreads;
+    float rdo[NE], rv[NE];
+    auto load_act_tiles = [&](int n0) {
+#pragma unroll
+        for (int i = 0; i < NE; ++i) {
+            const int e = tid + i * kThreads, r = e / DT, n = e % DT;
+            const size_t o = ((first + t0 + r) * H + h) * DV + n0 + n;
+            const bool ok = e < C * DT && r < nvalid;
+            rdo[i] = ok ? to_f32(dout[o]) : 0.f;
+            rv[i] = ok ? to_f32(v[o]) : 0.f;
+        }
+    };
     if (rp.enabled)
         for (int i = tid; i < DK / 2; i += kThreads) sfreq[i] = rp.turns[i];
-    // the record's T, M, P, Q' and K_end land while the chunk's rows are prepared; W goes to its
-    // padded rows through registers
+    // the record's W, K_end, T, M and P land while the chunk's rows are prepared again
     {
         using R = Rec<DK, C>;
         const float* rec = recs + ((size_t)bh * nchunks + ch) * R::floats;
@@ -333,125 +454,171 @@ bwd_grad_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
             cp16(sP + 4 * i, rec + R::P + 4 * i);
         }
         for (int i = tid; i < C * DK / 4; i += kThreads) {
-            cp16(sQp + 4 * i, rec + R::QP + 4 * i);
-            cp16(sKe + 4 * i, rec + R::KE + 4 * i);
+            const int r = i / (DK / 4), c4 = 4 * (i % (DK / 4));
+            cp16(sW + r * KP + c4, rec + R::W + r * DK + c4);
+            cp16(sKe + r * KP + c4, rec + R::KE + r * DK + c4);
         }
         cp_commit();
-        for (int e = tid; e < C * DK; e += kThreads) f.W[(e / DK) * LD + e % DK] = rec[R::W + e];
     }
+    load_state_tiles(0, 0);
+    load_act_tiles(0);
     simt::chunk_prep<T, DK, C>(f, q, k, alpha, beta, first, t0, nvalid, H, h, G, l2norm, rp,
-                               sfreq, pos_offset + t0, gate_logits);
-    cp_wait<0>();
-    auto gate = [&](int r, int c) {   // alpha of row r < nvalid, channel c
-        const size_t ia = ((first + t0 + r) * H + h) * DK + c;
-        return gate_logits ? gate_alpha(to_f32(static_cast<const T*>(alpha)[ia]))
-                           : static_cast<const float*>(alpha)[ia];
-    };
-    // the running sign products; zero the accumulators
+                               sfreq, pos_offset + t0, gate_logits, sAl);
+    cp_wait<1>();   // the record (the first state tiles may still be in flight)
+    // K_gamma = g k', the running sign products (bit r of a channel's word: negative through
+    // row r); zero the dbeta parts
     for (int e = tid; e < C * DK; e += kThreads) {
-        sdQp[e] = 0.f;
-        sdKe[e] = 0.f;
-        sdW[e] = 0.f;
+        const int r = e / DK, c = e % DK;
+        sKg[r * KP + c] = exp2f(f.L[r * LD + c]) * f.k[r * LD + c];
     }
     for (int c = tid; c < DK; c += kThreads) {
-        float s = 1.f;
+        uint32_t neg = 0, bits = 0;
         for (int r = 0; r < C; ++r) {
-            if (r < nvalid && gate(r, c) < 0.f) s = -s;
-            sSig[r * DK + c] = s;
+            if (sAl[r * DK + c] < 0.f) neg ^= 1u;
+            bits |= neg << r;
         }
-        sdgC[c] = 0.f;
+        sSgn[c] = bits;
     }
-    for (int e = tid; e < C * C; e += kThreads) {
-        sdM[e] = 0.f;
-        sdT[e] = 0.f;
-    }
-    for (int r = tid; r < C; r += kThreads) sdb[r] = 0.f;
+    for (int e = tid; e < NTT * C; e += kThreads) sYb[e] = 0.f;
+    float dgc_acc = 0.f;   // dgamma_C of channel tid (tid < DK)
+    float acc[QI][4];
+#pragma unroll
+    for (int i = 0; i < QI; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
     __syncthreads();
 
-    const float* S0 = ws_S + ((size_t)bh * nchunks + ch) * DK * DV;
-    const float* dS = ws_dS + ((size_t)bh * nchunks + ch) * DK * DV;
-    for (int n0 = 0; n0 < DV; n0 += DT) {
-        // tiles of S0, dS_out, dO, V; U = T B V
-        for (int e = tid; e < DK * DT; e += kThreads) {
-            const int c = e / DT, n = e % DT;
-            tS0[c * TP + n] = S0[(size_t)c * DV + n0 + n];
-            tdS[c * TP + n] = dS[(size_t)c * DV + n0 + n];
-        }
-        for (int e = tid; e < C * DT; e += kThreads) {
-            const int r = e / DT, n = e % DT;
-            const size_t o = ((first + t0 + r) * H + h) * DV + n0 + n;
-            tdO[r * TP + n] = r < nvalid ? to_f32(dout[o]) : 0.f;
-            tV[r * TP + n] = r < nvalid ? to_f32(v[o]) : 0.f;
-        }
-        __syncthreads();
-        for (int e = tid; e < C * DT; e += kThreads) {
-            const int j = e / DT, n = e % DT;
-            float u = 0.f, ws = 0.f, kd = 0.f;
-            for (int m = 0; m <= j; ++m) u += f.T[j * C + m] * f.b[m] * tV[m * TP + n];
-            for (int c = 0; c < DK; ++c) {
-                ws += f.W[j * LD + c] * tS0[c * TP + n];
-                kd += sKe[j * DK + c] * tdS[c * TP + n];
+    for (int n0 = 0, it = 0; n0 < DV; n0 += DT, ++it) {
+        // this tile's dO and V from registers; the next tile's into registers and its state
+        // tiles into the other buffer while this one is used
+        const float* tS0 = smem + Sh::off_s0 + (it & 1) * DK * TP;
+        const float* tdS = smem + Sh::off_ds + (it & 1) * DK * TP;
+#pragma unroll
+        for (int i = 0; i < NE; ++i) {
+            const int e = tid + i * kThreads, r = e / DT, n = e % DT;
+            if (e < C * DT) {
+                tdO[r * TP + n] = rdo[i];
+                tV[r * TP + n] = rv[i];
             }
-            tU[j * TP + n] = u;
-            tWS[j * TP + n] = ws;
-            tKd[j * TP + n] = kd;
+        }
+        if (n0 + DT < DV) {
+            load_act_tiles(n0 + DT);
+            load_state_tiles(n0 + DT, (it + 1) & 1);
+            cp_wait<1>();
+        } else {
+            cp_wait<0>();
         }
         __syncthreads();
-        // dU = scale M^T dO + K_end dS_out
-        for (int e = tid; e < C * DT; e += kThreads) {
-            const int j = e / DT, n = e % DT;
-            float acc = tKd[j * TP + n];
-            for (int r = j; r < C; ++r) acc += scale * f.M[r * C + j] * tdO[r * TP + n];
-            tdU[j * TP + n] = acc;
-        }
-        __syncthreads();
-        // accumulate dQ', dK_end, dW over the tile's columns
-        for (int e = tid; e < C * DK; e += kThreads) {
-            const int r = e / DK, c = e % DK;
-            float aq = 0.f, ak = 0.f, aw = 0.f;
-            for (int n = 0; n < DT; ++n) {
-                aq += tdO[r * TP + n] * tS0[c * TP + n];
-                ak += (tU[r * TP + n] - tWS[r * TP + n]) * tdS[c * TP + n];
-                aw += tKd[r * TP + n] * tS0[c * TP + n];
+        // U = T B V (K = C), W S0 and K_end dS_out (K = DK): 3 NTT tiles
+        for (int tt = warp; tt < 3 * NTT; tt += kThreads / 32) {
+            const int kind = tt / NTT, nt = tt % NTT;
+            float c[4] = {0.f, 0.f, 0.f, 0.f};
+            if (kind == 0) {
+                mma3_tile<C>(c, [&](int m, int kk) { return f.T[m * C + kk] * f.b[kk]; },
+                             [&](int kk, int n) { return tV[kk * TP + 8 * nt + n]; }, lane);
+                st_frag(tU, TP, 8 * nt, c, 1.f, lane);
+            } else if (kind == 1) {
+                mma3_tile<DK>(c, [&](int m, int kk) { return sW[m * KP + kk]; },
+                              [&](int kk, int n) { return tS0[kk * TP + 8 * nt + n]; }, lane);
+                st_frag(tWS, TP, 8 * nt, c, 1.f, lane);
+            } else {
+                mma3_tile<DK>(c, [&](int m, int kk) { return sKe[m * KP + kk]; },
+                              [&](int kk, int n) { return tdS[kk * TP + 8 * nt + n]; }, lane);
+                st_frag(tKd, TP, 8 * nt, c, 1.f, lane);
             }
-            sdQp[e] += scale * aq;
-            sdKe[e] += ak;
-            sdW[e] -= aw;
+        }
+        __syncthreads();
+        // dU = K_end dS_out + scale M^T dO (NTT tiles); the accumulated tiles but dT; dgamma_C
+        if (warp < NTT) {
+            float c[4] = {0.f, 0.f, 0.f, 0.f};
+            mma3_tile<C>(c, [&](int m, int kk) { return f.M[kk * C + m]; },
+                         [&](int kk, int n) { return tdO[kk * TP + 8 * warp + n]; }, lane);
+            const int g = lane >> 2, t = lane & 3, col = 8 * warp + 2 * t;
+            tdU[g * TP + col] = tKd[g * TP + col] + scale * c[0];
+            tdU[g * TP + col + 1] = tKd[g * TP + col + 1] + scale * c[1];
+            tdU[(g + 8) * TP + col] = tKd[(g + 8) * TP + col] + scale * c[2];
+            tdU[(g + 8) * TP + col + 1] = tKd[(g + 8) * TP + col + 1] + scale * c[3];
+        }
+#pragma unroll
+        for (int i = 0; i < QI; ++i) {
+            const int qt = warp + 8 * i;
+            if (qt < Q1) {                // dQ' += dO S0^T (scale at the end)
+                mma3_tile<DT>(acc[i], [&](int m, int kk) { return tdO[m * TP + kk]; },
+                              [&](int kk, int n) { return tS0[(8 * qt + n) * TP + kk]; }, lane);
+            } else if (qt < Q2) {         // dK_end += (U - W S0) dS_out^T
+                const int c0 = 8 * (qt - Q1);
+                mma3_tile<DT>(acc[i], [&](int m, int kk) { return tU[m * TP + kk] - tWS[m * TP + kk]; },
+                              [&](int kk, int n) { return tdS[(c0 + n) * TP + kk]; }, lane);
+            } else if (qt < Q3) {         // -dW += (K_end dS_out) S0^T
+                const int c0 = 8 * (qt - Q2);
+                mma3_tile<DT>(acc[i], [&](int m, int kk) { return tKd[m * TP + kk]; },
+                              [&](int kk, int n) { return tS0[(c0 + n) * TP + kk]; }, lane);
+            } else if (qt < Q3 + 2) {     // dM += dO U^T (scale at the end)
+                const int j0 = 8 * (qt - Q3);
+                mma3_tile<DT>(acc[i], [&](int m, int kk) { return tdO[m * TP + kk]; },
+                              [&](int kk, int n) { return tU[(j0 + n) * TP + kk]; }, lane);
+            }
         }
         for (int c = tid; c < DK; c += kThreads) {
-            float acc = 0.f;
-            for (int n = 0; n < DT; ++n) acc += tdS[c * TP + n] * tS0[c * TP + n];
-            sdgC[c] += acc;
+            float a = 0.f;
+            for (int n = 0; n < DT; ++n) a += tdS[c * TP + n] * tS0[c * TP + n];
+            dgc_acc += a;
         }
-        // dM += scale dO U^T;  dT += dU (B V)^T
-        for (int e = tid; e < C * C; e += kThreads) {
-            const int r = e / C, j = e % C;
-            float am = 0.f, at = 0.f;
-            for (int n = 0; n < DT; ++n) {
-                am += tdO[r * TP + n] * tU[j * TP + n];
-                at += tdU[r * TP + n] * tV[j * TP + n];
+        __syncthreads();
+        // dT += dU (B V)^T (its two tiles); Y = T^T dU (NTT tiles): dv = B Y, dbeta parts Y . V
+#pragma unroll
+        for (int i = 0; i < QI; ++i) {
+            const int qt = warp + 8 * i;
+            if (qt >= Q3 + 2 && qt < NQ) {
+                const int j0 = 8 * (qt - Q3 - 2);
+                mma3_tile<DT>(acc[i], [&](int m, int kk) { return tdU[m * TP + kk]; },
+                              [&](int kk, int n) { return f.b[j0 + n] * tV[(j0 + n) * TP + kk]; },
+                              lane);
             }
-            sdM[e] += scale * am;
-            sdT[e] += f.b[j] * at;
         }
-        // Y = T^T dU:  dv = B Y, dbeta += rowsum(Y . V)
-        for (int j = tid / DT; j < C; j += kThreads / DT) {
-            const int n = tid % DT;
-            float y = 0.f;
-            for (int r = j; r < C; ++r) y += f.T[r * C + j] * tdU[r * TP + n];
-            if (j < nvalid) dv_out[((first + t0 + j) * H + h) * DV + n0 + n] = f.b[j] * y;
-            float yv = y * tV[j * TP + n];
-            for (int o = DT / 2; o > 0; o >>= 1) yv += __shfl_xor_sync(0xffffffffu, yv, o);
-            if (n == 0) sdb[j] += yv;
+        if (warp >= 8 - NTT) {
+            const int nt = warp - (8 - NTT);
+            float c[4] = {0.f, 0.f, 0.f, 0.f};
+            mma3_tile<C>(c, [&](int m, int kk) { return f.T[kk * C + m]; },
+                         [&](int kk, int n) { return tdU[kk * TP + 8 * nt + n]; }, lane);
+            const int g = lane >> 2, t = lane & 3, col = 8 * nt + 2 * t;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                const int j = g + 8 * hf;
+                const float y0 = c[2 * hf], y1 = c[2 * hf + 1];
+                if (j < nvalid)
+                    *reinterpret_cast<float2*>(dv_out + ((first + t0 + j) * H + h) * DV + n0 + col) =
+                        make_float2(f.b[j] * y0, f.b[j] * y1);
+                float yv = y0 * tV[j * TP + col] + y1 * tV[j * TP + col + 1];
+                yv += __shfl_xor_sync(0xffffffffu, yv, 1);
+                yv += __shfl_xor_sync(0xffffffffu, yv, 2);
+                if (t == 0) sYb[nt * C + j] += yv;
+            }
         }
         __syncthreads();
     }
+    // the accumulated tiles into shared memory: dQ' (scaled), dK_end, dW (negated), dM
+    // (scaled), dT; dgamma_C; dbeta = the sum of the Y tiles' parts
+#pragma unroll
+    for (int i = 0; i < QI; ++i) {
+        const int qt = warp + 8 * i;
+        if (qt < Q1) st_frag(sdQp, DK, 8 * qt, acc[i], scale, lane);
+        else if (qt < Q2) st_frag(sdKe, DK, 8 * (qt - Q1), acc[i], 1.f, lane);
+        else if (qt < Q3) st_frag(sdW, DK, 8 * (qt - Q2), acc[i], -1.f, lane);
+        else if (qt < Q3 + 2) st_frag(sdM, C, 8 * (qt - Q3), acc[i], scale, lane);
+        else if (qt < NQ) st_frag(sdT, C, 8 * (qt - Q3 - 2), acc[i], 1.f, lane);
+    }
+    for (int c = tid; c < DK; c += kThreads) sdgC[c] = dgc_acc;
+    for (int r = tid; r < C; r += kThreads) {
+        float a = 0.f;
+        for (int nt = 0; nt < NTT; ++nt) a += sYb[nt * C + r];
+        sdb[r] = a;
+    }
+    __syncthreads();
 
     // Q' = Q_gamma - M W:  dM -= dQ' W^T,  dW -= M^T dQ'
     for (int e = tid; e < C * C; e += kThreads) {
         const int r = e / C, j = e % C;
         float acc = 0.f;
-        for (int c = 0; c < DK; ++c) acc += sdQp[r * DK + c] * f.W[j * LD + c];
+        for (int c = 0; c < DK; ++c) acc += sdQp[r * DK + c] * sW[j * KP + c];
         sdM[e] = j <= r ? sdM[e] - acc : 0.f;   // M is lower triangular (diagonal included)
     }
     for (int e = tid; e < C * DK; e += kThreads) {
@@ -465,7 +632,7 @@ bwd_grad_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
     for (int e = tid; e < C * C; e += kThreads) {
         const int r = e / C, j = e % C;
         float acc = 0.f;
-        for (int c = 0; c < DK; ++c) acc += sdW[r * DK + c] * exp2f(f.L[j * LD + c]) * f.k[j * LD + c];
+        for (int c = 0; c < DK; ++c) acc += sdW[r * DK + c] * sKg[j * KP + c];
         sdT[e] += f.b[j] * acc;
     }
     __syncthreads();
@@ -498,8 +665,7 @@ bwd_grad_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
     }
     for (int j = tid >> 5; j < C; j += kThreads / 32) {   // one warp per row, lanes over channels
         float acc = 0.f;
-        for (int c = tid & 31; c < DK; c += 32)
-            acc += sdW[j * DK + c] * exp2f(f.L[j * LD + c]) * f.k[j * LD + c];
+        for (int c = tid & 31; c < DK; c += 32) acc += sdW[j * DK + c] * sKg[j * KP + c];
         acc = warp_sum(acc);
         if ((tid & 31) == 0) sdb[j] += acc;
     }
@@ -538,27 +704,31 @@ bwd_grad_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
         dk += f.b[j] * sdW[e] * g + sdKe[e] * f.sg[c] * exp2f(f.LC[c] - Lj);
         dq += sdQp[e] * g;
         const size_t o = ((first + t0 + j) * H + h) * DK + c;
-        ws_dq[o] = sSig[e] * dq;
-        ws_dk[o] = sSig[e] * dk;
+        const float sgn = (sSgn[c] >> j) & 1u ? -1.f : 1.f;
+        ws_dq[o] = sgn * dq;
+        ws_dk[o] = sgn * dk;
     }
-    // dalpha, one thread per channel c, in the order t = 0 .. C-1:
+    // dalpha in the order t = 0 .. C-1, two threads per channel c (lanes 2 c, 2 c + 1 of a warp),
+    // thread half hh taking the rows a, r = hh mod 2 of the sums:
     //   dg_r = dK_gamma,r k'_r + dQ_gamma,r q'_r (+ dgamma_C sigma_C at the last row)
     //   dR_ab = E_ab k'_a k'_b + dM_ab q'_a k'_b (+ dK_end,b sigma_C k'_b at a = C-1), b <= a
     //   dalpha_t = sign(alpha_t) [g_{t-1} sum_{r>=t} dg_r R_rt + sum_{a>=t} R_at Z_at],
     //   Z_{a,t} = |alpha_{t-1}| Z_{a,t-1} + dR_{a,t-1},  Z_{a,0} = 0
-    for (int c = tid; c < DK; c += kThreads) {
+    static_assert(2 * DK <= kThreads, "two threads per channel");
+    if ((tid >> 1) < DK) {   // whole warps (DK is a multiple of 16)
+        const int c = tid >> 1, hh = tid & 1;
         const float sC = f.sg[c];
-        float Z[C];
+        float Z[C / 2], dgv[C / 2];
 #pragma unroll
-        for (int a = 0; a < C; ++a) Z[a] = 0.f;
+        for (int i = 0; i < C / 2; ++i) {
+            const int r = 2 * i + hh;
+            Z[i] = 0.f;
+            dgv[i] = f.b[r] * sdW[r * DK + c] * f.k[r * LD + c] + sdQp[r * DK + c] * f.q[r * LD + c];
+            if (r == C - 1) dgv[i] += sdgC[c] * sC;
+        }
         auto dR = [&](int a, int bb) {
             float x = (sE[a * C + bb] * f.k[a * LD + c] + sdM[a * C + bb] * f.q[a * LD + c]) * f.k[bb * LD + c];
             if (a == C - 1) x += sdKe[bb * DK + c] * sC * f.k[bb * LD + c];
-            return x;
-        };
-        auto dg = [&](int r) {
-            float x = f.b[r] * sdW[r * DK + c] * f.k[r * LD + c] + sdQp[r * DK + c] * f.q[r * LD + c];
-            if (r == C - 1) x += sdgC[c] * sC;
             return x;
         };
 #pragma unroll
@@ -566,20 +736,26 @@ bwd_grad_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
             if (t > 0) {
                 const float am = exp2f(f.L[(t - 1) * LD + c] - (t > 1 ? f.L[(t - 2) * LD + c] : 0.f));
 #pragma unroll
-                for (int a = 0; a < C; ++a) Z[a] = a >= t - 1 ? am * Z[a] + dR(a, t - 1) : 0.f;
+                for (int i = 0; i < C / 2; ++i) {
+                    const int a = 2 * i + hh;
+                    Z[i] = a >= t - 1 ? am * Z[i] + dR(a, t - 1) : 0.f;
+                }
             }
             const float Lt = f.L[t * LD + c];
-            const float gprev = t > 0 ? exp2f(f.L[(t - 1) * LD + c]) : 1.f;
             float s1 = 0.f, s2 = 0.f;
 #pragma unroll
-            for (int r = 0; r < C; ++r) {
+            for (int i = 0; i < C / 2; ++i) {
+                const int r = 2 * i + hh;
                 if (r < t) continue;
                 const float R = exp2f(f.L[r * LD + c] - Lt);
-                s1 += dg(r) * R;
-                s2 += Z[r] * R;
+                s1 += dgv[i] * R;
+                s2 += Z[i] * R;
             }
-            if (t < nvalid) {
-                const float a = gate(t, c);
+            s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+            s2 += __shfl_xor_sync(0xffffffffu, s2, 1);
+            if (hh == 0 && t < nvalid) {
+                const float gprev = t > 0 ? exp2f(f.L[(t - 1) * LD + c]) : 1.f;
+                const float a = sAl[t * DK + c];
                 float d = (a < 0.f ? -1.f : 1.f) * (gprev * s1 + s2);
                 if (gate_logits) d *= 0.5f * (1.f - a * a);   // alpha = 2 sigma(a) - 1
                 dalpha[((first + t0 + t) * H + h) * DK + c] = d;

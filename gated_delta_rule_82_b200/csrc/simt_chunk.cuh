@@ -42,13 +42,20 @@ struct Factors {
         q = p; k = q + C * LD; L = k + C * LD; W = L + C * LD; A = W + C * LD; M = A + C * C;
         T = M + C * C; b = T + C * C; sg = b + C; LC = sg + DK;
     }
+    // without W and A (for a kernel that takes M and T from elsewhere)
+    static constexpr int floats_nw = 3 * C * LD + 2 * C * C + C + 2 * DK;
+    __device__ void bind_nw(float* p) {
+        q = p; k = q + C * LD; L = k + C * LD; W = nullptr; A = nullptr; M = L + C * LD;
+        T = M + C * C; b = T + C * C; sg = b + C; LC = sg + DK;
+    }
 };
 
 // Rows r < nvalid of q and k (value head h reads q/k row (token * H + h) / G), beta of head h,
 // alpha from fp32 values or `dtype` logits; rows past nvalid are identity steps.  Then the
 // prologue (rotation at position pos0 + r, L2 norm) and the gate prefix with the signs absorbed:
-// q', k', L, beta, sigma_C and L_C.  `first` is the token index of row 0 on the token axis.  Ends
-// with a barrier.
+// q', k', L, beta, sigma_C and L_C.  `first` is the token index of row 0 on the token axis.
+// alpha_out (nullable, [C][DK]) receives the gates themselves (1 past nvalid).  Ends with a
+// barrier.
 template <typename Tin, int DK, int C>
 __device__ __forceinline__ void chunk_prep(const Factors<DK, C>& f, const Tin* __restrict__ q,
                                               const Tin* __restrict__ k,
@@ -56,7 +63,8 @@ __device__ __forceinline__ void chunk_prep(const Factors<DK, C>& f, const Tin* _
                                               const float* __restrict__ beta, size_t first, int t0,
                                               int nvalid, int H, int h, int G, int l2norm,
                                               const RopeParams& rp, const unsigned long long* sfreq,
-                                              long long pos0, int gate_logits) {
+                                              long long pos0, int gate_logits,
+                                              float* alpha_out = nullptr) {
     constexpr int LD = Factors<DK, C>::LD;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     constexpr int NW = kThreads / 32;
@@ -161,6 +169,7 @@ __device__ __forceinline__ void chunk_prep(const Factors<DK, C>& f, const Tin* _
 #pragma unroll
             for (int r = 0; r < AG; ++r) {
                 const float a = av[r];
+                if (alpha_out) alpha_out[(r0 + r) * DK + c] = a;
                 if (a < 0.f) sg = -sg;
                 L += log2f(fmaxf(fabsf(a), kFltMin));
                 f.L[(r0 + r) * LD + c] = L;

@@ -51,11 +51,6 @@ __device__ __forceinline__ void cp16(void* dst, const void* src) {
 __device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-// the first `floats` floats of a chunk record into shared memory (one commit group)
-__device__ __forceinline__ void load_record(float* dst, const float* src, int floats) {
-    for (int i = threadIdx.x; i < floats / 4; i += kThreads) cp16(dst + 4 * i, src + 4 * i);
-    cp_commit();
-}
 
 // ---- 0. every chunk's factors: one CTA per (b*h, chunk) -----------------------------------------
 template <typename T, int DK, int DV, int C>
@@ -94,176 +89,6 @@ bwd_factors_kernel(const T* __restrict__ q, const T* __restrict__ k, const void*
     }
     for (int r = tid; r < C; r += kThreads) rec[R::B + r] = f.b[r];
     for (int c = tid; c < DK; c += kThreads) rec[R::GC + c] = f.sg[c] * exp2f(f.LC[c]);
-}
-
-// ---- 1. the forward replay: one CTA per (b*h, DVS columns of the state) ----------------------------
-//   U~ = T B V,  U = U~ - W S,  S <- Diag(gamma_C) S + K_end^T U;  the state entering every chunk is
-//   written to ws_S.  The next chunk's record is fetched while this one is used.
-template <int DK, int DV, int C>
-struct ReplayShape {
-    static constexpr int DVS = DV < 16 ? DV : 16;
-    static constexpr int REC = Rec<DK, C>::QP;               // the part of a record the replay reads
-    static constexpr int off_v = 2 * REC;                    // two record stages, then V [C][DVS]
-    static constexpr int off_ut = off_v + C * DVS;           // U~ [C][DVS]
-    static constexpr int off_u = off_ut + C * DVS;           // U  [C][DVS]
-    static constexpr int off_s = off_u + C * DVS;            // S  [DK][DVS]
-    static constexpr int total = off_s + DK * DVS;
-    static constexpr size_t bytes = sizeof(float) * (size_t)total;
-};
-
-template <typename T, int DK, int DV, int C>
-__global__ void __launch_bounds__(kThreads)
-bwd_replay_kernel(const T* __restrict__ v, const float* __restrict__ h0,
-                  const float* __restrict__ recs, float* __restrict__ ws_S, int T_len, int H) {
-    using R = Rec<DK, C>;
-    using Sh = ReplayShape<DK, DV, C>;
-    constexpr int DVS = Sh::DVS;
-    extern __shared__ float smem[];
-    float* sv = smem + Sh::off_v;
-    float* sUt = smem + Sh::off_ut;
-    float* sU = smem + Sh::off_u;
-    float* sS = smem + Sh::off_s;
-    const int bh = blockIdx.x, b = bh / H, h = bh % H;
-    const int n0 = blockIdx.y * DVS;
-    const int tid = threadIdx.x;
-    const int nchunks = (T_len + C - 1) / C;
-    const float* rec0 = recs + (size_t)bh * nchunks * R::floats;
-    for (int e = tid; e < DK * DVS; e += kThreads)
-        sS[e] = h0 ? h0[((size_t)bh * DK + e / DVS) * DV + n0 + e % DVS] : 0.f;
-    load_record(smem, rec0, Sh::REC);
-    // this thread's elements of a chunk's V slice, read one chunk ahead into registers
-    constexpr int NE = (C * DVS + kThreads - 1) / kThreads;
-    float rv[NE];
-    auto load_v = [&](int ch) {
-        const int t0 = ch * C, nvalid = min(C, T_len - t0);
-#pragma unroll
-        for (int i = 0; i < NE; ++i) {
-            const int e = tid + i * kThreads, r = e / DVS, n = e % DVS;
-            rv[i] = e < C * DVS && r < nvalid
-                        ? to_f32(v[(((size_t)b * T_len + t0 + r) * H + h) * DV + n0 + n]) : 0.f;
-        }
-    };
-    load_v(0);
-    for (int ch = 0; ch < nchunks; ++ch) {
-        const float* rf = smem + (ch & 1) * Sh::REC;
-#pragma unroll
-        for (int i = 0; i < NE; ++i)
-            if (tid + i * kThreads < C * DVS) sv[tid + i * kThreads] = rv[i];
-        if (ch + 1 < nchunks) {
-            load_v(ch + 1);
-            load_record(smem + ((ch + 1) & 1) * Sh::REC, rec0 + (size_t)(ch + 1) * R::floats, Sh::REC);
-            cp_wait<1>();
-        } else {
-            cp_wait<0>();
-        }
-        float* dst = ws_S + ((size_t)bh * nchunks + ch) * DK * DV + n0;
-        for (int e = tid; e < DK * DVS; e += kThreads) dst[(e / DVS) * DV + e % DVS] = sS[e];
-        __syncthreads();
-        for (int e = tid; e < C * DVS; e += kThreads) {
-            const int r = e / DVS, n = e % DVS;
-            float acc = 0.f;
-            for (int j = 0; j <= r; ++j) acc += rf[R::T + r * C + j] * rf[R::B + j] * sv[j * DVS + n];
-            sUt[e] = acc;
-        }
-        __syncthreads();
-        for (int e = tid; e < C * DVS; e += kThreads) {
-            const int r = e / DVS, n = e % DVS;
-            float acc = sUt[e];
-            for (int c = 0; c < DK; ++c) acc -= rf[R::W + r * DK + c] * sS[c * DVS + n];
-            sU[e] = acc;
-        }
-        __syncthreads();
-        for (int e = tid; e < DK * DVS; e += kThreads) {
-            const int c = e / DVS, n = e % DVS;
-            float acc = rf[R::GC + c] * sS[e];
-            for (int r = 0; r < C; ++r) acc += rf[R::KE + r * DK + c] * sU[r * DVS + n];
-            sS[e] = acc;
-        }
-        __syncthreads();   // this stage is refilled by the next iteration's prefetch
-    }
-}
-
-// ---- 2. the state-gradient chain: one CTA per (b*h, DVS columns of the state) ----------------
-template <int DK, int DV, int C>
-struct ChainShape {
-    static constexpr int DVS = DV < 16 ? DV : 16;
-    static constexpr int REC = Rec<DK, C>::M;                 // the part of a record the chain reads
-    static constexpr int off_do = 2 * REC;                    // two record stages, then dO [C][DVS]
-    static constexpr int off_kd = off_do + C * DVS;           // K_end dS_out [C][DVS]
-    static constexpr int off_ds = off_kd + C * DVS;           // dS_out [DK][DVS]
-    static constexpr int total = off_ds + DK * DVS;
-    static constexpr size_t bytes = sizeof(float) * (size_t)total;
-};
-
-// ws_dS: [B*H][NT][DK][DV] fp32, the gradient with respect to each chunk's end state.
-template <typename T, int DK, int DV, int C>
-__global__ void __launch_bounds__(kThreads)
-bwd_chain_kernel(const T* __restrict__ dout, const float* __restrict__ dhT,
-                 float* __restrict__ dh0, const float* __restrict__ recs, float* __restrict__ ws_dS,
-                 int T_len, int H, float scale) {
-    using R = Rec<DK, C>;
-    using Sh = ChainShape<DK, DV, C>;
-    constexpr int DVS = Sh::DVS;
-    extern __shared__ float smem[];
-    float* sdO = smem + Sh::off_do;
-    float* sKd = smem + Sh::off_kd;
-    float* sdS = smem + Sh::off_ds;
-    const int bh = blockIdx.x, b = bh / H, h = bh % H;
-    const int n0 = blockIdx.y * DVS;
-    const int tid = threadIdx.x;
-    const int nchunks = (T_len + C - 1) / C;
-    const float* rec0 = recs + (size_t)bh * nchunks * R::floats;
-    for (int e = tid; e < DK * DVS; e += kThreads)
-        sdS[e] = dhT ? dhT[((size_t)bh * DK + e / DVS) * DV + n0 + e % DVS] : 0.f;
-    load_record(smem, rec0 + (size_t)(nchunks - 1) * R::floats, Sh::REC);
-    // this thread's elements of a chunk's dO slice, read one chunk ahead into registers
-    constexpr int NE = (C * DVS + kThreads - 1) / kThreads;
-    float rdo[NE];
-    auto load_do = [&](int ch) {
-        const int t0 = ch * C, nvalid = min(C, T_len - t0);
-#pragma unroll
-        for (int i = 0; i < NE; ++i) {
-            const int e = tid + i * kThreads, r = e / DVS, n = e % DVS;
-            rdo[i] = e < C * DVS && r < nvalid
-                         ? to_f32(dout[(((size_t)b * T_len + t0 + r) * H + h) * DV + n0 + n]) : 0.f;
-        }
-    };
-    load_do(nchunks - 1);
-    for (int ch = nchunks - 1, it = 0; ch >= 0; --ch, ++it) {
-        const float* rf = smem + (it & 1) * Sh::REC;
-#pragma unroll
-        for (int i = 0; i < NE; ++i)
-            if (tid + i * kThreads < C * DVS) sdO[tid + i * kThreads] = rdo[i];
-        if (ch > 0) {
-            load_do(ch - 1);
-            load_record(smem + ((it + 1) & 1) * Sh::REC, rec0 + (size_t)(ch - 1) * R::floats, Sh::REC);
-            cp_wait<1>();
-        } else {
-            cp_wait<0>();
-        }
-        float* dst = ws_dS + ((size_t)bh * nchunks + ch) * DK * DV + n0;
-        for (int e = tid; e < DK * DVS; e += kThreads) dst[(e / DVS) * DV + e % DVS] = sdS[e];
-        __syncthreads();
-        for (int e = tid; e < C * DVS; e += kThreads) {   // K_end dS_out
-            const int j = e / DVS, n = e % DVS;
-            float acc = 0.f;
-            for (int c = 0; c < DK; ++c) acc += rf[R::KE + j * DK + c] * sdS[c * DVS + n];
-            sKd[e] = acc;
-        }
-        __syncthreads();
-        // dS_in = scale Q'^T dO + Diag(gamma_C) dS_out - W^T (K_end dS_out)
-        for (int e = tid; e < DK * DVS; e += kThreads) {
-            const int c = e / DVS, n = e % DVS;
-            float acc = rf[R::GC + c] * sdS[e];
-            for (int r = 0; r < C; ++r)
-                acc += scale * rf[R::QP + r * DK + c] * sdO[r * DVS + n] - rf[R::W + r * DK + c] * sKd[r * DVS + n];
-            sdS[e] = acc;   // each element is read only by its own thread above
-        }
-        __syncthreads();   // this stage is refilled by the next iteration's prefetch
-    }
-    if (dh0)
-        for (int e = tid; e < DK * DVS; e += kThreads)
-            dh0[((size_t)bh * DK + e / DVS) * DV + n0 + e % DVS] = sdS[e];
 }
 
 // ---- warp-level tensor-core tiles with fp32-grade products ------------------------------------
@@ -315,6 +140,243 @@ __device__ __forceinline__ void st_frag(float* d, int ld, int col0, const float 
     d[g * ld + col0 + 2 * t + 1] = s * c[1];
     d[(g + 8) * ld + col0 + 2 * t] = s * c[2];
     d[(g + 8) * ld + col0 + 2 * t + 1] = s * c[3];
+}
+
+// ---- a chunk record in shared memory, for the serial passes ----------------------------------------
+// The rows of W, K_end (and Q') are RP = DK + 8 floats apart (the lanes of a warp tile's fragment
+// fall on distinct banks), then T, beta and gamma_C as in the record.
+template <int DK, int C>
+struct Stage {
+    static constexpr int RP = DK + 8;
+    static constexpr int W = 0, KE = C * RP, T = 2 * C * RP, B = T + C * C, GC = B + C;
+    static constexpr int QP = GC + DK;
+    static constexpr int floats_replay = QP, floats_chain = QP + C * RP;
+};
+// the record's W, K_end, T, beta, gamma_C (and Q' when with_qp) into a stage (one commit group)
+template <int DK, int C>
+__device__ __forceinline__ void load_stage(float* dst, const float* rec, bool with_qp) {
+    using R = Rec<DK, C>;
+    using S = Stage<DK, C>;
+    constexpr int RC = DK / 4;   // 16-byte pieces per row
+    const int nrows = with_qp ? 3 * C : 2 * C;
+    for (int i = threadIdx.x; i < nrows * RC; i += kThreads) {
+        const int row = i / RC, c4 = 4 * (i % RC), blk = row / C, r = row % C;
+        const int src = blk == 0 ? R::W : blk == 1 ? R::KE : R::QP;
+        const int d = blk == 0 ? S::W : blk == 1 ? S::KE : S::QP;
+        cp16(dst + d + r * S::RP + c4, rec + src + r * DK + c4);
+    }
+    for (int i = threadIdx.x; i < (C * C + C + DK) / 4; i += kThreads)
+        cp16(dst + S::T + 4 * i, rec + R::T + 4 * i);
+    cp_commit();
+}
+
+// ---- 1. the forward replay: one CTA per (b*h, DVS columns of the state) ----------------------------
+//   U = T B V - W S,  S <- Diag(gamma_C) S + K_end^T U  (warp tiles; the state entering every chunk
+//   is written to ws_S).  The next chunk's record and V slice are fetched while this one is used.
+template <int DK, int DV, int C>
+struct ReplayShape {
+    static constexpr int DVS = DV < 16 ? DV : 16;
+    static constexpr int NT = DVS / 8;                      // 8-column tiles
+    static constexpr int SP = DVS + 8;                      // rows of V, U, S (fragment banks)
+    // the W S product is split over KQ ranges of the state rows (one warp tile each), whose parts
+    // are summed where U is read
+    static constexpr int KQ = (8 / NT) < (DK / 8) ? (8 / NT) : (DK / 8);
+    static constexpr int KC = DK / KQ;
+    static constexpr int REC = Stage<DK, C>::floats_replay;
+    static constexpr int off_v = 2 * REC;                   // two stages, then V [C][SP]
+    static constexpr int off_u = off_v + C * SP;            // parts of U [KQ][C][SP]
+    static constexpr int off_s = off_u + KQ * C * SP;       // S  [DK][SP]
+    static constexpr int total = off_s + DK * SP;
+    static constexpr size_t bytes = sizeof(float) * (size_t)total;
+};
+
+template <typename T, int DK, int DV, int C>
+__global__ void __launch_bounds__(kThreads)
+bwd_replay_kernel(const T* __restrict__ v, const float* __restrict__ h0,
+                  const float* __restrict__ recs, float* __restrict__ ws_S, int T_len, int H) {
+    using R = Rec<DK, C>;
+    using St = Stage<DK, C>;
+    using Sh = ReplayShape<DK, DV, C>;
+    constexpr int DVS = Sh::DVS, NT = Sh::NT, SP = Sh::SP, RP = St::RP, KQ = Sh::KQ, KC = Sh::KC;
+    extern __shared__ float smem[];
+    float* sv = smem + Sh::off_v;
+    float* sU = smem + Sh::off_u;
+    float* sS = smem + Sh::off_s;
+    const int bh = blockIdx.x, b = bh / H, h = bh % H;
+    const int n0 = blockIdx.y * DVS;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int nchunks = (T_len + C - 1) / C;
+    const float* rec0 = recs + (size_t)bh * nchunks * R::floats;
+    for (int e = tid; e < DK * DVS; e += kThreads)
+        sS[(e / DVS) * SP + e % DVS] = h0 ? h0[((size_t)bh * DK + e / DVS) * DV + n0 + e % DVS] : 0.f;
+    load_stage<DK, C>(smem, rec0, false);
+    // this thread's elements of a chunk's V slice, read one chunk ahead into registers
+    constexpr int NE = (C * DVS + kThreads - 1) / kThreads;
+    float rv[NE];
+    auto load_v = [&](int ch) {
+        const int t0 = ch * C, nvalid = min(C, T_len - t0);
+#pragma unroll
+        for (int i = 0; i < NE; ++i) {
+            const int e = tid + i * kThreads, r = e / DVS, n = e % DVS;
+            rv[i] = e < C * DVS && r < nvalid
+                        ? to_f32(v[(((size_t)b * T_len + t0 + r) * H + h) * DV + n0 + n]) : 0.f;
+        }
+    };
+    load_v(0);
+    for (int ch = 0; ch < nchunks; ++ch) {
+        const float* rf = smem + (ch & 1) * Sh::REC;
+#pragma unroll
+        for (int i = 0; i < NE; ++i) {
+            const int e = tid + i * kThreads;
+            if (e < C * DVS) sv[(e / DVS) * SP + e % DVS] = rv[i];
+        }
+        if (ch + 1 < nchunks) {
+            load_v(ch + 1);
+            load_stage<DK, C>(smem + ((ch + 1) & 1) * Sh::REC, rec0 + (size_t)(ch + 1) * R::floats, false);
+            cp_wait<1>();
+        } else {
+            cp_wait<0>();
+        }
+        float* dst = ws_S + ((size_t)bh * nchunks + ch) * DK * DV + n0;
+        for (int e = tid; e < DK * DVS; e += kThreads) dst[(e / DVS) * DV + e % DVS] = sS[(e / DVS) * SP + e % DVS];
+        __syncthreads();
+        if (warp < NT * KQ) {   // part kq of U = T B V - W S, columns 8 nt ..
+            const int nt = warp % NT, kq = warp / NT;
+            float c[4] = {0.f, 0.f, 0.f, 0.f};
+            if (kq == 0)
+                mma3_tile<C>(c, [&](int m, int k) { return rf[St::T + m * C + k] * rf[St::B + k]; },
+                             [&](int k, int n) { return sv[k * SP + 8 * nt + n]; }, lane);
+            mma3_tile<KC>(c, [&](int m, int k) { return -rf[St::W + m * RP + kq * KC + k]; },
+                          [&](int k, int n) { return sS[(kq * KC + k) * SP + 8 * nt + n]; }, lane);
+            st_frag(sU + kq * C * SP, SP, 8 * nt, c, 1.f, lane);
+        }
+        __syncthreads();
+        auto u_at = [&](int r, int n) {
+            float x = 0.f;
+#pragma unroll
+            for (int kq = 0; kq < KQ; ++kq) x += sU[kq * C * SP + r * SP + n];
+            return x;
+        };
+        // S <- Diag(gamma_C) S + K_end^T U: (DK / 16) x NT tiles, each read and written in place
+        for (int id = warp; id < (DK / 16) * NT; id += kThreads / 32) {
+            const int r0 = 16 * (id / NT), c0 = 8 * (id % NT) + 2 * t;
+            float c[4];
+            c[0] = rf[St::GC + r0 + g] * sS[(r0 + g) * SP + c0];
+            c[1] = rf[St::GC + r0 + g] * sS[(r0 + g) * SP + c0 + 1];
+            c[2] = rf[St::GC + r0 + g + 8] * sS[(r0 + g + 8) * SP + c0];
+            c[3] = rf[St::GC + r0 + g + 8] * sS[(r0 + g + 8) * SP + c0 + 1];
+            mma3_tile<C>(c, [&](int m, int k) { return rf[St::KE + k * RP + r0 + m]; },
+                         [&](int k, int n) { return u_at(k, 8 * (id % NT) + n); }, lane);
+            st_frag(sS + r0 * SP, SP, 8 * (id % NT), c, 1.f, lane);
+        }
+        __syncthreads();   // this stage is refilled by the next iteration's prefetch
+    }
+}
+
+// ---- 2. the state-gradient chain: one CTA per (b*h, DVS columns of the state) ----------------
+//   K_d = K_end dS_out,  dS_in = Diag(gamma_C) dS_out + scale Q'^T dO - W^T K_d  (warp tiles)
+template <int DK, int DV, int C>
+struct ChainShape {
+    static constexpr int DVS = DV < 16 ? DV : 16;
+    static constexpr int NT = DVS / 8;
+    static constexpr int SP = DVS + 8;
+    static constexpr int KQ = (8 / NT) < (DK / 8) ? (8 / NT) : (DK / 8);   // as in the replay
+    static constexpr int KC = DK / KQ;
+    static constexpr int REC = Stage<DK, C>::floats_chain;
+    static constexpr int off_do = 2 * REC;                    // two stages, then dO [C][SP]
+    static constexpr int off_kd = off_do + C * SP;            // parts of K_end dS_out [KQ][C][SP]
+    static constexpr int off_ds = off_kd + KQ * C * SP;       // dS_out [DK][SP]
+    static constexpr int total = off_ds + DK * SP;
+    static constexpr size_t bytes = sizeof(float) * (size_t)total;
+};
+
+// ws_dS: [B*H][NT][DK][DV] fp32, the gradient with respect to each chunk's end state.
+template <typename T, int DK, int DV, int C>
+__global__ void __launch_bounds__(kThreads)
+bwd_chain_kernel(const T* __restrict__ dout, const float* __restrict__ dhT,
+                 float* __restrict__ dh0, const float* __restrict__ recs, float* __restrict__ ws_dS,
+                 int T_len, int H, float scale) {
+    using R = Rec<DK, C>;
+    using St = Stage<DK, C>;
+    using Sh = ChainShape<DK, DV, C>;
+    constexpr int DVS = Sh::DVS, NT = Sh::NT, SP = Sh::SP, RP = St::RP, KQ = Sh::KQ, KC = Sh::KC;
+    extern __shared__ float smem[];
+    float* sdO = smem + Sh::off_do;
+    float* sKd = smem + Sh::off_kd;
+    float* sdS = smem + Sh::off_ds;
+    const int bh = blockIdx.x, b = bh / H, h = bh % H;
+    const int n0 = blockIdx.y * DVS;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int nchunks = (T_len + C - 1) / C;
+    const float* rec0 = recs + (size_t)bh * nchunks * R::floats;
+    for (int e = tid; e < DK * DVS; e += kThreads)
+        sdS[(e / DVS) * SP + e % DVS] = dhT ? dhT[((size_t)bh * DK + e / DVS) * DV + n0 + e % DVS] : 0.f;
+    load_stage<DK, C>(smem, rec0 + (size_t)(nchunks - 1) * R::floats, true);
+    // this thread's elements of a chunk's dO slice, read one chunk ahead into registers
+    constexpr int NE = (C * DVS + kThreads - 1) / kThreads;
+    float rdo[NE];
+    auto load_do = [&](int ch) {
+        const int t0 = ch * C, nvalid = min(C, T_len - t0);
+#pragma unroll
+        for (int i = 0; i < NE; ++i) {
+            const int e = tid + i * kThreads, r = e / DVS, n = e % DVS;
+            rdo[i] = e < C * DVS && r < nvalid
+                         ? to_f32(dout[(((size_t)b * T_len + t0 + r) * H + h) * DV + n0 + n]) : 0.f;
+        }
+    };
+    load_do(nchunks - 1);
+    for (int ch = nchunks - 1, it = 0; ch >= 0; --ch, ++it) {
+        const float* rf = smem + (it & 1) * Sh::REC;
+#pragma unroll
+        for (int i = 0; i < NE; ++i) {
+            const int e = tid + i * kThreads;
+            if (e < C * DVS) sdO[(e / DVS) * SP + e % DVS] = rdo[i];
+        }
+        if (ch > 0) {
+            load_do(ch - 1);
+            load_stage<DK, C>(smem + ((it + 1) & 1) * Sh::REC, rec0 + (size_t)(ch - 1) * R::floats, true);
+            cp_wait<1>();
+        } else {
+            cp_wait<0>();
+        }
+        float* dst = ws_dS + ((size_t)bh * nchunks + ch) * DK * DV + n0;
+        for (int e = tid; e < DK * DVS; e += kThreads) dst[(e / DVS) * DV + e % DVS] = sdS[(e / DVS) * SP + e % DVS];
+        __syncthreads();
+        if (warp < NT * KQ) {   // part kq of K_end dS_out, columns 8 nt ..
+            const int nt = warp % NT, kq = warp / NT;
+            float c[4] = {0.f, 0.f, 0.f, 0.f};
+            mma3_tile<KC>(c, [&](int m, int k) { return rf[St::KE + m * RP + kq * KC + k]; },
+                          [&](int k, int n) { return sdS[(kq * KC + k) * SP + 8 * nt + n]; }, lane);
+            st_frag(sKd + kq * C * SP, SP, 8 * nt, c, 1.f, lane);
+        }
+        __syncthreads();
+        auto kd_at = [&](int r, int n) {
+            float x = 0.f;
+#pragma unroll
+            for (int kq = 0; kq < KQ; ++kq) x += sKd[kq * C * SP + r * SP + n];
+            return x;
+        };
+        // dS_in = Diag(gamma_C) dS_out + scale Q'^T dO - W^T K_d, tiles read and written in place
+        for (int id = warp; id < (DK / 16) * NT; id += kThreads / 32) {
+            const int r0 = 16 * (id / NT), nt = id % NT, c0 = 8 * nt + 2 * t;
+            float c[4];
+            c[0] = rf[St::GC + r0 + g] * sdS[(r0 + g) * SP + c0];
+            c[1] = rf[St::GC + r0 + g] * sdS[(r0 + g) * SP + c0 + 1];
+            c[2] = rf[St::GC + r0 + g + 8] * sdS[(r0 + g + 8) * SP + c0];
+            c[3] = rf[St::GC + r0 + g + 8] * sdS[(r0 + g + 8) * SP + c0 + 1];
+            mma3_tile<C>(c, [&](int m, int k) { return scale * rf[St::QP + k * RP + r0 + m]; },
+                         [&](int k, int n) { return sdO[k * SP + 8 * nt + n]; }, lane);
+            mma3_tile<C>(c, [&](int m, int k) { return -rf[St::W + k * RP + r0 + m]; },
+                         [&](int k, int n) { return kd_at(k, 8 * nt + n); }, lane);
+            st_frag(sdS + r0 * SP, SP, 8 * nt, c, 1.f, lane);
+        }
+        __syncthreads();   // this stage is refilled by the next iteration's prefetch
+    }
+    if (dh0)
+        for (int e = tid; e < DK * DVS; e += kThreads)
+            dh0[((size_t)bh * DK + e / DVS) * DV + n0 + e % DVS] = sdS[(e / DVS) * SP + e % DVS];
 }
 
 // ---- 3. the gradients of one chunk: one CTA per (b*h, chunk), all dv in tiles of DT ----------

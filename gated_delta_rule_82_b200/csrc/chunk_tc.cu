@@ -186,12 +186,14 @@ struct TcMaps {
 
 // Issue the TMA loads of the chunk of batch b, value head h (q/k head hk) starting at token t0:
 // alpha -> G, q -> QR, k -> KR on bar_in; V (two 64-column halves, 128-byte swizzle) on bar_v.
-// Rows past the sequence end read as zeros.
+// Rows past the sequence end read as zeros.  alpha, the largest input, is read once (one value
+// head), so its lines go first when L2 evicts (the workspace images stay).
 __device__ __forceinline__ void issue_inputs(const TcMaps& m, uint8_t* sm, uint64_t* bar_in,
                                              int b, int h, int hk, int t0, int gate_logits) {
     // gate values: fp32 [64][128] into G; logits: bf16 [64][128] into the upper half of G
     tc::mbar_arrive_expect_tx(bar_in, gate_logits ? kInBytes - 16384 : kInBytes);
-    tc::tma_load_4d(sm + S_G + (gate_logits ? 16384 : 0), &m.alpha, 0, h, t0, b, bar_in);
+    tc::tma_load_4d_hint(sm + S_G + (gate_logits ? 16384 : 0), &m.alpha, 0, h, t0, b, bar_in,
+                         tc::policy_evict_first());
     tc::tma_load_4d(sm + S_QR, &m.q, 0, hk, t0, b, bar_in);
     tc::tma_load_4d(sm + S_KR, &m.k, 0, hk, t0, b, bar_in);
 }
@@ -1133,14 +1135,17 @@ struct SegIter {
 };
 
 // kSeg: the items are the chunks of segment units (SegArgs) head0, head0 + hstride, ... instead of
-// whole head units; in the summary pass there are no outputs.
+// whole head units; in the summary pass there are no outputs.  discard: each chunk-head's image is
+// dropped from L2 once both of its copies have landed (the images of one fused launch are read
+// once; without it the dirty lines that L2 evicts are written back to DRAM).
 template <bool kSeg>
 __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, const uint8_t* __restrict__ ws,
                                            const int* __restrict__ flags, PackedTabs pt,
                                            const float* __restrict__ h0,
                                            __nv_bfloat16* __restrict__ out, float* __restrict__ hT,
                                            int T_len, int H, int NT, int BH, float scale, int head0,
-                                           int hstride, uint32_t tmem, SegArgs sa) {
+                                           int hstride, uint32_t tmem, SegArgs sa,
+                                           bool discard) {
     uint64_t* full_c = reinterpret_cast<uint64_t*>(sm + SS_BAR);   // [2] A_c, K_end, U~^T landed
     uint64_t* empty_c = full_c + 2;     // [2] chain stage read by the chain products (commit)
     uint64_t* full_o = empty_c + 2;     // [2] Q', U~^T, M landed
@@ -1370,7 +1375,8 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
         // ---- output issue: S^T Q'^T (A in TMEM) + U~^T M^T (both from shared memory) ----
         const uint32_t ido = tc::idesc_bf16_f32(128, 64, 0, 0);
         const uint64_t o_desc0 = tc::smem_desc_sw128(tc::smem_u32(sm + SS_O), 16, 1024);
-        for (int u = 0; u < (outputs ? U : 0); ++u) {
+        int nc = U > 0 && !kSeg ? units_chunks(head0) : 0;
+        for (int u = 0, c = 0, bh = head0; u < (outputs ? U : 0); ++u) {
             const int st = u & 1, ob = u & 3;
             if (!wait(&full_o[st], (u >> 1) & 1)) break;
             // issued once D_c(u) has completed, so it never shares the tensor pipe with a chain
@@ -1392,6 +1398,19 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
                                   ido, 1u);
             tc::mma_commit_warp(&mma_o[ob]);
             tc::mma_commit_warp(&empty_o[st]);
+            if constexpr (!kSeg) {
+                // both copies of this item's image have landed (its output stage above, its chain
+                // stage before D_c(u) completed)
+                if (discard) {
+                    const uint8_t* img = ws + ((size_t)bh * NT + c) * WS_CHUNK;
+                    for (int i = lane; i < (int)(WS_CHUNK / 128); i += 32) tc::discard_l2(img + 128 * i);
+                }
+                if (++c == nc) {
+                    c = 0;
+                    bh += hstride;
+                    if (u + 1 < U) nc = units_chunks(bh);
+                }
+            }
         }
     } else if (warp == 10 || warp == 11) {
         // ---- loads: warp 10 the chain stages, warp 11 the output stages ----
@@ -1561,7 +1580,7 @@ ckda_tc_state(const __grid_constant__ TcMaps maps, const uint8_t* __restrict__ w
     __shared__ uint32_t tmem_slot;
     const uint32_t tmem = kernel_tmem_alloc(&tmem_slot);
     state_role<false>(aligned_smem(smem_raw), maps, ws, flags, pt, h0, out, hT, T_len, H, NT, BH,
-                      scale, blockIdx.x, gridDim.x, tmem, SegArgs{});
+                      scale, blockIdx.x, gridDim.x, tmem, SegArgs{}, false);
     kernel_tmem_free(tmem);
 }
 
@@ -1592,7 +1611,7 @@ ckda_tc_fused(const __grid_constant__ TcMaps maps, const void* __restrict__ alph
                             rp, pos_offset, tmem);
     if (chain)
         state_role<false>(sm, maps, ws, flags, pt, h0, out, hT, T_len, H, NT, BH, scale, b, n_state,
-                          tmem, SegArgs{});
+                          tmem, SegArgs{}, (reinterpret_cast<uintptr_t>(ws) & 127) == 0);
     kernel_tmem_free(tmem);
 }
 
@@ -1606,7 +1625,7 @@ ckda_tc_seg(const __grid_constant__ TcMaps maps, const uint8_t* __restrict__ ws,
     __shared__ uint32_t tmem_slot;
     const uint32_t tmem = kernel_tmem_alloc(&tmem_slot);
     state_role<true>(aligned_smem(smem_raw), maps, ws, flags, PackedTabs{nullptr, nullptr, nullptr},
-                     h0, out, hT, T_len, H, NT, BH, scale, blockIdx.x, gridDim.x, tmem, sa);
+                     h0, out, hT, T_len, H, NT, BH, scale, blockIdx.x, gridDim.x, tmem, sa, false);
     kernel_tmem_free(tmem);
 }
 

@@ -86,6 +86,21 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const void* map, int c0, 
         ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2),
           "r"(c3), "r"(smem_u32(bar)) : "memory");
 }
+// The same with an L2 cache policy (createpolicy), e.g. evict-first for data read once.
+__device__ __forceinline__ void tma_load_4d_hint(void* dst, const void* map, int c0, int c1, int c2,
+                                                 int c3, uint64_t* bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6], %7;"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2),
+          "r"(c3), "r"(smem_u32(bar)), "l"(policy) : "memory");
+}
+// An L2 policy under which the accessed lines are the first to be evicted.
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
 __device__ __forceinline__ void prefetch_tensormap(const void* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -138,6 +153,11 @@ __device__ __forceinline__ void bulk_wait_read() {
 // Wait until every committed bulk store has completed.
 __device__ __forceinline__ void bulk_wait_all() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// Drop the 128-byte L2 line at p (128-byte aligned) without writing it back: its contents become
+// unspecified.  For data that is dead once read (it saves the write-back of a dirty line).
+__device__ __forceinline__ void discard_l2(const void* p) {
+    asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
 }
 // Ask the memory system to bring [p, p + bytes) into L2 (p and bytes 16-byte aligned).
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {

@@ -1135,17 +1135,14 @@ struct SegIter {
 };
 
 // kSeg: the items are the chunks of segment units (SegArgs) head0, head0 + hstride, ... instead of
-// whole head units; in the summary pass there are no outputs.  discard: each chunk-head's image is
-// dropped from L2 once both of its copies have landed (the images of one fused launch are read
-// once; without it the dirty lines that L2 evicts are written back to DRAM).
+// whole head units; in the summary pass there are no outputs.
 template <bool kSeg>
 __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, const uint8_t* __restrict__ ws,
                                            const int* __restrict__ flags, PackedTabs pt,
                                            const float* __restrict__ h0,
                                            __nv_bfloat16* __restrict__ out, float* __restrict__ hT,
                                            int T_len, int H, int NT, int BH, float scale, int head0,
-                                           int hstride, uint32_t tmem, SegArgs sa,
-                                           bool discard) {
+                                           int hstride, uint32_t tmem, SegArgs sa) {
     uint64_t* full_c = reinterpret_cast<uint64_t*>(sm + SS_BAR);   // [2] A_c, K_end, U~^T landed
     uint64_t* empty_c = full_c + 2;     // [2] chain stage read by the chain products (commit)
     uint64_t* full_o = empty_c + 2;     // [2] Q', U~^T, M landed
@@ -1375,8 +1372,7 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
         // ---- output issue: S^T Q'^T (A in TMEM) + U~^T M^T (both from shared memory) ----
         const uint32_t ido = tc::idesc_bf16_f32(128, 64, 0, 0);
         const uint64_t o_desc0 = tc::smem_desc_sw128(tc::smem_u32(sm + SS_O), 16, 1024);
-        int nc = U > 0 && !kSeg ? units_chunks(head0) : 0;
-        for (int u = 0, c = 0, bh = head0; u < (outputs ? U : 0); ++u) {
+        for (int u = 0; u < (outputs ? U : 0); ++u) {
             const int st = u & 1, ob = u & 3;
             if (!wait(&full_o[st], (u >> 1) & 1)) break;
             // issued once D_c(u) has completed, so it never shares the tensor pipe with a chain
@@ -1398,19 +1394,6 @@ __device__ __forceinline__ void state_role(uint8_t* sm, const TcMaps& maps, cons
                                   ido, 1u);
             tc::mma_commit_warp(&mma_o[ob]);
             tc::mma_commit_warp(&empty_o[st]);
-            if constexpr (!kSeg) {
-                // both copies of this item's image have landed (its output stage above, its chain
-                // stage before D_c(u) completed)
-                if (discard) {
-                    const uint8_t* img = ws + ((size_t)bh * NT + c) * WS_CHUNK;
-                    for (int i = lane; i < (int)(WS_CHUNK / 128); i += 32) tc::discard_l2(img + 128 * i);
-                }
-                if (++c == nc) {
-                    c = 0;
-                    bh += hstride;
-                    if (u + 1 < U) nc = units_chunks(bh);
-                }
-            }
         }
     } else if (warp == 10 || warp == 11) {
         // ---- loads: warp 10 the chain stages, warp 11 the output stages ----
@@ -1580,7 +1563,7 @@ ckda_tc_state(const __grid_constant__ TcMaps maps, const uint8_t* __restrict__ w
     __shared__ uint32_t tmem_slot;
     const uint32_t tmem = kernel_tmem_alloc(&tmem_slot);
     state_role<false>(aligned_smem(smem_raw), maps, ws, flags, pt, h0, out, hT, T_len, H, NT, BH,
-                      scale, blockIdx.x, gridDim.x, tmem, SegArgs{}, false);
+                      scale, blockIdx.x, gridDim.x, tmem, SegArgs{});
     kernel_tmem_free(tmem);
 }
 
@@ -1611,7 +1594,7 @@ ckda_tc_fused(const __grid_constant__ TcMaps maps, const void* __restrict__ alph
                             rp, pos_offset, tmem);
     if (chain)
         state_role<false>(sm, maps, ws, flags, pt, h0, out, hT, T_len, H, NT, BH, scale, b, n_state,
-                          tmem, SegArgs{}, (reinterpret_cast<uintptr_t>(ws) & 127) == 0);
+                          tmem, SegArgs{});
     kernel_tmem_free(tmem);
 }
 
@@ -1625,7 +1608,7 @@ ckda_tc_seg(const __grid_constant__ TcMaps maps, const uint8_t* __restrict__ ws,
     __shared__ uint32_t tmem_slot;
     const uint32_t tmem = kernel_tmem_alloc(&tmem_slot);
     state_role<true>(aligned_smem(smem_raw), maps, ws, flags, PackedTabs{nullptr, nullptr, nullptr},
-                     h0, out, hT, T_len, H, NT, BH, scale, blockIdx.x, gridDim.x, tmem, sa, false);
+                     h0, out, hT, T_len, H, NT, BH, scale, blockIdx.x, gridDim.x, tmem, sa);
     kernel_tmem_free(tmem);
 }
 

@@ -154,11 +154,6 @@ __device__ __forceinline__ void bulk_wait_read() {
 __device__ __forceinline__ void bulk_wait_all() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
-// Drop the 128-byte L2 line at p (128-byte aligned) without writing it back: its contents become
-// unspecified.  For data that is dead once read (it saves the write-back of a dirty line).
-__device__ __forceinline__ void discard_l2(const void* p) {
-    asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
-}
 // Ask the memory system to bring [p, p + bytes) into L2 (p and bytes 16-byte aligned).
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");

@@ -605,7 +605,8 @@ def main():
         ms_b = event_time_ms(fnB, nB, stream) / nB
         extras["backward"] = {
             "workload": f"{w['name']} (B={B},T={T},H={H},dk=dv={dk}) with h0, dout and dhT: dq, dk, "
-                        "dv, dalpha, dbeta, dh0 in fp32 (CUDA cores, 16-token chunks)",
+                        "dv, dalpha, dbeta, dh0, fp32-grade (CUDA cores and split-tf32 warp tiles, "
+                        "16-token chunks)",
             "ms": round(ms_b, 3), "mtok_s": round(B * T / (ms_b / 1e3) / 1e6, 3),
             "over_forward": round(ms_b / ms_local, 1)}
         del bw, dout, dhT, wsb

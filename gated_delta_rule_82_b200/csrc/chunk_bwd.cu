@@ -1,5 +1,6 @@
-// chunk_bwd.cu -- gradients of the CKDA forward on CUDA cores (fp32): of L = <dout, out> +
-// <dhT, hT> with respect to q, k, v, alpha, beta and h0.
+// chunk_bwd.cu -- gradients of the CKDA forward in fp32-grade arithmetic: of L = <dout, out> +
+// <dhT, hT> with respect to q, k, v, alpha, beta and h0.  fp32 on the CUDA cores, and the dense
+// products (one chunk is 16 rows) as warp-level tensor-core tiles with split tf32 operands.
 //
 // The backward runs the chunked form in reverse (derived from the transition of the "Complex
 // KDA" paper summary, "Background"; the chunk factors are those of simt_chunk.cuh, with the gate

@@ -61,6 +61,13 @@ def test_segments_ragged():
     check(2, 64 * 37 + 13, 2, 5, h0_std=0.05, seed=5)
 
 
+@pytest.mark.parametrize("T,segments", [(130, 50), (64, 8), (1, 4), (200, 0)])
+def test_segments_few_chunks(T, segments):
+    """More segments asked for than there are chunks (one chunk per segment, or the single
+    fused launch when there is one chunk), and the automatic count (0), without h0."""
+    check(1, T, 2, segments, h0_std=0.0, seed=T)
+
+
 def test_segments_long_memory():
     """Slowly decaying signed gates and strong reflections from a nonzero h0: the state entering
     a segment depends on every earlier one, so the transitions F_s and the scan are exercised."""

@@ -250,6 +250,7 @@ ckda_status ckda_fwd_segmented(const void* q, const void* k, const void* v, cons
                                size_t workspace_bytes, ckda_stream_t stream) {
     if (segments < 1) return CKDA_ERR_ARG;
     if (flags.path == CKDA_PATH_SIMT) return CKDA_ERR_UNSUPPORTED;
+    flags.stages = 0;   // (ignored here: segments = 1 is the single fused launch)
     const PackedSeqs none{nullptr, nullptr, 0};
     return fwd_impl(q, k, v, alpha, beta, h0, out, hT, B, T, H, dk, dv, 64, flags, dtype,
                     pos_offset, workspace, workspace_bytes, none, (cudaStream_t)stream, segments);

@@ -68,6 +68,8 @@ def _load():
     lib.ckda_fwd_segmented_workspace_bytes.argtypes = [I] * 6
     lib.ckda_fwd_segmented.restype = I
     lib.ckda_fwd_segmented.argtypes = [P] * 8 + [I] * 5 + [_Flags, I, LL, I, P, SZ, P]
+    lib.ckda_fwd_simt_workspace_bytes.restype = SZ
+    lib.ckda_fwd_simt_workspace_bytes.argtypes = [I] * 5
     lib.ckda_fwd_segments_auto.restype = I
     lib.ckda_fwd_segments_auto.argtypes = [I, I, I]
     lib.ckda_fwd_varlen_workspace_bytes.restype = SZ
@@ -195,6 +197,8 @@ def fwd_chunked(q, k, v, alpha, beta, h0=None, *, chunk=64, l2norm=True, rope_th
     code = _dtype_code(q)
     if workspace is None:   # (a workspace given is checked against the need by the library)
         need = workspace_bytes(B, T, H, dk, dv, chunk, q.dtype, path)
+        if need == 0:   # the CUDA-core path: the workspace of its record form
+            need = int(_load().ckda_fwd_simt_workspace_bytes(B, T, H, dk, dv))
         if need:
             workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()

@@ -6,6 +6,7 @@
 #include <string.h>
 
 #include "internal.cuh"
+#include "simt_records.h"
 
 using namespace ckda;
 
@@ -209,6 +210,21 @@ ckda_status fwd_impl(const void* q, const void* k, const void* v, const void* al
                                          scale, pos_offset, flags.gate_logits, workspace,
                                          flags.stages, pk, stream));
     }
+    // CUDA-core path: the record form when the caller gives it a workspace (batched sequences)
+    if (!packed && workspace) {
+        const size_t need = simt_records_bytes(B, T, H, dk);
+        if (workspace_bytes >= need) {
+            if (!aligned16(workspace)) return CKDA_ERR_ALIGN;
+            const void* all[] = {q, k, v, alpha, beta, h0, out, hT};
+            const size_t allsz[] = {nqk * es, nqk * es, nv * es, asz, (size_t)ntok * H * 4,
+                                    nst * 4, nv * es, nst * 4};
+            for (int i = 0; i < 8; ++i)
+                if (all[i] && overlap(workspace, need, all[i], allsz[i])) return CKDA_ERR_ARG;
+            const SimtArgs a{q, k, v, alpha, beta, h0, out, hT, B, T, nullptr, H, G, l2, rp,
+                             scale, pos_offset, flags.gate_logits};
+            return from_cuda(launch_chunk_simt_records(a, dk, dv, dtype, workspace, stream));
+        }
+    }
     return from_cuda(launch_chunk_simt(q, k, v, alpha, beta, h0, out, hT, B, T, H, G, dk, dv, chunk,
                                        l2, rp, scale, pos_offset, flags.gate_logits, dtype, pk,
                                        stream));
@@ -226,6 +242,13 @@ ckda_status ckda_fwd_chunked(const void* q, const void* k, const void* v, const 
     const PackedSeqs none{nullptr, nullptr, 0};
     return fwd_impl(q, k, v, alpha, beta, h0, out, hT, B, T, H, dk, dv, chunk, flags, dtype,
                     pos_offset, workspace, workspace_bytes, none, (cudaStream_t)stream);
+}
+
+size_t ckda_fwd_simt_workspace_bytes(int B, int T, int H, int dk, int dv) {
+    if (B < 1 || T < 1 || H < 1) return (size_t)-1;
+    if (!supported_dim(dk) || !supported_dim(dv)) return (size_t)-1;
+    if ((long long)B * T * H * 128 > (1ll << 40)) return (size_t)-1;
+    return simt_records_bytes(B, T, H, dk);
 }
 
 int ckda_fwd_segments_auto(int B, int T, int H) {

@@ -192,6 +192,18 @@ CKDA_API ckda_status ckda_fwd_chunked(const void* q, const void* k, const void* 
                              size_t workspace_bytes, ckda_stream_t stream);
 
 /*
+ * Bytes of the optional workspace of the CUDA-core path (flags.path = CKDA_PATH_SIMT, or sizes
+ * the tensor-core path does not take), or (size_t)-1 for invalid sizes.  Given to
+ * ckda_fwd_chunked as its workspace (at least this many bytes, 16-byte aligned), it selects the
+ * record form of that path: every 16-token chunk's factors formed once, chunk-parallel, and the
+ * serial pass over the chunks with the products on warp-level tensor-core tiles (split tf32
+ * operands, fp32-grade); without it (and for packed sequences) the path recomputes the chunk
+ * factors in plain fp32 loops per 16 state columns.  Both give the recurrence up to rounding.
+ * ckda_fwd_workspace_bytes reports 0 for this path (the workspace is not required).
+ */
+CKDA_API size_t ckda_fwd_simt_workspace_bytes(int B, int T, int H, int dk, int dv);
+
+/*
  * The chunked forward with a segment-parallel state pass (tensor-core path only: bf16,
  * dk = dv = 128, chunk 64; batched sequences).  The serial pass over the chunks of every
  * (batch, head) is split into `segments` segments of L = ceil(ceil(T/64) / segments) chunks

@@ -35,7 +35,8 @@ def test_header_declares_the_boundary():
                  "ckda_qk_prologue", "ckda_strerror", "ckda_abi_version", "ckda_fwd_varlen",
                  "ckda_fwd_varlen_workspace_bytes", "ckda_last_device_status",
                  "ckda_set_wait_limit_ns", "ckda_fwd_chunked_noalloc", "ckda_fwd_segmented",
-                 "ckda_fwd_segmented_workspace_bytes", "ckda_fwd_segments_auto"):
+                 "ckda_fwd_segmented_workspace_bytes", "ckda_fwd_segments_auto",
+                 "ckda_fwd_simt_workspace_bytes"):
         assert want in names
 
 
@@ -131,6 +132,15 @@ def fwd_seg(lib, q=P, k=9 * P, v=17 * P, a=25 * P, b=40 * P, h0=None, out=50 * P
 ])
 def test_segmented_validation(lib, kw, want):
     assert fwd_seg(lib, **kw) == want
+
+
+def test_simt_workspace_query(lib):
+    # the record form of the CUDA-core path: 7056 floats per 16-token chunk and head at dk = 128
+    assert lib.ckda_fwd_simt_workspace_bytes(2, 2048, 16, 128, 128) == 2 * 16 * 128 * 7056 * 4
+    assert lib.ckda_fwd_simt_workspace_bytes(1, 17, 1, 16, 16) == 2 * (3 * 16 * 16 + 3 * 256 + 16 + 16) * 4
+    bad = ctypes.c_size_t(-1).value
+    assert lib.ckda_fwd_simt_workspace_bytes(1, 0, 1, 16, 16) == bad
+    assert lib.ckda_fwd_simt_workspace_bytes(1, 64, 1, 24, 16) == bad
 
 
 def test_segmented_workspace_and_count(lib):

@@ -177,12 +177,15 @@ def test_decode_batched_all_steps():
 # ---- chunked forward, CUDA-core path --------------------------------------------------------
 
 def _fwd_check(B, T, H, dk, dv, chunk, *, dtype, kind="ckda", rope=(0.0, 0), pos=0, h0_std=0.0,
-               path="simt", seed=0, tol_o=None, tol_s=None, want_state=True):
+               path="simt", seed=0, tol_o=None, tol_s=None, want_state=True, plain=False):
+    """The CUDA-core path in its record form (the binding gives it its workspace), or with
+    plain=True in the form without a workspace (the chunk factors recomputed per column slice)."""
     theta, conv = rope
     d, g = fwd_case(B, T, H, dk, dv, kind=kind, dtype=dtype, h0_std=h0_std, seed=seed)
+    kw = {"workspace": torch.empty(0, dtype=torch.uint8, device="cuda")} if plain else {}
     out, hT = ck.fwd_chunked(g["q"], g["k"], g["v"], g["alpha"], g["beta"], g["h0"], chunk=chunk,
                              rope_theta=theta, rope_convention=conv, pos_offset=pos, path=path,
-                             want_state=want_state)
+                             want_state=want_state, **kw)
     torch.cuda.synchronize()
     o_ref, s_ref = oracle_fwd(d, rope_theta=theta, rope_convention=conv, pos_offset=pos)
     eo = rel_err(out, o_ref)
@@ -200,10 +203,12 @@ def test_fwd_tiny_fp32():
     _fwd_check(w["B"], w["T"], w["H"], w["dk"], w["dv"], w["chunk"], dtype="f32", kind="tiny")
 
 
+@pytest.mark.parametrize("plain", [False, True])
 @pytest.mark.parametrize("chunk", [16, 32, 64])
-@pytest.mark.parametrize("dk,dv", [(16, 16), (32, 64), (64, 32), (128, 128)])
-def test_fwd_simt_sizes(chunk, dk, dv):
-    _fwd_check(2, 100, 2, dk, dv, chunk, dtype="f32", kind="tiny", h0_std=0.5, seed=chunk + dk)
+@pytest.mark.parametrize("dk,dv", [(16, 16), (32, 64), (64, 32), (128, 128), (128, 16), (16, 128)])
+def test_fwd_simt_sizes(chunk, dk, dv, plain):
+    _fwd_check(2, 100, 2, dk, dv, chunk, dtype="f32", kind="tiny", h0_std=0.5, seed=chunk + dk,
+               plain=plain)
 
 
 @pytest.mark.parametrize("kind", ["ckda", "kda"])
@@ -211,15 +216,18 @@ def test_fwd_simt_bf16(kind):
     _fwd_check(2, 150, 3, 64, 64, 32, dtype="bf16", kind=kind, h0_std=0.02, seed=5)
 
 
+@pytest.mark.parametrize("plain", [False, True])
 @pytest.mark.parametrize("conv,pos", [(0, 0), (1, 17), (0, 65000)])
-def test_fwd_simt_rope(conv, pos):
+def test_fwd_simt_rope(conv, pos, plain):
     _fwd_check(1, 77, 2, 32, 32, 16, dtype="f32", kind="ckda", rope=(10000.0, conv), pos=pos,
-               h0_std=0.1, seed=9)
+               h0_std=0.1, seed=9, plain=plain)
 
 
 def test_fwd_simt_ragged_and_single_token():
     for T in (1, 15, 17, 63, 65):
-        _fwd_check(1, T, 2, 32, 16, 16, dtype="f32", kind="tiny", h0_std=0.3, seed=T)
+        for plain in (False, True):
+            _fwd_check(1, T, 2, 32, 16, 16, dtype="f32", kind="tiny", h0_std=0.3, seed=T,
+                       plain=plain)
 
 
 def test_fwd_simt_no_state_out():

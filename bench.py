@@ -609,7 +609,21 @@ def main():
                         "16-token chunks)",
             "ms": round(ms_b, 3), "mtok_s": round(B * T / (ms_b / 1e3) / 1e6, 3),
             "over_forward": round(ms_b / ms_local, 1)}
-        del bw, dout, dhT, wsb
+        # the same inputs through the CUDA-core forward (fp32-grade products; the path for
+        # workloads whose state does not decay), in its record form
+        wss = torch.empty(ck.simt_workspace_bytes(B, T, H, dk, dv), dtype=torch.uint8, device=dev)
+        outS, hS = torch.empty_like(bw["v"]), torch.empty_like(bw["h0"])
+        fnS = lambda i: ck.fwd_chunked(bw["q"], bw["k"], bw["v"], bw["alpha"], bw["beta"],
+                                       bw["h0"], path="simt", out=outS, hT=hS, workspace=wss)
+        for i in range(2):
+            fnS(i)
+        ms_s = event_time_ms(fnS, nB, stream) / nB
+        extras["simt_forward"] = {
+            "workload": f"{w['name']} (B={B},T={T},H={H},dk=dv={dk}) with h0, CUDA-core path, "
+                        "record form (16-token chunks, split-tf32 warp tiles)",
+            "ms": round(ms_s, 3), "mtok_s": round(B * T / (ms_s / 1e3) / 1e6, 2),
+            "over_forward": round(ms_s / ms_local, 1)}
+        del bw, dout, dhT, wsb, wss, outS, hS
 
         # ---- batched decode: 256 sequences x 32 heads, dk = dv = 128 ------------------------
         wd = synth.WORKLOADS["decode_bf16"]

@@ -212,6 +212,14 @@ def fwd_chunked(q, k, v, alpha, beta, h0=None, *, chunk=64, l2norm=True, rope_th
     return out, hT
 
 
+def simt_workspace_bytes(B, T, H, dk, dv) -> int:
+    """Bytes of the optional workspace that selects the record form of the CUDA-core path."""
+    n = _load().ckda_fwd_simt_workspace_bytes(B, T, H, dk, dv)
+    if n == ctypes.c_size_t(-1).value:
+        raise ValueError("unsupported problem for the CUDA-core path")
+    return int(n)
+
+
 def segments_auto(B, T, H) -> int:
     """Segment count ckda_fwd_segments_auto picks for a batch of B x H sequences of T tokens on the
     current device (1: the single fused launch is expected to be faster)."""

@@ -57,7 +57,7 @@ def parse():
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--no-extras", action="store_true",
                     help="skip decode / KDA-ratio / e2e / CPU-baseline legs")
-    ap.add_argument("--profile-case", choices=["fwd", "decode", "prologue", "bwd", "seg"], default=None,
+    ap.add_argument("--profile-case", choices=["fwd", "decode", "prologue", "bwd", "seg", "simt"], default=None,
                     help="run only a few calls of one entry point (for ncu captures) and exit")
     return ap.parse_args()
 
@@ -284,6 +284,15 @@ def profile_case(case, calls, dev):
         dhT = 0.02 * torch.randn((w["B"], w["H"], w["dk"], w["dv"]), generator=gen, device=dev)
         for _ in range(calls):
             ck.bwd_chunked(s["q"], s["k"], s["v"], s["alpha"], s["beta"], s["h0"], dout, dhT)
+    elif case == "simt":
+        w = WORKLOAD
+        s = synth.torch_fwd_inputs(w["B"], w["T"], w["H"], w["dk"], w["dv"], kind=w["kind"],
+                                   h0_std=0.02, seed=1, device=dev)
+        ws = torch.empty(ck.simt_workspace_bytes(w["B"], w["T"], w["H"], w["dk"], w["dv"]),
+                         dtype=torch.uint8, device=dev)
+        for _ in range(calls):
+            ck.fwd_chunked(s["q"], s["k"], s["v"], s["alpha"], s["beta"], s["h0"], path="simt",
+                           workspace=ws)
     elif case == "seg":
         wl = synth.WORKLOADS["long_rope_bf16"]
         s = synth.torch_fwd_inputs(1, wl["T"], 2, 128, 128, kind="ckda", dtype="bf16",

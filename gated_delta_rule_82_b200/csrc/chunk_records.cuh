@@ -32,19 +32,18 @@ __device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0
 
 // ---- warp-level tensor-core tiles with fp32-grade products ------------------------------------
 // mma.sync m16n8k8 with tf32 operands, each operand split into a tf32 head and a tf32 tail
-// (x = hi + lo, lo the rounded remainder): a b = a_hi b_hi + a_hi b_lo + a_lo b_hi up to a relative
-// 2^-21, i.e. the product of two fp32 values to about fp32 precision ("3xTF32").  Fragment layout
+// (x = hi + lo: hi is x with its 13 low mantissa bits cleared, lo the remainder x - hi, exact in
+// fp32, with its own 13 low bits cleared; each cut loses under 2^-10 of what it cuts):
+// a b = a_hi b_hi + a_hi b_lo + a_lo b_hi up to a relative 3 * 2^-20, i.e. the product of two
+// fp32 values to about fp32 precision ("3xTF32").  The cuts are integer masks on the full-rate
+// pipes.  Fragment layout
 // (PTX ISA, mma.m16n8k8 .tf32), g = lane / 4, t = lane % 4: A a0 = A[g][t], a1 = A[g+8][t],
 // a2 = A[g][t+4], a3 = A[g+8][t+4]; B b0 = B[t][g], b1 = B[t+4][g]; D d0 = D[g][2t],
 // d1 = D[g][2t+1], d2 = D[g+8][2t], d3 = D[g+8][2t+1].
-__device__ __forceinline__ uint32_t f2tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
-}
+constexpr uint32_t kTf32Mask = 0xffffe000u;   // sign, exponent and the 10 tf32 mantissa bits
 __device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
-    hi = f2tf32(x);
-    lo = f2tf32(x - __uint_as_float(hi));
+    hi = __float_as_uint(x) & kTf32Mask;
+    lo = __float_as_uint(x - __uint_as_float(hi)) & kTf32Mask;
 }
 __device__ __forceinline__ void mma_tf32(float c[4], const uint32_t a[4], const uint32_t b[2]) {
     asm volatile(

@@ -208,14 +208,15 @@ __device__ __forceinline__ void issue_v(const TcMaps& m, uint8_t* sm, uint64_t* 
 // Merge products of 16 x 16 and 32 x 32 blocks run on the warp-level tensor-core instruction
 // (mma.sync m16n8k8, tf32 operands rounded to nearest, fp32 accumulation): these blocks are below
 // the smallest tcgen05 tile (M = 64).  tf32 keeps 10 mantissa bits (the results become bf16 T').
+// The rounding (to nearest, ties away from zero) is integer arithmetic on the bit pattern: half a
+// tf32 unit added to the magnitude, then the 13 dropped bits cleared (a carry into the exponent
+// rounds up to the next binade) -- the operands are finite.
 // Fragment layout (PTX ISA, mma.m16n8k8 .tf32), g = lane / 4, t = lane % 4:
 //   A (16 x 8, row-major)  a0 = A[g][t], a1 = A[g+8][t], a2 = A[g][t+4], a3 = A[g+8][t+4]
 //   B (8 x 8)              b0 = B[t][g], b1 = B[t+4][g]
 //   C, D (16 x 8, fp32)    c0 = D[g][2t], c1 = D[g][2t+1], c2 = D[g+8][2t], c3 = D[g+8][2t+1]
 __device__ __forceinline__ uint32_t to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
+    return (__float_as_uint(x) + 0x1000u) & 0xffffe000u;
 }
 // c (+)= A[16 x K] B[K x 8]: A rows `lda` floats apart, B rows `ldb` floats apart (shared memory)
 template <int K>

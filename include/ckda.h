@@ -308,7 +308,7 @@ CKDA_API size_t ckda_bwd_workspace_bytes(int B, int T, int H, int dk, int dv);
  * q, k, v, the gates and h0, for the forward with the same inputs, sizes and flags (rotation,
  * norm, scale, grouped value heads, gate logits).  Computed in fp32-grade arithmetic (fp32 on
  * the CUDA cores; the dense products as warp-level tensor-core tiles whose tf32 operands are split
- * into a head and the rounded remainder, about 2^-21 relative per product) by the chunked form
+ * into a head and a remainder, about 3 * 2^-20 relative per product) by the chunked form
  * run in reverse (16-token chunks: the forward replay keeps each chunk's entering
  * state, a reverse chain carries the state gradient, every chunk forms its input gradients, and
  * the prologue -- rotation, then L2 norm -- is differentiated last).  There is no backward on

@@ -6,7 +6,7 @@ reverse in fp32 (chunk 16; the stable algebra is restated in float64 in test_chu
 Every gradient -- dq, dk, dv, dalpha, dbeta, dh0 -- is compared element by element with the
 parity metric max|g - g_ref| / max|g_ref|.  The backward's arithmetic is fp32 throughout (bf16
 inputs are read exactly), so every case is held to the fp32 bound, 1e-4; the measured errors are
-1e-7 to 1e-5.
+5e-7 to 2e-5.
 """
 import numpy as np
 import pytest

@@ -606,84 +606,181 @@ bwd_grad_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
     __syncthreads();
     const float* sE = sdT;
 
-    // dq^, dk^ of every row (signs taken back out of q', k'):
-    //   dk'_j = sum_{m<j} E_jm R_jm k'_m + sum_{r>j} E_rj R_rj k'_r + sum_{r>=j} dM_rj R_rj q'_r
-    //           + dK_gamma,j g_j + dK_end,j sigma_C R_{C-1,j}
-    //   dq'_j = sum_{m<=j} dM_jm R_jm k'_m + dQ_gamma,j g_j          (dQ_gamma = dQ')
-    for (int e = tid; e < C * DK; e += kThreads) {
-        const int j = e / DK, c = e % DK;
-        if (j >= nvalid) continue;
-        const float Lj = f.L[j * LD + c];
-        float dk = 0.f, dq = 0.f;
-        for (int m = 0; m < j; ++m) {
-            const float R = exp2f(Lj - f.L[m * LD + c]);
-            dk += sE[j * C + m] * R * f.k[m * LD + c];
-            dq += sdM[j * C + m] * R * f.k[m * LD + c];
+    // The ratios R_rj = g_r / g_j of a chunk whose decay stays >= 2^-60 in every channel factor
+    // into g_r and 1/g_j with room to spare in fp32 (products of a gradient and g stay normal), so
+    // the sums over rows become warp-tile products and staircase sums; other chunks take the
+    // ratios exactly, exp2(L_r - L_j) per channel.
+    const bool factored = __syncthreads_and(tid >= DK || f.LC[tid] >= -60.f) != 0;
+    if (factored) {
+        static_assert(Sh::off_tiles + 3 * Sh::CD + 2 * Sh::CK <= Sh::total, "K/g, Q_gamma fit");
+        // K / g and Q_gamma, rows KP apart, in the part of the tile region the loop left dead
+        float* sKi = smem + Sh::off_tiles + 3 * Sh::CD;
+        float* sQg = sKi + Sh::CK;
+        for (int e = tid; e < C * DK; e += kThreads) {
+            const int r = e / DK, c = e % DK;
+            const float L = f.L[r * LD + c];
+            sKi[r * KP + c] = f.k[r * LD + c] * exp2f(-L);
+            sQg[r * KP + c] = f.q[r * LD + c] * exp2f(L);
         }
-        dq += sdM[j * C + j] * f.k[j * LD + c];
-        for (int r = j; r < C; ++r) {
-            const float R = exp2f(f.L[r * LD + c] - Lj);
-            dk += (sE[r * C + j] * f.k[r * LD + c] + sdM[r * C + j] * f.q[r * LD + c]) * R;
-        }
-        const float g = exp2f(Lj);
-        dk += f.b[j] * sdW[e] * g + sdKe[e] * f.sg[c] * exp2f(f.LC[c] - Lj);
-        dq += sdQp[e] * g;
-        const size_t o = ((first + t0 + j) * H + h) * DK + c;
-        const float sgn = (sSgn[c] >> j) & 1u ? -1.f : 1.f;
-        ws_dq[o] = sgn * dq;
-        ws_dk[o] = sgn * dk;
-    }
-    // dalpha in the order t = 0 .. C-1, two threads per channel c (lanes 2 c, 2 c + 1 of a warp),
-    // thread half hh taking the rows a, r = hh mod 2 of the sums:
-    //   dg_r = dK_gamma,r k'_r + dQ_gamma,r q'_r (+ dgamma_C sigma_C at the last row)
-    //   dR_ab = E_ab k'_a k'_b + dM_ab q'_a k'_b (+ dK_end,b sigma_C k'_b at a = C-1), b <= a
-    //   dalpha_t = sign(alpha_t) [g_{t-1} sum_{r>=t} dg_r R_rt + sum_{a>=t} R_at Z_at],
-    //   Z_{a,t} = |alpha_{t-1}| Z_{a,t-1} + dR_{a,t-1},  Z_{a,0} = 0
-    static_assert(2 * DK <= kThreads, "two threads per channel");
-    if ((tid >> 1) < DK) {   // whole warps (DK is a multiple of 16)
-        const int c = tid >> 1, hh = tid & 1;
-        const float sC = f.sg[c];
-        float Z[C / 2], dgv[C / 2];
+        __syncthreads();
+        if (warp >= 4) {
+            // dq^, dk^ on warp tiles of 8 channels (signs taken back out of q', k'):
+            //   P1 = E (K/g),  P2 = E^T K_gamma + dM^T Q_gamma,  P3 = dM (K/g)
+            //   dk'_j = g_j P1_j + P2_j / g_j + dK_gamma,j g_j + dK_end,j sigma_C g_C / g_j
+            //   dq'_j = g_j (P3_j + dQ_gamma,j)
+            const int g = lane >> 2, t = lane & 3;
+            for (int id = warp - 4; id < DK / 8; id += kThreads / 32 - 4) {
+                const int n0 = 8 * id;
+                float p1[4] = {0.f, 0.f, 0.f, 0.f}, p2[4] = {0.f, 0.f, 0.f, 0.f};
+                float p3[4] = {0.f, 0.f, 0.f, 0.f};
+                mma3_tile<C>(p1, [&](int m, int kk) { return sE[m * C + kk]; },
+                             [&](int kk, int n) { return sKi[kk * KP + n0 + n]; }, lane);
+                mma3_tile<C>(p2, [&](int m, int kk) { return sE[kk * C + m]; },
+                             [&](int kk, int n) { return sKg[kk * KP + n0 + n]; }, lane);
+                mma3_tile<C>(p2, [&](int m, int kk) { return sdM[kk * C + m]; },
+                             [&](int kk, int n) { return sQg[kk * KP + n0 + n]; }, lane);
+                mma3_tile<C>(p3, [&](int m, int kk) { return sdM[m * C + kk]; },
+                             [&](int kk, int n) { return sKi[kk * KP + n0 + n]; }, lane);
 #pragma unroll
-        for (int i = 0; i < C / 2; ++i) {
-            const int r = 2 * i + hh;
-            Z[i] = 0.f;
-            dgv[i] = f.b[r] * sdW[r * DK + c] * f.k[r * LD + c] + sdQp[r * DK + c] * f.q[r * LD + c];
-            if (r == C - 1) dgv[i] += sdgC[c] * sC;
-        }
-        auto dR = [&](int a, int bb) {
-            float x = (sE[a * C + bb] * f.k[a * LD + c] + sdM[a * C + bb] * f.q[a * LD + c]) * f.k[bb * LD + c];
-            if (a == C - 1) x += sdKe[bb * DK + c] * sC * f.k[bb * LD + c];
-            return x;
-        };
+                for (int hf = 0; hf < 2; ++hf) {
+                    const int j = g + 8 * hf, c = n0 + 2 * t;
+                    if (j >= nvalid) continue;
+                    float dq2[2], dk2[2];
 #pragma unroll
-        for (int t = 0; t < C; ++t) {
-            if (t > 0) {
-                const float am = exp2f(f.L[(t - 1) * LD + c] - (t > 1 ? f.L[(t - 2) * LD + c] : 0.f));
-#pragma unroll
-                for (int i = 0; i < C / 2; ++i) {
-                    const int a = 2 * i + hh;
-                    Z[i] = a >= t - 1 ? am * Z[i] + dR(a, t - 1) : 0.f;
+                    for (int u = 0; u < 2; ++u) {
+                        const int cc = c + u, i = 2 * hf + u;
+                        const float L = f.L[j * LD + cc], gj = exp2f(L), hj = exp2f(-L);
+                        const float sgn = (sSgn[cc] >> j) & 1u ? -1.f : 1.f;
+                        dk2[u] = sgn * (gj * p1[i] + hj * p2[i] + f.b[j] * sdW[j * DK + cc] * gj +
+                                        sdKe[j * DK + cc] * f.sg[cc] * exp2f(f.LC[cc] - L));
+                        dq2[u] = sgn * gj * (p3[i] + sdQp[j * DK + cc]);
+                    }
+                    const size_t o = ((first + t0 + j) * H + h) * DK + c;
+                    *reinterpret_cast<float2*>(ws_dq + o) = make_float2(dq2[0], dq2[1]);
+                    *reinterpret_cast<float2*>(ws_dk + o) = make_float2(dk2[0], dk2[1]);
                 }
             }
-            const float Lt = f.L[t * LD + c];
-            float s1 = 0.f, s2 = 0.f;
+        } else if (tid < DK) {
+            // dalpha of channel c = tid.  With D_ab = R_ab dR_ab = (K_gamma,a E_ab + Q_gamma,a dM_ab
+            // (+ g_C sigma_C dK_end,b at a = C-1)) (K/g)_b and S_t = sum_{a>=t} sum_{b<t} D_ab
+            // (the sum of R_at Z_at over a >= t, times g_t / g_{t-1}):
+            //   dalpha_t = sign(alpha_t) (g_{t-1} / g_t) [sum_{r>=t} dg_r g_r + S_t]
+            const int c = tid;
+            float S[C];
 #pragma unroll
+            for (int b = 0; b < C; ++b) S[b] = 0.f;
+            const float gC = exp2f(f.LC[c]) * f.sg[c];
+#pragma unroll
+            for (int a = 1; a < C; ++a) {
+                const float ka = sKg[a * KP + c], qa = sQg[a * KP + c];
+                float pr = 0.f;   // sum_{b < tt} D_ab
+#pragma unroll
+                for (int tt = 0; tt <= a; ++tt) {
+                    S[tt] += pr;
+                    if (tt < a) {
+                        float d = ka * sE[a * C + tt] + qa * sdM[a * C + tt];
+                        if (a == C - 1) d += gC * sdKe[tt * DK + c];
+                        pr += d * sKi[tt * KP + c];
+                    }
+                }
+            }
+            float sfx = 0.f;   // sum_{r >= tt} dg_r g_r
+#pragma unroll
+            for (int tt = C - 1; tt >= 0; --tt) {
+                const float L = f.L[tt * LD + c];
+                float dg = f.b[tt] * sdW[tt * DK + c] * f.k[tt * LD + c] + sdQp[tt * DK + c] * f.q[tt * LD + c];
+                if (tt == C - 1) dg += sdgC[c] * f.sg[c];
+                sfx += dg * exp2f(L);
+                if (tt < nvalid) {
+                    const float Lp = tt > 0 ? f.L[(tt - 1) * LD + c] : 0.f;
+                    const float a = sAl[tt * DK + c];
+                    float d = (a < 0.f ? -1.f : 1.f) * exp2f(Lp - L) * (sfx + S[tt]);
+                    if (gate_logits) d *= 0.5f * (1.f - a * a);   // alpha = 2 sigma(a) - 1
+                    dalpha[((first + t0 + tt) * H + h) * DK + c] = d;
+                }
+            }
+        }
+    } else {
+
+        // dq^, dk^ of every row (signs taken back out of q', k'):
+        //   dk'_j = sum_{m<j} E_jm R_jm k'_m + sum_{r>j} E_rj R_rj k'_r + sum_{r>=j} dM_rj R_rj q'_r
+        //           + dK_gamma,j g_j + dK_end,j sigma_C R_{C-1,j}
+        //   dq'_j = sum_{m<=j} dM_jm R_jm k'_m + dQ_gamma,j g_j          (dQ_gamma = dQ')
+        for (int e = tid; e < C * DK; e += kThreads) {
+            const int j = e / DK, c = e % DK;
+            if (j >= nvalid) continue;
+            const float Lj = f.L[j * LD + c];
+            float dk = 0.f, dq = 0.f;
+            for (int m = 0; m < j; ++m) {
+                const float R = exp2f(Lj - f.L[m * LD + c]);
+                dk += sE[j * C + m] * R * f.k[m * LD + c];
+                dq += sdM[j * C + m] * R * f.k[m * LD + c];
+            }
+            dq += sdM[j * C + j] * f.k[j * LD + c];
+            for (int r = j; r < C; ++r) {
+                const float R = exp2f(f.L[r * LD + c] - Lj);
+                dk += (sE[r * C + j] * f.k[r * LD + c] + sdM[r * C + j] * f.q[r * LD + c]) * R;
+            }
+            const float g = exp2f(Lj);
+            dk += f.b[j] * sdW[e] * g + sdKe[e] * f.sg[c] * exp2f(f.LC[c] - Lj);
+            dq += sdQp[e] * g;
+            const size_t o = ((first + t0 + j) * H + h) * DK + c;
+            const float sgn = (sSgn[c] >> j) & 1u ? -1.f : 1.f;
+            ws_dq[o] = sgn * dq;
+            ws_dk[o] = sgn * dk;
+        }
+        // dalpha in the order t = 0 .. C-1, two threads per channel c (lanes 2 c, 2 c + 1 of a warp),
+        // thread half hh taking the rows a, r = hh mod 2 of the sums:
+        //   dg_r = dK_gamma,r k'_r + dQ_gamma,r q'_r (+ dgamma_C sigma_C at the last row)
+        //   dR_ab = E_ab k'_a k'_b + dM_ab q'_a k'_b (+ dK_end,b sigma_C k'_b at a = C-1), b <= a
+        //   dalpha_t = sign(alpha_t) [g_{t-1} sum_{r>=t} dg_r R_rt + sum_{a>=t} R_at Z_at],
+        //   Z_{a,t} = |alpha_{t-1}| Z_{a,t-1} + dR_{a,t-1},  Z_{a,0} = 0
+        static_assert(2 * DK <= kThreads, "two threads per channel");
+        if ((tid >> 1) < DK) {   // whole warps (DK is a multiple of 16)
+            const int c = tid >> 1, hh = tid & 1;
+            const float sC = f.sg[c];
+            float Z[C / 2], dgv[C / 2];
+    #pragma unroll
             for (int i = 0; i < C / 2; ++i) {
                 const int r = 2 * i + hh;
-                if (r < t) continue;
-                const float R = exp2f(f.L[r * LD + c] - Lt);
-                s1 += dgv[i] * R;
-                s2 += Z[i] * R;
+                Z[i] = 0.f;
+                dgv[i] = f.b[r] * sdW[r * DK + c] * f.k[r * LD + c] + sdQp[r * DK + c] * f.q[r * LD + c];
+                if (r == C - 1) dgv[i] += sdgC[c] * sC;
             }
-            s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
-            s2 += __shfl_xor_sync(0xffffffffu, s2, 1);
-            if (hh == 0 && t < nvalid) {
-                const float gprev = t > 0 ? exp2f(f.L[(t - 1) * LD + c]) : 1.f;
-                const float a = sAl[t * DK + c];
-                float d = (a < 0.f ? -1.f : 1.f) * (gprev * s1 + s2);
-                if (gate_logits) d *= 0.5f * (1.f - a * a);   // alpha = 2 sigma(a) - 1
-                dalpha[((first + t0 + t) * H + h) * DK + c] = d;
+            auto dR = [&](int a, int bb) {
+                float x = (sE[a * C + bb] * f.k[a * LD + c] + sdM[a * C + bb] * f.q[a * LD + c]) * f.k[bb * LD + c];
+                if (a == C - 1) x += sdKe[bb * DK + c] * sC * f.k[bb * LD + c];
+                return x;
+            };
+    #pragma unroll
+            for (int t = 0; t < C; ++t) {
+                if (t > 0) {
+                    const float am = exp2f(f.L[(t - 1) * LD + c] - (t > 1 ? f.L[(t - 2) * LD + c] : 0.f));
+    #pragma unroll
+                    for (int i = 0; i < C / 2; ++i) {
+                        const int a = 2 * i + hh;
+                        Z[i] = a >= t - 1 ? am * Z[i] + dR(a, t - 1) : 0.f;
+                    }
+                }
+                const float Lt = f.L[t * LD + c];
+                float s1 = 0.f, s2 = 0.f;
+    #pragma unroll
+                for (int i = 0; i < C / 2; ++i) {
+                    const int r = 2 * i + hh;
+                    if (r < t) continue;
+                    const float R = exp2f(f.L[r * LD + c] - Lt);
+                    s1 += dgv[i] * R;
+                    s2 += Z[i] * R;
+                }
+                s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+                s2 += __shfl_xor_sync(0xffffffffu, s2, 1);
+                if (hh == 0 && t < nvalid) {
+                    const float gprev = t > 0 ? exp2f(f.L[(t - 1) * LD + c]) : 1.f;
+                    const float a = sAl[t * DK + c];
+                    float d = (a < 0.f ? -1.f : 1.f) * (gprev * s1 + s2);
+                    if (gate_logits) d *= 0.5f * (1.f - a * a);   // alpha = 2 sigma(a) - 1
+                    dalpha[((first + t0 + t) * H + h) * DK + c] = d;
+                }
             }
         }
     }

@@ -94,8 +94,10 @@ def test_bwd_grouped_heads():
 
 
 def test_bwd_exact_zero_and_tiny_gates():
-    """Exact-zero gates and long runs of tiny gates: the chunked backward never divides by a
-    gate, so the gradients stay finite and match the token-by-token oracle."""
+    """Exact-zero gates and long runs of tiny gates: chunks holding them take the exact ratio
+    form, which never divides by a gate (the factored form is used only where every channel's
+    decay over the chunk stays >= 2^-60), so the gradients stay finite and match the
+    token-by-token oracle."""
     B, T, H, dk, dv = 1, 96, 2, 32, 32
     d, g = fwd_case(B, T, H, dk, dv, kind="tiny", dtype="f32", h0_std=0.3, seed=21)
     rng = np.random.default_rng(0)

@@ -182,7 +182,32 @@ def _stable_factors(qh, kh, V, a, b):
                 Qg=Qg, W=W, U=U, Kend=sig[-1] * R[-1] * kp, Qp=Qg - M @ W)
 
 
-def _stable_chunk_grads(F, V, a, b, S0, dO, dS1, scale):
+def _factored_gate_grads(F, a, E, dM, dQp, dKend, dKg, dg, reach=0):
+    """dq', dk' and dalpha of a chunk whose decay stays inside the fp32 range, with every ratio
+    factored as R_rj = g_r (1/g_j) (the GPU's form for chunks whose decay stays >= 2^-60):
+      dk' = g E (K/g) + (E^T K_gamma + dM^T Q_gamma) / g + dK_gamma g + dK_end sigma_C g_C / g
+      dq' = g (dM (K/g) + dQ')
+      dalpha_t = sign(alpha_t) (g_{t-1} / g_t) [sum_{r>=t} dg_r g_r + S_t],
+      S_t = sum_{a>=t} sum_{b<t} D_ab,  D_ab = R_ab dR_ab = (K_gamma,a E_ab + Q_gamma,a dM_ab
+            (+ g_C sigma_C dK_end,b at a = C-1)) (K/g)_b.
+    reach > 0 widens the staircase to b < t + reach (a planted mistake, for the test below)."""
+    g, kp, Kg, Qg, sC = F["g"], F["kp"], F["Kg"], F["Qg"], F["sC"]
+    C = g.shape[0]
+    Ki = kp / g
+    dkp = g * (E @ Ki) + (E.T @ Kg + dM.T @ Qg) / g + dKg * g + dKend * sC * g[-1] / g
+    dqp = g * (dM @ Ki + dQp)
+    D = (Kg[:, None, :] * E[:, :, None] + Qg[:, None, :] * dM[:, :, None]) * Ki[None, :, :]
+    D[-1] += (g[-1] * sC) * dKend * Ki
+    D *= np.tril(np.ones((C, C)), -1)[:, :, None]
+    da = np.zeros_like(a)
+    for t in range(C):
+        S_t = D[t:, :t + reach].sum((0, 1))
+        gprev = g[t - 1] if t > 0 else 1.0
+        da[t] = np.where(a[t] < 0, -1.0, 1.0) * (gprev / g[t]) * ((dg[t:] * g[t:]).sum(0) + S_t)
+    return dqp, dkp, da
+
+
+def _stable_chunk_grads(F, V, a, b, S0, dO, dS1, scale, factored=False, reach=0):
     C = V.shape[0]
     kp, qp, R, g, T, W, U, M, Kend, Kg = (F[x] for x in ("kp", "qp", "R", "g", "T", "W", "U",
                                                          "M", "Kend", "Kg"))
@@ -214,11 +239,14 @@ def _stable_chunk_grads(F, V, a, b, S0, dO, dS1, scale):
         gprev = g[t - 1] if t > 0 else 1.0
         da[t] = np.where(a[t] < 0, -1.0, 1.0) * (gprev * (dg[t:] * R[t:, t]).sum(0)
                                                  + (R[t:, t] * Z[t:]).sum(0))
+    if factored:
+        dqp, dkp, da = _factored_gate_grads(F, a, E, dM, dQp, dKend, dKg, dg, reach)
     dS0 = scale * F["Qp"].T @ dO + (F["sC"] * F["gC"])[:, None] * dS1 - W.T @ (Kend @ dS1)
     return F["sig"] * dqp, F["sig"] * dkp, b[:, None] * Y, da, db, dS0
 
 
-def _stable_chunked_bwd(q, k, v, alpha, beta, h0, dout, dhT, C, scale, l2norm, theta, pos0):
+def _stable_chunked_bwd(q, k, v, alpha, beta, h0, dout, dhT, C, scale, l2norm, theta, pos0,
+                        factored=False):
     T, dk = q.shape
     pos = pos0 + np.arange(T, dtype=np.float64)
     yq = _rot(q, pos, theta) if theta > 0 else q.copy()
@@ -238,7 +266,7 @@ def _stable_chunked_bwd(q, k, v, alpha, beta, h0, dout, dhT, C, scale, l2norm, t
         sl = slice(ci * C, min(T, ci * C + C))
         F = _stable_factors(qh[sl], kh[sl], v[sl], alpha[sl], beta[sl])
         *gs, dS = _stable_chunk_grads(F, v[sl], alpha[sl], beta[sl], S0s[ci], dout[sl], dS,
-                                      scale)
+                                      scale, factored)
         for G_, x in zip(grads, gs):
             G_[sl] = x
 
@@ -275,3 +303,49 @@ def test_stable_chunked_backward_equals_the_oracle(T, C, theta, l2, amin, zeros)
     for name, x, y in zip(("dq", "dk", "dv", "dalpha", "dbeta", "dh0"), got, want):
         err = np.abs(x - y).max() / max(np.abs(y).max(), 1e-12)
         assert err < 1e-9, (name, err)
+
+
+@pytest.mark.parametrize("T,C,theta,l2", [(32, 8, 0.0, True), (45, 16, 1000.0, True),
+                                          (40, 16, 0.0, False)])
+def test_factored_gate_gradients_equal_the_oracle(T, C, theta, l2):
+    """The factored form of the chunk gradients (ratios split into g_r and 1/g_j, the dalpha
+    recurrence as a staircase sum) on gates whose chunk decay stays far inside the fp32 range
+    (|alpha| >= 0.3: at most 2^-28 over 16 tokens), against the token-by-token oracle."""
+    rng = np.random.default_rng(T * 11 + C)
+    dk, dv = 6, 4
+    q, k = rng.standard_normal((T, dk)), rng.standard_normal((T, dk))
+    v = rng.standard_normal((T, dv))
+    alpha = rng.choice([-1.0, 1.0], (T, dk)) * rng.uniform(0.3, 1.0, (T, dk))
+    beta = rng.uniform(0.0, 2.0, T)
+    h0 = rng.standard_normal((dk, dv))
+    dout, dhT = rng.standard_normal((T, dv)), rng.standard_normal((dk, dv))
+    scale = oracle.default_scale(dk)
+    got = _stable_chunked_bwd(q, k, v, alpha, beta, h0, dout, dhT, C, scale, l2, theta, 5,
+                              factored=True)
+    ref = oracle.bwd(q[None, :, None], k[None, :, None], v[None, :, None], alpha[None, :, None],
+                     beta[None, :, None], h0[None, None], dout[None, :, None], dhT[None, None],
+                     l2norm=l2, rope_theta=theta, pos_offset=5)
+    want = (ref["dq"][0, :, 0], ref["dk"][0, :, 0], ref["dv"][0, :, 0], ref["dalpha"][0, :, 0],
+            ref["dbeta"][0, :, 0], ref["dh0"][0, 0])
+    for name, x, y in zip(("dq", "dk", "dv", "dalpha", "dbeta", "dh0"), got, want):
+        err = np.abs(x - y).max() / max(np.abs(y).max(), 1e-12)
+        assert err < 1e-9, (name, err)
+
+
+def test_factored_staircase_boundary_matters():
+    """The factored form equals the exact form chunk by chunk, and the staircase's boundary is
+    pinned: widening it to b <= t (one diagonal of D too many) moves dalpha well off."""
+    rng = np.random.default_rng(3)
+    C, dk, dv = 8, 4, 3
+    q, k = rng.standard_normal((C, dk)), rng.standard_normal((C, dk))
+    v = rng.standard_normal((C, dv))
+    a = rng.choice([-1.0, 1.0], (C, dk)) * rng.uniform(0.5, 1.0, (C, dk))
+    b = rng.uniform(0.5, 2.0, C)
+    S0, dO, dS1 = (rng.standard_normal(x) for x in ((dk, dv), (C, dv), (dk, dv)))
+    F = _stable_factors(q, k, v, a, b)
+    exact = _stable_chunk_grads(F, v, a, b, S0, dO, dS1, 0.5)
+    fact = _stable_chunk_grads(F, v, a, b, S0, dO, dS1, 0.5, factored=True)
+    for x, y in zip(exact, fact):
+        assert np.abs(x - y).max() <= 1e-10 * max(np.abs(x).max(), 1.0)
+    wide = _stable_chunk_grads(F, v, a, b, S0, dO, dS1, 0.5, factored=True, reach=1)
+    assert np.abs(wide[3] - exact[3]).max() > 1e-2 * np.abs(exact[3]).max()

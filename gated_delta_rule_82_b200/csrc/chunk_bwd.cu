@@ -115,12 +115,16 @@ bwd_replay_kernel(const T* __restrict__ v, const float* __restrict__ h0,
             st_frag(sU + kq * C * SP, SP, 8 * nt, c, 1.f, lane);
         }
         __syncthreads();
-        auto u_at = [&](int r, int n) {
-            float x = 0.f;
+        // the parts of U summed once (in the order kq = 0 ..), in place in part 0
+        for (int e = tid; e < C * DVS; e += kThreads) {
+            const int o = (e / DVS) * SP + e % DVS;
+            float x = sU[o];
 #pragma unroll
-            for (int kq = 0; kq < KQ; ++kq) x += sU[kq * C * SP + r * SP + n];
-            return x;
-        };
+            for (int kq = 1; kq < KQ; ++kq) x += sU[kq * C * SP + o];
+            sU[o] = x;
+        }
+        __syncthreads();
+        auto u_at = [&](int r, int n) { return sU[r * SP + n]; };
         // S <- Diag(gamma_C) S + K_end^T U: (DK / 16) x NT tiles, each read and written in place
         for (int id = warp; id < (DK / 16) * NT; id += kThreads / 32) {
             const int r0 = 16 * (id / NT), c0 = 8 * (id % NT) + 2 * t;
@@ -215,12 +219,16 @@ bwd_chain_kernel(const T* __restrict__ dout, const float* __restrict__ dhT,
             st_frag(sKd + kq * C * SP, SP, 8 * nt, c, 1.f, lane);
         }
         __syncthreads();
-        auto kd_at = [&](int r, int n) {
-            float x = 0.f;
+        // the parts of K_end dS_out summed once (in the order kq = 0 ..), in place in part 0
+        for (int e = tid; e < C * DVS; e += kThreads) {
+            const int o = (e / DVS) * SP + e % DVS;
+            float x = sKd[o];
 #pragma unroll
-            for (int kq = 0; kq < KQ; ++kq) x += sKd[kq * C * SP + r * SP + n];
-            return x;
-        };
+            for (int kq = 1; kq < KQ; ++kq) x += sKd[kq * C * SP + o];
+            sKd[o] = x;
+        }
+        __syncthreads();
+        auto kd_at = [&](int r, int n) { return sKd[r * SP + n]; };
         // dS_in = Diag(gamma_C) dS_out + scale Q'^T dO - W^T K_d, tiles read and written in place
         for (int id = warp; id < (DK / 16) * NT; id += kThreads / 32) {
             const int r0 = 16 * (id / NT), nt = id % NT, c0 = 8 * nt + 2 * t;
